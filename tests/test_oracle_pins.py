@@ -1,0 +1,362 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Each test ties one part of the oracle to a closed form, an invariant, a
+published known-answer value or finite differences, chosen so that a
+plausible slip (a dropped term, a wrong sign or index, a transposed operand,
+the wrong GELU or mask) fails at least one of them.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import gpt_oracle as O
+from scratch_decoder_only_b200 import configs as CF
+from scratch_decoder_only_b200 import synthetic as S
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def ocfg(mc: CF.ModelConfig) -> O.OracleConfig:
+    return O.OracleConfig(vocab=mc.vocab, vocab_padded=mc.vocab_padded, d_model=mc.d_model,
+                          n_heads=mc.n_heads, d_mlp=mc.d_mlp, n_layers=mc.n_layers,
+                          max_seq=mc.max_seq, tied=mc.tied, ln_eps=mc.ln_eps,
+                          init_std=mc.init_std)
+
+
+TINY = O.OracleConfig(vocab=11, vocab_padded=16, d_model=8, n_heads=2, d_mlp=16,
+                      n_layers=2, max_seq=6)
+
+
+def random_params(cfg, seed, scale=0.3):
+    """Every parameter random (not the standard init), so each one matters."""
+    rng = np.random.default_rng(seed)
+    flat = rng.normal(0.0, scale, O.num_params(cfg))
+    P = O.unflatten(cfg, flat)
+    for name in P:
+        if name.endswith("_g"):
+            P[name][...] = 1.0 + rng.normal(0, 0.2, P[name].shape)
+    P["wte"][cfg.vocab:] = 0.0
+    if not cfg.tied:
+        P["w_head"][cfg.vocab:] = 0.0
+    return flat
+
+
+# ---------------------------------------------------------------- generators
+
+def test_splitmix64_known_answer():
+    lines = [l for l in open(os.path.join(GOLDEN, "splitmix64_seed1234567.txt"))
+             if l.strip() and not l.startswith("#")]
+    seed = int(lines[0].split()[1])
+    want = np.array([int(x) for x in lines[1:]], dtype=np.uint64)
+    got = O.splitmix64(seed, np.arange(len(want), dtype=np.uint64))
+    assert np.array_equal(got, want)
+
+
+def test_box_muller_moments():
+    z = O.gaussian_for_elements(7, np.arange(1_000_000, dtype=np.uint64))
+    n = z.size
+    assert abs(z.mean()) < 4 / math.sqrt(n)
+    assert abs(z.std() - 1.0) < 4 * math.sqrt(0.5 / n)
+    # fourth moment of N(0,1) is 3 (rules out uniform-like or mis-scaled draws)
+    assert abs((z ** 4).mean() - 3.0) < 0.05
+    # symmetric: the fraction below 0 is 1/2
+    assert abs((z < 0).mean() - 0.5) < 4 * 0.5 / math.sqrt(n)
+
+
+@pytest.mark.parametrize("wl,n_expected", [(CF.TINY_BYTE, 473_728), (CF.PACKED_SMALL, 4_950_144),
+                                           (CF.BYTE_30M, 26_007_552), (CF.GPT2_124M, 124_475_904)])
+def test_param_counts(wl, n_expected):
+    assert O.num_params(ocfg(wl.model)) == n_expected
+    assert wl.model.num_params() == n_expected
+
+
+def test_init_statistics_and_constants():
+    cfg = ocfg(CF.TINY_BYTE.model)
+    flat = O.init_params(cfg, 42)
+    P = O.unflatten(cfg, flat)
+    for name, arr in P.items():
+        leaf = name.split(".")[-1]
+        if leaf.endswith("_g"):
+            assert np.all(arr == 1.0)
+        elif leaf.startswith("b_") or leaf.endswith("_b"):
+            assert np.all(arr == 0.0)
+        else:
+            a = arr[:cfg.vocab] if leaf in ("wte", "w_head") else arr
+            n = a.size
+            assert abs(a.mean()) < 4 * 0.02 / math.sqrt(n), name
+            assert abs(a.std() - 0.02) < 4 * 0.02 * math.sqrt(0.5 / n) + 1e-4, name
+    # deterministic and seed-dependent
+    assert np.array_equal(flat, O.init_params(cfg, 42))
+    assert not np.array_equal(flat, O.init_params(cfg, 43))
+
+
+def test_init_pad_rows_zero():
+    cfg = O.OracleConfig(vocab=50, vocab_padded=64, d_model=16, n_heads=2, d_mlp=32,
+                         n_layers=1, max_seq=8, tied=True)
+    P = O.unflatten(cfg, O.init_params(cfg, 1))
+    assert np.all(P["wte"][50:] == 0) and np.any(P["wte"][:50] != 0)
+
+
+# ---------------------------------------------------------------- pieces
+
+def test_positions_from_segments():
+    pos, seg = O.positions_from_segments(np.array([[0, 0, 0, 1, 1, 2]]), 1, 6)
+    assert pos.tolist() == [[0, 1, 2, 0, 1, 0]]
+    pos, _ = O.positions_from_segments(None, 2, 4)
+    assert pos.tolist() == [[0, 1, 2, 3]] * 2
+
+
+def test_layernorm_hand_example():
+    x = np.array([[1.0, 2.0, 3.0, 4.0]])
+    y, xhat, rstd = O.layernorm_fwd(x, np.ones(4), np.zeros(4), 1e-5)
+    # mean 2.5, biased variance 1.25
+    want = (x - 2.5) / math.sqrt(1.25 + 1e-5)
+    assert np.allclose(y, want, rtol=0, atol=1e-15)
+    g, b = np.array([2.0, 1.0, 0.5, 3.0]), np.array([0.1, -0.2, 0.3, 0.0])
+    y2, _, _ = O.layernorm_fwd(x, g, b, 1e-5)
+    assert np.allclose(y2, want * g + b, atol=1e-15)
+    rng = np.random.default_rng(0)
+    z = rng.normal(3.0, 5.0, (7, 64))
+    yz, _, _ = O.layernorm_fwd(z, np.ones(64), np.zeros(64), 0.0)
+    assert np.allclose(yz.mean(-1), 0, atol=1e-12)
+    assert np.allclose((yz ** 2).mean(-1), 1, atol=1e-12)
+
+
+def test_gelu_tanh_form():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "gelu_tanh_points.txt"))
+            if l.strip() and not l.startswith("#")]
+    for u, g in rows:
+        assert abs(O.gelu(np.float64(u)) - float(g)) < 1e-12
+    assert abs(O.gelu(np.float64(1.0)) - 0.8413447460685429) > 1e-4   # not the erf form
+    assert abs(O.gelu(np.float64(12.0)) - 12.0) < 1e-12
+    assert abs(O.gelu(np.float64(-12.0))) < 1e-12
+    u = np.linspace(-6, 6, 241)
+    h = 1e-6
+    fd = (O.gelu(u + h) - O.gelu(u - h)) / (2 * h)
+    assert np.allclose(O.gelu_grad(u), fd, atol=1e-8)
+
+
+def test_attention_hand_example():
+    # one head, d = 4: scores scaled by 1/sqrt(4) = 1/2
+    q = np.zeros((1, 1, 2, 4)); k = np.zeros((1, 1, 2, 4)); v = np.zeros((1, 1, 2, 4))
+    q[0, 0, 1] = [2.0, 0, 0, 0]
+    k[0, 0, 0] = [1.0, 0, 0, 0]
+    v[0, 0, 0] = [1.0, 2.0, 3.0, 4.0]
+    v[0, 0, 1] = [-1.0, 0.0, 1.0, 0.0]
+    seg = np.zeros((1, 2), dtype=np.int64)
+    o = O.attention_fwd(q, k, v, seg)
+    # query 0 sees only key 0
+    assert np.allclose(o[0, 0, 0], v[0, 0, 0], atol=0)
+    # query 1: scores (1, 0) -> weights (e, 1)/(e+1)
+    w0 = math.e / (math.e + 1)
+    assert np.allclose(o[0, 0, 1], w0 * v[0, 0, 0] + (1 - w0) * v[0, 0, 1], atol=1e-15)
+    # a new document at position 1: query 1 sees only itself
+    o2 = O.attention_fwd(q, k, v, np.array([[0, 1]]))
+    assert np.allclose(o2[0, 0, 1], v[0, 0, 1], atol=0)
+
+
+def test_softmax_rows_sum_to_one():
+    rng = np.random.default_rng(3)
+    q, k = rng.normal(size=(3, 9, 8)), rng.normal(size=(3, 9, 8))
+    seg = np.array([0, 0, 0, 1, 1, 1, 1, 2, 2])
+    p = O.attention_probs(q, k, O.allowed_mask(seg))
+    assert np.all(np.abs(p.sum(-1) - 1.0) <= 1e-12)
+    assert np.all(p[:, ~O.allowed_mask(seg)] == 0.0)
+    p32 = O.attention_probs(q.astype(np.float32), k.astype(np.float32), O.allowed_mask(seg))
+    assert np.all(np.abs(p32.sum(-1) - 1.0) <= 1e-6)
+    z = rng.normal(size=(5, 20))
+    _, dz = O.cross_entropy(z, np.array([1, 2, 3, 4, 5]), 20)
+    assert np.allclose(dz.sum(1), 0.0, atol=1e-15)   # softmax rows sum to 1 minus the one-hot
+
+
+def test_cross_entropy_closed_forms():
+    V = 7
+    z = np.zeros((3, 10))
+    loss, dz = O.cross_entropy(z, np.array([0, 6, -1]), V)
+    assert abs(loss - math.log(V)) < 1e-15
+    assert np.all(dz[:, V:] == 0) and np.all(dz[2] == 0)
+    assert abs(dz[0, 0] - (1 / V - 1) / 2) < 1e-15 and abs(dz[0, 1] - (1 / V) / 2) < 1e-15
+    # hand example, V = 3, logits (0, ln 2, 0), target 1: p = (1/4, 1/2, 1/4), loss = ln 2
+    z = np.array([[0.0, math.log(2.0), 0.0]])
+    loss, dz = O.cross_entropy(z, np.array([1]), 3)
+    assert abs(loss - math.log(2.0)) < 1e-15
+    assert np.allclose(dz, [[0.25, -0.5, 0.25]], atol=1e-15)
+
+
+# ---------------------------------------------------------------- whole model
+
+def _fd_check(cfg, seg, seed):
+    rng = np.random.default_rng(seed)
+    B, T = 2, cfg.max_seq
+    x = rng.integers(0, cfg.vocab, size=(B, T + 1))
+    tokens, targets = x[:, :-1], x[:, 1:].copy()
+    if seg is not None:
+        targets[:, :-1][seg[:, 1:] != seg[:, :-1]] = -1
+    targets[0, 2] = -1                       # an ignored position
+    flat = random_params(cfg, seed)
+    loss, g = O.loss_and_grads(cfg, flat, tokens, targets, seg)
+    h = 1e-5
+    fd = np.empty_like(g)
+    for i in range(flat.size):
+        old = flat[i]
+        flat[i] = old + h
+        lp, _ = O.cross_entropy(O.forward(cfg, flat, tokens, seg)[0], targets.reshape(-1), cfg.vocab)
+        flat[i] = old - h
+        lm, _ = O.cross_entropy(O.forward(cfg, flat, tokens, seg)[0], targets.reshape(-1), cfg.vocab)
+        flat[i] = old
+        fd[i] = (lp - lm) / (2 * h)
+    err = np.abs(fd - g) - 1e-6 * np.maximum(1.0, np.abs(g))
+    assert np.all(err <= 0), (np.max(np.abs(fd - g)), int(np.argmax(err)))
+    # the check must see real gradients in every tensor class
+    assert np.count_nonzero(g) > 0.5 * g.size
+    return g
+
+
+def test_fd_gradients_plain():
+    _fd_check(TINY, None, 11)
+
+
+def test_fd_gradients_packed():
+    seg = np.array([[0, 0, 0, 1, 1, 1], [0, 0, 1, 1, 1, 2]])
+    _fd_check(TINY, seg, 12)
+
+
+def test_fd_gradients_tied():
+    cfg = O.OracleConfig(**{**TINY.__dict__, "tied": True})
+    _fd_check(cfg, None, 13)
+
+
+def test_initial_loss_near_ln_v():
+    wl = CF.TINY_BYTE
+    cfg = ocfg(wl.model)
+    flat = O.init_params(cfg, wl.init_seed)
+    tok, tgt, seg = S.make_batch(wl)
+    logits, _ = O.forward(cfg, flat, tok, seg)
+    loss, _ = O.cross_entropy(logits, tgt.reshape(-1), cfg.vocab)
+    sigma2 = cfg.init_std ** 2 * cfg.d_model
+    assert abs(loss - (math.log(cfg.vocab) + sigma2 / 2)) <= 0.1
+    assert abs(math.log(257) - 5.5491) < 1e-4
+
+
+def test_mask_future_has_no_influence():
+    cfg = TINY
+    flat = random_params(cfg, 5)
+    rng = np.random.default_rng(5)
+    tok = rng.integers(0, cfg.vocab, size=(2, 6))
+    for seg in (None, np.array([[0, 0, 0, 1, 1, 1], [0, 1, 1, 1, 2, 2]])):
+        base, _ = O.forward(cfg, flat, tok, seg)
+        base = base.reshape(2, 6, -1)
+        for j in range(6):
+            t2 = tok.copy()
+            t2[:, j] = (t2[:, j] + 1) % cfg.vocab
+            alt = O.forward(cfg, flat, t2, seg)[0].reshape(2, 6, -1)
+            for b in range(2):
+                for i in range(6):
+                    same_doc = seg is None or seg[b, i] == seg[b, j]
+                    if i < j or not same_doc:
+                        assert np.array_equal(base[b, i], alt[b, i]), (b, i, j)
+                    elif i == j:
+                        assert not np.array_equal(base[b, i], alt[b, i])
+
+
+def test_packed_row_equals_separate_documents():
+    cfg = TINY
+    flat = random_params(cfg, 8)
+    rng = np.random.default_rng(8)
+    tok = rng.integers(0, cfg.vocab, size=(1, 6))
+    seg = np.array([[0, 0, 0, 0, 1, 1]])
+    packed, _ = O.forward(cfg, flat, tok, seg)
+    a, _ = O.forward(cfg, flat, tok[:, :4], None)
+    b, _ = O.forward(cfg, flat, tok[:, 4:], None)
+    assert np.allclose(packed[:4], a, rtol=0, atol=1e-12)
+    assert np.allclose(packed[4:], b, rtol=0, atol=1e-12)
+    # all-equal seg ids is plain causal
+    same, _ = O.forward(cfg, flat, tok, np.zeros((1, 6), dtype=np.int64))
+    plain, _ = O.forward(cfg, flat, tok, None)
+    assert np.array_equal(same, plain)
+
+
+# ---------------------------------------------------------------- optimiser
+
+def test_clip_coefficient_hand_vector():
+    norm, coef = O.clip_coefficient(np.array([3.0, 4.0]), 1.0)
+    assert norm == 5.0 and abs(coef - 1.0 / (5.0 + 1e-6)) < 1e-18
+    norm, coef = O.clip_coefficient(np.array([0.3, 0.4]), 1.0)
+    assert coef == 1.0
+
+
+def test_adamw_closed_forms():
+    lr, b1, b2, eps, wd = 1e-3, 0.9, 0.95, 1e-8, 0.1
+    p0 = np.array([0.5, -0.25, 0.0, 1.0])
+    g1 = np.array([0.2, -0.1, 0.0, 3.0])
+    p1, m1, v1 = O.adamw_update(p0, g1, np.zeros(4), np.zeros(4), 1, lr, b1, b2, eps, wd)
+    # step 1: m_hat = g, v_hat = g^2 -> update = g/(|g|+eps)
+    want1 = p0 - lr * (g1 / (np.abs(g1) + eps) + wd * p0)
+    assert np.allclose(p1, want1, rtol=0, atol=1e-15)
+    # step 2 by hand in plain Python floats for element 0
+    g2 = 0.05
+    m = b1 * (1 - b1) * 0.2 + (1 - b1) * g2
+    v = b2 * (1 - b2) * 0.04 + (1 - b2) * g2 * g2
+    mh, vh = m / (1 - b1 ** 2), v / (1 - b2 ** 2)
+    want = p1[0] - lr * (mh / (math.sqrt(vh) + eps) + wd * p1[0])
+    p2, _, _ = O.adamw_update(p1, np.array([g2, 0, 0, 0]), m1, v1, 2, lr, b1, b2, eps, wd)
+    assert abs(p2[0] - want) < 1e-16
+
+
+def test_clip_adamw_step_skips_nonfinite():
+    p = np.ones(3); g = np.array([1.0, np.inf, 0.0])
+    p2, m2, v2, norm, skipped = O.clip_adamw_step(p, g, np.zeros(3), np.zeros(3), 1,
+                                                  1e-3, 0.9, 0.999, 1e-8, 0.0, 1.0)
+    assert skipped and np.array_equal(p2, p)
+    # clipped step: clip coefficient cancels at t = 1 except through eps
+    g = np.array([30.0, 40.0, 0.0])
+    p2, _, _, norm, skipped = O.clip_adamw_step(p, g, np.zeros(3), np.zeros(3), 1,
+                                                1e-3, 0.9, 0.999, 1e-8, 0.0, 1.0)
+    assert not skipped and norm == 50.0
+    assert np.allclose(p2, [1 - 1e-3, 1 - 1e-3, 1.0], atol=1e-9)
+
+
+def test_loss_scale_rule():
+    s, good, skip = O.loss_scale_update(2.0 ** 15, 5, False)
+    assert (s, good, skip) == (2.0 ** 14, 0, True)
+    s, good = 2.0 ** 15, 0
+    for _ in range(1999):
+        s, good, skip = O.loss_scale_update(s, good, True)
+    assert s == 2.0 ** 15 and good == 1999
+    s, good, skip = O.loss_scale_update(s, good, True)
+    assert s == 2.0 ** 16 and good == 0 and not skip
+
+
+# ---------------------------------------------------------------- decoding
+
+def _successor_model(V, C):
+    """Blocks are identities (zero weights), positions are 0, token k embeds as
+    the k-th unit vector and the head row c reads coordinate (c-1) mod V, so the
+    next token after k is (k+1) mod V."""
+    cfg = O.OracleConfig(vocab=V, vocab_padded=V, d_model=C, n_heads=2, d_mlp=2 * C,
+                         n_layers=2, max_seq=16)
+    flat = np.zeros(O.num_params(cfg))
+    P = O.unflatten(cfg, flat)
+    for name in P:
+        if name.endswith("_g"):
+            P[name][...] = 1.0
+    P["wte"][np.arange(V), np.arange(V)] = 1.0
+    P["w_head"][np.arange(V), (np.arange(V) - 1) % V] = 1.0
+    return cfg, flat
+
+
+def test_greedy_decode_successor_model():
+    cfg, flat = _successor_model(V=6, C=8)
+    out, gaps = O.greedy_decode(cfg, flat, np.array([[0, 3], [2, 5]]), n_new=5, dtype=np.float64)
+    assert out.tolist() == [[4, 5, 0, 1, 2], [0, 1, 2, 3, 4]]
+    assert np.all(gaps > 0)
+
+
+def test_greedy_decode_tie_lowest_index():
+    cfg, flat = _successor_model(V=6, C=8)
+    P = O.unflatten(cfg, flat)
+    P["w_head"][2] = P["w_head"][5]          # column 2 ties with column 5
+    out, gaps = O.greedy_decode(cfg, flat, np.array([[4]]), n_new=1, dtype=np.float64)
+    assert out.tolist() == [[2]] and gaps[0, 0] == 0.0
