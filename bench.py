@@ -1,0 +1,353 @@
+"""Benchmark: GPT-2 124M training step (forward + backward + clip + AdamW) on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = gpt_forward_loss + gpt_backward + gpt_clip_adamw_step over one
+16 x 1024 batch of synthetic Zipf(1.0) tokens (bf16 operands, fp32 master
+weights).  `value` is whole-job train tokens/s with inputs resident in HBM;
+`e2e` repeats the measurement through the public API with the batch copied
+from pinned host memory and the loss read back every step.  With N > 1 the
+N ranks run independent replicas (the step has no exchange on one GPU);
+time is the max over ranks.  The CPU oracle is timed on a bounded sample as
+`cpu_baseline`; `--impl reference` times only the oracle.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from scratch_decoder_only_b200 import configs as CF  # noqa: E402
+from scratch_decoder_only_b200 import synthetic as S  # noqa: E402
+
+WL = CF.GPT2_124M
+METRIC = "train tokens/sec (fwd+bwd+AdamW) GPT-2 124M bf16, MFU %; decode tok/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        d["source"] = "measured"
+        return d
+    d = dict(PEAKS_FALLBACK)
+    d["source"] = "fallback"
+    return d
+
+
+def flops_per_token(mc: CF.ModelConfig, T: int) -> float:
+    """6 N (matmul weights incl. embeddings) + causal attention 6 L C (T+1)."""
+    return 6.0 * mc.num_params() + 6.0 * mc.n_layers * mc.d_model * (T + 1)
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- oracle arm
+
+def oracle_sample_step(seq=256):
+    """One bounded oracle step: 1 row x `seq` tokens of the GPT-2 124M model,
+    forward + backward + clip + AdamW over all parameters (fp64).  Returns
+    (seconds, tokens, threads)."""
+    from oracle import gpt_oracle as O
+    mc = WL.model
+    cfg = O.OracleConfig(vocab=mc.vocab, vocab_padded=mc.vocab_padded, d_model=mc.d_model,
+                         n_heads=mc.n_heads, d_mlp=mc.d_mlp, n_layers=mc.n_layers, max_seq=mc.max_seq,
+                         tied=mc.tied)
+    tok, tgt, _ = S.make_batch(WL, batch=1, seq=seq)
+    p0 = O.init_params(cfg, WL.init_seed).astype(np.float64)
+    hp = WL.adamw
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    loss, g = O.loss_and_grads(cfg, p0, tok, tgt)
+    O.clip_adamw_step(p0, g, np.zeros_like(g), np.zeros_like(g), 1, hp.lr, hp.beta1, hp.beta2, hp.eps,
+                      hp.weight_decay, hp.clip_norm)
+    dt = time.perf_counter() - t0
+    return dt, seq, threads
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    steps = max(1, min(args.steps, 3))
+    for _ in range(max(0, min(args.warmup, 1))):
+        oracle_sample_step()
+    times, toks, threads = [], 0, 1
+    for _ in range(steps):
+        dt, n, threads = oracle_sample_step()
+        times.append(dt)
+        toks += n
+    total = sum(times)
+    value = toks / total
+    sample = f"1 row x 256 tokens of the GPT-2 124M step per timed step (fwd+bwd+clip+AdamW over all params, fp64 numpy), {steps} steps"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": 1000 * total / steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WL.name, "global_batch": 1, "seq_len": 256,
+                                            "parallelism": "none (CPU oracle)"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from scratch_decoder_only_b200.gpt import GPT
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    mc = WL.model
+    B, T = WL.batch, WL.seq
+    tok, tgt, _ = S.make_batch(WL, seed=WL.data_seed + rank)
+    d_tok = torch.from_numpy(tok).to(dev)
+    d_tgt = torch.from_numpy(tgt).to(dev)
+    model = GPT(mc, WL.init_seed)
+    hp = WL.adamw
+    loss = torch.zeros(1, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        model.train_step(d_tok, d_tgt, None, hp, loss)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # warm-up (also fills the profiling event pool)
+    model.profile_enable(True)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    model.profile_enable(True)
+
+    # timed region: K steps, inputs resident in HBM (working set >> L2)
+    clocks = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    n0 = model.kernel_launches()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    n1 = model.kernel_launches()
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    clk = clocks.stop()
+    barrier()
+    prof = model.profile_read()
+    model.profile_enable(False)
+    final_loss = float(loss.item())
+    status = model.status()
+
+    tokens_per_step = B * T
+    value = world * tokens_per_step * args.steps / (ms / 1000.0)
+    ms_step = ms / args.steps
+    fpt = flops_per_token(mc, T)
+    peaks = load_peaks()
+    mfu = fpt * tokens_per_step / (ms_step / 1000.0) / (peaks["bf16_tflops"] * 1e12)
+    mfu_sust = fpt * tokens_per_step / (ms_step / 1000.0) / (peaks["bf16_tflops_sustained"] * 1e12)
+
+    # dominant kernel: the tcgen05 GEMMs (all GEMM launches of the step)
+    g_ms = sum(v["ms"] for k, v in prof.items() if k.startswith("gemm"))
+    g_fl = sum(v["flops"] for k, v in prof.items() if k.startswith("gemm"))
+    g_n = sum(v["launches"] for k, v in prof.items() if k.startswith("gemm"))
+    achieved = g_fl / (g_ms / 1000.0) / 1e12 if g_ms > 0 else 0.0
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"], "traffic": None,
+                "kernel": "gemm_tc (all GEMM launches)", "launches": g_n,
+                "avg_launch_ms": g_ms / max(1, g_n), "peak_source": peaks["source"] + " sustained"}
+    kernels = {k: {"launches": v["launches"], "ms_per_step": v["ms"] / args.steps,
+                   "share_of_step": v["ms"] / ms if ms > 0 else None,
+                   "tflops": (v["flops"] / (v["ms"] / 1000) / 1e12) if v["flops"] and v["ms"] else None,
+                   "gbs": (v["bytes"] / (v["ms"] / 1000) / 1e9) if v["bytes"] and v["ms"] else None,
+                   "hbm_frac": ((v["bytes"] / (v["ms"] / 1000) / 1e9) / peaks["hbm_gbs"])
+                   if v["bytes"] and v["ms"] else None}
+               for k, v in prof.items()}
+
+    # end-to-end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        h_tok = torch.from_numpy(tok).pin_memory()
+        h_tgt = torch.from_numpy(tgt).pin_memory()
+        h_loss = torch.zeros(1, dtype=torch.float32).pin_memory()
+        for _ in range(1):
+            d_tok.copy_(h_tok, non_blocking=True)
+            d_tgt.copy_(h_tgt, non_blocking=True)
+            step()
+            h_loss.copy_(loss, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier()
+        k2 = max(1, min(args.steps, 10))
+        e0.record(stream)
+        for _ in range(k2):
+            d_tok.copy_(h_tok, non_blocking=True)
+            d_tgt.copy_(h_tgt, non_blocking=True)
+            step()
+            h_loss.copy_(loss, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms2 = max_over_ranks(e0.elapsed_time(e1))
+        e2e = {"value": world * tokens_per_step * k2 / (ms2 / 1000.0), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h_tok.numel() * 4 + h_tgt.numel() * 4), "d2h_bytes_per_step": 4,
+               "steps": k2}
+
+    # greedy decode (secondary metric)
+    decode = None
+    if not args.no_decode:
+        decode = bench_decode(torch, dev, args)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, n, threads = oracle_sample_step()
+        cpu = {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": "1 row x 256 tokens of the GPT-2 124M step (fwd+bwd+clip+AdamW over all 124.5M "
+                         "params), numpy fp64, one step"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic (Zipf(1.0) tokens, random init)",
+                "config": {"workload": WL.name, "global_batch": B * world, "seq_len": T,
+                           "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                           "l2": "working set > L2 (no flush needed)"},
+                "mfu": mfu, "mfu_sustained_peak": mfu_sust, "flops_per_step": fpt * tokens_per_step,
+                "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": n1 - n0, "clocks": clk, "decode": decode,
+                "final_loss": final_loss, "status": status}
+        print(json.dumps(line), flush=True)
+    model.close()
+
+
+def bench_decode(torch, dev, args):
+    from scratch_decoder_only_b200.gpt import GPT
+    wl = CF.GPT2_DECODE
+    res = {}
+    model = GPT(wl.model, wl.init_seed)
+    for B in (1, 32):
+        prompt = torch.from_numpy(S.make_prompts(wl, B, 128)).to(dev)
+        out = torch.empty((B, 384), dtype=torch.int32, device=dev)
+        model.greedy_decode(prompt, 8, out[:, :8])
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        model.greedy_decode(prompt, 384, out)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        res[f"b{B}"] = {"tok_per_s": B * 384 / (ms / 1000.0), "ms": ms}
+    model.close()
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

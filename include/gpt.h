@@ -1,0 +1,257 @@
+/*
+ * gpt.h -- C ABI of libgpt.so: one training step of a GPT-style decoder-only
+ * transformer, and greedy decoding with a KV cache, on one NVIDIA B200
+ * (sm_100a).
+ *
+ * The calls follow the pages' statement of the problem: a language model is a
+ * function from the start of a text to a probability for every next token;
+ * generating means picking a token, appending it and repeating; training means
+ * raising the probability of the token that really came next ("Smallem -- Le
+ * projet et ses regles", section "Ce qu'est un modele de langage").
+ *
+ * Conventions for every call:
+ *  - Return value: 0 (GPT_OK) or a negative GPT_ERR_* code.  On error the
+ *    call has enqueued no work and gpt_last_error() describes the cause.
+ *  - Pointers documented as "device" must point to CUDA device memory of the
+ *    current device, owned by the caller, valid until the set stream reaches
+ *    the call.  Pointers documented as "host" are ordinary host memory.
+ *  - Work is enqueued asynchronously on the stream given to gpt_set_stream
+ *    (the default stream until then).  Only gpt_create, gpt_get_*,
+ *    gpt_set_*, gpt_status and gpt_greedy_decode's argument checks block.
+ *  - The library owns parameters, fp32 master weights, AdamW moments,
+ *    gradients, activations and the KV cache, in one device arena allocated
+ *    by gpt_create and freed by gpt_destroy.
+ *  - Bad token / target / segment ids found on the device are clamped (no
+ *    memory fault) and recorded in a sticky device error word, which
+ *    gpt_status reports (GPT_ERR_DEVICE) and clears.
+ *  - A model handle is not thread safe: one host thread at a time.
+ */
+#ifndef GPT_H_
+#define GPT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GPT_OK            0
+#define GPT_ERR_ARG      -1  /* NULL pointer, size out of range, bad config  */
+#define GPT_ERR_STATE    -2  /* call order violated (e.g. backward w/o loss) */
+#define GPT_ERR_CUDA     -3  /* a CUDA runtime call failed                   */
+#define GPT_ERR_TIMEOUT  -4  /* a bounded device-side wait gave up           */
+#define GPT_ERR_DEVICE   -5  /* sticky device flag: bad ids were clamped     */
+#define GPT_ERR_NOMEM    -6  /* the arena does not fit in device memory      */
+
+#define GPT_PRECISION_FP32 0
+#define GPT_PRECISION_BF16 1
+
+/* Device error word bits (reported through gpt_status / gpt_device_error). */
+#define GPT_DEVERR_TOKEN   1u   /* token id outside [0, vocab)                */
+#define GPT_DEVERR_TARGET  2u   /* target id outside [-1, vocab)              */
+#define GPT_DEVERR_SEGMENT 4u   /* seg_ids decrease inside a row              */
+#define GPT_DEVERR_TIMEOUT 8u   /* a bounded wait in a kernel gave up         */
+#define GPT_DEVERR_POS     16u  /* position beyond max_seq (decode)           */
+
+/*
+ * Model shape and numerics.  Architecture: token embedding plus a learned
+ * position embedding added to it, n_layers pre-LayerNorm blocks (causal
+ * multi-head attention, then a GELU MLP, each added back to the residual),
+ * a final LayerNorm and a projection to the vocabulary ("Feste: GPT-2 from
+ * scratch in Rust", section "Model Architecture mirrors GPT-2"; "LucilleAI",
+ * section "Architecture (from source)").
+ *
+ *  vocab          real vocabulary size V (softmax / argmax over 0..V-1)
+ *  vocab_padded   LM-head width Vp >= V; rows V..Vp-1 of the embedding and
+ *                 head are zero-initialised and receive zero gradient
+ *  d_model        C; must be a multiple of 8 and of n_heads, at most 1024
+ *  n_heads        H; head size d = C / H must be 16, 32, 64 or 128
+ *  d_mlp          F; multiple of 8
+ *  n_layers       L >= 1
+ *  max_seq        largest T (also the number of position-embedding rows)
+ *  max_batch      largest B accepted by gpt_forward_loss / decode
+ *  tied           1: the LM head reuses the token embedding matrix
+ *  precision      GPT_PRECISION_FP32 (fp32 everywhere, SIMT FFMA) or
+ *                 GPT_PRECISION_BF16 (bf16 GEMM/attention operands and
+ *                 activations, fp32 accumulate, fp32 master weights, moments
+ *                 and weight gradients; tcgen05 tensor cores)
+ *  loss_scaling   1: dynamic loss scale (x0.5 and skip on a non-finite
+ *                 gradient, x2 after 2000 finite steps); 0: scale fixed at 1
+ *                 (the non-finite skip stays on)
+ *  init_loss_scale  starting scale when loss_scaling = 1 (e.g. 32768)
+ *  ln_eps         LayerNorm epsilon (1e-5, biased variance)
+ *  init_std       std of the N(0, init_std) initial weight matrices (0.02)
+ */
+typedef struct {
+  int32_t vocab, vocab_padded, d_model, n_heads, d_mlp, n_layers, max_seq, max_batch;
+  int32_t tied, precision, loss_scaling;
+  float init_loss_scale;
+  float ln_eps, init_std;
+} gpt_config;
+
+/* AdamW with decoupled weight decay ("Feste", section "Manual
+ * Backpropagation from scratch") after global L2 clipping to clip_norm
+ * ("RustGPT", section "Technical implementation": L2 norm capped at 5.0):
+ * coef = min(1, clip_norm / (||g|| + 1e-6)).  Weight decay applies to every
+ * parameter. */
+typedef struct {
+  float lr, beta1, beta2, eps, weight_decay, clip_norm;
+} gpt_adamw;
+
+typedef struct gpt_model gpt_model;   /* opaque */
+
+/* Optimiser / loss-scale scalars, read back by gpt_get_scalars. */
+typedef struct {
+  float loss_scale;      /* current dynamic loss scale                       */
+  int32_t good_steps;    /* consecutive finite steps since the last change   */
+  int32_t step;          /* AdamW steps taken (skipped steps do not count)   */
+  float last_loss;       /* loss of the latest gpt_forward_loss with targets */
+  float last_grad_norm;  /* unscaled global L2 norm of the latest step       */
+  int32_t last_skipped;  /* 1 if the latest step was skipped (non-finite)    */
+} gpt_scalars;
+
+/* Validate cfg, size and allocate the device arena, initialise parameters
+ * from seed (weights N(0, init_std) drawn per canonical element from
+ * SplitMix64 + Box-Muller, LayerNorm gains 1, biases and shifts 0, padded
+ * vocabulary rows 0), and return a handle in *out.  Synchronous.
+ * Errors: GPT_ERR_ARG (bad cfg / NULL), GPT_ERR_NOMEM, GPT_ERR_CUDA. */
+int gpt_create(const gpt_config* cfg, uint64_t seed, gpt_model** out);
+
+/* Free the arena and the handle.  NULL is ignored.  Synchronises. */
+void gpt_destroy(gpt_model* m);
+
+/* Enqueue all later work on this cudaStream_t (NULL = legacy default). */
+int gpt_set_stream(gpt_model* m, void* cuda_stream);
+
+/* Forward pass over tokens [B, T] (device int32, row-major).
+ *  targets  device int32 [B, T]: next-token ids, -1 = ignored; NULL = no
+ *           loss (the logits of the last forward stay readable through
+ *           gpt_get_logits and no backward is possible).
+ *  seg_ids  device int32 [B, T]: document id of each token, non-decreasing
+ *           inside a row (sequence packing: a token attends only to earlier
+ *           tokens of its own document and its position restarts at 0 at
+ *           each document -- "LucilleAI", sections "What makes it special"
+ *           and "Real measured numbers"); NULL = one document per row.
+ *  loss_dev device float[1] receiving the mean cross-entropy over valid
+ *           targets ("RustGPT", "Technical implementation": cross-entropy
+ *           loss); may be NULL.
+ * Requires 1 <= B <= max_batch, 1 <= T <= max_seq.
+ * With targets the logits buffer is overwritten by the loss gradient. */
+int gpt_forward_loss(gpt_model* m, const int32_t* tokens, const int32_t* targets,
+                     const int32_t* seg_ids, int B, int T, float* loss_dev);
+
+/* Backward pass by the chain rule ("Feste", section "Manual Backpropagation
+ * from scratch") for the latest gpt_forward_loss with targets.  Overwrites
+ * all parameter gradients (fp32, canonical layout, multiplied by the current
+ * loss scale).  Errors: GPT_ERR_STATE if no forward with targets preceded. */
+int gpt_backward(gpt_model* m);
+
+/* Unscale, clip and update: g <- g / loss_scale; if any g is not finite the
+ * step is skipped (parameters and moments unchanged, scale halved when
+ * loss_scaling = 1); otherwise the global L2 norm is clipped and AdamW
+ * updates the fp32 master weights and refreshes the bf16 working copy.
+ *  grad_norm_dev  device float[1]: the unscaled global norm (may be NULL)
+ *  skipped_dev    device int32[1]: 1 if skipped, else 0 (may be NULL) */
+int gpt_clip_adamw_step(gpt_model* m, const gpt_adamw* hp, float* grad_norm_dev,
+                        int32_t* skipped_dev);
+
+/* Greedy decoding ("RustGPT", "Technical implementation": greedy decoding):
+ * prefill over prompt [B, Tp] (device int32), then n_new tokens, each the
+ * argmax (lowest index on ties) of the fp32 logits over 0..V-1 at the last
+ * position, appended and fed back through a per-layer KV cache.
+ *  out  device int32 [B, n_new].
+ * Requires 1 <= B <= max_batch, Tp >= 1, n_new >= 1, Tp + n_new - 1 <= max_seq.
+ * Errors: GPT_ERR_ARG, GPT_ERR_STATE (sequence too long). */
+int gpt_greedy_decode(gpt_model* m, const int32_t* prompt, int B, int Tp, int n_new,
+                      int32_t* out);
+
+/* Number of parameters N in the canonical layout:
+ *  wte[Vp,C], wpe[max_seq,C]; per layer ln1_g[C], ln1_b[C], w_qkv[3C,C]
+ *  (rows: q, then k, then v; head h = rows h*d..h*d+d-1 of each), b_qkv[3C],
+ *  w_o[C,C], b_o[C], ln2_g[C], ln2_b[C], w_fc[F,C], b_fc[F], w_fc2[C,F],
+ *  b_fc2[C]; then lnf_g[C], lnf_b[C]; then w_head[Vp,C] only if untied. */
+int gpt_num_params(const gpt_model* m, size_t* n);
+
+/* Copy N fp32 values (canonical layout) between the library and dst/src,
+ * which may be host or device memory (cudaMemcpyDefault).  Synchronous.
+ * n must equal gpt_num_params.
+ *  gpt_get_params / gpt_set_params : fp32 master weights (set also refreshes
+ *                                    the bf16 working copy)
+ *  gpt_get_grads  / gpt_set_grads  : gradients as stored (x loss scale)
+ *  gpt_get_adam_m / gpt_set_adam_m, gpt_get_adam_v / gpt_set_adam_v : moments */
+int gpt_get_params(gpt_model* m, float* dst, size_t n);
+int gpt_set_params(gpt_model* m, const float* src, size_t n);
+int gpt_get_grads(gpt_model* m, float* dst, size_t n);
+int gpt_set_grads(gpt_model* m, const float* src, size_t n);
+int gpt_get_adam_m(gpt_model* m, float* dst, size_t n);
+int gpt_set_adam_m(gpt_model* m, const float* src, size_t n);
+int gpt_get_adam_v(gpt_model* m, float* dst, size_t n);
+int gpt_set_adam_v(gpt_model* m, const float* src, size_t n);
+
+/* Copy the logits of the latest gpt_forward_loss called with targets = NULL,
+ * as fp32 [B*T, Vp] row-major, to dst (host or device).  n = B*T*Vp.
+ * Synchronous.  Errors: GPT_ERR_STATE if those logits were overwritten. */
+int gpt_get_logits(gpt_model* m, float* dst, size_t n);
+
+/* Copy the residual stream entering block `layer` of the latest forward
+ * (layer 0: the embedding sum wte[tok] + wpe[pos]; layer = n_layers: the
+ * input of the final LayerNorm) as fp32 [B*T, C] to dst (host or device).
+ * n = B*T*C.  Synchronous.  Errors: GPT_ERR_ARG (layer or n out of range),
+ * GPT_ERR_STATE (no forward yet). */
+int gpt_get_residual(gpt_model* m, int layer, float* dst, size_t n);
+
+/* Read / write the optimiser and loss-scale scalars.  Synchronous. */
+int gpt_get_scalars(gpt_model* m, gpt_scalars* out);
+int gpt_set_scalars(gpt_model* m, const gpt_scalars* in);
+
+/* Synchronise the stream, then return GPT_OK, GPT_ERR_CUDA, GPT_ERR_TIMEOUT
+ * or GPT_ERR_DEVICE from the sticky device error word, which is cleared. */
+int gpt_status(gpt_model* m);
+
+/* The sticky device error word (GPT_DEVERR_* bits) without clearing it.
+ * Synchronous. */
+int gpt_device_error(gpt_model* m, uint32_t* bits);
+
+/* Human-readable description of the last error on this handle ("" if none).
+ * The string lives until the next call on the handle. */
+const char* gpt_last_error(const gpt_model* m);
+
+/* Number of kernels libgpt has launched in this process (all handles).
+ * Benchmarks read it before and after a timed region. */
+int gpt_kernel_launches(uint64_t* out);
+
+/* Per-kernel-class device timing (tracing).  While enabled, every GEMM,
+ * attention, cross-entropy, LayerNorm and optimiser launch of later calls on
+ * this handle is bracketed by CUDA events recorded on the handle's stream,
+ * together with its algorithmic FLOPs and HBM bytes.  gpt_profile_enable(m, 1)
+ * starts a fresh record, (m, 0) stops recording and keeps the record. */
+typedef struct {
+  char name[24];      /* gemm_fwd, gemm_dgrad, gemm_wgrad, attn_fwd, attn_bwd,
+                         xent, ln_fwd, ln_bwd, clip_adamw                      */
+  int32_t launches;   /* bracketed calls                                      */
+  double ms;          /* summed event time                                    */
+  double flops;       /* summed algorithmic FLOPs (0 where not applicable)    */
+  double bytes;       /* summed algorithmic HBM bytes (0 where not applicable) */
+} gpt_prof_entry;
+int gpt_profile_enable(gpt_model* m, int on);
+
+/* Synchronise and summarise the record into out[0..max_entries), one entry
+ * per class with launches > 0; *n_out receives the number written. */
+int gpt_profile_read(gpt_model* m, gpt_prof_entry* out, int max_entries, int* n_out);
+
+/* Fault injection for tests: write value into gradient element index
+ * (e.g. +inf to exercise the skip path).  Synchronous, host-side. */
+int gpt_debug_poison_grad(gpt_model* m, size_t index, float value);
+
+/* Exercise a bounded device-side wait that can never complete: a kernel
+ * waits on a shared-memory mbarrier that nothing arrives on, gives up after
+ * about timeout_us microseconds, sets GPT_DEVERR_TIMEOUT and returns.  The
+ * call synchronises and returns GPT_ERR_TIMEOUT when the wait gave up as
+ * designed (the context stays usable).  For the failure-detection tests. */
+int gpt_debug_wait_timeout(gpt_model* m, int timeout_us);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GPT_H_ */

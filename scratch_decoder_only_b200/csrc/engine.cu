@@ -1,0 +1,882 @@
+// libgpt engine: the device arena, parameter initialisation, the forward /
+// backward / optimiser schedule of one training step, greedy decoding, and
+// the C ABI declared in include/gpt.h.
+//
+// Everything of a step is enqueued on one stream; nothing returns to the host
+// during a step (loss, grad norm, skip flag and loss scale live in device
+// scalars).  Layouts (row-major):
+//   parameters  fp32 master p32[N] in canonical order (see gpt.h); gradients,
+//               AdamW m and v share that layout; bf16 mode adds a bf16 working
+//               copy pw[N] that every GEMM reads.
+//   activations [B*T, C] per layer: x (residual input), h1 = LN1(x), qkv
+//               [B*T, 3C], att, x_mid, h2 = LN2(x_mid), u = pre-GELU [B*T, F],
+//               a = GELU(u); LayerNorm mean / rstd [B*T] fp32; lse [B, H, T].
+//   logits      [B*T, ldl], ldl = Vp rounded up to 8 (16-byte rows for TMA);
+//               overwritten in place by the loss gradient.
+#include <string.h>
+#include <math.h>
+#include <string>
+#include <vector>
+#include <thread>
+#include <algorithm>
+#include "gpt.h"
+#include "launch.h"
+
+struct LayerOff {
+  size_t ln1_g, ln1_b, w_qkv, b_qkv, w_o, b_o, ln2_g, ln2_b, w_fc, b_fc, w_fc2, b_fc2;
+};
+
+struct gpt_model {
+  gpt_config cfg;
+  int device = 0;
+  cudaStream_t stream = 0;
+  bool bf16 = false;
+  int V, Vp, C, H, d, F, NL, Tmax, Bmax, ldl;
+  long Mmax;
+  size_t N = 0;
+  size_t o_wte, o_wpe, o_lnf_g, o_lnf_b, o_head;
+  std::vector<LayerOff> L;
+  char* arena = nullptr;
+  size_t arena_bytes = 0;
+  float *p32, *g32, *m32, *v32;
+  void* pw;
+  void *xs, *xmid, *h1, *h2, *qkv, *att, *u, *a, *xf, *logits;
+  float *mu1, *rs1, *mu2, *rs2, *muf, *rsf, *lse;
+  int *tok, *tgt, *pos, *dstart;
+  float* dres32;
+  void *dres_t, *dC, *dF, *dqkv;
+  float *attD, *rowloss, *partials, *splitws;
+  size_t partials_n, splitws_n;
+  double* normpart;
+  int normblk = 592;
+  DevScalars* sc;
+  void *kc, *vc, *dx, *dh, *dq, *datt, *du, *da, *dxf;
+  float *dlogits, *dmu, *drs;
+  int* dtok;
+  int fwd_B = 0, fwd_T = 0;
+  bool have_targets = false, logits_valid = false;
+  std::string err;
+  // tracing: per-kernel-class CUDA-event brackets
+  bool seg_used = false;
+  bool prof = false;
+  struct ProfRec { int cls; cudaEvent_t a, b; double flops, bytes; };
+  std::vector<ProfRec> recs;
+  std::vector<cudaEvent_t> evpool;
+  size_t evused = 0;
+};
+
+enum ProfCls { PC_GEMM_FWD, PC_GEMM_DX, PC_GEMM_DW, PC_ATTN_FWD, PC_ATTN_BWD, PC_XENT, PC_LN_FWD, PC_LN_BWD,
+               PC_OPT, PC_COUNT };
+static const char* kProfNames[PC_COUNT] = {"gemm_fwd", "gemm_dgrad", "gemm_wgrad", "attn_fwd", "attn_bwd",
+                                           "xent", "ln_fwd", "ln_bwd", "clip_adamw"};
+
+static cudaEvent_t prof_event(gpt_model* m) {
+  if (m->evused == m->evpool.size()) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    m->evpool.push_back(e);
+  }
+  return m->evpool[m->evused++];
+}
+
+// Brackets the launches made during its lifetime with two events.
+struct ProfScope {
+  gpt_model* m;
+  long idx = -1;
+  ProfScope(gpt_model* mm, int cls, double flops, double bytes) : m(mm) {
+    if (!m->prof) return;
+    cudaEvent_t a = prof_event(m);
+    if (!a) return;
+    cudaEventRecord(a, m->stream);
+    m->recs.push_back({cls, a, nullptr, flops, bytes});
+    idx = (long)m->recs.size() - 1;
+  }
+  ~ProfScope() {
+    if (idx < 0) return;
+    cudaEvent_t b = prof_event(m);
+    if (!b) { m->recs.pop_back(); return; }
+    cudaEventRecord(b, m->stream);
+    m->recs[idx].b = b;
+  }
+};
+
+#define FAIL(code, msg)            \
+  do {                             \
+    m->err = (msg);                \
+    return (code);                 \
+  } while (0)
+#define CK(x)                                                                       \
+  do {                                                                              \
+    cudaError_t e_ = (x);                                                           \
+    if (e_ != cudaSuccess) {                                                        \
+      m->err = std::string(#x) + ": " + cudaGetErrorString(e_);                     \
+      return GPT_ERR_CUDA;                                                          \
+    }                                                                               \
+  } while (0)
+#define CKI(x)                   \
+  do {                           \
+    int r_ = (x);                \
+    if (r_ != GPT_OK) return r_; \
+  } while (0)
+
+// ---------------------------------------------------------------------------
+// Parameter layout and initialisation
+// ---------------------------------------------------------------------------
+static void layout_params(gpt_model* m) {
+  size_t o = 0;
+  size_t C = m->C, F = m->F, Vp = m->Vp;
+  m->o_wte = o; o += Vp * C;
+  m->o_wpe = o; o += (size_t)m->Tmax * C;
+  m->L.resize(m->NL);
+  for (int l = 0; l < m->NL; ++l) {
+    LayerOff& lo = m->L[l];
+    lo.ln1_g = o; o += C;
+    lo.ln1_b = o; o += C;
+    lo.w_qkv = o; o += 3 * C * C;
+    lo.b_qkv = o; o += 3 * C;
+    lo.w_o = o; o += C * C;
+    lo.b_o = o; o += C;
+    lo.ln2_g = o; o += C;
+    lo.ln2_b = o; o += C;
+    lo.w_fc = o; o += F * C;
+    lo.b_fc = o; o += F;
+    lo.w_fc2 = o; o += C * F;
+    lo.b_fc2 = o; o += C;
+  }
+  m->o_lnf_g = o; o += C;
+  m->o_lnf_b = o; o += C;
+  if (m->cfg.tied) {
+    m->o_head = m->o_wte;
+  } else {
+    m->o_head = o; o += Vp * C;
+  }
+  m->N = o;
+}
+
+// SplitMix64 output k for a seed (Steele, Lea, Flood 2014; Vigna's reference
+// splitmix64.c): state after k+1 golden-ratio increments, then the finaliser.
+static inline uint64_t splitmix64_at(uint64_t seed, uint64_t k) {
+  uint64_t z = seed + (k + 1) * 0x9E3779B97F4A7C15ULL;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+  return z ^ (z >> 31);
+}
+
+// Box-Muller (1958) normal deviate for canonical element e, from draws 2e, 2e+1.
+static inline double normal_at(uint64_t seed, uint64_t e) {
+  uint64_t x1 = splitmix64_at(seed, 2 * e), x2 = splitmix64_at(seed, 2 * e + 1);
+  double u1 = ((double)(x1 >> 11) + 1.0) * 0x1.0p-53;
+  double u2 = (double)(x2 >> 11) * 0x1.0p-53;
+  return sqrt(-2.0 * log(u1)) * cos(2.0 * M_PI * u2);
+}
+
+static void fill_normal(std::vector<float>& h, size_t off, size_t n, uint64_t seed, double stddev) {
+  unsigned nt = std::max(1u, std::min(32u, std::thread::hardware_concurrency()));
+  if (n < 65536) nt = 1;
+  std::vector<std::thread> th;
+  for (unsigned t = 0; t < nt; ++t) {
+    size_t a = off + n * t / nt, b = off + n * (t + 1) / nt;
+    th.emplace_back([&h, a, b, seed, stddev]() {
+      for (size_t e = a; e < b; ++e) h[e] = (float)(stddev * normal_at(seed, e));
+    });
+  }
+  for (auto& x : th) x.join();
+}
+
+static void init_host_params(gpt_model* m, uint64_t seed, std::vector<float>& h) {
+  h.assign(m->N, 0.f);
+  size_t C = m->C, F = m->F;
+  double sd = m->cfg.init_std;
+  auto zero_pad_rows = [&](size_t off) {
+    for (size_t r = (size_t)m->V; r < (size_t)m->Vp; ++r)
+      for (size_t c = 0; c < C; ++c) h[off + r * C + c] = 0.f;
+  };
+  fill_normal(h, m->o_wte, (size_t)m->Vp * C, seed, sd);
+  zero_pad_rows(m->o_wte);
+  fill_normal(h, m->o_wpe, (size_t)m->Tmax * C, seed, sd);
+  for (auto& lo : m->L) {
+    for (size_t i = 0; i < C; ++i) { h[lo.ln1_g + i] = 1.f; h[lo.ln2_g + i] = 1.f; }
+    fill_normal(h, lo.w_qkv, 3 * C * C, seed, sd);
+    fill_normal(h, lo.w_o, C * C, seed, sd);
+    fill_normal(h, lo.w_fc, F * C, seed, sd);
+    fill_normal(h, lo.w_fc2, C * F, seed, sd);
+  }
+  for (size_t i = 0; i < C; ++i) h[m->o_lnf_g + i] = 1.f;
+  if (!m->cfg.tied) {
+    fill_normal(h, m->o_head, (size_t)m->Vp * C, seed, sd);
+    zero_pad_rows(m->o_head);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Arena
+// ---------------------------------------------------------------------------
+struct Carver {
+  size_t off = 0;
+  std::vector<std::pair<void**, size_t>> items;
+  void add(void** p, size_t bytes) {
+    off = (off + 255) & ~(size_t)255;
+    items.push_back({p, off});
+    off += bytes;
+  }
+};
+
+static int build_arena(gpt_model* m) {
+  size_t es = m->bf16 ? 2 : 4;
+  size_t N = m->N, C = m->C, F = m->F, Mx = m->Mmax, NL = m->NL;
+  Carver cv;
+  cv.add((void**)&m->p32, N * 4);
+  cv.add((void**)&m->g32, N * 4);
+  cv.add((void**)&m->m32, N * 4);
+  cv.add((void**)&m->v32, N * 4);
+  if (m->bf16) cv.add(&m->pw, N * es);
+  cv.add(&m->xs, (NL + 1) * Mx * C * es);
+  cv.add(&m->xmid, NL * Mx * C * es);
+  cv.add(&m->h1, NL * Mx * C * es);
+  cv.add(&m->h2, NL * Mx * C * es);
+  cv.add(&m->qkv, NL * Mx * 3 * C * es);
+  cv.add(&m->att, NL * Mx * C * es);
+  cv.add(&m->u, NL * Mx * F * es);
+  cv.add(&m->a, NL * Mx * F * es);
+  cv.add(&m->xf, Mx * C * es);
+  cv.add(&m->logits, Mx * (size_t)m->ldl * es);
+  cv.add((void**)&m->mu1, NL * Mx * 4);
+  cv.add((void**)&m->rs1, NL * Mx * 4);
+  cv.add((void**)&m->mu2, NL * Mx * 4);
+  cv.add((void**)&m->rs2, NL * Mx * 4);
+  cv.add((void**)&m->muf, Mx * 4);
+  cv.add((void**)&m->rsf, Mx * 4);
+  cv.add((void**)&m->lse, NL * Mx * m->H * 4);
+  cv.add((void**)&m->tok, Mx * 4);
+  cv.add((void**)&m->tgt, Mx * 4);
+  cv.add((void**)&m->pos, Mx * 4);
+  cv.add((void**)&m->dstart, Mx * 4);
+  cv.add((void**)&m->dres32, Mx * C * 4);
+  cv.add(&m->dres_t, Mx * C * es);
+  cv.add(&m->dC, Mx * C * es);
+  cv.add(&m->dF, Mx * F * es);
+  cv.add(&m->dqkv, Mx * 3 * C * es);
+  cv.add((void**)&m->attD, Mx * m->H * 4);
+  cv.add((void**)&m->rowloss, Mx * 4);
+  m->partials_n = std::max((size_t)296 * 2 * C, (size_t)128 * std::max(3 * C, F));
+  cv.add((void**)&m->partials, m->partials_n * 4);
+  m->splitws_n = m->bf16 ? (size_t)8 * std::max(3 * C * C, F * C) : 0;
+  if (m->splitws_n) cv.add((void**)&m->splitws, m->splitws_n * 4);
+  else m->splitws = nullptr;
+  cv.add((void**)&m->normpart, m->normblk * 8);
+  cv.add((void**)&m->sc, sizeof(DevScalars));
+  size_t Bx = m->Bmax;
+  size_t kvn = NL * Bx * m->H * (size_t)m->Tmax * m->d;
+  cv.add(&m->kc, kvn * es);
+  cv.add(&m->vc, kvn * es);
+  cv.add(&m->dx, Bx * C * es);
+  cv.add(&m->dh, Bx * C * es);
+  cv.add(&m->dq, Bx * 3 * C * es);
+  cv.add(&m->datt, Bx * C * es);
+  cv.add(&m->du, Bx * F * es);
+  cv.add(&m->da, Bx * F * es);
+  cv.add(&m->dxf, Bx * C * es);
+  cv.add((void**)&m->dlogits, Bx * m->Vp * 4);
+  cv.add((void**)&m->dmu, Bx * 4);
+  cv.add((void**)&m->drs, Bx * 4);
+  cv.add((void**)&m->dtok, Bx * 4);
+  m->arena_bytes = cv.off + 256;
+  cudaError_t e = cudaMalloc((void**)&m->arena, m->arena_bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    m->arena = nullptr;
+    m->err = std::string("cudaMalloc of the arena (") + std::to_string(m->arena_bytes) +
+             " bytes) failed: " + cudaGetErrorString(e);
+    return GPT_ERR_NOMEM;
+  }
+  for (auto& it : cv.items) *it.first = m->arena + it.second;
+  if (!m->bf16) m->pw = m->p32;
+  return GPT_OK;
+}
+
+// ---------------------------------------------------------------------------
+// GEMM and attention dispatch
+// ---------------------------------------------------------------------------
+template <typename T>
+static EpiParams<T> epi_none() {
+  EpiParams<T> e;
+  memset(&e, 0, sizeof(e));
+  return e;
+}
+template <typename T>
+static EpiParams<T> epi_store(T* out, long ld, const float* bias, const T* resid, long ldr) {
+  EpiParams<T> e = epi_none<T>();
+  e.kind = EPI_STORE; e.out = out; e.ld_out = ld; e.bias = bias; e.resid = resid; e.ld_resid = ldr;
+  return e;
+}
+template <typename T>
+static EpiParams<T> epi_gelu(T* u, T* a, long ld, const float* bias) {
+  EpiParams<T> e = epi_none<T>();
+  e.kind = EPI_GELU; e.out = u; e.ld_out = ld; e.out2 = a; e.ld_out2 = ld; e.bias = bias;
+  return e;
+}
+template <typename T>
+static EpiParams<T> epi_dgelu(T* out, long ld, const T* u) {
+  EpiParams<T> e = epi_none<T>();
+  e.kind = EPI_DGELU; e.out = out; e.ld_out = ld; e.aux = u; e.ld_aux = ld;
+  return e;
+}
+template <typename T>
+static EpiParams<T> epi_f32(float* out, long ld) {
+  EpiParams<T> e = epi_none<T>();
+  e.kind = EPI_F32; e.outf = out; e.ld_outf = ld;
+  return e;
+}
+
+static int g_num_sms = 148;
+
+// C[M,N] = A(M x K) . B(N x K)^T; see launch.h for the operand conventions.
+static int gemm_cls(bool a_t, bool b_t) { return a_t ? PC_GEMM_DW : (b_t ? PC_GEMM_DX : PC_GEMM_FWD); }
+
+static int gemm(gpt_model* m, int M, int N, int K, const float* A, long lda, bool a_t, const float* B,
+                long ldb, bool b_t, EpiParams<float> epi) {
+  ProfScope ps(m, gemm_cls(a_t, b_t), 2.0 * M * N * K, 0.0);
+  CK(launch_gemm_simt<float>(M, N, K, A, lda, a_t, B, ldb, b_t, epi, 1, m->stream));
+  return GPT_OK;
+}
+
+static int gemm(gpt_model* m, int M, int N, int K, const bf16* A, long lda, bool a_t, const bf16* B,
+                long ldb, bool b_t, EpiParams<bf16> epi) {
+  ProfScope ps(m, gemm_cls(a_t, b_t), 2.0 * M * N * K, 0.0);
+  if (!gemm_tc_supported(M, N, K, lda, a_t, ldb, b_t)) {
+    CK(launch_gemm_simt<bf16>(M, N, K, A, lda, a_t, B, ldb, b_t, epi, 1, m->stream));
+    return GPT_OK;
+  }
+  int splits = 1;
+  if (epi.kind == EPI_F32) {
+    long tiles = (long)((M + 127) / 128) * ((N + 255) / 256);
+    while (splits < 8 && tiles * splits * 2 <= g_num_sms * 2 && K / (splits * 2) >= 512 &&
+           (size_t)(splits * 2) * M * N <= m->splitws_n)
+      splits *= 2;
+  }
+  if (splits > 1) {
+    EpiParams<bf16> e2 = epi;
+    e2.kind = EPI_F32_SPLIT;
+    e2.outf = m->splitws;
+    e2.ld_outf = N;
+    e2.split_stride = (long)M * N;
+    CK(launch_gemm_tc(M, N, K, A, lda, a_t, B, ldb, b_t, e2, splits, &m->sc->err, m->stream));
+    if (epi.ld_outf != N) FAIL(GPT_ERR_ARG, "split-K output must be dense");
+    CK(launch_sum_splits(m->splitws, splits, (long)M * N, (long)M * N, epi.outf, m->stream));
+  } else {
+    CK(launch_gemm_tc(M, N, K, A, lda, a_t, B, ldb, b_t, epi, 1, &m->sc->err, m->stream));
+  }
+  return GPT_OK;
+}
+
+static double attn_pairs(int B, int T, int H, bool seg) { return seg ? 0.0 : (double)B * H * T * (T + 1) / 2.0; }
+
+static int attn_fwd(gpt_model* m, const float* qkv, float* out, float* lse, int B, int T) {
+  ProfScope ps(m, PC_ATTN_FWD, 4.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0);
+  CK(launch_attn_fwd_simt<float>(qkv, out, lse, m->dstart, B, T, m->H, m->d, m->stream));
+  return GPT_OK;
+}
+static int attn_fwd(gpt_model* m, const bf16* qkv, bf16* out, float* lse, int B, int T) {
+  ProfScope ps(m, PC_ATTN_FWD, 4.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0);
+  if (attn_mma_supported(m->d)) CK(launch_attn_fwd_mma(qkv, out, lse, m->dstart, B, T, m->H, m->d, m->stream));
+  else CK(launch_attn_fwd_simt<bf16>(qkv, out, lse, m->dstart, B, T, m->H, m->d, m->stream));
+  return GPT_OK;
+}
+static int attn_bwd(gpt_model* m, const float* qkv, const float* out, const float* dout, const float* lse,
+                    float* dqkv, int B, int T) {
+  ProfScope ps(m, PC_ATTN_BWD, 8.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0);
+  CK(launch_attn_bwd_simt<float>(qkv, out, dout, lse, m->attD, m->dstart, dqkv, B, T, m->H, m->d, m->stream));
+  return GPT_OK;
+}
+static int attn_bwd(gpt_model* m, const bf16* qkv, const bf16* out, const bf16* dout, const float* lse,
+                    bf16* dqkv, int B, int T) {
+  ProfScope ps(m, PC_ATTN_BWD, 8.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0);
+  if (attn_mma_supported(m->d))
+    CK(launch_attn_bwd_mma(qkv, out, dout, lse, m->attD, m->dstart, dqkv, B, T, m->H, m->d, m->stream));
+  else
+    CK(launch_attn_bwd_simt<bf16>(qkv, out, dout, lse, m->attD, m->dstart, dqkv, B, T, m->H, m->d, m->stream));
+  return GPT_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Forward, loss, backward
+// ---------------------------------------------------------------------------
+template <typename T>
+struct Acts {
+  gpt_model* m;
+  size_t MC, M3C, MF, Mx;
+  explicit Acts(gpt_model* mm) : m(mm) {
+    Mx = m->Mmax; MC = Mx * m->C; M3C = 3 * MC; MF = Mx * m->F;
+  }
+  T* x(int l) const { return (T*)m->xs + l * MC; }
+  T* xmid(int l) const { return (T*)m->xmid + l * MC; }
+  T* h1(int l) const { return (T*)m->h1 + l * MC; }
+  T* h2(int l) const { return (T*)m->h2 + l * MC; }
+  T* qkv(int l) const { return (T*)m->qkv + l * M3C; }
+  T* att(int l) const { return (T*)m->att + l * MC; }
+  T* u(int l) const { return (T*)m->u + l * MF; }
+  T* a(int l) const { return (T*)m->a + l * MF; }
+  float* mu1(int l) const { return m->mu1 + l * Mx; }
+  float* rs1(int l) const { return m->rs1 + l * Mx; }
+  float* mu2(int l) const { return m->mu2 + l * Mx; }
+  float* rs2(int l) const { return m->rs2 + l * Mx; }
+  float* lse(int l) const { return m->lse + l * Mx * m->H; }
+  const T* W(size_t off) const { return (const T*)m->pw + off; }
+  const float* P(size_t off) const { return m->p32 + off; }
+  float* G(size_t off) const { return m->g32 + off; }
+};
+
+template <typename T>
+static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targets, const int32_t* seg, int B,
+                        int T_, float* loss_dev) {
+  cudaStream_t s = m->stream;
+  Acts<T> A(m);
+  const int M = B * T_, C = m->C, F = m->F;
+  const float eps = m->cfg.ln_eps;
+  const double es = sizeof(T), lnb = (double)M * C * 2 * es + 8.0 * M;
+  m->seg_used = seg != nullptr;
+  CK(launch_prep(tokens, targets, seg, B, T_, m->V, m->tok, m->tgt, m->pos, m->dstart, m->sc, s));
+  CK(launch_embed_fwd<T>(m->tok, m->pos, A.P(m->o_wte), A.P(m->o_wpe), A.x(0), M, C, s));
+  for (int l = 0; l < m->NL; ++l) {
+    const LayerOff& lo = m->L[l];
+    { ProfScope ps(m, PC_LN_FWD, 0, lnb);
+      CK(launch_ln_fwd<T>(A.x(l), A.P(lo.ln1_g), A.P(lo.ln1_b), A.h1(l), A.mu1(l), A.rs1(l), M, C, eps, s)); }
+    CKI(gemm(m, M, 3 * C, C, A.h1(l), C, false, A.W(lo.w_qkv), C, false,
+             epi_store<T>(A.qkv(l), 3 * C, A.P(lo.b_qkv), nullptr, 0)));
+    CKI(attn_fwd(m, A.qkv(l), A.att(l), A.lse(l), B, T_));
+    CKI(gemm(m, M, C, C, A.att(l), C, false, A.W(lo.w_o), C, false,
+             epi_store<T>(A.xmid(l), C, A.P(lo.b_o), A.x(l), C)));
+    { ProfScope ps(m, PC_LN_FWD, 0, lnb);
+      CK(launch_ln_fwd<T>(A.xmid(l), A.P(lo.ln2_g), A.P(lo.ln2_b), A.h2(l), A.mu2(l), A.rs2(l), M, C, eps, s)); }
+    CKI(gemm(m, M, F, C, A.h2(l), C, false, A.W(lo.w_fc), C, false,
+             epi_gelu<T>(A.u(l), A.a(l), F, A.P(lo.b_fc))));
+    CKI(gemm(m, M, C, F, A.a(l), F, false, A.W(lo.w_fc2), F, false,
+             epi_store<T>(A.x(l + 1), C, A.P(lo.b_fc2), A.xmid(l), C)));
+  }
+  { ProfScope ps(m, PC_LN_FWD, 0, lnb);
+    CK(launch_ln_fwd<T>(A.x(m->NL), A.P(m->o_lnf_g), A.P(m->o_lnf_b), (T*)m->xf, m->muf, m->rsf, M, C, eps, s)); }
+  CKI(gemm(m, M, m->Vp, C, (const T*)m->xf, C, false, A.W(m->o_head), C, false,
+           epi_store<T>((T*)m->logits, m->ldl, nullptr, nullptr, 0)));
+  if (targets) {
+    ProfScope ps(m, PC_XENT, 0, 2.0 * es * M * m->Vp);
+    CK(launch_xent<T>((T*)m->logits, m->ldl, m->tgt, M, m->V, m->Vp, m->rowloss, m->sc, s));
+    CK(launch_loss_finalize(m->rowloss, M, m->sc, loss_dev, s));
+  }
+  m->fwd_B = B;
+  m->fwd_T = T_;
+  m->have_targets = targets != nullptr;
+  m->logits_valid = targets == nullptr;
+  return GPT_OK;
+}
+
+template <typename T>
+static int backward_impl(gpt_model* m) {
+  cudaStream_t s = m->stream;
+  Acts<T> A(m);
+  const int B = m->fwd_B, T_ = m->fwd_T, M = B * T_, C = m->C, F = m->F, Vp = m->Vp;
+  T* dC = (T*)m->dC;
+  T* dF = (T*)m->dF;
+  T* dq = (T*)m->dqkv;
+  T* drt = (T*)m->dres_t;
+  const T* dz = (const T*)m->logits;
+  const T* xf = (const T*)m->xf;
+  int nblk = 0;
+  const double es = sizeof(T), lnbb = (double)M * C * (3 * es + 8) + 8.0 * M;
+  // LM head: dxf = dz . W_head;  dW_head = dz^T . xf  (into dwte when tied)
+  CKI(gemm(m, M, C, Vp, dz, m->ldl, false, A.W(m->o_head), C, true, epi_store<T>(dC, C, nullptr, nullptr, 0)));
+  CKI(gemm(m, Vp, C, M, dz, m->ldl, true, xf, C, true, epi_f32<T>(A.G(m->o_head), C)));
+  { ProfScope ps(m, PC_LN_BWD, 0, lnbb);
+    CK(launch_ln_bwd<T>(dC, A.x(m->NL), m->muf, m->rsf, A.P(m->o_lnf_g), nullptr, m->dres32, drt, m->partials,
+                      M, C, &nblk, s));
+    CK(launch_reduce_rows(m->partials, nblk, 2 * C, A.G(m->o_lnf_g), s)); }
+  for (int l = m->NL - 1; l >= 0; --l) {
+    const LayerOff& lo = m->L[l];
+    // MLP: x_out = x_mid + gelu(h2 W_fc^T + b_fc) W_fc2^T + b_fc2
+    CK(launch_colsum<float>(m->dres32, C, M, C, m->partials, A.G(lo.b_fc2), s));
+    CKI(gemm(m, C, F, M, drt, C, true, A.a(l), F, true, epi_f32<T>(A.G(lo.w_fc2), F)));
+    CKI(gemm(m, M, F, C, drt, C, false, A.W(lo.w_fc2), F, true, epi_dgelu<T>(dF, F, A.u(l))));
+    CK(launch_colsum<T>(dF, F, M, F, m->partials, A.G(lo.b_fc), s));
+    CKI(gemm(m, F, C, M, dF, F, true, A.h2(l), C, true, epi_f32<T>(A.G(lo.w_fc), C)));
+    CKI(gemm(m, M, C, F, dF, F, false, A.W(lo.w_fc), C, true, epi_store<T>(dC, C, nullptr, nullptr, 0)));
+    { ProfScope ps(m, PC_LN_BWD, 0, lnbb);
+      CK(launch_ln_bwd<T>(dC, A.xmid(l), A.mu2(l), A.rs2(l), A.P(lo.ln2_g), m->dres32, m->dres32, drt,
+                          m->partials, M, C, &nblk, s));
+      CK(launch_reduce_rows(m->partials, nblk, 2 * C, A.G(lo.ln2_g), s)); }
+    // attention: x_mid = x + attn(h1 W_qkv^T + b_qkv) W_o^T + b_o
+    CK(launch_colsum<float>(m->dres32, C, M, C, m->partials, A.G(lo.b_o), s));
+    CKI(gemm(m, C, C, M, drt, C, true, A.att(l), C, true, epi_f32<T>(A.G(lo.w_o), C)));
+    CKI(gemm(m, M, C, C, drt, C, false, A.W(lo.w_o), C, true, epi_store<T>(dC, C, nullptr, nullptr, 0)));
+    CKI(attn_bwd(m, A.qkv(l), A.att(l), dC, A.lse(l), dq, B, T_));
+    CK(launch_colsum<T>(dq, 3 * C, M, 3 * C, m->partials, A.G(lo.b_qkv), s));
+    CKI(gemm(m, 3 * C, C, M, dq, 3 * C, true, A.h1(l), C, true, epi_f32<T>(A.G(lo.w_qkv), C)));
+    CKI(gemm(m, M, C, 3 * C, dq, 3 * C, false, A.W(lo.w_qkv), C, true, epi_store<T>(dC, C, nullptr, nullptr, 0)));
+    { ProfScope ps(m, PC_LN_BWD, 0, lnbb);
+      CK(launch_ln_bwd<T>(dC, A.x(l), A.mu1(l), A.rs1(l), A.P(lo.ln1_g), m->dres32, m->dres32, drt,
+                          m->partials, M, C, &nblk, s));
+      CK(launch_reduce_rows(m->partials, nblk, 2 * C, A.G(lo.ln1_g), s)); }
+  }
+  // embeddings: scatter-add by token and by position
+  if (!m->cfg.tied) CK(cudaMemsetAsync(A.G(m->o_wte), 0, (size_t)Vp * C * 4, s));
+  CK(cudaMemsetAsync(A.G(m->o_wpe), 0, (size_t)m->Tmax * C * 4, s));
+  CK(launch_embed_bwd<T>(m->dres32, m->tok, m->pos, A.G(m->o_wte), A.G(m->o_wpe), M, C, s));
+  m->have_targets = false;
+  return GPT_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Greedy decoding
+// ---------------------------------------------------------------------------
+template <typename T>
+static int decode_impl(gpt_model* m, const int32_t* prompt, int B, int Tp, int n_new, int32_t* out) {
+  cudaStream_t s = m->stream;
+  Acts<T> A(m);
+  const int C = m->C, F = m->F, H = m->H, d = m->d;
+  const float eps = m->cfg.ln_eps;
+  CKI(forward_impl<T>(m, prompt, nullptr, nullptr, B, Tp, nullptr));
+  m->logits_valid = false;
+  size_t kvl = (size_t)m->Bmax * H * m->Tmax * d;
+  T* kc = (T*)m->kc;
+  T* vc = (T*)m->vc;
+  for (int l = 0; l < m->NL; ++l)
+    CK(launch_kv_fill<T>(A.qkv(l), kc + l * kvl, vc + l * kvl, B, Tp, H, d, m->Tmax, s));
+  T *x = (T*)m->dx, *h = (T*)m->dh, *q = (T*)m->dq, *att = (T*)m->datt, *u = (T*)m->du, *a = (T*)m->da,
+    *xf = (T*)m->dxf;
+  CK(launch_gather_last<T>((const T*)m->xf, B, Tp, C, xf, s));
+  CK(launch_gemv<T>(xf, B, C, A.W(m->o_head), m->Vp, nullptr, nullptr, 2, nullptr, nullptr, m->dlogits, s));
+  CK(launch_argmax(m->dlogits, B, m->V, m->Vp, m->dtok, out, n_new, 0, s));
+  for (int st = 1; st < n_new; ++st) {
+    int pos = Tp + st - 1;
+    CK(launch_dec_embed<T>(m->dtok, A.P(m->o_wte), A.P(m->o_wpe), x, B, C, pos, m->Tmax, &m->sc->err, s));
+    for (int l = 0; l < m->NL; ++l) {
+      const LayerOff& lo = m->L[l];
+      CK(launch_ln_fwd<T>(x, A.P(lo.ln1_g), A.P(lo.ln1_b), h, m->dmu, m->drs, B, C, eps, s));
+      CK(launch_gemv<T>(h, B, C, A.W(lo.w_qkv), 3 * C, A.P(lo.b_qkv), nullptr, 0, q, nullptr, nullptr, s));
+      CK(launch_dec_attn<T>(q, kc + l * kvl, vc + l * kvl, att, B, H, d, m->Tmax, pos, s));
+      CK(launch_gemv<T>(att, B, C, A.W(lo.w_o), C, A.P(lo.b_o), x, 0, x, nullptr, nullptr, s));
+      CK(launch_ln_fwd<T>(x, A.P(lo.ln2_g), A.P(lo.ln2_b), h, m->dmu, m->drs, B, C, eps, s));
+      CK(launch_gemv<T>(h, B, C, A.W(lo.w_fc), F, A.P(lo.b_fc), nullptr, 1, u, a, nullptr, s));
+      CK(launch_gemv<T>(a, B, F, A.W(lo.w_fc2), C, A.P(lo.b_fc2), x, 0, x, nullptr, nullptr, s));
+    }
+    CK(launch_ln_fwd<T>(x, A.P(m->o_lnf_g), A.P(m->o_lnf_b), xf, m->dmu, m->drs, B, C, eps, s));
+    CK(launch_gemv<T>(xf, B, C, A.W(m->o_head), m->Vp, nullptr, nullptr, 2, nullptr, nullptr, m->dlogits, s));
+    CK(launch_argmax(m->dlogits, B, m->V, m->Vp, m->dtok, out, n_new, st, s));
+  }
+  return GPT_OK;
+}
+
+// ---------------------------------------------------------------------------
+// C ABI
+// ---------------------------------------------------------------------------
+static int validate_cfg(const gpt_config* c, std::string& why) {
+  if (c->vocab < 1 || c->vocab_padded < c->vocab) { why = "vocab / vocab_padded"; return 0; }
+  if (c->d_model < 8 || c->d_model % 8 || c->d_model > 1024) { why = "d_model must be a multiple of 8 in [8, 1024]"; return 0; }
+  if (c->n_heads < 1 || c->d_model % c->n_heads) { why = "d_model must be a multiple of n_heads"; return 0; }
+  int d = c->d_model / c->n_heads;
+  if (d != 16 && d != 32 && d != 64 && d != 128) { why = "head size must be 16, 32, 64 or 128"; return 0; }
+  if (c->d_mlp < 8 || c->d_mlp % 8) { why = "d_mlp must be a positive multiple of 8"; return 0; }
+  if (c->n_layers < 1 || c->max_seq < 1 || c->max_batch < 1) { why = "n_layers, max_seq, max_batch >= 1"; return 0; }
+  if (c->precision != GPT_PRECISION_FP32 && c->precision != GPT_PRECISION_BF16) { why = "precision"; return 0; }
+  if (!(c->ln_eps > 0.f) || !(c->init_std >= 0.f)) { why = "ln_eps > 0, init_std >= 0"; return 0; }
+  if (c->loss_scaling && !(c->init_loss_scale > 0.f)) { why = "init_loss_scale > 0"; return 0; }
+  return 1;
+}
+
+static thread_local std::string g_create_err;
+
+extern "C" {
+
+int gpt_create(const gpt_config* cfg, uint64_t seed, gpt_model** out) {
+  if (!cfg || !out) return GPT_ERR_ARG;
+  *out = nullptr;
+  std::string why;
+  if (!validate_cfg(cfg, why)) { g_create_err = why; return GPT_ERR_ARG; }
+  gpt_model* m = new gpt_model();
+  m->cfg = *cfg;
+  if (cudaGetDevice(&m->device) != cudaSuccess) { delete m; cudaGetLastError(); return GPT_ERR_CUDA; }
+  int nsm = 0;
+  if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, m->device) == cudaSuccess && nsm > 0)
+    g_num_sms = nsm;
+  m->bf16 = cfg->precision == GPT_PRECISION_BF16;
+  m->V = cfg->vocab; m->Vp = cfg->vocab_padded; m->C = cfg->d_model; m->H = cfg->n_heads;
+  m->d = m->C / m->H; m->F = cfg->d_mlp; m->NL = cfg->n_layers; m->Tmax = cfg->max_seq;
+  m->Bmax = cfg->max_batch; m->Mmax = (long)m->Bmax * m->Tmax;
+  m->ldl = (m->Vp + 7) / 8 * 8;
+  layout_params(m);
+  int r = build_arena(m);
+  if (r != GPT_OK) { g_create_err = m->err; delete m; return r; }
+  std::vector<float> h;
+  init_host_params(m, seed, h);
+  cudaError_t e = cudaMemcpy(m->p32, h.data(), m->N * 4, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemset(m->g32, 0, m->N * 4);
+  if (e == cudaSuccess) e = cudaMemset(m->m32, 0, m->N * 4);
+  if (e == cudaSuccess) e = cudaMemset(m->v32, 0, m->N * 4);
+  if (e == cudaSuccess && m->bf16) e = launch_cast<bf16>(m->p32, (bf16*)m->pw, m->N, 0);
+  DevScalars sc;
+  memset(&sc, 0, sizeof(sc));
+  sc.loss_scale = cfg->loss_scaling ? cfg->init_loss_scale : 1.0f;
+  sc.loss_scaling = cfg->loss_scaling ? 1 : 0;
+  sc.coef = 1.f; sc.bc1 = 1.f; sc.bc2 = 1.f;
+  if (e == cudaSuccess) e = cudaMemcpy(m->sc, &sc, sizeof(sc), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    g_create_err = std::string("initialisation: ") + cudaGetErrorString(e);
+    cudaFree(m->arena);
+    delete m;
+    return GPT_ERR_CUDA;
+  }
+  *out = m;
+  return GPT_OK;
+}
+
+void gpt_destroy(gpt_model* m) {
+  if (!m) return;
+  cudaDeviceSynchronize();
+  for (auto e : m->evpool) cudaEventDestroy(e);
+  if (m->arena) cudaFree(m->arena);
+  delete m;
+}
+
+int gpt_set_stream(gpt_model* m, void* stream) {
+  if (!m) return GPT_ERR_ARG;
+  m->stream = (cudaStream_t)stream;
+  return GPT_OK;
+}
+
+int gpt_forward_loss(gpt_model* m, const int32_t* tokens, const int32_t* targets, const int32_t* seg_ids, int B,
+                     int T, float* loss_dev) {
+  if (!m) return GPT_ERR_ARG;
+  m->err.clear();
+  if (!tokens) FAIL(GPT_ERR_ARG, "tokens is NULL");
+  if (B < 1 || B > m->Bmax) FAIL(GPT_ERR_ARG, "B out of range [1, max_batch]");
+  if (T < 1 || T > m->Tmax) FAIL(GPT_ERR_ARG, "T out of range [1, max_seq]");
+  if (m->bf16) return forward_impl<bf16>(m, tokens, targets, seg_ids, B, T, loss_dev);
+  return forward_impl<float>(m, tokens, targets, seg_ids, B, T, loss_dev);
+}
+
+int gpt_backward(gpt_model* m) {
+  if (!m) return GPT_ERR_ARG;
+  m->err.clear();
+  if (!m->have_targets) FAIL(GPT_ERR_STATE, "gpt_backward needs a preceding gpt_forward_loss with targets");
+  if (m->bf16) return backward_impl<bf16>(m);
+  return backward_impl<float>(m);
+}
+
+int gpt_clip_adamw_step(gpt_model* m, const gpt_adamw* hp, float* grad_norm_dev, int32_t* skipped_dev) {
+  if (!m || !hp) return GPT_ERR_ARG;
+  m->err.clear();
+  if (!(hp->clip_norm > 0.f)) FAIL(GPT_ERR_ARG, "clip_norm must be > 0");
+  cudaStream_t s = m->stream;
+  ProfScope ps(m, PC_OPT, 0, (double)m->N * (m->bf16 ? 34.0 : 32.0));
+  CK(launch_sumsq(m->g32, m->N, m->normpart, m->normblk, s));
+  CK(launch_opt_finalize(m->normpart, m->normblk, hp->clip_norm, hp->beta1, hp->beta2, m->sc, grad_norm_dev,
+                         skipped_dev, s));
+  if (m->bf16)
+    CK(launch_adamw<bf16>(m->p32, m->g32, m->m32, m->v32, (bf16*)m->pw, m->N, hp->lr, hp->beta1, hp->beta2,
+                          hp->eps, hp->weight_decay, m->sc, s));
+  else
+    CK(launch_adamw<float>(m->p32, m->g32, m->m32, m->v32, nullptr, m->N, hp->lr, hp->beta1, hp->beta2,
+                           hp->eps, hp->weight_decay, m->sc, s));
+  return GPT_OK;
+}
+
+int gpt_greedy_decode(gpt_model* m, const int32_t* prompt, int B, int Tp, int n_new, int32_t* out) {
+  if (!m) return GPT_ERR_ARG;
+  m->err.clear();
+  if (!prompt || !out) FAIL(GPT_ERR_ARG, "prompt / out is NULL");
+  if (B < 1 || B > m->Bmax || B > 32) FAIL(GPT_ERR_ARG, "B out of range [1, min(max_batch, 32)]");
+  if (Tp < 1 || n_new < 1) FAIL(GPT_ERR_ARG, "Tp and n_new must be >= 1");
+  if ((long)Tp + n_new - 1 > m->Tmax) FAIL(GPT_ERR_STATE, "Tp + n_new - 1 exceeds max_seq");
+  m->have_targets = false;
+  if (m->bf16) return decode_impl<bf16>(m, prompt, B, Tp, n_new, out);
+  return decode_impl<float>(m, prompt, B, Tp, n_new, out);
+}
+
+int gpt_num_params(const gpt_model* m, size_t* n) {
+  if (!m || !n) return GPT_ERR_ARG;
+  *n = m->N;
+  return GPT_OK;
+}
+
+static int copy_state(gpt_model* m, void* dst, const void* src, size_t n) {
+  if (!dst || !src) FAIL(GPT_ERR_ARG, "NULL pointer");
+  if (n != m->N) FAIL(GPT_ERR_ARG, "n must equal gpt_num_params");
+  CK(cudaStreamSynchronize(m->stream));
+  CK(cudaMemcpy(dst, src, n * 4, cudaMemcpyDefault));
+  return GPT_OK;
+}
+
+int gpt_get_params(gpt_model* m, float* dst, size_t n) { return m ? copy_state(m, dst, m->p32, n) : GPT_ERR_ARG; }
+int gpt_get_grads(gpt_model* m, float* dst, size_t n) { return m ? copy_state(m, dst, m->g32, n) : GPT_ERR_ARG; }
+int gpt_get_adam_m(gpt_model* m, float* dst, size_t n) { return m ? copy_state(m, dst, m->m32, n) : GPT_ERR_ARG; }
+int gpt_get_adam_v(gpt_model* m, float* dst, size_t n) { return m ? copy_state(m, dst, m->v32, n) : GPT_ERR_ARG; }
+int gpt_set_grads(gpt_model* m, const float* src, size_t n) { return m ? copy_state(m, m->g32, src, n) : GPT_ERR_ARG; }
+int gpt_set_adam_m(gpt_model* m, const float* src, size_t n) { return m ? copy_state(m, m->m32, src, n) : GPT_ERR_ARG; }
+int gpt_set_adam_v(gpt_model* m, const float* src, size_t n) { return m ? copy_state(m, m->v32, src, n) : GPT_ERR_ARG; }
+
+int gpt_set_params(gpt_model* m, const float* src, size_t n) {
+  if (!m) return GPT_ERR_ARG;
+  CKI(copy_state(m, m->p32, src, n));
+  if (m->bf16) {
+    CK(launch_cast<bf16>(m->p32, (bf16*)m->pw, m->N, m->stream));
+    CK(cudaStreamSynchronize(m->stream));
+  }
+  return GPT_OK;
+}
+
+int gpt_get_logits(gpt_model* m, float* dst, size_t n) {
+  if (!m || !dst) return GPT_ERR_ARG;
+  m->err.clear();
+  if (!m->logits_valid) FAIL(GPT_ERR_STATE, "no logits: run gpt_forward_loss with targets = NULL first");
+  int M = m->fwd_B * m->fwd_T;
+  if (n != (size_t)M * m->Vp) FAIL(GPT_ERR_ARG, "n must be B*T*vocab_padded");
+  cudaPointerAttributes at;
+  bool dev = cudaPointerGetAttributes(&at, dst) == cudaSuccess && at.type == cudaMemoryTypeDevice;
+  cudaGetLastError();
+  float* tmp = dst;
+  if (!dev) CK(cudaMalloc((void**)&tmp, n * 4));
+  cudaError_t e;
+  if (m->bf16) e = launch_to_f32<bf16>((const bf16*)m->logits, m->ldl, M, m->Vp, tmp, m->stream);
+  else e = launch_to_f32<float>((const float*)m->logits, m->ldl, M, m->Vp, tmp, m->stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(m->stream);
+  if (e == cudaSuccess && !dev) e = cudaMemcpy(dst, tmp, n * 4, cudaMemcpyDeviceToHost);
+  if (!dev) cudaFree(tmp);
+  CK(e);
+  return GPT_OK;
+}
+
+int gpt_get_residual(gpt_model* m, int layer, float* dst, size_t n) {
+  if (!m || !dst) return GPT_ERR_ARG;
+  m->err.clear();
+  if (m->fwd_B == 0) FAIL(GPT_ERR_STATE, "no forward pass yet");
+  if (layer < 0 || layer > m->NL) FAIL(GPT_ERR_ARG, "layer out of range [0, n_layers]");
+  int M = m->fwd_B * m->fwd_T;
+  if (n != (size_t)M * m->C) FAIL(GPT_ERR_ARG, "n must be B*T*d_model");
+  size_t off = (size_t)layer * m->Mmax * m->C;
+  cudaPointerAttributes at;
+  bool dev = cudaPointerGetAttributes(&at, dst) == cudaSuccess && at.type == cudaMemoryTypeDevice;
+  cudaGetLastError();
+  float* tmp = dst;
+  if (!dev) CK(cudaMalloc((void**)&tmp, n * 4));
+  cudaError_t e;
+  if (m->bf16) e = launch_to_f32<bf16>((const bf16*)m->xs + off, m->C, M, m->C, tmp, m->stream);
+  else e = launch_to_f32<float>((const float*)m->xs + off, m->C, M, m->C, tmp, m->stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(m->stream);
+  if (e == cudaSuccess && !dev) e = cudaMemcpy(dst, tmp, n * 4, cudaMemcpyDeviceToHost);
+  if (!dev) cudaFree(tmp);
+  CK(e);
+  return GPT_OK;
+}
+
+int gpt_get_scalars(gpt_model* m, gpt_scalars* out) {
+  if (!m || !out) return GPT_ERR_ARG;
+  DevScalars sc;
+  CK(cudaStreamSynchronize(m->stream));
+  CK(cudaMemcpy(&sc, m->sc, sizeof(sc), cudaMemcpyDeviceToHost));
+  out->loss_scale = sc.loss_scale;
+  out->good_steps = sc.good_steps;
+  out->step = sc.step;
+  out->last_loss = sc.loss;
+  out->last_grad_norm = sc.grad_norm;
+  out->last_skipped = sc.skipped;
+  return GPT_OK;
+}
+
+int gpt_set_scalars(gpt_model* m, const gpt_scalars* in) {
+  if (!m || !in) return GPT_ERR_ARG;
+  DevScalars sc;
+  CK(cudaStreamSynchronize(m->stream));
+  CK(cudaMemcpy(&sc, m->sc, sizeof(sc), cudaMemcpyDeviceToHost));
+  sc.loss_scale = in->loss_scale;
+  sc.good_steps = in->good_steps;
+  sc.step = in->step;
+  CK(cudaMemcpy(m->sc, &sc, sizeof(sc), cudaMemcpyHostToDevice));
+  return GPT_OK;
+}
+
+int gpt_status(gpt_model* m) {
+  if (!m) return GPT_ERR_ARG;
+  cudaError_t e = cudaStreamSynchronize(m->stream);
+  if (e != cudaSuccess) {
+    m->err = std::string("stream: ") + cudaGetErrorString(e);
+    return GPT_ERR_CUDA;
+  }
+  unsigned bits = 0;
+  CK(cudaMemcpy(&bits, &m->sc->err, 4, cudaMemcpyDeviceToHost));
+  if (!bits) return GPT_OK;
+  CK(cudaMemset(&m->sc->err, 0, 4));
+  m->err = "device error word 0x" + std::to_string(bits);
+  return (bits & GPT_DEVERR_TIMEOUT) ? GPT_ERR_TIMEOUT : GPT_ERR_DEVICE;
+}
+
+int gpt_device_error(gpt_model* m, uint32_t* bits) {
+  if (!m || !bits) return GPT_ERR_ARG;
+  CK(cudaStreamSynchronize(m->stream));
+  CK(cudaMemcpy(bits, &m->sc->err, 4, cudaMemcpyDeviceToHost));
+  return GPT_OK;
+}
+
+const char* gpt_last_error(const gpt_model* m) {
+  if (!m) return g_create_err.c_str();
+  return m->err.c_str();
+}
+
+int gpt_kernel_launches(uint64_t* out) {
+  if (!out) return GPT_ERR_ARG;
+  *out = g_kernel_launches;
+  return GPT_OK;
+}
+
+int gpt_profile_enable(gpt_model* m, int on) {
+  if (!m) return GPT_ERR_ARG;
+  if (on) {
+    CK(cudaStreamSynchronize(m->stream));
+    m->recs.clear();
+    m->evused = 0;
+  }
+  m->prof = on != 0;
+  return GPT_OK;
+}
+
+int gpt_profile_read(gpt_model* m, gpt_prof_entry* out, int max_entries, int* n_out) {
+  if (!m || !out || !n_out || max_entries < 0) return GPT_ERR_ARG;
+  CK(cudaStreamSynchronize(m->stream));
+  gpt_prof_entry acc[PC_COUNT];
+  memset(acc, 0, sizeof(acc));
+  for (auto& r : m->recs) {
+    if (!r.b) continue;
+    float ms = 0.f;
+    CK(cudaEventElapsedTime(&ms, r.a, r.b));
+    acc[r.cls].launches += 1;
+    acc[r.cls].ms += ms;
+    acc[r.cls].flops += r.flops;
+    acc[r.cls].bytes += r.bytes;
+  }
+  int n = 0;
+  for (int c = 0; c < PC_COUNT && n < max_entries; ++c) {
+    if (!acc[c].launches) continue;
+    out[n] = acc[c];
+    strncpy(out[n].name, kProfNames[c], sizeof(out[n].name) - 1);
+    ++n;
+  }
+  *n_out = n;
+  return GPT_OK;
+}
+
+int gpt_debug_poison_grad(gpt_model* m, size_t index, float value) {
+  if (!m) return GPT_ERR_ARG;
+  if (index >= m->N) FAIL(GPT_ERR_ARG, "index out of range");
+  CK(cudaStreamSynchronize(m->stream));
+  CK(cudaMemcpy(m->g32 + index, &value, 4, cudaMemcpyHostToDevice));
+  return GPT_OK;
+}
+
+int gpt_debug_wait_timeout(gpt_model* m, int timeout_us) {
+  if (!m || timeout_us < 1 || timeout_us > 10000000) return GPT_ERR_ARG;
+  int khz = 0;
+  CK(cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, m->device));
+  long long cycles = (long long)khz * timeout_us / 1000;
+  CK(launch_wait_timeout_probe(&m->sc->err, cycles, m->stream));
+  return gpt_status(m);
+}
+
+}  // extern "C"

@@ -1,0 +1,688 @@
+// Memory-bound kernels of the training step: input preparation, embedding
+// gather / scatter, LayerNorm forward / backward, fused softmax
+// cross-entropy with its logits gradient, deterministic row reductions,
+// global-norm clip and AdamW.  All are HBM-bound: 16-byte vector loads, one
+// warp per row where a row is reduced, no fp32 copies of bf16 tensors.
+#include "launch.h"
+
+unsigned long long g_kernel_launches = 0;
+
+#define LN_MAXC 1024   // largest d_model the register-resident LayerNorm handles
+
+// ---------------------------------------------------------------------------
+// Input preparation: clamp ids, positions inside packed documents, targets.
+// Position restarts at 0 at the first token of each document ("LucilleAI",
+// sequence packing); dstart[m] = row index of the first token of m's document.
+// ---------------------------------------------------------------------------
+__global__ void prep_kernel(const int32_t* __restrict__ tokens, const int32_t* __restrict__ targets,
+                            const int32_t* __restrict__ seg, int B, int T, int V, int* tok_out,
+                            int* tgt_out, int* pos_out, int* dstart_out, DevScalars* sc) {
+  int nv = 0;
+  unsigned err = 0;
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    int pos = 0, prev = 0;
+    for (int t = 0; t < T; ++t) {
+      long m = (long)b * T + t;
+      int tok = tokens[m];
+      if (tok < 0 || tok >= V) { err |= GPT_DEVERR_TOKEN; tok = tok < 0 ? 0 : V - 1; }
+      tok_out[m] = tok;
+      if (targets) {
+        int tg = targets[m];
+        if (tg < -1 || tg >= V) { err |= GPT_DEVERR_TARGET; tg = -1; }
+        tgt_out[m] = tg;
+        nv += (tg >= 0);
+      }
+      if (seg) {
+        int sg = seg[m];
+        if (t > 0) {
+          if (sg < prev) err |= GPT_DEVERR_SEGMENT;
+          pos = (sg == prev) ? pos + 1 : 0;
+        }
+        prev = sg;
+      } else {
+        pos = t;
+      }
+      pos_out[m] = pos;
+      dstart_out[m] = t - pos;
+    }
+  }
+  if (err) atomicOr(&sc->err, err);
+  __shared__ int red[32];
+  for (int o = 16; o > 0; o >>= 1) nv += __shfl_xor_sync(0xffffffffu, nv, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = nv;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int tot = 0;
+    for (int w = 0; w < (int)(blockDim.x + 31) / 32; ++w) tot += red[w];
+    if (targets) sc->n_valid = tot;
+  }
+}
+
+cudaError_t launch_prep(const int32_t* tokens, const int32_t* targets, const int32_t* seg, int B, int T,
+                        int V, int* tok_out, int* tgt_out, int* pos_out, int* dstart_out,
+                        DevScalars* sc, cudaStream_t s) {
+  int th = B < 32 ? 32 : (B > 1024 ? 1024 : ((B + 31) / 32) * 32);
+  ++g_kernel_launches;
+  prep_kernel<<<1, th, 0, s>>>(tokens, targets, seg, B, T, V, tok_out, tgt_out, pos_out, dstart_out, sc);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Embedding: x[m] = wte[tok[m]] + wpe[pos[m]] ("Feste", "Model Architecture
+// mirrors GPT-2": the position embedding is added directly).  fp32 sources.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void embed_fwd_kernel(const int* __restrict__ tok, const int* __restrict__ pos,
+                                 const float* __restrict__ wte, const float* __restrict__ wpe,
+                                 T* __restrict__ x, int M, int C) {
+  int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const float* a = wte + (long)tok[row] * C;
+  const float* b = wpe + (long)pos[row] * C;
+  T* o = x + (long)row * C;
+  constexpr int NV = Vec<T>::N;
+  for (int c = lane * NV; c < C; c += 32 * NV) {
+    float va[NV], vb[NV];
+#pragma unroll
+    for (int i = 0; i < NV; i += 4) {
+      Vec<float>::load(a + c + i, va + i);
+      Vec<float>::load(b + c + i, vb + i);
+    }
+#pragma unroll
+    for (int i = 0; i < NV; ++i) va[i] += vb[i];
+    Vec<T>::store(o + c, va);
+  }
+}
+
+template <typename T>
+cudaError_t launch_embed_fwd(const int* tok, const int* pos, const float* wte, const float* wpe, T* x,
+                             int M, int C, cudaStream_t s) {
+  ++g_kernel_launches;
+  embed_fwd_kernel<T><<<(M + 7) / 8, 256, 0, s>>>(tok, pos, wte, wpe, x, M, C);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// LayerNorm forward: one warp per row, the row kept in registers.  Biased
+// variance, y = (x - mean) * rstd * g + b; mean and rstd kept for backward.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void ln_fwd_kernel(const T* __restrict__ x, const float* __restrict__ g,
+                              const float* __restrict__ b, T* __restrict__ y, float* __restrict__ mean,
+                              float* __restrict__ rstd, int M, int C, float eps) {
+  constexpr int NV = Vec<T>::N;
+  constexpr int NCH = LN_MAXC / (32 * NV);
+  int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const T* xr = x + (long)row * C;
+  float v[NCH][NV];
+  float sum = 0.f;
+  int nch = C / NV;
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) {
+    int ch = lane + i * 32;
+    if (ch < nch) {
+      Vec<T>::load(xr + ch * NV, v[i]);
+#pragma unroll
+      for (int j = 0; j < NV; ++j) sum += v[i][j];
+    }
+  }
+  float mu = warp_sum(sum) / C;
+  float sq = 0.f;
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) {
+    int ch = lane + i * 32;
+    if (ch < nch) {
+#pragma unroll
+      for (int j = 0; j < NV; ++j) { float d = v[i][j] - mu; sq += d * d; }
+    }
+  }
+  float rs = 1.0f / sqrtf(warp_sum(sq) / C + eps);
+  T* yr = y + (long)row * C;
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) {
+    int ch = lane + i * 32;
+    if (ch < nch) {
+      float o[NV], gg[NV], bb[NV];
+#pragma unroll
+      for (int j = 0; j < NV; j += 4) {
+        Vec<float>::load(g + ch * NV + j, gg + j);
+        Vec<float>::load(b + ch * NV + j, bb + j);
+      }
+#pragma unroll
+      for (int j = 0; j < NV; ++j) o[j] = (v[i][j] - mu) * rs * gg[j] + bb[j];
+      Vec<T>::store(yr + ch * NV, o);
+    }
+  }
+  if (lane == 0) { mean[row] = mu; rstd[row] = rs; }
+}
+
+template <typename T>
+cudaError_t launch_ln_fwd(const T* x, const float* g, const float* b, T* y, float* mean, float* rstd,
+                          int M, int C, float eps, cudaStream_t s) {
+  ++g_kernel_launches;
+  ln_fwd_kernel<T><<<(M + 7) / 8, 256, 0, s>>>(x, g, b, y, mean, rstd, M, C, eps);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// LayerNorm backward, fused with the residual-gradient add:
+//   dx = rstd (gh - mean(gh) - xhat mean(gh xhat)),  gh = dy * g
+//   dres_out = dres_in + dx (fp32) and its T copy (the next GEMM operand);
+// per-block partial sums of dg = sum dy*xhat and db = sum dy go to
+// partials[block][0..C) and [C..2C).
+// ---------------------------------------------------------------------------
+#define LNB_WARPS 8
+template <typename T>
+__global__ void __launch_bounds__(LNB_WARPS * 32)
+ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __restrict__ mean,
+              const float* __restrict__ rstd, const float* __restrict__ g, const float* dres_in,
+              float* dres_out, T* __restrict__ dres_out_t, float* __restrict__ partials, int M, int C) {
+  constexpr int NV = Vec<T>::N;
+  constexpr int NCH = LN_MAXC / (32 * NV);
+  int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int nch = C / NV;
+  float dg[NCH][NV], db[NCH][NV], gg[NCH][NV];
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) {
+    int ch = lane + i * 32;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) { dg[i][j] = 0.f; db[i][j] = 0.f; gg[i][j] = 0.f; }
+    if (ch < nch) {
+#pragma unroll
+      for (int j = 0; j < NV; j += 4) Vec<float>::load(g + ch * NV + j, gg[i] + j);
+    }
+  }
+  for (int row = blockIdx.x * LNB_WARPS + warp; row < M; row += gridDim.x * LNB_WARPS) {
+    float mu = mean[row], rs = rstd[row];
+    const T* dyr = dy + (long)row * C;
+    const T* xr = x + (long)row * C;
+    float xh[NCH][NV], gh[NCH][NV];
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      int ch = lane + i * 32;
+      if (ch < nch) {
+        float dv[NV];
+        Vec<T>::load(dyr + ch * NV, dv);
+        Vec<T>::load(xr + ch * NV, xh[i]);
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+          xh[i][j] = (xh[i][j] - mu) * rs;
+          gh[i][j] = dv[j] * gg[i][j];
+          s1 += gh[i][j];
+          s2 += gh[i][j] * xh[i][j];
+          dg[i][j] += dv[j] * xh[i][j];
+          db[i][j] += dv[j];
+        }
+      }
+    }
+    s1 = warp_sum(s1) / C;
+    s2 = warp_sum(s2) / C;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      int ch = lane + i * 32;
+      if (ch < nch) {
+        long off = (long)row * C + ch * NV;
+        float o[NV];
+        if (dres_in) {
+#pragma unroll
+          for (int j = 0; j < NV; j += 4) Vec<float>::load(dres_in + off + j, o + j);
+        } else {
+#pragma unroll
+          for (int j = 0; j < NV; ++j) o[j] = 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < NV; ++j) o[j] += rs * (gh[i][j] - s1 - xh[i][j] * s2);
+#pragma unroll
+        for (int j = 0; j < NV; j += 4) Vec<float>::store(dres_out + off + j, o + j);
+        Vec<T>::store(dres_out_t + off, o);
+      }
+    }
+  }
+  // block-level reduction of the dg / db partials through shared memory
+  __shared__ float red[LNB_WARPS][2 * LN_MAXC / 8];   // reused in column slabs
+  constexpr int SLAB = 2 * LN_MAXC / 8;                 // columns per pass (256)
+  for (int base = 0; base < 2 * C; base += SLAB) {
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      int ch = lane + i * 32;
+      if (ch < nch) {
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+          int c = ch * NV + j;
+          if (c >= base && c < base + SLAB) red[warp][c - base] = dg[i][j];
+          if (C + c >= base && C + c < base + SLAB) red[warp][C + c - base] = db[i][j];
+        }
+      }
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < SLAB && base + c < 2 * C; c += blockDim.x) {
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < LNB_WARPS; ++w) acc += red[w][c];
+      partials[(long)blockIdx.x * 2 * C + base + c] = acc;
+    }
+    __syncthreads();
+  }
+}
+
+template <typename T>
+cudaError_t launch_ln_bwd(const T* dy, const T* x, const float* mean, const float* rstd, const float* g,
+                          const float* dres_in, float* dres_out, T* dres_out_t, float* partials,
+                          int M, int C, int* nblk_out, cudaStream_t s) {
+  int nblk = (M + LNB_WARPS - 1) / LNB_WARPS;
+  if (nblk > 296) nblk = 296;
+  *nblk_out = nblk;
+  ++g_kernel_launches;
+  ln_bwd_kernel<T><<<nblk, LNB_WARPS * 32, 0, s>>>(dy, x, mean, rstd, g, dres_in, dres_out, dres_out_t,
+                                                    partials, M, C);
+  return cudaGetLastError();
+}
+
+// out[n] = sum over r of partials[r][n], in a fixed order (deterministic).
+__global__ void reduce_rows_kernel(const float* __restrict__ p, int rows, int N, float* __restrict__ out) {
+  int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  float acc = 0.f;
+  for (int r = 0; r < rows; ++r) acc += p[(long)r * N + n];
+  out[n] = acc;
+}
+
+cudaError_t launch_reduce_rows(const float* partials, int rows, int N, float* out, cudaStream_t s) {
+  ++g_kernel_launches;
+  reduce_rows_kernel<<<(N + 255) / 256, 256, 0, s>>>(partials, rows, N, out);
+  return cudaGetLastError();
+}
+
+// Column sums of x [M, N] (bias gradients): stage 1 writes per-row-chunk
+// partials, stage 2 is reduce_rows.
+template <typename Tin>
+__global__ void colsum_kernel(const Tin* __restrict__ x, long ldx, int M, int N, int chunk,
+                              float* __restrict__ partials) {
+  int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  int r0 = blockIdx.y * chunk, r1 = min(M, r0 + chunk);
+  float acc = 0.f;
+  for (int r = r0; r < r1; ++r) acc += to_f(x[(long)r * ldx + n]);
+  partials[(long)blockIdx.y * N + n] = acc;
+}
+
+template <typename Tin>
+cudaError_t launch_colsum(const Tin* x, long ldx, int M, int N, float* partials, float* out, cudaStream_t s) {
+  int rc = M < 128 ? M : 128;
+  int chunk = (M + rc - 1) / rc;
+  rc = (M + chunk - 1) / chunk;
+  dim3 grid((N + 127) / 128, rc);
+  ++g_kernel_launches;
+  colsum_kernel<Tin><<<grid, 128, 0, s>>>(x, ldx, M, N, chunk, partials);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_reduce_rows(partials, rc, N, out, s);
+}
+
+// ---------------------------------------------------------------------------
+// Fused softmax cross-entropy and its gradient, in place over the logits.
+// Per row: lse over the real vocabulary 0..V-1 (online max / sum), loss =
+// lse - z[target]; then dz = (softmax - onehot) * loss_scale / N_valid for
+// c < V, 0 for the padded columns and for ignored rows.  No fp32
+// probability tensor is written.  ("RustGPT", "Technical implementation":
+// cross-entropy loss.)
+// ---------------------------------------------------------------------------
+#define XENT_THREADS 512
+template <typename T>
+__global__ void __launch_bounds__(XENT_THREADS)
+xent_kernel(T* __restrict__ logits, long ldl, const int* __restrict__ tgt, int V, int Vp,
+            float* __restrict__ rowloss, const DevScalars* __restrict__ sc) {
+  constexpr int NV = Vec<T>::N;
+  int row = blockIdx.x;
+  T* z = logits + (long)row * ldl;
+  int tg = tgt[row];
+  float m = -INFINITY, ssum = 0.f;
+  int nvec = V / NV;
+  for (int i = threadIdx.x; i < nvec; i += XENT_THREADS) {
+    float v[NV];
+    Vec<T>::load(z + i * NV, v);
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      if (v[j] > m) { ssum = ssum * expf(m - v[j]) + 1.f; m = v[j]; }
+      else ssum += expf(v[j] - m);
+    }
+  }
+  for (int c = nvec * NV + threadIdx.x; c < V; c += XENT_THREADS) {
+    float v = to_f(z[c]);
+    if (v > m) { ssum = ssum * expf(m - v) + 1.f; m = v; }
+    else ssum += expf(v - m);
+  }
+  // merge (m, s) across the block
+  __shared__ float sm[XENT_THREADS / 32], ss[XENT_THREADS / 32];
+  __shared__ float s_lse, s_ztg;
+  float wm = warp_max(m);
+  float ws = warp_sum(m == -INFINITY ? 0.f : ssum * expf(m - wm));
+  int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) { sm[warp] = wm; ss[warp] = ws; }
+  __syncthreads();
+  if (warp == 0) {
+    float mm = lane < XENT_THREADS / 32 ? sm[lane] : -INFINITY;
+    float s2 = lane < XENT_THREADS / 32 ? ss[lane] : 0.f;
+    float gm = warp_max(mm);
+    float gs = warp_sum(mm == -INFINITY ? 0.f : s2 * expf(mm - gm));
+    if (lane == 0) {
+      s_lse = gm + logf(gs);
+      s_ztg = tg >= 0 ? to_f(z[tg]) : 0.f;
+    }
+  }
+  __syncthreads();
+  float lse = s_lse;
+  if (threadIdx.x == 0) rowloss[row] = tg >= 0 ? lse - s_ztg : 0.f;
+  int nv = sc->n_valid;
+  float scale = tg >= 0 ? sc->loss_scale / (float)(nv > 0 ? nv : 1) : 0.f;
+  int nvp = Vp / NV;
+  for (int i = threadIdx.x; i < nvp; i += XENT_THREADS) {
+    float v[NV];
+    Vec<T>::load(z + i * NV, v);
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      int c = i * NV + j;
+      float p = c < V ? expf(v[j] - lse) : 0.f;
+      v[j] = (p - (c == tg ? 1.f : 0.f)) * scale;
+    }
+    Vec<T>::store(z + i * NV, v);
+  }
+  for (int c = nvp * NV + threadIdx.x; c < Vp; c += XENT_THREADS) {
+    float p = c < V ? expf(to_f(z[c]) - lse) : 0.f;
+    z[c] = from_f<T>((p - (c == tg ? 1.f : 0.f)) * scale);
+  }
+}
+
+template <typename T>
+cudaError_t launch_xent(T* logits, long ldl, const int* tgt, int M, int V, int Vp, float* rowloss,
+                        DevScalars* sc, cudaStream_t s) {
+  ++g_kernel_launches;
+  xent_kernel<T><<<M, XENT_THREADS, 0, s>>>(logits, ldl, tgt, V, Vp, rowloss, sc);
+  return cudaGetLastError();
+}
+
+__global__ void loss_finalize_kernel(const float* __restrict__ rowloss, int M, DevScalars* sc, float* loss_out) {
+  __shared__ float red[32];
+  float acc = 0.f;
+  for (int i = threadIdx.x; i < M; i += blockDim.x) acc += rowloss[i];
+  acc = warp_sum(acc);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < blockDim.x / 32 ? red[threadIdx.x] : 0.f;
+    v = warp_sum(v);
+    if (threadIdx.x == 0) {
+      int nv = sc->n_valid;
+      float loss = nv > 0 ? v / (float)nv : 0.f;
+      sc->loss = loss;
+      if (loss_out) *loss_out = loss;
+    }
+  }
+}
+
+cudaError_t launch_loss_finalize(const float* rowloss, int M, DevScalars* sc, float* loss_out, cudaStream_t s) {
+  ++g_kernel_launches;
+  loss_finalize_kernel<<<1, 1024, 0, s>>>(rowloss, M, sc, loss_out);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Embedding backward: scatter-add of the residual gradient into the token
+// rows of dwte and the position rows of dwpe (fp32 atomics).
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void embed_bwd_kernel(const float* __restrict__ dres, const int* __restrict__ tok,
+                                 const int* __restrict__ pos, float* gwte, float* gwpe, int M, int C) {
+  int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const float* d = dres + (long)row * C;
+  float* a = gwte + (long)tok[row] * C;
+  float* b = gwpe + (long)pos[row] * C;
+  for (int c = lane * 4; c < C; c += 128) {
+    float v[4];
+    Vec<float>::load(d + c, v);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) { atomicAdd(a + c + j, v[j]); atomicAdd(b + c + j, v[j]); }
+  }
+}
+
+template <typename T>
+cudaError_t launch_embed_bwd(const float* dres, const int* tok, const int* pos, float* gwte, float* gwpe,
+                             int M, int C, cudaStream_t s) {
+  ++g_kernel_launches;
+  embed_bwd_kernel<T><<<(M + 7) / 8, 256, 0, s>>>(dres, tok, pos, gwte, gwpe, M, C);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Global L2 norm, clip, dynamic loss scale and AdamW over the flat fp32
+// parameter vector (one tensor: the canonical layout is contiguous).
+// ---------------------------------------------------------------------------
+__global__ void sumsq_kernel(const float* __restrict__ g, size_t n, double* __restrict__ partials) {
+  float acc = 0.f;
+  size_t n4 = n / 4;
+  const float4* g4 = reinterpret_cast<const float4*>(g);
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+    float4 v = g4[i];
+    acc += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  if (blockIdx.x == 0)
+    for (size_t i = n4 * 4 + threadIdx.x; i < n; i += blockDim.x) acc += g[i] * g[i];
+  double d = acc;
+  for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+  __shared__ double red[32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = d;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < (int)blockDim.x / 32; ++w) t += red[w];
+    partials[blockIdx.x] = t;
+  }
+}
+
+cudaError_t launch_sumsq(const float* g, size_t n, double* partials, int nblk, cudaStream_t s) {
+  ++g_kernel_launches;
+  sumsq_kernel<<<nblk, 512, 0, s>>>(g, n, partials);
+  return cudaGetLastError();
+}
+
+__global__ void opt_finalize_kernel(const double* __restrict__ partials, int nblk, float clip, float beta1,
+                                    float beta2, DevScalars* sc, float* norm_out, int32_t* skipped_out) {
+  __shared__ double red[32];
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < nblk; i += blockDim.x) acc += partials[i];
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  double tot = 0.0;
+  for (int w = 0; w < (int)blockDim.x / 32; ++w) tot += red[w];
+  double inv = 1.0 / (double)sc->loss_scale;
+  double norm = sqrt(tot) * inv;
+  bool finite = isfinite(norm);
+  sc->grad_norm = (float)norm;
+  if (!finite) {
+    sc->skipped = 1;
+    if (sc->loss_scaling) sc->loss_scale *= 0.5f;
+    sc->good_steps = 0;
+  } else {
+    sc->skipped = 0;
+    double coef = (double)clip / (norm + 1e-6);
+    if (coef > 1.0) coef = 1.0;
+    sc->coef = (float)(coef * inv);
+    int t = sc->step + 1;
+    sc->step = t;
+    sc->bc1 = (float)(1.0 - pow((double)beta1, (double)t));
+    sc->bc2 = (float)(1.0 - pow((double)beta2, (double)t));
+    if (sc->loss_scaling) {
+      sc->good_steps += 1;
+      if (sc->good_steps >= 2000) { sc->loss_scale *= 2.0f; sc->good_steps = 0; }
+    }
+  }
+  if (norm_out) *norm_out = (float)norm;
+  if (skipped_out) *skipped_out = sc->skipped;
+}
+
+cudaError_t launch_opt_finalize(const double* partials, int nblk, float clip, float beta1, float beta2,
+                                DevScalars* sc, float* norm_out, int32_t* skipped_out, cudaStream_t s) {
+  ++g_kernel_launches;
+  opt_finalize_kernel<<<1, 1024, 0, s>>>(partials, nblk, clip, beta1, beta2, sc, norm_out, skipped_out);
+  return cudaGetLastError();
+}
+
+// AdamW ("Feste", "Manual Backpropagation from scratch": decoupled weight
+// decay) on the clipped, unscaled gradient g * coef:
+//   m = b1 m + (1-b1) g;  v = b2 v + (1-b2) g^2;
+//   p -= lr (m / bc1 / (sqrt(v / bc2) + eps) + wd p);  pw = T(p).
+template <typename T>
+__global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g, float* __restrict__ m,
+                             float* __restrict__ v, T* __restrict__ pw, size_t n, float lr, float beta1,
+                             float beta2, float eps, float wd, const DevScalars* __restrict__ sc) {
+  if (sc->skipped) return;
+  float coef = sc->coef, bc1 = sc->bc1, bc2 = sc->bc2;
+  float ib1 = 1.0f / bc1, ib2 = 1.0f / bc2;
+  size_t n4 = n / 4;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+    float pp[4], gg[4], mm[4], vv[4];
+    Vec<float>::load(p + 4 * i, pp);
+    Vec<float>::load(g + 4 * i, gg);
+    Vec<float>::load(m + 4 * i, mm);
+    Vec<float>::load(v + 4 * i, vv);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float gj = gg[j] * coef;
+      mm[j] = beta1 * mm[j] + (1.f - beta1) * gj;
+      vv[j] = beta2 * vv[j] + (1.f - beta2) * gj * gj;
+      float upd = (mm[j] * ib1) / (sqrtf(vv[j] * ib2) + eps) + wd * pp[j];
+      pp[j] = pp[j] - lr * upd;
+    }
+    Vec<float>::store(p + 4 * i, pp);
+    Vec<float>::store(m + 4 * i, mm);
+    Vec<float>::store(v + 4 * i, vv);
+    if (pw) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) pw[4 * i + j] = from_f<T>(pp[j]);
+    }
+  }
+  if (blockIdx.x == 0) {
+    for (size_t i = n4 * 4 + threadIdx.x; i < n; i += blockDim.x) {
+      float gj = g[i] * coef;
+      float mj = beta1 * m[i] + (1.f - beta1) * gj;
+      float vj = beta2 * v[i] + (1.f - beta2) * gj * gj;
+      float pj = p[i] - lr * ((mj * ib1) / (sqrtf(vj * ib2) + eps) + wd * p[i]);
+      p[i] = pj; m[i] = mj; v[i] = vj;
+      if (pw) pw[i] = from_f<T>(pj);
+    }
+  }
+}
+
+template <typename T>
+cudaError_t launch_adamw(float* p, const float* g, float* m, float* v, T* pw, size_t n, float lr,
+                         float beta1, float beta2, float eps, float wd, const DevScalars* sc,
+                         cudaStream_t s) {
+  ++g_kernel_launches;
+  adamw_kernel<T><<<148 * 8, 256, 0, s>>>(p, g, m, v, pw, n, lr, beta1, beta2, eps, wd, sc);
+  return cudaGetLastError();
+}
+
+template <typename T>
+__global__ void cast_kernel(const float* __restrict__ src, T* __restrict__ dst, size_t n) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    dst[i] = from_f<T>(src[i]);
+}
+template <typename T>
+cudaError_t launch_cast(const float* src, T* dst, size_t n, cudaStream_t s) {
+  ++g_kernel_launches;
+  cast_kernel<T><<<148 * 8, 256, 0, s>>>(src, dst, n);
+  return cudaGetLastError();
+}
+
+template <typename T>
+__global__ void to_f32_kernel(const T* __restrict__ src, long ld, int rows, int cols, float* __restrict__ dst) {
+  size_t n = (size_t)rows * cols;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    size_t r = i / cols, c = i % cols;
+    dst[i] = to_f(src[r * ld + c]);
+  }
+}
+template <typename T>
+cudaError_t launch_to_f32(const T* src, long ld, int rows, int cols, float* dst, cudaStream_t s) {
+  ++g_kernel_launches;
+  to_f32_kernel<T><<<148 * 8, 256, 0, s>>>(src, ld, rows, cols, dst);
+  return cudaGetLastError();
+}
+
+// out[i] = sum over splits of ws[split * stride + i] (split-K reduction).
+__global__ void sum_splits_kernel(const float* __restrict__ ws, int splits, long stride, long n,
+                                  float* __restrict__ out) {
+  long n4 = n / 4;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n4; i += (long)gridDim.x * blockDim.x) {
+    float a[4], b[4];
+    Vec<float>::load(ws + 4 * i, a);
+    for (int s = 1; s < splits; ++s) {
+      Vec<float>::load(ws + s * stride + 4 * i, b);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) a[j] += b[j];
+    }
+    Vec<float>::store(out + 4 * i, a);
+  }
+  if (blockIdx.x == 0)
+    for (long i = n4 * 4 + threadIdx.x; i < n; i += blockDim.x) {
+      float a = 0.f;
+      for (int s = 0; s < splits; ++s) a += ws[s * stride + i];
+      out[i] = a;
+    }
+}
+cudaError_t launch_sum_splits(const float* ws, int splits, long stride, long n, float* out, cudaStream_t s) {
+  ++g_kernel_launches;
+  sum_splits_kernel<<<148 * 4, 256, 0, s>>>(ws, splits, stride, n, out);
+  return cudaGetLastError();
+}
+
+// A bounded wait that cannot complete: an mbarrier nobody arrives on.  The
+// waiting thread gives up after timeout_cycles, records GPT_DEVERR_TIMEOUT
+// and returns, leaving the context usable.
+__global__ void wait_timeout_probe_kernel(unsigned* err, long long timeout_cycles) {
+  __shared__ __align__(8) uint64_t bar;
+  uint32_t a = (uint32_t)__cvta_generic_to_shared(&bar);
+  if (threadIdx.x == 0) asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(1));
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long t0 = clock64();
+    uint32_t done = 0;
+    while (!done) {
+      asm volatile("{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+                   : "=r"(done) : "r"(a), "r"(0u));
+      if (!done && clock64() - t0 > timeout_cycles) { atomicOr(err, GPT_DEVERR_TIMEOUT); break; }
+    }
+  }
+}
+cudaError_t launch_wait_timeout_probe(unsigned* err, long long timeout_cycles, cudaStream_t s) {
+  ++g_kernel_launches;
+  wait_timeout_probe_kernel<<<1, 32, 0, s>>>(err, timeout_cycles);
+  return cudaGetLastError();
+}
+
+// ---- explicit instantiations
+#define INST(T)                                                                                          \
+  template cudaError_t launch_embed_fwd<T>(const int*, const int*, const float*, const float*, T*, int, int, \
+                                           cudaStream_t);                                                \
+  template cudaError_t launch_ln_fwd<T>(const T*, const float*, const float*, T*, float*, float*, int, int, \
+                                        float, cudaStream_t);                                            \
+  template cudaError_t launch_ln_bwd<T>(const T*, const T*, const float*, const float*, const float*,      \
+                                        const float*, float*, T*, float*, int, int, int*, cudaStream_t);  \
+  template cudaError_t launch_colsum<T>(const T*, long, int, int, float*, float*, cudaStream_t);          \
+  template cudaError_t launch_xent<T>(T*, long, const int*, int, int, int, float*, DevScalars*, cudaStream_t); \
+  template cudaError_t launch_embed_bwd<T>(const float*, const int*, const int*, float*, float*, int, int,  \
+                                           cudaStream_t);                                                \
+  template cudaError_t launch_adamw<T>(float*, const float*, float*, float*, T*, size_t, float, float,     \
+                                       float, float, float, const DevScalars*, cudaStream_t);            \
+  template cudaError_t launch_cast<T>(const float*, T*, size_t, cudaStream_t);                            \
+  template cudaError_t launch_to_f32<T>(const T*, long, int, int, float*, cudaStream_t);
+INST(float)
+INST(bf16)

@@ -1,0 +1,33 @@
+"""Shared helpers for the parity tests: config conversion and comparisons."""
+import numpy as np
+
+from oracle import gpt_oracle as O
+from scratch_decoder_only_b200 import configs as CF
+
+
+def ocfg(mc: CF.ModelConfig, max_seq=None) -> O.OracleConfig:
+    return O.OracleConfig(vocab=mc.vocab, vocab_padded=mc.vocab_padded, d_model=mc.d_model,
+                          n_heads=mc.n_heads, d_mlp=mc.d_mlp, n_layers=mc.n_layers,
+                          max_seq=max_seq or mc.max_seq, tied=mc.tied, ln_eps=mc.ln_eps,
+                          init_std=mc.init_std)
+
+
+def per_tensor_rel_l2(cfg: O.OracleConfig, g_gpu, g_ref):
+    """{name: ||g_gpu - g_ref|| / ||g_ref||}; tensors with a zero reference
+    must be exactly zero on the GPU (reported as 0.0 or inf)."""
+    out, o = {}, 0
+    for name, shape in O.param_shapes(cfg):
+        n = int(np.prod(shape))
+        a = np.asarray(g_gpu[o:o + n], dtype=np.float64)
+        b = np.asarray(g_ref[o:o + n], dtype=np.float64)
+        nb = np.linalg.norm(b)
+        if nb == 0.0:
+            out[name] = 0.0 if np.all(a == 0.0) else float("inf")
+        else:
+            out[name] = float(np.linalg.norm(a - b) / nb)
+        o += n
+    return out
+
+
+def rel(a, b):
+    return abs(a - b) / max(abs(b), 1e-30)
