@@ -161,18 +161,22 @@ def init_params(cfg: OracleConfig, seed: int) -> np.ndarray:
     """Initial fp32 parameter vector in canonical order.
 
     Weight matrices and embeddings ~ N(0, init_std) (value for canonical
-    element e from ``gaussian_for_elements(seed, e)``), LayerNorm gains 1,
+    element e: float32(std * gaussian_for_elements(seed, e)) with std the
+    float32 value of init_std), LayerNorm gains 1,
     LayerNorm shifts and biases 0, and the padded vocabulary rows V..Vp-1 of
     the embedding / LM head are 0.
     """
     flat = np.zeros(num_params(cfg), dtype=np.float32)
+    # the configured standard deviation at float32 precision, as a
+    # configuration record carries it (0.02 -> 0.0199999995529651...)
+    std = float(np.float32(cfg.init_std))
     o = 0
     for name, shape in param_shapes(cfg):
         n = int(np.prod(shape))
         leaf = name.split(".")[-1]
         if leaf in ("wte", "wpe", "w_qkv", "w_o", "w_fc", "w_fc2", "w_head"):
             z = gaussian_for_elements(seed, np.arange(o, o + n, dtype=np.uint64))
-            vals = (cfg.init_std * z).astype(np.float32)
+            vals = (std * z).astype(np.float32)
             if leaf in ("wte", "w_head"):
                 vals.reshape(shape)[cfg.vocab:, :] = 0.0
             flat[o:o + n] = vals
