@@ -217,6 +217,15 @@ int gpt_device_error(gpt_model* m, uint32_t* bits);
  * The string lives until the next call on the handle. */
 const char* gpt_last_error(const gpt_model* m);
 
+/* Stand-alone tensor-core GEMM (the library's tcgen05 path), enqueued on
+ * `stream` (a cudaStream_t; NULL = legacy default):
+ *   C[m, n] = sum_k A(m, k) * B(n, k),  fp32 C with row stride ldc >= N,
+ * bf16 A and B in device memory.  A(m, k) = a_t ? A[k*lda + m] : A[m*lda + k];
+ * B(n, k) = b_t ? B[k*ldb + n] : B[n*ldb + k].  lda and ldb must be multiples
+ * of 8 and A, B 16-byte aligned.  Errors: GPT_ERR_ARG, GPT_ERR_CUDA. */
+int gpt_gemm_bf16(int M, int N, int K, const void* A, long lda, int a_t, const void* B, long ldb, int b_t,
+                  float* C, long ldc, void* stream);
+
 /* Number of kernels libgpt has launched in this process (all handles).
  * Benchmarks read it before and after a timed region. */
 int gpt_kernel_launches(uint64_t* out);

@@ -349,10 +349,13 @@ static int gemm(gpt_model* m, int M, int N, int K, const bf16* A, long lda, bool
   }
   int splits = 1;
   if (epi.kind == EPI_F32) {
+    // weight gradients: short output, long contraction -> split K over the SMs
     long tiles = (long)((M + 127) / 128) * ((N + 255) / 256);
-    while (splits < 8 && tiles * splits * 2 <= g_num_sms * 2 && K / (splits * 2) >= 512 &&
+    while (splits < 8 && tiles * splits * 2 <= g_num_sms && K / (splits * 2) >= 512 &&
            (size_t)(splits * 2) * M * N <= m->splitws_n)
       splits *= 2;
+    int kb_total = (K + 63) / 64, kbs = (kb_total + splits - 1) / splits;
+    splits = (kb_total + kbs - 1) / kbs;   // no empty split
   }
   if (splits > 1) {
     EpiParams<bf16> e2 = epi;
@@ -818,6 +821,18 @@ int gpt_device_error(gpt_model* m, uint32_t* bits) {
 const char* gpt_last_error(const gpt_model* m) {
   if (!m) return g_create_err.c_str();
   return m->err.c_str();
+}
+
+int gpt_gemm_bf16(int M, int N, int K, const void* A, long lda, int a_t, const void* B, long ldb, int b_t,
+                  float* C, long ldc, void* stream) {
+  if (!A || !B || !C || M < 1 || N < 1 || K < 1 || ldc < N) return GPT_ERR_ARG;
+  if (!gemm_tc_supported(M, N, K, lda, a_t != 0, ldb, b_t != 0)) return GPT_ERR_ARG;
+  EpiParams<bf16> e = epi_f32<bf16>(C, ldc);
+  static unsigned* err = nullptr;
+  if (!err && cudaMalloc((void**)&err, 4) != cudaSuccess) return GPT_ERR_CUDA;
+  cudaError_t r = launch_gemm_tc(M, N, K, (const bf16*)A, lda, a_t != 0, (const bf16*)B, ldb, b_t != 0, e, 1, err,
+                                 (cudaStream_t)stream);
+  return r == cudaSuccess ? GPT_OK : GPT_ERR_CUDA;
 }
 
 int gpt_kernel_launches(uint64_t* out) {
