@@ -139,6 +139,27 @@ def test_mask_bit_identity_fp32(torch):
                     assert np.array_equal(base[:, i], alt[:, i]), (i, j)
 
 
+def test_mask_bit_identity_bf16(torch):
+    """Tensor-core path: a changed token leaves earlier positions' logits bit-identical."""
+    wl = CF.PACKED_SMALL
+    rng = np.random.default_rng(2)
+    tok = rng.integers(0, 8000, size=(2, 200)).astype(np.int32)
+    seg = np.zeros((2, 200), np.int32)
+    seg[:, 130:] = 1
+    model = new_model(wl.model, 1)
+    for sg in (None, seg):
+        model.forward_loss(dev(torch, tok), None, dev(torch, sg))
+        base = model.get_logits(2, 200).reshape(2, 200, -1)
+        for j in (70, 150):
+            t2 = tok.copy()
+            t2[:, j] = (t2[:, j] + 11) % 8000
+            model.forward_loss(dev(torch, t2), None, dev(torch, sg))
+            alt = model.get_logits(2, 200).reshape(2, 200, -1)
+            same = [i for i in range(200) if i < j or (sg is not None and (i >= 130) != (j >= 130))]
+            assert np.array_equal(base[:, same], alt[:, same]), j
+            assert not np.array_equal(base[:, j], alt[:, j])
+
+
 def test_greedy_decode_fp32_bit_exact(torch):
     mc = CF.ModelConfig(vocab=50257, vocab_padded=50304, d_model=64, n_heads=4, d_mlp=256, n_layers=2,
                         max_seq=64, max_batch=2, tied=True, precision="fp32", init_std=0.5)
