@@ -167,8 +167,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     mc = WL.model
-    B, T = WL.batch, WL.seq
-    tok, tgt, _ = S.make_batch(WL, seed=WL.data_seed + rank)
+    B, T = args.batch or WL.batch, WL.seq
+    tok, tgt, _ = S.make_batch(WL, batch=B, seed=WL.data_seed + rank)
     d_tok = torch.from_numpy(tok).to(dev)
     d_tgt = torch.from_numpy(tgt).to(dev)
     model = GPT(mc, WL.init_seed)
@@ -328,6 +328,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None, help="override the batch (profiling of small cases)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

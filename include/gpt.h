@@ -237,7 +237,7 @@ int gpt_kernel_launches(uint64_t* out);
  * starts a fresh record, (m, 0) stops recording and keeps the record. */
 typedef struct {
   char name[24];      /* gemm_fwd, gemm_dgrad, gemm_wgrad, attn_fwd, attn_bwd,
-                         xent, ln_fwd, ln_bwd, clip_adamw                      */
+                         xent, ln_fwd, ln_bwd, clip_adamw, bias_grad, embed   */
   int32_t launches;   /* bracketed calls                                      */
   double ms;          /* summed event time                                    */
   double flops;       /* summed algorithmic FLOPs (0 where not applicable)    */

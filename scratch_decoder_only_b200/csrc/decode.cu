@@ -44,9 +44,9 @@ gemv_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, int 
   for (int k0 = 0; k0 < K; k0 += KC) {
     int kend = min(KC, K - k0);
     __syncthreads();
-    for (int i = threadIdx.x; i < B * KC; i += blockDim.x) {
-      int b = i / KC, kk = i % KC;
-      xs[b * KC + kk] = kk < kend ? to_f(X[(long)b * K + k0 + kk]) : 0.f;
+    for (int i = threadIdx.x; i < B * kend; i += blockDim.x) {
+      int b = i / kend, kk = i % kend;
+      xs[b * KC + kk] = to_f(X[(long)b * K + k0 + kk]);
     }
     __syncthreads();
     if (n < N) {

@@ -66,9 +66,9 @@ struct gpt_model {
 };
 
 enum ProfCls { PC_GEMM_FWD, PC_GEMM_DX, PC_GEMM_DW, PC_ATTN_FWD, PC_ATTN_BWD, PC_XENT, PC_LN_FWD, PC_LN_BWD,
-               PC_OPT, PC_COUNT };
+               PC_OPT, PC_BIAS, PC_EMBED, PC_COUNT };
 static const char* kProfNames[PC_COUNT] = {"gemm_fwd", "gemm_dgrad", "gemm_wgrad", "attn_fwd", "attn_bwd",
-                                           "xent", "ln_fwd", "ln_bwd", "clip_adamw"};
+                                           "xent", "ln_fwd", "ln_bwd", "clip_adamw", "bias_grad", "embed"};
 
 static cudaEvent_t prof_event(gpt_model* m) {
   if (m->evused == m->evpool.size()) {
@@ -258,7 +258,7 @@ static int build_arena(gpt_model* m) {
   cv.add(&m->dqkv, Mx * 3 * C * es);
   cv.add((void**)&m->attD, Mx * m->H * 4);
   cv.add((void**)&m->rowloss, Mx * 4);
-  m->partials_n = std::max((size_t)296 * 2 * C, (size_t)128 * std::max(3 * C, F));
+  m->partials_n = std::max((size_t)444 * 3 * C, (size_t)((Mx + 255) / 256) * std::max(3 * C, F));
   cv.add((void**)&m->partials, m->partials_n * 4);
   m->splitws_n = m->bf16 ? (size_t)8 * std::max(3 * C * C, F * C) : 0;
   if (m->splitws_n) cv.add((void**)&m->splitws, m->splitws_n * 4);
@@ -438,8 +438,9 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
   const float eps = m->cfg.ln_eps;
   const double es = sizeof(T), lnb = (double)M * C * 2 * es + 8.0 * M;
   m->seg_used = seg != nullptr;
-  CK(launch_prep(tokens, targets, seg, B, T_, m->V, m->tok, m->tgt, m->pos, m->dstart, m->sc, s));
-  CK(launch_embed_fwd<T>(m->tok, m->pos, A.P(m->o_wte), A.P(m->o_wpe), A.x(0), M, C, s));
+  { ProfScope ps(m, PC_EMBED, 0, (double)M * C * (8 + es) + 16.0 * M);
+    CK(launch_prep(tokens, targets, seg, B, T_, m->V, m->tok, m->tgt, m->pos, m->dstart, m->sc, s));
+    CK(launch_embed_fwd<T>(m->tok, m->pos, A.P(m->o_wte), A.P(m->o_wpe), A.x(0), M, C, s)); }
   for (int l = 0; l < m->NL; ++l) {
     const LayerOff& lo = m->L[l];
     { ProfScope ps(m, PC_LN_FWD, 0, lnb);
@@ -490,35 +491,40 @@ static int backward_impl(gpt_model* m) {
   CKI(gemm(m, Vp, C, M, dz, m->ldl, true, xf, C, true, epi_f32<T>(A.G(m->o_head), C)));
   { ProfScope ps(m, PC_LN_BWD, 0, lnbb);
     CK(launch_ln_bwd<T>(dC, A.x(m->NL), m->muf, m->rsf, A.P(m->o_lnf_g), nullptr, m->dres32, drt, m->partials,
-                      M, C, &nblk, s));
-    CK(launch_reduce_rows(m->partials, nblk, 2 * C, A.G(m->o_lnf_g), s)); }
+                        M, C, &nblk, s));
+    CK(launch_reduce_rows(m->partials, nblk, 2 * C, 3 * C, A.G(m->o_lnf_g), s));
+    // column sums of the gradient entering the last block = its fc2 bias gradient
+    CK(launch_reduce_rows(m->partials + 2 * C, nblk, C, 3 * C, A.G(m->L[m->NL - 1].b_fc2), s)); }
   for (int l = m->NL - 1; l >= 0; --l) {
     const LayerOff& lo = m->L[l];
-    // MLP: x_out = x_mid + gelu(h2 W_fc^T + b_fc) W_fc2^T + b_fc2
-    CK(launch_colsum<float>(m->dres32, C, M, C, m->partials, A.G(lo.b_fc2), s));
+    // MLP: x_out = x_mid + gelu(h2 W_fc^T + b_fc) W_fc2^T + b_fc2  (b_fc2 gradient already summed)
     CKI(gemm(m, C, F, M, drt, C, true, A.a(l), F, true, epi_f32<T>(A.G(lo.w_fc2), F)));
     CKI(gemm(m, M, F, C, drt, C, false, A.W(lo.w_fc2), F, true, epi_dgelu<T>(dF, F, A.u(l))));
-    CK(launch_colsum<T>(dF, F, M, F, m->partials, A.G(lo.b_fc), s));
+    { ProfScope ps(m, PC_BIAS, 0, (double)M * F * es);
+      CK(launch_colsum<T>(dF, F, M, F, m->partials, A.G(lo.b_fc), s)); }
     CKI(gemm(m, F, C, M, dF, F, true, A.h2(l), C, true, epi_f32<T>(A.G(lo.w_fc), C)));
     CKI(gemm(m, M, C, F, dF, F, false, A.W(lo.w_fc), C, true, epi_store<T>(dC, C, nullptr, nullptr, 0)));
     { ProfScope ps(m, PC_LN_BWD, 0, lnbb);
       CK(launch_ln_bwd<T>(dC, A.xmid(l), A.mu2(l), A.rs2(l), A.P(lo.ln2_g), m->dres32, m->dres32, drt,
                           m->partials, M, C, &nblk, s));
-      CK(launch_reduce_rows(m->partials, nblk, 2 * C, A.G(lo.ln2_g), s)); }
-    // attention: x_mid = x + attn(h1 W_qkv^T + b_qkv) W_o^T + b_o
-    CK(launch_colsum<float>(m->dres32, C, M, C, m->partials, A.G(lo.b_o), s));
+      CK(launch_reduce_rows(m->partials, nblk, 2 * C, 3 * C, A.G(lo.ln2_g), s));
+      CK(launch_reduce_rows(m->partials + 2 * C, nblk, C, 3 * C, A.G(lo.b_o), s)); }
+    // attention: x_mid = x + attn(h1 W_qkv^T + b_qkv) W_o^T + b_o  (b_o gradient already summed)
     CKI(gemm(m, C, C, M, drt, C, true, A.att(l), C, true, epi_f32<T>(A.G(lo.w_o), C)));
     CKI(gemm(m, M, C, C, drt, C, false, A.W(lo.w_o), C, true, epi_store<T>(dC, C, nullptr, nullptr, 0)));
     CKI(attn_bwd(m, A.qkv(l), A.att(l), dC, A.lse(l), dq, B, T_));
-    CK(launch_colsum<T>(dq, 3 * C, M, 3 * C, m->partials, A.G(lo.b_qkv), s));
+    { ProfScope ps(m, PC_BIAS, 0, (double)M * 3 * C * es);
+      CK(launch_colsum<T>(dq, 3 * C, M, 3 * C, m->partials, A.G(lo.b_qkv), s)); }
     CKI(gemm(m, 3 * C, C, M, dq, 3 * C, true, A.h1(l), C, true, epi_f32<T>(A.G(lo.w_qkv), C)));
     CKI(gemm(m, M, C, 3 * C, dq, 3 * C, false, A.W(lo.w_qkv), C, true, epi_store<T>(dC, C, nullptr, nullptr, 0)));
     { ProfScope ps(m, PC_LN_BWD, 0, lnbb);
       CK(launch_ln_bwd<T>(dC, A.x(l), A.mu1(l), A.rs1(l), A.P(lo.ln1_g), m->dres32, m->dres32, drt,
                           m->partials, M, C, &nblk, s));
-      CK(launch_reduce_rows(m->partials, nblk, 2 * C, A.G(lo.ln1_g), s)); }
+      CK(launch_reduce_rows(m->partials, nblk, 2 * C, 3 * C, A.G(lo.ln1_g), s));
+      if (l > 0) CK(launch_reduce_rows(m->partials + 2 * C, nblk, C, 3 * C, A.G(m->L[l - 1].b_fc2), s)); }
   }
   // embeddings: scatter-add by token and by position
+  ProfScope ps_emb(m, PC_EMBED, 0, (double)M * C * 12);
   if (!m->cfg.tied) CK(cudaMemsetAsync(A.G(m->o_wte), 0, (size_t)Vp * C * 4, s));
   CK(cudaMemsetAsync(A.G(m->o_wpe), 0, (size_t)m->Tmax * C * 4, s));
   CK(launch_embed_bwd<T>(m->dres32, m->tok, m->pos, A.G(m->o_wte), A.G(m->o_wpe), M, C, s));

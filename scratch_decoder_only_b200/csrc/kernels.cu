@@ -180,21 +180,16 @@ __global__ void __launch_bounds__(LNB_WARPS * 32)
 ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __restrict__ mean,
               const float* __restrict__ rstd, const float* __restrict__ g, const float* dres_in,
               float* dres_out, T* __restrict__ dres_out_t, float* __restrict__ partials, int M, int C) {
+  // partial row of this block: [dg (C) | db (C) | column sums of dres_out (C)]
   constexpr int NV = Vec<T>::N;
   constexpr int NCH = LN_MAXC / (32 * NV);
   int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int nch = C / NV;
-  float dg[NCH][NV], db[NCH][NV], gg[NCH][NV];
+  float dg[NCH][NV], db[NCH][NV], dsm[NCH][NV];
 #pragma unroll
-  for (int i = 0; i < NCH; ++i) {
-    int ch = lane + i * 32;
+  for (int i = 0; i < NCH; ++i)
 #pragma unroll
-    for (int j = 0; j < NV; ++j) { dg[i][j] = 0.f; db[i][j] = 0.f; gg[i][j] = 0.f; }
-    if (ch < nch) {
-#pragma unroll
-      for (int j = 0; j < NV; j += 4) Vec<float>::load(g + ch * NV + j, gg[i] + j);
-    }
-  }
+    for (int j = 0; j < NV; ++j) { dg[i][j] = 0.f; db[i][j] = 0.f; dsm[i][j] = 0.f; }
   for (int row = blockIdx.x * LNB_WARPS + warp; row < M; row += gridDim.x * LNB_WARPS) {
     float mu = mean[row], rs = rstd[row];
     const T* dyr = dy + (long)row * C;
@@ -205,13 +200,15 @@ ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __
     for (int i = 0; i < NCH; ++i) {
       int ch = lane + i * 32;
       if (ch < nch) {
-        float dv[NV];
+        float dv[NV], gg[NV];
         Vec<T>::load(dyr + ch * NV, dv);
         Vec<T>::load(xr + ch * NV, xh[i]);
 #pragma unroll
+        for (int j = 0; j < NV; j += 4) Vec<float>::load(g + ch * NV + j, gg + j);
+#pragma unroll
         for (int j = 0; j < NV; ++j) {
           xh[i][j] = (xh[i][j] - mu) * rs;
-          gh[i][j] = dv[j] * gg[i][j];
+          gh[i][j] = dv[j] * gg[j];
           s1 += gh[i][j];
           s2 += gh[i][j] * xh[i][j];
           dg[i][j] += dv[j] * xh[i][j];
@@ -235,17 +232,20 @@ ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __
           for (int j = 0; j < NV; ++j) o[j] = 0.f;
         }
 #pragma unroll
-        for (int j = 0; j < NV; ++j) o[j] += rs * (gh[i][j] - s1 - xh[i][j] * s2);
+        for (int j = 0; j < NV; ++j) {
+          o[j] += rs * (gh[i][j] - s1 - xh[i][j] * s2);
+          dsm[i][j] += o[j];
+        }
 #pragma unroll
         for (int j = 0; j < NV; j += 4) Vec<float>::store(dres_out + off + j, o + j);
         Vec<T>::store(dres_out_t + off, o);
       }
     }
   }
-  // block-level reduction of the dg / db partials through shared memory
-  __shared__ float red[LNB_WARPS][2 * LN_MAXC / 8];   // reused in column slabs
-  constexpr int SLAB = 2 * LN_MAXC / 8;                 // columns per pass (256)
-  for (int base = 0; base < 2 * C; base += SLAB) {
+  // block-level reduction of the three partial rows through shared memory
+  constexpr int SLAB = 256;
+  __shared__ float red[LNB_WARPS][SLAB];
+  for (int base = 0; base < 3 * C; base += SLAB) {
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
       int ch = lane + i * 32;
@@ -255,15 +255,16 @@ ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __
           int c = ch * NV + j;
           if (c >= base && c < base + SLAB) red[warp][c - base] = dg[i][j];
           if (C + c >= base && C + c < base + SLAB) red[warp][C + c - base] = db[i][j];
+          if (2 * C + c >= base && 2 * C + c < base + SLAB) red[warp][2 * C + c - base] = dsm[i][j];
         }
       }
     }
     __syncthreads();
-    for (int c = threadIdx.x; c < SLAB && base + c < 2 * C; c += blockDim.x) {
+    for (int c = threadIdx.x; c < SLAB && base + c < 3 * C; c += blockDim.x) {
       float acc = 0.f;
 #pragma unroll
       for (int w = 0; w < LNB_WARPS; ++w) acc += red[w][c];
-      partials[(long)blockIdx.x * 2 * C + base + c] = acc;
+      partials[(long)blockIdx.x * 3 * C + base + c] = acc;
     }
     __syncthreads();
   }
@@ -274,7 +275,7 @@ cudaError_t launch_ln_bwd(const T* dy, const T* x, const float* mean, const floa
                           const float* dres_in, float* dres_out, T* dres_out_t, float* partials,
                           int M, int C, int* nblk_out, cudaStream_t s) {
   int nblk = (M + LNB_WARPS - 1) / LNB_WARPS;
-  if (nblk > 296) nblk = 296;
+  if (nblk > 148 * 3) nblk = 148 * 3;
   *nblk_out = nblk;
   ++g_kernel_launches;
   ln_bwd_kernel<T><<<nblk, LNB_WARPS * 32, 0, s>>>(dy, x, mean, rstd, g, dres_in, dres_out, dres_out_t,
@@ -282,45 +283,85 @@ cudaError_t launch_ln_bwd(const T* dy, const T* x, const float* mean, const floa
   return cudaGetLastError();
 }
 
-// out[n] = sum over r of partials[r][n], in a fixed order (deterministic).
-__global__ void reduce_rows_kernel(const float* __restrict__ p, int rows, int N, float* __restrict__ out) {
-  int n = blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= N) return;
-  float acc = 0.f;
-  for (int r = 0; r < rows; ++r) acc += p[(long)r * N + n];
-  out[n] = acc;
+// out[n] = sum over r of p[r * ld + n], in a fixed order (deterministic):
+// 32 columns per block, the rows split over 8 warps, 4 loads in flight.
+__global__ void __launch_bounds__(256) reduce_rows_kernel(const float* __restrict__ p, int rows, int N, long ld,
+                                                          float* __restrict__ out) {
+  __shared__ float red[8][33];
+  int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int n = blockIdx.x * 32 + lane;
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  if (n < N) {
+    int r = warp;
+    for (; r + 24 < rows; r += 32) {
+      a0 += p[(long)r * ld + n];
+      a1 += p[(long)(r + 8) * ld + n];
+      a2 += p[(long)(r + 16) * ld + n];
+      a3 += p[(long)(r + 24) * ld + n];
+    }
+    for (; r < rows; r += 8) a0 += p[(long)r * ld + n];
+  }
+  red[warp][lane] = (a0 + a1) + (a2 + a3);
+  __syncthreads();
+  if (warp == 0 && n < N) {
+    float acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) acc += red[w][lane];
+    out[n] = acc;
+  }
 }
 
-cudaError_t launch_reduce_rows(const float* partials, int rows, int N, float* out, cudaStream_t s) {
+cudaError_t launch_reduce_rows(const float* partials, int rows, int N, long ld, float* out, cudaStream_t s) {
   ++g_kernel_launches;
-  reduce_rows_kernel<<<(N + 255) / 256, 256, 0, s>>>(partials, rows, N, out);
+  reduce_rows_kernel<<<(N + 31) / 32, 256, 0, s>>>(partials, rows, N, ld, out);
   return cudaGetLastError();
 }
 
-// Column sums of x [M, N] (bias gradients): stage 1 writes per-row-chunk
-// partials, stage 2 is reduce_rows.
+// Column sums of x [M, N] (bias gradients): blocks of 128 columns x 256 rows
+// (4 columns per lane, 8 warps x 32 rows) write per-row-chunk partials;
+// reduce_rows sums the chunks.
+#define CS_ROWS 256
 template <typename Tin>
-__global__ void colsum_kernel(const Tin* __restrict__ x, long ldx, int M, int N, int chunk,
-                              float* __restrict__ partials) {
-  int n = blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= N) return;
-  int r0 = blockIdx.y * chunk, r1 = min(M, r0 + chunk);
-  float acc = 0.f;
-  for (int r = r0; r < r1; ++r) acc += to_f(x[(long)r * ldx + n]);
-  partials[(long)blockIdx.y * N + n] = acc;
+__global__ void __launch_bounds__(256) colsum_kernel(const Tin* __restrict__ x, long ldx, int M, int N,
+                                                     float* __restrict__ partials) {
+  __shared__ float red[8][128];
+  int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int c0 = blockIdx.x * 128 + lane * 4;
+  int r0 = blockIdx.y * CS_ROWS + warp * (CS_ROWS / 8);
+  int r1 = min(M, r0 + CS_ROWS / 8);
+  float a[4] = {0.f, 0.f, 0.f, 0.f};
+  if (c0 < N) {
+    bool full = c0 + 4 <= N && (ldx & 3) == 0;
+    for (int r = r0; r < r1; ++r) {
+      const Tin* row = x + (long)r * ldx + c0;
+      if (full) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) a[j] += to_f(row[j]);
+      } else {
+        for (int j = 0; j < 4 && c0 + j < N; ++j) a[j] += to_f(row[j]);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) red[warp][lane * 4 + j] = a[j];
+  __syncthreads();
+  if (threadIdx.x < 128) {
+    int c = blockIdx.x * 128 + threadIdx.x;
+    float acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) acc += red[w][threadIdx.x];
+    if (c < N) partials[(long)blockIdx.y * N + c] = acc;
+  }
 }
 
 template <typename Tin>
 cudaError_t launch_colsum(const Tin* x, long ldx, int M, int N, float* partials, float* out, cudaStream_t s) {
-  int rc = M < 128 ? M : 128;
-  int chunk = (M + rc - 1) / rc;
-  rc = (M + chunk - 1) / chunk;
-  dim3 grid((N + 127) / 128, rc);
+  dim3 grid((N + 127) / 128, (M + CS_ROWS - 1) / CS_ROWS);
   ++g_kernel_launches;
-  colsum_kernel<Tin><<<grid, 128, 0, s>>>(x, ldx, M, N, chunk, partials);
+  colsum_kernel<Tin><<<grid, 256, 0, s>>>(x, ldx, M, N, partials);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_reduce_rows(partials, rc, N, out, s);
+  return launch_reduce_rows(partials, grid.y, N, N, out, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -397,9 +438,89 @@ xent_kernel(T* __restrict__ logits, long ldl, const int* __restrict__ tgt, int V
   }
 }
 
+// Same computation with the row staged in shared memory: one HBM read and
+// one HBM write per logit (used when the padded row fits, e.g. 100 KB bf16).
+__device__ __forceinline__ float block_reduce(float v, bool is_max, float* red) {
+  int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  v = is_max ? warp_max(v) : warp_sum(v);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    float x = lane < (int)(blockDim.x >> 5) ? red[lane] : (is_max ? -INFINITY : 0.f);
+    x = is_max ? warp_max(x) : warp_sum(x);
+    if (lane == 0) red[32] = x;
+  }
+  __syncthreads();
+  return red[32];
+}
+
+template <typename T>
+__global__ void __launch_bounds__(XENT_THREADS)
+xent_smem_kernel(T* __restrict__ logits, long ldl, const int* __restrict__ tgt, int V, int Vp,
+                 float* __restrict__ rowloss, const DevScalars* __restrict__ sc) {
+  constexpr int NV = Vec<T>::N;
+  extern __shared__ __align__(16) uint8_t xent_raw[];
+  T* zs = reinterpret_cast<T*>(xent_raw);
+  __shared__ float red[33];
+  const int row = blockIdx.x;
+  T* z = logits + (long)row * ldl;
+  const int tg = tgt[row];
+  const int nvec = (Vp + NV - 1) / NV;   // ldl >= nvec * NV
+  float m = -INFINITY;
+  for (int i = threadIdx.x; i < nvec; i += XENT_THREADS) {
+    uint4 raw = *reinterpret_cast<const uint4*>(z + i * NV);
+    *reinterpret_cast<uint4*>(zs + i * NV) = raw;
+    float v[NV];
+    Vec<T>::load(zs + i * NV, v);
+#pragma unroll
+    for (int j = 0; j < NV; ++j)
+      if (i * NV + j < V) m = fmaxf(m, v[j]);
+  }
+  m = block_reduce(m, true, red);
+  float ssum = 0.f;
+  for (int i = threadIdx.x; i < nvec; i += XENT_THREADS) {
+    float v[NV];
+    Vec<T>::load(zs + i * NV, v);
+#pragma unroll
+    for (int j = 0; j < NV; ++j)
+      if (i * NV + j < V) ssum += exp2f((v[j] - m) * 1.4426950408889634f);
+  }
+  ssum = block_reduce(ssum, false, red);
+  const float lse = m + logf(ssum);
+  if (threadIdx.x == 0) rowloss[row] = tg >= 0 ? lse - to_f(zs[tg]) : 0.f;
+  const int nv = sc->n_valid;
+  const float scale = tg >= 0 ? sc->loss_scale / (float)(nv > 0 ? nv : 1) : 0.f;
+  for (int i = threadIdx.x; i < nvec; i += XENT_THREADS) {
+    float v[NV];
+    Vec<T>::load(zs + i * NV, v);
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      int c = i * NV + j;
+      float p = c < V ? exp2f((v[j] - lse) * 1.4426950408889634f) : 0.f;
+      v[j] = (p - (c == tg ? 1.f : 0.f)) * scale;
+    }
+    Vec<T>::store(z + i * NV, v);
+  }
+}
+
 template <typename T>
 cudaError_t launch_xent(T* logits, long ldl, const int* tgt, int M, int V, int Vp, float* rowloss,
                         DevScalars* sc, cudaStream_t s) {
+  constexpr int NV = Vec<T>::N;
+  size_t smem = (size_t)((Vp + NV - 1) / NV) * NV * sizeof(T);
+  if (smem <= 200 * 1024 && (ldl % NV) == 0) {
+    static size_t attr = 0;
+    if (smem > attr) {
+      cudaError_t e = cudaFuncSetAttribute(xent_smem_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)smem);
+      if (e != cudaSuccess) return e;
+      attr = smem;
+    }
+    ++g_kernel_launches;
+    xent_smem_kernel<T><<<M, XENT_THREADS, smem, s>>>(logits, ldl, tgt, V, Vp, rowloss, sc);
+    return cudaGetLastError();
+  }
   ++g_kernel_launches;
   xent_kernel<T><<<M, XENT_THREADS, 0, s>>>(logits, ldl, tgt, V, Vp, rowloss, sc);
   return cudaGetLastError();

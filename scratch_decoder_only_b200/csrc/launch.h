@@ -34,11 +34,14 @@ cudaError_t launch_embed_fwd(const int* tok, const int* pos, const float* wte, c
 template <typename T>
 cudaError_t launch_ln_fwd(const T* x, const float* g, const float* b, T* y, float* mean, float* rstd,
                           int M, int C, float eps, cudaStream_t s);
+// partials: [nblk][3C] = dg | db | column sums of dres_out (the bias gradient of
+// the layer whose output gradient dres_out is)
 template <typename T>
 cudaError_t launch_ln_bwd(const T* dy, const T* x, const float* mean, const float* rstd, const float* g,
                           const float* dres_in, float* dres_out, T* dres_out_t, float* partials,
                           int M, int C, int* nblk_out, cudaStream_t s);
-cudaError_t launch_reduce_rows(const float* partials, int rows, int N, float* out, cudaStream_t s);
+// out[n] = sum_r partials[r * ld + n]
+cudaError_t launch_reduce_rows(const float* partials, int rows, int N, long ld, float* out, cudaStream_t s);
 template <typename Tin>
 cudaError_t launch_colsum(const Tin* x, long ldx, int M, int N, float* partials, float* out, cudaStream_t s);
 template <typename T>
