@@ -175,44 +175,46 @@ cudaError_t launch_ln_fwd(const T* x, const float* g, const float* b, T* y, floa
 // partials[block][0..C) and [C..2C).
 // ---------------------------------------------------------------------------
 #define LNB_WARPS 8
-template <typename T>
+template <typename T, int NCH>
 __global__ void __launch_bounds__(LNB_WARPS * 32)
 ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __restrict__ mean,
               const float* __restrict__ rstd, const float* __restrict__ g, const float* dres_in,
               float* dres_out, T* __restrict__ dres_out_t, float* __restrict__ partials, int M, int C) {
-  // partial row of this block: [dg (C) | db (C) | column sums of dres_out (C)]
+  // partial row of this block: [dg (C) | db (C) | column sums of dres_out (C)].
+  // Each warp accumulates its rows' contributions in its own shared-memory
+  // row (a lane owns fixed columns, so no atomics); the block then sums the
+  // warps' rows.
   constexpr int NV = Vec<T>::N;
-  constexpr int NCH = LN_MAXC / (32 * NV);
-  int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int nch = C / NV;
-  float dg[NCH][NV], db[NCH][NV], dsm[NCH][NV];
-#pragma unroll
-  for (int i = 0; i < NCH; ++i)
-#pragma unroll
-    for (int j = 0; j < NV; ++j) { dg[i][j] = 0.f; db[i][j] = 0.f; dsm[i][j] = 0.f; }
+  extern __shared__ float acc_sm[];   // [LNB_WARPS][3C]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nch = C / NV;
+  float* my = acc_sm + (long)warp * 3 * C;
+  for (int c = lane; c < 3 * C; c += 32) my[c] = 0.f;
+  __syncwarp();
   for (int row = blockIdx.x * LNB_WARPS + warp; row < M; row += gridDim.x * LNB_WARPS) {
-    float mu = mean[row], rs = rstd[row];
+    const float mu = mean[row], rs = rstd[row];
     const T* dyr = dy + (long)row * C;
     const T* xr = x + (long)row * C;
     float xh[NCH][NV], gh[NCH][NV];
     float s1 = 0.f, s2 = 0.f;
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
-      int ch = lane + i * 32;
+      const int ch = lane + i * 32;
       if (ch < nch) {
         float dv[NV], gg[NV];
         Vec<T>::load(dyr + ch * NV, dv);
         Vec<T>::load(xr + ch * NV, xh[i]);
 #pragma unroll
         for (int j = 0; j < NV; j += 4) Vec<float>::load(g + ch * NV + j, gg + j);
+        float* a = my + ch * NV;
 #pragma unroll
         for (int j = 0; j < NV; ++j) {
           xh[i][j] = (xh[i][j] - mu) * rs;
           gh[i][j] = dv[j] * gg[j];
           s1 += gh[i][j];
           s2 += gh[i][j] * xh[i][j];
-          dg[i][j] += dv[j] * xh[i][j];
-          db[i][j] += dv[j];
+          a[j] += dv[j] * xh[i][j];
+          a[C + j] += dv[j];
         }
       }
     }
@@ -220,9 +222,9 @@ ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __
     s2 = warp_sum(s2) / C;
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
-      int ch = lane + i * 32;
+      const int ch = lane + i * 32;
       if (ch < nch) {
-        long off = (long)row * C + ch * NV;
+        const long off = (long)row * C + ch * NV;
         float o[NV];
         if (dres_in) {
 #pragma unroll
@@ -231,10 +233,11 @@ ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __
 #pragma unroll
           for (int j = 0; j < NV; ++j) o[j] = 0.f;
         }
+        float* a = my + 2 * C + ch * NV;
 #pragma unroll
         for (int j = 0; j < NV; ++j) {
           o[j] += rs * (gh[i][j] - s1 - xh[i][j] * s2);
-          dsm[i][j] += o[j];
+          a[j] += o[j];
         }
 #pragma unroll
         for (int j = 0; j < NV; j += 4) Vec<float>::store(dres_out + off + j, o + j);
@@ -242,32 +245,30 @@ ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __
       }
     }
   }
-  // block-level reduction of the three partial rows through shared memory
-  constexpr int SLAB = 256;
-  __shared__ float red[LNB_WARPS][SLAB];
-  for (int base = 0; base < 3 * C; base += SLAB) {
+  __syncthreads();
+  for (int c = threadIdx.x; c < 3 * C; c += blockDim.x) {
+    float acc = 0.f;
 #pragma unroll
-    for (int i = 0; i < NCH; ++i) {
-      int ch = lane + i * 32;
-      if (ch < nch) {
-#pragma unroll
-        for (int j = 0; j < NV; ++j) {
-          int c = ch * NV + j;
-          if (c >= base && c < base + SLAB) red[warp][c - base] = dg[i][j];
-          if (C + c >= base && C + c < base + SLAB) red[warp][C + c - base] = db[i][j];
-          if (2 * C + c >= base && 2 * C + c < base + SLAB) red[warp][2 * C + c - base] = dsm[i][j];
-        }
-      }
-    }
-    __syncthreads();
-    for (int c = threadIdx.x; c < SLAB && base + c < 3 * C; c += blockDim.x) {
-      float acc = 0.f;
-#pragma unroll
-      for (int w = 0; w < LNB_WARPS; ++w) acc += red[w][c];
-      partials[(long)blockIdx.x * 3 * C + base + c] = acc;
-    }
-    __syncthreads();
+    for (int w = 0; w < LNB_WARPS; ++w) acc += acc_sm[(long)w * 3 * C + c];
+    partials[(long)blockIdx.x * 3 * C + c] = acc;
   }
+}
+
+template <typename T, int NCH>
+static cudaError_t ln_bwd_launch(const T* dy, const T* x, const float* mean, const float* rstd, const float* g,
+                                 const float* dres_in, float* dres_out, T* dres_out_t, float* partials, int M,
+                                 int C, int nblk, cudaStream_t s) {
+  size_t smem = (size_t)LNB_WARPS * 3 * C * sizeof(float);
+  static size_t attr = 0;
+  if (smem > attr) {
+    cudaError_t e = cudaFuncSetAttribute(ln_bwd_kernel<T, NCH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr = smem;
+  }
+  ++g_kernel_launches;
+  ln_bwd_kernel<T, NCH><<<nblk, LNB_WARPS * 32, smem, s>>>(dy, x, mean, rstd, g, dres_in, dres_out, dres_out_t,
+                                                           partials, M, C);
+  return cudaGetLastError();
 }
 
 template <typename T>
@@ -277,10 +278,15 @@ cudaError_t launch_ln_bwd(const T* dy, const T* x, const float* mean, const floa
   int nblk = (M + LNB_WARPS - 1) / LNB_WARPS;
   if (nblk > 148 * 3) nblk = 148 * 3;
   *nblk_out = nblk;
-  ++g_kernel_launches;
-  ln_bwd_kernel<T><<<nblk, LNB_WARPS * 32, 0, s>>>(dy, x, mean, rstd, g, dres_in, dres_out, dres_out_t,
-                                                    partials, M, C);
-  return cudaGetLastError();
+  constexpr int NV = Vec<T>::N;
+  int per_lane = (C / NV + 31) / 32;   // 16-byte chunks per lane
+  switch (per_lane) {
+    case 1: return ln_bwd_launch<T, 1>(dy, x, mean, rstd, g, dres_in, dres_out, dres_out_t, partials, M, C, nblk, s);
+    case 2: return ln_bwd_launch<T, 2>(dy, x, mean, rstd, g, dres_in, dres_out, dres_out_t, partials, M, C, nblk, s);
+    case 3: return ln_bwd_launch<T, 3>(dy, x, mean, rstd, g, dres_in, dres_out, dres_out_t, partials, M, C, nblk, s);
+    case 4: return ln_bwd_launch<T, 4>(dy, x, mean, rstd, g, dres_in, dres_out, dres_out_t, partials, M, C, nblk, s);
+    default: return ln_bwd_launch<T, 8>(dy, x, mean, rstd, g, dres_in, dres_out, dres_out_t, partials, M, C, nblk, s);
+  }
 }
 
 // out[n] = sum over r of p[r * ld + n], in a fixed order (deterministic):
