@@ -183,7 +183,8 @@ ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __
   // partial row of this block: [dg (C) | db (C) | column sums of dres_out (C)].
   // Each warp accumulates its rows' contributions in its own shared-memory
   // row (a lane owns fixed columns, so no atomics); the block then sums the
-  // warps' rows.
+  // warps' rows.  Element j of 16-byte chunk ch of section s sits at
+  // s*C + j*nch + ch, so the 32 lanes of a warp touch 32 consecutive banks.
   constexpr int NV = Vec<T>::N;
   extern __shared__ float acc_sm[];   // [LNB_WARPS][3C]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -206,15 +207,15 @@ ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __
         Vec<T>::load(xr + ch * NV, xh[i]);
 #pragma unroll
         for (int j = 0; j < NV; j += 4) Vec<float>::load(g + ch * NV + j, gg + j);
-        float* a = my + ch * NV;
+        float* a = my + ch;
 #pragma unroll
         for (int j = 0; j < NV; ++j) {
           xh[i][j] = (xh[i][j] - mu) * rs;
           gh[i][j] = dv[j] * gg[j];
           s1 += gh[i][j];
           s2 += gh[i][j] * xh[i][j];
-          a[j] += dv[j] * xh[i][j];
-          a[C + j] += dv[j];
+          a[j * nch] += dv[j] * xh[i][j];
+          a[C + j * nch] += dv[j];
         }
       }
     }
@@ -233,11 +234,11 @@ ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __
 #pragma unroll
           for (int j = 0; j < NV; ++j) o[j] = 0.f;
         }
-        float* a = my + 2 * C + ch * NV;
+        float* a = my + 2 * C + ch;
 #pragma unroll
         for (int j = 0; j < NV; ++j) {
           o[j] += rs * (gh[i][j] - s1 - xh[i][j] * s2);
-          a[j] += o[j];
+          a[j * nch] += o[j];
         }
 #pragma unroll
         for (int j = 0; j < NV; j += 4) Vec<float>::store(dres_out + off + j, o + j);
@@ -247,9 +248,11 @@ ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __
   }
   __syncthreads();
   for (int c = threadIdx.x; c < 3 * C; c += blockDim.x) {
+    const int sec = c / C, cc = c % C;
+    const int idx = sec * C + (cc % NV) * nch + cc / NV;
     float acc = 0.f;
 #pragma unroll
-    for (int w = 0; w < LNB_WARPS; ++w) acc += acc_sm[(long)w * 3 * C + c];
+    for (int w = 0; w < LNB_WARPS; ++w) acc += acc_sm[(long)w * 3 * C + idx];
     partials[(long)blockIdx.x * 3 * C + c] = acc;
   }
 }
