@@ -6,21 +6,28 @@
 // KV cache layout: kc/vc [B][H][Tmax][d] per layer.
 #include "launch.h"
 
+// pos = pos0 + *step (the step counter lives on the device so that one
+// captured decode step can be replayed).
 template <typename T>
 __global__ void dec_embed_kernel(const int* __restrict__ tok, const float* __restrict__ wte,
-                                 const float* __restrict__ wpe, T* __restrict__ x, int C, int pos) {
+                                 const float* __restrict__ wpe, T* __restrict__ x, int C, int pos0,
+                                 const int* __restrict__ step, int max_seq, unsigned* err) {
   int b = blockIdx.x;
+  int pos = pos0 + *step;
+  if (pos < 0 || pos >= max_seq) {
+    if (b == 0 && threadIdx.x == 0) set_dev_err(err, GPT_DEVERR_POS);
+    pos = pos < 0 ? 0 : max_seq - 1;
+  }
   const float* a = wte + (long)tok[b] * C;
   const float* p = wpe + (long)pos * C;
   for (int c = threadIdx.x; c < C; c += blockDim.x) x[(long)b * C + c] = from_f<T>(a[c] + p[c]);
 }
 
 template <typename T>
-cudaError_t launch_dec_embed(const int* tok, const float* wte, const float* wpe, T* x, int B, int C, int pos,
-                             int max_seq, unsigned* err, cudaStream_t s) {
-  if (pos < 0 || pos >= max_seq) return cudaErrorInvalidValue;
+cudaError_t launch_dec_embed(const int* tok, const float* wte, const float* wpe, T* x, int B, int C, int pos0,
+                             const int* step, int max_seq, unsigned* err, cudaStream_t s) {
   ++g_kernel_launches;
-  dec_embed_kernel<T><<<B, 256, 0, s>>>(tok, wte, wpe, x, C, pos);
+  dec_embed_kernel<T><<<B, 256, 0, s>>>(tok, wte, wpe, x, C, pos0, step, max_seq, err);
   return cudaGetLastError();
 }
 
@@ -128,8 +135,11 @@ cudaError_t launch_kv_fill(const T* qkv, T* kc, T* vc, int B, int Tp, int H, int
 // is appended to the cache by the same warp.
 template <typename T, int D>
 __global__ void dec_attn_kernel(const T* __restrict__ qkv, T* kc, T* vc, T* __restrict__ out, int B, int H,
-                                int Tmax, int pos) {
+                                int Tmax, int pos0, const int* __restrict__ step) {
   int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int pos = pos0 + *step;
+  if (pos < 0) pos = 0;
+  if (pos >= Tmax) pos = Tmax - 1;
   int bh = blockIdx.x * 4 + warp;
   if (bh >= B * H) return;
   int b = bh / H, h = bh % H;
@@ -174,14 +184,14 @@ __global__ void dec_attn_kernel(const T* __restrict__ qkv, T* kc, T* vc, T* __re
 }
 
 template <typename T>
-cudaError_t launch_dec_attn(const T* qkv, T* kc, T* vc, T* out, int B, int H, int d, int Tmax, int pos,
-                            cudaStream_t s) {
+cudaError_t launch_dec_attn(const T* qkv, T* kc, T* vc, T* out, int B, int H, int d, int Tmax, int pos0,
+                            const int* step, cudaStream_t s) {
   unsigned g = (B * H + 3) / 4;
   switch (d) {
-    case 16: ++g_kernel_launches; dec_attn_kernel<T, 16><<<g, 128, 0, s>>>(qkv, kc, vc, out, B, H, Tmax, pos); break;
-    case 32: ++g_kernel_launches; dec_attn_kernel<T, 32><<<g, 128, 0, s>>>(qkv, kc, vc, out, B, H, Tmax, pos); break;
-    case 64: ++g_kernel_launches; dec_attn_kernel<T, 64><<<g, 128, 0, s>>>(qkv, kc, vc, out, B, H, Tmax, pos); break;
-    case 128: ++g_kernel_launches; dec_attn_kernel<T, 128><<<g, 128, 0, s>>>(qkv, kc, vc, out, B, H, Tmax, pos); break;
+    case 16: ++g_kernel_launches; dec_attn_kernel<T, 16><<<g, 128, 0, s>>>(qkv, kc, vc, out, B, H, Tmax, pos0, step); break;
+    case 32: ++g_kernel_launches; dec_attn_kernel<T, 32><<<g, 128, 0, s>>>(qkv, kc, vc, out, B, H, Tmax, pos0, step); break;
+    case 64: ++g_kernel_launches; dec_attn_kernel<T, 64><<<g, 128, 0, s>>>(qkv, kc, vc, out, B, H, Tmax, pos0, step); break;
+    case 128: ++g_kernel_launches; dec_attn_kernel<T, 128><<<g, 128, 0, s>>>(qkv, kc, vc, out, B, H, Tmax, pos0, step); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -190,8 +200,9 @@ cudaError_t launch_dec_attn(const T* qkv, T* kc, T* vc, T* out, int B, int H, in
 // Greedy choice: argmax over the real vocabulary of fp32 logits, lowest
 // index on ties.  Writes tok[b] and out[b * out_ld + col].
 __global__ void argmax_kernel(const float* __restrict__ logits, int V, int Vp, int* tok, int32_t* out,
-                              int out_ld, int col) {
+                              int out_ld, const int* __restrict__ step) {
   int b = blockIdx.x;
+  const int col = step ? *step : 0;
   const float* z = logits + (long)b * Vp;
   float best = -INFINITY;
   int bi = 0x7fffffff;
@@ -227,9 +238,16 @@ __global__ void argmax_kernel(const float* __restrict__ logits, int V, int Vp, i
 }
 
 cudaError_t launch_argmax(const float* logits, int B, int V, int Vp, int* tok, int32_t* out, int out_ld,
-                          int col, cudaStream_t s) {
+                          const int* step, cudaStream_t s) {
   ++g_kernel_launches;
-  argmax_kernel<<<B, 1024, 0, s>>>(logits, V, Vp, tok, out, out_ld, col);
+  argmax_kernel<<<B, 1024, 0, s>>>(logits, V, Vp, tok, out, out_ld, step);
+  return cudaGetLastError();
+}
+
+__global__ void step_advance_kernel(int* step) { *step += 1; }
+cudaError_t launch_step_advance(int* step, cudaStream_t s) {
+  ++g_kernel_launches;
+  step_advance_kernel<<<1, 1, 0, s>>>(step);
   return cudaGetLastError();
 }
 
@@ -247,12 +265,13 @@ cudaError_t launch_gather_last(const T* x, int B, int Tp, int C, T* out, cudaStr
 }
 
 #define INSTD(T)                                                                                         \
-  template cudaError_t launch_dec_embed<T>(const int*, const float*, const float*, T*, int, int, int, int, \
-                                           unsigned*, cudaStream_t);                                     \
+  template cudaError_t launch_dec_embed<T>(const int*, const float*, const float*, T*, int, int, int,      \
+                                           const int*, int, unsigned*, cudaStream_t);                    \
   template cudaError_t launch_gemv<T>(const T*, int, int, const T*, int, const float*, const T*, int, T*, T*, \
                                       float*, cudaStream_t);                                             \
   template cudaError_t launch_kv_fill<T>(const T*, T*, T*, int, int, int, int, int, cudaStream_t);         \
-  template cudaError_t launch_dec_attn<T>(const T*, T*, T*, T*, int, int, int, int, int, cudaStream_t);    \
+  template cudaError_t launch_dec_attn<T>(const T*, T*, T*, T*, int, int, int, int, int, const int*,      \
+                                          cudaStream_t);                                                 \
   template cudaError_t launch_gather_last<T>(const T*, int, int, int, T*, cudaStream_t);
 INSTD(float)
 INSTD(bf16)

@@ -45,7 +45,7 @@ struct gpt_model {
   int *tok, *tgt, *pos, *dstart;
   float* dres32;
   void *dres_t, *dC, *dF, *dqkv;
-  float *attD, *rowloss, *partials, *splitws;
+  float *attD, *rowloss, *partials, *splitws, *dq_acc;
   size_t partials_n, splitws_n;
   double* normpart;
   int normblk = 592;
@@ -58,6 +58,12 @@ struct gpt_model {
   std::string err;
   // tracing: per-kernel-class CUDA-event brackets
   bool seg_used = false;
+  // decode: one captured step replayed on an internal stream
+  cudaStream_t cap_stream = nullptr;
+  cudaEvent_t ev_a = nullptr, ev_b = nullptr;
+  cudaGraphExec_t dec_graph = nullptr;
+  int dec_B = 0, dec_Tp = 0, dec_nnew = 0, dec_kernels = 0;
+  int32_t* dec_out = nullptr;
   bool prof = false;
   struct ProfRec { int cls; cudaEvent_t a, b; double flops, bytes; };
   std::vector<ProfRec> recs;
@@ -257,6 +263,7 @@ static int build_arena(gpt_model* m) {
   cv.add(&m->dF, Mx * F * es);
   cv.add(&m->dqkv, Mx * 3 * C * es);
   cv.add((void**)&m->attD, Mx * m->H * 4);
+  cv.add((void**)&m->dq_acc, m->bf16 ? Mx * C * 4 : 4);
   cv.add((void**)&m->rowloss, Mx * 4);
   m->partials_n = std::max((size_t)444 * 3 * C, (size_t)((Mx + 255) / 256) * std::max(3 * C, F));
   cv.add((void**)&m->partials, m->partials_n * 4);
@@ -381,7 +388,8 @@ static int attn_fwd(gpt_model* m, const float* qkv, float* out, float* lse, int 
 }
 static int attn_fwd(gpt_model* m, const bf16* qkv, bf16* out, float* lse, int B, int T) {
   ProfScope ps(m, PC_ATTN_FWD, 4.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0);
-  if (attn_mma_supported(m->d)) CK(launch_attn_fwd_mma(qkv, out, lse, m->dstart, B, T, m->H, m->d, m->stream));
+  if (attn_tc_supported(m->d)) CK(launch_attn_fwd_tc(qkv, out, lse, m->dstart, B, T, m->H, &m->sc->err, m->stream));
+  else if (attn_mma_supported(m->d)) CK(launch_attn_fwd_mma(qkv, out, lse, m->dstart, B, T, m->H, m->d, m->stream));
   else CK(launch_attn_fwd_simt<bf16>(qkv, out, lse, m->dstart, B, T, m->H, m->d, m->stream));
   return GPT_OK;
 }
@@ -394,7 +402,10 @@ static int attn_bwd(gpt_model* m, const float* qkv, const float* out, const floa
 static int attn_bwd(gpt_model* m, const bf16* qkv, const bf16* out, const bf16* dout, const float* lse,
                     bf16* dqkv, int B, int T) {
   ProfScope ps(m, PC_ATTN_BWD, 8.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0);
-  if (attn_mma_supported(m->d))
+  if (attn_tc_supported(m->d))
+    CK(launch_attn_bwd_tc(qkv, out, dout, lse, m->attD, m->dq_acc, m->dstart, dqkv, B, T, m->H, &m->sc->err,
+                          m->stream));
+  else if (attn_mma_supported(m->d))
     CK(launch_attn_bwd_mma(qkv, out, dout, lse, m->attD, m->dstart, dqkv, B, T, m->H, m->d, m->stream));
   else
     CK(launch_attn_bwd_simt<bf16>(qkv, out, dout, lse, m->attD, m->dstart, dqkv, B, T, m->H, m->d, m->stream));
@@ -536,40 +547,81 @@ static int backward_impl(gpt_model* m) {
 // Greedy decoding
 // ---------------------------------------------------------------------------
 template <typename T>
-static int decode_impl(gpt_model* m, const int32_t* prompt, int B, int Tp, int n_new, int32_t* out) {
-  cudaStream_t s = m->stream;
+static int decode_step(gpt_model* m, int B, int Tp, int n_new, int32_t* out, cudaStream_t s) {
   Acts<T> A(m);
   const int C = m->C, F = m->F, H = m->H, d = m->d;
   const float eps = m->cfg.ln_eps;
-  CKI(forward_impl<T>(m, prompt, nullptr, nullptr, B, Tp, nullptr));
-  m->logits_valid = false;
   size_t kvl = (size_t)m->Bmax * H * m->Tmax * d;
   T* kc = (T*)m->kc;
   T* vc = (T*)m->vc;
-  for (int l = 0; l < m->NL; ++l)
-    CK(launch_kv_fill<T>(A.qkv(l), kc + l * kvl, vc + l * kvl, B, Tp, H, d, m->Tmax, s));
   T *x = (T*)m->dx, *h = (T*)m->dh, *q = (T*)m->dq, *att = (T*)m->datt, *u = (T*)m->du, *a = (T*)m->da,
     *xf = (T*)m->dxf;
-  CK(launch_gather_last<T>((const T*)m->xf, B, Tp, C, xf, s));
-  CK(launch_gemv<T>(xf, B, C, A.W(m->o_head), m->Vp, nullptr, nullptr, 2, nullptr, nullptr, m->dlogits, s));
-  CK(launch_argmax(m->dlogits, B, m->V, m->Vp, m->dtok, out, n_new, 0, s));
-  for (int st = 1; st < n_new; ++st) {
-    int pos = Tp + st - 1;
-    CK(launch_dec_embed<T>(m->dtok, A.P(m->o_wte), A.P(m->o_wpe), x, B, C, pos, m->Tmax, &m->sc->err, s));
-    for (int l = 0; l < m->NL; ++l) {
-      const LayerOff& lo = m->L[l];
-      CK(launch_ln_fwd<T>(x, A.P(lo.ln1_g), A.P(lo.ln1_b), h, m->dmu, m->drs, B, C, eps, s));
-      CK(launch_gemv<T>(h, B, C, A.W(lo.w_qkv), 3 * C, A.P(lo.b_qkv), nullptr, 0, q, nullptr, nullptr, s));
-      CK(launch_dec_attn<T>(q, kc + l * kvl, vc + l * kvl, att, B, H, d, m->Tmax, pos, s));
-      CK(launch_gemv<T>(att, B, C, A.W(lo.w_o), C, A.P(lo.b_o), x, 0, x, nullptr, nullptr, s));
-      CK(launch_ln_fwd<T>(x, A.P(lo.ln2_g), A.P(lo.ln2_b), h, m->dmu, m->drs, B, C, eps, s));
-      CK(launch_gemv<T>(h, B, C, A.W(lo.w_fc), F, A.P(lo.b_fc), nullptr, 1, u, a, nullptr, s));
-      CK(launch_gemv<T>(a, B, F, A.W(lo.w_fc2), C, A.P(lo.b_fc2), x, 0, x, nullptr, nullptr, s));
-    }
-    CK(launch_ln_fwd<T>(x, A.P(m->o_lnf_g), A.P(m->o_lnf_b), xf, m->dmu, m->drs, B, C, eps, s));
-    CK(launch_gemv<T>(xf, B, C, A.W(m->o_head), m->Vp, nullptr, nullptr, 2, nullptr, nullptr, m->dlogits, s));
-    CK(launch_argmax(m->dlogits, B, m->V, m->Vp, m->dtok, out, n_new, st, s));
+  int* stepc = &m->sc->dec_step;
+  // the token fed at step st sits at position Tp - 1 + st
+  CK(launch_dec_embed<T>(m->dtok, A.P(m->o_wte), A.P(m->o_wpe), x, B, C, Tp - 1, stepc, m->Tmax, &m->sc->err, s));
+  for (int l = 0; l < m->NL; ++l) {
+    const LayerOff& lo = m->L[l];
+    CK(launch_ln_fwd<T>(x, A.P(lo.ln1_g), A.P(lo.ln1_b), h, m->dmu, m->drs, B, C, eps, s));
+    CK(launch_gemv<T>(h, B, C, A.W(lo.w_qkv), 3 * C, A.P(lo.b_qkv), nullptr, 0, q, nullptr, nullptr, s));
+    CK(launch_dec_attn<T>(q, kc + l * kvl, vc + l * kvl, att, B, H, d, m->Tmax, Tp - 1, stepc, s));
+    CK(launch_gemv<T>(att, B, C, A.W(lo.w_o), C, A.P(lo.b_o), x, 0, x, nullptr, nullptr, s));
+    CK(launch_ln_fwd<T>(x, A.P(lo.ln2_g), A.P(lo.ln2_b), h, m->dmu, m->drs, B, C, eps, s));
+    CK(launch_gemv<T>(h, B, C, A.W(lo.w_fc), F, A.P(lo.b_fc), nullptr, 1, u, a, nullptr, s));
+    CK(launch_gemv<T>(a, B, F, A.W(lo.w_fc2), C, A.P(lo.b_fc2), x, 0, x, nullptr, nullptr, s));
   }
+  CK(launch_ln_fwd<T>(x, A.P(m->o_lnf_g), A.P(m->o_lnf_b), xf, m->dmu, m->drs, B, C, eps, s));
+  CK(launch_gemv<T>(xf, B, C, A.W(m->o_head), m->Vp, nullptr, nullptr, 2, nullptr, nullptr, m->dlogits, s));
+  CK(launch_argmax(m->dlogits, B, m->V, m->Vp, m->dtok, out, n_new, stepc, s));
+  CK(launch_step_advance(stepc, s));
+  return GPT_OK;
+}
+
+template <typename T>
+static int decode_impl(gpt_model* m, const int32_t* prompt, int B, int Tp, int n_new, int32_t* out) {
+  cudaStream_t s = m->stream;
+  Acts<T> A(m);
+  const int C = m->C, H = m->H, d = m->d;
+  CKI(forward_impl<T>(m, prompt, nullptr, nullptr, B, Tp, nullptr));
+  m->logits_valid = false;
+  size_t kvl = (size_t)m->Bmax * H * m->Tmax * d;
+  for (int l = 0; l < m->NL; ++l)
+    CK(launch_kv_fill<T>(A.qkv(l), (T*)m->kc + l * kvl, (T*)m->vc + l * kvl, B, Tp, H, d, m->Tmax, s));
+  // first new token: from the prefill's last position
+  CK(launch_gather_last<T>((const T*)m->xf, B, Tp, C, (T*)m->dxf, s));
+  CK(launch_gemv<T>((const T*)m->dxf, B, C, A.W(m->o_head), m->Vp, nullptr, nullptr, 2, nullptr, nullptr,
+                    m->dlogits, s));
+  CK(launch_argmax(m->dlogits, B, m->V, m->Vp, m->dtok, out, n_new, nullptr, s));
+  if (n_new == 1) return GPT_OK;
+  const int one = 1;
+  CK(cudaMemcpyAsync(&m->sc->dec_step, &one, sizeof(int), cudaMemcpyHostToDevice, s));
+  // later tokens: one captured step (about 7 L + 5 kernels), replayed n_new - 1 times
+  if (!m->cap_stream) CK(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking));
+  if (!m->ev_a) {
+    CK(cudaEventCreateWithFlags(&m->ev_a, cudaEventDisableTiming));
+    CK(cudaEventCreateWithFlags(&m->ev_b, cudaEventDisableTiming));
+  }
+  if (!m->dec_graph || m->dec_B != B || m->dec_Tp != Tp || m->dec_nnew != n_new || m->dec_out != out) {
+    if (m->dec_graph) { cudaGraphExecDestroy(m->dec_graph); m->dec_graph = nullptr; }
+    cudaGraph_t g = nullptr;
+    unsigned long long n0 = g_kernel_launches;
+    CK(cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
+    int r = decode_step<T>(m, B, Tp, n_new, out, m->cap_stream);
+    cudaError_t ec = cudaStreamEndCapture(m->cap_stream, &g);
+    if (r != GPT_OK) { if (g) cudaGraphDestroy(g); return r; }
+    CK(ec);
+    cudaError_t ei = cudaGraphInstantiate(&m->dec_graph, g, 0);
+    cudaGraphDestroy(g);
+    CK(ei);
+    g_kernel_launches = n0;
+    m->dec_kernels = 7 * m->NL + 5;
+    m->dec_B = B; m->dec_Tp = Tp; m->dec_nnew = n_new; m->dec_out = out;
+  }
+  CK(cudaEventRecord(m->ev_a, s));
+  CK(cudaStreamWaitEvent(m->cap_stream, m->ev_a, 0));
+  for (int st = 1; st < n_new; ++st) CK(cudaGraphLaunch(m->dec_graph, m->cap_stream));
+  g_kernel_launches += (unsigned long long)m->dec_kernels * (n_new - 1);
+  CK(cudaEventRecord(m->ev_b, m->cap_stream));
+  CK(cudaStreamWaitEvent(s, m->ev_b, 0));
   return GPT_OK;
 }
 
@@ -641,6 +693,10 @@ void gpt_destroy(gpt_model* m) {
   if (!m) return;
   cudaDeviceSynchronize();
   for (auto e : m->evpool) cudaEventDestroy(e);
+  if (m->dec_graph) cudaGraphExecDestroy(m->dec_graph);
+  if (m->ev_a) cudaEventDestroy(m->ev_a);
+  if (m->ev_b) cudaEventDestroy(m->ev_b);
+  if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
   if (m->arena) cudaFree(m->arena);
   delete m;
 }

@@ -174,24 +174,23 @@ cudaError_t launch_ln_fwd(const T* x, const float* g, const float* b, T* y, floa
 // per-block partial sums of dg = sum dy*xhat and db = sum dy go to
 // partials[block][0..C) and [C..2C).
 // ---------------------------------------------------------------------------
-#define LNB_WARPS 8
+#define LNB_WARPS 4
+// NCH = 16-byte chunks per lane (C <= 32 * NCH * Vec<T>::N): the row and the
+// warp's column accumulators stay in registers.
 template <typename T, int NCH>
 __global__ void __launch_bounds__(LNB_WARPS * 32)
 ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __restrict__ mean,
               const float* __restrict__ rstd, const float* __restrict__ g, const float* dres_in,
               float* dres_out, T* __restrict__ dres_out_t, float* __restrict__ partials, int M, int C) {
-  // partial row of this block: [dg (C) | db (C) | column sums of dres_out (C)].
-  // Each warp accumulates its rows' contributions in its own shared-memory
-  // row (a lane owns fixed columns, so no atomics); the block then sums the
-  // warps' rows.  Element j of 16-byte chunk ch of section s sits at
-  // s*C + j*nch + ch, so the 32 lanes of a warp touch 32 consecutive banks.
+  // partial row of this block: [dg (C) | db (C) | column sums of dres_out (C)]
   constexpr int NV = Vec<T>::N;
-  extern __shared__ float acc_sm[];   // [LNB_WARPS][3C]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nch = C / NV;
-  float* my = acc_sm + (long)warp * 3 * C;
-  for (int c = lane; c < 3 * C; c += 32) my[c] = 0.f;
-  __syncwarp();
+  float dg[NCH][NV], db[NCH][NV], dsm[NCH][NV];
+#pragma unroll
+  for (int i = 0; i < NCH; ++i)
+#pragma unroll
+    for (int j = 0; j < NV; ++j) { dg[i][j] = 0.f; db[i][j] = 0.f; dsm[i][j] = 0.f; }
   for (int row = blockIdx.x * LNB_WARPS + warp; row < M; row += gridDim.x * LNB_WARPS) {
     const float mu = mean[row], rs = rstd[row];
     const T* dyr = dy + (long)row * C;
@@ -207,15 +206,14 @@ ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __
         Vec<T>::load(xr + ch * NV, xh[i]);
 #pragma unroll
         for (int j = 0; j < NV; j += 4) Vec<float>::load(g + ch * NV + j, gg + j);
-        float* a = my + ch;
 #pragma unroll
         for (int j = 0; j < NV; ++j) {
           xh[i][j] = (xh[i][j] - mu) * rs;
           gh[i][j] = dv[j] * gg[j];
           s1 += gh[i][j];
           s2 += gh[i][j] * xh[i][j];
-          a[j * nch] += dv[j] * xh[i][j];
-          a[C + j * nch] += dv[j];
+          dg[i][j] += dv[j] * xh[i][j];
+          db[i][j] += dv[j];
         }
       }
     }
@@ -234,11 +232,10 @@ ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __
 #pragma unroll
           for (int j = 0; j < NV; ++j) o[j] = 0.f;
         }
-        float* a = my + 2 * C + ch;
 #pragma unroll
         for (int j = 0; j < NV; ++j) {
           o[j] += rs * (gh[i][j] - s1 - xh[i][j] * s2);
-          a[j * nch] += o[j];
+          dsm[i][j] += o[j];
         }
 #pragma unroll
         for (int j = 0; j < NV; j += 4) Vec<float>::store(dres_out + off + j, o + j);
@@ -246,14 +243,26 @@ ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __
       }
     }
   }
-  __syncthreads();
-  for (int c = threadIdx.x; c < 3 * C; c += blockDim.x) {
-    const int sec = c / C, cc = c % C;
-    const int idx = sec * C + (cc % NV) * nch + cc / NV;
-    float acc = 0.f;
+  // sum the warps' accumulators through shared memory, one section at a time
+  extern __shared__ float red_sm[];   // [LNB_WARPS][C]
+  for (int sec = 0; sec < 3; ++sec) {
 #pragma unroll
-    for (int w = 0; w < LNB_WARPS; ++w) acc += acc_sm[(long)w * 3 * C + idx];
-    partials[(long)blockIdx.x * 3 * C + c] = acc;
+    for (int i = 0; i < NCH; ++i) {
+      const int ch = lane + i * 32;
+      if (ch < nch) {
+#pragma unroll
+        for (int j = 0; j < NV; ++j)
+          red_sm[warp * C + ch * NV + j] = sec == 0 ? dg[i][j] : (sec == 1 ? db[i][j] : dsm[i][j]);
+      }
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < LNB_WARPS; ++w) acc += red_sm[w * C + c];
+      partials[(long)blockIdx.x * 3 * C + sec * C + c] = acc;
+    }
+    __syncthreads();
   }
 }
 
@@ -261,13 +270,7 @@ template <typename T, int NCH>
 static cudaError_t ln_bwd_launch(const T* dy, const T* x, const float* mean, const float* rstd, const float* g,
                                  const float* dres_in, float* dres_out, T* dres_out_t, float* partials, int M,
                                  int C, int nblk, cudaStream_t s) {
-  size_t smem = (size_t)LNB_WARPS * 3 * C * sizeof(float);
-  static size_t attr = 0;
-  if (smem > attr) {
-    cudaError_t e = cudaFuncSetAttribute(ln_bwd_kernel<T, NCH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr = smem;
-  }
+  size_t smem = (size_t)LNB_WARPS * C * sizeof(float);
   ++g_kernel_launches;
   ln_bwd_kernel<T, NCH><<<nblk, LNB_WARPS * 32, smem, s>>>(dy, x, mean, rstd, g, dres_in, dres_out, dres_out_t,
                                                            partials, M, C);
@@ -487,27 +490,33 @@ xent_smem_kernel(T* __restrict__ logits, long ldl, const int* __restrict__ tgt, 
       if (i * NV + j < V) m = fmaxf(m, v[j]);
   }
   m = block_reduce(m, true, red);
+  // e = exp(z - max), kept in place of z (z[target] is read first); the
+  // second pass only scales: dz = e / sum - onehot
+  const float zt = tg >= 0 ? to_f(zs[tg]) : 0.f;
+  __syncthreads();
   float ssum = 0.f;
   for (int i = threadIdx.x; i < nvec; i += XENT_THREADS) {
     float v[NV];
     Vec<T>::load(zs + i * NV, v);
 #pragma unroll
-    for (int j = 0; j < NV; ++j)
-      if (i * NV + j < V) ssum += exp2f((v[j] - m) * 1.4426950408889634f);
+    for (int j = 0; j < NV; ++j) {
+      v[j] = i * NV + j < V ? exp2f((v[j] - m) * 1.4426950408889634f) : 0.f;
+      ssum += v[j];
+    }
+    Vec<T>::store(zs + i * NV, v);
   }
   ssum = block_reduce(ssum, false, red);
-  const float lse = m + logf(ssum);
-  if (threadIdx.x == 0) rowloss[row] = tg >= 0 ? lse - to_f(zs[tg]) : 0.f;
+  if (threadIdx.x == 0) rowloss[row] = tg >= 0 ? m + logf(ssum) - zt : 0.f;
   const int nv = sc->n_valid;
   const float scale = tg >= 0 ? sc->loss_scale / (float)(nv > 0 ? nv : 1) : 0.f;
+  const float inv = scale / ssum;
   for (int i = threadIdx.x; i < nvec; i += XENT_THREADS) {
     float v[NV];
     Vec<T>::load(zs + i * NV, v);
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
       int c = i * NV + j;
-      float p = c < V ? exp2f((v[j] - lse) * 1.4426950408889634f) : 0.f;
-      v[j] = (p - (c == tg ? 1.f : 0.f)) * scale;
+      v[j] = v[j] * inv - (c == tg ? scale : 0.f);
     }
     Vec<T>::store(z + i * NV, v);
   }

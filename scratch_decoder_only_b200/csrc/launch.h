@@ -90,19 +90,30 @@ cudaError_t launch_attn_bwd_mma(const bf16* qkv, const bf16* out, const bf16* do
                                 float* Dbuf, const int* dstart, bf16* dqkv, int B, int T_, int H, int d,
                                 cudaStream_t s);
 
+// ---- attention_tc.cu: head size 64 on tcgen05 (dq_acc: fp32 [B*T, C] scratch)
+bool attn_tc_supported(int d);
+cudaError_t launch_attn_fwd_tc(const bf16* qkv, bf16* out, float* lse, const int* dstart, int B, int T, int H,
+                               unsigned* err, cudaStream_t s);
+cudaError_t launch_attn_bwd_tc(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* Dbuf,
+                               float* dq_acc, const int* dstart, bf16* dqkv, int B, int T, int H, unsigned* err,
+                               cudaStream_t s);
+
 // ---- decode.cu
+// decode kernels read the position as pos0 + *step (device counter)
 template <typename T>
-cudaError_t launch_dec_embed(const int* tok, const float* wte, const float* wpe, T* x, int B, int C, int pos,
-                             int max_seq, unsigned* err, cudaStream_t s);
+cudaError_t launch_dec_embed(const int* tok, const float* wte, const float* wpe, T* x, int B, int C, int pos0,
+                             const int* step, int max_seq, unsigned* err, cudaStream_t s);
 template <typename T>
 cudaError_t launch_gemv(const T* X, int B, int K, const T* W, int N, const float* bias, const T* resid,
                         int mode, T* out, T* out2, float* outf, cudaStream_t s);
 template <typename T>
 cudaError_t launch_kv_fill(const T* qkv, T* kc, T* vc, int B, int Tp, int H, int d, int Tmax, cudaStream_t s);
 template <typename T>
-cudaError_t launch_dec_attn(const T* qkv, T* kc, T* vc, T* out, int B, int H, int d, int Tmax, int pos,
-                            cudaStream_t s);
+cudaError_t launch_dec_attn(const T* qkv, T* kc, T* vc, T* out, int B, int H, int d, int Tmax, int pos0,
+                            const int* step, cudaStream_t s);
+// out[b * out_ld + (*step or 0)] = argmax; tok[b] = argmax
 cudaError_t launch_argmax(const float* logits, int B, int V, int Vp, int* tok, int32_t* out, int out_ld,
-                          int col, cudaStream_t s);
+                          const int* step, cudaStream_t s);
+cudaError_t launch_step_advance(int* step, cudaStream_t s);
 template <typename T>
 cudaError_t launch_gather_last(const T* x, int B, int Tp, int C, T* out, cudaStream_t s);
