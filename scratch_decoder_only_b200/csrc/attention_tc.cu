@@ -3,27 +3,26 @@
 // dstart[i] <= j <= i).  Same layouts as the other attention kernels: qkv
 // [B*T, 3C], out / dout [B*T, C], lse / D [B, H, T].
 //
-// One 192-thread CTA per tile, warp-specialised like the GEMM:
-//   warp 0     TMA producer (128-row tiles of Q, K, V, dO; 128-byte swizzle)
+// Every kernel is a 192-thread CTA, warp-specialised like the GEMM:
+//   warp 0     TMA producer (tiles of Q, K, V, dO with a 128-byte swizzle)
 //   warp 1     MMA issuer (one thread; tcgen05.mma kind::f16, M = 128)
-//   warps 2-5  "softmax" warps: thread t owns accumulator row t (TMEM lane t);
-//              they read scores from TMEM, form P (and dS), write them to
-//              shared memory as the next MMA's operand, and run the epilogues.
+//   warps 2-5  elementwise warps: thread t owns accumulator row t (TMEM lane
+//              t); they read scores from TMEM, write P or dS to shared memory
+//              as the next MMA's operand, and run the epilogue.
+// A CTA works through its blocks one after another; latency is hidden by
+// running 2-3 CTAs per SM (each takes 128-256 TMEM columns, 64-96 KB smem).
 //
-// Forward (CTA = 128 queries): per 128-key block, S = Q K^T into one of two
-// TMEM buffers (the next block's S is computed while this one is being
-// exponentiated), P = exp2(S log2e / sqrt(d) - m) to shared memory,
-// O_blk = P V into TMEM, accumulated in registers with the online-softmax
-// correction.  Writes O and the row log-sum-exp.
-//
-// Backward (CTA = 128 keys; K, V resident): per 128-query block, S^T = K Q^T
-// and dP^T = V dO^T into TMEM; P^T = exp2(S^T ... - lse), dS^T = P^T (dP^T - D)
-// to shared memory; dV += P^T dO and dK += dS^T Q accumulate in TMEM across
-// query blocks; dQ_blk = dS K goes to TMEM and is added into an fp32 dQ
-// accumulator in global memory with one TMA bulk reduce-add per tile (no
-// per-element atomics).  The same shared-memory tiles serve as K-major and
-// MN-major operands (a 64-wide bf16 row is exactly one 128-byte swizzle atom).
-// Key / query blocks outside the document ranges are skipped, not masked.
+//   forward  CTA = 128 queries, 64-key blocks: S = Q K^T (TMEM), P =
+//            exp2(S log2e / 8 - m) (smem), O_blk = P V (TMEM), accumulated in
+//            registers with the online-softmax correction; writes O, lse.
+//   dK / dV  CTA = 128 keys, 64-query blocks: S^T = K Q^T, dP^T = V dO^T
+//            (TMEM); P^T and dS^T = P^T (dP^T - D) (smem); dV += P^T dO and
+//            dK += dS^T Q accumulate in TMEM across query blocks.
+//   dQ       CTA = 128 queries, 64-key blocks: S, dP (TMEM); dS (smem);
+//            dQ += dS K in TMEM.
+// A 64-wide bf16 row is one 128-byte swizzle atom, so one shared-memory tile
+// serves as a K-major operand and as an MN-major one.  Blocks outside the
+// document ranges are skipped, not masked.
 #include "tc_common.cuh"
 
 #define AT_D 64
@@ -70,23 +69,51 @@ __device__ __forceinline__ void trap_timeout(volatile int* abort_flag, unsigned*
   atomicOr(err, GPT_DEVERR_TIMEOUT);
 }
 
+#define AT_BK 64                             // iterated block (keys in fwd / dQ, queries in dK dV)
+#define AT_HALF (AT_BK * AT_D * 2)           // 8 KB: 64 rows x 128 B
+
+// Write 32 bf16 values at columns c0..c0+31 (< 64) of row r of a 64-column
+// K-major operand (rows of 128 B, 128-byte swizzle).
+__device__ __forceinline__ void st_row32_64(uint32_t base, int r, int c0, const float* v) {
+  const uint32_t rowb = base + r * 128;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int u = (c0 >> 3) + q;
+    uint32_t a = rowb + ((u ^ (r & 7)) << 4);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk_bf16(v[8 * q], v[8 * q + 1])),
+                 "r"(pk_bf16(v[8 * q + 2], v[8 * q + 3])), "r"(pk_bf16(v[8 * q + 4], v[8 * q + 5])),
+                 "r"(pk_bf16(v[8 * q + 6], v[8 * q + 7]))
+                 : "memory");
+  }
+}
+
+__device__ __forceinline__ void tc_alloc(uint32_t slot, int cols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(cols));
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+}
+__device__ __forceinline__ void tc_dealloc(uint32_t tmem, int cols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(cols));
+}
+
 // ============================================================== forward
 struct FwdSmem {
-  static constexpr int Q = 0;                              // 16 KB
-  static constexpr int KV = Q + AT_TILE_BYTES;             // 2 stages x (K, V)
-  static constexpr int P = KV + 4 * AT_TILE_BYTES;         // 32 KB (two column blocks)
-  static constexpr int BAR = P + 2 * AT_TILE_BYTES;
+  static constexpr int Q = 0;                          // 16 KB: 128 queries
+  static constexpr int KV = Q + AT_TILE_BYTES;         // 2 stages x (K 8 KB, V 8 KB)
+  static constexpr int P = KV + 4 * AT_HALF;           // 16 KB: 128 queries x 64 keys
+  static constexpr int BAR = P + AT_TILE_BYTES;
   static constexpr int TOTAL = BAR + 256;
+  static constexpr int TMEM_COLS = 128;                // S 0..63, O 64..127
 };
 
-__global__ void __launch_bounds__(AT_THREADS, 1)
-attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, float* __restrict__ lse,
-            const int* __restrict__ dstart, int T, int H, unsigned* err) {
+__global__ void __launch_bounds__(AT_THREADS)
+attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV64,
+            bf16* __restrict__ out, float* __restrict__ lse, const int* __restrict__ dstart, int T, int H,
+            unsigned* err) {
   extern __shared__ __align__(1024) uint8_t at_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)at_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = (uint64_t*)(sm + FwdSmem::BAR);
-  // bars: 0 q_full, 1-2 kv_full, 3-4 kv_empty, 5-6 s_full, 7-8 s_free, 9 p_full, 10 o_full, 11 o_free, 12 drain
-  uint32_t* tmem_slot = (uint32_t*)(bars + 13);
+  // bars: 0 q_full, 1-2 kv_full, 3-4 kv_empty, 5 s_full, 6 s_free, 7 p_full, 8 o_full, 9 o_free, 10 drain
+  uint32_t* tmem_slot = (uint32_t*)(bars + 11);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   int* s_info = (int*)(tmem_slot + 2);
   const uint32_t b0 = smem_u32(bars);
@@ -104,47 +131,40 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
 
   if (threadIdx.x == 0) {
     mbar_init(bar(0), 1);
-    for (int i = 1; i <= 2; ++i) mbar_init(bar(i), 1);
-    for (int i = 3; i <= 4; ++i) mbar_init(bar(i), 1);
-    for (int i = 5; i <= 6; ++i) mbar_init(bar(i), 1);
-    for (int i = 7; i <= 8; ++i) mbar_init(bar(i), 4);
+    for (int i = 1; i <= 4; ++i) mbar_init(bar(i), 1);
+    mbar_init(bar(5), 1);
+    mbar_init(bar(6), 4);
+    mbar_init(bar(7), 4);
+    mbar_init(bar(8), 1);
     mbar_init(bar(9), 4);
     mbar_init(bar(10), 1);
-    mbar_init(bar(11), 4);
-    mbar_init(bar(12), 1);
     *abort_flag = 0;
-    const int kb_lo = dsr[q0] / AT_BLK, kb_hi = min(q0 + AT_BLK - 1, T - 1) / AT_BLK;
+    const int kb_lo = dsr[q0] / AT_BK, kb_hi = min(q0 + AT_BLK - 1, T - 1) / AT_BK;
     s_info[0] = kb_lo;
     s_info[1] = kb_hi - kb_lo + 1;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(512));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-  }
+  if (warp == 0) tc_alloc(smem_u32(tmem_slot), FwdSmem::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int kb_lo = s_info[0], nj = s_info[1];
-  // TMEM columns: S[0] 0..127, S[1] 128..255, O 256..319
 
   if (warp == 0 && lane == 0) {
     // ---------------- producer
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQKV)) : "memory");
     mbar_expect_tx(bar(0), AT_TILE_BYTES);
-    tma_load_2d(sQ, &tmQKV, bar(0), h * AT_D, (int)(rowbase + q0));
+    tma_load_2d(sQ, &tmQ, bar(0), h * AT_D, (int)(rowbase + q0));
     bool ok = true;
     for (int j = 0; j < nj && ok; ++j) {
       const int st = j & 1;
       if (!mbar_wait(bar(3 + st), ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-      mbar_expect_tx(bar(1 + st), 2 * AT_TILE_BYTES);
-      const int k0 = (kb_lo + j) * AT_BLK;
-      const uint32_t dst = sKV + st * 2 * AT_TILE_BYTES;
-      tma_load_2d(dst, &tmQKV, bar(1 + st), C + h * AT_D, (int)(rowbase + k0));
-      tma_load_2d(dst + AT_TILE_BYTES, &tmQKV, bar(1 + st), 2 * C + h * AT_D, (int)(rowbase + k0));
+      mbar_expect_tx(bar(1 + st), 2 * AT_HALF);
+      const int k0 = (kb_lo + j) * AT_BK;
+      const uint32_t dst = sKV + st * 2 * AT_HALF;
+      tma_load_2d(dst, &tmKV64, bar(1 + st), C + h * AT_D, (int)(rowbase + k0));
+      tma_load_2d(dst + AT_HALF, &tmKV64, bar(1 + st), 2 * C + h * AT_D, (int)(rowbase + k0));
     }
     if (!ok) trap_timeout(abort_flag, err);
     volatile int never = 0;
@@ -152,39 +172,31 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
     for (int j = max(0, nj - 2); j < nj; ++j) mbar_wait(bar(1 + (j & 1)), (j >> 1) & 1, &never, 1ll << 28);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
-    constexpr uint32_t ID_S = instr_desc(128, false, false);   // S = Q K^T: 128 x 128, K = 64
-    constexpr uint32_t ID_O = instr_desc(64, false, true);     // O = P V: 128 x 64, K = 128 (V MN-major)
+    constexpr uint32_t ID_S = instr_desc(64, false, false);   // S = Q K^T: 128 x 64, K = 64
+    constexpr uint32_t ID_O = instr_desc(64, false, true);    // O = P V: 128 x 64, K = 64 keys (V MN-major)
     bool ok = mbar_wait(bar(0), 0, abort_flag);
-    auto issue_s = [&](int j) -> bool {
-      const int st = j & 1;
-      if (!mbar_wait(bar(1 + st), (j >> 1) & 1, abort_flag)) return false;
-      if (!mbar_wait(bar(7 + st), ((j >> 1) & 1) ^ 1, abort_flag)) return false;
-      tc_fence_after();
-      const uint32_t sK = sKV + st * 2 * AT_TILE_BYTES;
-#pragma unroll
-      for (int k = 0; k < AT_D / 16; ++k) umma_bf16(tmem + st * 128, kdesc(sQ + k * 32), kdesc(sK + k * 32), ID_S, k > 0);
-      umma_commit(bar(5 + st));
-      return true;
-    };
-    if (ok) ok = issue_s(0);
     for (int j = 0; j < nj && ok; ++j) {
-      if (j + 1 < nj && !issue_s(j + 1)) { ok = false; break; }
-      if (!mbar_wait(bar(9), j & 1, abort_flag)) { ok = false; break; }
-      if (!mbar_wait(bar(11), (j & 1) ^ 1, abort_flag)) { ok = false; break; }
+      const int st = j & 1;
+      if (!mbar_wait(bar(1 + st), (j >> 1) & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(bar(6), (j & 1) ^ 1, abort_flag)) { ok = false; break; }   // S read by the softmax warps
       tc_fence_after();
-      const uint32_t sV = sKV + (j & 1) * 2 * AT_TILE_BYTES + AT_TILE_BYTES;
+      const uint32_t sK = sKV + st * 2 * AT_HALF, sV = sK + AT_HALF;
 #pragma unroll
-      for (int kk = 0; kk < AT_BLK / 16; ++kk) {
-        const uint32_t pa = sP + (kk >> 2) * AT_TILE_BYTES + (kk & 3) * 32;
-        umma_bf16(tmem + 256, kdesc(pa), mndesc(sV + kk * 2048, 8192), ID_O, kk > 0);
-      }
-      umma_commit(bar(10));
-      umma_commit(bar(3 + (j & 1)));
+      for (int k = 0; k < AT_D / 16; ++k) umma_bf16(tmem + 0, kdesc(sQ + k * 32), kdesc(sK + k * 32), ID_S, k > 0);
+      umma_commit(bar(5));
+      if (!mbar_wait(bar(7), j & 1, abort_flag)) { ok = false; break; }         // P written
+      if (!mbar_wait(bar(9), (j & 1) ^ 1, abort_flag)) { ok = false; break; }   // previous O read
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < AT_BK / 16; ++kk)
+        umma_bf16(tmem + 64, kdesc(sP + kk * 32), mndesc(sV + kk * 2048, 8192), ID_O, kk > 0);
+      umma_commit(bar(8));
+      umma_commit(bar(3 + st));
     }
     if (!ok) trap_timeout(abort_flag, err);
-    umma_commit(bar(12));
+    umma_commit(bar(10));
     volatile int never = 0;
-    mbar_wait(bar(12), 0, &never, 1ll << 28);
+    mbar_wait(bar(10), 0, &never, 1ll << 28);
   } else if (warp >= 2) {
     // ---------------- softmax warps: thread owns query row r
     const int quarter = warp & 3;
@@ -199,63 +211,54 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
 #pragma unroll
     for (int i = 0; i < AT_D; ++i) o[i] = 0.f;
     for (int j = 0; j < nj; ++j) {
-      const int st = j & 1;
-      const int k0 = (kb_lo + j) * AT_BLK;
-      if (!mbar_wait(bar(5 + st), (j >> 1) & 1, abort_flag)) { trap_timeout(abort_flag, err); break; }
+      const int k0 = (kb_lo + j) * AT_BK;
+      if (!mbar_wait(bar(5), j & 1, abort_flag)) { trap_timeout(abort_flag, err); break; }
       tc_fence_after();
-      const uint32_t tS = tmem + lane_off + st * 128;
-      // pass 1: masked row maximum
+      uint32_t sr[64];
+      tmem_ld32(tmem + lane_off, sr);
+      tmem_ld32(tmem + lane_off + 32, sr + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(6));   // S may be overwritten
       float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < AT_BLK; c += 32) {
-        uint32_t rr[32];
-        tmem_ld32(tS + c, rr);
-        tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int k = k0 + c + i;
-          if (k <= q && k >= ds_q) mx = fmaxf(mx, __uint_as_float(rr[i]) * sl2);
-        }
+      for (int i = 0; i < 64; ++i) {
+        const int k = k0 + i;
+        const float v = (k <= q && k >= ds_q) ? __uint_as_float(sr[i]) * sl2 : -INFINITY;
+        sr[i] = __float_as_uint(v);
+        mx = fmaxf(mx, v);
       }
       const float mn = fmaxf(m, mx);
       const float mu = mn == -INFINITY ? 0.f : mn;
       const float corr = exp2f(m - mu);
-      // pass 2: P = exp2(s - m) to shared memory (the previous P was consumed: o_full seen)
       float ps = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < AT_BLK; c += 32) {
-        uint32_t rr[32];
-        tmem_ld32(tS + c, rr);
-        tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 64; c += 32) {
         float p[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const int k = k0 + c + i;
-          p[i] = (k <= q && k >= ds_q) ? exp2f(__uint_as_float(rr[i]) * sl2 - mu) : 0.f;
+          p[i] = exp2f(__uint_as_float(sr[c + i]) - mu);
           ps += p[i];
         }
-        st_row32_bf16(sP, r, c, p);
+        st_row32_64(sP, r, c, p);
       }
-      tc_fence_before();
       fence_async_smem();
       __syncwarp();
-      if (lane == 0) { mbar_arrive(bar(7 + st)); mbar_arrive(bar(9)); }
+      if (lane == 0) mbar_arrive(bar(7));   // P ready
       l = l * corr + ps;
       m = mn;
-      // O_blk = P V
-      if (!mbar_wait(bar(10), j & 1, abort_flag)) { trap_timeout(abort_flag, err); break; }
+      if (!mbar_wait(bar(8), j & 1, abort_flag)) { trap_timeout(abort_flag, err); break; }
       tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < AT_D; c += 32) {
-        uint32_t rr[32];
-        tmem_ld32(tmem + lane_off + 256 + c, rr);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[c + i] = o[c + i] * corr + __uint_as_float(rr[i]);
-      }
+      uint32_t orr[64];
+      tmem_ld32(tmem + lane_off + 64, orr);
+      tmem_ld32(tmem + lane_off + 96, orr + 32);
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(11));
+      if (lane == 0) mbar_arrive(bar(9));   // O tile read, P buffer free
+#pragma unroll
+      for (int i = 0; i < 64; ++i) o[i] = o[i] * corr + __uint_as_float(orr[i]);
     }
     if (qv) {
       const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -275,39 +278,39 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  if (warp == 0) tc_dealloc(tmem, FwdSmem::TMEM_COLS);
 }
 
-// ============================================================== backward
-struct BwdSmem {
-  static constexpr int K = 0;                               // 16 KB
-  static constexpr int V = K + AT_TILE_BYTES;               // 16 KB
-  static constexpr int QD = V + AT_TILE_BYTES;              // 2 stages x (Q, dO)
-  static constexpr int PT = QD + 4 * AT_TILE_BYTES;         // 32 KB
-  static constexpr int DST = PT + 2 * AT_TILE_BYTES;        // 32 KB
-  static constexpr int DQ = DST + 2 * AT_TILE_BYTES;        // 32 KB fp32 staging (two 32-column boxes)
-  static constexpr int AUX = DQ + 2 * AT_TILE_BYTES;        // 2 x (lse2, D, dstart) x 128
-  static constexpr int BAR = AUX + 2 * 3 * AT_BLK * 4;
+// ============================================================== backward: dK, dV
+struct DkvSmem {
+  static constexpr int K = 0;                          // 16 KB: 128 keys
+  static constexpr int V = K + AT_TILE_BYTES;          // 16 KB
+  static constexpr int QD = V + AT_TILE_BYTES;         // 2 stages x (Q 8 KB, dO 8 KB)
+  static constexpr int PT = QD + 4 * AT_HALF;          // 16 KB: 128 keys x 64 queries
+  static constexpr int DST = PT + AT_TILE_BYTES;       // 16 KB
+  static constexpr int AUX = DST + AT_TILE_BYTES;      // 2 x (lse2, D, dstart) x 64
+  static constexpr int BAR = AUX + 2 * 3 * AT_BK * 4;
   static constexpr int TOTAL = BAR + 256;
+  static constexpr int TMEM_COLS = 256;                // S^T 0..63, dP^T 64..127, dV 128..191, dK 192..255
 };
 
-__global__ void __launch_bounds__(AT_THREADS, 1)
-attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
-            const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ lse, const float* __restrict__ Dbuf,
-            const int* __restrict__ dstart, bf16* __restrict__ dqkv, int T, int H, unsigned* err) {
+__global__ void __launch_bounds__(AT_THREADS)
+attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ64,
+                 const __grid_constant__ CUtensorMap tmDO64, const float* __restrict__ lse,
+                 const float* __restrict__ Dbuf, const int* __restrict__ dstart, bf16* __restrict__ dqkv, int T,
+                 int H, unsigned* err) {
   extern __shared__ __align__(1024) uint8_t at_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)at_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t* bars = (uint64_t*)(sm + BwdSmem::BAR);
-  // bars: 0 kv_full, 1-2 q_full, 3-4 q_empty, 5 s_full, 6 p_full, 7 dq_full, 8 tm_free, 9 drain,
-  //       10 softmax-group barrier
+  uint64_t* bars = (uint64_t*)(sm + DkvSmem::BAR);
+  // bars: 0 kv_full, 1-2 q_full, 3-4 q_empty, 5 s_full, 6 s_free, 7 p_full, 8 p_free, 9 drain, 10 group
   uint32_t* tmem_slot = (uint32_t*)(bars + 11);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   int* s_info = (int*)(tmem_slot + 2);
   const uint32_t b0 = smem_u32(bars);
   auto bar = [&](int i) { return b0 + 8u * i; };
-  const uint32_t sK = smem_u32(sm + BwdSmem::K), sV = smem_u32(sm + BwdSmem::V), sQD = smem_u32(sm + BwdSmem::QD);
-  const uint32_t sPT = smem_u32(sm + BwdSmem::PT), sDST = smem_u32(sm + BwdSmem::DST), sDQ = smem_u32(sm + BwdSmem::DQ);
-  float* aux = (float*)(sm + BwdSmem::AUX);
+  const uint32_t sK = smem_u32(sm + DkvSmem::K), sV = smem_u32(sm + DkvSmem::V), sQD = smem_u32(sm + DkvSmem::QD);
+  const uint32_t sPT = smem_u32(sm + DkvSmem::PT), sDST = smem_u32(sm + DkvSmem::DST);
+  float* aux = (float*)(sm + DkvSmem::AUX);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kb = blockIdx.x;   // earliest key blocks see the most queries: launched first
@@ -316,56 +319,50 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
   const int k0 = kb * AT_BLK;
   const long rowbase = (long)b * T;
   const int* dsr = dstart + rowbase;
-  const int nqb = (T + AT_BLK - 1) / AT_BLK;
+  const int nqb = (T + AT_BK - 1) / AT_BK;
+  const int qb_lo = k0 / AT_BK;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(0), 1);
     for (int i = 1; i <= 4; ++i) mbar_init(bar(i), 1);
     mbar_init(bar(5), 1);
     mbar_init(bar(6), 4);
-    mbar_init(bar(7), 1);
-    mbar_init(bar(8), 4);
+    mbar_init(bar(7), 4);
+    mbar_init(bar(8), 1);
     mbar_init(bar(9), 1);
     mbar_init(bar(10), 128);
     *abort_flag = 0;
     const int last_key = min(k0 + AT_BLK - 1, T - 1);
     int n = 0;
-    for (int qb = kb; qb < nqb; ++qb) {
-      if (dsr[qb * AT_BLK] > last_key) break;   // every later query lives in a later document
+    for (int qb = qb_lo; qb < nqb; ++qb) {
+      if (dsr[qb * AT_BK] > last_key) break;   // every later query lives in a later document
       ++n;
     }
     s_info[0] = n;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(512));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-  }
+  if (warp == 0) tc_alloc(smem_u32(tmem_slot), DkvSmem::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int niter = s_info[0];
-  // TMEM columns: S^T 0..127, dP^T 128..255, dV 256..319, dK 320..383, dQ 384..447
 
   if (warp == 0 && lane == 0) {
     // ---------------- producer
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQKV)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmDO)) : "memory");
     mbar_expect_tx(bar(0), 2 * AT_TILE_BYTES);
-    tma_load_2d(sK, &tmQKV, bar(0), C + h * AT_D, (int)(rowbase + k0));
-    tma_load_2d(sV, &tmQKV, bar(0), 2 * C + h * AT_D, (int)(rowbase + k0));
+    tma_load_2d(sK, &tmK, bar(0), C + h * AT_D, (int)(rowbase + k0));
+    tma_load_2d(sV, &tmK, bar(0), 2 * C + h * AT_D, (int)(rowbase + k0));
     bool ok = true;
     for (int i = 0; i < niter && ok; ++i) {
       const int st = i & 1;
       if (!mbar_wait(bar(3 + st), ((i >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-      mbar_expect_tx(bar(1 + st), 2 * AT_TILE_BYTES);
-      const int q0 = (kb + i) * AT_BLK;
-      const uint32_t dst = sQD + st * 2 * AT_TILE_BYTES;
-      tma_load_2d(dst, &tmQKV, bar(1 + st), h * AT_D, (int)(rowbase + q0));
-      tma_load_2d(dst + AT_TILE_BYTES, &tmDO, bar(1 + st), h * AT_D, (int)(rowbase + q0));
+      mbar_expect_tx(bar(1 + st), 2 * AT_HALF);
+      const int q0 = (qb_lo + i) * AT_BK;
+      const uint32_t dst = sQD + st * 2 * AT_HALF;
+      tma_load_2d(dst, &tmQ64, bar(1 + st), h * AT_D, (int)(rowbase + q0));
+      tma_load_2d(dst + AT_HALF, &tmDO64, bar(1 + st), h * AT_D, (int)(rowbase + q0));
     }
     if (!ok) trap_timeout(abort_flag, err);
     volatile int never = 0;
@@ -373,42 +370,37 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
     for (int i = max(0, niter - 2); i < niter; ++i) mbar_wait(bar(1 + (i & 1)), (i >> 1) & 1, &never, 1ll << 28);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
-    constexpr uint32_t ID_SS = instr_desc(128, false, false);   // S^T, dP^T: 128 keys x 128 queries, K = d
-    constexpr uint32_t ID_KV = instr_desc(64, false, true);     // dV, dK: 128 keys x 64, K = queries
-    constexpr uint32_t ID_Q = instr_desc(64, true, true);       // dQ: 128 queries x 64, K = keys
+    constexpr uint32_t ID_SS = instr_desc(64, false, false);   // S^T, dP^T: 128 keys x 64 queries, K = d
+    constexpr uint32_t ID_KV = instr_desc(64, false, true);    // dV, dK: 128 keys x 64, K = 64 queries
     bool ok = mbar_wait(bar(0), 0, abort_flag);
     for (int i = 0; i < niter && ok; ++i) {
       const int st = i & 1;
       if (!mbar_wait(bar(1 + st), (i >> 1) & 1, abort_flag)) { ok = false; break; }
-      if (!mbar_wait(bar(8), (i & 1) ^ 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(bar(6), (i & 1) ^ 1, abort_flag)) { ok = false; break; }   // S^T / dP^T read
       tc_fence_after();
-      const uint32_t sQ = sQD + st * 2 * AT_TILE_BYTES, sDO = sQ + AT_TILE_BYTES;
+      const uint32_t sQ = sQD + st * 2 * AT_HALF, sDO = sQ + AT_HALF;
 #pragma unroll
       for (int k = 0; k < AT_D / 16; ++k) {
         umma_bf16(tmem + 0, kdesc(sK + k * 32), kdesc(sQ + k * 32), ID_SS, k > 0);
-        umma_bf16(tmem + 128, kdesc(sV + k * 32), kdesc(sDO + k * 32), ID_SS, k > 0);
+        umma_bf16(tmem + 64, kdesc(sV + k * 32), kdesc(sDO + k * 32), ID_SS, k > 0);
       }
       umma_commit(bar(5));
-      if (!mbar_wait(bar(6), i & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(bar(7), i & 1, abort_flag)) { ok = false; break; }         // P^T, dS^T written
       tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < AT_BLK / 16; ++kk) {
-        const uint32_t koff = (kk >> 2) * AT_TILE_BYTES + (kk & 3) * 32;
-        umma_bf16(tmem + 256, kdesc(sPT + koff), mndesc(sDO + kk * 2048, 8192), ID_KV, (i > 0 || kk > 0));
-        umma_bf16(tmem + 320, kdesc(sDST + koff), mndesc(sQ + kk * 2048, 8192), ID_KV, (i > 0 || kk > 0));
+      for (int kk = 0; kk < AT_BK / 16; ++kk) {
+        umma_bf16(tmem + 128, kdesc(sPT + kk * 32), mndesc(sDO + kk * 2048, 8192), ID_KV, (i > 0 || kk > 0));
+        umma_bf16(tmem + 192, kdesc(sDST + kk * 32), mndesc(sQ + kk * 2048, 8192), ID_KV, (i > 0 || kk > 0));
       }
-#pragma unroll
-      for (int kk = 0; kk < AT_BLK / 16; ++kk)
-        umma_bf16(tmem + 384, mndesc(sDST + kk * 2048, AT_TILE_BYTES), mndesc(sK + kk * 2048, 8192), ID_Q, kk > 0);
-      umma_commit(bar(3 + st));
-      umma_commit(bar(7));
+      umma_commit(bar(8));        // P^T / dS^T buffers free
+      umma_commit(bar(3 + st));   // Q / dO stage free
     }
     if (!ok) trap_timeout(abort_flag, err);
     umma_commit(bar(9));
     volatile int never = 0;
     mbar_wait(bar(9), 0, &never, 1ll << 28);
   } else if (warp >= 2) {
-    // ---------------- softmax warps: thread owns key row r (S^T, dP^T, dK, dV) and query row r (dQ)
+    // ---------------- elementwise warps: thread owns key row r
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const int k = k0 + r;
@@ -417,79 +409,60 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
     const float sl2 = 0.125f * LOG2E_F;
     bool ok = true;
     uint32_t gph = 0;
+    // per-query values of the first block
+    float nl = 0.f, nd = 0.f;
+    int nds = 0x7fffffff;
+    if (tid < AT_BK && niter > 0) {
+      const int qq = qb_lo * AT_BK + tid;
+      if (qq < T) { nl = lse[(long)bh * T + qq] * LOG2E_F; nd = Dbuf[(long)bh * T + qq]; nds = dsr[qq]; }
+    }
     for (int i = 0; i < niter; ++i) {
-      const int q0 = (kb + i) * AT_BLK;
-      float* L2 = aux + (i & 1) * 3 * AT_BLK;
-      float* Dq = L2 + AT_BLK;
-      int* DSq = reinterpret_cast<int*>(Dq + AT_BLK);
-      {
-        const int qq = q0 + tid;
-        const bool v = qq < T;
-        L2[tid] = v ? lse[(long)bh * T + qq] * LOG2E_F : 0.f;
-        Dq[tid] = v ? Dbuf[(long)bh * T + qq] : 0.f;
-        DSq[tid] = v ? dsr[qq] : 0x7fffffff;
-      }
+      const int q0 = (qb_lo + i) * AT_BK;
+      float* L2 = aux + (i & 1) * 3 * AT_BK;
+      float* Dq = L2 + AT_BK;
+      int* DSq = reinterpret_cast<int*>(Dq + AT_BK);
+      if (tid < AT_BK) { L2[tid] = nl; Dq[tid] = nd; DSq[tid] = nds; }
       if (!group_sync(bar(10), gph, abort_flag)) { ok = false; break; }
+      // prefetch the next block's per-query values (consumed next iteration)
+      nl = 0.f; nd = 0.f; nds = 0x7fffffff;
+      if (tid < AT_BK && i + 1 < niter) {
+        const int qq = q0 + AT_BK + tid;
+        if (qq < T) { nl = lse[(long)bh * T + qq] * LOG2E_F; nd = Dbuf[(long)bh * T + qq]; nds = dsr[qq]; }
+      }
       if (!mbar_wait(bar(5), i & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < AT_BLK; c += 32) {
-        uint32_t sr[32], dr[32];
-        tmem_ld32(tmem + lane_off + c, sr);
-        tmem_ld32(tmem + lane_off + 128 + c, dr);
-        tmem_wait_ld();
+      uint32_t sr[64], dr[64];
+      tmem_ld32(tmem + lane_off, sr);
+      tmem_ld32(tmem + lane_off + 32, sr + 32);
+      tmem_ld32(tmem + lane_off + 64, dr);
+      tmem_ld32(tmem + lane_off + 96, dr + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(6));   // S^T / dP^T may be overwritten
+      // the previous block's P^T / dS^T have been consumed
+      if (i > 0 && !mbar_wait(bar(8), (i - 1) & 1, abort_flag)) { ok = false; break; }
+#pragma unroll
+      for (int c = 0; c < AT_BK; c += 32) {
         float p[32], ds[32];
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) {
           const int ql = c + jj, qq = q0 + ql;
           const bool allowed = qq < T && qq >= k && DSq[ql] <= k;
-          const float pv = allowed ? exp2f(__uint_as_float(sr[jj]) * sl2 - L2[ql]) : 0.f;
+          const float pv = allowed ? exp2f(__uint_as_float(sr[ql]) * sl2 - L2[ql]) : 0.f;
           p[jj] = pv;
-          ds[jj] = pv * (__uint_as_float(dr[jj]) - Dq[ql]);
+          ds[jj] = pv * (__uint_as_float(dr[ql]) - Dq[ql]);
         }
-        st_row32_bf16(sPT, r, c, p);
-        st_row32_bf16(sDST, r, c, ds);
+        st_row32_64(sPT, r, c, p);
+        st_row32_64(sDST, r, c, ds);
       }
-      tc_fence_before();
       fence_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(6));
-      // dQ block (row r = query q0 + r): stage and add into the fp32 accumulator
-      if (!mbar_wait(bar(7), i & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t qa[32], qb2[32];
-      tmem_ld32(tmem + lane_off + 384, qa);
-      tmem_ld32(tmem + lane_off + 416, qb2);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(8));   // S^T / dP^T / dQ tensor memory free
-      if (tid == 0) bulk_wait_read<0>();    // the previous reduce has read the staging buffer
-      if (!group_sync(bar(10), gph, abort_flag)) { ok = false; break; }
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const uint32_t* src = half ? qb2 : qa;
-        const uint32_t boxb = sDQ + half * AT_TILE_BYTES + r * 128;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          uint32_t a = boxb + ((u ^ (r & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(src[4 * u]), "r"(src[4 * u + 1]),
-                       "r"(src[4 * u + 2]), "r"(src[4 * u + 3])
-                       : "memory");
-        }
-      }
-      fence_async_smem();
-      if (!group_sync(bar(10), gph, abort_flag)) { ok = false; break; }
-      if (tid == 0) {
-        tma_reduce_add_2d(&tmDQ, sDQ, h * AT_D, (int)(rowbase + q0));
-        tma_reduce_add_2d(&tmDQ, sDQ + AT_TILE_BYTES, h * AT_D + 32, (int)(rowbase + q0));
-        bulk_commit();
-      }
+      if (lane == 0) mbar_arrive(bar(7));
     }
     if (!ok) trap_timeout(abort_flag, err);
-    if (ok && niter > 0) {
-      // dK (scaled by 1/sqrt(d)) and dV rows, accumulated over all query blocks;
-      // the tensor-memory loads are warp-collective, only the stores depend on k < T
+    // wait for the last dV / dK accumulation, then write the rows
+    if (ok && niter > 0 && mbar_wait(bar(8), (niter - 1) & 1, abort_flag)) {
       tc_fence_after();
       bf16* row = dqkv + (rowbase + k) * 3 * C;
 #pragma unroll
@@ -499,7 +472,7 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
 #pragma unroll
         for (int c = 0; c < AT_D; c += 32) {
           uint32_t rr[32];
-          tmem_ld32(tmem + lane_off + (part == 0 ? 320 : 256) + c, rr);
+          tmem_ld32(tmem + lane_off + (part == 0 ? 192 : 128) + c, rr);
           tmem_wait_ld();
           if (k < T) {
 #pragma unroll
@@ -515,12 +488,185 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
         }
       }
     }
-    if (tid == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  if (warp == 0) tc_dealloc(tmem, DkvSmem::TMEM_COLS);
+}
+
+// ============================================================== backward: dQ
+struct DqSmem {
+  static constexpr int Q = 0;                          // 16 KB: 128 queries
+  static constexpr int DO = Q + AT_TILE_BYTES;         // 16 KB
+  static constexpr int KV = DO + AT_TILE_BYTES;        // 2 stages x (K 8 KB, V 8 KB)
+  static constexpr int DS = KV + 4 * AT_HALF;          // 16 KB: 128 queries x 64 keys
+  static constexpr int BAR = DS + AT_TILE_BYTES;
+  static constexpr int TOTAL = BAR + 256;
+  static constexpr int TMEM_COLS = 256;                // S 0..63, dP 64..127, dQ 128..191
+};
+
+__global__ void __launch_bounds__(AT_THREADS)
+attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+               const __grid_constant__ CUtensorMap tmKV64, const float* __restrict__ lse,
+               const float* __restrict__ Dbuf, const int* __restrict__ dstart, bf16* __restrict__ dqkv, int T,
+               int H, unsigned* err) {
+  extern __shared__ __align__(1024) uint8_t at_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)at_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = (uint64_t*)(sm + DqSmem::BAR);
+  // bars: 0 q_full, 1-2 kv_full, 3-4 kv_empty, 5 s_full, 6 s_free, 7 ds_full, 8 ds_free, 9 drain
+  uint32_t* tmem_slot = (uint32_t*)(bars + 10);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  int* s_info = (int*)(tmem_slot + 2);
+  const uint32_t b0 = smem_u32(bars);
+  auto bar = [&](int i) { return b0 + 8u * i; };
+  const uint32_t sQ = smem_u32(sm + DqSmem::Q), sDO = smem_u32(sm + DqSmem::DO), sKV = smem_u32(sm + DqSmem::KV);
+  const uint32_t sDS = smem_u32(sm + DqSmem::DS);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nqb = (T + AT_BLK - 1) / AT_BLK;
+  const int qb = nqb - 1 - blockIdx.x;
+  const int bh = blockIdx.y, b = bh / H, h = bh % H;
+  const int C = H * AT_D;
+  const int q0 = qb * AT_BLK;
+  const long rowbase = (long)b * T;
+  const int* dsr = dstart + rowbase;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(0), 1);
+    for (int i = 1; i <= 4; ++i) mbar_init(bar(i), 1);
+    mbar_init(bar(5), 1);
+    mbar_init(bar(6), 4);
+    mbar_init(bar(7), 4);
+    mbar_init(bar(8), 1);
+    mbar_init(bar(9), 1);
+    *abort_flag = 0;
+    const int kb_lo = dsr[q0] / AT_BK, kb_hi = min(q0 + AT_BLK - 1, T - 1) / AT_BK;
+    s_info[0] = kb_lo;
+    s_info[1] = kb_hi - kb_lo + 1;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0) tc_alloc(smem_u32(tmem_slot), DqSmem::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int kb_lo = s_info[0], nj = s_info[1];
+
+  if (warp == 0 && lane == 0) {
+    mbar_expect_tx(bar(0), 2 * AT_TILE_BYTES);
+    tma_load_2d(sQ, &tmQ, bar(0), h * AT_D, (int)(rowbase + q0));
+    tma_load_2d(sDO, &tmDO, bar(0), h * AT_D, (int)(rowbase + q0));
+    bool ok = true;
+    for (int j = 0; j < nj && ok; ++j) {
+      const int st = j & 1;
+      if (!mbar_wait(bar(3 + st), ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+      mbar_expect_tx(bar(1 + st), 2 * AT_HALF);
+      const int k0 = (kb_lo + j) * AT_BK;
+      const uint32_t dst = sKV + st * 2 * AT_HALF;
+      tma_load_2d(dst, &tmKV64, bar(1 + st), C + h * AT_D, (int)(rowbase + k0));
+      tma_load_2d(dst + AT_HALF, &tmKV64, bar(1 + st), 2 * C + h * AT_D, (int)(rowbase + k0));
+    }
+    if (!ok) trap_timeout(abort_flag, err);
+    volatile int never = 0;
+    mbar_wait(bar(0), 0, &never, 1ll << 28);
+    for (int j = max(0, nj - 2); j < nj; ++j) mbar_wait(bar(1 + (j & 1)), (j >> 1) & 1, &never, 1ll << 28);
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t ID_S = instr_desc(64, false, false);   // S, dP: 128 queries x 64 keys, K = d
+    constexpr uint32_t ID_Q = instr_desc(64, false, true);    // dQ += dS K: 128 x 64, K = 64 keys (K MN-major)
+    bool ok = mbar_wait(bar(0), 0, abort_flag);
+    for (int j = 0; j < nj && ok; ++j) {
+      const int st = j & 1;
+      if (!mbar_wait(bar(1 + st), (j >> 1) & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(bar(6), (j & 1) ^ 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t sK = sKV + st * 2 * AT_HALF, sV = sK + AT_HALF;
+#pragma unroll
+      for (int k = 0; k < AT_D / 16; ++k) {
+        umma_bf16(tmem + 0, kdesc(sQ + k * 32), kdesc(sK + k * 32), ID_S, k > 0);
+        umma_bf16(tmem + 64, kdesc(sDO + k * 32), kdesc(sV + k * 32), ID_S, k > 0);
+      }
+      umma_commit(bar(5));
+      if (!mbar_wait(bar(7), j & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < AT_BK / 16; ++kk)
+        umma_bf16(tmem + 128, kdesc(sDS + kk * 32), mndesc(sK + kk * 2048, 8192), ID_Q, (j > 0 || kk > 0));
+      umma_commit(bar(8));
+      umma_commit(bar(3 + st));
+    }
+    if (!ok) trap_timeout(abort_flag, err);
+    umma_commit(bar(9));
+    volatile int never = 0;
+    mbar_wait(bar(9), 0, &never, 1ll << 28);
+  } else if (warp >= 2) {
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int q = q0 + r;
+    const bool qv = q < T;
+    const int ds_q = qv ? dsr[q] : 0;
+    const float Lq = qv ? lse[(long)bh * T + q] * LOG2E_F : 0.f;
+    const float Dv = qv ? Dbuf[(long)bh * T + q] : 0.f;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const float sl2 = 0.125f * LOG2E_F;
+    bool ok = true;
+    for (int j = 0; j < nj; ++j) {
+      const int k0 = (kb_lo + j) * AT_BK;
+      if (!mbar_wait(bar(5), j & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sr[64], dr[64];
+      tmem_ld32(tmem + lane_off, sr);
+      tmem_ld32(tmem + lane_off + 32, sr + 32);
+      tmem_ld32(tmem + lane_off + 64, dr);
+      tmem_ld32(tmem + lane_off + 96, dr + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(6));
+      if (j > 0 && !mbar_wait(bar(8), (j - 1) & 1, abort_flag)) { ok = false; break; }   // dS buffer free
+#pragma unroll
+      for (int c = 0; c < AT_BK; c += 32) {
+        float ds[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int kk = k0 + c + i;
+          const float p = (kk <= q && kk >= ds_q) ? exp2f(__uint_as_float(sr[c + i]) * sl2 - Lq) : 0.f;
+          ds[i] = p * (__uint_as_float(dr[c + i]) - Dv);
+        }
+        st_row32_64(sDS, r, c, ds);
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(7));
+    }
+    if (!ok) trap_timeout(abort_flag, err);
+    if (ok && nj > 0 && mbar_wait(bar(8), (nj - 1) & 1, abort_flag)) {
+      tc_fence_after();
+      bf16* dst = dqkv + (rowbase + q) * 3 * C + h * AT_D;
+#pragma unroll
+      for (int c = 0; c < AT_D; c += 32) {
+        uint32_t rr[32];
+        tmem_ld32(tmem + lane_off + 128 + c, rr);
+        tmem_wait_ld();
+        if (qv) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 w;
+            w.x = pk_bf16(__uint_as_float(rr[8 * u]) * 0.125f, __uint_as_float(rr[8 * u + 1]) * 0.125f);
+            w.y = pk_bf16(__uint_as_float(rr[8 * u + 2]) * 0.125f, __uint_as_float(rr[8 * u + 3]) * 0.125f);
+            w.z = pk_bf16(__uint_as_float(rr[8 * u + 4]) * 0.125f, __uint_as_float(rr[8 * u + 5]) * 0.125f);
+            w.w = pk_bf16(__uint_as_float(rr[8 * u + 6]) * 0.125f, __uint_as_float(rr[8 * u + 7]) * 0.125f);
+            *reinterpret_cast<uint4*>(dst + c + 8 * u) = w;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tc_dealloc(tmem, DqSmem::TMEM_COLS);
 }
 
 // D[b, h, t] = dO[b*T+t, head h] . O[b*T+t, head h]   (one thread per (row, head))
@@ -544,72 +690,61 @@ __global__ void attn_rowdot_kernel(const bf16* __restrict__ out, const bf16* __r
   Dbuf[((long)b * H + h) * T + t] = acc;
 }
 
-// dqkv[:, q part] = bf16(dQacc * 1/sqrt(d))
-__global__ void dq_convert_kernel(const float* __restrict__ acc, bf16* __restrict__ dqkv, long rows, int C) {
-  const long n8 = rows * C / 8;
-  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n8; i += (long)gridDim.x * blockDim.x) {
-    const long e = i * 8, row = e / C;
-    const int c = e % C;
-    float v[8];
-    Vec<float>::load(acc + e, v);
-    Vec<float>::load(acc + e + 4, v + 4);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] *= 0.125f;
-    Vec<bf16>::store(dqkv + row * 3 * C + c, v);
-  }
-}
-
 // ============================================================== launchers
 bool attn_tc_supported(int d) { return d == AT_D && get_encode() != nullptr; }
+
+template <typename K>
+static cudaError_t tc_smem_attr(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
 
 cudaError_t launch_attn_fwd_tc(const bf16* qkv, bf16* out, float* lse, const int* dstart, int B, int T, int H,
                                unsigned* err, cudaStream_t s) {
   const int C = H * AT_D;
-  CUtensorMap tm;
-  if (!make_map_ex(&tm, MapKey{qkv, (long)B * T, 3L * C, 3L * C, 1, 0, AT_D, AT_BLK, 0, 128}))
+  const long rows = (long)B * T;
+  CUtensorMap tq, tkv;
+  if (!make_map_ex(&tq, MapKey{qkv, rows, 3L * C, 3L * C, 1, 0, AT_D, AT_BLK, 0, 128}) ||
+      !make_map_ex(&tkv, MapKey{qkv, rows, 3L * C, 3L * C, 1, 0, AT_D, AT_BK, 0, 128}))
     return cudaErrorInvalidValue;
-  // more than half the shared memory: one CTA per SM, as each holds all 512 TMEM columns
-  const int smem = FwdSmem::TOTAL + 1024 > 120 * 1024 ? FwdSmem::TOTAL + 1024 : 120 * 1024;
+  const int smem = FwdSmem::TOTAL + 1024;
   static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  if (!attr) { cudaError_t e = tc_smem_attr(attn_fwd_tc, smem); if (e) return e; attr = true; }
   dim3 grid((T + AT_BLK - 1) / AT_BLK, B * H);
   ++g_kernel_launches;
-  attn_fwd_tc<<<grid, AT_THREADS, smem, s>>>(tm, out, lse, dstart, T, H, err);
+  attn_fwd_tc<<<grid, AT_THREADS, smem, s>>>(tq, tkv, out, lse, dstart, T, H, err);
   return cudaGetLastError();
 }
 
 cudaError_t launch_attn_bwd_tc(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* Dbuf,
                                float* dq_acc, const int* dstart, bf16* dqkv, int B, int T, int H, unsigned* err,
                                cudaStream_t s) {
+  (void)dq_acc;
   const int C = H * AT_D;
   const long rows = (long)B * T;
-  CUtensorMap tq, tdo, tdq;
-  if (!make_map_ex(&tq, MapKey{qkv, rows, 3L * C, 3L * C, 1, 0, AT_D, AT_BLK, 0, 128}) ||
-      !make_map_ex(&tdo, MapKey{dout, rows, (long)C, (long)C, 1, 0, AT_D, AT_BLK, 0, 128}) ||
-      !make_map_ex(&tdq, MapKey{dq_acc, rows, (long)C, (long)C, 1, 0, 32, AT_BLK, 1, 128}))
+  CUtensorMap tq128, tq64, tdo128, tdo64;
+  if (!make_map_ex(&tq128, MapKey{qkv, rows, 3L * C, 3L * C, 1, 0, AT_D, AT_BLK, 0, 128}) ||
+      !make_map_ex(&tq64, MapKey{qkv, rows, 3L * C, 3L * C, 1, 0, AT_D, AT_BK, 0, 128}) ||
+      !make_map_ex(&tdo128, MapKey{dout, rows, (long)C, (long)C, 1, 0, AT_D, AT_BLK, 0, 128}) ||
+      !make_map_ex(&tdo64, MapKey{dout, rows, (long)C, (long)C, 1, 0, AT_D, AT_BK, 0, 128}))
     return cudaErrorInvalidValue;
-  const int smem = BwdSmem::TOTAL + 1024;
+  const int smem_kv = DkvSmem::TOTAL + 1024, smem_q = DqSmem::TOTAL + 1024;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_bwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = tc_smem_attr(attn_bwd_dkdv_tc, smem_kv);
+    if (e == cudaSuccess) e = tc_smem_attr(attn_bwd_dq_tc, smem_q);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  cudaError_t e = cudaMemsetAsync(dq_acc, 0, rows * C * sizeof(float), s);
-  if (e != cudaSuccess) return e;
   long n = rows * H;
   ++g_kernel_launches;
   attn_rowdot_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(out, dout, Dbuf, B, T, H);
+  cudaError_t e;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   dim3 grid((T + AT_BLK - 1) / AT_BLK, B * H);
   ++g_kernel_launches;
-  attn_bwd_tc<<<grid, AT_THREADS, smem, s>>>(tq, tdo, tdq, lse, Dbuf, dstart, dqkv, T, H, err);
+  attn_bwd_dkdv_tc<<<grid, AT_THREADS, smem_kv, s>>>(tq128, tq64, tdo64, lse, Dbuf, dstart, dqkv, T, H, err);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   ++g_kernel_launches;
-  dq_convert_kernel<<<148 * 4, 256, 0, s>>>(dq_acc, dqkv, rows, C);
+  attn_bwd_dq_tc<<<grid, AT_THREADS, smem_q, s>>>(tq128, tdo128, tq64, lse, Dbuf, dstart, dqkv, T, H, err);
   return cudaGetLastError();
 }
