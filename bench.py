@@ -157,6 +157,24 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- multi-rank timing
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Slowest rank's value (the job's time): all-reduce MAX over the group."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_rank_step * steps / (max_ms / 1000.0)
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def run_ours(args, rank, world, local_rank):
@@ -183,13 +201,6 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     # warm-up (also fills the profiling event pool)
     model.profile_enable(True)
     for _ in range(args.warmup):
@@ -211,7 +222,7 @@ def run_ours(args, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize()
     n1 = model.kernel_launches()
-    ms = max_over_ranks(e0.elapsed_time(e1))
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     clk = clocks.stop()
     barrier()
     prof = model.profile_read()
@@ -220,7 +231,7 @@ def run_ours(args, rank, world, local_rank):
     status = model.status()
 
     tokens_per_step = B * T
-    value = world * tokens_per_step * args.steps / (ms / 1000.0)
+    value = job_throughput(tokens_per_step, args.steps, world, ms)
     ms_step = ms / args.steps
     fpt = flops_per_token(mc, T)
     peaks = load_peaks()
@@ -266,8 +277,8 @@ def run_ours(args, rank, world, local_rank):
             h_loss.copy_(loss, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
-        ms2 = max_over_ranks(e0.elapsed_time(e1))
-        e2e = {"value": world * tokens_per_step * k2 / (ms2 / 1000.0), "unit": "tokens/s",
+        ms2 = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": job_throughput(tokens_per_step, k2, world, ms2), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h_tok.numel() * 4 + h_tgt.numel() * 4), "d2h_bytes_per_step": 4,
                "steps": k2}
 

@@ -99,21 +99,22 @@ __device__ __forceinline__ void tc_dealloc(uint32_t tmem, int cols) {
 struct FwdSmem {
   static constexpr int Q = 0;                          // 16 KB: 128 queries
   static constexpr int KV = Q + AT_TILE_BYTES;         // 2 stages x (K 8 KB, V 8 KB)
-  static constexpr int P = KV + 4 * AT_HALF;           // 16 KB: 128 queries x 64 keys
-  static constexpr int BAR = P + AT_TILE_BYTES;
+  static constexpr int P = KV + 4 * AT_HALF;           // 2 x 16 KB: 128 queries x 64 keys
+  static constexpr int BAR = P + 2 * AT_TILE_BYTES;
   static constexpr int TOTAL = BAR + 256;
-  static constexpr int TMEM_COLS = 128;                // S 0..63, O 64..127
+  static constexpr int TMEM_COLS = 256;                // S 0..63, O[0] 64..127, O[1] 128..191
 };
 
-__global__ void __launch_bounds__(AT_THREADS)
+__global__ void __launch_bounds__(AT_THREADS, 2)
 attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV64,
             bf16* __restrict__ out, float* __restrict__ lse, const int* __restrict__ dstart, int T, int H,
             unsigned* err) {
   extern __shared__ __align__(1024) uint8_t at_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)at_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = (uint64_t*)(sm + FwdSmem::BAR);
-  // bars: 0 q_full, 1-2 kv_full, 3-4 kv_empty, 5 s_full, 6 s_free, 7 p_full, 8 o_full, 9 o_free, 10 drain
-  uint32_t* tmem_slot = (uint32_t*)(bars + 11);
+  // bars: 0 q_full, 1-2 kv_full, 3-4 kv_empty, 5 s_full, 6 s_free, 7-8 p_full, 9-10 o_full, 11-12 o_free,
+  //       13 drain
+  uint32_t* tmem_slot = (uint32_t*)(bars + 14);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   int* s_info = (int*)(tmem_slot + 2);
   const uint32_t b0 = smem_u32(bars);
@@ -135,9 +136,12 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     mbar_init(bar(5), 1);
     mbar_init(bar(6), 4);
     mbar_init(bar(7), 4);
-    mbar_init(bar(8), 1);
-    mbar_init(bar(9), 4);
+    mbar_init(bar(8), 4);
+    mbar_init(bar(9), 1);
     mbar_init(bar(10), 1);
+    mbar_init(bar(11), 4);
+    mbar_init(bar(12), 4);
+    mbar_init(bar(13), 1);
     *abort_flag = 0;
     const int kb_lo = dsr[q0] / AT_BK, kb_hi = min(q0 + AT_BLK - 1, T - 1) / AT_BK;
     s_info[0] = kb_lo;
@@ -171,34 +175,42 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     mbar_wait(bar(0), 0, &never, 1ll << 28);
     for (int j = max(0, nj - 2); j < nj; ++j) mbar_wait(bar(1 + (j & 1)), (j >> 1) & 1, &never, 1ll << 28);
   } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
+    // ---------------- MMA issuer: S(j+1) is issued before P V of block j
     constexpr uint32_t ID_S = instr_desc(64, false, false);   // S = Q K^T: 128 x 64, K = 64
     constexpr uint32_t ID_O = instr_desc(64, false, true);    // O = P V: 128 x 64, K = 64 keys (V MN-major)
     bool ok = mbar_wait(bar(0), 0, abort_flag);
-    for (int j = 0; j < nj && ok; ++j) {
+    auto issue_s = [&](int j) -> bool {
       const int st = j & 1;
-      if (!mbar_wait(bar(1 + st), (j >> 1) & 1, abort_flag)) { ok = false; break; }
-      if (!mbar_wait(bar(6), (j & 1) ^ 1, abort_flag)) { ok = false; break; }   // S read by the softmax warps
+      if (!mbar_wait(bar(1 + st), (j >> 1) & 1, abort_flag)) return false;
+      if (!mbar_wait(bar(6), (j & 1) ^ 1, abort_flag)) return false;   // previous S read
       tc_fence_after();
-      const uint32_t sK = sKV + st * 2 * AT_HALF, sV = sK + AT_HALF;
+      const uint32_t sK = sKV + st * 2 * AT_HALF;
 #pragma unroll
       for (int k = 0; k < AT_D / 16; ++k) umma_bf16(tmem + 0, kdesc(sQ + k * 32), kdesc(sK + k * 32), ID_S, k > 0);
       umma_commit(bar(5));
-      if (!mbar_wait(bar(7), j & 1, abort_flag)) { ok = false; break; }         // P written
-      if (!mbar_wait(bar(9), (j & 1) ^ 1, abort_flag)) { ok = false; break; }   // previous O read
+      return true;
+    };
+    if (ok && nj > 0) ok = issue_s(0);
+    for (int j = 0; j < nj && ok; ++j) {
+      const int st = j & 1;
+      if (j + 1 < nj && !issue_s(j + 1)) { ok = false; break; }
+      if (!mbar_wait(bar(7 + st), (j >> 1) & 1, abort_flag)) { ok = false; break; }         // P(j) written
+      if (!mbar_wait(bar(11 + st), ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }  // O buffer read
       tc_fence_after();
+      const uint32_t sV = sKV + st * 2 * AT_HALF + AT_HALF, sPj = sP + st * AT_TILE_BYTES;
 #pragma unroll
       for (int kk = 0; kk < AT_BK / 16; ++kk)
-        umma_bf16(tmem + 64, kdesc(sP + kk * 32), mndesc(sV + kk * 2048, 8192), ID_O, kk > 0);
-      umma_commit(bar(8));
+        umma_bf16(tmem + 64 + st * 64, kdesc(sPj + kk * 32), mndesc(sV + kk * 2048, 8192), ID_O, kk > 0);
+      umma_commit(bar(9 + st));
       umma_commit(bar(3 + st));
     }
     if (!ok) trap_timeout(abort_flag, err);
-    umma_commit(bar(10));
+    umma_commit(bar(13));
     volatile int never = 0;
-    mbar_wait(bar(10), 0, &never, 1ll << 28);
+    mbar_wait(bar(13), 0, &never, 1ll << 28);
   } else if (warp >= 2) {
-    // ---------------- softmax warps: thread owns query row r
+    // ---------------- softmax warps: thread owns query row r.  O of block j is
+    // accumulated during block j+1, so no wait follows the P V it enables.
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const int q = q0 + r;
@@ -206,13 +218,29 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     const int ds_q = qv ? dsr[q] : 0;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = 0.125f * LOG2E_F;   // 1/sqrt(64) in the exp2 domain
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY, l = 0.f, c_pend = 0.f;
     float o[AT_D];
 #pragma unroll
     for (int i = 0; i < AT_D; ++i) o[i] = 0.f;
+    bool ok = true;
+    auto accumulate = [&](int jj) -> bool {   // o = o * c(jj) + O(jj)
+      const int sb = jj & 1;
+      if (!mbar_wait(bar(9 + sb), (jj >> 1) & 1, abort_flag)) return false;
+      tc_fence_after();
+      uint32_t orr[64];
+      tmem_ld32(tmem + lane_off + 64 + sb * 64, orr);
+      tmem_ld32(tmem + lane_off + 96 + sb * 64, orr + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(11 + sb));
+#pragma unroll
+      for (int i = 0; i < 64; ++i) o[i] = o[i] * c_pend + __uint_as_float(orr[i]);
+      return true;
+    };
     for (int j = 0; j < nj; ++j) {
       const int k0 = (kb_lo + j) * AT_BK;
-      if (!mbar_wait(bar(5), j & 1, abort_flag)) { trap_timeout(abort_flag, err); break; }
+      if (!mbar_wait(bar(5), j & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[64];
       tmem_ld32(tmem + lane_off, sr);
@@ -231,8 +259,10 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
       }
       const float mn = fmaxf(m, mx);
       const float mu = mn == -INFINITY ? 0.f : mn;
-      const float corr = exp2f(m - mu);
+      const float cj = exp2f(m - mu);
       float ps = 0.f;
+      // P buffer j&1 was read by P V of block j-2, whose result was accumulated in block j-1
+      const uint32_t sPj = sP + (j & 1) * AT_TILE_BYTES;
 #pragma unroll
       for (int c = 0; c < 64; c += 32) {
         float p[32];
@@ -241,25 +271,18 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           p[i] = exp2f(__uint_as_float(sr[c + i]) - mu);
           ps += p[i];
         }
-        st_row32_64(sP, r, c, p);
+        st_row32_64(sPj, r, c, p);
       }
       fence_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(7));   // P ready
-      l = l * corr + ps;
+      if (lane == 0) mbar_arrive(bar(7 + (j & 1)));   // P(j) ready
+      l = l * cj + ps;
       m = mn;
-      if (!mbar_wait(bar(8), j & 1, abort_flag)) { trap_timeout(abort_flag, err); break; }
-      tc_fence_after();
-      uint32_t orr[64];
-      tmem_ld32(tmem + lane_off + 64, orr);
-      tmem_ld32(tmem + lane_off + 96, orr + 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(9));   // O tile read, P buffer free
-#pragma unroll
-      for (int i = 0; i < 64; ++i) o[i] = o[i] * corr + __uint_as_float(orr[i]);
+      if (j > 0 && !accumulate(j - 1)) { ok = false; break; }
+      c_pend = cj;
     }
+    if (ok && nj > 0) ok = accumulate(nj - 1);
+    if (!ok) trap_timeout(abort_flag, err);
     if (qv) {
       const float inv = l > 0.f ? 1.f / l : 0.f;
       bf16* orow = out + (rowbase + q) * C + h * AT_D;
@@ -294,7 +317,7 @@ struct DkvSmem {
   static constexpr int TMEM_COLS = 256;                // S^T 0..63, dP^T 64..127, dV 128..191, dK 192..255
 };
 
-__global__ void __launch_bounds__(AT_THREADS)
+__global__ void __launch_bounds__(AT_THREADS, 2)
 attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ64,
                  const __grid_constant__ CUtensorMap tmDO64, const float* __restrict__ lse,
                  const float* __restrict__ Dbuf, const int* __restrict__ dstart, bf16* __restrict__ dqkv, int T,
@@ -302,7 +325,8 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   extern __shared__ __align__(1024) uint8_t at_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)at_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = (uint64_t*)(sm + DkvSmem::BAR);
-  // bars: 0 kv_full, 1-2 q_full, 3-4 q_empty, 5 s_full, 6 s_free, 7 p_full, 8 p_free, 9 drain, 10 group
+  // bars: 0 kv_full, 1-2 q_full (TMA tiles + per-query values), 3-4 q_empty, 5 s_full, 6 s_free,
+  //       7 p_full, 8 p_free, 9 drain
   uint32_t* tmem_slot = (uint32_t*)(bars + 11);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   int* s_info = (int*)(tmem_slot + 2);
@@ -324,23 +348,30 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
 
   if (threadIdx.x == 0) {
     mbar_init(bar(0), 1);
-    for (int i = 1; i <= 4; ++i) mbar_init(bar(i), 1);
+    for (int i = 1; i <= 2; ++i) mbar_init(bar(i), 1 + 32);   // TMA arrival + 32 lanes of per-query values
+    for (int i = 3; i <= 4; ++i) mbar_init(bar(i), 1);
     mbar_init(bar(5), 1);
     mbar_init(bar(6), 4);
     mbar_init(bar(7), 4);
     mbar_init(bar(8), 1);
     mbar_init(bar(9), 1);
-    mbar_init(bar(10), 128);
     *abort_flag = 0;
-    const int last_key = min(k0 + AT_BLK - 1, T - 1);
-    int n = 0;
-    for (int qb = qb_lo; qb < nqb; ++qb) {
-      if (dsr[qb * AT_BK] > last_key) break;   // every later query lives in a later document
-      ++n;
-    }
-    s_info[0] = n;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0) {
+    // query blocks that can see these keys: a prefix (document starts never
+    // decrease), counted 32 blocks at a time with a ballot
+    const int last_key = min(k0 + AT_BLK - 1, T - 1);
+    int n = 0;
+    for (int base = qb_lo; base < nqb; base += 32) {
+      const int qb = base + lane;
+      const bool sees = qb < nqb && dsr[qb * AT_BK] <= last_key;
+      const unsigned m = __ballot_sync(0xffffffffu, sees);
+      n += __popc(m);
+      if (m != 0xffffffffu) break;
+    }
+    if (lane == 0) s_info[0] = n;
   }
   if (warp == 0) tc_alloc(smem_u32(tmem_slot), DkvSmem::TMEM_COLS);
   tc_fence_before();
@@ -349,34 +380,52 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   const uint32_t tmem = *tmem_slot;
   const int niter = s_info[0];
 
-  if (warp == 0 && lane == 0) {
-    // ---------------- producer
-    mbar_expect_tx(bar(0), 2 * AT_TILE_BYTES);
-    tma_load_2d(sK, &tmK, bar(0), C + h * AT_D, (int)(rowbase + k0));
-    tma_load_2d(sV, &tmK, bar(0), 2 * C + h * AT_D, (int)(rowbase + k0));
+  if (warp == 0) {
+    // ---------------- producer (lane 0: TMA; all lanes: per-query lse, D, dstart)
+    if (lane == 0) {
+      mbar_expect_tx(bar(0), 2 * AT_TILE_BYTES);
+      tma_load_2d(sK, &tmK, bar(0), C + h * AT_D, (int)(rowbase + k0));
+      tma_load_2d(sV, &tmK, bar(0), 2 * C + h * AT_D, (int)(rowbase + k0));
+    }
     bool ok = true;
-    for (int i = 0; i < niter && ok; ++i) {
+    for (int i = 0; i < niter; ++i) {
       const int st = i & 1;
       if (!mbar_wait(bar(3 + st), ((i >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-      mbar_expect_tx(bar(1 + st), 2 * AT_HALF);
       const int q0 = (qb_lo + i) * AT_BK;
-      const uint32_t dst = sQD + st * 2 * AT_HALF;
-      tma_load_2d(dst, &tmQ64, bar(1 + st), h * AT_D, (int)(rowbase + q0));
-      tma_load_2d(dst + AT_HALF, &tmDO64, bar(1 + st), h * AT_D, (int)(rowbase + q0));
+      if (lane == 0) {
+        mbar_expect_tx(bar(1 + st), 2 * AT_HALF);
+        const uint32_t dst = sQD + st * 2 * AT_HALF;
+        tma_load_2d(dst, &tmQ64, bar(1 + st), h * AT_D, (int)(rowbase + q0));
+        tma_load_2d(dst + AT_HALF, &tmDO64, bar(1 + st), h * AT_D, (int)(rowbase + q0));
+      }
+      float* L2 = aux + st * 3 * AT_BK;
+      float* Dq = L2 + AT_BK;
+      int* DSq = reinterpret_cast<int*>(Dq + AT_BK);
+#pragma unroll
+      for (int e = lane; e < AT_BK; e += 32) {
+        const int qq = q0 + e;
+        const bool v = qq < T;
+        L2[e] = v ? lse[(long)bh * T + qq] * LOG2E_F : 0.f;
+        Dq[e] = v ? Dbuf[(long)bh * T + qq] : 0.f;
+        DSq[e] = v ? dsr[qq] : 0x7fffffff;
+      }
+      mbar_arrive(bar(1 + st));   // release: the values above are visible to whoever waits on q_full
     }
-    if (!ok) trap_timeout(abort_flag, err);
-    volatile int never = 0;
-    mbar_wait(bar(0), 0, &never, 1ll << 28);
-    for (int i = max(0, niter - 2); i < niter; ++i) mbar_wait(bar(1 + (i & 1)), (i >> 1) & 1, &never, 1ll << 28);
+    if (!ok && lane == 0) trap_timeout(abort_flag, err);
+    if (lane == 0) {
+      volatile int never = 0;
+      mbar_wait(bar(0), 0, &never, 1ll << 28);
+      for (int i = max(0, niter - 2); i < niter; ++i) mbar_wait(bar(1 + (i & 1)), (i >> 1) & 1, &never, 1ll << 28);
+    }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
     constexpr uint32_t ID_SS = instr_desc(64, false, false);   // S^T, dP^T: 128 keys x 64 queries, K = d
     constexpr uint32_t ID_KV = instr_desc(64, false, true);    // dV, dK: 128 keys x 64, K = 64 queries
     bool ok = mbar_wait(bar(0), 0, abort_flag);
-    for (int i = 0; i < niter && ok; ++i) {
+    auto issue_s = [&](int i) -> bool {   // S^T and dP^T of query block i
       const int st = i & 1;
-      if (!mbar_wait(bar(1 + st), (i >> 1) & 1, abort_flag)) { ok = false; break; }
-      if (!mbar_wait(bar(6), (i & 1) ^ 1, abort_flag)) { ok = false; break; }   // S^T / dP^T read
+      if (!mbar_wait(bar(1 + st), (i >> 1) & 1, abort_flag)) return false;
+      if (!mbar_wait(bar(6), (i & 1) ^ 1, abort_flag)) return false;   // previous S^T / dP^T read
       tc_fence_after();
       const uint32_t sQ = sQD + st * 2 * AT_HALF, sDO = sQ + AT_HALF;
 #pragma unroll
@@ -385,8 +434,15 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         umma_bf16(tmem + 64, kdesc(sV + k * 32), kdesc(sDO + k * 32), ID_SS, k > 0);
       }
       umma_commit(bar(5));
+      return true;
+    };
+    if (ok && niter > 0) ok = issue_s(0);
+    for (int i = 0; i < niter && ok; ++i) {
+      const int st = i & 1;
+      if (i + 1 < niter && !issue_s(i + 1)) { ok = false; break; }
       if (!mbar_wait(bar(7), i & 1, abort_flag)) { ok = false; break; }         // P^T, dS^T written
       tc_fence_after();
+      const uint32_t sQ = sQD + st * 2 * AT_HALF, sDO = sQ + AT_HALF;
 #pragma unroll
       for (int kk = 0; kk < AT_BK / 16; ++kk) {
         umma_bf16(tmem + 128, kdesc(sPT + kk * 32), mndesc(sDO + kk * 2048, 8192), ID_KV, (i > 0 || kk > 0));
@@ -408,27 +464,13 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = 0.125f * LOG2E_F;
     bool ok = true;
-    uint32_t gph = 0;
-    // per-query values of the first block
-    float nl = 0.f, nd = 0.f;
-    int nds = 0x7fffffff;
-    if (tid < AT_BK && niter > 0) {
-      const int qq = qb_lo * AT_BK + tid;
-      if (qq < T) { nl = lse[(long)bh * T + qq] * LOG2E_F; nd = Dbuf[(long)bh * T + qq]; nds = dsr[qq]; }
-    }
     for (int i = 0; i < niter; ++i) {
       const int q0 = (qb_lo + i) * AT_BK;
-      float* L2 = aux + (i & 1) * 3 * AT_BK;
-      float* Dq = L2 + AT_BK;
-      int* DSq = reinterpret_cast<int*>(Dq + AT_BK);
-      if (tid < AT_BK) { L2[tid] = nl; Dq[tid] = nd; DSq[tid] = nds; }
-      if (!group_sync(bar(10), gph, abort_flag)) { ok = false; break; }
-      // prefetch the next block's per-query values (consumed next iteration)
-      nl = 0.f; nd = 0.f; nds = 0x7fffffff;
-      if (tid < AT_BK && i + 1 < niter) {
-        const int qq = q0 + AT_BK + tid;
-        if (qq < T) { nl = lse[(long)bh * T + qq] * LOG2E_F; nd = Dbuf[(long)bh * T + qq]; nds = dsr[qq]; }
-      }
+      const int st = i & 1;
+      const float* L2 = aux + st * 3 * AT_BK;
+      const float* Dq = L2 + AT_BK;
+      const int* DSq = reinterpret_cast<const int*>(Dq + AT_BK);
+      if (!mbar_wait(bar(1 + st), (i >> 1) & 1, abort_flag)) { ok = false; break; }   // per-query values
       if (!mbar_wait(bar(5), i & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[64], dr[64];
@@ -506,7 +548,7 @@ struct DqSmem {
   static constexpr int TMEM_COLS = 256;                // S 0..63, dP 64..127, dQ 128..191
 };
 
-__global__ void __launch_bounds__(AT_THREADS)
+__global__ void __launch_bounds__(AT_THREADS, 2)
 attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                const __grid_constant__ CUtensorMap tmKV64, const float* __restrict__ lse,
                const float* __restrict__ Dbuf, const int* __restrict__ dstart, bf16* __restrict__ dqkv, int T,
@@ -576,10 +618,10 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     constexpr uint32_t ID_S = instr_desc(64, false, false);   // S, dP: 128 queries x 64 keys, K = d
     constexpr uint32_t ID_Q = instr_desc(64, false, true);    // dQ += dS K: 128 x 64, K = 64 keys (K MN-major)
     bool ok = mbar_wait(bar(0), 0, abort_flag);
-    for (int j = 0; j < nj && ok; ++j) {
+    auto issue_s = [&](int j) -> bool {
       const int st = j & 1;
-      if (!mbar_wait(bar(1 + st), (j >> 1) & 1, abort_flag)) { ok = false; break; }
-      if (!mbar_wait(bar(6), (j & 1) ^ 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(bar(1 + st), (j >> 1) & 1, abort_flag)) return false;
+      if (!mbar_wait(bar(6), (j & 1) ^ 1, abort_flag)) return false;
       tc_fence_after();
       const uint32_t sK = sKV + st * 2 * AT_HALF, sV = sK + AT_HALF;
 #pragma unroll
@@ -588,8 +630,15 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         umma_bf16(tmem + 64, kdesc(sDO + k * 32), kdesc(sV + k * 32), ID_S, k > 0);
       }
       umma_commit(bar(5));
+      return true;
+    };
+    if (ok && nj > 0) ok = issue_s(0);
+    for (int j = 0; j < nj && ok; ++j) {
+      const int st = j & 1;
+      if (j + 1 < nj && !issue_s(j + 1)) { ok = false; break; }
       if (!mbar_wait(bar(7), j & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
+      const uint32_t sK = sKV + st * 2 * AT_HALF;
 #pragma unroll
       for (int kk = 0; kk < AT_BK / 16; ++kk)
         umma_bf16(tmem + 128, kdesc(sDS + kk * 32), mndesc(sK + kk * 2048, 8192), ID_Q, (j > 0 || kk > 0));
