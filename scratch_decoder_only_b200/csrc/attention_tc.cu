@@ -123,8 +123,8 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nqb = (T + AT_BLK - 1) / AT_BLK;
-  const int qb = nqb - 1 - blockIdx.x;   // heaviest query blocks first
-  const int bh = blockIdx.y, b = bh / H, h = bh % H;
+  const int qb = nqb - 1 - blockIdx.y;   // heaviest query blocks first (y is the slow grid index)
+  const int bh = blockIdx.x, b = bh / H, h = bh % H;
   const int C = H * AT_D;
   const int q0 = qb * AT_BLK;
   const long rowbase = (long)b * T;
@@ -337,8 +337,8 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   float* aux = (float*)(sm + DkvSmem::AUX);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kb = blockIdx.x;   // earliest key blocks see the most queries: launched first
-  const int bh = blockIdx.y, b = bh / H, h = bh % H;
+  const int kb = blockIdx.y;   // earliest key blocks see the most queries: launched first
+  const int bh = blockIdx.x, b = bh / H, h = bh % H;
   const int C = H * AT_D;
   const int k0 = kb * AT_BLK;
   const long rowbase = (long)b * T;
@@ -473,27 +473,28 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
       if (!mbar_wait(bar(1 + st), (i >> 1) & 1, abort_flag)) { ok = false; break; }   // per-query values
       if (!mbar_wait(bar(5), i & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[64], dr[64];
-      tmem_ld32(tmem + lane_off, sr);
-      tmem_ld32(tmem + lane_off + 32, sr + 32);
-      tmem_ld32(tmem + lane_off + 64, dr);
-      tmem_ld32(tmem + lane_off + 96, dr + 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(6));   // S^T / dP^T may be overwritten
-      // the previous block's P^T / dS^T have been consumed
+      // the previous block's P^T / dS^T have been consumed (checked before the first store)
       if (i > 0 && !mbar_wait(bar(8), (i - 1) & 1, abort_flag)) { ok = false; break; }
+      // two 32-query halves keep 64 score values live instead of 128
 #pragma unroll
       for (int c = 0; c < AT_BK; c += 32) {
+        uint32_t sr[32], dr[32];
+        tmem_ld32(tmem + lane_off + c, sr);
+        tmem_ld32(tmem + lane_off + 64 + c, dr);
+        tmem_wait_ld();
+        if (c + 32 == AT_BK) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(6));   // S^T / dP^T may be overwritten
+        }
         float p[32], ds[32];
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) {
           const int ql = c + jj, qq = q0 + ql;
           const bool allowed = qq < T && qq >= k && DSq[ql] <= k;
-          const float pv = allowed ? exp2f(__uint_as_float(sr[ql]) * sl2 - L2[ql]) : 0.f;
+          const float pv = allowed ? exp2f(__uint_as_float(sr[jj]) * sl2 - L2[ql]) : 0.f;
           p[jj] = pv;
-          ds[jj] = pv * (__uint_as_float(dr[ql]) - Dq[ql]);
+          ds[jj] = pv * (__uint_as_float(dr[jj]) - Dq[ql]);
         }
         st_row32_64(sPT, r, c, p);
         st_row32_64(sDST, r, c, ds);
@@ -567,8 +568,8 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nqb = (T + AT_BLK - 1) / AT_BLK;
-  const int qb = nqb - 1 - blockIdx.x;
-  const int bh = blockIdx.y, b = bh / H, h = bh % H;
+  const int qb = nqb - 1 - blockIdx.y;
+  const int bh = blockIdx.x, b = bh / H, h = bh % H;
   const int C = H * AT_D;
   const int q0 = qb * AT_BLK;
   const long rowbase = (long)b * T;
@@ -758,7 +759,7 @@ cudaError_t launch_attn_fwd_tc(const bf16* qkv, bf16* out, float* lse, const int
   const int smem = FwdSmem::TOTAL + 1024;
   static bool attr = false;
   if (!attr) { cudaError_t e = tc_smem_attr(attn_fwd_tc, smem); if (e) return e; attr = true; }
-  dim3 grid((T + AT_BLK - 1) / AT_BLK, B * H);
+  dim3 grid(B * H, (T + AT_BLK - 1) / AT_BLK);
   ++g_kernel_launches;
   attn_fwd_tc<<<grid, AT_THREADS, smem, s>>>(tq, tkv, out, lse, dstart, T, H, err);
   return cudaGetLastError();
@@ -789,7 +790,7 @@ cudaError_t launch_attn_bwd_tc(const bf16* qkv, const bf16* out, const bf16* dou
   attn_rowdot_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(out, dout, Dbuf, B, T, H);
   cudaError_t e;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  dim3 grid((T + AT_BLK - 1) / AT_BLK, B * H);
+  dim3 grid(B * H, (T + AT_BLK - 1) / AT_BLK);
   ++g_kernel_launches;
   attn_bwd_dkdv_tc<<<grid, AT_THREADS, smem_kv, s>>>(tq128, tq64, tdo64, lse, Dbuf, dstart, dqkv, T, H, err);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
