@@ -226,6 +226,27 @@ const char* gpt_last_error(const gpt_model* m);
 int gpt_gemm_bf16(int M, int N, int K, const void* A, long lda, int a_t, const void* B, long ldb, int b_t,
                   float* C, long ldc, void* stream);
 
+/* Split-K variant of gpt_gemm_bf16 that allocates no device memory, for
+ * callers that cannot call cudaMalloc where they need the product (a memory
+ * pool owns the device, an allocation would synchronise a real-time path, or
+ * a host application hands a plugin only the operands).  The paper has no
+ * counterpart: this is a deployment convenience, not a step of the method.
+ *
+ * Same operands, layouts and result as gpt_gemm_bf16 (fp32 C[M, N], row
+ * stride ldc >= N); the K range is split into `splits` slices (1..16, reduced
+ * so that no slice is empty) whose partial sums live in a fixed file-scope
+ * device array of 4194304 floats (16 MiB, held on every GPU that loads the
+ * library until the process exits), then summed into C in a fixed order.
+ * Requires splits * M * N <= 4194304, else GPT_ERR_ARG with the reason in
+ * gpt_last_error(NULL).  Calls no cudaMalloc / cudaFree.
+ * The first call on a device looks up the array's device address with that
+ * device current; make that first call before any stream capture.
+ * All calls share the array (it keeps the last call's partials): calls whose
+ * GPU work overlaps (unordered streams) race on it.
+ * Errors: GPT_ERR_ARG, GPT_ERR_CUDA. */
+int gpt_gemm_bf16_splitk_noalloc(int M, int N, int K, const void* A, long lda, int a_t, const void* B, long ldb,
+                                 int b_t, int splits, float* C, long ldc, void* stream);
+
 /* Number of kernels libgpt has launched in this process (all handles).
  * Benchmarks read it before and after a timed region. */
 int gpt_kernel_launches(uint64_t* out);

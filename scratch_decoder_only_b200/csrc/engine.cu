@@ -644,6 +644,9 @@ static int validate_cfg(const gpt_config* c, std::string& why) {
 
 static thread_local std::string g_create_err;
 
+// Error text for calls without a model handle (reported by gpt_last_error(NULL)).
+void set_global_error(const char* msg) { g_create_err = msg ? msg : ""; }
+
 extern "C" {
 
 int gpt_create(const gpt_config* cfg, uint64_t seed, gpt_model** out) {

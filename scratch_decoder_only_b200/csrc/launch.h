@@ -6,6 +6,9 @@
 #include <stdint.h>
 #include "common.cuh"
 
+// Error text for calls without a model handle (gpt_last_error(NULL)); engine.cu.
+void set_global_error(const char* msg);
+
 // Kernels launched by this library since load (bench / tracing counter).
 extern unsigned long long g_kernel_launches;
 

@@ -29,6 +29,7 @@ EXPORTED = [
     "gpt_set_adam_v", "gpt_get_logits", "gpt_get_residual", "gpt_get_scalars", "gpt_set_scalars", "gpt_status",
     "gpt_device_error", "gpt_last_error", "gpt_debug_poison_grad", "gpt_debug_wait_timeout",
     "gpt_kernel_launches", "gpt_profile_enable", "gpt_profile_read", "gpt_gemm_bf16",
+    "gpt_gemm_bf16_splitk_noalloc",
 ]
 
 
@@ -94,6 +95,8 @@ def load_library(path: str = LIB_PATH):
         "gpt_kernel_launches": ([ctypes.POINTER(ctypes.c_uint64)], I),
         "gpt_profile_enable": ([H, I], I),
         "gpt_gemm_bf16": ([I, I, I, P, ctypes.c_long, I, P, ctypes.c_long, I, P, ctypes.c_long, P], I),
+        "gpt_gemm_bf16_splitk_noalloc": ([I, I, I, P, ctypes.c_long, I, P, ctypes.c_long, I, I, P, ctypes.c_long, P],
+                                         I),
         "gpt_profile_read": ([H, ctypes.POINTER(gpt_prof_entry), I, ctypes.POINTER(I)], I),
     }
     for n in ("params", "grads", "adam_m", "adam_v"):
@@ -138,6 +141,27 @@ def gemm_bf16(A, B, a_t=False, b_t=False, M=None, N=None, K=None, lda=None, ldb=
                          ldb, int(b_t), ctypes.c_void_p(C.data_ptr()), N, ctypes.c_void_p(s))
     if rc != GPT_OK:
         raise GPTError(rc, "gpt_gemm_bf16")
+    return C
+
+
+def gemm_bf16_splitk_noalloc(A, B, a_t=False, b_t=False, splits=4, M=None, N=None, K=None, lda=None, ldb=None):
+    """Split-K form of gemm_bf16 whose partial sums use the library's fixed
+    device scratch array (no device allocation inside the call)."""
+    import torch
+    L = load_library()
+    if M is None:
+        M = A.shape[1] if a_t else A.shape[0]
+        K = A.shape[0] if a_t else A.shape[1]
+        N = B.shape[1] if b_t else B.shape[0]
+    lda = lda or A.stride(0)
+    ldb = ldb or B.stride(0)
+    C = torch.empty((M, N), dtype=torch.float32, device=A.device)
+    s = torch.cuda.current_stream().cuda_stream
+    rc = L.gpt_gemm_bf16_splitk_noalloc(M, N, K, ctypes.c_void_p(A.data_ptr()), lda, int(a_t),
+                                        ctypes.c_void_p(B.data_ptr()), ldb, int(b_t), splits,
+                                        ctypes.c_void_p(C.data_ptr()), N, ctypes.c_void_p(s))
+    if rc != GPT_OK:
+        raise GPTError(rc, L.gpt_last_error(None).decode())
     return C
 
 
