@@ -29,70 +29,85 @@
 #define TC_THREADS 192
 
 // ------------------------------------------------------------------ epilogue
-// Each epilogue warp owns 32 accumulator rows; it walks the tile in 32-column
-// chunks: TMEM -> registers -> epilogue arithmetic -> a 32 x 32 box in its
-// shared-memory staging buffer (swizzled like the TMA box) -> TMA store.
-// Two staging buffers per output alternate so a store can drain while the
-// next chunk is computed.
-#define EPI_WARP_BYTES 8192   // per epilogue warp: 2 buffers x 4 KB
+// The four epilogue warps cooperate on 128-row sub-tiles of the accumulator
+// (64 columns for bf16 outputs, 32 for fp32: 128-byte rows either way): each
+// thread owns one row (its TMEM lane), applies the epilogue and writes the
+// row into a 128-byte-swizzled staging buffer; after a barrier one thread
+// stores the whole 16 KB sub-tile with a single TMA bulk-tensor store.  Two
+// staging buffers per output alternate so a store drains while the next
+// sub-tile is computed (the second output of GELU uses buffers 2 and 3).
+#define EPI_BUF_BYTES 16384
 
-// Write 32 values of row r into a 32 x 32 bf16 box (64-byte rows, 64-byte swizzle).
-__device__ __forceinline__ void stage_bf16(uint32_t buf, int r, const float* v) {
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint4 w;
-    w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
-    w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
-    w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
-    w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
-    uint32_t a = buf + r * 64 + ((q ^ ((r >> 1) & 3)) << 4);
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(w.x), "r"(w.y), "r"(w.z), "r"(w.w)
-                 : "memory");
-  }
-}
-// Write 32 fp32 values of row r into a 32 x 32 fp32 box (128-byte rows, 128-byte swizzle).
-__device__ __forceinline__ void stage_f32(uint32_t buf, int r, const float* v) {
+// Row r (0..127) of a 128-row staging buffer: 8 x 16 bytes, 128-byte swizzle.
+__device__ __forceinline__ void stage_row128(uint32_t buf, int r, const uint4* w) {
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
     uint32_t a = buf + r * 128 + ((q ^ (r & 7)) << 4);
-    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(a), "f"(v[4 * q]), "f"(v[4 * q + 1]),
-                 "f"(v[4 * q + 2]), "f"(v[4 * q + 3])
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(w[q].x), "r"(w[q].y), "r"(w[q].z),
+                 "r"(w[q].w)
                  : "memory");
   }
 }
-
-// 32 consecutive bf16 of one row into registers (16-byte loads), zero past N.
-__device__ __forceinline__ void ld_row32(const bf16* src, int nvalid, uint4* raw) {
-  if (nvalid >= 32) {
+__device__ __forceinline__ void pack_bf16x64(const float* v, uint4* w) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) raw[q] = *reinterpret_cast<const uint4*>(src + 8 * q);
-  } else {
-    bf16* h = reinterpret_cast<bf16*>(raw);
-    for (int j = 0; j < 32; ++j) h[j] = j < nvalid ? src[j] : __float2bfloat16_rn(0.f);
+  for (int q = 0; q < 8; ++q) {
+    w[q].x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    w[q].y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    w[q].z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    w[q].w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
   }
 }
-__device__ __forceinline__ float4 load_bias4(const float* bias, int c, int N) {
-  if (c + 3 < N) return *reinterpret_cast<const float4*>(bias + c);
-  float4 b = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (c < N) b.x = bias[c];
-  if (c + 1 < N) b.y = bias[c + 1];
-  if (c + 2 < N) b.z = bias[c + 2];
-  return b;
-}
-__device__ __forceinline__ void unpack_row32(const uint4* raw, float* x) {
-#pragma unroll
-  for (int q = 0; q < 4; ++q) Vec<bf16>::load(reinterpret_cast<const bf16*>(raw + q), x + 8 * q);
+
+// Bounded barrier of the 128 epilogue threads (an mbarrier with count 128).
+__device__ __forceinline__ bool epi_sync(uint32_t bar, uint32_t& phase, volatile int* abort_flag) {
+  mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, phase, abort_flag);
+  phase ^= 1;
+  return ok;
 }
 
+// Row r of a 128-row, 128-byte-swizzled bf16 buffer (64 values) into fp32.
+__device__ __forceinline__ void load_row128_bf16(uint32_t buf, int r, float* x) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    uint4 w;
+    const uint32_t a = buf + r * 128 + ((q ^ (r & 7)) << 4);
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w) : "r"(a)
+                 : "memory");
+    Vec<bf16>::load(reinterpret_cast<const bf16*>(&w), x + 8 * q);
+  }
+}
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a)
+               : "memory");
+  return v;
+}
 // ------------------------------------------------------------------ the kernel
-template <int BN>
+// EPI_STORE with a residual is its own instantiation: its residual tiles come
+// in by TMA like the DGELU pre-activations.
+#define EPI_STORE_RES 5
+template <int KIND>
+struct EpiTraits {
+  static constexpr bool SIDE = (KIND == EPI_STORE_RES || KIND == EPI_DGELU);   // reads a bf16 [M, N] input
+  static constexpr bool BIAS = (KIND == EPI_STORE || KIND == EPI_STORE_RES || KIND == EPI_GELU);
+  static constexpr bool F32OUT = (KIND == EPI_F32 || KIND == EPI_F32_SPLIT);
+};
+
+template <int BN, int KIND>
 struct TcCfg {
-  static constexpr int STAGES = BN >= 256 ? 4 : 6;
+  // GELU's second output and the side input each take two more staging
+  // buffers; the other kinds keep one more mainloop stage instead
+  static constexpr bool WIDE = (KIND == EPI_GELU || EpiTraits<KIND>::SIDE);
+  static constexpr int EPI_BYTES = (WIDE ? 4 : 2) * EPI_BUF_BYTES;
+  static constexpr int STAGES = (BN >= 256 ? 3 : 4) + (WIDE ? 0 : 1);
+  static constexpr int BIAS_BYTES = EpiTraits<KIND>::BIAS ? BN * 4 : 0;
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;
   static constexpr int B_BYTES = BN * TC_BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
-  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 4 * EPI_WARP_BYTES + 256;
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + 256 + BIAS_BYTES;
+  static_assert(SMEM <= 232448, "shared memory per block");
 };
 
 template <int BN, bool A_MN, bool B_MN, int KIND>
@@ -100,15 +115,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2, int M, int N,
                int K, int splits, EpiParams<bf16> epi, unsigned* err) {
-  using Cfg = TcCfg<BN>;
+  using Cfg = TcCfg<BN, KIND>;
   constexpr int STAGES = Cfg::STAGES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* tile_mem = smem;
-  uint8_t* epi_mem = smem + STAGES * Cfg::STAGE_BYTES;   // 4 warps x EPI_WARP_BYTES, 1024-aligned
-  uint64_t* bars = (uint64_t*)(epi_mem + 4 * EPI_WARP_BYTES);
-  // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
-  uint32_t* tmem_slot = (uint32_t*)(bars + 2 * STAGES + 5);
+  uint8_t* epi_mem = smem + STAGES * Cfg::STAGE_BYTES;   // Cfg::EPI_BYTES of staging, 1024-aligned
+  uint64_t* bars = (uint64_t*)(epi_mem + Cfg::EPI_BYTES);
+  // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain, epilogue group, side[2]
+  uint32_t* tmem_slot = (uint32_t*)(bars + 2 * STAGES + 8);
+  float* bias_s = (float*)((uint8_t*)bars + 256);   // BN bias values of the current tile
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -118,11 +134,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
   auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
   const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+  const uint32_t group_bar = bar0 + 8u * (2 * STAGES + 5);
+  auto side_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 6 + b); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar(a), 1); mbar_init(tempty_bar(a), 4); }
     mbar_init(drain_bar, 1);
+    mbar_init(group_bar, 128);
+    mbar_init(side_bar(0), 1);
+    mbar_init(side_bar(1), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -236,111 +257,154 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     volatile int never = 0;
     mbar_wait(drain_bar, 0, &never, 1ll << 28);
   } else if (warp >= 2) {
-    // ---------------- epilogue: warp w reads TMEM lanes 32*(w%4) .. +31
+    // ---------------- epilogue: thread owns tile row 32*(warp%4) + lane (its TMEM lane)
+    using Tr = EpiTraits<KIND>;
     const int quarter = warp & 3;
-    const uint32_t sbuf = smem_u32(epi_mem + (warp - 2) * EPI_WARP_BYTES);
-    constexpr bool F32OUT = (KIND == EPI_F32 || KIND == EPI_F32_SPLIT);
-    constexpr uint32_t BOX_BYTES = F32OUT ? 4096 : 2048;   // one 32 x 32 box
+    const int rl = quarter * 32 + lane;
+    const int etid = threadIdx.x - 64;
+    constexpr int SW = Tr::F32OUT ? 32 : 64;   // sub-tile columns (128-byte rows)
+    const uint32_t sbase = smem_u32(epi_mem);
+    const uint32_t rbase = sbase + 2 * EPI_BUF_BYTES;   // side-input buffers
+    const uint32_t bias_sa = smem_u32(bias_s);
+    const bool has_bias = Tr::BIAS && epi.bias != nullptr;
+    uint32_t gph = 0;
+    int sub = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
-    int nbuf = 0;
-    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+    bool ok = true;
+    // side input: thread 0 loads sub-tile k into buffer k&1 one sub-tile ahead
+    int ld_u = blockIdx.x, ld_c = 0, issued = 0;
+    auto issue_side = [&]() {
+      if (ld_u >= units) return;
+      const int t = ld_u % tiles;
+      const int m0 = (t % tiles_m) * TC_BM, n0 = (t / tiles_m) * BN;
+      const uint32_t sb = side_bar(issued & 1);
+      mbar_expect_tx(sb, EPI_BUF_BYTES);
+      tma_load_2d(rbase + (issued & 1) * EPI_BUF_BYTES, &tmC2, sb, n0 + ld_c, m0);
+      ++issued;
+      ld_c += SW;
+      if (ld_c >= BN || n0 + ld_c >= N) { ld_c = 0; ld_u += gridDim.x; }
+    };
+    if (Tr::SIDE && etid == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmC2)) : "memory");
+      issue_side();
+    }
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
       const int split = u / tiles, t = u % tiles;
       const int m0 = (t % tiles_m) * TC_BM, n0 = (t / tiles_m) * BN;
-      const int rbase = m0 + quarter * 32;
-      const int row = rbase + lane;
-      const bool row_ok = row < M;
-      if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) {
-        *abort_flag = 1;
-        atomicOr(err, GPT_DEVERR_TIMEOUT);
-        break;
+      // this tile's bias: fetched before the accumulator wait, written to shared
+      // memory after it (every thread has finished the previous tile's reads:
+      // they precede its last group barrier)
+      float bv[BN / 128];
+      if (has_bias) {
+#pragma unroll
+        for (int j = 0; j < BN / 128; ++j) {
+          const int col = n0 + etid + 128 * j;
+          bv[j] = col < N ? epi.bias[col] : 0.f;
+        }
       }
+      if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) { ok = false; break; }
       tc_fence_after();
+      if (has_bias) {
+#pragma unroll
+        for (int j = 0; j < BN / 128; ++j) bias_s[etid + 128 * j] = bv[j];
+      }
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
-      // residual (STORE) or pre-activation (DGELU) row chunks, prefetched one chunk ahead
-      const bf16* side = nullptr;
-      long side_ld = 0;
-      if (KIND == EPI_STORE && epi.resid) { side = epi.resid; side_ld = epi.ld_resid; }
-      if (KIND == EPI_DGELU) { side = epi.aux; side_ld = epi.ld_aux; }
-      uint4 nxt[4];
-      if (side && row_ok) ld_row32(side + (long)row * side_ld + n0, N - n0, nxt);
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
+      for (int c = 0; c < BN; c += SW) {
         const int col0 = n0 + c;
         if (col0 >= N) break;
-        uint32_t r[32];
+        uint32_t r[SW];
         tmem_ld32(tbase + c, r);
-        uint4 cur[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) cur[q] = nxt[q];
-        if (side && row_ok && c + 32 < BN && col0 + 32 < N)
-          ld_row32(side + (long)row * side_ld + col0 + 32, N - col0 - 32, nxt);
+        if (SW == 64) tmem_ld32(tbase + c + 32, r + 32);
         tmem_wait_ld();
-        float v[32];
+        if (c + SW >= BN || col0 + SW >= N) {   // last sub-tile: the accumulator can be reused
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty_bar(acc));
+        }
+        // the store that last used this staging buffer has read it
+        if (etid == 0) bulk_wait_read<1>();
+        if (!epi_sync(group_bar, gph, abort_flag)) { ok = false; break; }
+        // every thread is past the previous sub-tile: its side buffer is free
+        if (Tr::SIDE && etid == 0) issue_side();
+        const uint32_t b0 = sbase + (sub & 1) * EPI_BUF_BYTES;
+        float v[SW];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-        // wait until the store that last used this staging buffer has read it
-        if (lane == 0) bulk_wait_read<1>();
-        __syncwarp();
-        const uint32_t b0 = sbuf + nbuf * BOX_BYTES;
-        if constexpr (KIND == EPI_STORE) {
-          if (epi.bias) {
+        for (int j = 0; j < SW; ++j) v[j] = __uint_as_float(r[j]);
+        if (has_bias) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              float4 bb = load_bias4(epi.bias, col0 + 4 * q, N);
-              v[4 * q] += bb.x; v[4 * q + 1] += bb.y; v[4 * q + 2] += bb.z; v[4 * q + 3] += bb.w;
-            }
-          }
-          if (side) {
-            float rr[32];
-            unpack_row32(cur, rr);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] += rr[j];
-          }
-          stage_bf16(b0, lane, v);
-        } else if constexpr (KIND == EPI_GELU) {
-          float a[32];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            float4 bb = load_bias4(epi.bias, col0 + 4 * q, N);
+          for (int q = 0; q < SW / 4; ++q) {
+            const float4 bb = ld_shared_f4(bias_sa + (c + 4 * q) * 4);
             v[4 * q] += bb.x; v[4 * q + 1] += bb.y; v[4 * q + 2] += bb.z; v[4 * q + 3] += bb.w;
           }
+        }
+        if constexpr (Tr::SIDE) {
+          if (!mbar_wait(side_bar(sub & 1), (sub >> 1) & 1, abort_flag)) { ok = false; break; }
+        }
+        uint4 w[8];
+        if constexpr (KIND == EPI_STORE || KIND == EPI_STORE_RES) {
+          if constexpr (KIND == EPI_STORE_RES) {
+            float rr[64];
+            load_row128_bf16(rbase + (sub & 1) * EPI_BUF_BYTES, rl, rr);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            float uq = __bfloat162float(__float2bfloat16_rn(v[j]));
+            for (int j = 0; j < 64; ++j) v[j] += rr[j];
+          }
+          pack_bf16x64(v, w);
+          stage_row128(b0, rl, w);
+        } else if constexpr (KIND == EPI_GELU) {
+          float a[64];
+#pragma unroll
+          for (int j = 0; j < 64; ++j) {
+            const float uq = __bfloat162float(__float2bfloat16_rn(v[j]));
             v[j] = uq;
             a[j] = gelu_fast(uq);
           }
-          stage_bf16(b0, lane, v);
-          stage_bf16(b0 + 2 * BOX_BYTES, lane, a);
+          pack_bf16x64(v, w);
+          stage_row128(b0, rl, w);
+          pack_bf16x64(a, w);
+          stage_row128(b0 + 2 * EPI_BUF_BYTES, rl, w);
         } else if constexpr (KIND == EPI_DGELU) {
-          float uu[32];
-          unpack_row32(cur, uu);
+          float uu[64];
+          load_row128_bf16(rbase + (sub & 1) * EPI_BUF_BYTES, rl, uu);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] *= gelu_grad_fast(uu[j]);
-          stage_bf16(b0, lane, v);
+          for (int j = 0; j < 64; ++j) v[j] *= gelu_grad_fast(uu[j]);
+          pack_bf16x64(v, w);
+          stage_row128(b0, rl, w);
         } else {
-          stage_f32(b0, lane, v);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            w[q] = make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]), __float_as_uint(v[4 * q + 2]),
+                              __float_as_uint(v[4 * q + 3]));
+          stage_row128(b0, rl, w);
         }
         fence_async_smem();
-        __syncwarp();
-        if (lane == 0) {
+        if (!epi_sync(group_bar, gph, abort_flag)) { ok = false; break; }
+        if (etid == 0) {
           if constexpr (KIND == EPI_F32_SPLIT) {
-            tma_store_3d(&tmC, b0, col0, rbase, split);
+            tma_store_3d(&tmC, b0, col0, m0, split);
           } else {
-            tma_store_2d(&tmC, b0, col0, rbase);
-            if constexpr (KIND == EPI_GELU) tma_store_2d(&tmC2, b0 + 2 * BOX_BYTES, col0, rbase);
+            tma_store_2d(&tmC, b0, col0, m0);
+            if constexpr (KIND == EPI_GELU) tma_store_2d(&tmC2, b0 + 2 * EPI_BUF_BYTES, col0, m0);
           }
           bulk_commit();
         }
-        nbuf ^= 1;
+        ++sub;
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tempty_bar(acc));
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
-    if (lane == 0) bulk_wait_all();
+    if (!ok) {
+      *abort_flag = 1;
+      atomicOr(err, GPT_DEVERR_TIMEOUT);
+    }
+    if (etid == 0) {
+      bulk_wait_all();
+      // side loads issued but not consumed (only after an abort): let them land
+      for (int k = sub; k < issued; ++k) {
+        volatile int never = 0;
+        mbar_wait(side_bar(k & 1), (k >> 1) & 1, &never, 1ll << 28);
+      }
+    }
     __syncwarp();
   }
   tc_fence_before();
@@ -366,7 +430,7 @@ template <int BN, bool A_MN, bool B_MN, int KIND>
 static cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc,
                              const CUtensorMap& tc2, int M, int N, int K, int splits, const EpiParams<bf16>& epi,
                              unsigned* err, cudaStream_t s) {
-  using Cfg = TcCfg<BN>;
+  using Cfg = TcCfg<BN, KIND>;
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, A_MN, B_MN, KIND>,
@@ -390,6 +454,8 @@ static cudaError_t launch_kind(const CUtensorMap& ta, const CUtensorMap& tb, con
                                unsigned* err, cudaStream_t s) {
   if (epi.kind == EPI_F32) return launch_tc<BN, A_MN, B_MN, EPI_F32>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
   if constexpr (!A_MN) {
+    if (epi.kind == EPI_STORE && epi.resid)
+      return launch_tc<BN, A_MN, B_MN, EPI_STORE_RES>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
     if (epi.kind == EPI_STORE) return launch_tc<BN, A_MN, B_MN, EPI_STORE>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
     if constexpr (!B_MN) {
       if (epi.kind == EPI_GELU) return launch_tc<BN, A_MN, B_MN, EPI_GELU>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
@@ -413,23 +479,28 @@ static cudaError_t launch_bn(int M, int N, int K, const bf16* A, long lda, bool 
   if (!ok) return cudaErrorInvalidValue;
   ok = b_t ? make_map(&tb, B, K, N, ldb, 64, TC_BK) : make_map(&tb, B, N, K, ldb, TC_BK, BN);
   if (!ok) return cudaErrorInvalidValue;
-  // output boxes: 32 x 32, bf16 with 64-byte swizzle or fp32 with 128-byte swizzle
+  // output boxes: 128 rows x 128 bytes (64 bf16 or 32 fp32 columns), 128-byte swizzle
   switch (epi.kind) {
     case EPI_STORE:
-    case EPI_DGELU:
-      ok = make_map_ex(&tc, MapKey{epi.out, M, N, epi.ld_out, 1, 0, 32, 32, 0, 64});
+      ok = make_map_ex(&tc, MapKey{epi.out, M, N, epi.ld_out, 1, 0, 64, TC_BM, 0, 128});
       tc2 = tc;
+      // the residual is read by TMA in the same 128 x 64 boxes
+      if (ok && epi.resid) ok = make_map_ex(&tc2, MapKey{epi.resid, M, N, epi.ld_resid, 1, 0, 64, TC_BM, 0, 128});
+      break;
+    case EPI_DGELU:
+      ok = make_map_ex(&tc, MapKey{epi.out, M, N, epi.ld_out, 1, 0, 64, TC_BM, 0, 128}) &&
+           make_map_ex(&tc2, MapKey{epi.aux, M, N, epi.ld_aux, 1, 0, 64, TC_BM, 0, 128});
       break;
     case EPI_GELU:
-      ok = make_map_ex(&tc, MapKey{epi.out, M, N, epi.ld_out, 1, 0, 32, 32, 0, 64}) &&
-           make_map_ex(&tc2, MapKey{epi.out2, M, N, epi.ld_out2, 1, 0, 32, 32, 0, 64});
+      ok = make_map_ex(&tc, MapKey{epi.out, M, N, epi.ld_out, 1, 0, 64, TC_BM, 0, 128}) &&
+           make_map_ex(&tc2, MapKey{epi.out2, M, N, epi.ld_out2, 1, 0, 64, TC_BM, 0, 128});
       break;
     case EPI_F32:
-      ok = make_map_ex(&tc, MapKey{epi.outf, M, N, epi.ld_outf, 1, 0, 32, 32, 1, 128});
+      ok = make_map_ex(&tc, MapKey{epi.outf, M, N, epi.ld_outf, 1, 0, 32, TC_BM, 1, 128});
       tc2 = tc;
       break;
     case EPI_F32_SPLIT:
-      ok = make_map_ex(&tc, MapKey{epi.outf, M, N, epi.ld_outf, splits, epi.split_stride, 32, 32, 1, 128});
+      ok = make_map_ex(&tc, MapKey{epi.outf, M, N, epi.ld_outf, splits, epi.split_stride, 32, TC_BM, 1, 128});
       tc2 = tc;
       break;
     default:
@@ -457,6 +528,10 @@ cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* A, long lda, bool a_
   for (const void* o : outs)
     if (o && ((uintptr_t)o & 15)) return cudaErrorInvalidValue;
   if (epi.kind >= EPI_F32 ? (epi.ld_outf & 3) : (epi.ld_out & 7)) return cudaErrorInvalidValue;
+  // residual / pre-activation inputs are read by TMA too
+  const bf16* side = epi.kind == EPI_STORE ? epi.resid : epi.kind == EPI_DGELU ? epi.aux : nullptr;
+  const long side_ld = epi.kind == EPI_STORE ? epi.ld_resid : epi.ld_aux;
+  if (side && (((uintptr_t)side & 15) || (side_ld & 7))) return cudaErrorInvalidValue;
   if (splits < 1) splits = 1;
   // tile width: prefer 256 columns unless 128 fills the machine's waves better
   long tm = (M + TC_BM - 1) / TC_BM;
