@@ -304,37 +304,60 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
   if (warp == 0) tc_dealloc(tmem, FwdSmem::TMEM_COLS);
 }
 
-// ============================================================== backward: dK, dV
-struct DkvSmem {
-  static constexpr int K = 0;                          // 16 KB: 128 keys
-  static constexpr int V = K + AT_TILE_BYTES;          // 16 KB
-  static constexpr int QD = V + AT_TILE_BYTES;         // 2 stages x (Q 8 KB, dO 8 KB)
-  static constexpr int PT = QD + 4 * AT_HALF;          // 16 KB: 128 keys x 64 queries
-  static constexpr int DST = PT + AT_TILE_BYTES;       // 16 KB
-  static constexpr int AUX = DST + AT_TILE_BYTES;      // 2 x (lse2, D, dstart) x 64
-  static constexpr int BAR = AUX + 2 * 3 * AT_BK * 4;
+// ============================================================== backward
+// One CTA per 128-key block: it walks the 128-query blocks that can see its
+// keys and, per block,
+//   S^T = K Q^T, dP^T = V dO^T                  (TMEM, 128 x 128 each)
+//   P^T = exp2(S^T log2e / 8 - lse log2e),  dS^T = P^T (dP^T - D)    (smem)
+//   dV += P^T dO,  dK += dS^T Q                  (TMEM, across query blocks)
+//   dQ_blk = dS K                                (TMEM; added in fp32 to a
+//                                                 global accumulator by a TMA
+//                                                 bulk reduce, scaled by 1/8
+//                                                 and rounded by a final pass)
+// 320 threads: warp 0 loads, warp 1 issues MMAs, warps 2-9 are two groups of
+// four elementwise warps; group g handles query columns 64g..64g+63 of the
+// score tiles and d columns 32g..32g+31 of the dQ, dK, dV accumulators.
+#define BW_THREADS 320
+#define BW_QB 128                                    // queries per iterated block
+struct BwdSmem {
+  static constexpr int K = 0;                        // 16 KB: 128 keys x 64
+  static constexpr int V = K + AT_TILE_BYTES;        // 16 KB
+  static constexpr int Q = V + AT_TILE_BYTES;        // 2 stages x 16 KB
+  static constexpr int DO = Q + 2 * AT_TILE_BYTES;   // 2 stages x 16 KB
+  static constexpr int PT = DO + 2 * AT_TILE_BYTES;  // 32 KB: [128 keys][128 queries] as two 64-query blocks
+  static constexpr int DST = PT + 2 * AT_TILE_BYTES; // 32 KB, same layout
+  static constexpr int DQS = DST + 2 * AT_TILE_BYTES;// 2 groups x 16 KB: [128 queries][32 fp32]
+  static constexpr int AUX = DQS + 2 * AT_TILE_BYTES;// 2 stages x (lse2, D, dstart) x 128
+  static constexpr int BAR = AUX + 2 * 3 * BW_QB * 4;
   static constexpr int TOTAL = BAR + 256;
-  static constexpr int TMEM_COLS = 256;                // S^T 0..63, dP^T 64..127, dV 128..191, dK 192..255
+  static constexpr int TMEM_COLS = 512;              // S^T 0, dP^T 128, dV 256, dK 320, dQ 384
 };
 
-__global__ void __launch_bounds__(AT_THREADS, 2)
-attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ64,
-                 const __grid_constant__ CUtensorMap tmDO64, const float* __restrict__ lse,
-                 const float* __restrict__ Dbuf, const int* __restrict__ dstart, bf16* __restrict__ dqkv, int T,
-                 int H, unsigned* err) {
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__global__ void __launch_bounds__(BW_THREADS, 1)
+attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
+            const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ lse, const float* __restrict__ Dbuf,
+            const int* __restrict__ dstart, bf16* __restrict__ dqkv, int T, int H, unsigned* err) {
   extern __shared__ __align__(1024) uint8_t at_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)at_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t* bars = (uint64_t*)(sm + DkvSmem::BAR);
+  uint64_t* bars = (uint64_t*)(sm + BwdSmem::BAR);
   // bars: 0 kv_full, 1-2 q_full (TMA tiles + per-query values), 3-4 q_empty, 5 s_full, 6 s_free,
-  //       7 p_full, 8 p_free, 9 drain
-  uint32_t* tmem_slot = (uint32_t*)(bars + 11);
+  //       7 p_full, 8 mma_done (P^T / dS^T read, dQ_blk complete), 9 dq_free, 10 drain,
+  //       11-12 group barriers
+  uint32_t* tmem_slot = (uint32_t*)(bars + 13);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   int* s_info = (int*)(tmem_slot + 2);
   const uint32_t b0 = smem_u32(bars);
   auto bar = [&](int i) { return b0 + 8u * i; };
-  const uint32_t sK = smem_u32(sm + DkvSmem::K), sV = smem_u32(sm + DkvSmem::V), sQD = smem_u32(sm + DkvSmem::QD);
-  const uint32_t sPT = smem_u32(sm + DkvSmem::PT), sDST = smem_u32(sm + DkvSmem::DST);
-  float* aux = (float*)(sm + DkvSmem::AUX);
+  const uint32_t sK = smem_u32(sm + BwdSmem::K), sV = smem_u32(sm + BwdSmem::V);
+  const uint32_t sQ = smem_u32(sm + BwdSmem::Q), sDO = smem_u32(sm + BwdSmem::DO);
+  const uint32_t sPT = smem_u32(sm + BwdSmem::PT), sDST = smem_u32(sm + BwdSmem::DST);
+  const uint32_t sDQ = smem_u32(sm + BwdSmem::DQS);
+  float* aux = (float*)(sm + BwdSmem::AUX);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kb = blockIdx.y;   // earliest key blocks see the most queries: launched first
@@ -343,18 +366,21 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   const int k0 = kb * AT_BLK;
   const long rowbase = (long)b * T;
   const int* dsr = dstart + rowbase;
-  const int nqb = (T + AT_BK - 1) / AT_BK;
-  const int qb_lo = k0 / AT_BK;
+  const int nqb = (T + BW_QB - 1) / BW_QB;
+  const int qb_lo = k0 / BW_QB;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(0), 1);
     for (int i = 1; i <= 2; ++i) mbar_init(bar(i), 1 + 32);   // TMA arrival + 32 lanes of per-query values
     for (int i = 3; i <= 4; ++i) mbar_init(bar(i), 1);
     mbar_init(bar(5), 1);
-    mbar_init(bar(6), 4);
-    mbar_init(bar(7), 4);
+    mbar_init(bar(6), 8);
+    mbar_init(bar(7), 8);
     mbar_init(bar(8), 1);
-    mbar_init(bar(9), 1);
+    mbar_init(bar(9), 8);
+    mbar_init(bar(10), 1);
+    mbar_init(bar(11), 128);
+    mbar_init(bar(12), 128);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -366,14 +392,14 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     int n = 0;
     for (int base = qb_lo; base < nqb; base += 32) {
       const int qb = base + lane;
-      const bool sees = qb < nqb && dsr[qb * AT_BK] <= last_key;
+      const bool sees = qb < nqb && dsr[qb * BW_QB] <= last_key;
       const unsigned m = __ballot_sync(0xffffffffu, sees);
       n += __popc(m);
       if (m != 0xffffffffu) break;
     }
     if (lane == 0) s_info[0] = n;
   }
-  if (warp == 0) tc_alloc(smem_u32(tmem_slot), DkvSmem::TMEM_COLS);
+  if (warp == 0) tc_alloc(smem_u32(tmem_slot), BwdSmem::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -381,33 +407,43 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   const int niter = s_info[0];
 
   if (warp == 0) {
-    // ---------------- producer (lane 0: TMA; all lanes: per-query lse, D, dstart)
+    // ---------------- producer (lane 0: TMA; all lanes: per-query lse2, D, dstart)
     if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQKV)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmDO)) : "memory");
       mbar_expect_tx(bar(0), 2 * AT_TILE_BYTES);
-      tma_load_2d(sK, &tmK, bar(0), C + h * AT_D, (int)(rowbase + k0));
-      tma_load_2d(sV, &tmK, bar(0), 2 * C + h * AT_D, (int)(rowbase + k0));
+      tma_load_2d(sK, &tmQKV, bar(0), C + h * AT_D, (int)(rowbase + k0));
+      tma_load_2d(sV, &tmQKV, bar(0), 2 * C + h * AT_D, (int)(rowbase + k0));
     }
     bool ok = true;
     for (int i = 0; i < niter; ++i) {
       const int st = i & 1;
-      if (!mbar_wait(bar(3 + st), ((i >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-      const int q0 = (qb_lo + i) * AT_BK;
-      if (lane == 0) {
-        mbar_expect_tx(bar(1 + st), 2 * AT_HALF);
-        const uint32_t dst = sQD + st * 2 * AT_HALF;
-        tma_load_2d(dst, &tmQ64, bar(1 + st), h * AT_D, (int)(rowbase + q0));
-        tma_load_2d(dst + AT_HALF, &tmDO64, bar(1 + st), h * AT_D, (int)(rowbase + q0));
-      }
-      float* L2 = aux + st * 3 * AT_BK;
-      float* Dq = L2 + AT_BK;
-      int* DSq = reinterpret_cast<int*>(Dq + AT_BK);
+      const int q0 = (qb_lo + i) * BW_QB;
+      // per-query values into registers before the stage is free
+      float l2v[4], dv[4];
+      int dsv[4];
 #pragma unroll
-      for (int e = lane; e < AT_BK; e += 32) {
-        const int qq = q0 + e;
+      for (int e = 0; e < 4; ++e) {
+        const int qq = q0 + lane + 32 * e;
         const bool v = qq < T;
-        L2[e] = v ? lse[(long)bh * T + qq] * LOG2E_F : 0.f;
-        Dq[e] = v ? Dbuf[(long)bh * T + qq] : 0.f;
-        DSq[e] = v ? dsr[qq] : 0x7fffffff;
+        l2v[e] = v ? lse[(long)bh * T + qq] * LOG2E_F : 0.f;
+        dv[e] = v ? Dbuf[(long)bh * T + qq] : 0.f;
+        dsv[e] = v ? dsr[qq] : 0x7fffffff;
+      }
+      if (!mbar_wait(bar(3 + st), ((i >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+      if (lane == 0) {
+        mbar_expect_tx(bar(1 + st), 2 * AT_TILE_BYTES);
+        tma_load_2d(sQ + st * AT_TILE_BYTES, &tmQKV, bar(1 + st), h * AT_D, (int)(rowbase + q0));
+        tma_load_2d(sDO + st * AT_TILE_BYTES, &tmDO, bar(1 + st), h * AT_D, (int)(rowbase + q0));
+      }
+      float* L2 = aux + st * 3 * BW_QB;
+      float* Dq = L2 + BW_QB;
+      int* DSq = reinterpret_cast<int*>(Dq + BW_QB);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        L2[lane + 32 * e] = l2v[e];
+        Dq[lane + 32 * e] = dv[e];
+        DSq[lane + 32 * e] = dsv[e];
       }
       mbar_arrive(bar(1 + st));   // release: the values above are visible to whoever waits on q_full
     }
@@ -419,19 +455,20 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
-    constexpr uint32_t ID_SS = instr_desc(64, false, false);   // S^T, dP^T: 128 keys x 64 queries, K = d
-    constexpr uint32_t ID_KV = instr_desc(64, false, true);    // dV, dK: 128 keys x 64, K = 64 queries
+    constexpr uint32_t ID_SS = instr_desc(128, false, false);   // S^T, dP^T: 128 keys x 128 queries, K = d
+    constexpr uint32_t ID_KV = instr_desc(64, false, true);     // dV, dK: 128 keys x 64, K = 128 queries
+    constexpr uint32_t ID_DQ = instr_desc(64, true, true);      // dQ: 128 queries x 64, K = 128 keys
     bool ok = mbar_wait(bar(0), 0, abort_flag);
     auto issue_s = [&](int i) -> bool {   // S^T and dP^T of query block i
       const int st = i & 1;
       if (!mbar_wait(bar(1 + st), (i >> 1) & 1, abort_flag)) return false;
       if (!mbar_wait(bar(6), (i & 1) ^ 1, abort_flag)) return false;   // previous S^T / dP^T read
       tc_fence_after();
-      const uint32_t sQ = sQD + st * 2 * AT_HALF, sDO = sQ + AT_HALF;
+      const uint32_t q = sQ + st * AT_TILE_BYTES, o = sDO + st * AT_TILE_BYTES;
 #pragma unroll
       for (int k = 0; k < AT_D / 16; ++k) {
-        umma_bf16(tmem + 0, kdesc(sK + k * 32), kdesc(sQ + k * 32), ID_SS, k > 0);
-        umma_bf16(tmem + 64, kdesc(sV + k * 32), kdesc(sDO + k * 32), ID_SS, k > 0);
+        umma_bf16(tmem + 0, kdesc(sK + k * 32), kdesc(q + k * 32), ID_SS, k > 0);
+        umma_bf16(tmem + 128, kdesc(sV + k * 32), kdesc(o + k * 32), ID_SS, k > 0);
       }
       umma_commit(bar(5));
       return true;
@@ -440,283 +477,206 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     for (int i = 0; i < niter && ok; ++i) {
       const int st = i & 1;
       if (i + 1 < niter && !issue_s(i + 1)) { ok = false; break; }
-      if (!mbar_wait(bar(7), i & 1, abort_flag)) { ok = false; break; }         // P^T, dS^T written
+      if (!mbar_wait(bar(7), i & 1, abort_flag)) { ok = false; break; }   // P^T, dS^T written
       tc_fence_after();
-      const uint32_t sQ = sQD + st * 2 * AT_HALF, sDO = sQ + AT_HALF;
+      const uint32_t q = sQ + st * AT_TILE_BYTES, o = sDO + st * AT_TILE_BYTES;
 #pragma unroll
-      for (int kk = 0; kk < AT_BK / 16; ++kk) {
-        umma_bf16(tmem + 128, kdesc(sPT + kk * 32), mndesc(sDO + kk * 2048, 8192), ID_KV, (i > 0 || kk > 0));
-        umma_bf16(tmem + 192, kdesc(sDST + kk * 32), mndesc(sQ + kk * 2048, 8192), ID_KV, (i > 0 || kk > 0));
+      for (int kk = 0; kk < BW_QB / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * AT_TILE_BYTES + (kk & 3) * 32;
+        umma_bf16(tmem + 256, kdesc(sPT + off), mndesc(o + kk * 2048, 8192), ID_KV, (i > 0 || kk > 0));
+        umma_bf16(tmem + 320, kdesc(sDST + off), mndesc(q + kk * 2048, 8192), ID_KV, (i > 0 || kk > 0));
       }
-      umma_commit(bar(8));        // P^T / dS^T buffers free
       umma_commit(bar(3 + st));   // Q / dO stage free
+      // dQ_blk = dS K once the previous block's dQ has been read out
+      if (i > 0 && !mbar_wait(bar(9), (i - 1) & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < AT_BLK / 16; ++kk)
+        umma_bf16(tmem + 384, mndesc(sDST + kk * 2048, AT_TILE_BYTES), mndesc(sK + kk * 2048, 8192), ID_DQ, kk > 0);
+      umma_commit(bar(8));
     }
     if (!ok) trap_timeout(abort_flag, err);
-    umma_commit(bar(9));
+    umma_commit(bar(10));
     volatile int never = 0;
-    mbar_wait(bar(9), 0, &never, 1ll << 28);
+    mbar_wait(bar(10), 0, &never, 1ll << 28);
   } else if (warp >= 2) {
-    // ---------------- elementwise warps: thread owns key row r
+    // ---------------- elementwise warps: thread owns key row r (and query row r of dQ)
     const int quarter = warp & 3;
+    const int grp = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
     const int k = k0 + r;
-    const int tid = threadIdx.x - 64;
+    const int gtid = threadIdx.x - 64 - 128 * grp;   // 0..127 inside the group
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = 0.125f * LOG2E_F;
+    const uint32_t gbar = bar(11 + grp);
+    const uint32_t sDQg = sDQ + grp * AT_TILE_BYTES;
+    uint32_t gph = 0;
     bool ok = true;
-    for (int i = 0; i < niter; ++i) {
-      const int q0 = (qb_lo + i) * AT_BK;
-      const int st = i & 1;
-      const float* L2 = aux + st * 3 * AT_BK;
-      const float* Dq = L2 + AT_BK;
-      const int* DSq = reinterpret_cast<const int*>(Dq + AT_BK);
-      if (!mbar_wait(bar(1 + st), (i >> 1) & 1, abort_flag)) { ok = false; break; }   // per-query values
-      if (!mbar_wait(bar(5), i & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      // the previous block's P^T / dS^T have been consumed (checked before the first store)
-      if (i > 0 && !mbar_wait(bar(8), (i - 1) & 1, abort_flag)) { ok = false; break; }
-      // two 32-query halves keep 64 score values live instead of 128
+    // waits are voted warp-wide so that the .sync.aligned TMEM loads after them
+    // are never reached by part of a warp
+    auto wait_w = [&](uint32_t bb, uint32_t parity) { return __all_sync(0xffffffffu, mbar_wait(bb, parity, abort_flag)); };
+    // dQ of block j: TMEM -> fp32 staging (128-byte swizzle) -> bulk reduce-add
+    auto flush_dq = [&](int j) -> bool {
+      uint32_t rr[32];
+      tmem_ld32(tmem + lane_off + 384 + 32 * grp, rr);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(9));   // the dQ accumulator may be overwritten
+      if (gtid == 0) bulk_wait_read<0>();   // the previous reduce has read the staging
+      if (!__all_sync(0xffffffffu, group_sync(gbar, gph, abort_flag))) return false;
 #pragma unroll
-      for (int c = 0; c < AT_BK; c += 32) {
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t a = sDQg + r * 128 + ((u ^ (r & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(rr[4 * u]), "r"(rr[4 * u + 1]),
+                     "r"(rr[4 * u + 2]), "r"(rr[4 * u + 3])
+                     : "memory");
+      }
+      fence_async_smem();
+      if (!__all_sync(0xffffffffu, group_sync(gbar, gph, abort_flag))) return false;
+      if (gtid == 0) {
+        tma_reduce_add_2d(&tmDQ, sDQg, h * AT_D + 32 * grp, (int)(rowbase + (qb_lo + j) * BW_QB));
+        bulk_commit();
+      }
+      return true;
+    };
+    for (int i = 0; i < niter; ++i) {
+      const int q0 = (qb_lo + i) * BW_QB;
+      const int st = i & 1;
+      const float4* aL2 = reinterpret_cast<const float4*>(aux + st * 3 * BW_QB + grp * 64);
+      const float4* aD = aL2 + BW_QB / 4;
+      const int4* aDS = reinterpret_cast<const int4*>(aL2 + BW_QB / 2);
+      if (!wait_w(bar(1 + st), (i >> 1) & 1)) { ok = false; break; }   // per-query values
+      if (!wait_w(bar(5), i & 1)) { ok = false; break; }
+      tc_fence_after();
+      // masking only where a key can be later than a query or before its document
+      // (document starts never decrease, queries past T carry INT_MAX)
+      const int ds_last = reinterpret_cast<const int*>(aux)[st * 3 * BW_QB + 2 * BW_QB + BW_QB - 1];
+      const bool need_mask = q0 < k0 + AT_BLK || ds_last > k0;
+      // P^T and dS^T as packed bf16 pairs, 32 columns at a time (64 score
+      // registers live); the score buffers are released after the second load
+      uint32_t pw[32], dw[32];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
         uint32_t sr[32], dr[32];
-        tmem_ld32(tmem + lane_off + c, sr);
-        tmem_ld32(tmem + lane_off + 64 + c, dr);
+        tmem_ld32(tmem + lane_off + 64 * grp + 32 * half, sr);
+        tmem_ld32(tmem + lane_off + 128 + 64 * grp + 32 * half, dr);
         tmem_wait_ld();
-        if (c + 32 == AT_BK) {
+        if (half == 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(6));   // S^T / dP^T may be overwritten
         }
-        float p[32], ds[32];
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const int ql = c + jj, qq = q0 + ql;
-          const bool allowed = qq < T && qq >= k && DSq[ql] <= k;
-          const float pv = allowed ? exp2f(__uint_as_float(sr[jj]) * sl2 - L2[ql]) : 0.f;
-          p[jj] = pv;
-          ds[jj] = pv * (__uint_as_float(dr[jj]) - Dq[ql]);
-        }
-        st_row32_64(sPT, r, c, p);
-        st_row32_64(sDST, r, c, ds);
-      }
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(7));
-    }
-    if (!ok) trap_timeout(abort_flag, err);
-    // wait for the last dV / dK accumulation, then write the rows
-    if (ok && niter > 0 && mbar_wait(bar(8), (niter - 1) & 1, abort_flag)) {
-      tc_fence_after();
-      bf16* row = dqkv + (rowbase + k) * 3 * C;
+        for (int c8 = 0; c8 < 32; c8 += 8) {
+          const int c = 32 * half + c8;
+          float lv[8], dv[8];
+          int dsq[8];
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        const float sc = part == 0 ? 0.125f : 1.f;
-        bf16* dst = row + (part == 0 ? C : 2 * C) + h * AT_D;
+          for (int hh = 0; hh < 2; ++hh) {
+            const float4 l4 = aL2[c / 4 + hh];
+            const float4 d4 = aD[c / 4 + hh];
+            lv[4 * hh] = l4.x; lv[4 * hh + 1] = l4.y; lv[4 * hh + 2] = l4.z; lv[4 * hh + 3] = l4.w;
+            dv[4 * hh] = d4.x; dv[4 * hh + 1] = d4.y; dv[4 * hh + 2] = d4.z; dv[4 * hh + 3] = d4.w;
+            int4 s4 = make_int4(0, 0, 0, 0);
+            if (need_mask) s4 = aDS[c / 4 + hh];
+            dsq[4 * hh] = s4.x; dsq[4 * hh + 1] = s4.y; dsq[4 * hh + 2] = s4.z; dsq[4 * hh + 3] = s4.w;
+          }
+          float pv[8], gv[8];
 #pragma unroll
-        for (int c = 0; c < AT_D; c += 32) {
-          uint32_t rr[32];
-          tmem_ld32(tmem + lane_off + (part == 0 ? 192 : 128) + c, rr);
-          tmem_wait_ld();
-          if (k < T) {
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              uint4 w;
-              w.x = pk_bf16(__uint_as_float(rr[8 * u]) * sc, __uint_as_float(rr[8 * u + 1]) * sc);
-              w.y = pk_bf16(__uint_as_float(rr[8 * u + 2]) * sc, __uint_as_float(rr[8 * u + 3]) * sc);
-              w.z = pk_bf16(__uint_as_float(rr[8 * u + 4]) * sc, __uint_as_float(rr[8 * u + 5]) * sc);
-              w.w = pk_bf16(__uint_as_float(rr[8 * u + 6]) * sc, __uint_as_float(rr[8 * u + 7]) * sc);
-              *reinterpret_cast<uint4*>(dst + c + 8 * u) = w;
+          for (int e = 0; e < 8; ++e) {
+            float x = ex2_approx(fmaf(__uint_as_float(sr[c8 + e]), sl2, -lv[e]));
+            if (need_mask) {
+              const int qq = q0 + 64 * grp + c + e;
+              if (!(qq >= k && dsq[e] <= k)) x = 0.f;
             }
+            pv[e] = x;
+            gv[e] = x * (__uint_as_float(dr[c8 + e]) - dv[e]);
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            pw[c / 2 + e] = pk_bf16(pv[2 * e], pv[2 * e + 1]);
+            dw[c / 2 + e] = pk_bf16(gv[2 * e], gv[2 * e + 1]);
           }
         }
       }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 0) tc_dealloc(tmem, DkvSmem::TMEM_COLS);
-}
-
-// ============================================================== backward: dQ
-struct DqSmem {
-  static constexpr int Q = 0;                          // 16 KB: 128 queries
-  static constexpr int DO = Q + AT_TILE_BYTES;         // 16 KB
-  static constexpr int KV = DO + AT_TILE_BYTES;        // 2 stages x (K 8 KB, V 8 KB)
-  static constexpr int DS = KV + 4 * AT_HALF;          // 16 KB: 128 queries x 64 keys
-  static constexpr int BAR = DS + AT_TILE_BYTES;
-  static constexpr int TOTAL = BAR + 256;
-  static constexpr int TMEM_COLS = 256;                // S 0..63, dP 64..127, dQ 128..191
-};
-
-__global__ void __launch_bounds__(AT_THREADS, 2)
-attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
-               const __grid_constant__ CUtensorMap tmKV64, const float* __restrict__ lse,
-               const float* __restrict__ Dbuf, const int* __restrict__ dstart, bf16* __restrict__ dqkv, int T,
-               int H, unsigned* err) {
-  extern __shared__ __align__(1024) uint8_t at_raw[];
-  uint8_t* sm = (uint8_t*)(((uintptr_t)at_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t* bars = (uint64_t*)(sm + DqSmem::BAR);
-  // bars: 0 q_full, 1-2 kv_full, 3-4 kv_empty, 5 s_full, 6 s_free, 7 ds_full, 8 ds_free, 9 drain
-  uint32_t* tmem_slot = (uint32_t*)(bars + 10);
-  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
-  int* s_info = (int*)(tmem_slot + 2);
-  const uint32_t b0 = smem_u32(bars);
-  auto bar = [&](int i) { return b0 + 8u * i; };
-  const uint32_t sQ = smem_u32(sm + DqSmem::Q), sDO = smem_u32(sm + DqSmem::DO), sKV = smem_u32(sm + DqSmem::KV);
-  const uint32_t sDS = smem_u32(sm + DqSmem::DS);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nqb = (T + AT_BLK - 1) / AT_BLK;
-  const int qb = nqb - 1 - blockIdx.y;
-  const int bh = blockIdx.x, b = bh / H, h = bh % H;
-  const int C = H * AT_D;
-  const int q0 = qb * AT_BLK;
-  const long rowbase = (long)b * T;
-  const int* dsr = dstart + rowbase;
-
-  if (threadIdx.x == 0) {
-    mbar_init(bar(0), 1);
-    for (int i = 1; i <= 4; ++i) mbar_init(bar(i), 1);
-    mbar_init(bar(5), 1);
-    mbar_init(bar(6), 4);
-    mbar_init(bar(7), 4);
-    mbar_init(bar(8), 1);
-    mbar_init(bar(9), 1);
-    *abort_flag = 0;
-    const int kb_lo = dsr[q0] / AT_BK, kb_hi = min(q0 + AT_BLK - 1, T - 1) / AT_BK;
-    s_info[0] = kb_lo;
-    s_info[1] = kb_hi - kb_lo + 1;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  }
-  if (warp == 0) tc_alloc(smem_u32(tmem_slot), DqSmem::TMEM_COLS);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const int kb_lo = s_info[0], nj = s_info[1];
-
-  if (warp == 0 && lane == 0) {
-    mbar_expect_tx(bar(0), 2 * AT_TILE_BYTES);
-    tma_load_2d(sQ, &tmQ, bar(0), h * AT_D, (int)(rowbase + q0));
-    tma_load_2d(sDO, &tmDO, bar(0), h * AT_D, (int)(rowbase + q0));
-    bool ok = true;
-    for (int j = 0; j < nj && ok; ++j) {
-      const int st = j & 1;
-      if (!mbar_wait(bar(3 + st), ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-      mbar_expect_tx(bar(1 + st), 2 * AT_HALF);
-      const int k0 = (kb_lo + j) * AT_BK;
-      const uint32_t dst = sKV + st * 2 * AT_HALF;
-      tma_load_2d(dst, &tmKV64, bar(1 + st), C + h * AT_D, (int)(rowbase + k0));
-      tma_load_2d(dst + AT_HALF, &tmKV64, bar(1 + st), 2 * C + h * AT_D, (int)(rowbase + k0));
-    }
-    if (!ok) trap_timeout(abort_flag, err);
-    volatile int never = 0;
-    mbar_wait(bar(0), 0, &never, 1ll << 28);
-    for (int j = max(0, nj - 2); j < nj; ++j) mbar_wait(bar(1 + (j & 1)), (j >> 1) & 1, &never, 1ll << 28);
-  } else if (warp == 1 && lane == 0) {
-    constexpr uint32_t ID_S = instr_desc(64, false, false);   // S, dP: 128 queries x 64 keys, K = d
-    constexpr uint32_t ID_Q = instr_desc(64, false, true);    // dQ += dS K: 128 x 64, K = 64 keys (K MN-major)
-    bool ok = mbar_wait(bar(0), 0, abort_flag);
-    auto issue_s = [&](int j) -> bool {
-      const int st = j & 1;
-      if (!mbar_wait(bar(1 + st), (j >> 1) & 1, abort_flag)) return false;
-      if (!mbar_wait(bar(6), (j & 1) ^ 1, abort_flag)) return false;
-      tc_fence_after();
-      const uint32_t sK = sKV + st * 2 * AT_HALF, sV = sK + AT_HALF;
+      // the previous block's P^T / dS^T have been consumed and its dQ is complete
+      if (i > 0 && !wait_w(bar(8), (i - 1) & 1)) { ok = false; break; }
+      {
+        const uint32_t pb = sPT + grp * AT_TILE_BYTES + r * 128, db = sDST + grp * AT_TILE_BYTES + r * 128;
 #pragma unroll
-      for (int k = 0; k < AT_D / 16; ++k) {
-        umma_bf16(tmem + 0, kdesc(sQ + k * 32), kdesc(sK + k * 32), ID_S, k > 0);
-        umma_bf16(tmem + 64, kdesc(sDO + k * 32), kdesc(sV + k * 32), ID_S, k > 0);
-      }
-      umma_commit(bar(5));
-      return true;
-    };
-    if (ok && nj > 0) ok = issue_s(0);
-    for (int j = 0; j < nj && ok; ++j) {
-      const int st = j & 1;
-      if (j + 1 < nj && !issue_s(j + 1)) { ok = false; break; }
-      if (!mbar_wait(bar(7), j & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t sK = sKV + st * 2 * AT_HALF;
-#pragma unroll
-      for (int kk = 0; kk < AT_BK / 16; ++kk)
-        umma_bf16(tmem + 128, kdesc(sDS + kk * 32), mndesc(sK + kk * 2048, 8192), ID_Q, (j > 0 || kk > 0));
-      umma_commit(bar(8));
-      umma_commit(bar(3 + st));
-    }
-    if (!ok) trap_timeout(abort_flag, err);
-    umma_commit(bar(9));
-    volatile int never = 0;
-    mbar_wait(bar(9), 0, &never, 1ll << 28);
-  } else if (warp >= 2) {
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    const int q = q0 + r;
-    const bool qv = q < T;
-    const int ds_q = qv ? dsr[q] : 0;
-    const float Lq = qv ? lse[(long)bh * T + q] * LOG2E_F : 0.f;
-    const float Dv = qv ? Dbuf[(long)bh * T + q] : 0.f;
-    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const float sl2 = 0.125f * LOG2E_F;
-    bool ok = true;
-    for (int j = 0; j < nj; ++j) {
-      const int k0 = (kb_lo + j) * AT_BK;
-      if (!mbar_wait(bar(5), j & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sr[64], dr[64];
-      tmem_ld32(tmem + lane_off, sr);
-      tmem_ld32(tmem + lane_off + 32, sr + 32);
-      tmem_ld32(tmem + lane_off + 64, dr);
-      tmem_ld32(tmem + lane_off + 96, dr + 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(6));
-      if (j > 0 && !mbar_wait(bar(8), (j - 1) & 1, abort_flag)) { ok = false; break; }   // dS buffer free
-#pragma unroll
-      for (int c = 0; c < AT_BK; c += 32) {
-        float ds[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int kk = k0 + c + i;
-          const float p = (kk <= q && kk >= ds_q) ? exp2f(__uint_as_float(sr[c + i]) * sl2 - Lq) : 0.f;
-          ds[i] = p * (__uint_as_float(dr[c + i]) - Dv);
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t sw = (u ^ (r & 7)) << 4;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pb + sw), "r"(pw[4 * u]), "r"(pw[4 * u + 1]),
+                       "r"(pw[4 * u + 2]), "r"(pw[4 * u + 3])
+                       : "memory");
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(db + sw), "r"(dw[4 * u]), "r"(dw[4 * u + 1]),
+                       "r"(dw[4 * u + 2]), "r"(dw[4 * u + 3])
+                       : "memory");
         }
-        st_row32_64(sDS, r, c, ds);
       }
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(7));
+      if (i > 0) {
+        tc_fence_after();
+        if (!flush_dq(i - 1)) { ok = false; break; }
+      }
     }
-    if (!ok) trap_timeout(abort_flag, err);
-    if (ok && nj > 0 && mbar_wait(bar(8), (nj - 1) & 1, abort_flag)) {
+    // the last block's dQ, then dK and dV
+    if (ok && niter > 0 && wait_w(bar(8), (niter - 1) & 1)) {
       tc_fence_after();
-      bf16* dst = dqkv + (rowbase + q) * 3 * C + h * AT_D;
+      ok = flush_dq(niter - 1);
+      if (ok) {
+        bf16* row = dqkv + (rowbase + k) * 3 * C;
 #pragma unroll
-      for (int c = 0; c < AT_D; c += 32) {
-        uint32_t rr[32];
-        tmem_ld32(tmem + lane_off + 128 + c, rr);
-        tmem_wait_ld();
-        if (qv) {
+        for (int part = 0; part < 2; ++part) {
+          const float sc = part == 0 ? 0.125f : 1.f;
+          bf16* dst = row + (part == 0 ? C : 2 * C) + h * AT_D + 32 * grp;
+          uint32_t rr[32];
+          tmem_ld32(tmem + lane_off + (part == 0 ? 320 : 256) + 32 * grp, rr);
+          tmem_wait_ld();
+          if (k >= T) continue;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             uint4 w;
-            w.x = pk_bf16(__uint_as_float(rr[8 * u]) * 0.125f, __uint_as_float(rr[8 * u + 1]) * 0.125f);
-            w.y = pk_bf16(__uint_as_float(rr[8 * u + 2]) * 0.125f, __uint_as_float(rr[8 * u + 3]) * 0.125f);
-            w.z = pk_bf16(__uint_as_float(rr[8 * u + 4]) * 0.125f, __uint_as_float(rr[8 * u + 5]) * 0.125f);
-            w.w = pk_bf16(__uint_as_float(rr[8 * u + 6]) * 0.125f, __uint_as_float(rr[8 * u + 7]) * 0.125f);
-            *reinterpret_cast<uint4*>(dst + c + 8 * u) = w;
+            w.x = pk_bf16(__uint_as_float(rr[8 * u]) * sc, __uint_as_float(rr[8 * u + 1]) * sc);
+            w.y = pk_bf16(__uint_as_float(rr[8 * u + 2]) * sc, __uint_as_float(rr[8 * u + 3]) * sc);
+            w.z = pk_bf16(__uint_as_float(rr[8 * u + 4]) * sc, __uint_as_float(rr[8 * u + 5]) * sc);
+            w.w = pk_bf16(__uint_as_float(rr[8 * u + 6]) * sc, __uint_as_float(rr[8 * u + 7]) * sc);
+            *reinterpret_cast<uint4*>(dst + 8 * u) = w;
           }
         }
       }
+    } else if (niter > 0) {
+      ok = false;
     }
+    if (!ok) trap_timeout(abort_flag, err);
+    if (gtid == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tc_dealloc(tmem, DqSmem::TMEM_COLS);
+  if (warp == 0) tc_dealloc(tmem, BwdSmem::TMEM_COLS);
+}
+
+// dq[row, head h] = bf16(dQacc / 8); the accumulator is cleared for the next use.
+__global__ void attn_dq_finish_kernel(float* __restrict__ dq_acc, bf16* __restrict__ dqkv, long rows, int C) {
+  const long n8 = rows * C / 8;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n8; i += (long)gridDim.x * blockDim.x) {
+    const long e = i * 8, row = e / C;
+    const int c = (int)(e % C);
+    float4* src = reinterpret_cast<float4*>(dq_acc + e);
+    const float4 a = src[0], bq = src[1];
+    uint4 w;
+    w.x = pk_bf16(a.x * 0.125f, a.y * 0.125f);
+    w.y = pk_bf16(a.z * 0.125f, a.w * 0.125f);
+    w.z = pk_bf16(bq.x * 0.125f, bq.y * 0.125f);
+    w.w = pk_bf16(bq.z * 0.125f, bq.w * 0.125f);
+    *reinterpret_cast<uint4*>(dqkv + row * 3 * C + c) = w;
+    src[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    src[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 }
 
 // D[b, h, t] = dO[b*T+t, head h] . O[b*T+t, head h]   (one thread per (row, head))
@@ -768,20 +728,17 @@ cudaError_t launch_attn_fwd_tc(const bf16* qkv, bf16* out, float* lse, const int
 cudaError_t launch_attn_bwd_tc(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* Dbuf,
                                float* dq_acc, const int* dstart, bf16* dqkv, int B, int T, int H, unsigned* err,
                                cudaStream_t s) {
-  (void)dq_acc;
   const int C = H * AT_D;
   const long rows = (long)B * T;
-  CUtensorMap tq128, tq64, tdo128, tdo64;
-  if (!make_map_ex(&tq128, MapKey{qkv, rows, 3L * C, 3L * C, 1, 0, AT_D, AT_BLK, 0, 128}) ||
-      !make_map_ex(&tq64, MapKey{qkv, rows, 3L * C, 3L * C, 1, 0, AT_D, AT_BK, 0, 128}) ||
-      !make_map_ex(&tdo128, MapKey{dout, rows, (long)C, (long)C, 1, 0, AT_D, AT_BLK, 0, 128}) ||
-      !make_map_ex(&tdo64, MapKey{dout, rows, (long)C, (long)C, 1, 0, AT_D, AT_BK, 0, 128}))
+  CUtensorMap tqkv, tdo, tdq;
+  if (!make_map_ex(&tqkv, MapKey{qkv, rows, 3L * C, 3L * C, 1, 0, AT_D, AT_BLK, 0, 128}) ||
+      !make_map_ex(&tdo, MapKey{dout, rows, (long)C, (long)C, 1, 0, AT_D, BW_QB, 0, 128}) ||
+      !make_map_ex(&tdq, MapKey{dq_acc, rows, (long)C, (long)C, 1, 0, 32, BW_QB, 1, 128}))
     return cudaErrorInvalidValue;
-  const int smem_kv = DkvSmem::TOTAL + 1024, smem_q = DqSmem::TOTAL + 1024;
+  const int smem = BwdSmem::TOTAL + 1024;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = tc_smem_attr(attn_bwd_dkdv_tc, smem_kv);
-    if (e == cudaSuccess) e = tc_smem_attr(attn_bwd_dq_tc, smem_q);
+    cudaError_t e = tc_smem_attr(attn_bwd_tc, smem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
@@ -792,9 +749,9 @@ cudaError_t launch_attn_bwd_tc(const bf16* qkv, const bf16* out, const bf16* dou
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   dim3 grid(B * H, (T + AT_BLK - 1) / AT_BLK);
   ++g_kernel_launches;
-  attn_bwd_dkdv_tc<<<grid, AT_THREADS, smem_kv, s>>>(tq128, tq64, tdo64, lse, Dbuf, dstart, dqkv, T, H, err);
+  attn_bwd_tc<<<grid, BW_THREADS, smem, s>>>(tqkv, tdo, tdq, lse, Dbuf, dstart, dqkv, T, H, err);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   ++g_kernel_launches;
-  attn_bwd_dq_tc<<<grid, AT_THREADS, smem_q, s>>>(tq128, tdo128, tq64, lse, Dbuf, dstart, dqkv, T, H, err);
+  attn_dq_finish_kernel<<<148 * 8, 256, 0, s>>>(dq_acc, dqkv, rows, C);
   return cudaGetLastError();
 }
