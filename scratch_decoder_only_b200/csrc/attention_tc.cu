@@ -308,7 +308,8 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 // One CTA per 128-key block: it walks the 128-query blocks that can see its
 // keys and, per block,
 //   S^T = K Q^T, dP^T = V dO^T                  (TMEM, 128 x 128 each)
-//   P^T = exp2(S^T log2e / 8 - lse log2e),  dS^T = P^T (dP^T - D)    (smem)
+//   P^T = exp2(S^T log2e / 8 - lse log2e)       (bf16, back into TMEM)
+//   dS^T = P^T (dP^T - D)                       (bf16, shared memory)
 //   dV += P^T dO,  dK += dS^T Q                  (TMEM, across query blocks)
 //   dQ_blk = dS K                                (TMEM; added in fp32 to a
 //                                                 global accumulator by a TMA
@@ -319,18 +320,19 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 // score tiles and d columns 32g..32g+31 of the dQ, dK, dV accumulators.
 #define BW_THREADS 320
 #define BW_QB 128                                    // queries per iterated block
+#define BW_ST 3                                      // Q / dO pipeline stages
 struct BwdSmem {
   static constexpr int K = 0;                        // 16 KB: 128 keys x 64
   static constexpr int V = K + AT_TILE_BYTES;        // 16 KB
-  static constexpr int Q = V + AT_TILE_BYTES;        // 2 stages x 16 KB
-  static constexpr int DO = Q + 2 * AT_TILE_BYTES;   // 2 stages x 16 KB
-  static constexpr int PT = DO + 2 * AT_TILE_BYTES;  // 32 KB: [128 keys][128 queries] as two 64-query blocks
-  static constexpr int DST = PT + 2 * AT_TILE_BYTES; // 32 KB, same layout
-  static constexpr int DQS = DST + 2 * AT_TILE_BYTES;// 2 groups x 16 KB: [128 queries][32 fp32]
-  static constexpr int AUX = DQS + 2 * AT_TILE_BYTES;// 2 stages x (lse2, D, dstart) x 128
-  static constexpr int BAR = AUX + 2 * 3 * BW_QB * 4;
+  static constexpr int Q = V + AT_TILE_BYTES;        // BW_ST stages x 16 KB
+  static constexpr int DO = Q + BW_ST * AT_TILE_BYTES;
+  static constexpr int DST = DO + BW_ST * AT_TILE_BYTES;   // 32 KB: [128 keys][128 queries] as two 64-query blocks
+  static constexpr int DQS = DST + 2 * AT_TILE_BYTES;      // 2 groups x 16 KB: [128 queries][32 fp32]
+  static constexpr int AUX = DQS + 2 * AT_TILE_BYTES;      // BW_ST stages x (lse2, D, dstart) x 128
+  static constexpr int BAR = AUX + BW_ST * 3 * BW_QB * 4;
   static constexpr int TOTAL = BAR + 256;
-  static constexpr int TMEM_COLS = 512;              // S^T 0, dP^T 128, dV 256, dK 320, dQ 384
+  // TMEM columns: S^T 0, dP^T 128, dV 256, dK 320, dQ 384, P^T (bf16 pairs) 448
+  static constexpr int TMEM_COLS = 512;
 };
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -338,6 +340,60 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// D[tmem] (+)= A[tmem] * B[smem]: A is read from tensor memory (128 lanes x 16 bf16).
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t acc) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 32 columns of P^T and dS^T for one key row: p = exp2(s sl2 - lse2), ds = p (dp - D),
+// packed into bf16 pairs.  MASK applies causality and document starts.
+template <bool MASK>
+__device__ __forceinline__ void bwd_elementwise32(const uint32_t* sr, const uint32_t* dr, const float* L2,
+                                                  const float* Dq, const int* DSq, int q_first, int k, float sl2,
+                                                  uint32_t* pw, uint32_t* dw) {
+#pragma unroll
+  for (int c8 = 0; c8 < 32; c8 += 8) {
+    const float4 la = *reinterpret_cast<const float4*>(L2 + c8), lb = *reinterpret_cast<const float4*>(L2 + c8 + 4);
+    const float4 da = *reinterpret_cast<const float4*>(Dq + c8), db = *reinterpret_cast<const float4*>(Dq + c8 + 4);
+    const float lv[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
+    const float dv[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+    int dsq[8];
+    if (MASK) {
+      const int4 sa = *reinterpret_cast<const int4*>(DSq + c8), sb = *reinterpret_cast<const int4*>(DSq + c8 + 4);
+      dsq[0] = sa.x; dsq[1] = sa.y; dsq[2] = sa.z; dsq[3] = sa.w;
+      dsq[4] = sb.x; dsq[5] = sb.y; dsq[6] = sb.z; dsq[7] = sb.w;
+    }
+    float pv[8], gv[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float x = ex2_approx(fmaf(__uint_as_float(sr[c8 + e]), sl2, -lv[e]));
+      if (MASK && !(q_first + c8 + e >= k && dsq[e] <= k)) x = 0.f;
+      pv[e] = x;
+      gv[e] = x * (__uint_as_float(dr[c8 + e]) - dv[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      pw[c8 / 2 + e] = pk_bf16(pv[2 * e], pv[2 * e + 1]);
+      dw[c8 / 2 + e] = pk_bf16(gv[2 * e], gv[2 * e + 1]);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(BW_THREADS, 1)
 attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
             const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ lse, const float* __restrict__ Dbuf,
@@ -345,17 +401,19 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
   extern __shared__ __align__(1024) uint8_t at_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)at_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = (uint64_t*)(sm + BwdSmem::BAR);
-  // bars: 0 kv_full, 1-2 q_full (TMA tiles + per-query values), 3-4 q_empty, 5 s_full, 6 s_free,
-  //       7 p_full, 8 mma_done (P^T / dS^T read, dQ_blk complete), 9 dq_free, 10 drain,
-  //       11-12 group barriers
-  uint32_t* tmem_slot = (uint32_t*)(bars + 13);
+  // bars: 0 kv_full, 1-3 q_full (TMA tiles + per-query values), 4-6 q_empty, 7 s_full, 8 s_free,
+  //       9 p_full, 10 mma_done (P^T / dS^T read, dQ_blk complete), 11 dq_free, 12 drain,
+  //       13-14 staging written (per group, 128 arrivals), 15-16 staging free (per group)
+  uint32_t* tmem_slot = (uint32_t*)(bars + 17);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   int* s_info = (int*)(tmem_slot + 2);
   const uint32_t b0 = smem_u32(bars);
   auto bar = [&](int i) { return b0 + 8u * i; };
+  enum { KV_FULL = 0, Q_FULL = 1, Q_EMPTY = 4, S_FULL = 7, S_FREE = 8, P_FULL = 9, MMA_DONE = 10, DQ_FREE = 11,
+         DRAIN = 12, ST_FULL = 13, ST_FREE = 15 };
   const uint32_t sK = smem_u32(sm + BwdSmem::K), sV = smem_u32(sm + BwdSmem::V);
   const uint32_t sQ = smem_u32(sm + BwdSmem::Q), sDO = smem_u32(sm + BwdSmem::DO);
-  const uint32_t sPT = smem_u32(sm + BwdSmem::PT), sDST = smem_u32(sm + BwdSmem::DST);
+  const uint32_t sDST = smem_u32(sm + BwdSmem::DST);
   const uint32_t sDQ = smem_u32(sm + BwdSmem::DQS);
   float* aux = (float*)(sm + BwdSmem::AUX);
 
@@ -370,17 +428,21 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
   const int qb_lo = k0 / BW_QB;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(0), 1);
-    for (int i = 1; i <= 2; ++i) mbar_init(bar(i), 1 + 32);   // TMA arrival + 32 lanes of per-query values
-    for (int i = 3; i <= 4; ++i) mbar_init(bar(i), 1);
-    mbar_init(bar(5), 1);
-    mbar_init(bar(6), 8);
-    mbar_init(bar(7), 8);
-    mbar_init(bar(8), 1);
-    mbar_init(bar(9), 8);
-    mbar_init(bar(10), 1);
-    mbar_init(bar(11), 128);
-    mbar_init(bar(12), 128);
+    mbar_init(bar(KV_FULL), 1);
+    for (int i = 0; i < BW_ST; ++i) {
+      mbar_init(bar(Q_FULL + i), 1 + 32);   // TMA arrival + 32 lanes of per-query values
+      mbar_init(bar(Q_EMPTY + i), 1);
+    }
+    mbar_init(bar(S_FULL), 1);
+    mbar_init(bar(S_FREE), 8);
+    mbar_init(bar(P_FULL), 8);
+    mbar_init(bar(MMA_DONE), 1);
+    mbar_init(bar(DQ_FREE), 8);
+    mbar_init(bar(DRAIN), 1);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(bar(ST_FULL + g), 128);
+      mbar_init(bar(ST_FREE + g), 1);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -411,13 +473,14 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQKV)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmDO)) : "memory");
-      mbar_expect_tx(bar(0), 2 * AT_TILE_BYTES);
-      tma_load_2d(sK, &tmQKV, bar(0), C + h * AT_D, (int)(rowbase + k0));
-      tma_load_2d(sV, &tmQKV, bar(0), 2 * C + h * AT_D, (int)(rowbase + k0));
+      mbar_expect_tx(bar(KV_FULL), 2 * AT_TILE_BYTES);
+      tma_load_2d(sK, &tmQKV, bar(KV_FULL), C + h * AT_D, (int)(rowbase + k0));
+      tma_load_2d(sV, &tmQKV, bar(KV_FULL), 2 * C + h * AT_D, (int)(rowbase + k0));
     }
     bool ok = true;
     for (int i = 0; i < niter; ++i) {
-      const int st = i & 1;
+      const int st = i % BW_ST;
+      const uint32_t ph = (i / BW_ST) & 1;
       const int q0 = (qb_lo + i) * BW_QB;
       // per-query values into registers before the stage is free
       float l2v[4], dv[4];
@@ -430,11 +493,11 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
         dv[e] = v ? Dbuf[(long)bh * T + qq] : 0.f;
         dsv[e] = v ? dsr[qq] : 0x7fffffff;
       }
-      if (!mbar_wait(bar(3 + st), ((i >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(bar(Q_EMPTY + st), ph ^ 1, abort_flag)) { ok = false; break; }
       if (lane == 0) {
-        mbar_expect_tx(bar(1 + st), 2 * AT_TILE_BYTES);
-        tma_load_2d(sQ + st * AT_TILE_BYTES, &tmQKV, bar(1 + st), h * AT_D, (int)(rowbase + q0));
-        tma_load_2d(sDO + st * AT_TILE_BYTES, &tmDO, bar(1 + st), h * AT_D, (int)(rowbase + q0));
+        mbar_expect_tx(bar(Q_FULL + st), 2 * AT_TILE_BYTES);
+        tma_load_2d(sQ + st * AT_TILE_BYTES, &tmQKV, bar(Q_FULL + st), h * AT_D, (int)(rowbase + q0));
+        tma_load_2d(sDO + st * AT_TILE_BYTES, &tmDO, bar(Q_FULL + st), h * AT_D, (int)(rowbase + q0));
       }
       float* L2 = aux + st * 3 * BW_QB;
       float* Dq = L2 + BW_QB;
@@ -445,24 +508,25 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
         Dq[lane + 32 * e] = dv[e];
         DSq[lane + 32 * e] = dsv[e];
       }
-      mbar_arrive(bar(1 + st));   // release: the values above are visible to whoever waits on q_full
+      mbar_arrive(bar(Q_FULL + st));   // release: the values above are visible to whoever waits on q_full
     }
     if (!ok && lane == 0) trap_timeout(abort_flag, err);
     if (lane == 0) {
       volatile int never = 0;
-      mbar_wait(bar(0), 0, &never, 1ll << 28);
-      for (int i = max(0, niter - 2); i < niter; ++i) mbar_wait(bar(1 + (i & 1)), (i >> 1) & 1, &never, 1ll << 28);
+      mbar_wait(bar(KV_FULL), 0, &never, 1ll << 28);
+      for (int i = max(0, niter - BW_ST); i < niter; ++i)
+        mbar_wait(bar(Q_FULL + i % BW_ST), (i / BW_ST) & 1, &never, 1ll << 28);
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
     constexpr uint32_t ID_SS = instr_desc(128, false, false);   // S^T, dP^T: 128 keys x 128 queries, K = d
     constexpr uint32_t ID_KV = instr_desc(64, false, true);     // dV, dK: 128 keys x 64, K = 128 queries
     constexpr uint32_t ID_DQ = instr_desc(64, true, true);      // dQ: 128 queries x 64, K = 128 keys
-    bool ok = mbar_wait(bar(0), 0, abort_flag);
+    bool ok = mbar_wait(bar(KV_FULL), 0, abort_flag);
     auto issue_s = [&](int i) -> bool {   // S^T and dP^T of query block i
-      const int st = i & 1;
-      if (!mbar_wait(bar(1 + st), (i >> 1) & 1, abort_flag)) return false;
-      if (!mbar_wait(bar(6), (i & 1) ^ 1, abort_flag)) return false;   // previous S^T / dP^T read
+      const int st = i % BW_ST;
+      if (!mbar_wait(bar(Q_FULL + st), (i / BW_ST) & 1, abort_flag)) return false;
+      if (!mbar_wait(bar(S_FREE), (i & 1) ^ 1, abort_flag)) return false;   // previous S^T / dP^T read
       tc_fence_after();
       const uint32_t q = sQ + st * AT_TILE_BYTES, o = sDO + st * AT_TILE_BYTES;
 #pragma unroll
@@ -470,35 +534,35 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
         umma_bf16(tmem + 0, kdesc(sK + k * 32), kdesc(q + k * 32), ID_SS, k > 0);
         umma_bf16(tmem + 128, kdesc(sV + k * 32), kdesc(o + k * 32), ID_SS, k > 0);
       }
-      umma_commit(bar(5));
+      umma_commit(bar(S_FULL));
       return true;
     };
     if (ok && niter > 0) ok = issue_s(0);
     for (int i = 0; i < niter && ok; ++i) {
-      const int st = i & 1;
+      const int st = i % BW_ST;
       if (i + 1 < niter && !issue_s(i + 1)) { ok = false; break; }
-      if (!mbar_wait(bar(7), i & 1, abort_flag)) { ok = false; break; }   // P^T, dS^T written
+      if (!mbar_wait(bar(P_FULL), i & 1, abort_flag)) { ok = false; break; }   // P^T, dS^T written
       tc_fence_after();
       const uint32_t q = sQ + st * AT_TILE_BYTES, o = sDO + st * AT_TILE_BYTES;
 #pragma unroll
       for (int kk = 0; kk < BW_QB / 16; ++kk) {
         const uint32_t off = (kk >> 2) * AT_TILE_BYTES + (kk & 3) * 32;
-        umma_bf16(tmem + 256, kdesc(sPT + off), mndesc(o + kk * 2048, 8192), ID_KV, (i > 0 || kk > 0));
+        umma_bf16_ts(tmem + 256, tmem + 448 + 8 * kk, mndesc(o + kk * 2048, 8192), ID_KV, (i > 0 || kk > 0));
         umma_bf16(tmem + 320, kdesc(sDST + off), mndesc(q + kk * 2048, 8192), ID_KV, (i > 0 || kk > 0));
       }
-      umma_commit(bar(3 + st));   // Q / dO stage free
+      umma_commit(bar(Q_EMPTY + st));   // Q / dO stage free
       // dQ_blk = dS K once the previous block's dQ has been read out
-      if (i > 0 && !mbar_wait(bar(9), (i - 1) & 1, abort_flag)) { ok = false; break; }
+      if (i > 0 && !mbar_wait(bar(DQ_FREE), (i - 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < AT_BLK / 16; ++kk)
         umma_bf16(tmem + 384, mndesc(sDST + kk * 2048, AT_TILE_BYTES), mndesc(sK + kk * 2048, 8192), ID_DQ, kk > 0);
-      umma_commit(bar(8));
+      umma_commit(bar(MMA_DONE));
     }
     if (!ok) trap_timeout(abort_flag, err);
-    umma_commit(bar(10));
+    umma_commit(bar(DRAIN));
     volatile int never = 0;
-    mbar_wait(bar(10), 0, &never, 1ll << 28);
+    mbar_wait(bar(DRAIN), 0, &never, 1ll << 28);
   } else if (warp >= 2) {
     // ---------------- elementwise warps: thread owns key row r (and query row r of dQ)
     const int quarter = warp & 3;
@@ -508,23 +572,23 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
     const int gtid = threadIdx.x - 64 - 128 * grp;   // 0..127 inside the group
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = 0.125f * LOG2E_F;
-    const uint32_t gbar = bar(11 + grp);
+    const uint32_t st_full = bar(ST_FULL + grp), st_free = bar(ST_FREE + grp);
     const uint32_t sDQg = sDQ + grp * AT_TILE_BYTES;
-    uint32_t gph = 0;
     bool ok = true;
-    // waits are voted warp-wide so that the .sync.aligned TMEM loads after them
-    // are never reached by part of a warp
+    // waits are voted warp-wide so that the .sync.aligned TMEM accesses after
+    // them are never reached by part of a warp
     auto wait_w = [&](uint32_t bb, uint32_t parity) { return __all_sync(0xffffffffu, mbar_wait(bb, parity, abort_flag)); };
     // dQ of block j: TMEM -> fp32 staging (128-byte swizzle) -> bulk reduce-add
+    // issued by the group's first thread once all 128 rows are written
     auto flush_dq = [&](int j) -> bool {
       uint32_t rr[32];
       tmem_ld32(tmem + lane_off + 384 + 32 * grp, rr);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(9));   // the dQ accumulator may be overwritten
-      if (gtid == 0) bulk_wait_read<0>();   // the previous reduce has read the staging
-      if (!__all_sync(0xffffffffu, group_sync(gbar, gph, abort_flag))) return false;
+      if (lane == 0) mbar_arrive(bar(DQ_FREE));   // the dQ accumulator may be overwritten
+      // the reduce of block j-1 has read the staging (signalled by the first thread)
+      if (j > 0 && !wait_w(st_free, (j - 1) & 1)) return false;
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const uint32_t a = sDQg + r * 128 + ((u ^ (r & 7)) << 4);
@@ -533,28 +597,34 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
                      : "memory");
       }
       fence_async_smem();
-      if (!__all_sync(0xffffffffu, group_sync(gbar, gph, abort_flag))) return false;
+      mbar_arrive(st_full);
       if (gtid == 0) {
+        if (!mbar_wait(st_full, j & 1, abort_flag)) return false;
         tma_reduce_add_2d(&tmDQ, sDQg, h * AT_D + 32 * grp, (int)(rowbase + (qb_lo + j) * BW_QB));
         bulk_commit();
       }
       return true;
     };
+    // first thread: once the reduce of the previous flush has read the staging, free it
+    auto release_staging = [&]() {
+      if (gtid == 0) {
+        bulk_wait_read<0>();
+        mbar_arrive(st_free);
+      }
+    };
     for (int i = 0; i < niter; ++i) {
       const int q0 = (qb_lo + i) * BW_QB;
-      const int st = i & 1;
-      const float4* aL2 = reinterpret_cast<const float4*>(aux + st * 3 * BW_QB + grp * 64);
-      const float4* aD = aL2 + BW_QB / 4;
-      const int4* aDS = reinterpret_cast<const int4*>(aL2 + BW_QB / 2);
-      if (!wait_w(bar(1 + st), (i >> 1) & 1)) { ok = false; break; }   // per-query values
-      if (!wait_w(bar(5), i & 1)) { ok = false; break; }
+      const int st = i % BW_ST;
+      if (i >= 2) release_staging();   // reduce of block i-2, before the flush of block i-1
+      const float* L2 = aux + st * 3 * BW_QB + 64 * grp;
+      const float* Dq = L2 + BW_QB;
+      const int* DSq = reinterpret_cast<const int*>(L2 + 2 * BW_QB);
+      if (!wait_w(bar(Q_FULL + st), (i / BW_ST) & 1)) { ok = false; break; }   // per-query values
+      if (!wait_w(bar(S_FULL), i & 1)) { ok = false; break; }
       tc_fence_after();
       // masking only where a key can be later than a query or before its document
       // (document starts never decrease, queries past T carry INT_MAX)
-      const int ds_last = reinterpret_cast<const int*>(aux)[st * 3 * BW_QB + 2 * BW_QB + BW_QB - 1];
-      const bool need_mask = q0 < k0 + AT_BLK || ds_last > k0;
-      // P^T and dS^T as packed bf16 pairs, 32 columns at a time (64 score
-      // registers live); the score buffers are released after the second load
+      const bool need_mask = q0 < k0 + AT_BLK || DSq[BW_QB - 1 - 64 * grp] > k0;
       uint32_t pw[32], dw[32];
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
@@ -565,67 +635,44 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
         if (half == 1) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(6));   // S^T / dP^T may be overwritten
+          if (lane == 0) mbar_arrive(bar(S_FREE));   // S^T / dP^T may be overwritten
         }
-#pragma unroll
-        for (int c8 = 0; c8 < 32; c8 += 8) {
-          const int c = 32 * half + c8;
-          float lv[8], dv[8];
-          int dsq[8];
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const float4 l4 = aL2[c / 4 + hh];
-            const float4 d4 = aD[c / 4 + hh];
-            lv[4 * hh] = l4.x; lv[4 * hh + 1] = l4.y; lv[4 * hh + 2] = l4.z; lv[4 * hh + 3] = l4.w;
-            dv[4 * hh] = d4.x; dv[4 * hh + 1] = d4.y; dv[4 * hh + 2] = d4.z; dv[4 * hh + 3] = d4.w;
-            int4 s4 = make_int4(0, 0, 0, 0);
-            if (need_mask) s4 = aDS[c / 4 + hh];
-            dsq[4 * hh] = s4.x; dsq[4 * hh + 1] = s4.y; dsq[4 * hh + 2] = s4.z; dsq[4 * hh + 3] = s4.w;
-          }
-          float pv[8], gv[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            float x = ex2_approx(fmaf(__uint_as_float(sr[c8 + e]), sl2, -lv[e]));
-            if (need_mask) {
-              const int qq = q0 + 64 * grp + c + e;
-              if (!(qq >= k && dsq[e] <= k)) x = 0.f;
-            }
-            pv[e] = x;
-            gv[e] = x * (__uint_as_float(dr[c8 + e]) - dv[e]);
-          }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            pw[c / 2 + e] = pk_bf16(pv[2 * e], pv[2 * e + 1]);
-            dw[c / 2 + e] = pk_bf16(gv[2 * e], gv[2 * e + 1]);
-          }
-        }
+        const int qf = q0 + 64 * grp + 32 * half;
+        if (need_mask)
+          bwd_elementwise32<true>(sr, dr, L2 + 32 * half, Dq + 32 * half, DSq + 32 * half, qf, k, sl2, pw + 16 * half,
+                                  dw + 16 * half);
+        else
+          bwd_elementwise32<false>(sr, dr, L2 + 32 * half, Dq + 32 * half, DSq + 32 * half, qf, k, sl2,
+                                   pw + 16 * half, dw + 16 * half);
       }
       // the previous block's P^T / dS^T have been consumed and its dQ is complete
-      if (i > 0 && !wait_w(bar(8), (i - 1) & 1)) { ok = false; break; }
+      if (i > 0 && !wait_w(bar(MMA_DONE), (i - 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      tmem_st32(tmem + lane_off + 448 + 32 * grp, pw);
       {
-        const uint32_t pb = sPT + grp * AT_TILE_BYTES + r * 128, db = sDST + grp * AT_TILE_BYTES + r * 128;
+        const uint32_t db = sDST + grp * AT_TILE_BYTES + r * 128;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const uint32_t sw = (u ^ (r & 7)) << 4;
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pb + sw), "r"(pw[4 * u]), "r"(pw[4 * u + 1]),
-                       "r"(pw[4 * u + 2]), "r"(pw[4 * u + 3])
-                       : "memory");
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(db + sw), "r"(dw[4 * u]), "r"(dw[4 * u + 1]),
                        "r"(dw[4 * u + 2]), "r"(dw[4 * u + 3])
                        : "memory");
         }
       }
+      tmem_wait_st();
       fence_async_smem();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(7));
+      if (lane == 0) mbar_arrive(bar(P_FULL));
       if (i > 0) {
         tc_fence_after();
         if (!flush_dq(i - 1)) { ok = false; break; }
       }
     }
     // the last block's dQ, then dK and dV
-    if (ok && niter > 0 && wait_w(bar(8), (niter - 1) & 1)) {
+    if (ok && niter > 0 && wait_w(bar(MMA_DONE), (niter - 1) & 1)) {
       tc_fence_after();
+      if (niter >= 2) release_staging();
       ok = flush_dq(niter - 1);
       if (ok) {
         bf16* row = dqkv + (rowbase + k) * 3 * C;
