@@ -95,246 +95,11 @@ __device__ __forceinline__ void tc_dealloc(uint32_t tmem, int cols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(cols));
 }
 
-// ============================================================== forward
-struct FwdSmem {
-  static constexpr int Q = 0;                          // 16 KB: 128 queries
-  static constexpr int KV = Q + AT_TILE_BYTES;         // 2 stages x (K 8 KB, V 8 KB)
-  static constexpr int P = KV + 4 * AT_HALF;           // 2 x 16 KB: 128 queries x 64 keys
-  static constexpr int BAR = P + 2 * AT_TILE_BYTES;
-  static constexpr int TOTAL = BAR + 256;
-  static constexpr int TMEM_COLS = 256;                // S 0..63, O[0] 64..127, O[1] 128..191
-};
-
-__global__ void __launch_bounds__(AT_THREADS, 2)
-attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV64,
-            bf16* __restrict__ out, float* __restrict__ lse, const int* __restrict__ dstart, int T, int H,
-            unsigned* err) {
-  extern __shared__ __align__(1024) uint8_t at_raw[];
-  uint8_t* sm = (uint8_t*)(((uintptr_t)at_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t* bars = (uint64_t*)(sm + FwdSmem::BAR);
-  // bars: 0 q_full, 1-2 kv_full, 3-4 kv_empty, 5 s_full, 6 s_free, 7-8 p_full, 9-10 o_full, 11-12 o_free,
-  //       13 drain
-  uint32_t* tmem_slot = (uint32_t*)(bars + 14);
-  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
-  int* s_info = (int*)(tmem_slot + 2);
-  const uint32_t b0 = smem_u32(bars);
-  auto bar = [&](int i) { return b0 + 8u * i; };
-  const uint32_t sQ = smem_u32(sm + FwdSmem::Q), sKV = smem_u32(sm + FwdSmem::KV), sP = smem_u32(sm + FwdSmem::P);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nqb = (T + AT_BLK - 1) / AT_BLK;
-  const int qb = nqb - 1 - blockIdx.y;   // heaviest query blocks first (y is the slow grid index)
-  const int bh = blockIdx.x, b = bh / H, h = bh % H;
-  const int C = H * AT_D;
-  const int q0 = qb * AT_BLK;
-  const long rowbase = (long)b * T;
-  const int* dsr = dstart + rowbase;
-
-  if (threadIdx.x == 0) {
-    mbar_init(bar(0), 1);
-    for (int i = 1; i <= 4; ++i) mbar_init(bar(i), 1);
-    mbar_init(bar(5), 1);
-    mbar_init(bar(6), 4);
-    mbar_init(bar(7), 4);
-    mbar_init(bar(8), 4);
-    mbar_init(bar(9), 1);
-    mbar_init(bar(10), 1);
-    mbar_init(bar(11), 4);
-    mbar_init(bar(12), 4);
-    mbar_init(bar(13), 1);
-    *abort_flag = 0;
-    const int kb_lo = dsr[q0] / AT_BK, kb_hi = min(q0 + AT_BLK - 1, T - 1) / AT_BK;
-    s_info[0] = kb_lo;
-    s_info[1] = kb_hi - kb_lo + 1;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  }
-  if (warp == 0) tc_alloc(smem_u32(tmem_slot), FwdSmem::TMEM_COLS);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const int kb_lo = s_info[0], nj = s_info[1];
-
-  if (warp == 0 && lane == 0) {
-    // ---------------- producer
-    mbar_expect_tx(bar(0), AT_TILE_BYTES);
-    tma_load_2d(sQ, &tmQ, bar(0), h * AT_D, (int)(rowbase + q0));
-    bool ok = true;
-    for (int j = 0; j < nj && ok; ++j) {
-      const int st = j & 1;
-      if (!mbar_wait(bar(3 + st), ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-      mbar_expect_tx(bar(1 + st), 2 * AT_HALF);
-      const int k0 = (kb_lo + j) * AT_BK;
-      const uint32_t dst = sKV + st * 2 * AT_HALF;
-      tma_load_2d(dst, &tmKV64, bar(1 + st), C + h * AT_D, (int)(rowbase + k0));
-      tma_load_2d(dst + AT_HALF, &tmKV64, bar(1 + st), 2 * C + h * AT_D, (int)(rowbase + k0));
-    }
-    if (!ok) trap_timeout(abort_flag, err);
-    volatile int never = 0;
-    mbar_wait(bar(0), 0, &never, 1ll << 28);
-    for (int j = max(0, nj - 2); j < nj; ++j) mbar_wait(bar(1 + (j & 1)), (j >> 1) & 1, &never, 1ll << 28);
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer: S(j+1) is issued before P V of block j
-    constexpr uint32_t ID_S = instr_desc(64, false, false);   // S = Q K^T: 128 x 64, K = 64
-    constexpr uint32_t ID_O = instr_desc(64, false, true);    // O = P V: 128 x 64, K = 64 keys (V MN-major)
-    bool ok = mbar_wait(bar(0), 0, abort_flag);
-    auto issue_s = [&](int j) -> bool {
-      const int st = j & 1;
-      if (!mbar_wait(bar(1 + st), (j >> 1) & 1, abort_flag)) return false;
-      if (!mbar_wait(bar(6), (j & 1) ^ 1, abort_flag)) return false;   // previous S read
-      tc_fence_after();
-      const uint32_t sK = sKV + st * 2 * AT_HALF;
-#pragma unroll
-      for (int k = 0; k < AT_D / 16; ++k) umma_bf16(tmem + 0, kdesc(sQ + k * 32), kdesc(sK + k * 32), ID_S, k > 0);
-      umma_commit(bar(5));
-      return true;
-    };
-    if (ok && nj > 0) ok = issue_s(0);
-    for (int j = 0; j < nj && ok; ++j) {
-      const int st = j & 1;
-      if (j + 1 < nj && !issue_s(j + 1)) { ok = false; break; }
-      if (!mbar_wait(bar(7 + st), (j >> 1) & 1, abort_flag)) { ok = false; break; }         // P(j) written
-      if (!mbar_wait(bar(11 + st), ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }  // O buffer read
-      tc_fence_after();
-      const uint32_t sV = sKV + st * 2 * AT_HALF + AT_HALF, sPj = sP + st * AT_TILE_BYTES;
-#pragma unroll
-      for (int kk = 0; kk < AT_BK / 16; ++kk)
-        umma_bf16(tmem + 64 + st * 64, kdesc(sPj + kk * 32), mndesc(sV + kk * 2048, 8192), ID_O, kk > 0);
-      umma_commit(bar(9 + st));
-      umma_commit(bar(3 + st));
-    }
-    if (!ok) trap_timeout(abort_flag, err);
-    umma_commit(bar(13));
-    volatile int never = 0;
-    mbar_wait(bar(13), 0, &never, 1ll << 28);
-  } else if (warp >= 2) {
-    // ---------------- softmax warps: thread owns query row r.  O of block j is
-    // accumulated during block j+1, so no wait follows the P V it enables.
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    const int q = q0 + r;
-    const bool qv = q < T;
-    const int ds_q = qv ? dsr[q] : 0;
-    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const float sl2 = 0.125f * LOG2E_F;   // 1/sqrt(64) in the exp2 domain
-    float m = -INFINITY, l = 0.f, c_pend = 0.f;
-    float o[AT_D];
-#pragma unroll
-    for (int i = 0; i < AT_D; ++i) o[i] = 0.f;
-    bool ok = true;
-    auto accumulate = [&](int jj) -> bool {   // o = o * c(jj) + O(jj)
-      const int sb = jj & 1;
-      if (!mbar_wait(bar(9 + sb), (jj >> 1) & 1, abort_flag)) return false;
-      tc_fence_after();
-      uint32_t orr[64];
-      tmem_ld32(tmem + lane_off + 64 + sb * 64, orr);
-      tmem_ld32(tmem + lane_off + 96 + sb * 64, orr + 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(11 + sb));
-#pragma unroll
-      for (int i = 0; i < 64; ++i) o[i] = o[i] * c_pend + __uint_as_float(orr[i]);
-      return true;
-    };
-    for (int j = 0; j < nj; ++j) {
-      const int k0 = (kb_lo + j) * AT_BK;
-      if (!mbar_wait(bar(5), j & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld32(tmem + lane_off, sr);
-      tmem_ld32(tmem + lane_off + 32, sr + 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(6));   // S may be overwritten
-      float mx = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const int k = k0 + i;
-        const float v = (k <= q && k >= ds_q) ? __uint_as_float(sr[i]) * sl2 : -INFINITY;
-        sr[i] = __float_as_uint(v);
-        mx = fmaxf(mx, v);
-      }
-      const float mn = fmaxf(m, mx);
-      const float mu = mn == -INFINITY ? 0.f : mn;
-      const float cj = exp2f(m - mu);
-      float ps = 0.f;
-      // P buffer j&1 was read by P V of block j-2, whose result was accumulated in block j-1
-      const uint32_t sPj = sP + (j & 1) * AT_TILE_BYTES;
-#pragma unroll
-      for (int c = 0; c < 64; c += 32) {
-        float p[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          p[i] = exp2f(__uint_as_float(sr[c + i]) - mu);
-          ps += p[i];
-        }
-        st_row32_64(sPj, r, c, p);
-      }
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(7 + (j & 1)));   // P(j) ready
-      l = l * cj + ps;
-      m = mn;
-      if (j > 0 && !accumulate(j - 1)) { ok = false; break; }
-      c_pend = cj;
-    }
-    if (ok && nj > 0) ok = accumulate(nj - 1);
-    if (!ok) trap_timeout(abort_flag, err);
-    if (qv) {
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      bf16* orow = out + (rowbase + q) * C + h * AT_D;
-#pragma unroll
-      for (int c = 0; c < AT_D; c += 8) {
-        uint4 w;
-        w.x = pk_bf16(o[c] * inv, o[c + 1] * inv);
-        w.y = pk_bf16(o[c + 2] * inv, o[c + 3] * inv);
-        w.z = pk_bf16(o[c + 4] * inv, o[c + 5] * inv);
-        w.w = pk_bf16(o[c + 6] * inv, o[c + 7] * inv);
-        *reinterpret_cast<uint4*>(orow + c) = w;
-      }
-      lse[(long)bh * T + q] = (m + log2f(l)) * LN2_F;
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 0) tc_dealloc(tmem, FwdSmem::TMEM_COLS);
+__device__ __forceinline__ int ld_once(const int* p) {
+  int v;
+  asm volatile("ld.global.nc.s32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
 }
-
-// ============================================================== backward
-// One CTA per 128-key block: it walks the 128-query blocks that can see its
-// keys and, per block,
-//   S^T = K Q^T, dP^T = V dO^T                  (TMEM, 128 x 128 each)
-//   P^T = exp2(S^T log2e / 8 - lse log2e)       (bf16, back into TMEM)
-//   dS^T = P^T (dP^T - D)                       (bf16, shared memory)
-//   dV += P^T dO,  dK += dS^T Q                  (TMEM, across query blocks)
-//   dQ_blk = dS K                                (TMEM; added in fp32 to a
-//                                                 global accumulator by a TMA
-//                                                 bulk reduce, scaled by 1/8
-//                                                 and rounded by a final pass)
-// 320 threads: warp 0 loads, warp 1 issues MMAs, warps 2-9 are two groups of
-// four elementwise warps; group g handles query columns 64g..64g+63 of the
-// score tiles and d columns 32g..32g+31 of the dQ, dK, dV accumulators.
-#define BW_THREADS 320
-#define BW_QB 128                                    // queries per iterated block
-#define BW_ST 3                                      // Q / dO pipeline stages
-struct BwdSmem {
-  static constexpr int K = 0;                        // 16 KB: 128 keys x 64
-  static constexpr int V = K + AT_TILE_BYTES;        // 16 KB
-  static constexpr int Q = V + AT_TILE_BYTES;        // BW_ST stages x 16 KB
-  static constexpr int DO = Q + BW_ST * AT_TILE_BYTES;
-  static constexpr int DST = DO + BW_ST * AT_TILE_BYTES;   // 32 KB: [128 keys][128 queries] as two 64-query blocks
-  static constexpr int DQS = DST + 2 * AT_TILE_BYTES;      // 2 groups x 16 KB: [128 queries][32 fp32]
-  static constexpr int AUX = DQS + 2 * AT_TILE_BYTES;      // BW_ST stages x (lse2, D, dstart) x 128
-  static constexpr int BAR = AUX + BW_ST * 3 * BW_QB * 4;
-  static constexpr int TOTAL = BAR + 256;
-  // TMEM columns: S^T 0, dP^T 128, dV 256, dK 320, dQ 384, P^T (bf16 pairs) 448
-  static constexpr int TMEM_COLS = 512;
-};
-
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -360,6 +125,336 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// Forward softmax over one 32-key chunk of a score row.  Masked chunks keep
+// key e (0..31) when lo <= e <= hi (lo, hi relative to the chunk start); the
+// test is branch-free: ((e - lo) | (hi - e)) >= 0.
+template <bool MASK>
+__device__ __forceinline__ float fwd_chunk_max(const uint32_t* sr, int lo, int hi) {
+  float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent chains
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    const float v = __uint_as_float(sr[e]);
+    m4[e & 3] = fmaxf(m4[e & 3], (!MASK || ((e - lo) | (hi - e)) >= 0) ? v : -INFINITY);
+  }
+  return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+}
+template <bool MASK>
+__device__ __forceinline__ float fwd_chunk_exp(const uint32_t* sr, int lo, int hi, float sl2, float mb, uint32_t* pw) {
+  float l2[2] = {0.f, 0.f};
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    float p0 = ex2_approx(fmaf(__uint_as_float(sr[e]), sl2, -mb));
+    float p1 = ex2_approx(fmaf(__uint_as_float(sr[e + 1]), sl2, -mb));
+    if (MASK) {
+      p0 = ((e - lo) | (hi - e)) >= 0 ? p0 : 0.f;
+      p1 = ((e + 1 - lo) | (hi - e - 1)) >= 0 ? p1 : 0.f;
+    }
+    l2[(e >> 1) & 1] += p0 + p1;
+    pw[e / 2] = pk_bf16(p0, p1);
+  }
+  return l2[0] + l2[1];
+}
+
+// ============================================================== forward
+// CTA = two 128-query tiles (256 queries) sharing each 128-key block of K
+// and V.  Per tile g and key block j:
+//   S_g = Q_g K_j^T                (TMEM, 128 x 128 fp32)
+//   P_g = exp2(S_g log2e / 8 - m)  (bf16 pairs written back over S_g)
+//   O_g += P_g V_j                 (TMEM, 128 x 64 fp32, A operand from TMEM)
+// The MMA warp alternates between the tiles so that one tile's softmax runs
+// while the other tile's products are computed.  The running max m is only
+// raised (and O, l rescaled) when a row's block max exceeds it by more than
+// 2^8; otherwise the stale max is kept, which bounds every P by 256.
+// 320 threads: warp 0 loads, warp 1 issues MMAs, warps 2-5 (tile 0) and 6-9
+// (tile 1) run the softmax, thread t of a group owning query row t.
+#define FW_THREADS 320
+#define FW_QT 256                                    // queries per CTA
+#define FW_ST 3                                      // K / V stages
+#define FW_RESCALE 8.0f                              // log2 of the largest tolerated P
+struct FwdSmem {
+  static constexpr int Q = 0;                        // 2 tiles x 16 KB
+  static constexpr int KV = Q + 2 * AT_TILE_BYTES;   // FW_ST stages x (K 16 KB, V 16 KB)
+  static constexpr int BAR = KV + FW_ST * 2 * AT_TILE_BYTES;
+  static constexpr int TOTAL = BAR + 256;
+  static constexpr int TMEM_COLS = 512;              // tile g: S (P over its first 64 columns) at 256g, O at 256g + 128
+};
+
+__global__ void __launch_bounds__(FW_THREADS, 1)
+attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, float* __restrict__ lse,
+            const int* __restrict__ dstart, int T, int H, unsigned* err) {
+  extern __shared__ __align__(1024) uint8_t at_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)at_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = (uint64_t*)(sm + FwdSmem::BAR);
+  enum { Q_FULL = 0, KV_FULL = 1, KV_EMPTY = 1 + FW_ST, S_FULL = 1 + 2 * FW_ST, P_FULL = S_FULL + 2,
+         O_DONE = P_FULL + 2, DRAIN = O_DONE + 2, NBARS = DRAIN + 1 };
+  uint32_t* tmem_slot = (uint32_t*)(bars + NBARS);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  int* s_info = (int*)(tmem_slot + 2);
+  const uint32_t b0 = smem_u32(bars);
+  auto bar = [&](int i) { return b0 + 8u * i; };
+  const uint32_t sQ = smem_u32(sm + FwdSmem::Q), sKV = smem_u32(sm + FwdSmem::KV);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nqt = (T + FW_QT - 1) / FW_QT;
+  const int qt = nqt - 1 - blockIdx.y;   // heaviest query tiles first (y is the slow grid index)
+  const int bh = blockIdx.x, b = bh / H, h = bh % H;
+  const int C = H * AT_D;
+  const int q0 = qt * FW_QT;
+  const long rowbase = (long)b * T;
+  const int* dsr = dstart + rowbase;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(Q_FULL), 1);
+    for (int i = 0; i < FW_ST; ++i) {
+      mbar_init(bar(KV_FULL + i), 1);
+      mbar_init(bar(KV_EMPTY + i), 1);
+    }
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(bar(S_FULL + g), 1);
+      mbar_init(bar(P_FULL + g), 4);
+      mbar_init(bar(O_DONE + g), 1);
+    }
+    mbar_init(bar(DRAIN), 1);
+    *abort_flag = 0;
+    // key blocks of each tile: from its first query's document start to its last query
+    for (int g = 0; g < 2; ++g) {
+      const int qa = min(q0 + 128 * g, T - 1), qz = min(q0 + 128 * g + 127, T - 1);
+      s_info[2 * g] = dsr[qa] / AT_BLK;
+      s_info[2 * g + 1] = qz / AT_BLK;
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0) tc_alloc(smem_u32(tmem_slot), FwdSmem::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int lo0 = s_info[0], hi0 = s_info[1], lo1 = s_info[2], hi1 = s_info[3];
+  const bool two = q0 + 128 < T;          // the second tile has queries
+  const int jlo = lo0, jhi = two ? hi1 : hi0;
+  auto in_tile = [&](int g, int j) { return g == 0 ? (j >= lo0 && j <= hi0) : (two && j >= lo1 && j <= hi1); };
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- producer
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQKV)) : "memory");
+    mbar_expect_tx(bar(Q_FULL), 2 * AT_TILE_BYTES);
+    tma_load_2d(sQ, &tmQKV, bar(Q_FULL), h * AT_D, (int)(rowbase + q0));
+    tma_load_2d(sQ + AT_TILE_BYTES, &tmQKV, bar(Q_FULL), h * AT_D, (int)(rowbase + q0 + 128));
+    bool ok = true;
+    for (int j = jlo; j <= jhi && ok; ++j) {
+      const int n = j - jlo, st = n % FW_ST;
+      if (!mbar_wait(bar(KV_EMPTY + st), ((n / FW_ST) & 1) ^ 1, abort_flag)) { ok = false; break; }
+      mbar_expect_tx(bar(KV_FULL + st), 2 * AT_TILE_BYTES);
+      const uint32_t dst = sKV + st * 2 * AT_TILE_BYTES;
+      tma_load_2d(dst, &tmQKV, bar(KV_FULL + st), C + h * AT_D, (int)(rowbase + j * AT_BLK));
+      tma_load_2d(dst + AT_TILE_BYTES, &tmQKV, bar(KV_FULL + st), 2 * C + h * AT_D, (int)(rowbase + j * AT_BLK));
+    }
+    if (!ok) trap_timeout(abort_flag, err);
+    volatile int never = 0;
+    mbar_wait(bar(Q_FULL), 0, &never, 1ll << 28);
+    const int nj = jhi - jlo + 1;
+    for (int n = max(0, nj - FW_ST); n < nj; ++n) mbar_wait(bar(KV_FULL + n % FW_ST), (n / FW_ST) & 1, &never, 1ll << 28);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer: S_0(j+1) is issued right after P_0 V(j), then P_1 V(j), S_1(j+1)
+    constexpr uint32_t ID_S = instr_desc(128, false, false);   // S = Q K^T: 128 x 128, K = 64
+    constexpr uint32_t ID_O = instr_desc(64, false, true);     // O = P V: 128 x 64, K = 128 keys (V MN-major)
+    bool ok = mbar_wait(bar(Q_FULL), 0, abort_flag);
+    int ns[2] = {0, 0}, np[2] = {0, 0};   // S and P V products issued per tile
+    auto kv_wait = [&](int j) {
+      const int n = j - jlo;
+      return mbar_wait(bar(KV_FULL + n % FW_ST), (n / FW_ST) & 1, abort_flag);
+    };
+    auto issue_s = [&](int g, int j) -> bool {
+      if (!in_tile(g, j)) return true;
+      // the softmax has turned the previous S into P (and P V was issued before this)
+      if (ns[g] > 0 && !mbar_wait(bar(P_FULL + g), (ns[g] - 1) & 1, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t sK = sKV + ((j - jlo) % FW_ST) * 2 * AT_TILE_BYTES, q = sQ + g * AT_TILE_BYTES;
+#pragma unroll
+      for (int k = 0; k < AT_D / 16; ++k)
+        umma_bf16(tmem + 256 * g, kdesc(q + k * 32), kdesc(sK + k * 32), ID_S, k > 0);
+      umma_commit(bar(S_FULL + g));
+      ++ns[g];
+      return true;
+    };
+    auto issue_pv = [&](int g, int j) -> bool {
+      if (!in_tile(g, j)) return true;
+      if (!mbar_wait(bar(P_FULL + g), np[g] & 1, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t sV = sKV + ((j - jlo) % FW_ST) * 2 * AT_TILE_BYTES + AT_TILE_BYTES;
+#pragma unroll
+      for (int kk = 0; kk < AT_BLK / 16; ++kk)
+        umma_bf16_ts(tmem + 256 * g + 128, tmem + 256 * g + 8 * kk, mndesc(sV + kk * 2048, 8192), ID_O,
+                     (np[g] > 0 || kk > 0));
+      umma_commit(bar(O_DONE + g));
+      ++np[g];
+      return true;
+    };
+    if (ok && jlo <= jhi) ok = kv_wait(jlo) && issue_s(0, jlo) && issue_s(1, jlo);
+    for (int j = jlo; j <= jhi && ok; ++j) {
+      const bool next = j + 1 <= jhi;
+      if (!issue_pv(0, j)) { ok = false; break; }
+      if (next && !(kv_wait(j + 1) && issue_s(0, j + 1))) { ok = false; break; }
+      if (!issue_pv(1, j)) { ok = false; break; }
+      umma_commit(bar(KV_EMPTY + (j - jlo) % FW_ST));   // K / V of block j no longer read
+      if (next && !issue_s(1, j + 1)) { ok = false; break; }
+    }
+    if (!ok) trap_timeout(abort_flag, err);
+    umma_commit(bar(DRAIN));
+    volatile int never = 0;
+    mbar_wait(bar(DRAIN), 0, &never, 1ll << 28);
+  } else if (warp >= 2) {
+    // ---------------- softmax warps: thread owns query row r of tile g
+    const int quarter = warp & 3;
+    const int g = (warp - 2) >> 2;
+    const int r = quarter * 32 + lane;
+    const int q = q0 + 128 * g + r;
+    const bool qv = q < T;
+    // document starts are read once into registers (a volatile load: the
+    // compiler must not re-issue it inside the per-element mask)
+    const int ds_q = qv ? ld_once(dsr + q) : 0x7fffffff;
+    const int lo = g == 0 ? lo0 : lo1, hi = g == 0 ? hi0 : hi1;
+    const int qlast = min(q0 + 128 * g + 127, T - 1);
+    const int ds_last = ld_once(dsr + qlast);
+    const uint32_t tS = tmem + 256 * g + ((uint32_t)(quarter * 32) << 16), tO = tS + 128;
+    const float sl2 = 0.125f * LOG2E_F;   // 1/sqrt(64) in the exp2 domain
+    auto wait_w = [&](uint32_t bb, uint32_t parity) { return __all_sync(0xffffffffu, mbar_wait(bb, parity, abort_flag)); };
+    float m_use = -INFINITY, l = 0.f;
+    bool ok = true;
+    int n = 0;
+    if (g == 0 || two) {
+      for (int j = lo; j <= hi; ++j, ++n) {
+        if (!wait_w(bar(S_FULL + g), n & 1)) { ok = false; break; }
+        tc_fence_after();
+        const int kb0 = j * AT_BLK;
+        // masked blocks: a key may be later than a query or before its document
+        // (voted warp-wide so the warp runs one code path)
+        const bool need_mask = __any_sync(0xffffffffu, kb0 + AT_BLK - 1 > q0 + 128 * g || ds_last > kb0 || !qv);
+        // pass 1: row max of the block
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t sr[32];
+          tmem_ld32(tS + 32 * c, sr);
+          tmem_wait_ld();
+          const int base = kb0 + 32 * c;
+          mx = fmaxf(mx, need_mask ? fwd_chunk_max<true>(sr, ds_q - base, q - base) : fwd_chunk_max<false>(sr, 0, 0));
+        }
+        mx *= sl2;
+        // raise the max (rescaling O and l) only when it grew by more than 2^FW_RESCALE
+        const bool raise = mx > m_use + FW_RESCALE;
+        if (__any_sync(0xffffffffu, raise)) {
+          const float m_new = fmaxf(m_use, mx);
+          const float sc = m_use == -INFINITY ? 0.f : exp2f(m_use - m_new);
+          if (n > 0) {
+            // O holds P V of every earlier block: wait for the last one, then scale it
+            if (!wait_w(bar(O_DONE + g), (n - 1) & 1)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              uint32_t orr[32];
+              tmem_ld32(tO + 32 * c, orr);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * sc);
+              tmem_st32(tO + 32 * c, orr);
+            }
+            tmem_wait_st();
+          }
+          l *= sc;
+          m_use = m_new;
+        }
+        const float mb = m_use == -INFINITY ? 0.f : m_use;
+        // pass 2: P = exp2(S sl2 - m) as bf16 pairs over the first 64 columns of S
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t sr[32], pw[16];
+          tmem_ld32(tS + 32 * c, sr);
+          tmem_wait_ld();
+          const int base = kb0 + 32 * c;
+          l += need_mask ? fwd_chunk_exp<true>(sr, ds_q - base, q - base, sl2, mb, pw)
+                         : fwd_chunk_exp<false>(sr, 0, 0, sl2, mb, pw);
+          tmem_st16(tS + 16 * c, pw);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(P_FULL + g));
+      }
+    }
+    if (!ok) trap_timeout(abort_flag, err);
+    // O / l for the row, after the last P V
+    if (ok && n > 0 && wait_w(bar(O_DONE + g), (n - 1) & 1)) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      bf16* orow = out + (rowbase + q) * C + h * AT_D;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t orr[32];
+        tmem_ld32(tO + 32 * c, orr);
+        tmem_wait_ld();
+        if (qv) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 w;
+            w.x = pk_bf16(__uint_as_float(orr[8 * u]) * inv, __uint_as_float(orr[8 * u + 1]) * inv);
+            w.y = pk_bf16(__uint_as_float(orr[8 * u + 2]) * inv, __uint_as_float(orr[8 * u + 3]) * inv);
+            w.z = pk_bf16(__uint_as_float(orr[8 * u + 4]) * inv, __uint_as_float(orr[8 * u + 5]) * inv);
+            w.w = pk_bf16(__uint_as_float(orr[8 * u + 6]) * inv, __uint_as_float(orr[8 * u + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + 32 * c + 8 * u) = w;
+          }
+        }
+      }
+      if (qv) lse[(long)bh * T + q] = (m_use + log2f(l)) * LN2_F;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tc_dealloc(tmem, FwdSmem::TMEM_COLS);
+}
+
+// ============================================================== backward
+// One CTA per 128-key block: it walks the 128-query blocks that can see its
+// keys and, per block,
+//   S^T = K Q^T, dP^T = V dO^T                  (TMEM, 128 x 128 each)
+//   P^T = exp2(S^T log2e / 8 - lse log2e)       (bf16, back into TMEM)
+//   dS^T = P^T (dP^T - D)                       (bf16, shared memory)
+//   dV += P^T dO,  dK += dS^T Q                  (TMEM, across query blocks)
+//   dQ_blk = dS K                                (TMEM; added in fp32 to a
+//                                                 global accumulator by a TMA
+//                                                 bulk reduce, scaled by 1/8
+//                                                 and rounded by a final pass)
+// 352 threads: warp 0 loads, warp 1 issues MMAs, warps 2-9 are two groups of
+// four elementwise warps (group g handles query columns 64g..64g+63 of the
+// score tiles and d columns 32g..32g+31 of the dQ, dK, dV accumulators) and
+// warp 10 issues the dQ bulk reduces.
+#define BW_THREADS 352
+#define BW_QB 128                                    // queries per iterated block
+#define BW_ST 3                                      // Q / dO pipeline stages
+struct BwdSmem {
+  static constexpr int K = 0;                        // 16 KB: 128 keys x 64
+  static constexpr int V = K + AT_TILE_BYTES;        // 16 KB
+  static constexpr int Q = V + AT_TILE_BYTES;        // BW_ST stages x 16 KB
+  static constexpr int DO = Q + BW_ST * AT_TILE_BYTES;
+  static constexpr int DST = DO + BW_ST * AT_TILE_BYTES;   // 32 KB: [128 keys][128 queries] as two 64-query blocks
+  static constexpr int DQS = DST + 2 * AT_TILE_BYTES;      // 2 groups x 16 KB: [128 queries][32 fp32]
+  static constexpr int AUX = DQS + 2 * AT_TILE_BYTES;      // BW_ST stages x (lse2, D, dstart) x 128
+  static constexpr int BAR = AUX + BW_ST * 3 * BW_QB * 4;
+  static constexpr int TOTAL = BAR + 256;
+  // TMEM columns: S^T 0, dP^T 128, dV 256, dK 320, dQ 384, P^T (bf16 pairs) 448
+  static constexpr int TMEM_COLS = 512;
+};
+
 // 32 columns of P^T and dS^T for one key row: p = exp2(s sl2 - lse2), ds = p (dp - D),
 // packed into bf16 pairs.  MASK applies causality and document starts.
 template <bool MASK>
@@ -382,7 +477,7 @@ __device__ __forceinline__ void bwd_elementwise32(const uint32_t* sr, const uint
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       float x = ex2_approx(fmaf(__uint_as_float(sr[c8 + e]), sl2, -lv[e]));
-      if (MASK && !(q_first + c8 + e >= k && dsq[e] <= k)) x = 0.f;
+      if (MASK) x = ((q_first + c8 + e - k) | (k - dsq[e])) >= 0 ? x : 0.f;   // q >= k and dstart[q] <= k
       pv[e] = x;
       gv[e] = x * (__uint_as_float(dr[c8 + e]) - dv[e]);
     }
@@ -563,13 +658,12 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
     umma_commit(bar(DRAIN));
     volatile int never = 0;
     mbar_wait(bar(DRAIN), 0, &never, 1ll << 28);
-  } else if (warp >= 2) {
+  } else if (warp >= 2 && warp < 10) {
     // ---------------- elementwise warps: thread owns key row r (and query row r of dQ)
     const int quarter = warp & 3;
     const int grp = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
     const int k = k0 + r;
-    const int gtid = threadIdx.x - 64 - 128 * grp;   // 0..127 inside the group
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = 0.125f * LOG2E_F;
     const uint32_t st_full = bar(ST_FULL + grp), st_free = bar(ST_FREE + grp);
@@ -578,8 +672,8 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
     // waits are voted warp-wide so that the .sync.aligned TMEM accesses after
     // them are never reached by part of a warp
     auto wait_w = [&](uint32_t bb, uint32_t parity) { return __all_sync(0xffffffffu, mbar_wait(bb, parity, abort_flag)); };
-    // dQ of block j: TMEM -> fp32 staging (128-byte swizzle) -> bulk reduce-add
-    // issued by the group's first thread once all 128 rows are written
+    // dQ of block j: TMEM -> fp32 staging (128-byte swizzle); warp 10 issues
+    // the bulk reduce-add once all 128 rows of the group are written
     auto flush_dq = [&](int j) -> bool {
       uint32_t rr[32];
       tmem_ld32(tmem + lane_off + 384 + 32 * grp, rr);
@@ -587,7 +681,7 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(DQ_FREE));   // the dQ accumulator may be overwritten
-      // the reduce of block j-1 has read the staging (signalled by the first thread)
+      // the reduce of block j-1 has read the staging
       if (j > 0 && !wait_w(st_free, (j - 1) & 1)) return false;
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
@@ -598,24 +692,11 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
       }
       fence_async_smem();
       mbar_arrive(st_full);
-      if (gtid == 0) {
-        if (!mbar_wait(st_full, j & 1, abort_flag)) return false;
-        tma_reduce_add_2d(&tmDQ, sDQg, h * AT_D + 32 * grp, (int)(rowbase + (qb_lo + j) * BW_QB));
-        bulk_commit();
-      }
       return true;
-    };
-    // first thread: once the reduce of the previous flush has read the staging, free it
-    auto release_staging = [&]() {
-      if (gtid == 0) {
-        bulk_wait_read<0>();
-        mbar_arrive(st_free);
-      }
     };
     for (int i = 0; i < niter; ++i) {
       const int q0 = (qb_lo + i) * BW_QB;
       const int st = i % BW_ST;
-      if (i >= 2) release_staging();   // reduce of block i-2, before the flush of block i-1
       const float* L2 = aux + st * 3 * BW_QB + 64 * grp;
       const float* Dq = L2 + BW_QB;
       const int* DSq = reinterpret_cast<const int*>(L2 + 2 * BW_QB);
@@ -672,7 +753,6 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
     // the last block's dQ, then dK and dV
     if (ok && niter > 0 && wait_w(bar(MMA_DONE), (niter - 1) & 1)) {
       tc_fence_after();
-      if (niter >= 2) release_staging();
       ok = flush_dq(niter - 1);
       if (ok) {
         bf16* row = dqkv + (rowbase + k) * 3 * C;
@@ -699,7 +779,23 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
       ok = false;
     }
     if (!ok) trap_timeout(abort_flag, err);
-    if (gtid == 0) bulk_wait_all();
+  } else if (warp == 10 && lane == 0) {
+    // ---------------- dQ reducer: per block, both groups' staging -> global fp32 accumulator
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmDQ)) : "memory");
+    bool ok = true;
+    for (int j = 0; j < niter && ok; ++j) {
+      for (int gg = 0; gg < 2; ++gg) {
+        if (!mbar_wait(bar(ST_FULL + gg), j & 1, abort_flag)) { ok = false; break; }
+        tma_reduce_add_2d(&tmDQ, sDQ + gg * AT_TILE_BYTES, h * AT_D + 32 * gg, (int)(rowbase + (qb_lo + j) * BW_QB));
+        bulk_commit();
+      }
+      if (!ok) break;
+      bulk_wait_read<0>();   // both stagings read: the groups may overwrite them
+      mbar_arrive(bar(ST_FREE + 0));
+      mbar_arrive(bar(ST_FREE + 1));
+    }
+    if (!ok) trap_timeout(abort_flag, err);
+    bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -759,16 +855,14 @@ cudaError_t launch_attn_fwd_tc(const bf16* qkv, bf16* out, float* lse, const int
                                unsigned* err, cudaStream_t s) {
   const int C = H * AT_D;
   const long rows = (long)B * T;
-  CUtensorMap tq, tkv;
-  if (!make_map_ex(&tq, MapKey{qkv, rows, 3L * C, 3L * C, 1, 0, AT_D, AT_BLK, 0, 128}) ||
-      !make_map_ex(&tkv, MapKey{qkv, rows, 3L * C, 3L * C, 1, 0, AT_D, AT_BK, 0, 128}))
-    return cudaErrorInvalidValue;
+  CUtensorMap tqkv;
+  if (!make_map_ex(&tqkv, MapKey{qkv, rows, 3L * C, 3L * C, 1, 0, AT_D, AT_BLK, 0, 128})) return cudaErrorInvalidValue;
   const int smem = FwdSmem::TOTAL + 1024;
   static bool attr = false;
   if (!attr) { cudaError_t e = tc_smem_attr(attn_fwd_tc, smem); if (e) return e; attr = true; }
-  dim3 grid(B * H, (T + AT_BLK - 1) / AT_BLK);
+  dim3 grid(B * H, (T + FW_QT - 1) / FW_QT);
   ++g_kernel_launches;
-  attn_fwd_tc<<<grid, AT_THREADS, smem, s>>>(tq, tkv, out, lse, dstart, T, H, err);
+  attn_fwd_tc<<<grid, FW_THREADS, smem, s>>>(tqkv, out, lse, dstart, T, H, err);
   return cudaGetLastError();
 }
 

@@ -4,6 +4,7 @@
 // global-norm clip and AdamW.  All are HBM-bound: 16-byte vector loads, one
 // warp per row where a row is reduced, no fp32 copies of bf16 tensors.
 #include "launch.h"
+#include "tc_common.cuh"
 
 unsigned long long g_kernel_launches = 0;
 
@@ -195,6 +196,25 @@ ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __
     const float mu = mean[row], rs = rstd[row];
     const T* dyr = dy + (long)row * C;
     const T* xr = x + (long)row * C;
+    // every load of the row is issued before the first use (one memory latency
+    // per row); dy and x stay packed until they are used
+    uint4 dyp[NCH], xp[NCH];
+    float o[NCH][NV];
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int ch = lane + i * 32;
+      if (ch < nch) {
+        dyp[i] = *reinterpret_cast<const uint4*>(dyr + ch * NV);
+        xp[i] = *reinterpret_cast<const uint4*>(xr + ch * NV);
+        if (dres_in) {
+#pragma unroll
+          for (int j = 0; j < NV; j += 4) Vec<float>::load(dres_in + (long)row * C + ch * NV + j, o[i] + j);
+        } else {
+#pragma unroll
+          for (int j = 0; j < NV; ++j) o[i][j] = 0.f;
+        }
+      }
+    }
     float xh[NCH][NV], gh[NCH][NV];
     float s1 = 0.f, s2 = 0.f;
 #pragma unroll
@@ -202,8 +222,8 @@ ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __
       const int ch = lane + i * 32;
       if (ch < nch) {
         float dv[NV], gg[NV];
-        Vec<T>::load(dyr + ch * NV, dv);
-        Vec<T>::load(xr + ch * NV, xh[i]);
+        Vec<T>::load(reinterpret_cast<const T*>(&dyp[i]), dv);
+        Vec<T>::load(reinterpret_cast<const T*>(&xp[i]), xh[i]);
 #pragma unroll
         for (int j = 0; j < NV; j += 4) Vec<float>::load(g + ch * NV + j, gg + j);
 #pragma unroll
@@ -224,22 +244,14 @@ ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __
       const int ch = lane + i * 32;
       if (ch < nch) {
         const long off = (long)row * C + ch * NV;
-        float o[NV];
-        if (dres_in) {
-#pragma unroll
-          for (int j = 0; j < NV; j += 4) Vec<float>::load(dres_in + off + j, o + j);
-        } else {
-#pragma unroll
-          for (int j = 0; j < NV; ++j) o[j] = 0.f;
-        }
 #pragma unroll
         for (int j = 0; j < NV; ++j) {
-          o[j] += rs * (gh[i][j] - s1 - xh[i][j] * s2);
-          dsm[i][j] += o[j];
+          o[i][j] += rs * (gh[i][j] - s1 - xh[i][j] * s2);
+          dsm[i][j] += o[i][j];
         }
 #pragma unroll
-        for (int j = 0; j < NV; j += 4) Vec<float>::store(dres_out + off + j, o + j);
-        Vec<T>::store(dres_out_t + off, o);
+        for (int j = 0; j < NV; j += 4) Vec<float>::store(dres_out + off + j, o[i] + j);
+        Vec<T>::store(dres_out_t + off, o[i]);
       }
     }
   }
@@ -277,21 +289,156 @@ static cudaError_t ln_bwd_launch(const T* dy, const T* x, const float* mean, con
   return cudaGetLastError();
 }
 
+// LayerNorm backward, row-group form: TPR = C / NV threads (one 16-byte chunk
+// each) share a row, G groups per block walk rows with a stride; the next
+// row's loads are issued before the current row's reduction, and the row sums
+// go through a per-group named barrier with double-buffered slots.  Column
+// accumulators (dgamma, dbeta, column sums of the residual gradient) are 24
+// registers per thread, summed over groups into one partial row per block.
+#define LNB2_THREADS 288
+template <typename T>
+__global__ void __launch_bounds__(LNB2_THREADS, 2)
+ln_bwd2_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __restrict__ mean,
+               const float* __restrict__ rstd, const float* __restrict__ g, const float* dres_in, float* dres_out,
+               T* __restrict__ dres_out_t, float* __restrict__ partials, int M, int C, int TPR, int G) {
+  constexpr int NV = Vec<T>::N;
+  __shared__ float2 slot[2][LNB2_THREADS / 32];
+  const int grp = threadIdx.x / TPR, t = threadIdx.x % TPR;
+  const int nch = C / NV;
+  const bool act = grp < G && t < nch;
+  const int wpg = TPR / 32, wig = t / 32, lane = threadIdx.x & 31;
+  const int col = t * NV;
+  float gg[NV], dg[NV], db[NV], dsm[NV];
+#pragma unroll
+  for (int j = 0; j < NV; ++j) { gg[j] = 0.f; dg[j] = 0.f; db[j] = 0.f; dsm[j] = 0.f; }
+  if (act) {
+#pragma unroll
+    for (int j = 0; j < NV; j += 4) Vec<float>::load(g + col + j, gg + j);
+  }
+  const int stride = gridDim.x * G;
+  int row = blockIdx.x * G + grp;
+  // prefetch of a row: dy, x packed, the residual gradient in fp32, mean, rstd
+  uint4 dyp = make_uint4(0, 0, 0, 0), xp = make_uint4(0, 0, 0, 0);
+  float dr[NV], mu = 0.f, rs = 0.f;
+  auto fetch = [&](int r) {
+    if (act && r < M) {
+      dyp = *reinterpret_cast<const uint4*>(dy + (long)r * C + col);
+      xp = *reinterpret_cast<const uint4*>(x + (long)r * C + col);
+      if (dres_in) {
+#pragma unroll
+        for (int j = 0; j < NV; j += 4) Vec<float>::load(dres_in + (long)r * C + col + j, dr + j);
+      } else {
+#pragma unroll
+        for (int j = 0; j < NV; ++j) dr[j] = 0.f;
+      }
+      mu = mean[r];
+      rs = rstd[r];
+    }
+  };
+  fetch(row);
+  int it = 0;
+  // every group runs the same number of iterations (rows past M are idle) so
+  // its named barrier always sees all of its threads
+  const int iters = (M + stride - 1) / stride;
+  for (; it < iters; ++it, row += stride) {
+    float dv[NV], xh[NV], o[NV];
+    Vec<T>::load(reinterpret_cast<const T*>(&dyp), dv);
+    Vec<T>::load(reinterpret_cast<const T*>(&xp), xh);
+#pragma unroll
+    for (int j = 0; j < NV; ++j) o[j] = dr[j];
+    const float mu_r = mu, rs_r = rs;
+    const bool live = act && row < M;
+    fetch(row + stride);
+    float s1 = 0.f, s2 = 0.f, gh[NV];
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      xh[j] = (xh[j] - mu_r) * rs_r;
+      gh[j] = dv[j] * gg[j];
+      s1 += gh[j];
+      s2 += gh[j] * xh[j];
+      if (live) { dg[j] += dv[j] * xh[j]; db[j] += dv[j]; }
+    }
+    s1 = warp_sum(live ? s1 : 0.f);
+    s2 = warp_sum(live ? s2 : 0.f);
+    if (lane == 0 && grp < G) slot[it & 1][grp * wpg + wig] = make_float2(s1, s2);
+    if (grp < G) asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(TPR) : "memory");
+    s1 = 0.f; s2 = 0.f;
+    for (int w = 0; w < wpg; ++w) {
+      const float2 v = slot[it & 1][grp * wpg + w];
+      s1 += v.x;
+      s2 += v.y;
+    }
+    s1 /= C;
+    s2 /= C;
+    if (live) {
+      const long off = (long)row * C + col;
+#pragma unroll
+      for (int j = 0; j < NV; ++j) {
+        o[j] += rs_r * (gh[j] - s1 - xh[j] * s2);
+        dsm[j] += o[j];
+      }
+#pragma unroll
+      for (int j = 0; j < NV; j += 4) Vec<float>::store(dres_out + off + j, o + j);
+      Vec<T>::store(dres_out_t + off, o);
+    }
+  }
+  // sum the groups' accumulators: [dg | db | dsm] per block
+  __syncthreads();
+  extern __shared__ float red2[];   // [G][3C]
+  if (act) {
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      red2[grp * 3 * C + col + j] = dg[j];
+      red2[grp * 3 * C + C + col + j] = db[j];
+      red2[grp * 3 * C + 2 * C + col + j] = dsm[j];
+    }
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < 3 * C; c += blockDim.x) {
+    float acc = 0.f;
+    for (int gi = 0; gi < G; ++gi) acc += red2[gi * 3 * C + c];
+    partials[(long)blockIdx.x * 3 * C + c] = acc;
+  }
+}
+
 template <typename T>
 cudaError_t launch_ln_bwd(const T* dy, const T* x, const float* mean, const float* rstd, const float* g,
                           const float* dres_in, float* dres_out, T* dres_out_t, float* partials,
                           int M, int C, int* nblk_out, cudaStream_t s) {
+  constexpr int NV = Vec<T>::N;
+  {
+    // row-group kernel: C / NV threads per row (whole warps), several rows per block
+    const int tpr = ((C / NV + 31) / 32) * 32;
+    if (C % NV == 0 && tpr <= LNB2_THREADS) {
+      const int G = LNB2_THREADS / tpr;
+      int nblk = (M + G - 1) / G;
+      if (nblk > 148 * 2) nblk = 148 * 2;
+      *nblk_out = nblk;
+      const size_t smem = (size_t)G * 3 * C * sizeof(float);
+      static size_t attr = 0;
+      if (smem > 48 * 1024 && smem > attr) {
+        cudaError_t e = cudaFuncSetAttribute(ln_bwd2_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr = smem;
+      }
+      ++g_kernel_launches;
+      ln_bwd2_kernel<T><<<nblk, G * tpr, smem, s>>>(dy, x, mean, rstd, g, dres_in, dres_out, dres_out_t, partials, M,
+                                                    C, tpr, G);
+      return cudaGetLastError();
+    }
+  }
   int nblk = (M + LNB_WARPS - 1) / LNB_WARPS;
   if (nblk > 148 * 3) nblk = 148 * 3;
   *nblk_out = nblk;
-  constexpr int NV = Vec<T>::N;
   int per_lane = (C / NV + 31) / 32;   // 16-byte chunks per lane
   switch (per_lane) {
     case 1: return ln_bwd_launch<T, 1>(dy, x, mean, rstd, g, dres_in, dres_out, dres_out_t, partials, M, C, nblk, s);
     case 2: return ln_bwd_launch<T, 2>(dy, x, mean, rstd, g, dres_in, dres_out, dres_out_t, partials, M, C, nblk, s);
     case 3: return ln_bwd_launch<T, 3>(dy, x, mean, rstd, g, dres_in, dres_out, dres_out_t, partials, M, C, nblk, s);
     case 4: return ln_bwd_launch<T, 4>(dy, x, mean, rstd, g, dres_in, dres_out, dres_out_t, partials, M, C, nblk, s);
-    default: return ln_bwd_launch<T, 8>(dy, x, mean, rstd, g, dres_in, dres_out, dres_out_t, partials, M, C, nblk, s);
+    default:   // C <= 1024: at most 4 chunks of 8 bf16 or 8 chunks of 4 fp32
+      if constexpr (NV >= 8) return cudaErrorInvalidValue;
+      else return ln_bwd_launch<T, 8>(dy, x, mean, rstd, g, dres_in, dres_out, dres_out_t, partials, M, C, nblk, s);
   }
 }
 
@@ -522,10 +669,110 @@ xent_smem_kernel(T* __restrict__ logits, long ldl, const int* __restrict__ tgt, 
   }
 }
 
+// bf16 logits: the row moves between HBM and shared memory as one bulk copy
+// each way (the copy engine keeps the whole row in flight); the three passes
+// over it (max, exp and sum, scale) run on shared memory.  exp(z - max) is
+// kept in place as bf16 and summed in fp32.
+#define XB_THREADS 512
+__global__ void __launch_bounds__(XB_THREADS, 2)
+xent_bulk_kernel(bf16* __restrict__ logits, long ldl, const int* __restrict__ tgt, int V, int Vp,
+                 float* __restrict__ rowloss, DevScalars* __restrict__ sc) {
+  extern __shared__ __align__(128) uint8_t xb_raw[];
+  __shared__ float red[33];
+  __shared__ __align__(8) uint64_t bar;
+  bf16* zs = reinterpret_cast<bf16*>(xb_raw);
+  const int row = blockIdx.x;
+  bf16* z = logits + (long)row * ldl;
+  const int tg = tgt[row];
+  const int nvec = Vp / 8;
+  const uint32_t bytes = (uint32_t)nvec * 16;
+  const uint32_t sbar = smem_u32(&bar), sz = smem_u32(zs);
+  if (threadIdx.x == 0) {
+    mbar_init(sbar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_expect_tx(sbar, bytes);
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(sz),
+                 "l"(reinterpret_cast<uint64_t>(z)), "r"(bytes), "r"(sbar)
+                 : "memory");
+  }
+  __syncthreads();
+  {
+    volatile int never = 0;
+    if (!mbar_wait(sbar, 0, &never, 1ll << 30)) atomicOr(&sc->err, GPT_DEVERR_TIMEOUT);
+  }
+  const uint4* zv = reinterpret_cast<const uint4*>(zs);
+  float m = -INFINITY;
+  for (int i = threadIdx.x; i < nvec; i += XB_THREADS) {
+    float v[8];
+    const uint4 w = zv[i];
+    Vec<bf16>::load(reinterpret_cast<const bf16*>(&w), v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (i * 8 + j < V) m = fmaxf(m, v[j]);
+  }
+  m = block_reduce(m, true, red);
+  const float zt = tg >= 0 ? to_f(zs[tg]) : 0.f;
+  __syncthreads();   // z[target] is read before the exp pass overwrites it
+  const float ml2 = m * 1.4426950408889634f;
+  float ssum = 0.f;
+  for (int i = threadIdx.x; i < nvec; i += XB_THREADS) {
+    float v[8];
+    uint4 w = zv[i];
+    Vec<bf16>::load(reinterpret_cast<const bf16*>(&w), v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float e;
+      asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(fmaf(v[j], 1.4426950408889634f, -ml2)));
+      v[j] = i * 8 + j < V ? e : 0.f;
+      ssum += v[j];
+    }
+    Vec<bf16>::store(reinterpret_cast<bf16*>(&w), v);
+    reinterpret_cast<uint4*>(zs)[i] = w;
+  }
+  ssum = block_reduce(ssum, false, red);
+  if (threadIdx.x == 0) rowloss[row] = tg >= 0 ? m + logf(ssum) - zt : 0.f;
+  const int nv = sc->n_valid;
+  const float scale = tg >= 0 ? sc->loss_scale / (float)(nv > 0 ? nv : 1) : 0.f;
+  const float inv = scale / ssum;
+  for (int i = threadIdx.x; i < nvec; i += XB_THREADS) {
+    float v[8];
+    uint4 w = zv[i];
+    Vec<bf16>::load(reinterpret_cast<const bf16*>(&w), v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = v[j] * inv - (i * 8 + j == tg ? scale : 0.f);
+    Vec<bf16>::store(reinterpret_cast<bf16*>(&w), v);
+    reinterpret_cast<uint4*>(zs)[i] = w;
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(reinterpret_cast<uint64_t>(z)),
+                 "r"(sz), "r"(bytes)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");   // shared memory stays live until read
+  }
+}
+
 template <typename T>
 cudaError_t launch_xent(T* logits, long ldl, const int* tgt, int M, int V, int Vp, float* rowloss,
                         DevScalars* sc, cudaStream_t s) {
   constexpr int NV = Vec<T>::N;
+  if constexpr (NV == 8) {
+    // bulk copies: 16-byte aligned rows, whole row within 110 KB (two blocks per SM)
+    const size_t bytes = (size_t)Vp * 2;
+    if (Vp % 8 == 0 && ldl % 8 == 0 && bytes <= 110 * 1024) {
+      static size_t attr = 0;
+      if (bytes > attr) {
+        cudaError_t e = cudaFuncSetAttribute(xent_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        if (e != cudaSuccess) return e;
+        attr = bytes;
+      }
+      ++g_kernel_launches;
+      xent_bulk_kernel<<<M, XB_THREADS, bytes, s>>>(logits, ldl, tgt, V, Vp, rowloss, sc);
+      return cudaGetLastError();
+    }
+  }
   size_t smem = (size_t)((Vp + NV - 1) / NV) * NV * sizeof(T);
   if (smem <= 200 * 1024 && (ldl % NV) == 0) {
     static size_t attr = 0;
