@@ -94,28 +94,33 @@ struct EpiTraits {
   static constexpr bool F32OUT = (KIND == EPI_F32 || KIND == EPI_F32_SPLIT);
 };
 
-template <int BN, int KIND>
+template <int BN, int KIND, int CG = 1>
 struct TcCfg {
   // GELU's second output and the side input each take two more staging
   // buffers; the other kinds keep one more mainloop stage instead
   static constexpr bool WIDE = (KIND == EPI_GELU || EpiTraits<KIND>::SIDE);
   static constexpr int EPI_BYTES = (WIDE ? 4 : 2) * EPI_BUF_BYTES;
-  static constexpr int STAGES = (BN >= 256 ? 3 : 4) + (WIDE ? 0 : 1);
   static constexpr int BIAS_BYTES = EpiTraits<KIND>::BIAS ? BN * 4 : 0;
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;
-  static constexpr int B_BYTES = BN * TC_BK * 2;
+  static constexpr int B_BYTES = (BN / CG) * TC_BK * 2;   // a CTA pair splits B along N
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int FREE = 232448 - 1024 - EPI_BYTES - 256 - BIAS_BYTES;
+  static constexpr int STAGES = FREE / STAGE_BYTES > 8 ? 8 : FREE / STAGE_BYTES;
   static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
   static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + 256 + BIAS_BYTES;
   static_assert(SMEM <= 232448, "shared memory per block");
 };
 
-template <int BN, bool A_MN, bool B_MN, int KIND>
+// CG = 2: a cluster of two CTAs computes a 256-row tile with one
+// tcgen05.mma.cta_group::2 stream issued by the even CTA; each CTA loads its
+// 128 rows of A and half of the tile's B columns, and holds its 128 rows of
+// the accumulator in its own TMEM.
+template <int BN, bool A_MN, bool B_MN, int KIND, int CG>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2, int M, int N,
                int K, int splits, EpiParams<bf16> epi, unsigned* err) {
-  using Cfg = TcCfg<BN, KIND>;
+  using Cfg = TcCfg<BN, KIND, CG>;
   constexpr int STAGES = Cfg::STAGES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -137,9 +142,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const uint32_t group_bar = bar0 + 8u * (2 * STAGES + 5);
   auto side_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 6 + b); };
 
+  const uint32_t rank = CG == 2 ? cluster_rank() : 0u;   // CTA inside the pair; 0 issues the MMAs
+  const int cid = CG == 2 ? (int)(blockIdx.x >> 1) : (int)blockIdx.x, ncl = CG == 2 ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar(a), 1); mbar_init(tempty_bar(a), 4); }
+    for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar(a), 1); mbar_init(tempty_bar(a), 4 * CG); }
     mbar_init(drain_bar, 1);
     mbar_init(group_bar, 128);
     mbar_init(side_bar(0), 1);
@@ -149,16 +156,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(Cfg::TMEM_COLS));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    if constexpr (CG == 2) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                   "r"(Cfg::TMEM_COLS));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                   "r"(Cfg::TMEM_COLS));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (CG == 2) cluster_sync_all();   // both CTAs' barriers exist before any remote arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int tiles_m = (M + TC_BM - 1) / TC_BM, tiles_n = (N + BN - 1) / BN;
+  constexpr int TM = TC_BM * CG;   // output rows per work unit
+  const int tiles_m = (M + TM - 1) / TM, tiles_n = (N + BN - 1) / BN;
   const int tiles = tiles_m * tiles_n;
   const int units = tiles * splits;
   const int kb_total = (K + TC_BK - 1) / TC_BK;
@@ -172,28 +187,33 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     uint32_t phase = 0;
     long issued = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    for (int u = cid; u < units && ok; u += ncl) {
       const int split = u / tiles, t = u % tiles;
-      const int m0 = (t % tiles_m) * TC_BM, n0 = (t / tiles_m) * BN;
+      const int m0 = (t % tiles_m) * TM + TC_BM * (int)rank, n0 = (t / tiles_m) * BN + (BN / CG) * (int)rank;
       const int kb0 = split * kbs, kb1 = min(kb_total, kb0 + kbs);
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(empty_bar(stage), phase ^ 1, abort_flag)) { ok = false; break; }
-        const uint32_t fb = full_bar(stage);
-        mbar_expect_tx(fb, Cfg::STAGE_BYTES);
+        // a pair completes both CTAs' bytes on the even CTA's barrier
+        const uint32_t fb = CG == 2 ? cluster_addr(full_bar(stage), 0) : full_bar(stage);
+        if (rank == 0) mbar_expect_tx(full_bar(stage), CG * Cfg::STAGE_BYTES);
         const uint32_t sa = smem_u32(tile_mem + stage * Cfg::STAGE_BYTES);
         const uint32_t sb = sa + Cfg::A_BYTES;
         const int k0 = kb * TC_BK;
+        auto load = [&](uint32_t dst, const CUtensorMap* map, int x, int y) {
+          if constexpr (CG == 2) tma_load_2d_pair(dst, map, fb, x, y);
+          else tma_load_2d(dst, map, fb, x, y);
+        };
         if (!A_MN) {
-          tma_load_2d(sa, &tmA, fb, k0, m0);
+          load(sa, &tmA, k0, m0);
         } else {
 #pragma unroll
-          for (int j = 0; j < TC_BM / 64; ++j) tma_load_2d(sa + j * 64 * TC_BK * 2, &tmA, fb, m0 + 64 * j, k0);
+          for (int j = 0; j < TC_BM / 64; ++j) load(sa + j * 64 * TC_BK * 2, &tmA, m0 + 64 * j, k0);
         }
         if (!B_MN) {
-          tma_load_2d(sb, &tmB, fb, k0, n0);
+          load(sb, &tmB, k0, n0);
         } else {
 #pragma unroll
-          for (int j = 0; j < BN / 64; ++j) tma_load_2d(sb + j * 64 * TC_BK * 2, &tmB, fb, n0 + 64 * j, k0);
+          for (int j = 0; j < BN / CG / 64; ++j) load(sb + j * 64 * TC_BK * 2, &tmB, n0 + 64 * j, k0);
         }
         ++issued;
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -204,7 +224,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       atomicOr(err, GPT_DEVERR_TIMEOUT);
     }
     // drain: wait (bounded) for the most recent loads of every stage to land
-    long nd = issued < STAGES ? issued : STAGES;
+    // (a pair's loads all complete on the even CTA's barriers)
+    long nd = rank == 0 ? (issued < STAGES ? issued : STAGES) : 0;
     int s = stage;
     uint32_t ph = phase;
     for (long i = 0; i < nd; ++i) {
@@ -212,9 +233,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       volatile int never = 0;
       mbar_wait(full_bar(s), ph, &never, 1ll << 28);
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
-    constexpr uint32_t IDESC = instr_desc(BN, A_MN, B_MN);
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ---------------- MMA issuer (the even CTA of a pair issues for both)
+    constexpr uint32_t IDESC = instr_desc(BN, A_MN, B_MN, TM);
     // K-major: SBO = 8 rows x 128 B; k step (16 elements) = 32 B inside the swizzle row.
     // MN-major: LBO = one 64-element box (64 k-rows x 128 B), SBO = 8 k-rows x 128 B; k step = 16 rows.
     constexpr uint32_t A_LBO = A_MN ? 64 * TC_BK * 2 : 16, A_SBO = 1024, A_KSTEP = A_MN ? 16 * 128 : 32;
@@ -224,7 +245,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    for (int u = cid; u < units && ok; u += ncl) {
       const int split = u / tiles;
       const int kb0 = split * kbs, kb1 = min(kb_total, kb0 + kbs);
       if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1, abort_flag)) { ok = false; break; }
@@ -239,13 +260,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         for (int k = 0; k < TC_BK / 16; ++k) {
           uint64_t ad = smem_desc(sa + k * A_KSTEP, A_LBO, A_SBO);
           uint64_t bd = smem_desc(sb + k * B_KSTEP, B_LBO, B_SBO);
-          umma_bf16(tmem_d, ad, bd, IDESC, (kb > kb0 || k > 0) ? 1u : 0u);
+          if constexpr (CG == 2) umma_bf16_pair(tmem_d, ad, bd, IDESC, (kb > kb0 || k > 0) ? 1u : 0u);
+          else umma_bf16(tmem_d, ad, bd, IDESC, (kb > kb0 || k > 0) ? 1u : 0u);
         }
-        umma_commit(empty_bar(stage));
+        if constexpr (CG == 2) umma_commit_pair_both(empty_bar(stage));
+        else umma_commit(empty_bar(stage));
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
       if (!ok) break;
-      umma_commit(tfull_bar(acc));
+      if constexpr (CG == 2) umma_commit_pair_both(tfull_bar(acc));
+      else umma_commit(tfull_bar(acc));
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
     if (!ok) {
@@ -253,7 +277,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       atomicOr(err, GPT_DEVERR_TIMEOUT);
     }
     // drain: all MMAs this thread issued have completed once this commit arrives
-    umma_commit(drain_bar);
+    if constexpr (CG == 2) umma_commit_pair_local(drain_bar);
+    else umma_commit(drain_bar);
     volatile int never = 0;
     mbar_wait(drain_bar, 0, &never, 1ll << 28);
   } else if (warp >= 2) {
@@ -273,25 +298,31 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     uint32_t acc_phase = 0;
     bool ok = true;
     // side input: thread 0 loads sub-tile k into buffer k&1 one sub-tile ahead
-    int ld_u = blockIdx.x, ld_c = 0, issued = 0;
+    int ld_u = cid, ld_c = 0, issued = 0;
     auto issue_side = [&]() {
       if (ld_u >= units) return;
       const int t = ld_u % tiles;
-      const int m0 = (t % tiles_m) * TC_BM, n0 = (t / tiles_m) * BN;
+      const int m0 = (t % tiles_m) * TM + TC_BM * (int)rank, n0 = (t / tiles_m) * BN;
       const uint32_t sb = side_bar(issued & 1);
       mbar_expect_tx(sb, EPI_BUF_BYTES);
       tma_load_2d(rbase + (issued & 1) * EPI_BUF_BYTES, &tmC2, sb, n0 + ld_c, m0);
       ++issued;
       ld_c += SW;
-      if (ld_c >= BN || n0 + ld_c >= N) { ld_c = 0; ld_u += gridDim.x; }
+      if (ld_c >= BN || n0 + ld_c >= N) { ld_c = 0; ld_u += ncl; }
     };
     if (Tr::SIDE && etid == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmC2)) : "memory");
       issue_side();
     }
-    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    // the even CTA's barrier that frees an accumulator (both CTAs' epilogues arrive)
+    auto tempty_arrive = [&](int a) {
+      if constexpr (CG == 2) mbar_arrive_cluster(cluster_addr(tempty_bar(a), 0));
+      else mbar_arrive(tempty_bar(a));
+    };
+    for (int u = cid; u < units && ok; u += ncl) {
       const int split = u / tiles, t = u % tiles;
-      const int m0 = (t % tiles_m) * TC_BM, n0 = (t / tiles_m) * BN;
+      const int m0 = (t % tiles_m) * TM + TC_BM * (int)rank, n0 = (t / tiles_m) * BN;
+      const bool rows_in = m0 < M;   // a pair's second half can lie past the last row
       // this tile's bias: fetched before the accumulator wait, written to shared
       // memory after it (every thread has finished the previous tile's reads:
       // they precede its last group barrier)
@@ -321,7 +352,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if (c + SW >= BN || col0 + SW >= N) {   // last sub-tile: the accumulator can be reused
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(tempty_bar(acc));
+          if (lane == 0) tempty_arrive(acc);
         }
         // the store that last used this staging buffer has read it
         if (etid == 0) bulk_wait_read<1>();
@@ -380,7 +411,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
         fence_async_smem();
         if (!epi_sync(group_bar, gph, abort_flag)) { ok = false; break; }
-        if (etid == 0) {
+        if (etid == 0 && rows_in) {
           if constexpr (KIND == EPI_F32_SPLIT) {
             tma_store_3d(&tmC, b0, col0, m0, split);
           } else {
@@ -409,9 +440,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   }
   tc_fence_before();
   __syncthreads();
+  // a pair leaves together: the even CTA's MMAs read the odd CTA's shared
+  // memory and write its TMEM until the drain above
+  if constexpr (CG == 2) cluster_sync_all();
   tc_fence_after();
   if (warp == 0) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(Cfg::TMEM_COLS));
+    if constexpr (CG == 2)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(Cfg::TMEM_COLS));
+    else
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(Cfg::TMEM_COLS));
   }
 }
 
@@ -426,50 +463,69 @@ bool gemm_tc_supported(int M, int N, int K, long lda, bool a_t, long ldb, bool b
 
 static int g_sms = 0;
 
-template <int BN, bool A_MN, bool B_MN, int KIND>
+template <int BN, bool A_MN, bool B_MN, int KIND, int CG>
 static cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc,
                              const CUtensorMap& tc2, int M, int N, int K, int splits, const EpiParams<bf16>& epi,
                              unsigned* err, cudaStream_t s) {
-  using Cfg = TcCfg<BN, KIND>;
+  using Cfg = TcCfg<BN, KIND, CG>;
+  auto kern = gemm_tc_kernel<BN, A_MN, B_MN, KIND, CG>;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, A_MN, B_MN, KIND>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  int units = ((M + TC_BM - 1) / TC_BM) * ((N + BN - 1) / BN) * splits;
-  int grid = units < g_sms ? units : g_sms;
+  const int units = ((M + TC_BM * CG - 1) / (TC_BM * CG)) * ((N + BN - 1) / BN) * splits;
+  const int slots = g_sms / CG;
+  const int grid = CG * (units < slots ? units : slots);
   ++g_kernel_launches;
-  gemm_tc_kernel<BN, A_MN, B_MN, KIND><<<grid, TC_THREADS, Cfg::SMEM, s>>>(ta, tb, tc, tc2, M, N, K, splits, epi,
-                                                                          err);
-  return cudaGetLastError();
+  if constexpr (CG == 1) {
+    kern<<<grid, TC_THREADS, Cfg::SMEM, s>>>(ta, tb, tc, tc2, M, N, K, splits, epi, err);
+    return cudaGetLastError();
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(TC_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = Cfg::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute la[1];
+    la[0].id = cudaLaunchAttributeClusterDimension;
+    la[0].val.clusterDim.x = 2;
+    la[0].val.clusterDim.y = 1;
+    la[0].val.clusterDim.z = 1;
+    cfg.attrs = la;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, tc2, M, N, K, splits, epi, err);
+  }
 }
 
 // The (layout, epilogue) combinations the training step and the stand-alone
 // GEMM use; any other returns cudaErrorNotSupported.
-template <int BN, bool A_MN, bool B_MN>
+template <int BN, bool A_MN, bool B_MN, int CG>
 static cudaError_t launch_kind(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc,
                                const CUtensorMap& tc2, int M, int N, int K, int splits, const EpiParams<bf16>& epi,
                                unsigned* err, cudaStream_t s) {
-  if (epi.kind == EPI_F32) return launch_tc<BN, A_MN, B_MN, EPI_F32>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+  if (epi.kind == EPI_F32) return launch_tc<BN, A_MN, B_MN, EPI_F32, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
   if constexpr (!A_MN) {
     if (epi.kind == EPI_STORE && epi.resid)
-      return launch_tc<BN, A_MN, B_MN, EPI_STORE_RES>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
-    if (epi.kind == EPI_STORE) return launch_tc<BN, A_MN, B_MN, EPI_STORE>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+      return launch_tc<BN, A_MN, B_MN, EPI_STORE_RES, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+    if (epi.kind == EPI_STORE)
+      return launch_tc<BN, A_MN, B_MN, EPI_STORE, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
     if constexpr (!B_MN) {
-      if (epi.kind == EPI_GELU) return launch_tc<BN, A_MN, B_MN, EPI_GELU>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+      if (epi.kind == EPI_GELU)
+        return launch_tc<BN, A_MN, B_MN, EPI_GELU, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
     } else {
-      if (epi.kind == EPI_DGELU) return launch_tc<BN, A_MN, B_MN, EPI_DGELU>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+      if (epi.kind == EPI_DGELU)
+        return launch_tc<BN, A_MN, B_MN, EPI_DGELU, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
     }
   } else if constexpr (B_MN) {
     if (epi.kind == EPI_F32_SPLIT)
-      return launch_tc<BN, A_MN, B_MN, EPI_F32_SPLIT>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+      return launch_tc<BN, A_MN, B_MN, EPI_F32_SPLIT, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
   }
   return cudaErrorNotSupported;
 }
 
-template <int BN>
+template <int BN, int CG>
 static cudaError_t launch_bn(int M, int N, int K, const bf16* A, long lda, bool a_t, const bf16* B, long ldb,
                              bool b_t, const EpiParams<bf16>& epi, int splits, unsigned* err, cudaStream_t s) {
   CUtensorMap ta, tb, tc, tc2;
@@ -477,7 +533,8 @@ static cudaError_t launch_bn(int M, int N, int K, const bf16* A, long lda, bool 
   // A: K-major [M rows][K cols] (box 64 x 128) or MN-major [K rows][M cols] (box 64 x 64)
   ok = a_t ? make_map(&ta, A, K, M, lda, 64, TC_BK) : make_map(&ta, A, M, K, lda, TC_BK, TC_BM);
   if (!ok) return cudaErrorInvalidValue;
-  ok = b_t ? make_map(&tb, B, K, N, ldb, 64, TC_BK) : make_map(&tb, B, N, K, ldb, TC_BK, BN);
+  // B: K-major [N rows][K cols] (box 64 x BN/CG: a pair splits the tile's columns) or MN-major (box 64 x 64)
+  ok = b_t ? make_map(&tb, B, K, N, ldb, 64, TC_BK) : make_map(&tb, B, N, K, ldb, TC_BK, BN / CG);
   if (!ok) return cudaErrorInvalidValue;
   // output boxes: 128 rows x 128 bytes (64 bf16 or 32 fp32 columns), 128-byte swizzle
   switch (epi.kind) {
@@ -507,10 +564,10 @@ static cudaError_t launch_bn(int M, int N, int K, const bf16* A, long lda, bool 
       ok = false;
   }
   if (!ok) return cudaErrorInvalidValue;
-  if (!a_t && !b_t) return launch_kind<BN, false, false>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
-  if (!a_t && b_t) return launch_kind<BN, false, true>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
-  if (a_t && b_t) return launch_kind<BN, true, true>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
-  return launch_kind<BN, true, false>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+  if (!a_t && !b_t) return launch_kind<BN, false, false, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+  if (!a_t && b_t) return launch_kind<BN, false, true, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+  if (a_t && b_t) return launch_kind<BN, true, true, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+  return launch_kind<BN, true, false, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
 }
 
 cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* A, long lda, bool a_t, const bf16* B, long ldb,
@@ -541,6 +598,16 @@ cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* A, long lda, bool a_
     return (double)units * per / ((double)waves * g_sms * 256);
   };
   bool use128 = N <= 128 || eff(u128, 128) > eff(u256, 256) * 1.15;
-  if (use128) return launch_bn<128>(M, N, K, A, lda, a_t, B, ldb, b_t, epi, splits, err, s);
-  return launch_bn<256>(M, N, K, A, lda, a_t, B, ldb, b_t, epi, splits, err, s);
+  if (use128) return launch_bn<128, 1>(M, N, K, A, lda, a_t, B, ldb, b_t, epi, splits, err, s);
+  // 256-row tiles on CTA pairs: each SM streams half of B, so the MMA is not
+  // held back by shared-memory bandwidth; taken unless the pairs fill the
+  // machine much worse than single CTAs
+  long u2 = ((M + 255) / 256) * ((N + 255) / 256) * splits;
+  auto eff2 = [](long units) {
+    long slots = g_sms / 2, waves = (units + slots - 1) / slots;
+    return (double)units / ((double)waves * slots);
+  };
+  bool pair = M > 128 && eff2(u2) * 1.2 >= eff(u256, 256);
+  if (pair) return launch_bn<256, 2>(M, N, K, A, lda, a_t, B, ldb, b_t, epi, splits, err, s);
+  return launch_bn<256, 1>(M, N, K, A, lda, a_t, B, ldb, b_t, epi, splits, err, s);
 }

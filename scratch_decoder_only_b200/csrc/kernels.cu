@@ -513,8 +513,62 @@ __global__ void __launch_bounds__(256) colsum_kernel(const Tin* __restrict__ x, 
   }
 }
 
+// bf16 column sums with 16-byte loads: a block covers 256 columns (32 lanes
+// x 8 columns) and CS2_ROWS rows split over 8 warps, four rows in flight per
+// thread; one partial row per block row-chunk.
+#define CS2_ROWS 512
+__global__ void __launch_bounds__(256) colsum_bf16_kernel(const bf16* __restrict__ x, long ldx, int M, int N,
+                                                         float* __restrict__ partials) {
+  __shared__ float red[8][257];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c0 = blockIdx.x * 256 + lane * 8;
+  const int rb = blockIdx.y * CS2_ROWS, re = min(M, rb + CS2_ROWS);
+  float a[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) a[j] = 0.f;
+  if (c0 < N) {
+    int r = rb + warp;
+    for (; r + 24 < re; r += 32) {
+      uint4 w[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) w[u] = *reinterpret_cast<const uint4*>(x + (long)(r + 8 * u) * ldx + c0);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        float v[8];
+        Vec<bf16>::load(reinterpret_cast<const bf16*>(&w[u]), v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) a[j] += v[j];
+      }
+    }
+    for (; r < re; r += 8) {
+      float v[8];
+      Vec<bf16>::load(x + (long)r * ldx + c0, v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[j] += v[j];
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) red[warp][lane * 8 + j] = a[j];
+  __syncthreads();
+  const int c = blockIdx.x * 256 + threadIdx.x;
+  float acc = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) acc += red[w][threadIdx.x];
+  if (c < N) partials[(long)blockIdx.y * N + c] = acc;
+}
+
 template <typename Tin>
 cudaError_t launch_colsum(const Tin* x, long ldx, int M, int N, float* partials, float* out, cudaStream_t s) {
+  if constexpr (sizeof(Tin) == 2) {
+    if (N % 8 == 0 && ldx % 8 == 0 && ((uintptr_t)x & 15) == 0) {
+      dim3 g2((N + 255) / 256, (M + CS2_ROWS - 1) / CS2_ROWS);
+      ++g_kernel_launches;
+      colsum_bf16_kernel<<<g2, 256, 0, s>>>(reinterpret_cast<const bf16*>(x), ldx, M, N, partials);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+      return launch_reduce_rows(partials, g2.y, N, N, out, s);
+    }
+  }
   dim3 grid((N + 127) / 128, (M + CS_ROWS - 1) / CS_ROWS);
   ++g_kernel_launches;
   colsum_kernel<Tin><<<grid, 256, 0, s>>>(x, ldx, M, N, partials);
