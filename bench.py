@@ -177,6 +177,13 @@ def job_throughput(tokens_per_rank_step: int, steps: int, world: int, max_ms: fl
 
 # ----------------------------------------------------------------------------- our arm
 
+# DRAM bytes per GEMM launch of the training step at batch 16: the cold-cache
+# ncu capture of all 147 GEMM launches of a batch-4 step (37.67 MB per
+# launch, profiles/gemm_tc_traffic_b4.txt) scaled by the 4x token count.
+# Re-measure, or set to None, whenever the GEMM kernel changes.
+GEMM_TRAFFIC_BYTES_PER_LAUNCH = 150.7e6
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -258,7 +265,10 @@ def run_ours(args, rank, world, local_rank):
     g_n = sum(v["launches"] for k, v in prof.items() if k.startswith("gemm"))
     achieved = g_fl / (g_ms / 1000.0) / 1e12 if g_ms > 0 else 0.0
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
-                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"], "traffic": None,
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"],
+                "traffic": GEMM_TRAFFIC_BYTES_PER_LAUNCH if B == WL.batch else None,
+                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum over the 147 GEMM launches of "
+                                  "a batch-4 step, per launch, x4 for batch 16 (profiles/gemm_tc_traffic_b4.txt)",
                 "kernel": "gemm_tc (all GEMM launches)", "launches": g_n,
                 "avg_launch_ms": g_ms / max(1, g_n), "peak_source": peaks["source"] + " sustained",
                 "measured": "CUDA events around each launch in a second timed region of the same K steps "
