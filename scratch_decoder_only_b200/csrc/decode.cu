@@ -131,67 +131,155 @@ cudaError_t launch_kv_fill(const T* qkv, T* kc, T* vc, int B, int Tp, int H, int
   return cudaGetLastError();
 }
 
-// One query per (row, head) against keys 0..pos; the new key/value (at pos)
-// is appended to the cache by the same warp.
+// Split decode attention: grid (B*H, DA_SPLITS); block (bh, sp) takes keys
+// sp, sp + DA_SPLITS, ... in chunks of DA_CHUNK and keeps an online softmax
+// (max, sum, output) per 8-lane group, each lane holding 8 of the head's
+// dimensions (one 16-byte load of a key or value row).  Its partial
+// (m, l, o[D]) goes to part[bh][sp]; dec_attn_combine merges the splits.
+// The new key / value of this step are read from qkv, and written to the
+// cache by split 0.
+#define DA_SPLITS 16
+#define DA_THREADS 128
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float* v) {
+#pragma unroll
+  for (int i = 0; i < 8; i += Vec<T>::N) Vec<T>::load(p + i, v + i);
+}
 template <typename T, int D>
-__global__ void dec_attn_kernel(const T* __restrict__ qkv, T* kc, T* vc, T* __restrict__ out, int B, int H,
-                                int Tmax, int pos0, const int* __restrict__ step) {
-  int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+__global__ void __launch_bounds__(DA_THREADS)
+dec_attn_split_kernel(const T* __restrict__ qkv, T* kc, T* vc, float* __restrict__ part, int B, int H, int Tmax,
+                      int pos0, const int* __restrict__ step) {
+  static_assert(D % 8 == 0 && D <= 256, "head size");
+  constexpr int LPK = D / 8;            // lanes per key row (16 bytes each)
+  constexpr int KPW = 32 / LPK;         // keys per warp pass
+  constexpr int NW = DA_THREADS / 32;
   int pos = pos0 + *step;
   if (pos < 0) pos = 0;
   if (pos >= Tmax) pos = Tmax - 1;
-  int bh = blockIdx.x * 4 + warp;
-  if (bh >= B * H) return;
-  int b = bh / H, h = bh % H;
+  const int bh = blockIdx.x, sp = blockIdx.y;
+  const int b = bh / H, h = bh % H;
   const int C = H * D;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = lane / LPK, sub = lane % LPK;
   const T* q = qkv + (long)b * 3 * C + h * D;
   const T* knew = q + C;
   const T* vnew = q + 2 * C;
   T* kcb = kc + (long)bh * Tmax * D;
   T* vcb = vc + (long)bh * Tmax * D;
-  for (int i = lane; i < D; i += 32) {
-    kcb[(long)pos * D + i] = knew[i];
-    vcb[(long)pos * D + i] = vnew[i];
+  if (sp == 0 && threadIdx.x < D) {
+    kcb[(long)pos * D + threadIdx.x] = knew[threadIdx.x];
+    vcb[(long)pos * D + threadIdx.x] = vnew[threadIdx.x];
   }
-  const float scale = 1.0f / sqrtf((float)D);
-  float qv[D];
+  const float scale = rsqrtf((float)D);
+  float qv[8];
+  load8(q + sub * 8, qv);
 #pragma unroll
-  for (int i = 0; i < D; ++i) qv[i] = to_f(q[i]) * scale;
-  float mloc = -INFINITY, sloc = 0.f, acc[D];
+  for (int i = 0; i < 8; ++i) qv[i] *= scale;
+  float m = -INFINITY, l = 0.f, o[8];
 #pragma unroll
-  for (int i = 0; i < D; ++i) acc[i] = 0.f;
-  for (int j = lane; j <= pos; j += 32) {
+  for (int i = 0; i < 8; ++i) o[i] = 0.f;
+  // key j belongs to this split when (j / KPW) % (DA_SPLITS * NW) == sp * NW + warp
+  for (int j0 = (sp * NW + warp) * KPW; j0 <= pos; j0 += DA_SPLITS * NW * KPW) {
+    const int j = j0 + grp;
+    const bool live = j <= pos;
     const T* kr = j == pos ? knew : kcb + (long)j * D;
     const T* vr = j == pos ? vnew : vcb + (long)j * D;
+    float kv[8], vv[8];
+    if (live) {
+      load8(kr + sub * 8, kv);
+      load8(vr + sub * 8, vv);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { kv[i] = 0.f; vv[i] = 0.f; }
+    }
     float sc = 0.f;
 #pragma unroll
-    for (int i = 0; i < D; ++i) sc = fmaf(qv[i], to_f(kr[i]), sc);
-    float mn = fmaxf(mloc, sc);
-    float corr = expf(mloc - mn), p = expf(sc - mn);
-    sloc = sloc * corr + p;
+    for (int i = 0; i < 8; ++i) sc = fmaf(qv[i], kv[i], sc);
 #pragma unroll
-    for (int i = 0; i < D; ++i) acc[i] = acc[i] * corr + p * to_f(vr[i]);
-    mloc = mn;
+    for (int o2 = LPK / 2; o2 > 0; o2 >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o2);
+    if (live) {
+      const float mn = fmaxf(m, sc);
+      const float corr = expf(m - mn), p = expf(sc - mn);
+      l = l * corr + p;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = o[i] * corr + p * vv[i];
+      m = mn;
+    }
   }
-  float mw = warp_max(mloc);
-  float f = mloc == -INFINITY ? 0.f : expf(mloc - mw);
-  float ssum = warp_sum(sloc * f);
+  // merge the key groups of the warp (lanes with the same sub hold the same dimensions)
 #pragma unroll
-  for (int i = 0; i < D; ++i) {
-    float v = warp_sum(acc[i] * f);
-    if ((i & 31) == lane) out[(long)b * C + h * D + i] = from_f<T>(v / ssum);
+  for (int o2 = LPK; o2 < 32; o2 <<= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o2);
+    const float l2 = __shfl_xor_sync(0xffffffffu, l, o2);
+    const float mn = fmaxf(m, m2);
+    const float f1 = m == -INFINITY ? 0.f : expf(m - mn), f2 = m2 == -INFINITY ? 0.f : expf(m2 - mn);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = o[i] * f1 + __shfl_xor_sync(0xffffffffu, o[i], o2) * f2;
+    l = l * f1 + l2 * f2;
+    m = mn;
+  }
+  // merge the warps through shared memory
+  __shared__ float sm_m[NW], sm_l[NW], sm_o[NW][D];
+  if (lane < LPK) {
+    if (lane == 0) { sm_m[warp] = m; sm_l[warp] = l; }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) sm_o[warp][sub * 8 + i] = o[i];
+  }
+  __syncthreads();
+  float* dst = part + ((long)bh * DA_SPLITS + sp) * (D + 2);
+  if (threadIdx.x < D) {
+    float mm = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) mm = fmaxf(mm, sm_m[w]);
+    float ll = 0.f, oo = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float f = sm_m[w] == -INFINITY ? 0.f : expf(sm_m[w] - mm);
+      ll += sm_l[w] * f;
+      oo += sm_o[w][threadIdx.x] * f;
+    }
+    dst[2 + threadIdx.x] = oo;
+    if (threadIdx.x == 0) { dst[0] = mm; dst[1] = ll; }
   }
 }
 
+// out[b, head h] = merge of the DA_SPLITS partials of (b, h).
+template <typename T, int D>
+__global__ void dec_attn_combine_kernel(const float* __restrict__ part, T* __restrict__ out, int H) {
+  const int bh = blockIdx.x, b = bh / H, h = bh % H;
+  const float* p = part + (long)bh * DA_SPLITS * (D + 2);
+  float mm = -INFINITY;
+  for (int s2 = 0; s2 < DA_SPLITS; ++s2) mm = fmaxf(mm, p[s2 * (D + 2)]);
+  for (int i = threadIdx.x; i < D; i += blockDim.x) {
+    float ll = 0.f, oo = 0.f;
+    for (int s2 = 0; s2 < DA_SPLITS; ++s2) {
+      const float ms = p[s2 * (D + 2)];
+      const float f = ms == -INFINITY ? 0.f : expf(ms - mm);
+      ll += p[s2 * (D + 2) + 1] * f;
+      oo += p[s2 * (D + 2) + 2 + i] * f;
+    }
+    out[(long)b * H * D + h * D + i] = from_f<T>(oo / ll);
+  }
+}
+
+size_t dec_attn_part_floats(int B, int H, int d) { return (size_t)B * H * DA_SPLITS * (d + 2); }
+
 template <typename T>
-cudaError_t launch_dec_attn(const T* qkv, T* kc, T* vc, T* out, int B, int H, int d, int Tmax, int pos0,
+cudaError_t launch_dec_attn(const T* qkv, T* kc, T* vc, T* out, float* part, int B, int H, int d, int Tmax, int pos0,
                             const int* step, cudaStream_t s) {
-  unsigned g = (B * H + 3) / 4;
+  dim3 g(B * H, DA_SPLITS);
   switch (d) {
-    case 16: ++g_kernel_launches; dec_attn_kernel<T, 16><<<g, 128, 0, s>>>(qkv, kc, vc, out, B, H, Tmax, pos0, step); break;
-    case 32: ++g_kernel_launches; dec_attn_kernel<T, 32><<<g, 128, 0, s>>>(qkv, kc, vc, out, B, H, Tmax, pos0, step); break;
-    case 64: ++g_kernel_launches; dec_attn_kernel<T, 64><<<g, 128, 0, s>>>(qkv, kc, vc, out, B, H, Tmax, pos0, step); break;
-    case 128: ++g_kernel_launches; dec_attn_kernel<T, 128><<<g, 128, 0, s>>>(qkv, kc, vc, out, B, H, Tmax, pos0, step); break;
+#define DA_CASE(DD)                                                                                               \
+  case DD:                                                                                                        \
+    g_kernel_launches += 2;                                                                                       \
+    dec_attn_split_kernel<T, DD><<<g, DA_THREADS, 0, s>>>(qkv, kc, vc, part, B, H, Tmax, pos0, step);             \
+    dec_attn_combine_kernel<T, DD><<<B * H, 64, 0, s>>>(part, out, H);                                            \
+    break;
+    DA_CASE(16)
+    DA_CASE(32)
+    DA_CASE(64)
+    DA_CASE(128)
+#undef DA_CASE
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -270,7 +358,7 @@ cudaError_t launch_gather_last(const T* x, int B, int Tp, int C, T* out, cudaStr
   template cudaError_t launch_gemv<T>(const T*, int, int, const T*, int, const float*, const T*, int, T*, T*, \
                                       float*, cudaStream_t);                                             \
   template cudaError_t launch_kv_fill<T>(const T*, T*, T*, int, int, int, int, int, cudaStream_t);         \
-  template cudaError_t launch_dec_attn<T>(const T*, T*, T*, T*, int, int, int, int, int, const int*,      \
+  template cudaError_t launch_dec_attn<T>(const T*, T*, T*, T*, float*, int, int, int, int, int, const int*,      \
                                           cudaStream_t);                                                 \
   template cudaError_t launch_gather_last<T>(const T*, int, int, int, T*, cudaStream_t);
 INSTD(float)

@@ -51,7 +51,7 @@ struct gpt_model {
   int normblk = 592;
   DevScalars* sc;
   void *kc, *vc, *dx, *dh, *dq, *datt, *du, *da, *dxf;
-  float *dlogits, *dmu, *drs;
+  float *dlogits, *dmu, *drs, *dpart;
   int* dtok;
   int fwd_B = 0, fwd_T = 0;
   bool have_targets = false, logits_valid = false;
@@ -287,6 +287,7 @@ static int build_arena(gpt_model* m) {
   cv.add((void**)&m->dmu, Bx * 4);
   cv.add((void**)&m->drs, Bx * 4);
   cv.add((void**)&m->dtok, Bx * 4);
+  cv.add((void**)&m->dpart, dec_attn_part_floats((int)Bx, m->H, m->d) * 4);
   m->arena_bytes = cv.off + 256;
   cudaError_t e = cudaMalloc((void**)&m->arena, m->arena_bytes);
   if (e != cudaSuccess) {
@@ -546,6 +547,23 @@ static int backward_impl(gpt_model* m) {
 // ---------------------------------------------------------------------------
 // Greedy decoding
 // ---------------------------------------------------------------------------
+// One projection of a decode step: y = x W^T with the gemv epilogue `mode`
+// (0: + bias + residual, 1: u = + bias and gelu(u), 2: fp32 logits).  A batch
+// of more than 8 rows runs on the tensor-core GEMM (rows past B are zero
+// tiles), fewer rows on the GEMV that streams each weight row once.
+template <typename T>
+static cudaError_t dec_proj(gpt_model* m, const T* X, int B, int K, const T* W, int N, const float* bias,
+                            const T* resid, int mode, T* out, T* out2, float* outf, cudaStream_t s) {
+  if constexpr (sizeof(T) == 2) {
+    if (B > 8 && gemm_tc_supported(B, N, K, K, false, K, false)) {
+      EpiParams<T> e = mode == 2 ? epi_f32<T>(outf, N)
+                                 : mode == 1 ? epi_gelu<T>(out, out2, N, bias) : epi_store<T>(out, N, bias, resid, N);
+      return launch_gemm_tc(B, N, K, X, K, false, W, K, false, e, 1, &m->sc->err, s);
+    }
+  }
+  return launch_gemv<T>(X, B, K, W, N, bias, resid, mode, out, out2, outf, s);
+}
+
 template <typename T>
 static int decode_step(gpt_model* m, int B, int Tp, int n_new, int32_t* out, cudaStream_t s) {
   Acts<T> A(m);
@@ -562,15 +580,15 @@ static int decode_step(gpt_model* m, int B, int Tp, int n_new, int32_t* out, cud
   for (int l = 0; l < m->NL; ++l) {
     const LayerOff& lo = m->L[l];
     CK(launch_ln_fwd<T>(x, A.P(lo.ln1_g), A.P(lo.ln1_b), h, m->dmu, m->drs, B, C, eps, s));
-    CK(launch_gemv<T>(h, B, C, A.W(lo.w_qkv), 3 * C, A.P(lo.b_qkv), nullptr, 0, q, nullptr, nullptr, s));
-    CK(launch_dec_attn<T>(q, kc + l * kvl, vc + l * kvl, att, B, H, d, m->Tmax, Tp - 1, stepc, s));
-    CK(launch_gemv<T>(att, B, C, A.W(lo.w_o), C, A.P(lo.b_o), x, 0, x, nullptr, nullptr, s));
+    CK(dec_proj<T>(m, h, B, C, A.W(lo.w_qkv), 3 * C, A.P(lo.b_qkv), nullptr, 0, q, nullptr, nullptr, s));
+    CK(launch_dec_attn<T>(q, kc + l * kvl, vc + l * kvl, att, m->dpart, B, H, d, m->Tmax, Tp - 1, stepc, s));
+    CK(dec_proj<T>(m, att, B, C, A.W(lo.w_o), C, A.P(lo.b_o), x, 0, x, nullptr, nullptr, s));
     CK(launch_ln_fwd<T>(x, A.P(lo.ln2_g), A.P(lo.ln2_b), h, m->dmu, m->drs, B, C, eps, s));
-    CK(launch_gemv<T>(h, B, C, A.W(lo.w_fc), F, A.P(lo.b_fc), nullptr, 1, u, a, nullptr, s));
-    CK(launch_gemv<T>(a, B, F, A.W(lo.w_fc2), C, A.P(lo.b_fc2), x, 0, x, nullptr, nullptr, s));
+    CK(dec_proj<T>(m, h, B, C, A.W(lo.w_fc), F, A.P(lo.b_fc), nullptr, 1, u, a, nullptr, s));
+    CK(dec_proj<T>(m, a, B, F, A.W(lo.w_fc2), C, A.P(lo.b_fc2), x, 0, x, nullptr, nullptr, s));
   }
   CK(launch_ln_fwd<T>(x, A.P(m->o_lnf_g), A.P(m->o_lnf_b), xf, m->dmu, m->drs, B, C, eps, s));
-  CK(launch_gemv<T>(xf, B, C, A.W(m->o_head), m->Vp, nullptr, nullptr, 2, nullptr, nullptr, m->dlogits, s));
+  CK(dec_proj<T>(m, xf, B, C, A.W(m->o_head), m->Vp, nullptr, nullptr, 2, nullptr, nullptr, m->dlogits, s));
   CK(launch_argmax(m->dlogits, B, m->V, m->Vp, m->dtok, out, n_new, stepc, s));
   CK(launch_step_advance(stepc, s));
   return GPT_OK;
@@ -588,8 +606,8 @@ static int decode_impl(gpt_model* m, const int32_t* prompt, int B, int Tp, int n
     CK(launch_kv_fill<T>(A.qkv(l), (T*)m->kc + l * kvl, (T*)m->vc + l * kvl, B, Tp, H, d, m->Tmax, s));
   // first new token: from the prefill's last position
   CK(launch_gather_last<T>((const T*)m->xf, B, Tp, C, (T*)m->dxf, s));
-  CK(launch_gemv<T>((const T*)m->dxf, B, C, A.W(m->o_head), m->Vp, nullptr, nullptr, 2, nullptr, nullptr,
-                    m->dlogits, s));
+  CK(dec_proj<T>(m, (const T*)m->dxf, B, C, A.W(m->o_head), m->Vp, nullptr, nullptr, 2, nullptr, nullptr,
+                 m->dlogits, s));
   CK(launch_argmax(m->dlogits, B, m->V, m->Vp, m->dtok, out, n_new, nullptr, s));
   if (n_new == 1) return GPT_OK;
   const int one = 1;

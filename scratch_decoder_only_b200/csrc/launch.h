@@ -111,8 +111,9 @@ cudaError_t launch_gemv(const T* X, int B, int K, const T* W, int N, const float
                         int mode, T* out, T* out2, float* outf, cudaStream_t s);
 template <typename T>
 cudaError_t launch_kv_fill(const T* qkv, T* kc, T* vc, int B, int Tp, int H, int d, int Tmax, cudaStream_t s);
+size_t dec_attn_part_floats(int B, int H, int d);
 template <typename T>
-cudaError_t launch_dec_attn(const T* qkv, T* kc, T* vc, T* out, int B, int H, int d, int Tmax, int pos0,
+cudaError_t launch_dec_attn(const T* qkv, T* kc, T* vc, T* out, float* part, int B, int H, int d, int Tmax, int pos0,
                             const int* step, cudaStream_t s);
 // out[b * out_ld + (*step or 0)] = argmax; tok[b] = argmax
 cudaError_t launch_argmax(const float* logits, int B, int V, int Vp, int* tok, int32_t* out, int out_ld,
