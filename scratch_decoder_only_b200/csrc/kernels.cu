@@ -15,15 +15,27 @@ unsigned long long g_kernel_launches = 0;
 // Position restarts at 0 at the first token of each document ("LucilleAI",
 // sequence packing); dstart[m] = row index of the first token of m's document.
 // ---------------------------------------------------------------------------
-__global__ void prep_kernel(const int32_t* __restrict__ tokens, const int32_t* __restrict__ targets,
-                            const int32_t* __restrict__ seg, int B, int T, int V, int* tok_out,
-                            int* tgt_out, int* pos_out, int* dstart_out, DevScalars* sc) {
-  int nv = 0;
+__global__ void __launch_bounds__(1024) prep_kernel(const int32_t* __restrict__ tokens,
+                                                    const int32_t* __restrict__ targets,
+                                                    const int32_t* __restrict__ seg, int B, int T, int V,
+                                                    int* tok_out, int* tgt_out, int* pos_out, int* dstart_out,
+                                                    DevScalars* sc) {
+  // one block per row; the document start of t is the largest run start <= t
+  // (an inclusive max-scan of "t if a document starts at t"), carried across
+  // chunks of blockDim.x positions
+  __shared__ int wscan[32];
+  __shared__ int carry_s;
+  __shared__ int nv_s[32];
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   unsigned err = 0;
-  for (int b = threadIdx.x; b < B; b += blockDim.x) {
-    int pos = 0, prev = 0;
-    for (int t = 0; t < T; ++t) {
-      long m = (long)b * T + t;
+  int nv = 0;
+  int carry = 0;
+  for (int t0 = 0; t0 < T; t0 += blockDim.x) {
+    const int t = t0 + threadIdx.x;
+    int start = 0;
+    if (t < T) {
+      const long m = (long)b * T + t;
       int tok = tokens[m];
       if (tok < 0 || tok >= V) { err |= GPT_DEVERR_TOKEN; tok = tok < 0 ? 0 : V - 1; }
       tok_out[m] = tok;
@@ -34,37 +46,67 @@ __global__ void prep_kernel(const int32_t* __restrict__ tokens, const int32_t* _
         nv += (tg >= 0);
       }
       if (seg) {
-        int sg = seg[m];
+        const int sg = seg[m];
         if (t > 0) {
-          if (sg < prev) err |= GPT_DEVERR_SEGMENT;
-          pos = (sg == prev) ? pos + 1 : 0;
+          const int pv = seg[m - 1];
+          if (sg < pv) err |= GPT_DEVERR_SEGMENT;
+          if (sg != pv) start = t;
         }
-        prev = sg;
-      } else {
-        pos = t;
       }
-      pos_out[m] = pos;
-      dstart_out[m] = t - pos;
     }
+    // inclusive max-scan over the chunk
+    int v = start;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v = max(v, u);
+    }
+    if (lane == 31) wscan[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+      int w = lane < nw ? wscan[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w = max(w, u);
+      }
+      if (lane < nw) wscan[lane] = w;
+    }
+    __syncthreads();
+    if (warp > 0) v = max(v, wscan[warp - 1]);
+    v = max(v, carry);
+    if (t < T) {
+      const long m = (long)b * T + t;
+      const int ds = seg ? v : 0;
+      dstart_out[m] = ds;
+      pos_out[m] = t - ds;
+    }
+    if (threadIdx.x == blockDim.x - 1) carry_s = v;
+    __syncthreads();
+    carry = carry_s;
+    __syncthreads();
   }
   if (err) atomicOr(&sc->err, err);
-  __shared__ int red[32];
   for (int o = 16; o > 0; o >>= 1) nv += __shfl_xor_sync(0xffffffffu, nv, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = nv;
+  if (lane == 0) nv_s[warp] = nv;
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0 && targets) {
     int tot = 0;
-    for (int w = 0; w < (int)(blockDim.x + 31) / 32; ++w) tot += red[w];
-    if (targets) sc->n_valid = tot;
+    for (int w = 0; w < nw; ++w) tot += nv_s[w];
+    atomicAdd(&sc->n_valid, tot);   // cleared before the launch
   }
 }
 
 cudaError_t launch_prep(const int32_t* tokens, const int32_t* targets, const int32_t* seg, int B, int T,
                         int V, int* tok_out, int* tgt_out, int* pos_out, int* dstart_out,
                         DevScalars* sc, cudaStream_t s) {
-  int th = B < 32 ? 32 : (B > 1024 ? 1024 : ((B + 31) / 32) * 32);
+  if (targets) {
+    cudaError_t e = cudaMemsetAsync(&sc->n_valid, 0, sizeof(int), s);
+    if (e != cudaSuccess) return e;
+  }
+  int th = T >= 1024 ? 1024 : ((T + 31) / 32) * 32;
   ++g_kernel_launches;
-  prep_kernel<<<1, th, 0, s>>>(tokens, targets, seg, B, T, V, tok_out, tgt_out, pos_out, dstart_out, sc);
+  prep_kernel<<<B, th, 0, s>>>(tokens, targets, seg, B, T, V, tok_out, tgt_out, pos_out, dstart_out, sc);
   return cudaGetLastError();
 }
 
@@ -444,35 +486,35 @@ cudaError_t launch_ln_bwd(const T* dy, const T* x, const float* mean, const floa
 
 // out[n] = sum over r of p[r * ld + n], in a fixed order (deterministic):
 // 32 columns per block, the rows split over 8 warps, 4 loads in flight.
-__global__ void __launch_bounds__(256) reduce_rows_kernel(const float* __restrict__ p, int rows, int N, long ld,
-                                                          float* __restrict__ out) {
-  __shared__ float red[8][33];
+__global__ void __launch_bounds__(1024) reduce_rows_kernel(const float* __restrict__ p, int rows, int N, long ld,
+                                                           float* __restrict__ out) {
+  __shared__ float red[32][33];
   int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int n = blockIdx.x * 32 + lane;
   float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
   if (n < N) {
     int r = warp;
-    for (; r + 24 < rows; r += 32) {
+    for (; r + 96 < rows; r += 128) {
       a0 += p[(long)r * ld + n];
-      a1 += p[(long)(r + 8) * ld + n];
-      a2 += p[(long)(r + 16) * ld + n];
-      a3 += p[(long)(r + 24) * ld + n];
+      a1 += p[(long)(r + 32) * ld + n];
+      a2 += p[(long)(r + 64) * ld + n];
+      a3 += p[(long)(r + 96) * ld + n];
     }
-    for (; r < rows; r += 8) a0 += p[(long)r * ld + n];
+    for (; r < rows; r += 32) a0 += p[(long)r * ld + n];
   }
   red[warp][lane] = (a0 + a1) + (a2 + a3);
   __syncthreads();
   if (warp == 0 && n < N) {
     float acc = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) acc += red[w][lane];
+    for (int w = 0; w < 32; ++w) acc += red[w][lane];
     out[n] = acc;
   }
 }
 
 cudaError_t launch_reduce_rows(const float* partials, int rows, int N, long ld, float* out, cudaStream_t s) {
   ++g_kernel_launches;
-  reduce_rows_kernel<<<(N + 31) / 32, 256, 0, s>>>(partials, rows, N, ld, out);
+  reduce_rows_kernel<<<(N + 31) / 32, 1024, 0, s>>>(partials, rows, N, ld, out);
   return cudaGetLastError();
 }
 
