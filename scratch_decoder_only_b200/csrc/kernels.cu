@@ -150,63 +150,103 @@ cudaError_t launch_embed_fwd(const int* tok, const int* pos, const float* wte, c
 // LayerNorm forward: one warp per row, the row kept in registers.  Biased
 // variance, y = (x - mean) * rstd * g + b; mean and rstd kept for backward.
 // ---------------------------------------------------------------------------
-template <typename T>
-__global__ void ln_fwd_kernel(const T* __restrict__ x, const float* __restrict__ g,
-                              const float* __restrict__ b, T* __restrict__ y, float* __restrict__ mean,
-                              float* __restrict__ rstd, int M, int C, float eps) {
+template <typename T, int NCH>
+__global__ void __launch_bounds__(256) ln_fwd_kernel(const T* __restrict__ x, const float* __restrict__ g,
+                                                     const float* __restrict__ b, T* __restrict__ y,
+                                                     float* __restrict__ mean, float* __restrict__ rstd, int M, int C,
+                                                     float eps) {
+  // one warp per row, warps walk rows with a grid stride; gamma and beta stay
+  // in registers and the next row's x is loaded before the current row is
+  // reduced (one memory latency per row, overlapped with the previous row)
   constexpr int NV = Vec<T>::N;
-  constexpr int NCH = LN_MAXC / (32 * NV);
-  int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  int lane = threadIdx.x & 31;
-  if (row >= M) return;
-  const T* xr = x + (long)row * C;
-  float v[NCH][NV];
-  float sum = 0.f;
-  int nch = C / NV;
+  const int lane = threadIdx.x & 31;
+  const int nch = C / NV;
+  const int stride = gridDim.x * (blockDim.x >> 5);
+  float gg[NCH][NV], bb[NCH][NV];
 #pragma unroll
   for (int i = 0; i < NCH; ++i) {
-    int ch = lane + i * 32;
-    if (ch < nch) {
-      Vec<T>::load(xr + ch * NV, v[i]);
+    const int ch = lane + i * 32;
+#pragma unroll
+    for (int j = 0; j < NV; j += 4) {
+      if (ch < nch) {
+        Vec<float>::load(g + ch * NV + j, gg[i] + j);
+        Vec<float>::load(b + ch * NV + j, bb[i] + j);
+      } else {
+        gg[i][j] = gg[i][j + 1] = gg[i][j + 2] = gg[i][j + 3] = 0.f;
+        bb[i][j] = bb[i][j + 1] = bb[i][j + 2] = bb[i][j + 3] = 0.f;
+      }
+    }
+  }
+  int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  uint4 nxt[NCH];
+  auto fetch = [&](int r) {
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int ch = lane + i * 32;
+      if (r < M && ch < nch) nxt[i] = *reinterpret_cast<const uint4*>(x + (long)r * C + ch * NV);
+    }
+  };
+  fetch(row);
+  for (; row < M; row += stride) {
+    float v[NCH][NV];
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      if (lane + i * 32 < nch) Vec<T>::load(reinterpret_cast<const T*>(&nxt[i]), v[i]);
+      else
+#pragma unroll
+        for (int j = 0; j < NV; ++j) v[i][j] = 0.f;
+    }
+    fetch(row + stride);
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i)
 #pragma unroll
       for (int j = 0; j < NV; ++j) sum += v[i][j];
-    }
-  }
-  float mu = warp_sum(sum) / C;
-  float sq = 0.f;
+    const float mu = warp_sum(sum) / C;
+    float sq = 0.f;
 #pragma unroll
-  for (int i = 0; i < NCH; ++i) {
-    int ch = lane + i * 32;
-    if (ch < nch) {
+    for (int i = 0; i < NCH; ++i) {
+      if (lane + i * 32 < nch) {
 #pragma unroll
-      for (int j = 0; j < NV; ++j) { float d = v[i][j] - mu; sq += d * d; }
-    }
-  }
-  float rs = 1.0f / sqrtf(warp_sum(sq) / C + eps);
-  T* yr = y + (long)row * C;
-#pragma unroll
-  for (int i = 0; i < NCH; ++i) {
-    int ch = lane + i * 32;
-    if (ch < nch) {
-      float o[NV], gg[NV], bb[NV];
-#pragma unroll
-      for (int j = 0; j < NV; j += 4) {
-        Vec<float>::load(g + ch * NV + j, gg + j);
-        Vec<float>::load(b + ch * NV + j, bb + j);
+        for (int j = 0; j < NV; ++j) { const float d = v[i][j] - mu; sq += d * d; }
       }
-#pragma unroll
-      for (int j = 0; j < NV; ++j) o[j] = (v[i][j] - mu) * rs * gg[j] + bb[j];
-      Vec<T>::store(yr + ch * NV, o);
     }
+    const float rs = 1.0f / sqrtf(warp_sum(sq) / C + eps);
+    T* yr = y + (long)row * C;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int ch = lane + i * 32;
+      if (ch < nch) {
+        float o[NV];
+#pragma unroll
+        for (int j = 0; j < NV; ++j) o[j] = (v[i][j] - mu) * rs * gg[i][j] + bb[i][j];
+        Vec<T>::store(yr + ch * NV, o);
+      }
+    }
+    if (lane == 0) { mean[row] = mu; rstd[row] = rs; }
   }
-  if (lane == 0) { mean[row] = mu; rstd[row] = rs; }
 }
 
 template <typename T>
 cudaError_t launch_ln_fwd(const T* x, const float* g, const float* b, T* y, float* mean, float* rstd,
                           int M, int C, float eps, cudaStream_t s) {
+  constexpr int NV = Vec<T>::N;
+  const int per = (C / NV + 31) / 32;   // 16-byte chunks per lane
+  int blocks = (M + 7) / 8;
+  if (blocks > 148 * 8) blocks = 148 * 8;
   ++g_kernel_launches;
-  ln_fwd_kernel<T><<<(M + 7) / 8, 256, 0, s>>>(x, g, b, y, mean, rstd, M, C, eps);
+#define LNF_CASE(K) \
+  case K: ln_fwd_kernel<T, K><<<blocks, 256, 0, s>>>(x, g, b, y, mean, rstd, M, C, eps); break;
+  switch (per) {
+    LNF_CASE(1)
+    LNF_CASE(2)
+    LNF_CASE(3)
+    LNF_CASE(4)
+    default:
+      if constexpr (NV >= 8) return cudaErrorInvalidValue;
+      else { ln_fwd_kernel<T, 8><<<blocks, 256, 0, s>>>(x, g, b, y, mean, rstd, M, C, eps); break; }
+  }
+#undef LNF_CASE
   return cudaGetLastError();
 }
 
