@@ -75,6 +75,33 @@ __device__ __forceinline__ float gelu_grad_f(float u) {
   return 0.5f * (1.0f + t) + 0.5f * u * (1.0f - t * t) * GELU_K * (1.0f + 3.0f * GELU_C * u * u);
 }
 
+// Programmatic dependent launch: a kernel launched with the programmatic
+// serialization attribute may start while its predecessor in the stream
+// finishes; griddep_wait() holds it until the predecessor has completed and
+// its writes are visible (a no-op for a normal launch), and
+// griddep_release() lets the successor start launching.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+extern bool g_pdl;   // set while the decode step is captured: its launches overlap their predecessors
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  if (!g_pdl) {
+    kern<<<grid, block, smem, s>>>(args...);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 __device__ __forceinline__ void set_dev_err(unsigned* err, unsigned bit) {
   if (err) atomicOr(err, bit);
 }

@@ -12,6 +12,8 @@ template <typename T>
 __global__ void dec_embed_kernel(const int* __restrict__ tok, const float* __restrict__ wte,
                                  const float* __restrict__ wpe, T* __restrict__ x, int C, int pos0,
                                  const int* __restrict__ step, int max_seq, unsigned* err) {
+  griddep_wait();
+  griddep_release();
   int b = blockIdx.x;
   int pos = pos0 + *step;
   if (pos < 0 || pos >= max_seq) {
@@ -27,7 +29,8 @@ template <typename T>
 cudaError_t launch_dec_embed(const int* tok, const float* wte, const float* wpe, T* x, int B, int C, int pos0,
                              const int* step, int max_seq, unsigned* err, cudaStream_t s) {
   ++g_kernel_launches;
-  dec_embed_kernel<T><<<B, 256, 0, s>>>(tok, wte, wpe, x, C, pos0, step, max_seq, err);
+  cudaError_t e = launch_k(dec_embed_kernel<T>, dim3(B), dim3(256), 0, s, tok, wte, wpe, x, C, pos0, step, max_seq, err);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -40,6 +43,8 @@ template <typename T, int BB>
 __global__ void __launch_bounds__(GEMV_WARPS * 32)
 gemv_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, int N,
             const float* __restrict__ bias, const T* resid, int mode, T* out, T* out2, float* outf) {
+  griddep_wait();
+  griddep_release();
   constexpr int KC = 8192 / BB;
   constexpr int NV = Vec<T>::N;
   __shared__ __align__(16) float xs[BB * KC];
@@ -100,11 +105,14 @@ template <typename T>
 cudaError_t launch_gemv(const T* X, int B, int K, const T* W, int N, const float* bias, const T* resid,
                         int mode, T* out, T* out2, float* outf, cudaStream_t s) {
   unsigned g = (N + GEMV_WARPS - 1) / GEMV_WARPS;
-  if (B <= 1) { ++g_kernel_launches; gemv_kernel<T, 1><<<g, GEMV_WARPS * 32, 0, s>>>(X, B, K, W, N, bias, resid, mode, out, out2, outf); }
-  else if (B <= 8) { ++g_kernel_launches; gemv_kernel<T, 8><<<g, GEMV_WARPS * 32, 0, s>>>(X, B, K, W, N, bias, resid, mode, out, out2, outf); }
-  else if (B <= 32) { ++g_kernel_launches; gemv_kernel<T, 32><<<g, GEMV_WARPS * 32, 0, s>>>(X, B, K, W, N, bias, resid, mode, out, out2, outf); }
+  cudaError_t e;
+  const dim3 gb(GEMV_WARPS * 32);
+  if (B <= 1) e = launch_k(gemv_kernel<T, 1>, dim3(g), gb, 0, s, X, B, K, W, N, bias, resid, mode, out, out2, outf);
+  else if (B <= 8) e = launch_k(gemv_kernel<T, 8>, dim3(g), gb, 0, s, X, B, K, W, N, bias, resid, mode, out, out2, outf);
+  else if (B <= 32) e = launch_k(gemv_kernel<T, 32>, dim3(g), gb, 0, s, X, B, K, W, N, bias, resid, mode, out, out2, outf);
   else return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  ++g_kernel_launches;
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // Copy the prompt's K and V (from the prefill's qkv [B*Tp, 3C]) into the cache.
@@ -149,6 +157,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(DA_THREADS)
 dec_attn_split_kernel(const T* __restrict__ qkv, T* kc, T* vc, float* __restrict__ part, int B, int H, int Tmax,
                       int pos0, const int* __restrict__ step) {
+  griddep_wait();
+  griddep_release();
   static_assert(D % 8 == 0 && D <= 256, "head size");
   constexpr int LPK = D / 8;            // lanes per key row (16 bytes each)
   constexpr int KPW = 32 / LPK;         // keys per warp pass
@@ -246,6 +256,8 @@ dec_attn_split_kernel(const T* __restrict__ qkv, T* kc, T* vc, float* __restrict
 // out[b, head h] = merge of the DA_SPLITS partials of (b, h).
 template <typename T, int D>
 __global__ void dec_attn_combine_kernel(const float* __restrict__ part, T* __restrict__ out, int H) {
+  griddep_wait();
+  griddep_release();
   const int bh = blockIdx.x, b = bh / H, h = bh % H;
   const float* p = part + (long)bh * DA_SPLITS * (D + 2);
   float mm = -INFINITY;
@@ -268,12 +280,13 @@ template <typename T>
 cudaError_t launch_dec_attn(const T* qkv, T* kc, T* vc, T* out, float* part, int B, int H, int d, int Tmax, int pos0,
                             const int* step, cudaStream_t s) {
   dim3 g(B * H, DA_SPLITS);
+  cudaError_t e = cudaSuccess;
   switch (d) {
 #define DA_CASE(DD)                                                                                               \
   case DD:                                                                                                        \
     g_kernel_launches += 2;                                                                                       \
-    dec_attn_split_kernel<T, DD><<<g, DA_THREADS, 0, s>>>(qkv, kc, vc, part, B, H, Tmax, pos0, step);             \
-    dec_attn_combine_kernel<T, DD><<<B * H, 64, 0, s>>>(part, out, H);                                            \
+    e = launch_k(dec_attn_split_kernel<T, DD>, g, dim3(DA_THREADS), 0, s, qkv, kc, vc, part, B, H, Tmax, pos0, step); \
+    if (e == cudaSuccess) e = launch_k(dec_attn_combine_kernel<T, DD>, dim3(B * H), dim3(64), 0, s, (const float*)part, out, H); \
     break;
     DA_CASE(16)
     DA_CASE(32)
@@ -282,13 +295,15 @@ cudaError_t launch_dec_attn(const T* qkv, T* kc, T* vc, T* out, float* part, int
 #undef DA_CASE
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // Greedy choice: argmax over the real vocabulary of fp32 logits, lowest
 // index on ties.  Writes tok[b] and out[b * out_ld + col].
 __global__ void argmax_kernel(const float* __restrict__ logits, int V, int Vp, int* tok, int32_t* out,
                               int out_ld, const int* __restrict__ step) {
+  griddep_wait();
+  griddep_release();
   int b = blockIdx.x;
   const int col = step ? *step : 0;
   const float* z = logits + (long)b * Vp;
@@ -328,14 +343,16 @@ __global__ void argmax_kernel(const float* __restrict__ logits, int V, int Vp, i
 cudaError_t launch_argmax(const float* logits, int B, int V, int Vp, int* tok, int32_t* out, int out_ld,
                           const int* step, cudaStream_t s) {
   ++g_kernel_launches;
-  argmax_kernel<<<B, 1024, 0, s>>>(logits, V, Vp, tok, out, out_ld, step);
+  cudaError_t e = launch_k(argmax_kernel, dim3(B), dim3(1024), 0, s, logits, V, Vp, tok, out, out_ld, step);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
-__global__ void step_advance_kernel(int* step) { *step += 1; }
+__global__ void step_advance_kernel(int* step) { griddep_wait(); griddep_release(); *step += 1; }
 cudaError_t launch_step_advance(int* step, cudaStream_t s) {
   ++g_kernel_launches;
-  step_advance_kernel<<<1, 1, 0, s>>>(step);
+  cudaError_t e = launch_k(step_advance_kernel, dim3(1), dim3(1), 0, s, step);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -623,7 +623,9 @@ static int decode_impl(gpt_model* m, const int32_t* prompt, int B, int Tp, int n
     cudaGraph_t g = nullptr;
     unsigned long long n0 = g_kernel_launches;
     CK(cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
+    g_pdl = true;   // each captured kernel may start while its predecessor drains
     int r = decode_step<T>(m, B, Tp, n_new, out, m->cap_stream);
+    g_pdl = false;
     cudaError_t ec = cudaStreamEndCapture(m->cap_stream, &g);
     if (r != GPT_OK) { if (g) cudaGraphDestroy(g); return r; }
     CK(ec);

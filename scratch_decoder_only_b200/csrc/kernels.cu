@@ -7,6 +7,7 @@
 #include "tc_common.cuh"
 
 unsigned long long g_kernel_launches = 0;
+bool g_pdl = false;
 
 #define LN_MAXC 1024   // largest d_model the register-resident LayerNorm handles
 
@@ -159,6 +160,8 @@ __global__ void __launch_bounds__(256) ln_fwd_kernel(const T* __restrict__ x, co
   // in registers and the next row's x is loaded before the current row is
   // reduced (one memory latency per row, overlapped with the previous row)
   constexpr int NV = Vec<T>::N;
+  griddep_wait();
+  griddep_release();
   const int lane = threadIdx.x & 31;
   const int nch = C / NV;
   const int stride = gridDim.x * (blockDim.x >> 5);
@@ -235,8 +238,9 @@ cudaError_t launch_ln_fwd(const T* x, const float* g, const float* b, T* y, floa
   int blocks = (M + 7) / 8;
   if (blocks > 148 * 8) blocks = 148 * 8;
   ++g_kernel_launches;
+  cudaError_t e = cudaSuccess;
 #define LNF_CASE(K) \
-  case K: ln_fwd_kernel<T, K><<<blocks, 256, 0, s>>>(x, g, b, y, mean, rstd, M, C, eps); break;
+  case K: e = launch_k(ln_fwd_kernel<T, K>, dim3(blocks), dim3(256), 0, s, x, g, b, y, mean, rstd, M, C, eps); break;
   switch (per) {
     LNF_CASE(1)
     LNF_CASE(2)
@@ -244,10 +248,10 @@ cudaError_t launch_ln_fwd(const T* x, const float* g, const float* b, T* y, floa
     LNF_CASE(4)
     default:
       if constexpr (NV >= 8) return cudaErrorInvalidValue;
-      else { ln_fwd_kernel<T, 8><<<blocks, 256, 0, s>>>(x, g, b, y, mean, rstd, M, C, eps); break; }
+      else { e = launch_k(ln_fwd_kernel<T, 8>, dim3(blocks), dim3(256), 0, s, x, g, b, y, mean, rstd, M, C, eps); break; }
   }
 #undef LNF_CASE
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
