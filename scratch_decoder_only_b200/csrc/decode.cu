@@ -101,13 +101,90 @@ gemv_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, int 
   }
 }
 
+// Small-batch form (B <= 8): each warp computes R consecutive outputs for all
+// rows, every lane streaming 16-byte chunks of the R weight rows and of X
+// straight from global memory (no staging, no block barrier), so a warp has
+// R weight chunks in flight per step of the k loop.
+template <typename T, int BB, int R>
+__global__ void __launch_bounds__(GEMV_WARPS * 32)
+gemv_rows_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, int N,
+                 const float* __restrict__ bias, const T* resid, int mode, T* out, T* out2, float* outf) {
+  griddep_wait();
+  griddep_release();
+  constexpr int NV = Vec<T>::N;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = (blockIdx.x * GEMV_WARPS + warp) * R;
+  if (n0 >= N) return;
+  float acc[R][BB];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int b = 0; b < BB; ++b) acc[r][b] = 0.f;
+#pragma unroll 4
+  for (int kk = lane * NV; kk < K; kk += 32 * NV) {
+    float w[R][NV];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (n0 + r < N) Vec<T>::load(W + (long)(n0 + r) * K + kk, w[r]);
+      else
+#pragma unroll
+        for (int j = 0; j < NV; ++j) w[r][j] = 0.f;
+    }
+#pragma unroll
+    for (int b = 0; b < BB; ++b) {
+      if (b < B) {
+        float x[NV];
+        Vec<T>::load(X + (long)b * K + kk, x);
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+          for (int j = 0; j < NV; ++j) acc[r][b] = fmaf(w[r][j], x[j], acc[r][b]);
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int n = n0 + r;
+#pragma unroll
+    for (int b = 0; b < BB; ++b) {
+      if (b < B) {
+        const float y = warp_sum(acc[r][b]);
+        if (lane == 0 && n < N) {
+          const long o = (long)b * N + n;
+          if (mode == 2) {
+            outf[o] = y;
+          } else if (mode == 1) {
+            const float u = y + bias[n];
+            const T uq = from_f<T>(u);
+            out[o] = uq;
+            out2[o] = from_f<T>(gelu_f(to_f(uq)));
+          } else {
+            const float v = y + (bias ? bias[n] : 0.f) + (resid ? to_f(resid[o]) : 0.f);
+            out[o] = from_f<T>(v);
+          }
+        }
+      }
+    }
+  }
+}
+
 template <typename T>
 cudaError_t launch_gemv(const T* X, int B, int K, const T* W, int N, const float* bias, const T* resid,
                         int mode, T* out, T* out2, float* outf, cudaStream_t s) {
   unsigned g = (N + GEMV_WARPS - 1) / GEMV_WARPS;
   cudaError_t e;
   const dim3 gb(GEMV_WARPS * 32);
-  if (B <= 1) e = launch_k(gemv_kernel<T, 1>, dim3(g), gb, 0, s, X, B, K, W, N, bias, resid, mode, out, out2, outf);
+  const bool chunks = K % Vec<T>::N == 0 && ((uintptr_t)X & 15) == 0 && ((uintptr_t)W & 15) == 0;
+  const unsigned g2 = (N + GEMV_WARPS * 2 - 1) / (GEMV_WARPS * 2), g4 = (N + GEMV_WARPS * 4 - 1) / (GEMV_WARPS * 4);
+  if (chunks && B <= 1 && N >= 4096)
+    e = launch_k(gemv_rows_kernel<T, 1, 4>, dim3(g4), gb, 0, s, X, B, K, W, N, bias, resid, mode, out, out2, outf);
+  else if (chunks && B <= 1)
+    e = launch_k(gemv_rows_kernel<T, 1, 2>, dim3(g2), gb, 0, s, X, B, K, W, N, bias, resid, mode, out, out2, outf);
+  else if (chunks && B <= 8 && N >= 4096)
+    e = launch_k(gemv_rows_kernel<T, 8, 4>, dim3(g4), gb, 0, s, X, B, K, W, N, bias, resid, mode, out, out2, outf);
+  else if (chunks && B <= 8)
+    e = launch_k(gemv_rows_kernel<T, 8, 2>, dim3(g2), gb, 0, s, X, B, K, W, N, bias, resid, mode, out, out2, outf);
+  else if (B <= 1) e = launch_k(gemv_kernel<T, 1>, dim3(g), gb, 0, s, X, B, K, W, N, bias, resid, mode, out, out2, outf);
   else if (B <= 8) e = launch_k(gemv_kernel<T, 8>, dim3(g), gb, 0, s, X, B, K, W, N, bias, resid, mode, out, out2, outf);
   else if (B <= 32) e = launch_k(gemv_kernel<T, 32>, dim3(g), gb, 0, s, X, B, K, W, N, bias, resid, mode, out, out2, outf);
   else return cudaErrorInvalidValue;
