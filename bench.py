@@ -149,8 +149,9 @@ def run_reference(args, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": steps, "warmup": args.warmup, "ms_per_step": 1000 * total / steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": WL.name, "global_batch": 1, "seq_len": 256,
-                                            "parallelism": "none (CPU oracle)"},
+            "data": "synthetic", "config": {"workload": WL.name, "global_batch": WL.batch * world, "seq_len": WL.seq,
+                                            "parallelism": "none (CPU oracle on the host cores)",
+                                            "timed_sample": "one row x 256 tokens of this workload per step"},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
