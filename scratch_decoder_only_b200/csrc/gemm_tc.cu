@@ -7,21 +7,24 @@
 // MN-major: both activations read transposed in place), so no transposed
 // copy of any tensor is ever written.
 //
-// Structure (one 192-thread CTA per SM, persistent over output tiles):
+// Structure (192-thread CTAs, persistent over output tiles; a CTA alone or a
+// cluster of two sharing one MMA stream):
 //   warp 0      TMA producer: 2-D tiled loads (128-byte swizzle) of A and B
 //               k-blocks into a ring of shared-memory stages, completion
 //               signalled on "full" mbarriers; also allocates tensor memory.
-//   warp 1      MMA issuer: one thread issues tcgen05.mma (kind::f16,
-//               M = 128, N = BN, K = 16) into a TMEM accumulator, and
-//               tcgen05.commit frees each stage ("empty") and hands a finished
-//               accumulator to the epilogue ("tfull").
+//   warp 1      MMA issuer: one thread issues tcgen05.mma (kind::f16, M = 128
+//               for a CTA, 256 for a pair, N = BN, K = 16) into a TMEM
+//               accumulator, and tcgen05.commit frees each stage ("empty")
+//               and hands a finished accumulator to the epilogue ("tfull").
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator (one row per thread),
-//               epilogue arithmetic, 16-byte global stores; "tempty" returns
-//               the accumulator.  Two accumulators (2 x BN columns) let the
+//               epilogue arithmetic into a swizzled staging buffer, one TMA
+//               bulk-tensor store per 128-row sub-tile; "tempty" returns the
+//               accumulator.  Two accumulators (2 x BN columns) let the
 //               epilogue of one tile overlap the MMAs of the next.
-// TMA loads never use cluster multicast.  Every mbarrier wait is bounded:
-// on timeout the kernel records GPT_DEVERR_TIMEOUT, drains what it started,
-// frees its tensor memory and returns.
+// Every TMA load is a plain tile load into the issuing CTA's own shared
+// memory.  Every mbarrier wait is bounded: on timeout the kernel records
+// GPT_DEVERR_TIMEOUT, drains what it started, frees its tensor memory and
+// returns.
 #include "tc_common.cuh"
 
 #define TC_BM 128
