@@ -125,6 +125,7 @@ struct EpiParams {
   const T* aux; long ld_aux;
   float* outf; long ld_outf;
   long split_stride;
+  float* colsum;   // GELU' epilogue of the tensor-core GEMM: [ceil(M/128)][N] column sums of out (fp32), or null
 };
 
 // Apply the epilogue to one element (used by the SIMT GEMM).

@@ -511,9 +511,18 @@ static int backward_impl(gpt_model* m) {
     const LayerOff& lo = m->L[l];
     // MLP: x_out = x_mid + gelu(h2 W_fc^T + b_fc) W_fc2^T + b_fc2  (b_fc2 gradient already summed)
     CKI(gemm(m, C, F, M, drt, C, true, A.a(l), F, true, epi_f32<T>(A.G(lo.w_fc2), F)));
-    CKI(gemm(m, M, F, C, drt, C, false, A.W(lo.w_fc2), F, true, epi_dgelu<T>(dF, F, A.u(l))));
-    { ProfScope ps(m, PC_BIAS, 0, (double)M * F * es);
-      CK(launch_colsum<T>(dF, F, M, F, m->partials, A.G(lo.b_fc), s)); }
+    // on the tensor-core path the GELU' epilogue also sums dF per column over
+    // each 128-row tile (the fc bias gradient before the final reduction)
+    const bool fused_bfc = sizeof(T) == 2 && gemm_tc_supported(M, F, C, C, false, F, true) &&
+                           (size_t)((M + 127) / 128) * F <= m->partials_n;
+    {
+      EpiParams<T> e = epi_dgelu<T>(dF, F, A.u(l));
+      if (fused_bfc) e.colsum = m->partials;
+      CKI(gemm(m, M, F, C, drt, C, false, A.W(lo.w_fc2), F, true, e));
+    }
+    { ProfScope ps(m, PC_BIAS, 0, fused_bfc ? (double)((M + 127) / 128) * F * 4 : (double)M * F * es);
+      if (fused_bfc) CK(launch_reduce_rows(m->partials, (M + 127) / 128, F, F, A.G(lo.b_fc), s));
+      else CK(launch_colsum<T>(dF, F, M, F, m->partials, A.G(lo.b_fc), s)); }
     CKI(gemm(m, F, C, M, dF, F, true, A.h2(l), C, true, epi_f32<T>(A.G(lo.w_fc), C)));
     CKI(gemm(m, M, C, F, dF, F, false, A.W(lo.w_fc), C, true, epi_store<T>(dC, C, nullptr, nullptr, 0)));
     { ProfScope ps(m, PC_LN_BWD, 0, lnbb);

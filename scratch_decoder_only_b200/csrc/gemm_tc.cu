@@ -61,6 +61,25 @@ __device__ __forceinline__ void pack_bf16x64(const float* v, uint4* w) {
   }
 }
 
+// Column sums of a warp's 32 rows x 64 columns (lane = row, v = its 64 values):
+// five halving exchange steps leave lane l with the sums of columns 2l, 2l+1.
+__device__ __forceinline__ float2 warp_colsum64(const float* v, int lane) {
+  float t[64];
+#pragma unroll
+  for (int i = 0; i < 64; ++i) t[i] = v[i];
+#pragma unroll
+  for (int o = 16, n = 32; o >= 1; o >>= 1, n >>= 1) {
+    const bool hi = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < n; ++i) {
+      const float send = hi ? t[i] : t[i + n];
+      const float keep = hi ? t[i + n] : t[i];
+      t[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  return make_float2(t[0], t[1]);
+}
+
 // Bounded barrier of the 128 epilogue threads (an mbarrier with count 128).
 __device__ __forceinline__ bool epi_sync(uint32_t bar, uint32_t& phase, volatile int* abort_flag) {
   mbar_arrive(bar);
@@ -103,7 +122,8 @@ struct TcCfg {
   // buffers; the other kinds keep one more mainloop stage instead
   static constexpr bool WIDE = (KIND == EPI_GELU || EpiTraits<KIND>::SIDE);
   static constexpr int EPI_BYTES = (WIDE ? 4 : 2) * EPI_BUF_BYTES;
-  static constexpr int BIAS_BYTES = EpiTraits<KIND>::BIAS ? BN * 4 : 0;
+  // bias of the tile, or (GELU') the four row quarters' column sums of a sub-tile
+  static constexpr int BIAS_BYTES = EpiTraits<KIND>::BIAS ? BN * 4 : (KIND == EPI_DGELU ? 4 * 64 * 4 : 0);
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;
   static constexpr int B_BYTES = (BN / CG) * TC_BK * 2;   // a CTA pair splits B along N
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -405,6 +425,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           for (int j = 0; j < 64; ++j) v[j] *= gelu_grad_fast(uu[j]);
           pack_bf16x64(v, w);
           stage_row128(b0, rl, w);
+          if (epi.colsum) {   // this warp's 32 rows, summed per column, to shared memory
+            const float2 cs = warp_colsum64(v, lane);
+            bias_s[quarter * 64 + 2 * lane] = cs.x;
+            bias_s[quarter * 64 + 2 * lane + 1] = cs.y;
+          }
         } else {
 #pragma unroll
           for (int q = 0; q < 8; ++q)
@@ -414,6 +439,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
         fence_async_smem();
         if (!epi_sync(group_bar, gph, abort_flag)) { ok = false; break; }
+        if constexpr (KIND == EPI_DGELU) {
+          // the sub-tile's column sums over its 128 rows: one partial row per row tile
+          if (epi.colsum && etid < 64 && rows_in && col0 + etid < N)
+            epi.colsum[(long)(m0 / TC_BM) * N + col0 + etid] =
+                (bias_s[etid] + bias_s[64 + etid]) + (bias_s[128 + etid] + bias_s[192 + etid]);
+        }
         if (etid == 0 && rows_in) {
           if constexpr (KIND == EPI_F32_SPLIT) {
             tma_store_3d(&tmC, b0, col0, m0, split);

@@ -602,7 +602,7 @@ __global__ void __launch_bounds__(256) colsum_kernel(const Tin* __restrict__ x, 
 // bf16 column sums with 16-byte loads: a block covers 256 columns (32 lanes
 // x 8 columns) and CS2_ROWS rows split over 8 warps, four rows in flight per
 // thread; one partial row per block row-chunk.
-#define CS2_ROWS 512
+#define CS2_ROWS 256
 __global__ void __launch_bounds__(256) colsum_bf16_kernel(const bf16* __restrict__ x, long ldx, int M, int N,
                                                          float* __restrict__ partials) {
   __shared__ float red[8][257];
