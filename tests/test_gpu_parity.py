@@ -406,3 +406,31 @@ def test_greedy_decode_bf16_batched(torch):
     clear = gaps[:, 0] >= 0.1
     assert clear.sum() >= 9, gaps[:, 0]
     assert np.array_equal(out[clear, 0], ref[clear, 0]), (out[:, 0], ref[:, 0], gaps[:, 0])
+
+
+def test_byte30m_bf16_trajectory(torch):
+    """Several AdamW steps of the byte-level 30M model, compared step by step
+    with the oracle's own trajectory from the same initial weights (one row of
+    256 tokens per step: the oracle's cost bounds the size)."""
+    wl = CF.BYTE_30M
+    cfg = ocfg(wl.model)
+    hp = wl.adamw
+    steps = 5
+    batches = [S.make_batch(wl, batch=1, seq=256, seed=wl.data_seed + s) for s in range(steps)]
+    model = new_model(wl.model, wl.init_seed)
+    p0 = model.get_params().astype(np.float64)
+    p, m, v = p0.copy(), np.zeros_like(p0), np.zeros_like(p0)
+    for s, (tok, tgt, seg) in enumerate(batches):
+        g = gpu_step(torch, model, tok, tgt, seg, hp)
+        loss_r, grads_r = O.loss_and_grads(cfg, p, tok, tgt, seg, np.float64)
+        p, m, v, norm_r, skipped = O.clip_adamw_step(p, grads_r, m, v, s + 1, hp.lr, hp.beta1, hp.beta2, hp.eps,
+                                                     hp.weight_decay, hp.clip_norm)
+        assert not skipped and g["skipped"] == 0
+        assert rel(g["loss"], loss_r) <= 1e-2, (s, g["loss"], loss_r)
+        assert rel(g["norm"], norm_r) <= 3e-2, (s, g["norm"], norm_r)
+    # each step moves an element by at most about lr, so two trajectories stay
+    # within 2 lr per step of each other; the total update has the oracle's direction
+    pg = model.get_params().astype(np.float64)
+    assert np.max(np.abs(pg - p)) <= 2 * hp.lr * steps
+    du_gpu, du_ref = pg - p0, p - p0
+    assert np.linalg.norm(du_gpu - du_ref) <= 0.2 * np.linalg.norm(du_ref)
