@@ -112,7 +112,8 @@ enum EpiKind {
   EPI_GELU = 1,    // u = acc + bias[n]; out[m,n] = T(u); out2[m,n] = T(gelu(u))
   EPI_DGELU = 2,   // out[m,n] = T(acc * gelu'(aux[m,n]))
   EPI_F32 = 3,     // outf[m,n] = acc                                 (fp32)
-  EPI_F32_SPLIT = 4  // outf[split][m,n] = acc: split-K partial slab   (fp32)
+  EPI_F32_SPLIT = 4, // outf[split][m,n] = acc: split-K partial slab   (fp32)
+  EPI_F32_ADD = 5    // outf[m,n] += acc (fp32; split-K slices added in no fixed order onto a zeroed output)
 };
 
 template <typename T>
@@ -154,6 +155,9 @@ __device__ __forceinline__ void epi_apply1(const EpiParams<T>& p, int m, int n, 
       break;
     case EPI_F32_SPLIT:
       p.outf[(long)split * p.split_stride + (long)m * p.ld_outf + n] = acc;
+      break;
+    case EPI_F32_ADD:
+      atomicAdd(&p.outf[(long)m * p.ld_outf + n], acc);
       break;
   }
 }

@@ -45,8 +45,8 @@ struct gpt_model {
   int *tok, *tgt, *pos, *dstart;
   float* dres32;
   void *dres_t, *dC, *dF, *dqkv;
-  float *attD, *rowloss, *partials, *splitws, *dq_acc;
-  size_t partials_n, splitws_n;
+  float *attD, *rowloss, *partials, *dq_acc;
+  size_t partials_n;
   double* normpart;
   int normblk = 592;
   DevScalars* sc;
@@ -267,9 +267,6 @@ static int build_arena(gpt_model* m) {
   cv.add((void**)&m->rowloss, Mx * 4);
   m->partials_n = std::max((size_t)444 * 3 * C, (size_t)((Mx + 255) / 256) * std::max(3 * C, F));
   cv.add((void**)&m->partials, m->partials_n * 4);
-  m->splitws_n = m->bf16 ? (size_t)8 * std::max(3 * C * C, F * C) : 0;
-  if (m->splitws_n) cv.add((void**)&m->splitws, m->splitws_n * 4);
-  else m->splitws = nullptr;
   cv.add((void**)&m->normpart, m->normblk * 8);
   cv.add((void**)&m->sc, sizeof(DevScalars));
   size_t Bx = m->Bmax;
@@ -357,23 +354,27 @@ static int gemm(gpt_model* m, int M, int N, int K, const bf16* A, long lda, bool
   }
   int splits = 1;
   if (epi.kind == EPI_F32) {
-    // weight gradients: short output, long contraction -> split K over the SMs
-    long tiles = (long)((M + 127) / 128) * ((N + 255) / 256);
-    while (splits < 8 && tiles * splits * 2 <= g_num_sms && K / (splits * 2) >= 512 &&
-           (size_t)(splits * 2) * M * N <= m->splitws_n)
-      splits *= 2;
+    // weight gradients: short output, long contraction -> split K so the
+    // 256 x 256 CTA-pair tiles fill the machine's pairs in whole waves
+    const long tiles = (long)((M + 255) / 256) * ((N + 255) / 256), slots = g_num_sms / 2;
+    double best = 0.0;
+    for (int sp = 1; sp <= 8; sp *= 2) {
+      if (sp > 1 && K / sp < 512) break;
+      const long u = tiles * sp, waves = (u + slots - 1) / slots;
+      const double eff = (double)u / ((double)waves * slots);
+      if (eff > best * 1.05) { best = eff; splits = sp; }
+    }
     int kb_total = (K + 63) / 64, kbs = (kb_total + splits - 1) / splits;
     splits = (kb_total + kbs - 1) / kbs;   // no empty split
+    if (splits > 1 && epi.ld_outf != N) splits = 1;   // the zeroing below wants a dense output
   }
   if (splits > 1) {
+    // K slices add their products onto the zeroed weight gradient (TMA bulk
+    // reduce-add): no partial slabs, no separate summation pass
     EpiParams<bf16> e2 = epi;
-    e2.kind = EPI_F32_SPLIT;
-    e2.outf = m->splitws;
-    e2.ld_outf = N;
-    e2.split_stride = (long)M * N;
+    e2.kind = EPI_F32_ADD;
+    CK(cudaMemsetAsync(epi.outf, 0, (size_t)M * N * 4, m->stream));
     CK(launch_gemm_tc(M, N, K, A, lda, a_t, B, ldb, b_t, e2, splits, &m->sc->err, m->stream));
-    if (epi.ld_outf != N) FAIL(GPT_ERR_ARG, "split-K output must be dense");
-    CK(launch_sum_splits(m->splitws, splits, (long)M * N, (long)M * N, epi.outf, m->stream));
   } else {
     CK(launch_gemm_tc(M, N, K, A, lda, a_t, B, ldb, b_t, epi, 1, &m->sc->err, m->stream));
   }

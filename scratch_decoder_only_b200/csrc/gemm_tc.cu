@@ -108,12 +108,12 @@ __device__ __forceinline__ float4 ld_shared_f4(uint32_t a) {
 // ------------------------------------------------------------------ the kernel
 // EPI_STORE with a residual is its own instantiation: its residual tiles come
 // in by TMA like the DGELU pre-activations.
-#define EPI_STORE_RES 5
+#define EPI_STORE_RES 7
 template <int KIND>
 struct EpiTraits {
   static constexpr bool SIDE = (KIND == EPI_STORE_RES || KIND == EPI_DGELU);   // reads a bf16 [M, N] input
   static constexpr bool BIAS = (KIND == EPI_STORE || KIND == EPI_STORE_RES || KIND == EPI_GELU);
-  static constexpr bool F32OUT = (KIND == EPI_F32 || KIND == EPI_F32_SPLIT);
+  static constexpr bool F32OUT = (KIND == EPI_F32 || KIND == EPI_F32_SPLIT || KIND == EPI_F32_ADD);
 };
 
 template <int BN, int KIND, int CG = 1>
@@ -448,6 +448,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if (etid == 0 && rows_in) {
           if constexpr (KIND == EPI_F32_SPLIT) {
             tma_store_3d(&tmC, b0, col0, m0, split);
+          } else if constexpr (KIND == EPI_F32_ADD) {
+            tma_reduce_add_2d(&tmC, b0, col0, m0);
           } else {
             tma_store_2d(&tmC, b0, col0, m0);
             if constexpr (KIND == EPI_GELU) tma_store_2d(&tmC2, b0 + 2 * EPI_BUF_BYTES, col0, m0);
@@ -555,6 +557,8 @@ static cudaError_t launch_kind(const CUtensorMap& ta, const CUtensorMap& tb, con
   } else if constexpr (B_MN) {
     if (epi.kind == EPI_F32_SPLIT)
       return launch_tc<BN, A_MN, B_MN, EPI_F32_SPLIT, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+    if (epi.kind == EPI_F32_ADD)
+      return launch_tc<BN, A_MN, B_MN, EPI_F32_ADD, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
   }
   return cudaErrorNotSupported;
 }
@@ -587,6 +591,7 @@ static cudaError_t launch_bn(int M, int N, int K, const bf16* A, long lda, bool 
            make_map_ex(&tc2, MapKey{epi.out2, M, N, epi.ld_out2, 1, 0, 64, TC_BM, 0, 128});
       break;
     case EPI_F32:
+    case EPI_F32_ADD:
       ok = make_map_ex(&tc, MapKey{epi.outf, M, N, epi.ld_outf, 1, 0, 32, TC_BM, 1, 128});
       tc2 = tc;
       break;

@@ -1143,32 +1143,6 @@ cudaError_t launch_to_f32(const T* src, long ld, int rows, int cols, float* dst,
   return cudaGetLastError();
 }
 
-// out[i] = sum over splits of ws[split * stride + i] (split-K reduction).
-__global__ void sum_splits_kernel(const float* __restrict__ ws, int splits, long stride, long n,
-                                  float* __restrict__ out) {
-  long n4 = n / 4;
-  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n4; i += (long)gridDim.x * blockDim.x) {
-    float a[4], b[4];
-    Vec<float>::load(ws + 4 * i, a);
-    for (int s = 1; s < splits; ++s) {
-      Vec<float>::load(ws + s * stride + 4 * i, b);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) a[j] += b[j];
-    }
-    Vec<float>::store(out + 4 * i, a);
-  }
-  if (blockIdx.x == 0)
-    for (long i = n4 * 4 + threadIdx.x; i < n; i += blockDim.x) {
-      float a = 0.f;
-      for (int s = 0; s < splits; ++s) a += ws[s * stride + i];
-      out[i] = a;
-    }
-}
-cudaError_t launch_sum_splits(const float* ws, int splits, long stride, long n, float* out, cudaStream_t s) {
-  ++g_kernel_launches;
-  sum_splits_kernel<<<148 * 4, 256, 0, s>>>(ws, splits, stride, n, out);
-  return cudaGetLastError();
-}
 
 // A bounded wait that cannot complete: an mbarrier nobody arrives on.  The
 // waiting thread gives up after timeout_cycles, records GPT_DEVERR_TIMEOUT

@@ -65,7 +65,6 @@ template <typename T>
 cudaError_t launch_cast(const float* src, T* dst, size_t n, cudaStream_t s);
 template <typename T>
 cudaError_t launch_to_f32(const T* src, long ld, int rows, int cols, float* dst, cudaStream_t s);
-cudaError_t launch_sum_splits(const float* ws, int splits, long stride, long n, float* out, cudaStream_t s);
 cudaError_t launch_wait_timeout_probe(unsigned* err, long long timeout_cycles, cudaStream_t s);
 
 // ---- gemm_simt.cu: C[M,N] = A(M x K) . B(N x K)^T with epilogue, SIMT FFMA
