@@ -179,10 +179,10 @@ def job_throughput(tokens_per_rank_step: int, steps: int, world: int, max_ms: fl
 # ----------------------------------------------------------------------------- our arm
 
 # DRAM bytes per GEMM launch of the training step at batch 16: the cold-cache
-# ncu capture of all 147 GEMM launches of a batch-4 step (37.67 MB per
+# ncu capture of all 147 GEMM launches of a batch-4 step (39.98 MB per
 # launch, profiles/gemm_tc_traffic_b4.txt) scaled by the 4x token count.
 # Re-measure, or set to None, whenever the GEMM kernel changes.
-GEMM_TRAFFIC_BYTES_PER_LAUNCH = 150.7e6
+GEMM_TRAFFIC_BYTES_PER_LAUNCH = 159.9e6
 
 
 def run_ours(args, rank, world, local_rank):

@@ -69,6 +69,7 @@ struct gpt_model {
   std::vector<ProfRec> recs;
   std::vector<cudaEvent_t> evpool;
   size_t evused = 0;
+  std::vector<RedSeg> redsegs;   // deferred column reductions of the current backward pass
 };
 
 enum ProfCls { PC_GEMM_FWD, PC_GEMM_DX, PC_GEMM_DW, PC_ATTN_FWD, PC_ATTN_BWD, PC_XENT, PC_LN_FWD, PC_LN_BWD,
@@ -265,7 +266,13 @@ static int build_arena(gpt_model* m) {
   cv.add((void**)&m->attD, Mx * m->H * 4);
   cv.add((void**)&m->dq_acc, m->bf16 ? Mx * C * 4 : 4);
   cv.add((void**)&m->rowloss, Mx * 4);
-  m->partials_n = std::max((size_t)444 * 3 * C, (size_t)((Mx + 255) / 256) * std::max(3 * C, F));
+  {
+    // partial rows of every deferred column reduction of one backward pass:
+    // LayerNorm blocks (at most 444 rows of 3C) and bias column sums (at most
+    // one row per 128 tokens), each region rounded to 16 bytes
+    const size_t ln = (size_t)444 * 3 * C + 4, cs = (size_t)(Mx + 127) / 128;
+    m->partials_n = ln + NL * (2 * ln + cs * F + 4 + cs * 3 * C + 4);
+  }
   cv.add((void**)&m->partials, m->partials_n * 4);
   cv.add((void**)&m->normpart, m->normblk * 8);
   cv.add((void**)&m->sc, sizeof(DevScalars));
@@ -499,51 +506,85 @@ static int backward_impl(gpt_model* m) {
   const T* xf = (const T*)m->xf;
   int nblk = 0;
   const double es = sizeof(T), lnbb = (double)M * C * (3 * es + 8) + 8.0 * M;
+  // Partial rows (LayerNorm dg/db, bias column sums) take consecutive regions
+  // of the partials arena; one deferred launch reduces them all at the end.
+  std::vector<RedSeg>& segs = m->redsegs;
+  segs.clear();
+  float* pp = m->partials;
+  float* const pend = m->partials + m->partials_n;
+  auto take = [&](size_t n) -> float* {
+    float* p = pp;
+    pp += (n + 3) & ~(size_t)3;
+    return pp <= pend ? p : nullptr;
+  };
+  auto seg = [&](const float* src, float* dst, int rows, int cols, int ld) {
+    segs.push_back({src, dst, rows, cols, ld, 0});
+  };
+  // LayerNorm backward; its partial rows are [dg | db | column sums of the
+  // outgoing residual gradient] (the latter = the bias gradient `bias_dst`)
+  auto ln_bwd = [&](const T* x, const float* mu, const float* rs, const float* g, const float* din, float* gdst,
+                    float* bias_dst) -> int {
+    float* part = take((size_t)444 * 3 * C);
+    if (!part) FAIL(GPT_ERR_NOMEM, "partials arena too small");
+    ProfScope ps(m, PC_LN_BWD, 0, lnbb);
+    CK(launch_ln_bwd<T>(dC, x, mu, rs, g, din, m->dres32, drt, part, M, C, &nblk, s));
+    seg(part, gdst, nblk, 2 * C, 3 * C);
+    if (bias_dst) seg(part + 2 * C, bias_dst, nblk, C, 3 * C);
+    return GPT_OK;
+  };
   // LM head: dxf = dz . W_head;  dW_head = dz^T . xf  (into dwte when tied)
   CKI(gemm(m, M, C, Vp, dz, m->ldl, false, A.W(m->o_head), C, true, epi_store<T>(dC, C, nullptr, nullptr, 0)));
   CKI(gemm(m, Vp, C, M, dz, m->ldl, true, xf, C, true, epi_f32<T>(A.G(m->o_head), C)));
-  { ProfScope ps(m, PC_LN_BWD, 0, lnbb);
-    CK(launch_ln_bwd<T>(dC, A.x(m->NL), m->muf, m->rsf, A.P(m->o_lnf_g), nullptr, m->dres32, drt, m->partials,
-                        M, C, &nblk, s));
-    CK(launch_reduce_rows(m->partials, nblk, 2 * C, 3 * C, A.G(m->o_lnf_g), s));
-    // column sums of the gradient entering the last block = its fc2 bias gradient
-    CK(launch_reduce_rows(m->partials + 2 * C, nblk, C, 3 * C, A.G(m->L[m->NL - 1].b_fc2), s)); }
+  // column sums of the gradient entering the last block = its fc2 bias gradient
+  CKI(ln_bwd(A.x(m->NL), m->muf, m->rsf, A.P(m->o_lnf_g), nullptr, A.G(m->o_lnf_g), A.G(m->L[m->NL - 1].b_fc2)));
   for (int l = m->NL - 1; l >= 0; --l) {
     const LayerOff& lo = m->L[l];
-    // MLP: x_out = x_mid + gelu(h2 W_fc^T + b_fc) W_fc2^T + b_fc2  (b_fc2 gradient already summed)
+    // MLP: x_out = x_mid + gelu(h2 W_fc^T + b_fc) W_fc2^T + b_fc2  (b_fc2 gradient already taken)
     CKI(gemm(m, C, F, M, drt, C, true, A.a(l), F, true, epi_f32<T>(A.G(lo.w_fc2), F)));
     // on the tensor-core path the GELU' epilogue also sums dF per column over
-    // each 128-row tile (the fc bias gradient before the final reduction)
-    const bool fused_bfc = sizeof(T) == 2 && gemm_tc_supported(M, F, C, C, false, F, true) &&
-                           (size_t)((M + 127) / 128) * F <= m->partials_n;
+    // each 128-row tile (the fc bias gradient's partial rows)
+    const bool fused_bfc = sizeof(T) == 2 && gemm_tc_supported(M, F, C, C, false, F, true);
+    float* bpart = take((size_t)((M + 127) / 128) * F);
+    if (!bpart) FAIL(GPT_ERR_NOMEM, "partials arena too small");
     {
       EpiParams<T> e = epi_dgelu<T>(dF, F, A.u(l));
-      if (fused_bfc) e.colsum = m->partials;
+      if (fused_bfc) e.colsum = bpart;
       CKI(gemm(m, M, F, C, drt, C, false, A.W(lo.w_fc2), F, true, e));
     }
-    { ProfScope ps(m, PC_BIAS, 0, fused_bfc ? (double)((M + 127) / 128) * F * 4 : (double)M * F * es);
-      if (fused_bfc) CK(launch_reduce_rows(m->partials, (M + 127) / 128, F, F, A.G(lo.b_fc), s));
-      else CK(launch_colsum<T>(dF, F, M, F, m->partials, A.G(lo.b_fc), s)); }
+    if (fused_bfc) {
+      seg(bpart, A.G(lo.b_fc), (M + 127) / 128, F, F);
+    } else {
+      ProfScope ps(m, PC_BIAS, 0, (double)M * F * es);
+      int rows = 0;
+      CK(launch_colsum<T>(dF, F, M, F, bpart, &rows, s));
+      seg(bpart, A.G(lo.b_fc), rows, F, F);
+    }
     CKI(gemm(m, F, C, M, dF, F, true, A.h2(l), C, true, epi_f32<T>(A.G(lo.w_fc), C)));
     CKI(gemm(m, M, C, F, dF, F, false, A.W(lo.w_fc), C, true, epi_store<T>(dC, C, nullptr, nullptr, 0)));
-    { ProfScope ps(m, PC_LN_BWD, 0, lnbb);
-      CK(launch_ln_bwd<T>(dC, A.xmid(l), A.mu2(l), A.rs2(l), A.P(lo.ln2_g), m->dres32, m->dres32, drt,
-                          m->partials, M, C, &nblk, s));
-      CK(launch_reduce_rows(m->partials, nblk, 2 * C, 3 * C, A.G(lo.ln2_g), s));
-      CK(launch_reduce_rows(m->partials + 2 * C, nblk, C, 3 * C, A.G(lo.b_o), s)); }
-    // attention: x_mid = x + attn(h1 W_qkv^T + b_qkv) W_o^T + b_o  (b_o gradient already summed)
+    CKI(ln_bwd(A.xmid(l), A.mu2(l), A.rs2(l), A.P(lo.ln2_g), m->dres32, A.G(lo.ln2_g), A.G(lo.b_o)));
+    // attention: x_mid = x + attn(h1 W_qkv^T + b_qkv) W_o^T + b_o  (b_o gradient already taken)
     CKI(gemm(m, C, C, M, drt, C, true, A.att(l), C, true, epi_f32<T>(A.G(lo.w_o), C)));
     CKI(gemm(m, M, C, C, drt, C, false, A.W(lo.w_o), C, true, epi_store<T>(dC, C, nullptr, nullptr, 0)));
     CKI(attn_bwd(m, A.qkv(l), A.att(l), dC, A.lse(l), dq, B, T_));
-    { ProfScope ps(m, PC_BIAS, 0, (double)M * 3 * C * es);
-      CK(launch_colsum<T>(dq, 3 * C, M, 3 * C, m->partials, A.G(lo.b_qkv), s)); }
+    {
+      float* qpart = take((size_t)((M + 127) / 128) * 3 * C);
+      if (!qpart) FAIL(GPT_ERR_NOMEM, "partials arena too small");
+      ProfScope ps(m, PC_BIAS, 0, (double)M * 3 * C * es);
+      int rows = 0;
+      CK(launch_colsum<T>(dq, 3 * C, M, 3 * C, qpart, &rows, s));
+      seg(qpart, A.G(lo.b_qkv), rows, 3 * C, 3 * C);
+    }
     CKI(gemm(m, 3 * C, C, M, dq, 3 * C, true, A.h1(l), C, true, epi_f32<T>(A.G(lo.w_qkv), C)));
     CKI(gemm(m, M, C, 3 * C, dq, 3 * C, false, A.W(lo.w_qkv), C, true, epi_store<T>(dC, C, nullptr, nullptr, 0)));
-    { ProfScope ps(m, PC_LN_BWD, 0, lnbb);
-      CK(launch_ln_bwd<T>(dC, A.x(l), A.mu1(l), A.rs1(l), A.P(lo.ln1_g), m->dres32, m->dres32, drt,
-                          m->partials, M, C, &nblk, s));
-      CK(launch_reduce_rows(m->partials, nblk, 2 * C, 3 * C, A.G(lo.ln1_g), s));
-      if (l > 0) CK(launch_reduce_rows(m->partials + 2 * C, nblk, C, 3 * C, A.G(m->L[l - 1].b_fc2), s)); }
+    CKI(ln_bwd(A.x(l), A.mu1(l), A.rs1(l), A.P(lo.ln1_g), m->dres32, A.G(lo.ln1_g),
+               l > 0 ? A.G(m->L[l - 1].b_fc2) : nullptr));
+  }
+  // all LayerNorm and bias gradients from their partial rows, one launch
+  {
+    double pb = 0;
+    for (const RedSeg& g : segs) pb += (double)g.rows * g.cols * 4;
+    ProfScope ps(m, PC_BIAS, 0, pb);
+    CK(launch_reduce_segs(segs.data(), (int)segs.size(), s));
   }
   // embeddings: scatter-add by token and by position
   ProfScope ps_emb(m, PC_EMBED, 0, (double)M * C * 12);

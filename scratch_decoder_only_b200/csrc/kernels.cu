@@ -152,34 +152,23 @@ cudaError_t launch_embed_fwd(const int* tok, const int* pos, const float* wte, c
 // variance, y = (x - mean) * rstd * g + b; mean and rstd kept for backward.
 // ---------------------------------------------------------------------------
 template <typename T, int NCH>
-__global__ void __launch_bounds__(256) ln_fwd_kernel(const T* __restrict__ x, const float* __restrict__ g,
-                                                     const float* __restrict__ b, T* __restrict__ y,
-                                                     float* __restrict__ mean, float* __restrict__ rstd, int M, int C,
-                                                     float eps) {
-  // one warp per row, warps walk rows with a grid stride; gamma and beta stay
-  // in registers and the next row's x is loaded before the current row is
-  // reduced (one memory latency per row, overlapped with the previous row)
+__global__ void __launch_bounds__(256, (NCH * Vec<T>::N <= 24 ? 4 : 2)) ln_fwd_kernel(const T* __restrict__ x, const float* __restrict__ g,
+                                                        const float* __restrict__ b, T* __restrict__ y,
+                                                        float* __restrict__ mean, float* __restrict__ rstd, int M,
+                                                        int C, float eps) {
+  // one warp per row, warps walk rows with a grid stride over a grid of one
+  // resident wave; the next row's x is loaded before the current row is
+  // reduced, so each warp keeps two rows in flight.  gamma and beta are read
+  // per row through L1 (a few KB, always resident) rather than held in
+  // registers: for rows of up to 24 values per lane (C = 768 in bf16) the
+  // kernel fits in 64 registers and four 256-thread blocks share an SM, which
+  // is what keeps enough bytes in flight to cover HBM latency.
   constexpr int NV = Vec<T>::N;
   griddep_wait();
   griddep_release();
   const int lane = threadIdx.x & 31;
   const int nch = C / NV;
   const int stride = gridDim.x * (blockDim.x >> 5);
-  float gg[NCH][NV], bb[NCH][NV];
-#pragma unroll
-  for (int i = 0; i < NCH; ++i) {
-    const int ch = lane + i * 32;
-#pragma unroll
-    for (int j = 0; j < NV; j += 4) {
-      if (ch < nch) {
-        Vec<float>::load(g + ch * NV + j, gg[i] + j);
-        Vec<float>::load(b + ch * NV + j, bb[i] + j);
-      } else {
-        gg[i][j] = gg[i][j + 1] = gg[i][j + 2] = gg[i][j + 3] = 0.f;
-        bb[i][j] = bb[i][j + 1] = bb[i][j + 2] = bb[i][j + 3] = 0.f;
-      }
-    }
-  }
   int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   uint4 nxt[NCH];
   auto fetch = [&](int r) {
@@ -222,7 +211,14 @@ __global__ void __launch_bounds__(256) ln_fwd_kernel(const T* __restrict__ x, co
       if (ch < nch) {
         float o[NV];
 #pragma unroll
-        for (int j = 0; j < NV; ++j) o[j] = (v[i][j] - mu) * rs * gg[i][j] + bb[i][j];
+        for (int j = 0; j < NV; j += 4) {
+          const float4 gv = __ldg(reinterpret_cast<const float4*>(g + ch * NV + j));
+          const float4 bv = __ldg(reinterpret_cast<const float4*>(b + ch * NV + j));
+          o[j] = (v[i][j] - mu) * rs * gv.x + bv.x;
+          o[j + 1] = (v[i][j + 1] - mu) * rs * gv.y + bv.y;
+          o[j + 2] = (v[i][j + 2] - mu) * rs * gv.z + bv.z;
+          o[j + 3] = (v[i][j + 3] - mu) * rs * gv.w + bv.w;
+        }
         Vec<T>::store(yr + ch * NV, o);
       }
     }
@@ -230,17 +226,36 @@ __global__ void __launch_bounds__(256) ln_fwd_kernel(const T* __restrict__ x, co
   }
 }
 
+// Blocks of one resident wave for a kernel of 256-thread blocks (occupancy
+// queried once per kernel).
+template <auto KERN>
+static int resident_blocks(int want) {
+  static int per_sm = 0, sms = 0;
+  if (!per_sm) {
+    int dev = 0, n = 0, occ = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, KERN, 256, 0);
+    sms = n > 0 ? n : 148;
+    per_sm = occ > 0 ? occ : 1;
+  }
+  const int cap = per_sm * sms;
+  return want < cap ? want : cap;
+}
+
 template <typename T>
 cudaError_t launch_ln_fwd(const T* x, const float* g, const float* b, T* y, float* mean, float* rstd,
                           int M, int C, float eps, cudaStream_t s) {
   constexpr int NV = Vec<T>::N;
   const int per = (C / NV + 31) / 32;   // 16-byte chunks per lane
-  int blocks = (M + 7) / 8;
-  if (blocks > 148 * 8) blocks = 148 * 8;
+  const int want = (M + 7) / 8;
   ++g_kernel_launches;
   cudaError_t e = cudaSuccess;
-#define LNF_CASE(K) \
-  case K: e = launch_k(ln_fwd_kernel<T, K>, dim3(blocks), dim3(256), 0, s, x, g, b, y, mean, rstd, M, C, eps); break;
+#define LNF_CASE(K)                                                                                  \
+  case K:                                                                                            \
+    e = launch_k(ln_fwd_kernel<T, K>, dim3(resident_blocks<ln_fwd_kernel<T, K>>(want)), dim3(256), 0, s, x, g, b, \
+                 y, mean, rstd, M, C, eps);                                                          \
+    break;
   switch (per) {
     LNF_CASE(1)
     LNF_CASE(2)
@@ -248,7 +263,11 @@ cudaError_t launch_ln_fwd(const T* x, const float* g, const float* b, T* y, floa
     LNF_CASE(4)
     default:
       if constexpr (NV >= 8) return cudaErrorInvalidValue;
-      else { e = launch_k(ln_fwd_kernel<T, 8>, dim3(blocks), dim3(256), 0, s, x, g, b, y, mean, rstd, M, C, eps); break; }
+      else {
+        e = launch_k(ln_fwd_kernel<T, 8>, dim3(resident_blocks<ln_fwd_kernel<T, 8>>(want)), dim3(256), 0, s, x, g, b,
+                     y, mean, rstd, M, C, eps);
+        break;
+      }
   }
 #undef LNF_CASE
   return e != cudaSuccess ? e : cudaGetLastError();
@@ -528,38 +547,62 @@ cudaError_t launch_ln_bwd(const T* dy, const T* x, const float* mean, const floa
   }
 }
 
-// out[n] = sum over r of p[r * ld + n], in a fixed order (deterministic):
-// 32 columns per block, the rows split over 8 warps, 4 loads in flight.
-__global__ void __launch_bounds__(1024) reduce_rows_kernel(const float* __restrict__ p, int rows, int N, long ld,
-                                                           float* __restrict__ out) {
-  __shared__ float red[32][33];
-  int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int n = blockIdx.x * 32 + lane;
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-  if (n < N) {
-    int r = warp;
-    for (; r + 96 < rows; r += 128) {
-      a0 += p[(long)r * ld + n];
-      a1 += p[(long)(r + 32) * ld + n];
-      a2 += p[(long)(r + 64) * ld + n];
-      a3 += p[(long)(r + 96) * ld + n];
+// Deferred column reductions: every segment is dst[n] = sum over r < rows of
+// src[r * ld + n], n < cols, summed in a fixed order (deterministic).  All
+// the per-block partial rows a backward pass leaves (LayerNorm dg/db, bias
+// gradients) are reduced by one launch instead of one small launch each.
+// A block takes 128 columns of one segment: 32 column quads x 8 row groups,
+// row group g summing rows g, g+8, ...; the groups are then added in order.
+__global__ void __launch_bounds__(256) reduce_segs_kernel(RedSegList L) {
+  __shared__ float red[8][129];
+  int si = 0;
+  while (si + 1 < L.n && (int)blockIdx.x >= L.seg[si + 1].blk0) ++si;
+  const RedSeg& sg = L.seg[si];
+  const int q = threadIdx.x & 31, grp = threadIdx.x >> 5;
+  const int c = ((int)blockIdx.x - sg.blk0) * 128 + 4 * q;
+  float a[4] = {0.f, 0.f, 0.f, 0.f};
+  if (c < sg.cols) {
+    const bool vec = c + 4 <= sg.cols && (sg.ld & 3) == 0 && ((uintptr_t)sg.src & 15) == 0;
+    if (vec) {
+#pragma unroll 4
+      for (int r = grp; r < sg.rows; r += 8) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(sg.src + (long)r * sg.ld + c));
+        a[0] += v.x; a[1] += v.y; a[2] += v.z; a[3] += v.w;
+      }
+    } else {
+      for (int r = grp; r < sg.rows; r += 8)
+        for (int j = 0; j < 4 && c + j < sg.cols; ++j) a[j] += sg.src[(long)r * sg.ld + c + j];
     }
-    for (; r < rows; r += 32) a0 += p[(long)r * ld + n];
   }
-  red[warp][lane] = (a0 + a1) + (a2 + a3);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) red[grp][4 * q + j] = a[j];
   __syncthreads();
-  if (warp == 0 && n < N) {
+  if (threadIdx.x < 128) {
+    const int n = ((int)blockIdx.x - sg.blk0) * 128 + threadIdx.x;
     float acc = 0.f;
 #pragma unroll
-    for (int w = 0; w < 32; ++w) acc += red[w][lane];
-    out[n] = acc;
+    for (int w = 0; w < 8; ++w) acc += red[w][threadIdx.x];
+    if (n < sg.cols) sg.dst[n] = acc;
   }
 }
 
-cudaError_t launch_reduce_rows(const float* partials, int rows, int N, long ld, float* out, cudaStream_t s) {
-  ++g_kernel_launches;
-  reduce_rows_kernel<<<(N + 31) / 32, 1024, 0, s>>>(partials, rows, N, ld, out);
-  return cudaGetLastError();
+cudaError_t launch_reduce_segs(const RedSeg* segs, int n, cudaStream_t s) {
+  for (int i0 = 0; i0 < n; i0 += RED_MAX_SEGS) {
+    RedSegList L;
+    L.n = n - i0 < RED_MAX_SEGS ? n - i0 : RED_MAX_SEGS;
+    int blk = 0;
+    for (int i = 0; i < L.n; ++i) {
+      L.seg[i] = segs[i0 + i];
+      L.seg[i].blk0 = blk;
+      blk += (L.seg[i].cols + 127) / 128;
+    }
+    if (blk == 0) continue;
+    ++g_kernel_launches;
+    reduce_segs_kernel<<<blk, 256, 0, s>>>(L);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 // Column sums of x [M, N] (bias gradients): blocks of 128 columns x 256 rows
@@ -644,23 +687,21 @@ __global__ void __launch_bounds__(256) colsum_bf16_kernel(const bf16* __restrict
 }
 
 template <typename Tin>
-cudaError_t launch_colsum(const Tin* x, long ldx, int M, int N, float* partials, float* out, cudaStream_t s) {
+cudaError_t launch_colsum(const Tin* x, long ldx, int M, int N, float* partials, int* rows_out, cudaStream_t s) {
   if constexpr (sizeof(Tin) == 2) {
     if (N % 8 == 0 && ldx % 8 == 0 && ((uintptr_t)x & 15) == 0) {
       dim3 g2((N + 255) / 256, (M + CS2_ROWS - 1) / CS2_ROWS);
+      *rows_out = (int)g2.y;
       ++g_kernel_launches;
       colsum_bf16_kernel<<<g2, 256, 0, s>>>(reinterpret_cast<const bf16*>(x), ldx, M, N, partials);
-      cudaError_t e = cudaGetLastError();
-      if (e != cudaSuccess) return e;
-      return launch_reduce_rows(partials, g2.y, N, N, out, s);
+      return cudaGetLastError();
     }
   }
   dim3 grid((N + 127) / 128, (M + CS_ROWS - 1) / CS_ROWS);
+  *rows_out = (int)grid.y;
   ++g_kernel_launches;
   colsum_kernel<Tin><<<grid, 256, 0, s>>>(x, ldx, M, N, partials);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  return launch_reduce_rows(partials, grid.y, N, N, out, s);
+  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
@@ -1176,7 +1217,7 @@ cudaError_t launch_wait_timeout_probe(unsigned* err, long long timeout_cycles, c
                                         float, cudaStream_t);                                            \
   template cudaError_t launch_ln_bwd<T>(const T*, const T*, const float*, const float*, const float*,      \
                                         const float*, float*, T*, float*, int, int, int*, cudaStream_t);  \
-  template cudaError_t launch_colsum<T>(const T*, long, int, int, float*, float*, cudaStream_t);          \
+  template cudaError_t launch_colsum<T>(const T*, long, int, int, float*, int*, cudaStream_t);            \
   template cudaError_t launch_xent<T>(T*, long, const int*, int, int, int, float*, DevScalars*, cudaStream_t); \
   template cudaError_t launch_embed_bwd<T>(const float*, const int*, const int*, float*, float*, int, int,  \
                                            cudaStream_t);                                                \

@@ -43,10 +43,24 @@ template <typename T>
 cudaError_t launch_ln_bwd(const T* dy, const T* x, const float* mean, const float* rstd, const float* g,
                           const float* dres_in, float* dres_out, T* dres_out_t, float* partials,
                           int M, int C, int* nblk_out, cudaStream_t s);
-// out[n] = sum_r partials[r * ld + n]
-cudaError_t launch_reduce_rows(const float* partials, int rows, int N, long ld, float* out, cudaStream_t s);
+// Deferred column reductions: for each segment, dst[n] = sum_r src[r * ld + n]
+// (n < cols, r < rows, fixed summation order).  Segments are launched in
+// lists of RED_MAX_SEGS (the list travels as the kernel parameter).
+struct RedSeg {
+  const float* src;
+  float* dst;
+  int rows, cols, ld, blk0;   // blk0: first block of the segment (set by the launcher)
+};
+#define RED_MAX_SEGS 96
+struct RedSegList {
+  int n;
+  RedSeg seg[RED_MAX_SEGS];
+};
+cudaError_t launch_reduce_segs(const RedSeg* segs, int n, cudaStream_t s);
+// Column sums of x [M, N] as partial rows: partials[r][0..N), *rows_out rows
+// (at most (M + 127) / 128), to be summed by a reduction segment.
 template <typename Tin>
-cudaError_t launch_colsum(const Tin* x, long ldx, int M, int N, float* partials, float* out, cudaStream_t s);
+cudaError_t launch_colsum(const Tin* x, long ldx, int M, int N, float* partials, int* rows_out, cudaStream_t s);
 template <typename T>
 cudaError_t launch_xent(T* logits, long ldl, const int* tgt, int M, int V, int Vp, float* rowloss,
                         DevScalars* sc, cudaStream_t s);
