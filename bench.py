@@ -178,11 +178,14 @@ def job_throughput(tokens_per_rank_step: int, steps: int, world: int, max_ms: fl
 
 # ----------------------------------------------------------------------------- our arm
 
-# DRAM bytes per GEMM launch of the training step at batch 16: the cold-cache
-# ncu capture of all 147 GEMM launches of a batch-4 step (39.98 MB per
-# launch, profiles/gemm_tc_traffic_b4.txt) scaled by the 4x token count.
-# Re-measure, or set to None, whenever the GEMM kernel changes.
-GEMM_TRAFFIC_BYTES_PER_LAUNCH = 159.9e6
+# DRAM bytes per GEMM launch of the training step at batch 16, from a
+# cold-cache ncu capture of all 147 GEMM launches of a batch-4 step scaled by
+# the 4x token count (profiles/gemm_tc_traffic_b4.txt).  None while the GEMM
+# launch set differs from the one captured: the attention-output gradient
+# GEMMs have since taken the row-dot epilogue (kind 8), which reads one more
+# [M, C] bf16 operand; the capture (159.9 MB per launch, 160.0 algorithmic)
+# covers the set before that change.
+GEMM_TRAFFIC_BYTES_PER_LAUNCH = None
 
 
 def run_ours(args, rank, world, local_rank):
@@ -268,8 +271,12 @@ def run_ours(args, rank, world, local_rank):
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"],
                 "traffic": GEMM_TRAFFIC_BYTES_PER_LAUNCH if B == WL.batch else None,
-                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum over the 147 GEMM launches of "
-                                  "a batch-4 step, per launch, x4 for batch 16 (profiles/gemm_tc_traffic_b4.txt)",
+                "traffic_source": ("ncu dram__bytes_read.sum + dram__bytes_write.sum over the 147 GEMM launches of "
+                                   "a batch-4 step, per launch, x4 for batch 16 (profiles/gemm_tc_traffic_b4.txt)")
+                if GEMM_TRAFFIC_BYTES_PER_LAUNCH is not None else
+                "null: the GEMM launch set changed after the last capture (row-dot epilogue on the attention-output "
+                "gradient GEMMs); that capture, of the set before it, read 159.9 MB per launch against 160.0 MB "
+                "algorithmic (profiles/gemm_tc_traffic_b4.txt)",
                 "kernel": "gemm_tc (all GEMM launches)", "launches": g_n,
                 "avg_launch_ms": g_ms / max(1, g_n), "peak_source": peaks["source"] + " sustained",
                 "measured": "CUDA events around each launch in a second timed region of the same K steps "

@@ -867,8 +867,8 @@ cudaError_t launch_attn_fwd_tc(const bf16* qkv, bf16* out, float* lse, const int
 }
 
 cudaError_t launch_attn_bwd_tc(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* Dbuf,
-                               float* dq_acc, const int* dstart, bf16* dqkv, int B, int T, int H, unsigned* err,
-                               cudaStream_t s) {
+                               bool d_ready, float* dq_acc, const int* dstart, bf16* dqkv, int B, int T, int H,
+                               unsigned* err, cudaStream_t s) {
   const int C = H * AT_D;
   const long rows = (long)B * T;
   CUtensorMap tqkv, tdo, tdq;
@@ -883,11 +883,13 @@ cudaError_t launch_attn_bwd_tc(const bf16* qkv, const bf16* out, const bf16* dou
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  long n = rows * H;
-  ++g_kernel_launches;
-  attn_rowdot_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(out, dout, Dbuf, B, T, H);
   cudaError_t e;
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (!d_ready) {   // D = rowsum(dO o O), unless the producer of dO already wrote it
+    long n = rows * H;
+    ++g_kernel_launches;
+    attn_rowdot_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(out, dout, Dbuf, B, T, H);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   dim3 grid(B * H, (T + AT_BLK - 1) / AT_BLK);
   ++g_kernel_launches;
   attn_bwd_tc<<<grid, BW_THREADS, smem, s>>>(tqkv, tdo, tdq, lse, Dbuf, dstart, dqkv, T, H, err);

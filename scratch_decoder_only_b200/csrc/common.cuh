@@ -127,6 +127,11 @@ struct EpiParams {
   float* outf; long ld_outf;
   long split_stride;
   float* colsum;   // GELU' epilogue of the tensor-core GEMM: [ceil(M/128)][N] column sums of out (fp32), or null
+  // EPI_STORE on the tensor-core GEMM, no bias or residual: with rowdot set,
+  // also rowdot[(b * N/64 + h) * rd_T + t] = out[row, head h] . aux[row, head h]
+  // over 64-wide heads, row = b * rd_T + t (out rounded to T first)
+  float* rowdot;
+  int rd_T;
 };
 
 // Apply the epilogue to one element (used by the SIMT GEMM).

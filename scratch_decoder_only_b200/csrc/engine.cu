@@ -356,6 +356,7 @@ static int gemm(gpt_model* m, int M, int N, int K, const bf16* A, long lda, bool
                 long ldb, bool b_t, EpiParams<bf16> epi) {
   ProfScope ps(m, gemm_cls(a_t, b_t), 2.0 * M * N * K, 0.0);
   if (!gemm_tc_supported(M, N, K, lda, a_t, ldb, b_t)) {
+    if (epi.rowdot) FAIL(GPT_ERR_ARG, "row-dot epilogue needs the tensor-core GEMM");
     CK(launch_gemm_simt<bf16>(M, N, K, A, lda, a_t, B, ldb, b_t, epi, 1, m->stream));
     return GPT_OK;
   }
@@ -403,17 +404,18 @@ static int attn_fwd(gpt_model* m, const bf16* qkv, bf16* out, float* lse, int B,
   return GPT_OK;
 }
 static int attn_bwd(gpt_model* m, const float* qkv, const float* out, const float* dout, const float* lse,
-                    float* dqkv, int B, int T) {
+                    float* dqkv, int B, int T, bool) {
   ProfScope ps(m, PC_ATTN_BWD, 8.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0);
   CK(launch_attn_bwd_simt<float>(qkv, out, dout, lse, m->attD, m->dstart, dqkv, B, T, m->H, m->d, m->stream));
   return GPT_OK;
 }
+// d_ready: m->attD already holds D = rowsum(dO o O) (tensor-core path only)
 static int attn_bwd(gpt_model* m, const bf16* qkv, const bf16* out, const bf16* dout, const float* lse,
-                    bf16* dqkv, int B, int T) {
+                    bf16* dqkv, int B, int T, bool d_ready) {
   ProfScope ps(m, PC_ATTN_BWD, 8.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0);
   if (attn_tc_supported(m->d))
-    CK(launch_attn_bwd_tc(qkv, out, dout, lse, m->attD, m->dq_acc, m->dstart, dqkv, B, T, m->H, &m->sc->err,
-                          m->stream));
+    CK(launch_attn_bwd_tc(qkv, out, dout, lse, m->attD, d_ready, m->dq_acc, m->dstart, dqkv, B, T, m->H,
+                          &m->sc->err, m->stream));
   else if (attn_mma_supported(m->d))
     CK(launch_attn_bwd_mma(qkv, out, dout, lse, m->attD, m->dstart, dqkv, B, T, m->H, m->d, m->stream));
   else
@@ -564,8 +566,15 @@ static int backward_impl(gpt_model* m) {
     CKI(ln_bwd(A.xmid(l), A.mu2(l), A.rs2(l), A.P(lo.ln2_g), m->dres32, A.G(lo.ln2_g), A.G(lo.b_o)));
     // attention: x_mid = x + attn(h1 W_qkv^T + b_qkv) W_o^T + b_o  (b_o gradient already taken)
     CKI(gemm(m, C, C, M, drt, C, true, A.att(l), C, true, epi_f32<T>(A.G(lo.w_o), C)));
-    CKI(gemm(m, M, C, C, drt, C, false, A.W(lo.w_o), C, true, epi_store<T>(dC, C, nullptr, nullptr, 0)));
-    CKI(attn_bwd(m, A.qkv(l), A.att(l), dC, A.lse(l), dq, B, T_));
+    // dO = d(attention output); on the tensor-core path its GEMM epilogue also
+    // takes D = rowsum(dO o O) per row and head for the attention backward
+    const bool fuse_d = sizeof(T) == 2 && attn_tc_supported(m->d) && gemm_tc_supported(M, C, C, C, false, C, true);
+    {
+      EpiParams<T> e = epi_store<T>(dC, C, nullptr, nullptr, 0);
+      if (fuse_d) { e.aux = A.att(l); e.ld_aux = C; e.rowdot = m->attD; e.rd_T = T_; }
+      CKI(gemm(m, M, C, C, drt, C, false, A.W(lo.w_o), C, true, e));
+    }
+    CKI(attn_bwd(m, A.qkv(l), A.att(l), dC, A.lse(l), dq, B, T_, fuse_d));
     {
       float* qpart = take((size_t)((M + 127) / 128) * 3 * C);
       if (!qpart) FAIL(GPT_ERR_NOMEM, "partials arena too small");

@@ -109,9 +109,13 @@ __device__ __forceinline__ float4 ld_shared_f4(uint32_t a) {
 // EPI_STORE with a residual is its own instantiation: its residual tiles come
 // in by TMA like the DGELU pre-activations.
 #define EPI_STORE_RES 7
+// EPI_STORE with a row-dot output (the attention backward's D = dO . O per
+// row and head, taken while the dO tile is in registers): its own
+// instantiation, the second operand of the dot read by TMA as a side input.
+#define EPI_STORE_DOT 8
 template <int KIND>
 struct EpiTraits {
-  static constexpr bool SIDE = (KIND == EPI_STORE_RES || KIND == EPI_DGELU);   // reads a bf16 [M, N] input
+  static constexpr bool SIDE = (KIND == EPI_STORE_RES || KIND == EPI_DGELU || KIND == EPI_STORE_DOT);   // reads a bf16 [M, N] input
   static constexpr bool BIAS = (KIND == EPI_STORE || KIND == EPI_STORE_RES || KIND == EPI_GELU);
   static constexpr bool F32OUT = (KIND == EPI_F32 || KIND == EPI_F32_SPLIT || KIND == EPI_F32_ADD);
 };
@@ -406,6 +410,22 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           }
           pack_bf16x64(v, w);
           stage_row128(b0, rl, w);
+        } else if constexpr (KIND == EPI_STORE_DOT) {
+          float oo[64];
+          load_row128_bf16(rbase + (sub & 1) * EPI_BUF_BYTES, rl, oo);
+          float dot = 0.f;
+#pragma unroll
+          for (int j = 0; j < 64; ++j) {
+            v[j] = __bfloat162float(__float2bfloat16_rn(v[j]));
+            dot += v[j] * oo[j];
+          }
+          pack_bf16x64(v, w);
+          stage_row128(b0, rl, w);
+          const int row = m0 + rl;
+          if (rows_in && row < M) {
+            const int Tq = epi.rd_T, b = row / Tq;
+            epi.rowdot[((long)b * (N / 64) + col0 / 64) * Tq + (row - b * Tq)] = dot;
+          }
         } else if constexpr (KIND == EPI_GELU) {
           float a[64];
 #pragma unroll
@@ -545,6 +565,11 @@ static cudaError_t launch_kind(const CUtensorMap& ta, const CUtensorMap& tb, con
   if constexpr (!A_MN) {
     if (epi.kind == EPI_STORE && epi.resid)
       return launch_tc<BN, A_MN, B_MN, EPI_STORE_RES, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+    if constexpr (B_MN) {
+      if (epi.kind == EPI_STORE && epi.rowdot)
+        return launch_tc<BN, A_MN, B_MN, EPI_STORE_DOT, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+    }
+    if (epi.rowdot) return cudaErrorNotSupported;
     if (epi.kind == EPI_STORE)
       return launch_tc<BN, A_MN, B_MN, EPI_STORE, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
     if constexpr (!B_MN) {
@@ -581,6 +606,10 @@ static cudaError_t launch_bn(int M, int N, int K, const bf16* A, long lda, bool 
       tc2 = tc;
       // the residual is read by TMA in the same 128 x 64 boxes
       if (ok && epi.resid) ok = make_map_ex(&tc2, MapKey{epi.resid, M, N, epi.ld_resid, 1, 0, 64, TC_BM, 0, 128});
+      // so is the row-dot's second operand (heads of 64 columns, no bias or residual)
+      if (ok && epi.rowdot)
+        ok = !epi.resid && !epi.bias && N % 64 == 0 && epi.rd_T > 0 && epi.aux &&
+             make_map_ex(&tc2, MapKey{epi.aux, M, N, epi.ld_aux, 1, 0, 64, TC_BM, 0, 128});
       break;
     case EPI_DGELU:
       ok = make_map_ex(&tc, MapKey{epi.out, M, N, epi.ld_out, 1, 0, 64, TC_BM, 0, 128}) &&

@@ -110,9 +110,11 @@ cudaError_t launch_attn_bwd_mma(const bf16* qkv, const bf16* out, const bf16* do
 bool attn_tc_supported(int d);
 cudaError_t launch_attn_fwd_tc(const bf16* qkv, bf16* out, float* lse, const int* dstart, int B, int T, int H,
                                unsigned* err, cudaStream_t s);
+// d_ready: Dbuf [B, H, T] already holds rowsum(dO o O) (written by the GEMM
+// epilogue that produced dO); otherwise a row-dot kernel computes it first
 cudaError_t launch_attn_bwd_tc(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* Dbuf,
-                               float* dq_acc, const int* dstart, bf16* dqkv, int B, int T, int H, unsigned* err,
-                               cudaStream_t s);
+                               bool d_ready, float* dq_acc, const int* dstart, bf16* dqkv, int B, int T, int H,
+                               unsigned* err, cudaStream_t s);
 
 // ---- decode.cu
 // decode kernels read the position as pos0 + *step (device counter)
