@@ -107,51 +107,103 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- oracle arm
 
-def oracle_sample_step(seq=256):
-    """One bounded oracle step: 1 row x `seq` tokens of the GPT-2 124M model,
-    forward + backward + clip + AdamW over all parameters (fp64).  Returns
-    (seconds, tokens, threads)."""
+def _oracle_cfg(mc):
     from oracle import gpt_oracle as O
-    mc = WL.model
-    cfg = O.OracleConfig(vocab=mc.vocab, vocab_padded=mc.vocab_padded, d_model=mc.d_model,
-                         n_heads=mc.n_heads, d_mlp=mc.d_mlp, n_layers=mc.n_layers, max_seq=mc.max_seq,
-                         tied=mc.tied)
-    tok, tgt, _ = S.make_batch(WL, batch=1, seq=seq)
-    p0 = O.init_params(cfg, WL.init_seed).astype(np.float64)
-    hp = WL.adamw
+    return O.OracleConfig(vocab=mc.vocab, vocab_padded=mc.vocab_padded, d_model=mc.d_model,
+                          n_heads=mc.n_heads, d_mlp=mc.d_mlp, n_layers=mc.n_layers, max_seq=mc.max_seq,
+                          tied=mc.tied)
+
+
+def _blas_threads():
     try:
         from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:
-        threads = os.cpu_count() or 1
-    t0 = time.perf_counter()
-    loss, g = O.loss_and_grads(cfg, p0, tok, tgt)
-    O.clip_adamw_step(p0, g, np.zeros_like(g), np.zeros_like(g), 1, hp.lr, hp.beta1, hp.beta2, hp.eps,
-                      hp.weight_decay, hp.clip_norm)
-    dt = time.perf_counter() - t0
-    return dt, seq, threads
+        return os.cpu_count() or 1
+
+
+class OracleTrainer:
+    """The oracle training the workload's model on a bounded sample per step:
+    1 row x `seq` tokens forward + backward, then clip + AdamW over all
+    parameters (fp64), with the parameters and the AdamW moments carried from
+    step to step.  step(seq) returns (seconds of fwd+bwd, seconds of the
+    optimiser)."""
+
+    def __init__(self, wl):
+        from oracle import gpt_oracle as O
+        self.O, self.wl = O, wl
+        self.cfg = _oracle_cfg(wl.model)
+        self.p = O.init_params(self.cfg, wl.init_seed).astype(np.float64)
+        self.m = np.zeros_like(self.p)
+        self.v = np.zeros_like(self.p)
+        self.t = 0
+
+    def step(self, seq):
+        O, hp = self.O, self.wl.adamw
+        tok, tgt, _ = S.make_batch(self.wl, batch=1, seq=seq)
+        t0 = time.perf_counter()
+        _, g = O.loss_and_grads(self.cfg, self.p, tok, tgt)
+        t1 = time.perf_counter()
+        self.t += 1
+        self.p, self.m, self.v, _, _ = O.clip_adamw_step(self.p, g, self.m, self.v, self.t, hp.lr, hp.beta1,
+                                                         hp.beta2, hp.eps, hp.weight_decay, hp.clip_norm)
+        t2 = time.perf_counter()
+        return t1 - t0, t2 - t1
+
+
+def oracle_sample_step(seq=256):
+    """One bounded oracle step of the workload (the `cpu_baseline` of our arm):
+    1 row x `seq` tokens, forward + backward + clip + AdamW over all parameters.
+    Returns (seconds, tokens, threads)."""
+    tr = OracleTrainer(WL)
+    fb, opt = tr.step(seq)
+    return fb + opt, seq, _blas_threads()
+
+
+# wall-clock budget of the reference arm's W + K steps (the sample per step is
+# sized from a calibration step to fit it)
+REF_BUDGET_S = 150.0
+REF_SEQS = (256, 128, 64, 32, 16)
+
+
+def ref_sample_seq(fb0, opt, per_step_budget, seqs=None):
+    """Largest sample length whose predicted step time (forward + backward
+    linear in the tokens, measured as fb0 seconds at seqs[0]; the optimiser
+    fixed at opt seconds) fits the per-step budget; the smallest one when none
+    does."""
+    seqs = seqs or REF_SEQS
+    for seq in seqs:
+        if opt + fb0 * seq / seqs[0] <= per_step_budget:
+            return seq
+    return seqs[-1]
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    steps = max(1, min(args.steps, 3))
-    for _ in range(max(0, min(args.warmup, 1))):
-        oracle_sample_step()
-    times, toks, threads = [], 0, 1
-    for _ in range(steps):
-        dt, n, threads = oracle_sample_step()
-        times.append(dt)
-        toks += n
+    tr = OracleTrainer(WL)
+    # calibration: the first warm-up step, on the longest sample
+    fb0, opt = tr.step(REF_SEQS[0])
+    seq = ref_sample_seq(fb0, opt, REF_BUDGET_S / max(1, args.warmup - 1 + args.steps))
+    for _ in range(args.warmup - 1):
+        tr.step(seq)
+    times = []
+    for _ in range(args.steps):
+        fb, op = tr.step(seq)
+        times.append(fb + op)
     total = sum(times)
+    toks = seq * args.steps
     value = toks / total
-    sample = f"1 row x 256 tokens of the GPT-2 124M step per timed step (fwd+bwd+clip+AdamW over all params, fp64 numpy), {steps} steps"
+    threads = _blas_threads()
+    sample = (f"1 row x {seq} tokens of the {WL.name} step per timed step (fwd+bwd+clip+AdamW over all params, "
+              f"fp64 numpy), {args.steps} timed steps after {max(1, args.warmup)} warm-up; the sample length "
+              f"is chosen from a {REF_SEQS[0]}-token calibration step so the run fits about {REF_BUDGET_S:.0f} s")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": steps, "warmup": args.warmup, "ms_per_step": 1000 * total / steps,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": WL.name, "global_batch": WL.batch * world, "seq_len": WL.seq,
                                             "parallelism": "none (CPU oracle on the host cores)",
-                                            "timed_sample": "one row x 256 tokens of this workload per step"},
+                                            "timed_sample": f"one row x {seq} tokens of this workload per step"},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
