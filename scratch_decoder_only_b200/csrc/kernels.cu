@@ -606,8 +606,8 @@ cudaError_t launch_reduce_segs(const RedSeg* segs, int n, cudaStream_t s) {
 }
 
 // Column sums of x [M, N] (bias gradients): blocks of 128 columns x 256 rows
-// (4 columns per lane, 8 warps x 32 rows) write per-row-chunk partials;
-// reduce_rows sums the chunks.
+// (4 columns per lane, 8 warps x 32 rows) write per-row-chunk partials; a
+// deferred reduction segment sums the chunks.
 #define CS_ROWS 256
 template <typename Tin>
 __global__ void __launch_bounds__(256) colsum_kernel(const Tin* __restrict__ x, long ldx, int M, int N,
