@@ -24,7 +24,11 @@
  *  - Bad token / target / segment ids found on the device are clamped (no
  *    memory fault) and recorded in a sticky device error word, which
  *    gpt_status reports (GPT_ERR_DEVICE) and clears.
- *  - A model handle is not thread safe: one host thread at a time.
+ *  - A model handle is not thread safe: one host thread at a time.  Some
+ *    launch state is process-wide (the decode-graph capture switches on
+ *    programmatic dependent launch for the kernels it records; per-kernel
+ *    occupancy and tensor-map caches), so drive all handles of a process
+ *    from one host thread.
  */
 #ifndef GPT_H_
 #define GPT_H_
