@@ -228,6 +228,37 @@ def test_fd_gradients_tied():
     _fd_check(cfg, None, 13)
 
 
+@pytest.mark.parametrize("tied", [False, True])
+def test_padded_vocab_columns_take_no_part(tied):
+    """Columns V..Vp-1 of the LM head are padding: the loss, the gradient of
+    every real parameter and greedy decoding ignore whatever sits in the pad
+    rows, and the pad rows' own gradient is exactly zero."""
+    cfg = O.OracleConfig(**{**TINY.__dict__, "tied": tied})
+    flat = random_params(cfg, 21)
+    rng = np.random.default_rng(22)
+    tok = rng.integers(0, cfg.vocab, size=(2, 6))
+    tgt = rng.integers(0, cfg.vocab, size=(2, 6))
+    loss0, g0 = O.loss_and_grads(cfg, flat, tok, tgt)
+    head = "wte" if tied else "w_head"
+    flat_big = flat.copy()
+    big = O.unflatten(cfg, flat_big)              # views into flat_big
+    big[head][cfg.vocab:] = rng.normal(0.0, 50.0, big[head][cfg.vocab:].shape)   # huge pad logits
+    loss1, g1 = O.loss_and_grads(cfg, flat_big, tok, tgt)
+    assert loss1 == loss0
+    G0, G1 = O.unflatten(cfg, g0), O.unflatten(cfg, g1)
+    for k in G0:
+        if tied and k == "w_head":               # an alias of wte
+            continue
+        if k == head:
+            assert np.array_equal(G1[k][:cfg.vocab], G0[k][:cfg.vocab])
+            assert not np.any(G1[k][cfg.vocab:]) and not np.any(G0[k][cfg.vocab:])
+        else:
+            assert np.array_equal(G1[k], G0[k]), k
+    d0, _ = O.greedy_decode(cfg, flat, tok[:, :3], 3, dtype=np.float64)
+    d1, _ = O.greedy_decode(cfg, flat_big, tok[:, :3], 3, dtype=np.float64)
+    assert np.array_equal(d0, d1) and d1.max() < cfg.vocab
+
+
 def test_initial_loss_near_ln_v():
     wl = CF.TINY_BYTE
     cfg = ocfg(wl.model)
