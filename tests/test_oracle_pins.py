@@ -228,6 +228,42 @@ def test_fd_gradients_tied():
     _fd_check(cfg, None, 13)
 
 
+def test_block_structure_with_zero_input_weights():
+    """With every block's input projections zero (W_qkv = W_fc = 0) each block
+    adds a position-independent vector to the residual stream, computable by
+    hand: attention rows are convex combinations of identical value rows, so
+    each head returns its slice of the value bias b_qkv[2C:3C]; the MLP sees
+    u = b_fc.  Hence x_L = wte[tok] + wpe[pos] + sum over blocks of
+    (b_v W_o^T + b_o + gelu(b_fc) W_fc2^T + b_fc2) and the logits are
+    LN_f(x_L) W_head^T.  Pins the pre-LN residual wiring, the [out, in]
+    weight orientation, the q/k/v order inside W_qkv and b_qkv, the final
+    LayerNorm and the head, none of which finite differences can see."""
+    cfg = O.OracleConfig(vocab=13, vocab_padded=16, d_model=8, n_heads=2, d_mlp=12, n_layers=3, max_seq=7)
+    flat = random_params(cfg, 31)
+    P = O.unflatten(cfg, flat)                     # views into flat
+    C = cfg.d_model
+    for l in range(cfg.n_layers):
+        P[f"h{l}.w_qkv"][...] = 0.0
+        P[f"h{l}.w_fc"][...] = 0.0
+    rng = np.random.default_rng(32)
+    tok = rng.integers(0, cfg.vocab, size=(2, 7))
+    logits, _ = O.forward(cfg, flat, tok)
+
+    def gelu_tanh(u):
+        return 0.5 * u * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (u + 0.044715 * u ** 3)))
+
+    x = P["wte"][tok] + P["wpe"][np.arange(7)][None, :, :]
+    for l in range(cfg.n_layers):
+        b_v = P[f"h{l}.b_qkv"][2 * C:3 * C]
+        x = x + b_v @ P[f"h{l}.w_o"].T + P[f"h{l}.b_o"]
+        x = x + gelu_tanh(P[f"h{l}.b_fc"]) @ P[f"h{l}.w_fc2"].T + P[f"h{l}.b_fc2"]
+    mu = x.mean(axis=-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
+    xf = (x - mu) / np.sqrt(var + cfg.ln_eps) * P["lnf_g"] + P["lnf_b"]
+    want = xf.reshape(-1, C) @ P["w_head"].T
+    assert np.allclose(logits, want, rtol=0, atol=1e-12)
+
+
 @pytest.mark.parametrize("tied", [False, True])
 def test_padded_vocab_columns_take_no_part(tied):
     """Columns V..Vp-1 of the LM head are padding: the loss, the gradient of
