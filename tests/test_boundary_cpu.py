@@ -56,6 +56,38 @@ def test_struct_sizes_match_header():
     assert ctypes.sizeof(G.gpt_scalars) == 6 * 4
 
 
+def test_header_is_plain_c_and_matches_the_binding(tmp_path):
+    """include/gpt.h compiles as C99 on its own, and every struct's size and
+    field offsets seen by a C compiler equal the ctypes mirrors'."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    structs = {"gpt_config": G.gpt_config, "gpt_adamw": G.gpt_adamw, "gpt_scalars": G.gpt_scalars,
+               "gpt_prof_entry": G.gpt_prof_entry}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "gpt.h"', "int main(void) {"]
+    for sname, cls in structs.items():
+        lines.append(f'  printf("{sname} size %zu\\n", sizeof({sname}));')
+        for fname, _ in cls._fields_:
+            lines.append(f'  printf("{sname} {fname} %zu\\n", offsetof({sname}, {fname}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+                        "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    got = {}
+    for ln in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.splitlines():
+        parts = ln.split()
+        got[tuple(parts[:-1])] = int(parts[-1])
+    for sname, cls in structs.items():
+        assert got[(sname, "size")] == ctypes.sizeof(cls), sname
+        for fname, _ in cls._fields_:
+            assert got[(sname, fname)] == getattr(cls, fname).offset, (sname, fname)
+
+
 def _create(lib, **over):
     mc = CF.TINY_BYTE.model
     cfg = G.make_config(mc)
