@@ -7,8 +7,6 @@ import contextlib
 import io
 import json
 
-import pytest
-
 
 def test_sample_length_fits_budget():
     import bench
