@@ -237,19 +237,30 @@ int gpt_gemm_bf16(int M, int N, int K, const void* A, long lda, int a_t, const v
  * counterpart: this is a deployment convenience, not a step of the method.
  *
  * Same operands, layouts and result as gpt_gemm_bf16 (fp32 C[M, N], row
- * stride ldc >= N); the K range is split into `splits` slices (1..16, reduced
- * so that no slice is empty) whose partial sums live in a fixed file-scope
- * device array of 4194304 floats (16 MiB, held on every GPU that loads the
- * library until the process exits), then summed into C in a fixed order.
- * Requires splits * M * N <= 4194304, else GPT_ERR_ARG with the reason in
- * gpt_last_error(NULL).  Calls no cudaMalloc / cudaFree.
+ * stride ldc >= N, any N >= 1); the K range is split into `splits` slices
+ * (1..16, reduced so that no slice is empty) whose partial sums live in a
+ * fixed file-scope device array of 4194304 floats (16 MiB, held on every GPU
+ * that loads the library until the process exits), with rows padded to a
+ * multiple of 4 floats, then summed into C in a fixed order.
+ * Requires splits * M * round_up(N, 4) <= 4194304, else GPT_ERR_ARG with the
+ * reason in gpt_last_error(NULL).  Calls no cudaMalloc / cudaFree.
  * The first call on a device looks up the array's device address with that
  * device current; make that first call before any stream capture.
  * All calls share the array (it keeps the last call's partials): calls whose
  * GPU work overlaps (unordered streams) race on it.
+ * A bounded wait inside the GEMM that gives up makes that call write NaN to
+ * every element of C and sets a sticky error word, read and cleared by
+ * gpt_noalloc_status.
  * Errors: GPT_ERR_ARG, GPT_ERR_CUDA. */
 int gpt_gemm_bf16_splitk_noalloc(int M, int N, int K, const void* A, long lda, int a_t, const void* B, long ldb,
                                  int b_t, int splits, float* C, long ldc, void* stream);
+
+/* Status of gpt_gemm_bf16_splitk_noalloc on the current device: synchronises
+ * `stream` (a cudaStream_t; NULL = legacy default), then returns
+ * GPT_ERR_TIMEOUT if any call since the last gpt_noalloc_status had a bounded
+ * device wait give up (its C holds NaN), else GPT_OK, and clears the word.
+ * Allocates nothing.  Errors: GPT_ERR_CUDA. */
+int gpt_noalloc_status(void* stream);
 
 /* Number of kernels libgpt has launched in this process (all handles).
  * Benchmarks read it before and after a timed region. */

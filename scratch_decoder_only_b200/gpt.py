@@ -29,7 +29,7 @@ EXPORTED = [
     "gpt_set_adam_v", "gpt_get_logits", "gpt_get_residual", "gpt_get_scalars", "gpt_set_scalars", "gpt_status",
     "gpt_device_error", "gpt_last_error", "gpt_debug_poison_grad", "gpt_debug_wait_timeout",
     "gpt_kernel_launches", "gpt_profile_enable", "gpt_profile_read", "gpt_gemm_bf16",
-    "gpt_gemm_bf16_splitk_noalloc",
+    "gpt_gemm_bf16_splitk_noalloc", "gpt_noalloc_status",
 ]
 
 
@@ -97,6 +97,7 @@ def load_library(path: str = LIB_PATH):
         "gpt_gemm_bf16": ([I, I, I, P, ctypes.c_long, I, P, ctypes.c_long, I, P, ctypes.c_long, P], I),
         "gpt_gemm_bf16_splitk_noalloc": ([I, I, I, P, ctypes.c_long, I, P, ctypes.c_long, I, I, P, ctypes.c_long, P],
                                          I),
+        "gpt_noalloc_status": ([P], I),
         "gpt_profile_read": ([H, ctypes.POINTER(gpt_prof_entry), I, ctypes.POINTER(I)], I),
     }
     for n in ("params", "grads", "adam_m", "adam_v"):
@@ -163,6 +164,14 @@ def gemm_bf16_splitk_noalloc(A, B, a_t=False, b_t=False, splits=4, M=None, N=Non
     if rc != GPT_OK:
         raise GPTError(rc, L.gpt_last_error(None).decode())
     return C
+
+
+def noalloc_status():
+    """Synchronise the current stream and return (and clear) the no-allocation
+    GEMM's sticky status: GPT_OK, or GPT_ERR_TIMEOUT after a wait gave up."""
+    import torch
+    L = load_library()
+    return L.gpt_noalloc_status(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
 class GPT:
