@@ -454,6 +454,25 @@ def loss_scale_update(scale, good_steps, finite, growth_interval=2000):
     return scale, good_steps, False
 
 
+def lr_at(step, kind, warmup, total, max_lr, min_lr, lr_const=0.0):
+    """Learning rate of the AdamW step that follows ``step`` taken steps.
+
+    The pages' SFT recipe uses a cosine schedule with warm-up steps and a
+    minimum learning rate ("LucilleAI", "Getting started": --lr-scheduler
+    cosine --warmup-steps 100 --min-lr 0.00003).  Read plainly: a linear ramp
+    to max_lr over the warm-up steps, then half a cosine period from max_lr
+    down to min_lr at step ``total``, then min_lr.  kind 0 = constant.
+    """
+    if kind == 0:
+        return lr_const
+    if step < warmup:
+        return max_lr * (step + 1) / warmup
+    if step >= total:
+        return min_lr
+    r = (step - warmup) / (total - warmup)
+    return min_lr + 0.5 * (max_lr - min_lr) * (1.0 + math.cos(math.pi * r))
+
+
 def clip_adamw_step(params, grads, m, v, t, lr, beta1, beta2, eps, wd, clip_norm):
     """Clip by the global L2 norm, then AdamW.  Skips (no change) when the
     gradient is not finite.  Returns (p, m, v, norm, skipped)."""

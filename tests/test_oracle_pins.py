@@ -427,3 +427,27 @@ def test_greedy_decode_tie_lowest_index():
     P["w_head"][2] = P["w_head"][5]          # column 2 ties with column 5
     out, gaps = O.greedy_decode(cfg, flat, np.array([[4]]), n_new=1, dtype=np.float64)
     assert out.tolist() == [[2]] and gaps[0, 0] == 0.0
+
+
+def test_lr_schedule_special_points():
+    """Cosine schedule with warm-up ("LucilleAI", "Getting started": cosine,
+    warm-up steps, min-lr): checked at points fixed by the shape alone, not by
+    retyping the formula -- the ramp's first value and its top, the decay's
+    start at max_lr, its end at min_lr, the midpoint at the mean of the two,
+    the mirror symmetry lr(r) + lr(1 - r) = max + min of half a cosine period,
+    monotone decay, and the constant kind."""
+    kw = dict(kind=1, warmup=100, total=1100, max_lr=6e-4, min_lr=3e-5)
+    assert O.lr_at(0, **kw) == pytest.approx(6e-6, rel=1e-12)
+    assert O.lr_at(99, **kw) == pytest.approx(6e-4, rel=1e-12)
+    assert O.lr_at(100, **kw) == pytest.approx(6e-4, rel=1e-12)
+    assert O.lr_at(600, **kw) == pytest.approx((6e-4 + 3e-5) / 2, rel=1e-12)
+    assert O.lr_at(1100, **kw) == pytest.approx(3e-5, rel=1e-12)
+    assert O.lr_at(5000, **kw) == pytest.approx(3e-5, rel=1e-12)
+    for d in (1, 37, 250, 499):
+        assert O.lr_at(100 + d, **kw) + O.lr_at(1100 - d, **kw) == pytest.approx(6e-4 + 3e-5, rel=1e-12)
+    seq = [O.lr_at(s, **kw) for s in range(100, 1101)]
+    assert all(a >= b for a, b in zip(seq, seq[1:]))
+    # the ramp is linear: equal increments
+    ramp = np.diff([O.lr_at(s, **kw) for s in range(100)])
+    assert np.allclose(ramp, 6e-6, rtol=1e-9)
+    assert O.lr_at(12, kind=0, warmup=0, total=1, max_lr=1.0, min_lr=0.0, lr_const=2.5e-4) == 2.5e-4
