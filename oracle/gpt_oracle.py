@@ -73,10 +73,17 @@ class OracleConfig:
     tied: bool = False
     ln_eps: float = 1e-5
     init_std: float = 0.02
+    arch: str = "gpt2"          # "gpt2" or "llama"
+    n_kv_heads: int = 0         # llama: key / value heads (0: n_heads)
+    rope_base: float = 10000.0  # llama: rotary base
 
     @property
     def head_dim(self) -> int:
         return self.d_model // self.n_heads
+
+    @property
+    def kv_heads(self) -> int:
+        return self.n_kv_heads or self.n_heads
 
 
 # ---------------------------------------------------------------------------
@@ -86,6 +93,19 @@ class OracleConfig:
 def param_shapes(cfg: OracleConfig):
     """Canonical parameter order (row-major, linear weights stored [out, in])."""
     C, F, Vp = cfg.d_model, cfg.d_mlp, cfg.vocab_padded
+    if cfg.arch == "llama":
+        # no position table, no biases; q rows, then the key heads', then the
+        # value heads' rows; gate rows, then up rows
+        kvd = cfg.kv_heads * cfg.head_dim
+        out = [("wte", (Vp, C))]
+        for l in range(cfg.n_layers):
+            p = f"h{l}."
+            out += [(p + "attn_norm_g", (C,)), (p + "w_qkv", (C + 2 * kvd, C)), (p + "w_o", (C, C)),
+                    (p + "mlp_norm_g", (C,)), (p + "w_gu", (2 * F, C)), (p + "w_down", (C, F))]
+        out += [("norm_g", (C,))]
+        if not cfg.tied:
+            out.append(("w_head", (Vp, C)))
+        return out
     out = [("wte", (Vp, C)), ("wpe", (cfg.max_seq, C))]
     for l in range(cfg.n_layers):
         p = f"h{l}."
@@ -174,7 +194,7 @@ def init_params(cfg: OracleConfig, seed: int) -> np.ndarray:
     for name, shape in param_shapes(cfg):
         n = int(np.prod(shape))
         leaf = name.split(".")[-1]
-        if leaf in ("wte", "wpe", "w_qkv", "w_o", "w_fc", "w_fc2", "w_head"):
+        if leaf in ("wte", "wpe", "w_qkv", "w_o", "w_fc", "w_fc2", "w_head", "w_gu", "w_down"):
             z = gaussian_for_elements(seed, np.arange(o, o + n, dtype=np.uint64))
             vals = (std * z).astype(np.float32)
             if leaf in ("wte", "w_head"):
@@ -325,6 +345,8 @@ def _merge_heads(x, B, T, H, d):
 
 def forward(cfg: OracleConfig, flat_params, tokens, seg_ids=None, dtype=np.float64):
     """Logits [B*T, Vp] and the cache the backward pass needs."""
+    if cfg.arch == "llama":
+        return forward_llama(cfg, flat_params, tokens, seg_ids, dtype)
     P = {k: v.astype(dtype) for k, v in unflatten(cfg, np.asarray(flat_params)).items()}
     tokens = np.asarray(tokens, dtype=np.int64)
     B, T = tokens.shape
@@ -361,6 +383,8 @@ def forward(cfg: OracleConfig, flat_params, tokens, seg_ids=None, dtype=np.float
 
 def backward(cfg: OracleConfig, cache, dlogits):
     """Gradients of every parameter (dict by name, untied names only)."""
+    if cfg.arch == "llama":
+        return backward_llama(cfg, cache, dlogits)
     P = cache["P"]
     B, T = cache["B"], cache["T"]
     C, H, d = cfg.d_model, cfg.n_heads, cfg.head_dim
@@ -404,6 +428,159 @@ def backward(cfg: OracleConfig, cache, dlogits):
         G["w_head"] = g_head
     G["wpe"] = g_wpe
     return G
+
+
+# ---------------------------------------------------------------------------
+# Llama-style block: RMSNorm, rotary positions, grouped key / value heads,
+# SwiGLU MLP ("NTransformer" page, key features: Llama architecture with RoPE,
+# GQA and SwiGLU, KV cache; "RustGPT" roadmap: architecture extensions)
+# ---------------------------------------------------------------------------
+
+def rmsnorm_fwd(x, g, eps):
+    """x / sqrt(mean(x^2) + eps) * g over the last axis (Zhang and Sennrich 2019)."""
+    rstd = 1.0 / np.sqrt((x * x).mean(axis=-1, keepdims=True) + eps)
+    xhat = x * rstd
+    return xhat * g, xhat, rstd
+
+
+def rmsnorm_bwd(dy, xhat, rstd, g):
+    """Chain rule through RMSNorm: returns dx, dg (dg summed over rows)."""
+    gh = dy * g
+    C = xhat.shape[-1]
+    dx = rstd * (gh - xhat * (gh * xhat).sum(-1, keepdims=True) / C)
+    dg = (dy * xhat).reshape(-1, C).sum(0)
+    return dx, dg
+
+
+def rope_angles(pos, d, base):
+    """Angle pos * theta_i of dimension pair i = 0..d/2-1, theta_i = base^(-2i/d)
+    (Su et al., RoFormer), for positions pos [B, T] -> [B, T, d/2]."""
+    i = np.arange(d // 2, dtype=np.float64)
+    theta = base ** (-2.0 * i / d)
+    return np.asarray(pos, dtype=np.float64)[..., None] * theta
+
+
+def rope_apply(x, ang, inverse=False):
+    """Rotate the consecutive pairs (x[2i], x[2i+1]) of the last axis by ang
+    (or by -ang: the transpose, for the backward pass).  x: [B, H, T, d],
+    ang: [B, T, d/2]."""
+    c = np.cos(ang)[:, None]
+    s = np.sin(ang)[:, None]
+    if inverse:
+        s = -s
+    x0, x1 = x[..., 0::2], x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = x0 * c - x1 * s
+    out[..., 1::2] = x0 * s + x1 * c
+    return out
+
+
+def silu(z):
+    return z / (1.0 + np.exp(-z))
+
+
+def silu_grad(z):
+    sg = 1.0 / (1.0 + np.exp(-z))
+    return sg * (1.0 + z * (1.0 - sg))
+
+
+def _expand_kv(x, G):
+    """[B, Hkv, T, d] -> [B, Hkv * G, T, d]: query head h reads key head h // G."""
+    return np.repeat(x, G, axis=1)
+
+
+def forward_llama(cfg: OracleConfig, flat_params, tokens, seg_ids=None, dtype=np.float64):
+    """Logits [B*T, Vp] of the Llama-style model and the backward cache.
+
+    Block: h = RMSNorm(x) g1; q, k, v = h W_qkv^T (H query heads, Hkv key /
+    value heads); q, k rotated by their position inside the document; causal
+    (block-diagonal when packed) attention with query head h on key / value
+    head h // (H / Hkv); x += o W_o^T; h2 = RMSNorm(x) g2; gate, up = h2
+    W_gu^T; x += (silu(gate) * up) W_down^T.  Then RMSNorm and the head.
+    """
+    P = {k: v.astype(dtype) for k, v in unflatten(cfg, np.asarray(flat_params)).items()}
+    tokens = np.asarray(tokens, dtype=np.int64)
+    B, T = tokens.shape
+    C, H, d, F = cfg.d_model, cfg.n_heads, cfg.head_dim, cfg.d_mlp
+    Hkv = cfg.kv_heads
+    G = H // Hkv
+    pos, seg = positions_from_segments(seg_ids, B, T)
+    ang = rope_angles(pos, d, cfg.rope_base)
+    x = P["wte"][tokens.reshape(-1)]
+    cache = dict(B=B, T=T, tokens=tokens, pos=pos, seg=seg, ang=ang, layers=[], P=P)
+    for l in range(cfg.n_layers):
+        p = f"h{l}."
+        lc = {}
+        h1, lc["xhat1"], lc["rstd1"] = rmsnorm_fwd(x, P[p + "attn_norm_g"], cfg.ln_eps)
+        lc["h1"] = h1
+        qkv = h1 @ P[p + "w_qkv"].T
+        q = rope_apply(_split_heads(qkv[:, :C], B, T, H, d), ang)
+        k = rope_apply(_split_heads(qkv[:, C:C + Hkv * d], B, T, Hkv, d), ang)
+        v = _split_heads(qkv[:, C + Hkv * d:], B, T, Hkv, d)
+        lc["q"], lc["k"], lc["v"] = q, k, v
+        o = _merge_heads(attention_fwd(q, _expand_kv(k, G), _expand_kv(v, G), seg), B, T, H, d)
+        lc["o"] = o
+        x = x + o @ P[p + "w_o"].T
+        h2, lc["xhat2"], lc["rstd2"] = rmsnorm_fwd(x, P[p + "mlp_norm_g"], cfg.ln_eps)
+        lc["h2"] = h2
+        gu = h2 @ P[p + "w_gu"].T
+        lc["gate"], lc["up"] = gu[:, :F], gu[:, F:]
+        a = silu(lc["gate"]) * lc["up"]
+        lc["a"] = a
+        x = x + a @ P[p + "w_down"].T
+        cache["layers"].append(lc)
+    xf, cache["xhatf"], cache["rstdf"] = rmsnorm_fwd(x, P["norm_g"], cfg.ln_eps)
+    cache["xf"] = xf
+    return xf @ P["w_head"].T, cache
+
+
+def backward_llama(cfg: OracleConfig, cache, dlogits):
+    """Gradients of every parameter of the Llama-style model (by name)."""
+    P = cache["P"]
+    B, T, ang = cache["B"], cache["T"], cache["ang"]
+    C, H, d, F = cfg.d_model, cfg.n_heads, cfg.head_dim, cfg.d_mlp
+    Hkv = cfg.kv_heads
+    G = H // Hkv
+    Gr = {}
+    g_head = dlogits.T @ cache["xf"]
+    dxf = dlogits @ P["w_head"]
+    dx, Gr["norm_g"] = rmsnorm_bwd(dxf, cache["xhatf"], cache["rstdf"], P["norm_g"])
+    for l in reversed(range(cfg.n_layers)):
+        p = f"h{l}."
+        lc = cache["layers"][l]
+        # MLP: x_out = x_mid + (silu(gate) * up) W_down^T
+        Gr[p + "w_down"] = dx.T @ lc["a"]
+        da = dx @ P[p + "w_down"]
+        dgate = da * lc["up"] * silu_grad(lc["gate"])
+        dup = da * silu(lc["gate"])
+        dgu = np.concatenate([dgate, dup], axis=1)
+        Gr[p + "w_gu"] = dgu.T @ lc["h2"]
+        dh2 = dgu @ P[p + "w_gu"]
+        dln, Gr[p + "mlp_norm_g"] = rmsnorm_bwd(dh2, lc["xhat2"], lc["rstd2"], P[p + "mlp_norm_g"])
+        dx = dx + dln
+        # attention: x_mid = x_in + attn(RMSNorm(x_in)) W_o^T
+        Gr[p + "w_o"] = dx.T @ lc["o"]
+        do = _split_heads(dx @ P[p + "w_o"], B, T, H, d)
+        dq, dke, dve = attention_bwd(lc["q"], _expand_kv(lc["k"], G), _expand_kv(lc["v"], G), cache["seg"], do)
+        # a key / value head's gradient sums over the query heads that read it
+        dk = dke.reshape(B, Hkv, G, T, d).sum(axis=2)
+        dv = dve.reshape(B, Hkv, G, T, d).sum(axis=2)
+        dq = rope_apply(dq, ang, inverse=True)
+        dk = rope_apply(dk, ang, inverse=True)
+        dqkv = np.concatenate([_merge_heads(dq, B, T, H, d), _merge_heads(dk, B, T, Hkv, d),
+                               _merge_heads(dv, B, T, Hkv, d)], axis=1)
+        Gr[p + "w_qkv"] = dqkv.T @ lc["h1"]
+        dh1 = dqkv @ P[p + "w_qkv"]
+        dln, Gr[p + "attn_norm_g"] = rmsnorm_bwd(dh1, lc["xhat1"], lc["rstd1"], P[p + "attn_norm_g"])
+        dx = dx + dln
+    g_wte = np.zeros_like(P["wte"])
+    np.add.at(g_wte, cache["tokens"].reshape(-1), dx)
+    if cfg.tied:
+        Gr["wte"] = g_wte + g_head
+    else:
+        Gr["wte"] = g_wte
+        Gr["w_head"] = g_head
+    return Gr
 
 
 def flatten_grads(cfg: OracleConfig, G: dict, dtype=np.float64) -> np.ndarray:
@@ -510,3 +687,71 @@ def greedy_decode(cfg: OracleConfig, flat_params, prompt, n_new, dtype=np.float3
         out[:, s] = nxt
         seq = np.concatenate([seq, nxt[:, None]], axis=1)
     return out, gaps
+
+
+# ---------------------------------------------------------------------------
+# Sampling decode: temperature, top-k, top-p
+# ---------------------------------------------------------------------------
+
+def sample_token(z, V, temperature, top_k, top_p, u):
+    """One sampled token from a row of logits ``z`` (real vocabulary 0..V-1).
+
+    The pages list temperature scaling, top-k and top-p among the generation
+    features a from-scratch model should gain after greedy decoding
+    ("RustGPT", roadmap "high-priority feature requests"; "LucilleAI" names a
+    sampler in its GPU stack).  Read plainly, in this order:
+
+    * temperature <= 0: greedy (argmax, lowest index on ties);
+    * x = z / temperature;
+    * top-k (0 < top_k < V): keep the top_k largest x, ties at the cut going
+      to the lower indices;
+    * weights w_i = exp(x_i - max x) over the kept tokens;
+    * top-p (top_p < 1): order the kept tokens by (w descending, index
+      ascending) and keep the shortest prefix whose weight reaches top_p times
+      the kept total (ties at the cut again to the lower indices);
+    * with the uniform draw u in [0, 1) (an input: the method's random
+      numbers are passed in), return the first kept token, in ascending token
+      order, at which the running sum of kept weights exceeds u times their
+      total.
+    """
+    z = np.asarray(z, dtype=np.float64)[:V]
+    if temperature <= 0.0:
+        return int(np.argmax(z))
+    x = z / temperature
+    order = np.lexsort((np.arange(V), -x))          # x descending, index ascending
+    keep = np.zeros(V, dtype=bool)
+    k = V if (top_k <= 0 or top_k >= V) else top_k
+    keep[order[:k]] = True
+    w = np.where(keep, np.exp(x - np.max(x)), 0.0)
+    if top_p < 1.0:
+        total = w.sum()
+        kept = order[:k]
+        wk = w[kept]
+        sub = np.lexsort((kept, -wk))                # weight descending, index ascending
+        csum = np.cumsum(wk[sub])
+        n = int(np.searchsorted(csum, top_p * total, side="left")) + 1
+        keep2 = np.zeros(V, dtype=bool)
+        keep2[kept[sub[:min(n, len(sub))]]] = True
+        w = np.where(keep2, w, 0.0)
+    c = np.cumsum(w)
+    t = int(np.searchsorted(c, u * c[-1], side="right"))
+    if t >= V:
+        t = int(np.nonzero(w)[0][-1])
+    return t
+
+
+def sample_decode(cfg: OracleConfig, flat_params, prompt, n_new, temperature, top_k, top_p, uniforms,
+                  dtype=np.float64):
+    """Sampled continuation by full-prefix recomputation (no cache): each step
+    draws the next token of every row with ``sample_token`` from the last
+    position's logits and the row's uniform ``uniforms[b, step]``."""
+    seq = np.asarray(prompt, dtype=np.int64)
+    B = seq.shape[0]
+    out = np.zeros((B, n_new), dtype=np.int64)
+    for s in range(n_new):
+        logits, _ = forward(cfg, flat_params, seq, None, dtype)
+        last = logits.reshape(B, seq.shape[1], -1)[:, -1, :]
+        for b in range(B):
+            out[b, s] = sample_token(last[b], cfg.vocab, temperature, top_k, top_p, float(uniforms[b, s]))
+        seq = np.concatenate([seq, out[:, s:s + 1]], axis=1)
+    return out

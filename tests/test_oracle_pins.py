@@ -451,3 +451,151 @@ def test_lr_schedule_special_points():
     ramp = np.diff([O.lr_at(s, **kw) for s in range(100)])
     assert np.allclose(ramp, 6e-6, rtol=1e-9)
     assert O.lr_at(12, kind=0, warmup=0, total=1, max_lr=1.0, min_lr=0.0, lr_const=2.5e-4) == 2.5e-4
+
+
+def test_sampling_reduces_to_greedy_and_inverse_cdf():
+    """Sampling ("RustGPT" roadmap: temperature scaling, top-k, top-p):
+    pinned by the cases that reduce to something known -- temperature 0 and
+    top-k = 1 are greedy (lowest index on ties); with no top-k / top-p, a grid
+    of N uniforms (i + 1/2)/N lands on each token about N * softmax(z / T)
+    times (the inverse-CDF property), at T = 1 and T = 2; top-k keeps exactly
+    the k largest logits with ties to the lower index; top-p on a hand example
+    keeps the smallest high-probability prefix."""
+    rng = np.random.default_rng(12)
+    z = rng.normal(0, 2.0, 50)
+    V = 50
+    assert O.sample_token(z, V, 0.0, 0, 1.0, 0.7) == int(np.argmax(z))
+    for u in (0.0, 0.3, 0.999):
+        assert O.sample_token(z, V, 1.3, 1, 1.0, u) == int(np.argmax(z))
+    zt = np.array([1.0, 2.0, 2.0, 0.0])
+    assert O.sample_token(zt, 4, 1.0, 1, 1.0, 0.9) == 1
+    assert {O.sample_token(zt, 4, 1.0, 2, 1.0, u) for u in np.linspace(0, 0.999, 200)} == {1, 2}
+    N = 20000
+    for T in (1.0, 2.0):
+        p = np.exp(z / T - np.max(z / T))
+        p /= p.sum()
+        counts = np.bincount([O.sample_token(z, V, T, 0, 1.0, (i + 0.5) / N) for i in range(N)], minlength=V)
+        assert np.all(np.abs(counts - N * p) <= 1.0 + 1e-9), np.max(np.abs(counts - N * p))
+    # top-k = 5 at T = 1: only the five largest appear, in proportion to their renormalised softmax
+    top5 = np.argsort(-z)[:5]
+    p5 = np.exp(z[top5] - z[top5].max())
+    p5 /= p5.sum()
+    counts = np.bincount([O.sample_token(z, V, 1.0, 5, 1.0, (i + 0.5) / N) for i in range(N)], minlength=V)
+    assert set(np.nonzero(counts)[0]) == set(top5)
+    assert np.all(np.abs(counts[top5] - N * p5) <= 1.0 + 1e-9)
+    # top-p: probabilities (0.5, 0.3, 0.15, 0.05)
+    zp = np.log([0.15, 0.5, 0.05, 0.3])
+    assert {O.sample_token(zp, 4, 1.0, 0, 0.6, u) for u in np.linspace(0, 0.999, 100)} == {1, 3}
+    assert {O.sample_token(zp, 4, 1.0, 0, 0.85, u) for u in np.linspace(0, 0.999, 100)} == {0, 1, 3}
+    assert {O.sample_token(zp, 4, 1.0, 0, 0.4, u) for u in np.linspace(0, 0.999, 100)} == {1}
+    # in ascending token order: with (1, 3) kept, u below 0.5 / 0.8 gives token 1
+    assert O.sample_token(zp, 4, 1.0, 0, 0.6, 0.6) == 1 and O.sample_token(zp, 4, 1.0, 0, 0.6, 0.65) == 3
+
+
+# ---------------------------------------------------------------- Llama-style block
+
+LLAMA = O.OracleConfig(vocab=11, vocab_padded=16, d_model=16, n_heads=4, d_mlp=12, n_layers=2, max_seq=6,
+                       arch="llama", n_kv_heads=2)
+
+
+@pytest.mark.parametrize("variant", ["plain", "packed", "tied", "mha"])
+def test_llama_fd_gradients(variant):
+    """Central finite differences on every parameter element of the Llama-style
+    block (RMSNorm, rotary positions, two query heads per key / value head,
+    SwiGLU); packed rows restart the rotary positions at each document."""
+    cfg = LLAMA
+    seg = None
+    if variant == "packed":
+        seg = np.array([[0, 0, 0, 1, 1, 1], [0, 0, 1, 1, 1, 2]])
+    elif variant == "tied":
+        cfg = O.OracleConfig(**{**LLAMA.__dict__, "tied": True})
+    elif variant == "mha":
+        cfg = O.OracleConfig(**{**LLAMA.__dict__, "n_kv_heads": 4})
+    _fd_check(cfg, seg, 21)
+
+
+def test_rope_scores_depend_on_relative_position_only():
+    """Rotary positions (Su et al., RoFormer): a rotated query at position i
+    against a rotated key at position j gives the same score for every shift
+    (i + s, j + s), and the rotation keeps the vector norm; the inverse
+    rotation undoes it."""
+    rng = np.random.default_rng(5)
+    d = 16
+    q = rng.normal(size=(1, 1, 1, d))
+    k = rng.normal(size=(1, 1, 1, d))
+
+    def rot(x, p):
+        return O.rope_apply(x, O.rope_angles(np.array([[p]]), d, 10000.0))
+
+    base = float((rot(q, 7) * rot(k, 3)).sum())
+    for s in (1, 5, 100, 1000):
+        assert float((rot(q, 7 + s) * rot(k, 3 + s)).sum()) == pytest.approx(base, rel=1e-9, abs=1e-9)
+    assert float((rot(q, 7) * rot(k, 4)).sum()) != pytest.approx(base, rel=1e-6)
+    assert np.linalg.norm(rot(q, 123)) == pytest.approx(np.linalg.norm(q), rel=1e-12)
+    ang = O.rope_angles(np.array([[9]]), d, 10000.0)
+    assert np.allclose(O.rope_apply(O.rope_apply(q, ang), ang, inverse=True), q, atol=1e-12)
+    # position 0 is the identity
+    assert np.array_equal(rot(q, 0), q)
+
+
+def test_gqa_equals_mha_with_repeated_key_value_heads():
+    """Two query heads per key / value head give exactly the logits of the
+    multi-head model whose key and value weights repeat each shared head."""
+    cfg = LLAMA
+    mha = O.OracleConfig(**{**LLAMA.__dict__, "n_kv_heads": 4})
+    flat = random_params(cfg, 41)
+    P = O.unflatten(cfg, flat)
+    Q = O.unflatten(mha, np.zeros(O.num_params(mha)))
+    C, d, Hkv, G = cfg.d_model, cfg.head_dim, cfg.kv_heads, cfg.n_heads // cfg.kv_heads
+    for name in P:
+        if name.endswith("w_qkv"):
+            w = P[name]
+            q_rows = w[:C]
+            k_rows = w[C:C + Hkv * d].reshape(Hkv, d, C)
+            v_rows = w[C + Hkv * d:].reshape(Hkv, d, C)
+            Q[name][...] = np.concatenate([q_rows, np.repeat(k_rows, G, axis=0).reshape(-1, C),
+                                           np.repeat(v_rows, G, axis=0).reshape(-1, C)])
+        else:
+            Q[name][...] = P[name]
+    tok = np.random.default_rng(42).integers(0, cfg.vocab, size=(2, 6))
+    qflat = np.concatenate([Q[n].reshape(-1) for n, _ in O.param_shapes(mha)])
+    a, _ = O.forward(cfg, flat, tok)
+    b, _ = O.forward(mha, qflat, tok)
+    assert np.allclose(a, b, rtol=1e-12, atol=1e-12)
+
+
+def test_rmsnorm_and_silu_special_cases():
+    """RMSNorm of a constant row c is sign(c) |c| / sqrt(c^2 + eps) times the
+    gain, and scaling a row leaves RMSNorm unchanged when eps = 0; silu(0) = 0,
+    silu(z) -> z for large z and -> 0 for very negative z; silu' matches a
+    central difference."""
+    g = np.arange(1, 9, dtype=np.float64)
+    y, _, _ = O.rmsnorm_fwd(np.full((1, 8), -3.0), g, 1e-5)
+    assert np.allclose(y, -3.0 / math.sqrt(9.0 + 1e-5) * g)
+    x = np.random.default_rng(3).normal(size=(2, 8))
+    assert np.allclose(O.rmsnorm_fwd(x, g, 0.0)[0], O.rmsnorm_fwd(7.5 * x, g, 0.0)[0])
+    assert O.silu(np.array(0.0)) == 0.0
+    assert O.silu(np.array(40.0)) == pytest.approx(40.0, rel=1e-12)
+    assert abs(O.silu(np.array(-40.0))) < 1e-15
+    z = np.linspace(-6, 6, 25)
+    fd = (O.silu(z + 1e-6) - O.silu(z - 1e-6)) / 2e-6
+    assert np.allclose(O.silu_grad(z), fd, atol=1e-8)
+
+
+def test_llama_mask_and_packing_bit_identity():
+    """Changing token j leaves the logits of earlier positions bit-identical,
+    and a packed row equals its documents run separately (positions restart)."""
+    cfg = LLAMA
+    flat = random_params(cfg, 43)
+    rng = np.random.default_rng(44)
+    tok = rng.integers(0, cfg.vocab, size=(1, 6))
+    a, _ = O.forward(cfg, flat, tok)
+    t2 = tok.copy()
+    t2[0, 4] = (t2[0, 4] + 1) % cfg.vocab
+    b, _ = O.forward(cfg, flat, t2)
+    assert np.array_equal(a[:4], b[:4]) and not np.array_equal(a[4], b[4])
+    seg = np.array([[0, 0, 0, 1, 1, 1]])
+    p, _ = O.forward(cfg, flat, tok, seg)
+    d0, _ = O.forward(cfg, flat, tok[:, :3])
+    d1, _ = O.forward(cfg, flat, tok[:, 3:])
+    assert np.array_equal(p[:3], d0) and np.array_equal(p[3:], d1)
