@@ -235,14 +235,13 @@ def job_throughput(tokens_per_rank_step: int, steps: int, world: int, max_ms: fl
 
 # ----------------------------------------------------------------------------- our arm
 
-# DRAM bytes per GEMM launch of the training step at batch 16, from a
-# cold-cache ncu capture of all 147 GEMM launches of a batch-4 step scaled by
-# the 4x token count (profiles/gemm_tc_traffic_b4.txt).  None while the GEMM
-# launch set differs from the one captured: the attention-output gradient
-# GEMMs have since taken the row-dot epilogue (kind 8), which reads one more
-# [M, C] bf16 operand; the capture (159.9 MB per launch, 160.0 algorithmic)
-# covers the set before that change.
-GEMM_TRAFFIC_BYTES_PER_LAUNCH = None
+# DRAM bytes per GEMM launch at the headline size: the ncu capture of a
+# batch-4 step (dram__bytes_read.sum + dram__bytes_write.sum over its 147
+# gemm_tc_kernel launches: 40.50 MB per launch) scaled by the 4x token count
+# (profiles/train_step_gpt2_124m_b4_dram_traffic.txt); the algorithmic bytes
+# per launch at batch 16 are 162.0 MB (23.82 GB over the 147 launches).
+GEMM_TRAFFIC_BYTES_PER_LAUNCH = 162.0e6
+GEMM_ALGO_BYTES_PER_LAUNCH = 162.0e6
 
 
 def run_ours(args, rank, world, local_rank):
@@ -328,12 +327,10 @@ def run_ours(args, rank, world, local_rank):
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"],
                 "traffic": GEMM_TRAFFIC_BYTES_PER_LAUNCH if B == WL.batch else None,
-                "traffic_source": ("ncu dram__bytes_read.sum + dram__bytes_write.sum over the 147 GEMM launches of "
-                                   "a batch-4 step, per launch, x4 for batch 16 (profiles/gemm_tc_traffic_b4.txt)")
-                if GEMM_TRAFFIC_BYTES_PER_LAUNCH is not None else
-                "null: the GEMM launch set changed after the last capture (row-dot epilogue on the attention-output "
-                "gradient GEMMs); that capture, of the set before it, read 159.9 MB per launch against 160.0 MB "
-                "algorithmic (profiles/gemm_tc_traffic_b4.txt)",
+                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum over the 147 GEMM launches of "
+                                  "a batch-4 step, per launch, x4 for batch 16 "
+                                  "(profiles/train_step_gpt2_124m_b4_dram_traffic.txt)",
+                "algorithmic_bytes_per_launch": GEMM_ALGO_BYTES_PER_LAUNCH,
                 "kernel": "gemm_tc (all GEMM launches)", "launches": g_n,
                 "avg_launch_ms": g_ms / max(1, g_n), "peak_source": peaks["source"] + " sustained",
                 "measured": "CUDA events around each launch in a second timed region of the same K steps "
@@ -373,10 +370,13 @@ def run_ours(args, rank, world, local_rank):
                "h2d_bytes_per_step": int(h_tok.numel() * 4 + h_tgt.numel() * 4), "d2h_bytes_per_step": 4,
                "steps": k2}
 
-    # greedy decode (secondary metric)
+    # greedy decode (secondary metric) and the other training workloads
     decode = None
     if not args.no_decode:
         decode = bench_decode(torch, dev, args)
+    configs = None
+    if not args.no_configs and B == WL.batch:
+        configs = bench_configs(torch, dev, args)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -394,16 +394,74 @@ def run_ours(args, rank, world, local_rank):
                            "l2": "working set > L2 (no flush needed)"},
                 "mfu": mfu, "mfu_sustained_peak": mfu_sust, "flops_per_step": fpt * tokens_per_step,
                 "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": n1 - n0, "clocks": clk, "decode": decode,
+                "gpu_launches": n1 - n0, "clocks": clk, "decode": decode, "other_workloads": configs,
                 "final_loss": final_loss, "status": status}
         print(json.dumps(line), flush=True)
     model.close()
+
+
+def bench_configs(torch, dev, args):
+    """The other training workloads, timed the same way (CUDA events over K
+    steps after W warm-up steps, inputs resident): the tiny byte model (fp32,
+    100 timed steps), the packed model (bf16, block-diagonal attention, loss
+    scale 2^15) and the byte-level 30M model (bf16, 32 x 1024).  MFU counts 6N
+    + attention FLOPs (causal pairs; the packed model's from its documents)."""
+    from scratch_decoder_only_b200.gpt import GPT
+    peaks = load_peaks()
+    res = {}
+    for wl, steps in ((CF.TINY_BYTE, 100), (CF.PACKED_SMALL, args.steps), (CF.BYTE_30M, args.steps)):
+        mc = wl.model
+        tok, tgt, seg = S.make_batch(wl)
+        d_tok, d_tgt = torch.from_numpy(tok).to(dev), torch.from_numpy(tgt).to(dev)
+        d_seg = None if seg is None else torch.from_numpy(seg).to(dev)
+        model = GPT(mc, wl.init_seed)
+        loss = torch.zeros(1, dtype=torch.float32, device=dev)
+        for _ in range(max(3, args.warmup)):
+            model.train_step(d_tok, d_tgt, d_seg, wl.adamw, loss)
+        torch.cuda.synchronize()
+        times = []
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        e[0].record()
+        for i in range(steps):
+            model.train_step(d_tok, d_tgt, d_seg, wl.adamw, loss)
+            e[i + 1].record()
+        torch.cuda.synchronize()
+        times = [e[i].elapsed_time(e[i + 1]) for i in range(steps)]
+        ms = float(np.mean(times))
+        B, T = tok.shape
+        if seg is None:
+            pairs = B * T * (T + 1) / 2.0
+        else:
+            pairs = 0.0
+            for b in range(B):
+                _, counts = np.unique(seg[b], return_counts=True)
+                pairs += float(np.sum(counts * (counts + 1) / 2.0))
+        flops = 6.0 * mc.num_params() * B * T + 12.0 * mc.n_layers * mc.d_model * pairs
+        entry = {"workload": wl.name, "tokens_per_s": B * T / (ms / 1000.0), "ms_per_step": ms,
+                 "ms_per_step_median": float(np.median(times)), "steps": steps, "final_loss": float(loss.item()),
+                 "flops_per_step": flops}
+        if mc.precision != "fp32":
+            entry["mfu"] = flops / (ms / 1000.0) / (peaks["bf16_tflops"] * 1e12)
+        res[wl.name] = entry
+        model.close()
+    return res
+
+
+def decode_bytes(mc: CF.ModelConfig, B: int, Tp: int, n_new: int) -> float:
+    """Algorithmic HBM bytes of one greedy decode call: the bf16 matmul weights
+    (tied head included) once for the prefill and once per later token, the
+    K and V rows of the cache each step reads (bf16), and the fp32 logits."""
+    C, F, L, Vp = mc.d_model, mc.d_mlp, mc.n_layers, mc.vocab_padded
+    w = 2.0 * (L * (4 * C * C + 2 * F * C) + Vp * C)
+    kv = sum(B * L * 2 * (Tp + s + 1) * C * 2.0 for s in range(n_new - 1))
+    return n_new * w + kv + n_new * B * Vp * 4.0
 
 
 def bench_decode(torch, dev, args):
     from scratch_decoder_only_b200.gpt import GPT
     wl = CF.GPT2_DECODE
     res = {}
+    hbm = load_peaks()["hbm_gbs"]
     model = GPT(wl.model, wl.init_seed)
     for B in (1, 32):
         prompt = torch.from_numpy(S.make_prompts(wl, B, 128)).to(dev)
@@ -416,7 +474,11 @@ def bench_decode(torch, dev, args):
         e1.record()
         torch.cuda.synchronize()
         ms = e0.elapsed_time(e1)
-        res[f"b{B}"] = {"tok_per_s": B * 384 / (ms / 1000.0), "ms": ms}
+        nbytes = decode_bytes(wl.model, B, 128, 384)
+        gbs = nbytes / (ms / 1000.0) / 1e9
+        res[f"b{B}"] = {"tok_per_s": B * 384 / (ms / 1000.0), "ms": ms, "bytes": nbytes, "gbs": gbs,
+                        "hbm_frac": gbs / hbm,
+                        "ceiling_tok_per_s": B * 384 / (nbytes / (hbm * 1e9))}
     model.close()
     return res
 
@@ -428,6 +490,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other training workloads")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None, help="override the batch (profiling of small cases)")

@@ -50,6 +50,7 @@ extern "C" {
 
 #define GPT_PRECISION_FP32 0
 #define GPT_PRECISION_BF16 1
+#define GPT_PRECISION_FP16 2
 
 /* Device error word bits (reported through gpt_status / gpt_device_error). */
 #define GPT_DEVERR_TOKEN   1u   /* token id outside [0, vocab)                */
@@ -76,22 +77,42 @@ extern "C" {
  *  max_seq        largest T (also the number of position-embedding rows)
  *  max_batch      largest B accepted by gpt_forward_loss / decode
  *  tied           1: the LM head reuses the token embedding matrix
- *  precision      GPT_PRECISION_FP32 (fp32 everywhere, SIMT FFMA) or
+ *  precision      GPT_PRECISION_FP32 (fp32 everywhere, SIMT FFMA),
  *                 GPT_PRECISION_BF16 (bf16 GEMM/attention operands and
  *                 activations, fp32 accumulate, fp32 master weights, moments
- *                 and weight gradients; tcgen05 tensor cores)
+ *                 and weight gradients; tcgen05 tensor cores) or
+ *                 GPT_PRECISION_FP16 (the same with fp16 in place of bf16:
+ *                 the pages' FP16 AMP with a loss scaler, "LucilleAI",
+ *                 "Architecture (from source)": autocast FP16 + GradScaler;
+ *                 use loss_scaling = 1)
  *  loss_scaling   1: dynamic loss scale (x0.5 and skip on a non-finite
  *                 gradient, x2 after 2000 finite steps); 0: scale fixed at 1
  *                 (the non-finite skip stays on)
  *  init_loss_scale  starting scale when loss_scaling = 1 (e.g. 32768)
  *  ln_eps         LayerNorm epsilon (1e-5, biased variance)
  *  init_std       std of the N(0, init_std) initial weight matrices (0.02)
+ *  arch           GPT_ARCH_GPT2 (the block above) or GPT_ARCH_LLAMA: a
+ *                 Llama-style block ("NTransformer" page, "key features":
+ *                 Llama architecture with RoPE, GQA, SwiGLU and a KV cache)
+ *                 -- RMSNorm in place of LayerNorm (gains only), no position
+ *                 table: queries and keys rotated by their position inside
+ *                 the document (consecutive pairs (2i, 2i+1) by pos *
+ *                 rope_base^(-2i/d)), n_kv_heads key/value heads shared by
+ *                 n_heads / n_kv_heads query heads each, a SwiGLU MLP
+ *                 (silu(x W_gate^T) * (x W_up^T)) W_down^T, no biases.
+ *                 Needs 16-bit precision and head size 64.
+ *  n_kv_heads     Llama: key/value heads, dividing n_heads (0: n_heads)
+ *  rope_base      Llama: rotary base (10000)
  */
+#define GPT_ARCH_GPT2  0
+#define GPT_ARCH_LLAMA 1
 typedef struct {
   int32_t vocab, vocab_padded, d_model, n_heads, d_mlp, n_layers, max_seq, max_batch;
   int32_t tied, precision, loss_scaling;
   float init_loss_scale;
   float ln_eps, init_std;
+  int32_t arch, n_kv_heads;
+  float rope_base;
 } gpt_config;
 
 /* AdamW with decoupled weight decay ("Feste", section "Manual
@@ -113,7 +134,30 @@ typedef struct {
   float last_loss;       /* loss of the latest gpt_forward_loss with targets */
   float last_grad_norm;  /* unscaled global L2 norm of the latest step       */
   int32_t last_skipped;  /* 1 if the latest step was skipped (non-finite)    */
+  float last_lr;         /* learning rate the latest taken step used         */
 } gpt_scalars;
+
+/* Learning-rate schedule evaluated on the device from the AdamW step counter
+ * (the number of steps taken before the one being computed, s = 0, 1, ...;
+ * skipped steps do not advance it), so that a step captured in a CUDA graph
+ * still follows the schedule when replayed.  The pages' SFT recipe trains
+ * with a cosine schedule, warm-up steps and a floor ("LucilleAI", "Getting
+ * started": --lr-scheduler cosine --warmup-steps 100 --min-lr 0.00003):
+ *   GPT_LR_CONSTANT  lr = gpt_adamw.lr of each gpt_clip_adamw_step call
+ *   GPT_LR_COSINE    s <  warmup_steps: lr = max_lr * (s + 1) / warmup_steps
+ *                    s >= total_steps:  lr = min_lr
+ *                    otherwise, with r = (s - warmup_steps) / (total_steps -
+ *                    warmup_steps): lr = min_lr + (max_lr - min_lr) *
+ *                    (1 + cos(pi r)) / 2
+ * With a cosine schedule set, gpt_adamw.lr is ignored. */
+#define GPT_LR_CONSTANT 0
+#define GPT_LR_COSINE   1
+typedef struct {
+  int32_t kind;            /* GPT_LR_CONSTANT or GPT_LR_COSINE             */
+  int32_t warmup_steps;    /* >= 0                                          */
+  int32_t total_steps;     /* > warmup_steps                                */
+  float max_lr, min_lr;    /* 0 <= min_lr <= max_lr                         */
+} gpt_lr_schedule;
 
 /* Validate cfg, size and allocate the device arena, initialise parameters
  * from seed (weights N(0, init_std) drawn per canonical element from
@@ -151,6 +195,21 @@ int gpt_forward_loss(gpt_model* m, const int32_t* tokens, const int32_t* targets
  * loss scale).  Errors: GPT_ERR_STATE if no forward with targets preceded. */
 int gpt_backward(gpt_model* m);
 
+/* Gradient accumulation over micro-batches.  gpt_backward_accumulate is
+ * gpt_backward except that it adds this micro-batch's gradient to the stored
+ * gradients instead of overwriting them; gpt_set_loss_weight(w) multiplies
+ * the loss gradient of every later gpt_forward_loss by w (default 1; the
+ * reported loss stays the plain mean).  With k micro-batches of equal valid
+ * target counts, weight 1/k, one gpt_backward and k - 1 accumulating
+ * backwards give the gradient of the mean loss over all of them, which one
+ * gpt_clip_adamw_step then applies (the pages train with FP16 accumulation
+ * and a loss scaler on a 4 GB GPU: "LucilleAI", "Why it matters",
+ * "Architecture (from source)").  gpt_set_loss_weight synchronises.
+ * Errors: GPT_ERR_STATE (no forward with targets), GPT_ERR_ARG (w <= 0 or
+ * not finite). */
+int gpt_backward_accumulate(gpt_model* m);
+int gpt_set_loss_weight(gpt_model* m, float w);
+
 /* Unscale, clip and update: g <- g / loss_scale; if any g is not finite the
  * step is skipped (parameters and moments unchanged, scale halved when
  * loss_scaling = 1); otherwise the global L2 norm is clipped and AdamW
@@ -170,11 +229,40 @@ int gpt_clip_adamw_step(gpt_model* m, const gpt_adamw* hp, float* grad_norm_dev,
 int gpt_greedy_decode(gpt_model* m, const int32_t* prompt, int B, int Tp, int n_new,
                       int32_t* out);
 
+/* Sampling controls for gpt_sample_decode. */
+typedef struct {
+  float temperature;   /* > 0: logits divided by it; 0: greedy            */
+  int32_t top_k;       /* keep the top_k largest logits (0: no top-k)     */
+  float top_p;         /* keep the smallest top-probability prefix whose  */
+                       /* mass reaches top_p (1: no top-p); 0 < top_p <= 1 */
+} gpt_sampling;
+
+/* Sampled decoding: as gpt_greedy_decode, but every new token is drawn from
+ * the fp32 logits of the last position ("RustGPT", roadmap "high-priority
+ * feature requests": temperature scaling, top-k, top-p; "LucilleAI" lists a
+ * sampler in its GPU stack), in this order: x = z / temperature over the real
+ * vocabulary; top-k keeps the top_k largest x (ties at the cut to the lower
+ * index); weights w = exp(x - max x) over the kept tokens; top-p keeps the
+ * shortest prefix, in (w descending, index ascending) order, whose weight
+ * reaches top_p times the kept total; the token is the first kept one, in
+ * ascending token order, at which the running weight exceeds u times the
+ * kept total.  The random numbers are inputs:
+ *  uniforms  device float [B, n_new], values in [0, 1): column s is the draw
+ *            for new token s of each row.
+ * Requires vocab <= 55000 (the row is held in shared memory).
+ * Errors: as gpt_greedy_decode; GPT_ERR_ARG for bad controls. */
+int gpt_sample_decode(gpt_model* m, const int32_t* prompt, int B, int Tp, int n_new, const gpt_sampling* sp,
+                      const float* uniforms, int32_t* out);
+
 /* Number of parameters N in the canonical layout:
  *  wte[Vp,C], wpe[max_seq,C]; per layer ln1_g[C], ln1_b[C], w_qkv[3C,C]
  *  (rows: q, then k, then v; head h = rows h*d..h*d+d-1 of each), b_qkv[3C],
  *  w_o[C,C], b_o[C], ln2_g[C], ln2_b[C], w_fc[F,C], b_fc[F], w_fc2[C,F],
- *  b_fc2[C]; then lnf_g[C], lnf_b[C]; then w_head[Vp,C] only if untied. */
+ *  b_fc2[C]; then lnf_g[C], lnf_b[C]; then w_head[Vp,C] only if untied.
+ * Llama-style (Hkv key/value heads): wte[Vp,C]; per layer attn_norm_g[C],
+ *  w_qkv[C + 2*Hkv*d, C] (q rows, then the key heads', then the value
+ *  heads'), w_o[C,C], mlp_norm_g[C], w_gu[2F,C] (gate rows, then up rows),
+ *  w_down[C,F]; then norm_g[C]; then w_head[Vp,C] only if untied. */
 int gpt_num_params(const gpt_model* m, size_t* n);
 
 /* Copy N fp32 values (canonical layout) between the library and dst/src,
@@ -205,9 +293,28 @@ int gpt_get_logits(gpt_model* m, float* dst, size_t n);
  * GPT_ERR_STATE (no forward yet). */
 int gpt_get_residual(gpt_model* m, int layer, float* dst, size_t n);
 
-/* Read / write the optimiser and loss-scale scalars.  Synchronous. */
+/* Read / write the optimiser and loss-scale scalars.  Synchronous.
+ * gpt_set_scalars writes loss_scale, good_steps and step only. */
 int gpt_get_scalars(gpt_model* m, gpt_scalars* out);
 int gpt_set_scalars(gpt_model* m, const gpt_scalars* in);
+
+/* Set (or, with NULL, clear to GPT_LR_CONSTANT) the learning-rate schedule
+ * used by later gpt_clip_adamw_step calls.  Synchronous.
+ * Errors: GPT_ERR_ARG (kind unknown, warmup_steps < 0, total_steps <=
+ * warmup_steps, or not 0 <= min_lr <= max_lr). */
+int gpt_set_lr_schedule(gpt_model* m, const gpt_lr_schedule* sched);
+
+/* K training steps in one call, all enqueued without a host round trip:
+ * for k = 0..K-1, gpt_forward_loss on tokens + k*B*T (targets, seg_ids
+ * likewise; seg_ids may be NULL), gpt_backward and gpt_clip_adamw_step.
+ *  tokens, targets  device int32 [K, B, T];  seg_ids device int32 [K, B, T] or NULL
+ *  losses_dev       device float [K] (may be NULL): loss of each step
+ *  grad_norms_dev   device float [K] (may be NULL): unscaled norm of each step
+ *  skipped_dev      device int32 [K] (may be NULL): 1 where a step was skipped
+ * Errors: as the three calls, GPT_ERR_ARG for K < 1 or NULL targets. */
+int gpt_train_steps(gpt_model* m, const int32_t* tokens, const int32_t* targets, const int32_t* seg_ids, int K,
+                    int B, int T, const gpt_adamw* hp, float* losses_dev, float* grad_norms_dev,
+                    int32_t* skipped_dev);
 
 /* Synchronise the stream, then return GPT_OK, GPT_ERR_CUDA, GPT_ERR_TIMEOUT
  * or GPT_ERR_DEVICE from the sticky device error word, which is cleared. */

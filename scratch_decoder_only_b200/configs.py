@@ -24,11 +24,14 @@ class ModelConfig:
     max_seq: int
     max_batch: int
     tied: bool = False
-    precision: str = "fp32"          # "fp32" or "bf16"
+    precision: str = "fp32"          # "fp32", "bf16" or "fp16"
     loss_scaling: bool = False       # dynamic loss scale
     init_loss_scale: float = 1.0
     ln_eps: float = 1e-5
     init_std: float = 0.02
+    arch: str = "gpt2"               # "gpt2" or "llama" (RMSNorm, rotary positions, grouped K/V heads, SwiGLU)
+    n_kv_heads: int = 0              # llama: key / value heads (0: n_heads)
+    rope_base: float = 10000.0       # llama: rotary base
 
     @property
     def head_dim(self) -> int:
@@ -36,8 +39,13 @@ class ModelConfig:
 
     def num_params(self) -> int:
         C, F, Vp = self.d_model, self.d_mlp, self.vocab_padded
-        per_layer = 4 * C * C + 2 * F * C + 9 * C + F
-        n = Vp * C + self.max_seq * C + self.n_layers * per_layer + 2 * C
+        if self.arch == "llama":
+            kv = (self.n_kv_heads or self.n_heads) * self.head_dim
+            per_layer = C * (C + 2 * kv) + C * C + 3 * F * C + 2 * C
+            n = Vp * C + self.n_layers * per_layer + C
+        else:
+            per_layer = 4 * C * C + 2 * F * C + 9 * C + F
+            n = Vp * C + self.max_seq * C + self.n_layers * per_layer + 2 * C
         if not self.tied:
             n += Vp * C
         return n

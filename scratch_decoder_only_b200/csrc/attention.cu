@@ -234,3 +234,7 @@ template cudaError_t launch_attn_bwd_simt<float>(const float*, const float*, con
                                                  const int*, float*, int, int, int, int, cudaStream_t);
 template cudaError_t launch_attn_bwd_simt<bf16>(const bf16*, const bf16*, const bf16*, const float*, float*,
                                                 const int*, bf16*, int, int, int, int, cudaStream_t);
+template cudaError_t launch_attn_fwd_simt<f16>(const f16*, f16*, float*, const int*, int, int, int, int,
+                                               cudaStream_t);
+template cudaError_t launch_attn_bwd_simt<f16>(const f16*, const f16*, const f16*, const float*, float*,
+                                               const int*, f16*, int, int, int, int, cudaStream_t);

@@ -40,21 +40,6 @@ __device__ __forceinline__ uint32_t pk_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Row r of a [128 rows x 128 bf16] K-major operand stored as two 16 KB
-// 128-byte-swizzled column blocks; write 32 values at columns c0..c0+31.
-__device__ __forceinline__ void st_row32_bf16(uint32_t base, int r, int c0, const float* v) {
-  const uint32_t blk = base + (c0 >> 6) * AT_TILE_BYTES + r * 128;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int u = ((c0 & 63) >> 3) + q;
-    uint32_t a = blk + ((u ^ (r & 7)) << 4);
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk_bf16(v[8 * q], v[8 * q + 1])),
-                 "r"(pk_bf16(v[8 * q + 2], v[8 * q + 3])), "r"(pk_bf16(v[8 * q + 4], v[8 * q + 5])),
-                 "r"(pk_bf16(v[8 * q + 6], v[8 * q + 7]))
-                 : "memory");
-  }
-}
-
 // Bounded barrier among the 128 softmax threads (an mbarrier with count 128):
 // every thread arrives, then waits for the phase to complete.
 __device__ __forceinline__ bool group_sync(uint32_t bar, uint32_t& phase, volatile int* abort_flag) {
@@ -71,21 +56,6 @@ __device__ __forceinline__ void trap_timeout(volatile int* abort_flag, unsigned*
 
 #define AT_BK 64                             // iterated block (keys in fwd / dQ, queries in dK dV)
 #define AT_HALF (AT_BK * AT_D * 2)           // 8 KB: 64 rows x 128 B
-
-// Write 32 bf16 values at columns c0..c0+31 (< 64) of row r of a 64-column
-// K-major operand (rows of 128 B, 128-byte swizzle).
-__device__ __forceinline__ void st_row32_64(uint32_t base, int r, int c0, const float* v) {
-  const uint32_t rowb = base + r * 128;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int u = (c0 >> 3) + q;
-    uint32_t a = rowb + ((u ^ (r & 7)) << 4);
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk_bf16(v[8 * q], v[8 * q + 1])),
-                 "r"(pk_bf16(v[8 * q + 2], v[8 * q + 3])), "r"(pk_bf16(v[8 * q + 4], v[8 * q + 5])),
-                 "r"(pk_bf16(v[8 * q + 6], v[8 * q + 7]))
-                 : "memory");
-  }
-}
 
 __device__ __forceinline__ void tc_alloc(uint32_t slot, int cols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(cols));
@@ -133,46 +103,139 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
-// Forward softmax over one 32-key chunk of a score row.  Masked chunks keep
-// key e (0..31) when lo <= e <= hi (lo, hi relative to the chunk start); the
-// test is branch-free: ((e - lo) | (hi - e)) >= 0.
-template <bool MASK>
-__device__ __forceinline__ float fwd_chunk_max(const uint32_t* sr, int lo, int hi) {
-  float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent chains
-#pragma unroll
-  for (int e = 0; e < 32; ++e) {
-    const float v = __uint_as_float(sr[e]);
-    m4[e & 3] = fmaxf(m4[e & 3], (!MASK || ((e - lo) | (hi - e)) >= 0) ? v : -INFINITY);
-  }
-  return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+// Packed fp32 pairs (sm_100): (d0, d1) = (a0, a1) * b + c and (a0, a1) + (b0, b1).
+__device__ __forceinline__ void fma_x2(float& d0, float& d1, float a0, float a1, float b, float c) {
+  asm("{\n.reg .b64 ra, rb, rc, rd;\nmov.b64 ra, {%2, %3};\nmov.b64 rb, {%4, %4};\nmov.b64 rc, {%5, %5};\n"
+      "fma.rn.f32x2 rd, ra, rb, rc;\nmov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b), "f"(c));
 }
-template <bool MASK>
-__device__ __forceinline__ float fwd_chunk_exp(const uint32_t* sr, int lo, int hi, float sl2, float mb, uint32_t* pw) {
-  float l2[2] = {0.f, 0.f};
+__device__ __forceinline__ void add_x2(float& a0, float& a1, float b0, float b1) {
+  asm("{\n.reg .b64 ra, rb;\nmov.b64 ra, {%0, %1};\nmov.b64 rb, {%2, %3};\n"
+      "add.rn.f32x2 ra, ra, rb;\nmov.b64 {%0, %1}, ra;\n}\n"
+      : "+f"(a0), "+f"(a1) : "f"(b0), "f"(b1));
+}
+
+__device__ __forceinline__ void fma_x2v(float& d0, float& d1, float a0, float a1, float b0, float b1, float c) {
+  asm("{\n.reg .b64 ra, rb, rc, rd;\nmov.b64 ra, {%2, %3};\nmov.b64 rb, {%4, %5};\nmov.b64 rc, {%6, %6};\n"
+      "fma.rn.f32x2 rd, ra, rb, rc;\nmov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c));
+}
+
+// 2^x for a pair of arguments on the FMA pipe instead of the MUFU unit:
+// x = n + f with n = round(x) (the 1.5 * 2^23 rounding trick) and f in
+// [-1/2, 1/2]; 2^f by a cubic fitted here as a near-minimax relative
+// approximation on that interval (max relative error 7.7e-5, about 2^-13.7,
+// far below the 2^-9 of the bf16 P it feeds); 2^n is added to the exponent
+// field.  Arguments below -126 are clamped (their P is 0 in bf16 anyway).
+#define EXP2_C0 0.99992877245f
+#define EXP2_C1 0.69326078892f
+#define EXP2_C2 0.24260069430f
+#define EXP2_C3 0.05516735464f
+__device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& y0, float& y1) {
+  const float RND = 12582912.0f;   // 1.5 * 2^23
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  float t0 = x0, t1 = x1;
+  add_x2(t0, t1, RND, RND);
+  float n0 = t0, n1 = t1;
+  add_x2(n0, n1, -RND, -RND);
+  float f0 = x0, f1 = x1;
+  add_x2(f0, f1, -n0, -n1);
+  float p0, p1;
+  fma_x2v(p0, p1, f0, f1, EXP2_C3, EXP2_C3, EXP2_C2);
+  fma_x2v(p0, p1, p0, p1, f0, f1, EXP2_C1);
+  fma_x2v(p0, p1, p0, p1, f0, f1, EXP2_C0);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+// Pairs k of a 32-score chunk (k = 0..15) with (k & 7) < FW_POLY_PAIRS take
+// the polynomial, the others the MUFU ex2: the two units run side by side.
+#ifndef FW_POLY_PAIRS
+#define FW_POLY_PAIRS 3
+#endif
+
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// One 32-score chunk of a row: fold the (masked) raw scores into mx
+// (three-input max), write P = exp2(s sl2 - mb) as 16 packed 16-bit pairs at
+// TMEM column tP and add their sum to sum.  Masked chunks keep key e (0..31)
+// when lo <= e <= hi (relative to the chunk), branch-free:
+// ((e - lo) | (hi - e)) >= 0.  The exponent arguments and the sums run as
+// packed fp32 pairs.
+template <bool MASK, bool F16>
+__device__ __forceinline__ void fwd_chunk(const uint32_t* sr, int lo, int hi, float sl2, float mb, uint32_t tP,
+                                          float& mx, float& sum) {
+  float l0 = 0.f, l1 = 0.f;
+  uint32_t pw[16];
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
-    float p0 = ex2_approx(fmaf(__uint_as_float(sr[e]), sl2, -mb));
-    float p1 = ex2_approx(fmaf(__uint_as_float(sr[e + 1]), sl2, -mb));
+    float s0 = __uint_as_float(sr[e]), s1 = __uint_as_float(sr[e + 1]);
     if (MASK) {
-      p0 = ((e - lo) | (hi - e)) >= 0 ? p0 : 0.f;
-      p1 = ((e + 1 - lo) | (hi - e - 1)) >= 0 ? p1 : 0.f;
+      s0 = ((e - lo) | (hi - e)) >= 0 ? s0 : -INFINITY;
+      s1 = ((e + 1 - lo) | (hi - e - 1)) >= 0 ? s1 : -INFINITY;
     }
-    l2[(e >> 1) & 1] += p0 + p1;
-    pw[e / 2] = pk_bf16(p0, p1);
+    mx = fmax3f(mx, s0, s1);
+    float x0, x1;
+    fma_x2(x0, x1, s0, s1, sl2, -mb);
+    float p0, p1;
+    if (((e >> 1) & 7) < FW_POLY_PAIRS) {
+      exp2_poly_x2(x0, x1, p0, p1);
+      if (MASK) {   // the polynomial maps -inf to a tiny value, not 0
+        p0 = s0 == -INFINITY ? 0.f : p0;
+        p1 = s1 == -INFINITY ? 0.f : p1;
+      }
+    } else {
+      p0 = ex2_approx(x0);
+      p1 = ex2_approx(x1);
+    }
+    add_x2(l0, l1, p0, p1);
+    pw[e / 2] = pack16x2<F16>(p0, p1);
   }
-  return l2[0] + l2[1];
+  sum += l0 + l1;
+  tmem_st16(tP, pw);
+}
+
+// One pass over a row's 128 scores at tS (writing P at tP): four chunks of
+// 32, each chunk's TMEM load issued before the previous chunk's arithmetic
+// (tcgen05.wait::ld waits for every load in flight, so each wait covers a
+// load that had a chunk of arithmetic to land).  One code body per mask
+// variant keeps the score loop within the instruction cache.
+template <bool MASK, bool F16>
+__device__ __forceinline__ void fwd_pass(uint32_t tS, uint32_t tP, int lo, int hi, float sl2, float mb, float& mx,
+                                         float& sum) {
+  uint32_t ra[32], rb[32];
+  tmem_ld32(tS, ra);
+  tmem_wait_ld();
+#pragma unroll 1
+  for (int c = 0; c < 4; c += 2) {
+    tmem_ld32(tS + 32 * (c + 1), rb);
+    fwd_chunk<MASK, F16>(ra, lo - 32 * c, hi - 32 * c, sl2, mb, tP + 16 * c, mx, sum);
+    tmem_wait_ld();
+    if (c + 2 < 4) tmem_ld32(tS + 32 * (c + 2), ra);
+    fwd_chunk<MASK, F16>(rb, lo - 32 * (c + 1), hi - 32 * (c + 1), sl2, mb, tP + 16 * (c + 1), mx, sum);
+    tmem_wait_ld();
+  }
 }
 
 // ============================================================== forward
 // CTA = two 128-query tiles (256 queries) sharing each 128-key block of K
 // and V.  Per tile g and key block j:
 //   S_g = Q_g K_j^T                (TMEM, 128 x 128 fp32)
-//   P_g = exp2(S_g log2e / 8 - m)  (bf16 pairs written back over S_g)
+//   P_g = exp2(S_g log2e / 8 - m)  (bf16 pairs, TMEM columns beside O_g)
 //   O_g += P_g V_j                 (TMEM, 128 x 64 fp32, A operand from TMEM)
 // The MMA warp alternates between the tiles so that one tile's softmax runs
 // while the other tile's products are computed.  The running max m is only
 // raised (and O, l rescaled) when a row's block max exceeds it by more than
-// 2^8; otherwise the stale max is kept, which bounds every P by 256.
+// 2^8; otherwise the stale max is kept, which bounds every P by 256.  After a
+// row's first block, each half of the score row is read from TMEM once: the
+// exponentials use the running max while the block max is tracked, and only a
+// block whose max rose past the threshold is exponentiated again (S is still
+// intact, since P has its own columns).
 // 320 threads: warp 0 loads, warp 1 issues MMAs, warps 2-5 (tile 0) and 6-9
 // (tile 1) run the softmax, thread t of a group owning query row t.
 #define FW_THREADS 320
@@ -184,12 +247,13 @@ struct FwdSmem {
   static constexpr int KV = Q + 2 * AT_TILE_BYTES;   // FW_ST stages x (K 16 KB, V 16 KB)
   static constexpr int BAR = KV + FW_ST * 2 * AT_TILE_BYTES;
   static constexpr int TOTAL = BAR + 256;
-  static constexpr int TMEM_COLS = 512;              // tile g: S (P over its first 64 columns) at 256g, O at 256g + 128
+  static constexpr int TMEM_COLS = 512;              // tile g: S at 256g, O at 256g + 128, P at 256g + 192
 };
 
+template <bool F16>
 __global__ void __launch_bounds__(FW_THREADS, 1)
 attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, float* __restrict__ lse,
-            const int* __restrict__ dstart, int T, int H, unsigned* err) {
+            const int* __restrict__ dstart, int T, int H, int kcol0, int vcol0, int G, unsigned* err) {
   extern __shared__ __align__(1024) uint8_t at_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)at_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = (uint64_t*)(sm + FwdSmem::BAR);
@@ -255,8 +319,8 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
       if (!mbar_wait(bar(KV_EMPTY + st), ((n / FW_ST) & 1) ^ 1, abort_flag)) { ok = false; break; }
       mbar_expect_tx(bar(KV_FULL + st), 2 * AT_TILE_BYTES);
       const uint32_t dst = sKV + st * 2 * AT_TILE_BYTES;
-      tma_load_2d(dst, &tmQKV, bar(KV_FULL + st), C + h * AT_D, (int)(rowbase + j * AT_BLK));
-      tma_load_2d(dst + AT_TILE_BYTES, &tmQKV, bar(KV_FULL + st), 2 * C + h * AT_D, (int)(rowbase + j * AT_BLK));
+      tma_load_2d(dst, &tmQKV, bar(KV_FULL + st), kcol0 + (h / G) * AT_D, (int)(rowbase + j * AT_BLK));
+      tma_load_2d(dst + AT_TILE_BYTES, &tmQKV, bar(KV_FULL + st), vcol0 + (h / G) * AT_D, (int)(rowbase + j * AT_BLK));
     }
     if (!ok) trap_timeout(abort_flag, err);
     volatile int never = 0;
@@ -265,8 +329,8 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
     for (int n = max(0, nj - FW_ST); n < nj; ++n) mbar_wait(bar(KV_FULL + n % FW_ST), (n / FW_ST) & 1, &never, 1ll << 28);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer: S_0(j+1) is issued right after P_0 V(j), then P_1 V(j), S_1(j+1)
-    constexpr uint32_t ID_S = instr_desc(128, false, false);   // S = Q K^T: 128 x 128, K = 64
-    constexpr uint32_t ID_O = instr_desc(64, false, true);     // O = P V: 128 x 64, K = 128 keys (V MN-major)
+    constexpr uint32_t ID_S = instr_desc_t(F16, 128, false, false);   // S = Q K^T: 128 x 128, K = 64
+    constexpr uint32_t ID_O = instr_desc_t(F16, 64, false, true);     // O = P V: 128 x 64, K = 128 keys (V MN-major)
     bool ok = mbar_wait(bar(Q_FULL), 0, abort_flag);
     int ns[2] = {0, 0}, np[2] = {0, 0};   // S and P V products issued per tile
     auto kv_wait = [&](int j) {
@@ -293,7 +357,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
       const uint32_t sV = sKV + ((j - jlo) % FW_ST) * 2 * AT_TILE_BYTES + AT_TILE_BYTES;
 #pragma unroll
       for (int kk = 0; kk < AT_BLK / 16; ++kk)
-        umma_bf16_ts(tmem + 256 * g + 128, tmem + 256 * g + 8 * kk, mndesc(sV + kk * 2048, 8192), ID_O,
+        umma_bf16_ts(tmem + 256 * g + 128, tmem + 256 * g + 192 + 8 * kk, mndesc(sV + kk * 2048, 8192), ID_O,
                      (np[g] > 0 || kk > 0));
       umma_commit(bar(O_DONE + g));
       ++np[g];
@@ -325,7 +389,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
     const int lo = g == 0 ? lo0 : lo1, hi = g == 0 ? hi0 : hi1;
     const int qlast = min(q0 + 128 * g + 127, T - 1);
     const int ds_last = ld_once(dsr + qlast);
-    const uint32_t tS = tmem + 256 * g + ((uint32_t)(quarter * 32) << 16), tO = tS + 128;
+    const uint32_t tS = tmem + 256 * g + ((uint32_t)(quarter * 32) << 16), tO = tS + 128, tP = tS + 192;
     const float sl2 = 0.125f * LOG2E_F;   // 1/sqrt(64) in the exp2 domain
     auto wait_w = [&](uint32_t bb, uint32_t parity) { return __all_sync(0xffffffffu, mbar_wait(bb, parity, abort_flag)); };
     float m_use = -INFINITY, l = 0.f;
@@ -339,27 +403,28 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
         // masked blocks: a key may be later than a query or before its document
         // (voted warp-wide so the warp runs one code path)
         const bool need_mask = __any_sync(0xffffffffu, kb0 + AT_BLK - 1 > q0 + 128 * g || ds_last > kb0 || !qv);
-        // pass 1: row max of the block
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t sr[32];
-          tmem_ld32(tS + 32 * c, sr);
-          tmem_wait_ld();
-          const int base = kb0 + 32 * c;
-          mx = fmaxf(mx, need_mask ? fwd_chunk_max<true>(sr, ds_q - base, q - base) : fwd_chunk_max<false>(sr, 0, 0));
-        }
-        mx *= sl2;
-        // raise the max (rescaling O and l) only when it grew by more than 2^FW_RESCALE
-        const bool raise = mx > m_use + FW_RESCALE;
-        if (__any_sync(0xffffffffu, raise)) {
+        const int lo_h = ds_q - kb0, hi_h = q - kb0;   // allowed keys relative to the block
+        // exponentiate with the running max while tracking the block max; a
+        // block whose max rose more than 2^FW_RESCALE above the running one
+        // (always the row's first block, whose running max is -inf) raises
+        // it, rescales O and l, and is exponentiated again (S is intact: P
+        // has its own columns)
+        float bsum, mx;
+        float mb = m_use == -INFINITY ? 0.f : m_use;
+        while (true) {
+          bsum = 0.f;
+          mx = -INFINITY;
+          if (need_mask) fwd_pass<true, F16>(tS, tP, lo_h, hi_h, sl2, mb, mx, bsum);
+          else fwd_pass<false, F16>(tS, tP, lo_h, hi_h, sl2, mb, mx, bsum);
+          mx *= sl2;
+          if (!__any_sync(0xffffffffu, mx > m_use + FW_RESCALE)) break;
           const float m_new = fmaxf(m_use, mx);
-          const float sc = m_use == -INFINITY ? 0.f : exp2f(m_use - m_new);
           if (n > 0) {
             // O holds P V of every earlier block: wait for the last one, then scale it
+            const float sc = m_use == -INFINITY ? 0.f : exp2f(m_use - m_new);
             if (!wait_w(bar(O_DONE + g), (n - 1) & 1)) { ok = false; break; }
             tc_fence_after();
-#pragma unroll
+#pragma unroll 1
             for (int c = 0; c < 2; ++c) {
               uint32_t orr[32];
               tmem_ld32(tO + 32 * c, orr);
@@ -368,23 +433,14 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
               for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * sc);
               tmem_st32(tO + 32 * c, orr);
             }
-            tmem_wait_st();
+            l *= sc;
           }
-          l *= sc;
           m_use = m_new;
+          mb = m_use == -INFINITY ? 0.f : m_use;
+          tmem_wait_st();   // the first P of this block is replaced by the next pass
         }
-        const float mb = m_use == -INFINITY ? 0.f : m_use;
-        // pass 2: P = exp2(S sl2 - m) as bf16 pairs over the first 64 columns of S
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t sr[32], pw[16];
-          tmem_ld32(tS + 32 * c, sr);
-          tmem_wait_ld();
-          const int base = kb0 + 32 * c;
-          l += need_mask ? fwd_chunk_exp<true>(sr, ds_q - base, q - base, sl2, mb, pw)
-                         : fwd_chunk_exp<false>(sr, 0, 0, sl2, mb, pw);
-          tmem_st16(tS + 16 * c, pw);
-        }
+        if (!ok) break;
+        l += bsum;
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -406,10 +462,10 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             uint4 w;
-            w.x = pk_bf16(__uint_as_float(orr[8 * u]) * inv, __uint_as_float(orr[8 * u + 1]) * inv);
-            w.y = pk_bf16(__uint_as_float(orr[8 * u + 2]) * inv, __uint_as_float(orr[8 * u + 3]) * inv);
-            w.z = pk_bf16(__uint_as_float(orr[8 * u + 4]) * inv, __uint_as_float(orr[8 * u + 5]) * inv);
-            w.w = pk_bf16(__uint_as_float(orr[8 * u + 6]) * inv, __uint_as_float(orr[8 * u + 7]) * inv);
+            w.x = pack16x2<F16>(__uint_as_float(orr[8 * u]) * inv, __uint_as_float(orr[8 * u + 1]) * inv);
+            w.y = pack16x2<F16>(__uint_as_float(orr[8 * u + 2]) * inv, __uint_as_float(orr[8 * u + 3]) * inv);
+            w.z = pack16x2<F16>(__uint_as_float(orr[8 * u + 4]) * inv, __uint_as_float(orr[8 * u + 5]) * inv);
+            w.w = pack16x2<F16>(__uint_as_float(orr[8 * u + 6]) * inv, __uint_as_float(orr[8 * u + 7]) * inv);
             *reinterpret_cast<uint4*>(orow + 32 * c + 8 * u) = w;
           }
         }
@@ -455,14 +511,14 @@ struct BwdSmem {
   static constexpr int TMEM_COLS = 512;
 };
 
-// 32 columns of P^T and dS^T for one key row: p = exp2(s sl2 - lse2), ds = p (dp - D),
-// packed into bf16 pairs.  MASK applies causality and document starts.
-template <bool MASK>
-__device__ __forceinline__ void bwd_elementwise32(const uint32_t* sr, const uint32_t* dr, const float* L2,
-                                                  const float* Dq, const int* DSq, int q_first, int k, float sl2,
-                                                  uint32_t* pw, uint32_t* dw) {
+// NC columns of P^T and dS^T for one key row: p = exp2(s sl2 - lse2), ds = p (dp - D),
+// packed into 16-bit pairs.  MASK applies causality and document starts.
+template <bool MASK, bool F16, int NC>
+__device__ __forceinline__ void bwd_elementwise(const uint32_t* sr, const uint32_t* dr, const float* L2,
+                                                const float* Dq, const int* DSq, int q_first, int k, float sl2,
+                                                uint32_t* pw, uint32_t* dw) {
 #pragma unroll
-  for (int c8 = 0; c8 < 32; c8 += 8) {
+  for (int c8 = 0; c8 < NC; c8 += 8) {
     const float4 la = *reinterpret_cast<const float4*>(L2 + c8), lb = *reinterpret_cast<const float4*>(L2 + c8 + 4);
     const float4 da = *reinterpret_cast<const float4*>(Dq + c8), db = *reinterpret_cast<const float4*>(Dq + c8 + 4);
     const float lv[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
@@ -483,16 +539,18 @@ __device__ __forceinline__ void bwd_elementwise32(const uint32_t* sr, const uint
     }
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      pw[c8 / 2 + e] = pk_bf16(pv[2 * e], pv[2 * e + 1]);
-      dw[c8 / 2 + e] = pk_bf16(gv[2 * e], gv[2 * e + 1]);
+      pw[c8 / 2 + e] = pack16x2<F16>(pv[2 * e], pv[2 * e + 1]);
+      dw[c8 / 2 + e] = pack16x2<F16>(gv[2 * e], gv[2 * e + 1]);
     }
   }
 }
 
+template <bool F16>
 __global__ void __launch_bounds__(BW_THREADS, 1)
 attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
             const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ lse, const float* __restrict__ Dbuf,
-            const int* __restrict__ dstart, bf16* __restrict__ dqkv, int T, int H, unsigned* err) {
+            const int* __restrict__ dstart, int T, int H, int kcol0, int vcol0, int G, bf16* __restrict__ dkv,
+            long ld_kv, int v_off, unsigned* err) {
   extern __shared__ __align__(1024) uint8_t at_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)at_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = (uint64_t*)(sm + BwdSmem::BAR);
@@ -569,8 +627,8 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQKV)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmDO)) : "memory");
       mbar_expect_tx(bar(KV_FULL), 2 * AT_TILE_BYTES);
-      tma_load_2d(sK, &tmQKV, bar(KV_FULL), C + h * AT_D, (int)(rowbase + k0));
-      tma_load_2d(sV, &tmQKV, bar(KV_FULL), 2 * C + h * AT_D, (int)(rowbase + k0));
+      tma_load_2d(sK, &tmQKV, bar(KV_FULL), kcol0 + (h / G) * AT_D, (int)(rowbase + k0));
+      tma_load_2d(sV, &tmQKV, bar(KV_FULL), vcol0 + (h / G) * AT_D, (int)(rowbase + k0));
     }
     bool ok = true;
     for (int i = 0; i < niter; ++i) {
@@ -614,9 +672,9 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
-    constexpr uint32_t ID_SS = instr_desc(128, false, false);   // S^T, dP^T: 128 keys x 128 queries, K = d
-    constexpr uint32_t ID_KV = instr_desc(64, false, true);     // dV, dK: 128 keys x 64, K = 128 queries
-    constexpr uint32_t ID_DQ = instr_desc(64, true, true);      // dQ: 128 queries x 64, K = 128 keys
+    constexpr uint32_t ID_SS = instr_desc_t(F16, 128, false, false);   // S^T, dP^T: 128 keys x 128 queries, K = d
+    constexpr uint32_t ID_KV = instr_desc_t(F16, 64, false, true);     // dV, dK: 128 keys x 64, K = 128 queries
+    constexpr uint32_t ID_DQ = instr_desc_t(F16, 64, true, true);      // dQ: 128 queries x 64, K = 128 keys
     bool ok = mbar_wait(bar(KV_FULL), 0, abort_flag);
     auto issue_s = [&](int i) -> bool {   // S^T and dP^T of query block i
       const int st = i % BW_ST;
@@ -706,25 +764,43 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
       // masking only where a key can be later than a query or before its document
       // (document starts never decrease, queries past T carry INT_MAX)
       const bool need_mask = q0 < k0 + AT_BLK || DSq[BW_QB - 1 - 64 * grp] > k0;
+      // four 16-column quarters of the group's 64 query columns, each
+      // quarter's S^T / dP^T loads issued before the previous quarter's
+      // arithmetic (a TMEM load wait covers every load in flight)
       uint32_t pw[32], dw[32];
+      uint32_t sa[16], da[16], sb[16], db[16];
+      const uint32_t tSg = tmem + lane_off + 64 * grp, tDg = tmem + lane_off + 128 + 64 * grp;
+      const int qf = q0 + 64 * grp;
+      tmem_ld16(tSg, sa);
+      tmem_ld16(tDg, da);
+      tmem_wait_ld();
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t sr[32], dr[32];
-        tmem_ld32(tmem + lane_off + 64 * grp + 32 * half, sr);
-        tmem_ld32(tmem + lane_off + 128 + 64 * grp + 32 * half, dr);
+      for (int qt = 0; qt < 4; qt += 2) {
+        tmem_ld16(tSg + 16 * (qt + 1), sb);
+        tmem_ld16(tDg + 16 * (qt + 1), db);
+        if (need_mask)
+          bwd_elementwise<true, F16, 16>(sa, da, L2 + 16 * qt, Dq + 16 * qt, DSq + 16 * qt, qf + 16 * qt, k, sl2,
+                                         pw + 8 * qt, dw + 8 * qt);
+        else
+          bwd_elementwise<false, F16, 16>(sa, da, L2 + 16 * qt, Dq + 16 * qt, DSq + 16 * qt, qf + 16 * qt, k, sl2,
+                                          pw + 8 * qt, dw + 8 * qt);
         tmem_wait_ld();
-        if (half == 1) {
+        if (qt + 2 < 4) {
+          tmem_ld16(tSg + 16 * (qt + 2), sa);
+          tmem_ld16(tDg + 16 * (qt + 2), da);
+        } else {
+          // every S^T / dP^T value of this block is in registers
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(S_FREE));   // S^T / dP^T may be overwritten
         }
-        const int qf = q0 + 64 * grp + 32 * half;
         if (need_mask)
-          bwd_elementwise32<true>(sr, dr, L2 + 32 * half, Dq + 32 * half, DSq + 32 * half, qf, k, sl2, pw + 16 * half,
-                                  dw + 16 * half);
+          bwd_elementwise<true, F16, 16>(sb, db, L2 + 16 * (qt + 1), Dq + 16 * (qt + 1), DSq + 16 * (qt + 1),
+                                         qf + 16 * (qt + 1), k, sl2, pw + 8 * (qt + 1), dw + 8 * (qt + 1));
         else
-          bwd_elementwise32<false>(sr, dr, L2 + 32 * half, Dq + 32 * half, DSq + 32 * half, qf, k, sl2,
-                                   pw + 16 * half, dw + 16 * half);
+          bwd_elementwise<false, F16, 16>(sb, db, L2 + 16 * (qt + 1), Dq + 16 * (qt + 1), DSq + 16 * (qt + 1),
+                                          qf + 16 * (qt + 1), k, sl2, pw + 8 * (qt + 1), dw + 8 * (qt + 1));
+        if (qt + 2 < 4) tmem_wait_ld();
       }
       // the previous block's P^T / dS^T have been consumed and its dQ is complete
       if (i > 0 && !wait_w(bar(MMA_DONE), (i - 1) & 1)) { ok = false; break; }
@@ -755,11 +831,11 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
       tc_fence_after();
       ok = flush_dq(niter - 1);
       if (ok) {
-        bf16* row = dqkv + (rowbase + k) * 3 * C;
+        bf16* row = dkv + (rowbase + k) * ld_kv;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
           const float sc = part == 0 ? 0.125f : 1.f;
-          bf16* dst = row + (part == 0 ? C : 2 * C) + h * AT_D + 32 * grp;
+          bf16* dst = row + (part == 0 ? 0 : v_off) + h * AT_D + 32 * grp;
           uint32_t rr[32];
           tmem_ld32(tmem + lane_off + (part == 0 ? 320 : 256) + 32 * grp, rr);
           tmem_wait_ld();
@@ -767,10 +843,10 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             uint4 w;
-            w.x = pk_bf16(__uint_as_float(rr[8 * u]) * sc, __uint_as_float(rr[8 * u + 1]) * sc);
-            w.y = pk_bf16(__uint_as_float(rr[8 * u + 2]) * sc, __uint_as_float(rr[8 * u + 3]) * sc);
-            w.z = pk_bf16(__uint_as_float(rr[8 * u + 4]) * sc, __uint_as_float(rr[8 * u + 5]) * sc);
-            w.w = pk_bf16(__uint_as_float(rr[8 * u + 6]) * sc, __uint_as_float(rr[8 * u + 7]) * sc);
+            w.x = pack16x2<F16>(__uint_as_float(rr[8 * u]) * sc, __uint_as_float(rr[8 * u + 1]) * sc);
+            w.y = pack16x2<F16>(__uint_as_float(rr[8 * u + 2]) * sc, __uint_as_float(rr[8 * u + 3]) * sc);
+            w.z = pack16x2<F16>(__uint_as_float(rr[8 * u + 4]) * sc, __uint_as_float(rr[8 * u + 5]) * sc);
+            w.w = pack16x2<F16>(__uint_as_float(rr[8 * u + 6]) * sc, __uint_as_float(rr[8 * u + 7]) * sc);
             *reinterpret_cast<uint4*>(dst + 8 * u) = w;
           }
         }
@@ -803,8 +879,9 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
   if (warp == 0) tc_dealloc(tmem, BwdSmem::TMEM_COLS);
 }
 
-// dq[row, head h] = bf16(dQacc / 8); the accumulator is cleared for the next use.
-__global__ void attn_dq_finish_kernel(float* __restrict__ dq_acc, bf16* __restrict__ dqkv, long rows, int C) {
+// dq[row, head h] = bf16 or fp16 (F16) of dQacc / 8; the accumulator is cleared for the next use.
+template <bool F16>
+__global__ void attn_dq_finish_kernel(float* __restrict__ dq_acc, bf16* __restrict__ dqkv, long rows, int C, long ld_q) {
   const long n8 = rows * C / 8;
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n8; i += (long)gridDim.x * blockDim.x) {
     const long e = i * 8, row = e / C;
@@ -812,17 +889,18 @@ __global__ void attn_dq_finish_kernel(float* __restrict__ dq_acc, bf16* __restri
     float4* src = reinterpret_cast<float4*>(dq_acc + e);
     const float4 a = src[0], bq = src[1];
     uint4 w;
-    w.x = pk_bf16(a.x * 0.125f, a.y * 0.125f);
-    w.y = pk_bf16(a.z * 0.125f, a.w * 0.125f);
-    w.z = pk_bf16(bq.x * 0.125f, bq.y * 0.125f);
-    w.w = pk_bf16(bq.z * 0.125f, bq.w * 0.125f);
-    *reinterpret_cast<uint4*>(dqkv + row * 3 * C + c) = w;
+    w.x = pack16x2<F16>(a.x * 0.125f, a.y * 0.125f);
+    w.y = pack16x2<F16>(a.z * 0.125f, a.w * 0.125f);
+    w.z = pack16x2<F16>(bq.x * 0.125f, bq.y * 0.125f);
+    w.w = pack16x2<F16>(bq.z * 0.125f, bq.w * 0.125f);
+    *reinterpret_cast<uint4*>(dqkv + row * ld_q + c) = w;
     src[0] = make_float4(0.f, 0.f, 0.f, 0.f);
     src[1] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 
 // D[b, h, t] = dO[b*T+t, head h] . O[b*T+t, head h]   (one thread per (row, head))
+template <bool F16>
 __global__ void attn_rowdot_kernel(const bf16* __restrict__ out, const bf16* __restrict__ dout, float* __restrict__ Dbuf,
                                    int B, int T, int H) {
   long i = blockIdx.x * (long)blockDim.x + threadIdx.x;
@@ -835,8 +913,8 @@ __global__ void attn_rowdot_kernel(const bf16* __restrict__ out, const bf16* __r
 #pragma unroll
   for (int c = 0; c < AT_D; c += 8) {
     float x[8], y[8];
-    Vec<bf16>::load(dout + off + c, x);
-    Vec<bf16>::load(out + off + c, y);
+    unpack16x8<F16>(*reinterpret_cast<const uint4*>(dout + off + c), x);
+    unpack16x8<F16>(*reinterpret_cast<const uint4*>(out + off + c), y);
 #pragma unroll
     for (int k = 0; k < 8; ++k) acc += x[k] * y[k];
   }
@@ -851,35 +929,58 @@ static cudaError_t tc_smem_attr(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-cudaError_t launch_attn_fwd_tc(const bf16* qkv, bf16* out, float* lse, const int* dstart, int B, int T, int H,
-                               unsigned* err, cudaStream_t s) {
-  const int C = H * AT_D;
+AttnLayout attn_layout_mha(bf16* dqkv, int C) {
+  AttnLayout a;
+  a.qw = 3 * C; a.kcol = C; a.vcol = 2 * C; a.G = 1;
+  a.dkv = dqkv ? dqkv + C : nullptr; a.ld_kv = 3L * C; a.v_off = C;
+  return a;
+}
+
+template <bool F16>
+static cudaError_t attn_fwd_tc_t(const bf16* qkv, bf16* out, float* lse, const int* dstart, int B, int T, int H,
+                                 unsigned* err, cudaStream_t s, const AttnLayout& L) {
   const long rows = (long)B * T;
   CUtensorMap tqkv;
-  if (!make_map_ex(&tqkv, MapKey{qkv, rows, 3L * C, 3L * C, 1, 0, AT_D, AT_BLK, 0, 128})) return cudaErrorInvalidValue;
+  if (!make_map_ex(&tqkv, MapKey{qkv, rows, (long)L.qw, (long)L.qw, 1, 0, AT_D, AT_BLK, 0, 128}))
+    return cudaErrorInvalidValue;
   const int smem = FwdSmem::TOTAL + 1024;
   static bool attr = false;
-  if (!attr) { cudaError_t e = tc_smem_attr(attn_fwd_tc, smem); if (e) return e; attr = true; }
+  if (!attr) { cudaError_t e = tc_smem_attr(attn_fwd_tc<F16>, smem); if (e) return e; attr = true; }
   dim3 grid(B * H, (T + FW_QT - 1) / FW_QT);
   ++g_kernel_launches;
-  attn_fwd_tc<<<grid, FW_THREADS, smem, s>>>(tqkv, out, lse, dstart, T, H, err);
+  attn_fwd_tc<F16><<<grid, FW_THREADS, smem, s>>>(tqkv, out, lse, dstart, T, H, L.kcol, L.vcol, L.G, err);
   return cudaGetLastError();
 }
 
-cudaError_t launch_attn_bwd_tc(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* Dbuf,
-                               bool d_ready, float* dq_acc, const int* dstart, bf16* dqkv, int B, int T, int H,
-                               unsigned* err, cudaStream_t s) {
+static bool layout_ok(const AttnLayout& L, int H) {
+  // 16-byte aligned TMA columns and row strides; whole key / value groups
+  return L.G >= 1 && H % L.G == 0 && L.qw % 8 == 0 && L.kcol % 8 == 0 && L.vcol % 8 == 0 && L.ld_kv % 8 == 0 &&
+         L.v_off % 8 == 0;
+}
+
+cudaError_t launch_attn_fwd_tc(const bf16* qkv, bf16* out, float* lse, const int* dstart, int B, int T, int H,
+                               unsigned* err, cudaStream_t s, bool f16, const AttnLayout* lay) {
+  const AttnLayout L = lay ? *lay : attn_layout_mha(nullptr, H * AT_D);
+  if (!layout_ok(L, H)) return cudaErrorInvalidValue;
+  return f16 ? attn_fwd_tc_t<true>(qkv, out, lse, dstart, B, T, H, err, s, L)
+             : attn_fwd_tc_t<false>(qkv, out, lse, dstart, B, T, H, err, s, L);
+}
+
+template <bool F16>
+static cudaError_t attn_bwd_tc_t(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* Dbuf,
+                                 bool d_ready, float* dq_acc, const int* dstart, bf16* dqkv, int B, int T, int H,
+                                 unsigned* err, cudaStream_t s, const AttnLayout& L) {
   const int C = H * AT_D;
   const long rows = (long)B * T;
   CUtensorMap tqkv, tdo, tdq;
-  if (!make_map_ex(&tqkv, MapKey{qkv, rows, 3L * C, 3L * C, 1, 0, AT_D, AT_BLK, 0, 128}) ||
+  if (!make_map_ex(&tqkv, MapKey{qkv, rows, (long)L.qw, (long)L.qw, 1, 0, AT_D, AT_BLK, 0, 128}) ||
       !make_map_ex(&tdo, MapKey{dout, rows, (long)C, (long)C, 1, 0, AT_D, BW_QB, 0, 128}) ||
       !make_map_ex(&tdq, MapKey{dq_acc, rows, (long)C, (long)C, 1, 0, 32, BW_QB, 1, 128}))
     return cudaErrorInvalidValue;
   const int smem = BwdSmem::TOTAL + 1024;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = tc_smem_attr(attn_bwd_tc, smem);
+    cudaError_t e = tc_smem_attr(attn_bwd_tc<F16>, smem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
@@ -887,14 +988,24 @@ cudaError_t launch_attn_bwd_tc(const bf16* qkv, const bf16* out, const bf16* dou
   if (!d_ready) {   // D = rowsum(dO o O), unless the producer of dO already wrote it
     long n = rows * H;
     ++g_kernel_launches;
-    attn_rowdot_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(out, dout, Dbuf, B, T, H);
+    attn_rowdot_kernel<F16><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(out, dout, Dbuf, B, T, H);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   dim3 grid(B * H, (T + AT_BLK - 1) / AT_BLK);
   ++g_kernel_launches;
-  attn_bwd_tc<<<grid, BW_THREADS, smem, s>>>(tqkv, tdo, tdq, lse, Dbuf, dstart, dqkv, T, H, err);
+  attn_bwd_tc<F16><<<grid, BW_THREADS, smem, s>>>(tqkv, tdo, tdq, lse, Dbuf, dstart, T, H, L.kcol, L.vcol, L.G,
+                                                  L.dkv, L.ld_kv, L.v_off, err);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   ++g_kernel_launches;
-  attn_dq_finish_kernel<<<148 * 8, 256, 0, s>>>(dq_acc, dqkv, rows, C);
+  attn_dq_finish_kernel<F16><<<148 * 8, 256, 0, s>>>(dq_acc, dqkv, rows, C, (long)L.qw);
   return cudaGetLastError();
+}
+
+cudaError_t launch_attn_bwd_tc(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* Dbuf,
+                               bool d_ready, float* dq_acc, const int* dstart, bf16* dqkv, int B, int T, int H,
+                               unsigned* err, cudaStream_t s, bool f16, const AttnLayout* lay) {
+  const AttnLayout L = lay ? *lay : attn_layout_mha(dqkv, H * AT_D);
+  if (!layout_ok(L, H) || !L.dkv) return cudaErrorInvalidValue;
+  return f16 ? attn_bwd_tc_t<true>(qkv, out, dout, lse, Dbuf, d_ready, dq_acc, dstart, dqkv, B, T, H, err, s, L)
+             : attn_bwd_tc_t<false>(qkv, out, dout, lse, Dbuf, d_ready, dq_acc, dstart, dqkv, B, T, H, err, s, L);
 }

@@ -4,10 +4,12 @@
 #pragma once
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 #include <math.h>
 
 typedef __nv_bfloat16 bf16;
+typedef __half f16;
 
 #define GPT_DEVERR_TOKEN 1u
 #define GPT_DEVERR_TARGET 2u
@@ -17,9 +19,11 @@ typedef __nv_bfloat16 bf16;
 
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(bf16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_f(f16 x) { return __half2float(x); }
 template <typename T> __device__ __forceinline__ T from_f(float x);
 template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
 template <> __device__ __forceinline__ bf16 from_f<bf16>(float x) { return __float2bfloat16_rn(x); }
+template <> __device__ __forceinline__ f16 from_f<f16>(float x) { return __float2half_rn(x); }
 
 // 16 bytes of T moved as one vector and widened to fp32.
 template <typename T> struct Vec;
@@ -49,6 +53,26 @@ template <> struct Vec<bf16> {
     __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
 #pragma unroll
     for (int k = 0; k < 4; ++k) h[k] = __floats2bfloat162_rn(i[2 * k], i[2 * k + 1]);
+    *reinterpret_cast<uint4*>(p) = v;
+  }
+};
+
+template <> struct Vec<f16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void load(const f16* p, float* o) {
+    uint4 v = *reinterpret_cast<const uint4*>(p);
+    const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __half22float2(h[i]);
+      o[2 * i] = f.x; o[2 * i + 1] = f.y;
+    }
+  }
+  __device__ __forceinline__ static void store(f16* p, const float* i) {
+    uint4 v;
+    __half2* h = reinterpret_cast<__half2*>(&v);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) h[k] = __floats2half2_rn(i[2 * k], i[2 * k + 1]);
     *reinterpret_cast<uint4*>(p) = v;
   }
 };
@@ -132,6 +156,7 @@ struct EpiParams {
   // over 64-wide heads, row = b * rd_T + t (out rounded to T first)
   float* rowdot;
   int rd_T;
+  int f16;   // tensor-core GEMM: the 16-bit operands and outputs are fp16 (0: bf16)
 };
 
 // Apply the epilogue to one element (used by the SIMT GEMM).

@@ -21,8 +21,8 @@ __global__ void dec_embed_kernel(const int* __restrict__ tok, const float* __res
     pos = pos < 0 ? 0 : max_seq - 1;
   }
   const float* a = wte + (long)tok[b] * C;
-  const float* p = wpe + (long)pos * C;
-  for (int c = threadIdx.x; c < C; c += blockDim.x) x[(long)b * C + c] = from_f<T>(a[c] + p[c]);
+  const float* p = wpe ? wpe + (long)pos * C : nullptr;
+  for (int c = threadIdx.x; c < C; c += blockDim.x) x[(long)b * C + c] = from_f<T>(a[c] + (p ? p[c] : 0.f));
 }
 
 template <typename T>
@@ -195,24 +195,25 @@ cudaError_t launch_gemv(const T* X, int B, int K, const T* W, int N, const float
 // Copy the prompt's K and V (from the prefill's qkv [B*Tp, 3C]) into the cache.
 template <typename T>
 __global__ void kv_fill_kernel(const T* __restrict__ qkv, T* __restrict__ kc, T* __restrict__ vc, int B, int Tp,
-                               int H, int d, int Tmax) {
-  int C = H * d;
-  long n = (long)B * Tp * C;
+                               int d, int Tmax, DecLayout L) {
+  const int KC = L.Hkv * d;
+  long n = (long)B * Tp * KC;
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
-    int c = i % C;
-    long bt = i / C;
+    int c = i % KC;
+    long bt = i / KC;
     int t = bt % Tp, b = bt / Tp;
     int h = c / d, e = c % d;
-    long dst = (((long)b * H + h) * Tmax + t) * d + e;
-    kc[dst] = qkv[bt * 3 * C + C + c];
-    vc[dst] = qkv[bt * 3 * C + 2 * C + c];
+    long dst = (((long)b * L.Hkv + h) * Tmax + t) * d + e;
+    kc[dst] = qkv[bt * L.qw + L.kcol + c];
+    vc[dst] = qkv[bt * L.qw + L.vcol + c];
   }
 }
 
 template <typename T>
-cudaError_t launch_kv_fill(const T* qkv, T* kc, T* vc, int B, int Tp, int H, int d, int Tmax, cudaStream_t s) {
+cudaError_t launch_kv_fill(const T* qkv, T* kc, T* vc, int B, int Tp, int d, int Tmax, const DecLayout& L,
+                           cudaStream_t s) {
   ++g_kernel_launches;
-  kv_fill_kernel<T><<<148 * 4, 256, 0, s>>>(qkv, kc, vc, B, Tp, H, d, Tmax);
+  kv_fill_kernel<T><<<148 * 4, 256, 0, s>>>(qkv, kc, vc, B, Tp, d, Tmax, L);
   return cudaGetLastError();
 }
 
@@ -233,7 +234,7 @@ __device__ __forceinline__ void load8(const T* p, float* v) {
 template <typename T, int D>
 __global__ void __launch_bounds__(DA_THREADS)
 dec_attn_split_kernel(const T* __restrict__ qkv, T* kc, T* vc, float* __restrict__ part, int B, int H, int Tmax,
-                      int pos0, const int* __restrict__ step) {
+                      int pos0, const int* __restrict__ step, DecLayout Ly) {
   griddep_wait();
   griddep_release();
   static_assert(D % 8 == 0 && D <= 256, "head size");
@@ -245,15 +246,15 @@ dec_attn_split_kernel(const T* __restrict__ qkv, T* kc, T* vc, float* __restrict
   if (pos >= Tmax) pos = Tmax - 1;
   const int bh = blockIdx.x, sp = blockIdx.y;
   const int b = bh / H, h = bh % H;
-  const int C = H * D;
+  const int G = H / Ly.Hkv, hk = h / G;   // query head h reads key/value head hk
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = lane / LPK, sub = lane % LPK;
-  const T* q = qkv + (long)b * 3 * C + h * D;
-  const T* knew = q + C;
-  const T* vnew = q + 2 * C;
-  T* kcb = kc + (long)bh * Tmax * D;
-  T* vcb = vc + (long)bh * Tmax * D;
-  if (sp == 0 && threadIdx.x < D) {
+  const T* q = qkv + (long)b * Ly.qw + h * D;
+  const T* knew = qkv + (long)b * Ly.qw + Ly.kcol + hk * D;
+  const T* vnew = qkv + (long)b * Ly.qw + Ly.vcol + hk * D;
+  T* kcb = kc + ((long)b * Ly.Hkv + hk) * Tmax * D;
+  T* vcb = vc + ((long)b * Ly.Hkv + hk) * Tmax * D;
+  if (sp == 0 && h % G == 0 && threadIdx.x < D) {
     kcb[(long)pos * D + threadIdx.x] = knew[threadIdx.x];
     vcb[(long)pos * D + threadIdx.x] = vnew[threadIdx.x];
   }
@@ -355,14 +356,14 @@ size_t dec_attn_part_floats(int B, int H, int d) { return (size_t)B * H * DA_SPL
 
 template <typename T>
 cudaError_t launch_dec_attn(const T* qkv, T* kc, T* vc, T* out, float* part, int B, int H, int d, int Tmax, int pos0,
-                            const int* step, cudaStream_t s) {
+                            const int* step, const DecLayout& L, cudaStream_t s) {
   dim3 g(B * H, DA_SPLITS);
   cudaError_t e = cudaSuccess;
   switch (d) {
 #define DA_CASE(DD)                                                                                               \
   case DD:                                                                                                        \
     g_kernel_launches += 2;                                                                                       \
-    e = launch_k(dec_attn_split_kernel<T, DD>, g, dim3(DA_THREADS), 0, s, qkv, kc, vc, part, B, H, Tmax, pos0, step); \
+    e = launch_k(dec_attn_split_kernel<T, DD>, g, dim3(DA_THREADS), 0, s, qkv, kc, vc, part, B, H, Tmax, pos0, step, L); \
     if (e == cudaSuccess) e = launch_k(dec_attn_combine_kernel<T, DD>, dim3(B * H), dim3(64), 0, s, (const float*)part, out, H); \
     break;
     DA_CASE(16)
@@ -425,6 +426,258 @@ cudaError_t launch_argmax(const float* logits, int B, int V, int Vp, int* tok, i
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ sampling
+// Sampled choice of the next token ("RustGPT" roadmap: temperature scaling,
+// top-k, top-p; "LucilleAI": sampler), one CTA per row, the row's values in
+// shared memory.  In order: x = z / temperature over the real vocabulary;
+// top-k keeps the k largest x (ties at the cut to the lower index); weights
+// w = exp(x - max x) over the kept tokens; top-p keeps the shortest prefix,
+// in (w descending, index ascending) order, whose weight reaches top_p times
+// the kept total; the token is the first kept one, in ascending token order,
+// at which the running weight exceeds u times the kept total.  Thresholds
+// are found by bisection over order-preserving 32-bit keys, every sum by a
+// fixed-order block reduction (deterministic).  temperature <= 0: greedy.
+#define SMP_THREADS 1024
+#define SMP_WARPS (SMP_THREADS / 32)
+
+__device__ __forceinline__ uint32_t smp_key(float x) {
+  const uint32_t b = __float_as_uint(x);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+// Fixed-order block sums (the same thread-to-element map every call).
+__device__ __forceinline__ float smp_bsum(float v, float* red) {
+  v = warp_sum(v);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float t = lane < SMP_WARPS ? red[lane] : 0.f;
+  return warp_sum(t);
+}
+__device__ __forceinline__ int smp_bcount(int v, int* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  int t = lane < SMP_WARPS ? red[lane] : 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  return t;
+}
+// Exclusive block scan of one value per thread (in thread order).
+__device__ __forceinline__ float smp_bscan_excl(float v, float* red, float* total) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float t = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  __syncthreads();
+  if (lane == 31) red[warp] = inc;
+  __syncthreads();
+  float wsum = lane < SMP_WARPS ? red[lane] : 0.f, winc = wsum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float t = __shfl_up_sync(0xffffffffu, winc, o);
+    if (lane >= o) winc += t;
+  }
+  const float wex = __shfl_sync(0xffffffffu, winc - wsum, warp);
+  *total = __shfl_sync(0xffffffffu, winc, SMP_WARPS - 1);
+  return wex + inc - v;
+}
+__device__ __forceinline__ int smp_bscan_excl_i(int v, int* red) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  __syncthreads();
+  if (lane == 31) red[warp] = inc;
+  __syncthreads();
+  int wsum = lane < SMP_WARPS ? red[lane] : 0, winc = wsum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, winc, o);
+    if (lane >= o) winc += t;
+  }
+  const int wex = __shfl_sync(0xffffffffu, winc - wsum, warp);
+  return wex + inc - v;
+}
+
+__global__ void __launch_bounds__(SMP_THREADS) sample_kernel(const float* __restrict__ logits, int V, int Vp,
+                                                             float temp, int top_k, float top_p,
+                                                             const float* __restrict__ uni, int u_ld, int* tok,
+                                                             int32_t* out, int out_ld, const int* __restrict__ step) {
+  griddep_wait();
+  griddep_release();
+  extern __shared__ float w[];   // [V]
+  __shared__ float redf[SMP_WARPS];
+  __shared__ int redi[SMP_WARPS];
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int col = step ? *step : 0;
+  const float* z = logits + (long)b * Vp;
+  // thread tid owns the contiguous indices [c0, c1)
+  const int chunk = (V + SMP_THREADS - 1) / SMP_THREADS;
+  const int c0 = min(V, tid * chunk), c1 = min(V, c0 + chunk);
+  int choice = 0;
+  if (!(temp > 0.f)) {
+    // greedy: largest logit, lowest index on ties
+    float best = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int i = c0; i < c1; ++i) {
+      const float v = z[i];
+      if (v > best) { best = v; bi = i; }
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > best || (ov == best && oi < bi)) { best = ov; bi = oi; }
+    }
+    __shared__ float sv[SMP_WARPS];
+    __shared__ int si[SMP_WARPS];
+    if ((tid & 31) == 0) { sv[tid >> 5] = best; si[tid >> 5] = bi; }
+    __syncthreads();
+    if (tid < 32) {
+      best = sv[tid];
+      bi = si[tid];
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > best || (ov == best && oi < bi)) { best = ov; bi = oi; }
+      }
+      if (tid == 0) choice = (bi >= 0 && bi < V) ? bi : 0;
+    }
+  } else {
+    const float it = 1.0f / temp;
+    float mx = -INFINITY;
+    for (int i = c0; i < c1; ++i) {
+      const float x = z[i] * it;
+      w[i] = x;
+      mx = fmaxf(mx, x);
+    }
+    {
+      mx = warp_max(mx);
+      __syncthreads();
+      if ((tid & 31) == 0) redf[tid >> 5] = mx;
+      __syncthreads();
+      mx = warp_max((tid & 31) < SMP_WARPS ? redf[tid & 31] : -INFINITY);
+    }
+    // top-k: the largest key tk with count(key >= tk) >= k
+    const bool use_k = top_k > 0 && top_k < V;
+    uint32_t tk = 0;
+    int need_k = 0;
+    if (use_k) {
+      for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = tk | (1u << bit);
+        int cnt = 0;
+        for (int i = c0; i < c1; ++i) cnt += smp_key(w[i]) >= cand;
+        if (smp_bcount(cnt, redi) >= top_k) tk = cand;
+      }
+      int gt = 0;
+      for (int i = c0; i < c1; ++i) gt += smp_key(w[i]) > tk;
+      need_k = top_k - smp_bcount(gt, redi);
+    }
+    // weights of the kept tokens (ties at the top-k cut: lower indices first)
+    {
+      int eq = 0;
+      if (use_k)
+        for (int i = c0; i < c1; ++i) eq += smp_key(w[i]) == tk;
+      int rank = use_k ? smp_bscan_excl_i(eq, redi) : 0;
+      for (int i = c0; i < c1; ++i) {
+        bool keep = true;
+        if (use_k) {
+          const uint32_t k = smp_key(w[i]);
+          keep = k > tk || (k == tk && rank++ < need_k);
+        }
+        w[i] = keep ? __expf(w[i] - mx) : 0.f;
+      }
+    }
+    float part = 0.f;
+    for (int i = c0; i < c1; ++i) part += w[i];
+    const float Z = smp_bsum(part, redf);
+    if (top_p < 1.f) {
+      // the largest weight threshold tp with mass(w >= tp) >= top_p Z
+      const float target = top_p * Z;
+      uint32_t tp = 0;
+      for (int bit = 30; bit >= 0; --bit) {
+        const uint32_t cand = tp | (1u << bit);
+        float m = 0.f;
+        for (int i = c0; i < c1; ++i) m += __float_as_uint(w[i]) >= cand ? w[i] : 0.f;
+        if (smp_bsum(m, redf) >= target) tp = cand;
+      }
+      const float pstar = __uint_as_float(tp);
+      float gt = 0.f;
+      int eq = 0;
+      for (int i = c0; i < c1; ++i) {
+        gt += w[i] > pstar ? w[i] : 0.f;
+        eq += w[i] == pstar;
+      }
+      const float mgt = smp_bsum(gt, redf);
+      const int neq = smp_bcount(eq, redi);
+      int need = pstar > 0.f ? (int)ceilf((target - mgt) / pstar) : neq;
+      need = max(1, min(need, neq));
+      int rank = smp_bscan_excl_i(eq, redi);
+      for (int i = c0; i < c1; ++i) {
+        const bool keep = w[i] > pstar || (w[i] == pstar && rank++ < need);
+        if (!keep) w[i] = 0.f;
+      }
+    }
+    // inverse CDF in ascending token order
+    part = 0.f;
+    int last = -1;
+    for (int i = c0; i < c1; ++i) {
+      part += w[i];
+      if (w[i] > 0.f) last = i;
+    }
+    float Z2;
+    const float before = smp_bscan_excl(part, redf, &Z2);
+    const float u = uni[(long)b * u_ld + col];
+    const float target = u * Z2;
+    __shared__ int s_choice, s_last;
+    if (tid == 0) { s_choice = -1; s_last = -1; }
+    __syncthreads();
+    if (last >= 0) atomicMax(&s_last, last);
+    if (before <= target && target < before + part) {
+      float run = before;
+      for (int i = c0; i < c1; ++i) {
+        run += w[i];
+        if (w[i] > 0.f && run > target) { s_choice = i; break; }
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int c = s_choice >= 0 ? s_choice : s_last;
+      choice = (c >= 0 && c < V) ? c : 0;
+    }
+  }
+  if (tid == 0) {
+    tok[b] = choice;
+    out[(long)b * out_ld + col] = choice;
+  }
+}
+
+cudaError_t launch_sample(const float* logits, int B, int V, int Vp, float temp, int top_k, float top_p,
+                          const float* uni, int u_ld, int* tok, int32_t* out, int out_ld, const int* step,
+                          cudaStream_t s) {
+  const size_t smem = (size_t)V * 4;
+  static size_t attr = 0;
+  if (smem > attr) {
+    cudaError_t e = cudaFuncSetAttribute(sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr = smem;
+  }
+  ++g_kernel_launches;
+  cudaError_t e = launch_k(sample_kernel, dim3(B), dim3(SMP_THREADS), smem, s, logits, V, Vp, temp, top_k, top_p,
+                           uni, u_ld, tok, out, out_ld, step);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 __global__ void step_advance_kernel(int* step) { griddep_wait(); griddep_release(); *step += 1; }
 cudaError_t launch_step_advance(int* step, cudaStream_t s) {
   ++g_kernel_launches;
@@ -451,9 +704,10 @@ cudaError_t launch_gather_last(const T* x, int B, int Tp, int C, T* out, cudaStr
                                            const int*, int, unsigned*, cudaStream_t);                    \
   template cudaError_t launch_gemv<T>(const T*, int, int, const T*, int, const float*, const T*, int, T*, T*, \
                                       float*, cudaStream_t);                                             \
-  template cudaError_t launch_kv_fill<T>(const T*, T*, T*, int, int, int, int, int, cudaStream_t);         \
+  template cudaError_t launch_kv_fill<T>(const T*, T*, T*, int, int, int, int, const DecLayout&, cudaStream_t); \
   template cudaError_t launch_dec_attn<T>(const T*, T*, T*, T*, float*, int, int, int, int, int, const int*,      \
-                                          cudaStream_t);                                                 \
+                                          const DecLayout&, cudaStream_t);                               \
   template cudaError_t launch_gather_last<T>(const T*, int, int, int, T*, cudaStream_t);
 INSTD(float)
 INSTD(bf16)
+INSTD(f16)

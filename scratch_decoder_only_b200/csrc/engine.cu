@@ -19,6 +19,7 @@
 #include <vector>
 #include <thread>
 #include <algorithm>
+#include <type_traits>
 #include "gpt.h"
 #include "launch.h"
 
@@ -30,7 +31,13 @@ struct gpt_model {
   gpt_config cfg;
   int device = 0;
   cudaStream_t stream = 0;
-  bool bf16 = false;
+  bool lp = false;     // 16-bit operands and activations (bf16 or fp16)
+  bool fp16 = false;   // ... and those are fp16
+  // Llama-style block: RMSNorm, rotary positions, Hkv key/value heads, SwiGLU
+  bool llama = false;
+  int Hkv = 0, QW = 0, UW = 0;     // key/value heads; q|k|v row width; MLP up-projection width (F or 2F)
+  float2* rope_tab = nullptr;      // [max_seq][d/2] (cos, sin)
+  void* dkvq = nullptr;            // [Mmax, 2C] per-query-head key/value gradients (grouped heads)
   int V, Vp, C, H, d, F, NL, Tmax, Bmax, ldl;
   long Mmax;
   size_t N = 0;
@@ -52,6 +59,7 @@ struct gpt_model {
   DevScalars* sc;
   void *kc, *vc, *dx, *dh, *dq, *datt, *du, *da, *dxf;
   float *dlogits, *dmu, *drs, *dpart;
+  float* dam;      // fused decode: per-CTA argmax partials [Bmax][DF_MAX_GRID] values, then indices
   int* dtok;
   int fwd_B = 0, fwd_T = 0;
   bool have_targets = false, logits_valid = false;
@@ -64,12 +72,24 @@ struct gpt_model {
   cudaGraphExec_t dec_graph = nullptr;
   int dec_B = 0, dec_Tp = 0, dec_nnew = 0, dec_kernels = 0;
   int32_t* dec_out = nullptr;
+  // sampling decode (gpt_sample_decode); smp_on = false: greedy
+  bool smp_on = false;
+  float smp_temp = 0.f, smp_topp = 1.f;
+  int smp_topk = 0;
+  const float* smp_u = nullptr;
+  bool dec_smp_on = false;   // the sampling state the captured graph was built with
+  float dec_smp_temp = 0.f, dec_smp_topp = 1.f;
+  int dec_smp_topk = 0;
+  const float* dec_smp_u = nullptr;
   bool prof = false;
-  struct ProfRec { int cls; cudaEvent_t a, b; double flops, bytes; };
+  // pair_mult: FLOPs per allowed (query, key) pair of the latest packed
+  // forward, whose count the device holds (added at gpt_profile_read)
+  struct ProfRec { int cls; cudaEvent_t a, b; double flops, bytes, pair_mult; };
   std::vector<ProfRec> recs;
   std::vector<cudaEvent_t> evpool;
   size_t evused = 0;
   std::vector<RedSeg> redsegs;   // deferred column reductions of the current backward pass
+  bool accum_now = false;        // the backward in progress adds to the stored gradients
 };
 
 enum ProfCls { PC_GEMM_FWD, PC_GEMM_DX, PC_GEMM_DW, PC_ATTN_FWD, PC_ATTN_BWD, PC_XENT, PC_LN_FWD, PC_LN_BWD,
@@ -90,12 +110,12 @@ static cudaEvent_t prof_event(gpt_model* m) {
 struct ProfScope {
   gpt_model* m;
   long idx = -1;
-  ProfScope(gpt_model* mm, int cls, double flops, double bytes) : m(mm) {
+  ProfScope(gpt_model* mm, int cls, double flops, double bytes, double pair_mult = 0.0) : m(mm) {
     if (!m->prof) return;
     cudaEvent_t a = prof_event(m);
     if (!a) return;
     cudaEventRecord(a, m->stream);
-    m->recs.push_back({cls, a, nullptr, flops, bytes});
+    m->recs.push_back({cls, a, nullptr, flops, bytes, pair_mult});
     idx = (long)m->recs.size() - 1;
   }
   ~ProfScope() {
@@ -132,6 +152,32 @@ struct ProfScope {
 static void layout_params(gpt_model* m) {
   size_t o = 0;
   size_t C = m->C, F = m->F, Vp = m->Vp;
+  if (m->llama) {
+    // wte; per layer attn_norm_g, w_qkv [QW, C], w_o, mlp_norm_g, w_gu [2F, C],
+    // w_down [C, F]; norm_g; head if untied (no position table, no biases:
+    // the unused offsets are left at 0 and never read)
+    m->o_wte = o; o += Vp * C;
+    m->o_wpe = 0;
+    m->L.assign(m->NL, LayerOff{});
+    for (int l = 0; l < m->NL; ++l) {
+      LayerOff& lo = m->L[l];
+      lo.ln1_g = o; o += C;
+      lo.w_qkv = o; o += (size_t)m->QW * C;
+      lo.w_o = o; o += C * C;
+      lo.ln2_g = o; o += C;
+      lo.w_fc = o; o += 2 * F * C;
+      lo.w_fc2 = o; o += C * F;
+    }
+    m->o_lnf_g = o; o += C;
+    m->o_lnf_b = 0;
+    if (m->cfg.tied) {
+      m->o_head = m->o_wte;
+    } else {
+      m->o_head = o; o += Vp * C;
+    }
+    m->N = o;
+    return;
+  }
   m->o_wte = o; o += Vp * C;
   m->o_wpe = o; o += (size_t)m->Tmax * C;
   m->L.resize(m->NL);
@@ -198,6 +244,23 @@ static void init_host_params(gpt_model* m, uint64_t seed, std::vector<float>& h)
     for (size_t r = (size_t)m->V; r < (size_t)m->Vp; ++r)
       for (size_t c = 0; c < C; ++c) h[off + r * C + c] = 0.f;
   };
+  if (m->llama) {
+    fill_normal(h, m->o_wte, (size_t)m->Vp * C, seed, sd);
+    zero_pad_rows(m->o_wte);
+    for (auto& lo : m->L) {
+      for (size_t i = 0; i < C; ++i) { h[lo.ln1_g + i] = 1.f; h[lo.ln2_g + i] = 1.f; }
+      fill_normal(h, lo.w_qkv, (size_t)m->QW * C, seed, sd);
+      fill_normal(h, lo.w_o, C * C, seed, sd);
+      fill_normal(h, lo.w_fc, 2 * F * C, seed, sd);
+      fill_normal(h, lo.w_fc2, C * F, seed, sd);
+    }
+    for (size_t i = 0; i < C; ++i) h[m->o_lnf_g + i] = 1.f;
+    if (!m->cfg.tied) {
+      fill_normal(h, m->o_head, (size_t)m->Vp * C, seed, sd);
+      zero_pad_rows(m->o_head);
+    }
+    return;
+  }
   fill_normal(h, m->o_wte, (size_t)m->Vp * C, seed, sd);
   zero_pad_rows(m->o_wte);
   fill_normal(h, m->o_wpe, (size_t)m->Tmax * C, seed, sd);
@@ -229,21 +292,21 @@ struct Carver {
 };
 
 static int build_arena(gpt_model* m) {
-  size_t es = m->bf16 ? 2 : 4;
+  size_t es = m->lp ? 2 : 4;
   size_t N = m->N, C = m->C, F = m->F, Mx = m->Mmax, NL = m->NL;
   Carver cv;
   cv.add((void**)&m->p32, N * 4);
   cv.add((void**)&m->g32, N * 4);
   cv.add((void**)&m->m32, N * 4);
   cv.add((void**)&m->v32, N * 4);
-  if (m->bf16) cv.add(&m->pw, N * es);
+  if (m->lp) cv.add(&m->pw, N * es);
   cv.add(&m->xs, (NL + 1) * Mx * C * es);
   cv.add(&m->xmid, NL * Mx * C * es);
   cv.add(&m->h1, NL * Mx * C * es);
   cv.add(&m->h2, NL * Mx * C * es);
   cv.add(&m->qkv, NL * Mx * 3 * C * es);
   cv.add(&m->att, NL * Mx * C * es);
-  cv.add(&m->u, NL * Mx * F * es);
+  cv.add(&m->u, NL * Mx * (size_t)m->UW * es);
   cv.add(&m->a, NL * Mx * F * es);
   cv.add(&m->xf, Mx * C * es);
   cv.add(&m->logits, Mx * (size_t)m->ldl * es);
@@ -261,10 +324,14 @@ static int build_arena(gpt_model* m) {
   cv.add((void**)&m->dres32, Mx * C * 4);
   cv.add(&m->dres_t, Mx * C * es);
   cv.add(&m->dC, Mx * C * es);
-  cv.add(&m->dF, Mx * F * es);
+  cv.add(&m->dF, Mx * (size_t)(m->UW + (m->llama ? F : 0)) * es);   // llama: dgu [M, 2F] then da [M, F]
+  if (m->llama) {
+    cv.add((void**)&m->rope_tab, (size_t)m->Tmax * (m->d / 2) * sizeof(float2));
+    if (m->Hkv < m->H) cv.add(&m->dkvq, Mx * 2 * C * es);
+  }
   cv.add(&m->dqkv, Mx * 3 * C * es);
   cv.add((void**)&m->attD, Mx * m->H * 4);
-  cv.add((void**)&m->dq_acc, m->bf16 ? Mx * C * 4 : 4);
+  cv.add((void**)&m->dq_acc, m->lp ? Mx * C * 4 : 4);
   cv.add((void**)&m->rowloss, Mx * 4);
   {
     // partial rows of every deferred column reduction of one backward pass:
@@ -284,7 +351,7 @@ static int build_arena(gpt_model* m) {
   cv.add(&m->dh, Bx * C * es);
   cv.add(&m->dq, Bx * 3 * C * es);
   cv.add(&m->datt, Bx * C * es);
-  cv.add(&m->du, Bx * F * es);
+  cv.add(&m->du, Bx * (size_t)m->UW * es);
   cv.add(&m->da, Bx * F * es);
   cv.add(&m->dxf, Bx * C * es);
   cv.add((void**)&m->dlogits, Bx * m->Vp * 4);
@@ -292,6 +359,7 @@ static int build_arena(gpt_model* m) {
   cv.add((void**)&m->drs, Bx * 4);
   cv.add((void**)&m->dtok, Bx * 4);
   cv.add((void**)&m->dpart, dec_attn_part_floats((int)Bx, m->H, m->d) * 4);
+  cv.add((void**)&m->dam, Bx * DF_MAX_GRID * 8 + Bx * m->H * 4);   // argmax partials, then split counters
   m->arena_bytes = cv.off + 256;
   cudaError_t e = cudaMalloc((void**)&m->arena, m->arena_bytes);
   if (e != cudaSuccess) {
@@ -302,7 +370,7 @@ static int build_arena(gpt_model* m) {
     return GPT_ERR_NOMEM;
   }
   for (auto& it : cv.items) *it.first = m->arena + it.second;
-  if (!m->bf16) m->pw = m->p32;
+  if (!m->lp) m->pw = m->p32;
   return GPT_OK;
 }
 
@@ -348,16 +416,34 @@ static int gemm_cls(bool a_t, bool b_t) { return a_t ? PC_GEMM_DW : (b_t ? PC_GE
 static int gemm(gpt_model* m, int M, int N, int K, const float* A, long lda, bool a_t, const float* B,
                 long ldb, bool b_t, EpiParams<float> epi) {
   ProfScope ps(m, gemm_cls(a_t, b_t), 2.0 * M * N * K, 0.0);
+  if (epi.kind == EPI_F32 && m->accum_now) epi.kind = EPI_F32_ADD;   // gradient accumulation
   CK(launch_gemm_simt<float>(M, N, K, A, lda, a_t, B, ldb, b_t, epi, 1, m->stream));
   return GPT_OK;
 }
 
-static int gemm(gpt_model* m, int M, int N, int K, const bf16* A, long lda, bool a_t, const bf16* B,
-                long ldb, bool b_t, EpiParams<bf16> epi) {
+// The tensor-core GEMM for either 16-bit type (fp16 is flagged in the
+// epilogue record; the operand and output layouts are the same).
+template <typename T16>
+static cudaError_t tc_gemm(int M, int N, int K, const T16* A, long lda, bool a_t, const T16* B, long ldb, bool b_t,
+                           const EpiParams<T16>& epi, int splits, unsigned* err, cudaStream_t s) {
+  static_assert(sizeof(EpiParams<T16>) == sizeof(EpiParams<bf16>), "one layout for both 16-bit types");
+  EpiParams<bf16> e;
+  memcpy(&e, &epi, sizeof(e));
+  e.f16 = std::is_same<T16, f16>::value ? 1 : 0;
+  return launch_gemm_tc(M, N, K, reinterpret_cast<const bf16*>(A), lda, a_t, reinterpret_cast<const bf16*>(B), ldb,
+                        b_t, e, splits, err, s);
+}
+
+template <typename T16>
+static int gemm16(gpt_model* m, int M, int N, int K, const T16* A, long lda, bool a_t, const T16* B,
+                  long ldb, bool b_t, EpiParams<T16> epi) {
   ProfScope ps(m, gemm_cls(a_t, b_t), 2.0 * M * N * K, 0.0);
+  // gradient accumulation: weight gradients are added onto the stored ones
+  const bool add_f32 = epi.kind == EPI_F32 && m->accum_now;
   if (!gemm_tc_supported(M, N, K, lda, a_t, ldb, b_t)) {
     if (epi.rowdot) FAIL(GPT_ERR_ARG, "row-dot epilogue needs the tensor-core GEMM");
-    CK(launch_gemm_simt<bf16>(M, N, K, A, lda, a_t, B, ldb, b_t, epi, 1, m->stream));
+    if (add_f32) epi.kind = EPI_F32_ADD;
+    CK(launch_gemm_simt<T16>(M, N, K, A, lda, a_t, B, ldb, b_t, epi, 1, m->stream));
     return GPT_OK;
   }
   int splits = 1;
@@ -374,52 +460,77 @@ static int gemm(gpt_model* m, int M, int N, int K, const bf16* A, long lda, bool
     }
     int kb_total = (K + 63) / 64, kbs = (kb_total + splits - 1) / splits;
     splits = (kb_total + kbs - 1) / kbs;   // no empty split
-    if (splits > 1 && epi.ld_outf != N) splits = 1;   // the zeroing below wants a dense output
+    if (splits > 1 && epi.ld_outf != N && !m->accum_now) splits = 1;   // the zeroing below wants a dense output
   }
-  if (splits > 1) {
+  if (splits > 1 || add_f32) {
     // K slices add their products onto the zeroed weight gradient (TMA bulk
-    // reduce-add): no partial slabs, no separate summation pass
-    EpiParams<bf16> e2 = epi;
+    // reduce-add): no partial slabs, no separate summation pass; when
+    // accumulating, onto the stored gradient instead
+    EpiParams<T16> e2 = epi;
     e2.kind = EPI_F32_ADD;
-    CK(cudaMemsetAsync(epi.outf, 0, (size_t)M * N * 4, m->stream));
-    CK(launch_gemm_tc(M, N, K, A, lda, a_t, B, ldb, b_t, e2, splits, &m->sc->err, m->stream));
+    if (!add_f32) CK(cudaMemsetAsync(epi.outf, 0, (size_t)M * N * 4, m->stream));
+    CK(tc_gemm<T16>(M, N, K, A, lda, a_t, B, ldb, b_t, e2, splits, &m->sc->err, m->stream));
   } else {
-    CK(launch_gemm_tc(M, N, K, A, lda, a_t, B, ldb, b_t, epi, 1, &m->sc->err, m->stream));
+    CK(tc_gemm<T16>(M, N, K, A, lda, a_t, B, ldb, b_t, epi, 1, &m->sc->err, m->stream));
   }
   return GPT_OK;
 }
 
+static int gemm(gpt_model* m, int M, int N, int K, const bf16* A, long lda, bool a_t, const bf16* B, long ldb,
+                bool b_t, EpiParams<bf16> epi) {
+  return gemm16<bf16>(m, M, N, K, A, lda, a_t, B, ldb, b_t, epi);
+}
+static int gemm(gpt_model* m, int M, int N, int K, const f16* A, long lda, bool a_t, const f16* B, long ldb,
+                bool b_t, EpiParams<f16> epi) {
+  return gemm16<f16>(m, M, N, K, A, lda, a_t, B, ldb, b_t, epi);
+}
+
+// Allowed (query, key) pairs of a causal pass, all heads; a packed pass has
+// fewer, counted on the device by the input preparation (see ProfRec)
 static double attn_pairs(int B, int T, int H, bool seg) { return seg ? 0.0 : (double)B * H * T * (T + 1) / 2.0; }
+static double attn_pair_mult(const gpt_model* m, double per_pair) { return m->seg_used ? per_pair * m->H : 0.0; }
 
 static int attn_fwd(gpt_model* m, const float* qkv, float* out, float* lse, int B, int T) {
-  ProfScope ps(m, PC_ATTN_FWD, 4.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0);
+  ProfScope ps(m, PC_ATTN_FWD, 4.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0, attn_pair_mult(m, 4.0 * m->d));
   CK(launch_attn_fwd_simt<float>(qkv, out, lse, m->dstart, B, T, m->H, m->d, m->stream));
   return GPT_OK;
 }
-static int attn_fwd(gpt_model* m, const bf16* qkv, bf16* out, float* lse, int B, int T) {
-  ProfScope ps(m, PC_ATTN_FWD, 4.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0);
-  if (attn_tc_supported(m->d)) CK(launch_attn_fwd_tc(qkv, out, lse, m->dstart, B, T, m->H, &m->sc->err, m->stream));
-  else if (attn_mma_supported(m->d)) CK(launch_attn_fwd_mma(qkv, out, lse, m->dstart, B, T, m->H, m->d, m->stream));
-  else CK(launch_attn_fwd_simt<bf16>(qkv, out, lse, m->dstart, B, T, m->H, m->d, m->stream));
+template <typename T16>
+static int attn_fwd(gpt_model* m, const T16* qkv, T16* out, float* lse, int B, int T, const AttnLayout* lay = nullptr) {
+  ProfScope ps(m, PC_ATTN_FWD, 4.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0, attn_pair_mult(m, 4.0 * m->d));
+  constexpr bool F16 = std::is_same<T16, f16>::value;
+  if (lay && !attn_tc_supported(m->d)) FAIL(GPT_ERR_ARG, "grouped key/value heads need the tensor-core attention");
+  if (attn_tc_supported(m->d))
+    CK(launch_attn_fwd_tc(reinterpret_cast<const bf16*>(qkv), reinterpret_cast<bf16*>(out), lse, m->dstart, B, T,
+                          m->H, &m->sc->err, m->stream, F16, lay));
+  else if (!F16 && attn_mma_supported(m->d))
+    CK(launch_attn_fwd_mma(reinterpret_cast<const bf16*>(qkv), reinterpret_cast<bf16*>(out), lse, m->dstart, B, T,
+                           m->H, m->d, m->stream));
+  else CK(launch_attn_fwd_simt<T16>(qkv, out, lse, m->dstart, B, T, m->H, m->d, m->stream));
   return GPT_OK;
 }
 static int attn_bwd(gpt_model* m, const float* qkv, const float* out, const float* dout, const float* lse,
                     float* dqkv, int B, int T, bool) {
-  ProfScope ps(m, PC_ATTN_BWD, 8.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0);
+  ProfScope ps(m, PC_ATTN_BWD, 8.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0, attn_pair_mult(m, 8.0 * m->d));
   CK(launch_attn_bwd_simt<float>(qkv, out, dout, lse, m->attD, m->dstart, dqkv, B, T, m->H, m->d, m->stream));
   return GPT_OK;
 }
 // d_ready: m->attD already holds D = rowsum(dO o O) (tensor-core path only)
-static int attn_bwd(gpt_model* m, const bf16* qkv, const bf16* out, const bf16* dout, const float* lse,
-                    bf16* dqkv, int B, int T, bool d_ready) {
-  ProfScope ps(m, PC_ATTN_BWD, 8.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0);
+template <typename T16>
+static int attn_bwd(gpt_model* m, const T16* qkv, const T16* out, const T16* dout, const float* lse,
+                    T16* dqkv, int B, int T, bool d_ready, const AttnLayout* lay = nullptr) {
+  ProfScope ps(m, PC_ATTN_BWD, 8.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0, attn_pair_mult(m, 8.0 * m->d));
+  constexpr bool F16 = std::is_same<T16, f16>::value;
+  auto cb = [](const T16* p) { return reinterpret_cast<const bf16*>(p); };
+  if (lay && !attn_tc_supported(m->d)) FAIL(GPT_ERR_ARG, "grouped key/value heads need the tensor-core attention");
   if (attn_tc_supported(m->d))
-    CK(launch_attn_bwd_tc(qkv, out, dout, lse, m->attD, d_ready, m->dq_acc, m->dstart, dqkv, B, T, m->H,
-                          &m->sc->err, m->stream));
-  else if (attn_mma_supported(m->d))
-    CK(launch_attn_bwd_mma(qkv, out, dout, lse, m->attD, m->dstart, dqkv, B, T, m->H, m->d, m->stream));
+    CK(launch_attn_bwd_tc(cb(qkv), cb(out), cb(dout), lse, m->attD, d_ready, m->dq_acc, m->dstart,
+                          reinterpret_cast<bf16*>(dqkv), B, T, m->H, &m->sc->err, m->stream, F16, lay));
+  else if (!F16 && attn_mma_supported(m->d))
+    CK(launch_attn_bwd_mma(cb(qkv), cb(out), cb(dout), lse, m->attD, m->dstart, reinterpret_cast<bf16*>(dqkv), B, T,
+                           m->H, m->d, m->stream));
   else
-    CK(launch_attn_bwd_simt<bf16>(qkv, out, dout, lse, m->attD, m->dstart, dqkv, B, T, m->H, m->d, m->stream));
+    CK(launch_attn_bwd_simt<T16>(qkv, out, dout, lse, m->attD, m->dstart, dqkv, B, T, m->H, m->d, m->stream));
   return GPT_OK;
 }
 
@@ -429,9 +540,9 @@ static int attn_bwd(gpt_model* m, const bf16* qkv, const bf16* out, const bf16* 
 template <typename T>
 struct Acts {
   gpt_model* m;
-  size_t MC, M3C, MF, Mx;
+  size_t MC, M3C, MF, MU, Mx;
   explicit Acts(gpt_model* mm) : m(mm) {
-    Mx = m->Mmax; MC = Mx * m->C; M3C = 3 * MC; MF = Mx * m->F;
+    Mx = m->Mmax; MC = Mx * m->C; M3C = 3 * MC; MF = Mx * m->F; MU = Mx * m->UW;
   }
   T* x(int l) const { return (T*)m->xs + l * MC; }
   T* xmid(int l) const { return (T*)m->xmid + l * MC; }
@@ -439,7 +550,7 @@ struct Acts {
   T* h2(int l) const { return (T*)m->h2 + l * MC; }
   T* qkv(int l) const { return (T*)m->qkv + l * M3C; }
   T* att(int l) const { return (T*)m->att + l * MC; }
-  T* u(int l) const { return (T*)m->u + l * MF; }
+  T* u(int l) const { return (T*)m->u + l * MU; }
   T* a(int l) const { return (T*)m->a + l * MF; }
   float* mu1(int l) const { return m->mu1 + l * Mx; }
   float* rs1(int l) const { return m->rs1 + l * Mx; }
@@ -452,8 +563,17 @@ struct Acts {
 };
 
 template <typename T>
+static int forward_llama(gpt_model* m, const int32_t* tokens, const int32_t* targets, const int32_t* seg, int B,
+                         int T_, float* loss_dev);
+template <typename T>
+static int backward_llama(gpt_model* m);
+
+template <typename T>
 static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targets, const int32_t* seg, int B,
                         int T_, float* loss_dev) {
+  if constexpr (sizeof(T) == 2) {
+    if (m->llama) return forward_llama<T>(m, tokens, targets, seg, B, T_, loss_dev);
+  }
   cudaStream_t s = m->stream;
   Acts<T> A(m);
   const int M = B * T_, C = m->C, F = m->F;
@@ -497,6 +617,9 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
 
 template <typename T>
 static int backward_impl(gpt_model* m) {
+  if constexpr (sizeof(T) == 2) {
+    if (m->llama) return backward_llama<T>(m);
+  }
   cudaStream_t s = m->stream;
   Acts<T> A(m);
   const int B = m->fwd_B, T_ = m->fwd_T, M = B * T_, C = m->C, F = m->F, Vp = m->Vp;
@@ -593,13 +716,161 @@ static int backward_impl(gpt_model* m) {
     double pb = 0;
     for (const RedSeg& g : segs) pb += (double)g.rows * g.cols * 4;
     ProfScope ps(m, PC_BIAS, 0, pb);
-    CK(launch_reduce_segs(segs.data(), (int)segs.size(), s));
+    CK(launch_reduce_segs(segs.data(), (int)segs.size(), m->accum_now, s));
   }
   // embeddings: scatter-add by token and by position
   ProfScope ps_emb(m, PC_EMBED, 0, (double)M * C * 12);
-  if (!m->cfg.tied) CK(cudaMemsetAsync(A.G(m->o_wte), 0, (size_t)Vp * C * 4, s));
-  CK(cudaMemsetAsync(A.G(m->o_wpe), 0, (size_t)m->Tmax * C * 4, s));
+  if (!m->accum_now) {
+    if (!m->cfg.tied) CK(cudaMemsetAsync(A.G(m->o_wte), 0, (size_t)Vp * C * 4, s));
+    CK(cudaMemsetAsync(A.G(m->o_wpe), 0, (size_t)m->Tmax * C * 4, s));
+  }
   CK(launch_embed_bwd<T>(m->dres32, m->tok, m->pos, A.G(m->o_wte), A.G(m->o_wpe), M, C, s));
+  m->have_targets = false;
+  return GPT_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Llama-style block ("NTransformer" page, key features: RoPE, GQA, SwiGLU):
+// RMSNorm (the LayerNorm kernels without mean and shift), rotary positions
+// applied in place to the q and k heads after the qkv GEMM (and their inverse
+// to dq, dk), grouped key/value heads read by the tensor-core attention
+// through its column layout, SwiGLU between the up and down GEMMs; no biases.
+// ---------------------------------------------------------------------------
+// q|k|v column layout of the grouped heads; dkv: where the attention backward
+// writes the per-query-head key/value gradients
+static AttnLayout llama_layout(const gpt_model* m, void* dqkv) {
+  AttnLayout a;
+  a.qw = m->QW;
+  a.kcol = m->C;
+  a.vcol = m->C + m->Hkv * m->d;
+  a.G = m->H / m->Hkv;
+  if (a.G == 1) {
+    a.dkv = dqkv ? (bf16*)dqkv + m->C : nullptr;   // dK, dV straight into dqkv (same columns)
+    a.ld_kv = m->QW;
+    a.v_off = m->C;
+  } else {
+    a.dkv = (bf16*)m->dkvq;                       // per query head; summed by launch_gqa_reduce
+    a.ld_kv = 2L * m->C;
+    a.v_off = m->C;
+  }
+  return a;
+}
+
+template <typename T>
+static int forward_llama(gpt_model* m, const int32_t* tokens, const int32_t* targets, const int32_t* seg, int B,
+                         int T_, float* loss_dev) {
+  cudaStream_t s = m->stream;
+  Acts<T> A(m);
+  const int M = B * T_, C = m->C, F = m->F, QW = m->QW;
+  const float eps = m->cfg.ln_eps;
+  const double es = sizeof(T), lnb = (double)M * C * 2 * es + 8.0 * M;
+  m->seg_used = seg != nullptr;
+  const AttnLayout lay = llama_layout(m, nullptr);
+  { ProfScope ps(m, PC_EMBED, 0, (double)M * C * (4 + es) + 16.0 * M);
+    CK(launch_prep(tokens, targets, seg, B, T_, m->V, m->tok, m->tgt, m->pos, m->dstart, m->sc, s));
+    CK(launch_embed_fwd<T>(m->tok, m->pos, A.P(m->o_wte), nullptr, A.x(0), M, C, s)); }
+  for (int l = 0; l < m->NL; ++l) {
+    const LayerOff& lo = m->L[l];
+    { ProfScope ps(m, PC_LN_FWD, 0, lnb);
+      CK(launch_ln_fwd<T>(A.x(l), A.P(lo.ln1_g), nullptr, A.h1(l), A.mu1(l), A.rs1(l), M, C, eps, s)); }
+    CKI(gemm(m, M, QW, C, A.h1(l), C, false, A.W(lo.w_qkv), C, false, epi_store<T>(A.qkv(l), QW, nullptr, nullptr, 0)));
+    CK(launch_rope<T>(A.qkv(l), QW, M, m->H, C, m->Hkv, m->d, m->pos, 0, nullptr, m->rope_tab, m->Tmax, false, s));
+    CKI(attn_fwd(m, A.qkv(l), A.att(l), A.lse(l), B, T_, &lay));
+    CKI(gemm(m, M, C, C, A.att(l), C, false, A.W(lo.w_o), C, false, epi_store<T>(A.xmid(l), C, nullptr, A.x(l), C)));
+    { ProfScope ps(m, PC_LN_FWD, 0, lnb);
+      CK(launch_ln_fwd<T>(A.xmid(l), A.P(lo.ln2_g), nullptr, A.h2(l), A.mu2(l), A.rs2(l), M, C, eps, s)); }
+    CKI(gemm(m, M, 2 * F, C, A.h2(l), C, false, A.W(lo.w_fc), C, false,
+             epi_store<T>(A.u(l), 2 * F, nullptr, nullptr, 0)));
+    CK(launch_swiglu<T>(A.u(l), A.a(l), M, F, s));
+    CKI(gemm(m, M, C, F, A.a(l), F, false, A.W(lo.w_fc2), F, false,
+             epi_store<T>(A.x(l + 1), C, nullptr, A.xmid(l), C)));
+  }
+  { ProfScope ps(m, PC_LN_FWD, 0, lnb);
+    CK(launch_ln_fwd<T>(A.x(m->NL), A.P(m->o_lnf_g), nullptr, (T*)m->xf, m->muf, m->rsf, M, C, eps, s)); }
+  CKI(gemm(m, M, m->Vp, C, (const T*)m->xf, C, false, A.W(m->o_head), C, false,
+           epi_store<T>((T*)m->logits, m->ldl, nullptr, nullptr, 0)));
+  if (targets) {
+    ProfScope ps(m, PC_XENT, 0, 2.0 * es * M * m->Vp);
+    CK(launch_xent<T>((T*)m->logits, m->ldl, m->tgt, M, m->V, m->Vp, m->rowloss, m->sc, s));
+    CK(launch_loss_finalize(m->rowloss, M, m->sc, loss_dev, s));
+  }
+  m->fwd_B = B;
+  m->fwd_T = T_;
+  m->have_targets = targets != nullptr;
+  m->logits_valid = targets == nullptr;
+  return GPT_OK;
+}
+
+template <typename T>
+static int backward_llama(gpt_model* m) {
+  cudaStream_t s = m->stream;
+  Acts<T> A(m);
+  const int B = m->fwd_B, T_ = m->fwd_T, M = B * T_, C = m->C, F = m->F, Vp = m->Vp, QW = m->QW;
+  T* dC = (T*)m->dC;
+  T* dgu = (T*)m->dF;                       // [M, 2F]
+  T* da = (T*)m->dF + (size_t)m->Mmax * 2 * F;   // [M, F]
+  T* dq = (T*)m->dqkv;                      // [M, QW]
+  T* drt = (T*)m->dres_t;
+  const T* dz = (const T*)m->logits;
+  const T* xf = (const T*)m->xf;
+  int nblk = 0;
+  const double es = sizeof(T), lnbb = (double)M * C * (3 * es + 8) + 8.0 * M;
+  const AttnLayout lay = llama_layout(m, m->dqkv);
+  std::vector<RedSeg>& segs = m->redsegs;
+  segs.clear();
+  float* pp = m->partials;
+  float* const pend = m->partials + m->partials_n;
+  auto take = [&](size_t n) -> float* {
+    float* p = pp;
+    pp += (n + 3) & ~(size_t)3;
+    return pp <= pend ? p : nullptr;
+  };
+  // RMSNorm backward; its partial rows are [dg | (unused) | column sums]
+  auto rms_bwd = [&](const T* x, const float* mu, const float* rs, const float* g, const float* din,
+                     float* gdst) -> int {
+    float* part = take((size_t)444 * 3 * C);
+    if (!part) FAIL(GPT_ERR_NOMEM, "partials arena too small");
+    ProfScope ps(m, PC_LN_BWD, 0, lnbb);
+    CK(launch_ln_bwd<T>(dC, x, mu, rs, g, din, m->dres32, drt, part, M, C, &nblk, s, true));
+    segs.push_back({part, gdst, nblk, C, 3 * C, 0});
+    return GPT_OK;
+  };
+  CKI(gemm(m, M, C, Vp, dz, m->ldl, false, A.W(m->o_head), C, true, epi_store<T>(dC, C, nullptr, nullptr, 0)));
+  CKI(gemm(m, Vp, C, M, dz, m->ldl, true, xf, C, true, epi_f32<T>(A.G(m->o_head), C)));
+  CKI(rms_bwd(A.x(m->NL), m->muf, m->rsf, A.P(m->o_lnf_g), nullptr, A.G(m->o_lnf_g)));
+  for (int l = m->NL - 1; l >= 0; --l) {
+    const LayerOff& lo = m->L[l];
+    // MLP: x_out = x_mid + swiglu(h2 W_gu^T) W_down^T
+    CKI(gemm(m, C, F, M, drt, C, true, A.a(l), F, true, epi_f32<T>(A.G(lo.w_fc2), F)));
+    CKI(gemm(m, M, F, C, drt, C, false, A.W(lo.w_fc2), F, true, epi_store<T>(da, F, nullptr, nullptr, 0)));
+    CK(launch_swiglu_bwd<T>(da, A.u(l), dgu, M, F, s));
+    CKI(gemm(m, 2 * F, C, M, dgu, 2 * F, true, A.h2(l), C, true, epi_f32<T>(A.G(lo.w_fc), C)));
+    CKI(gemm(m, M, C, 2 * F, dgu, 2 * F, false, A.W(lo.w_fc), C, true, epi_store<T>(dC, C, nullptr, nullptr, 0)));
+    CKI(rms_bwd(A.xmid(l), A.mu2(l), A.rs2(l), A.P(lo.ln2_g), m->dres32, A.G(lo.ln2_g)));
+    // attention: x_mid = x + attn(rope(h1 W_qkv^T)) W_o^T
+    CKI(gemm(m, C, C, M, drt, C, true, A.att(l), C, true, epi_f32<T>(A.G(lo.w_o), C)));
+    {
+      EpiParams<T> e = epi_store<T>(dC, C, nullptr, nullptr, 0);
+      e.aux = A.att(l); e.ld_aux = C; e.rowdot = m->attD; e.rd_T = T_;
+      CKI(gemm(m, M, C, C, drt, C, false, A.W(lo.w_o), C, true, e));
+    }
+    CKI(attn_bwd(m, A.qkv(l), A.att(l), dC, A.lse(l), dq, B, T_, true, &lay));
+    if (lay.G > 1)
+      CK(launch_gqa_reduce<T>((const T*)m->dkvq, dq, QW, lay.kcol, lay.vcol, M, m->Hkv, lay.G, m->d, s));
+    CK(launch_rope<T>(dq, QW, M, m->H, C, m->Hkv, m->d, m->pos, 0, nullptr, m->rope_tab, m->Tmax, true, s));
+    CKI(gemm(m, QW, C, M, dq, QW, true, A.h1(l), C, true, epi_f32<T>(A.G(lo.w_qkv), C)));
+    CKI(gemm(m, M, C, QW, dq, QW, false, A.W(lo.w_qkv), C, true, epi_store<T>(dC, C, nullptr, nullptr, 0)));
+    CKI(rms_bwd(A.x(l), A.mu1(l), A.rs1(l), A.P(lo.ln1_g), m->dres32, A.G(lo.ln1_g)));
+  }
+  {
+    double pb = 0;
+    for (const RedSeg& g : segs) pb += (double)g.rows * g.cols * 4;
+    ProfScope ps(m, PC_BIAS, 0, pb);
+    CK(launch_reduce_segs(segs.data(), (int)segs.size(), m->accum_now, s));
+  }
+  ProfScope ps_emb(m, PC_EMBED, 0, (double)M * C * 8);
+  if (!m->cfg.tied && !m->accum_now) CK(cudaMemsetAsync(A.G(m->o_wte), 0, (size_t)Vp * C * 4, s));
+  CK(launch_embed_bwd<T>(m->dres32, m->tok, m->pos, A.G(m->o_wte), nullptr, M, C, s));
   m->have_targets = false;
   return GPT_OK;
 }
@@ -618,38 +889,76 @@ static cudaError_t dec_proj(gpt_model* m, const T* X, int B, int K, const T* W, 
     if (B > 8 && gemm_tc_supported(B, N, K, K, false, K, false)) {
       EpiParams<T> e = mode == 2 ? epi_f32<T>(outf, N)
                                  : mode == 1 ? epi_gelu<T>(out, out2, N, bias) : epi_store<T>(out, N, bias, resid, N);
-      return launch_gemm_tc(B, N, K, X, K, false, W, K, false, e, 1, &m->sc->err, s);
+      return tc_gemm<T>(B, N, K, X, K, false, W, K, false, e, 1, &m->sc->err, s);
     }
   }
   return launch_gemv<T>(X, B, K, W, N, bias, resid, mode, out, out2, outf, s);
 }
 
+// The Llama-style kernels exist for the 16-bit types only (the block needs
+// 16-bit precision; create() refuses it in fp32 mode).
+template <typename T>
+static cudaError_t rope16(T* x, long ld, int rows, int nq, int kcol, int nk, int d, const int* pos, int pos0,
+                          const int* step, const float2* tab, int max_seq, bool inverse, cudaStream_t s) {
+  if constexpr (sizeof(T) == 2) return launch_rope<T>(x, ld, rows, nq, kcol, nk, d, pos, pos0, step, tab, max_seq, inverse, s);
+  else return cudaErrorNotSupported;
+}
+template <typename T>
+static cudaError_t swiglu16(const T* gu, T* a, int rows, int F, cudaStream_t s) {
+  if constexpr (sizeof(T) == 2) return launch_swiglu<T>(gu, a, rows, F, s);
+  else return cudaErrorNotSupported;
+}
+
+static DecLayout dec_layout(const gpt_model* m) {
+  DecLayout L;
+  L.qw = m->QW;
+  L.kcol = m->C;
+  L.vcol = m->C + m->Hkv * m->d;
+  L.Hkv = m->Hkv;
+  return L;
+}
+
 template <typename T>
 static int decode_step(gpt_model* m, int B, int Tp, int n_new, int32_t* out, cudaStream_t s) {
   Acts<T> A(m);
-  const int C = m->C, F = m->F, H = m->H, d = m->d;
+  const int C = m->C, F = m->F, H = m->H, d = m->d, QW = m->QW;
   const float eps = m->cfg.ln_eps;
-  size_t kvl = (size_t)m->Bmax * H * m->Tmax * d;
+  const bool ll = m->llama;
+  const DecLayout DL = dec_layout(m);
+  size_t kvl = (size_t)m->Bmax * m->Hkv * m->Tmax * d;
   T* kc = (T*)m->kc;
   T* vc = (T*)m->vc;
   T *x = (T*)m->dx, *h = (T*)m->dh, *q = (T*)m->dq, *att = (T*)m->datt, *u = (T*)m->du, *a = (T*)m->da,
     *xf = (T*)m->dxf;
   int* stepc = &m->sc->dec_step;
+  // LayerNorm parameters (Llama: RMSNorm, gains only) and biases (Llama: none)
+  auto P0 = [&](size_t off) -> const float* { return ll ? nullptr : A.P(off); };
   // the token fed at step st sits at position Tp - 1 + st
-  CK(launch_dec_embed<T>(m->dtok, A.P(m->o_wte), A.P(m->o_wpe), x, B, C, Tp - 1, stepc, m->Tmax, &m->sc->err, s));
+  CK(launch_dec_embed<T>(m->dtok, A.P(m->o_wte), ll ? nullptr : A.P(m->o_wpe), x, B, C, Tp - 1, stepc, m->Tmax,
+                         &m->sc->err, s));
   for (int l = 0; l < m->NL; ++l) {
     const LayerOff& lo = m->L[l];
-    CK(launch_ln_fwd<T>(x, A.P(lo.ln1_g), A.P(lo.ln1_b), h, m->dmu, m->drs, B, C, eps, s));
-    CK(dec_proj<T>(m, h, B, C, A.W(lo.w_qkv), 3 * C, A.P(lo.b_qkv), nullptr, 0, q, nullptr, nullptr, s));
-    CK(launch_dec_attn<T>(q, kc + l * kvl, vc + l * kvl, att, m->dpart, B, H, d, m->Tmax, Tp - 1, stepc, s));
-    CK(dec_proj<T>(m, att, B, C, A.W(lo.w_o), C, A.P(lo.b_o), x, 0, x, nullptr, nullptr, s));
-    CK(launch_ln_fwd<T>(x, A.P(lo.ln2_g), A.P(lo.ln2_b), h, m->dmu, m->drs, B, C, eps, s));
-    CK(dec_proj<T>(m, h, B, C, A.W(lo.w_fc), F, A.P(lo.b_fc), nullptr, 1, u, a, nullptr, s));
-    CK(dec_proj<T>(m, a, B, F, A.W(lo.w_fc2), C, A.P(lo.b_fc2), x, 0, x, nullptr, nullptr, s));
+    CK(launch_ln_fwd<T>(x, A.P(lo.ln1_g), P0(lo.ln1_b), h, m->dmu, m->drs, B, C, eps, s));
+    CK(dec_proj<T>(m, h, B, C, A.W(lo.w_qkv), QW, P0(lo.b_qkv), nullptr, 0, q, nullptr, nullptr, s));
+    if (ll) CK(rope16<T>(q, QW, B, H, C, m->Hkv, d, nullptr, Tp - 1, stepc, m->rope_tab, m->Tmax, false, s));
+    CK(launch_dec_attn<T>(q, kc + l * kvl, vc + l * kvl, att, m->dpart, B, H, d, m->Tmax, Tp - 1, stepc, DL, s));
+    CK(dec_proj<T>(m, att, B, C, A.W(lo.w_o), C, P0(lo.b_o), x, 0, x, nullptr, nullptr, s));
+    CK(launch_ln_fwd<T>(x, A.P(lo.ln2_g), P0(lo.ln2_b), h, m->dmu, m->drs, B, C, eps, s));
+    if (ll) {
+      CK(dec_proj<T>(m, h, B, C, A.W(lo.w_fc), 2 * F, nullptr, nullptr, 0, u, nullptr, nullptr, s));
+      CK(swiglu16<T>(u, a, B, F, s));
+    } else {
+      CK(dec_proj<T>(m, h, B, C, A.W(lo.w_fc), F, A.P(lo.b_fc), nullptr, 1, u, a, nullptr, s));
+    }
+    CK(dec_proj<T>(m, a, B, F, A.W(lo.w_fc2), C, P0(lo.b_fc2), x, 0, x, nullptr, nullptr, s));
   }
-  CK(launch_ln_fwd<T>(x, A.P(m->o_lnf_g), A.P(m->o_lnf_b), xf, m->dmu, m->drs, B, C, eps, s));
+  CK(launch_ln_fwd<T>(x, A.P(m->o_lnf_g), P0(m->o_lnf_b), xf, m->dmu, m->drs, B, C, eps, s));
   CK(dec_proj<T>(m, xf, B, C, A.W(m->o_head), m->Vp, nullptr, nullptr, 2, nullptr, nullptr, m->dlogits, s));
-  CK(launch_argmax(m->dlogits, B, m->V, m->Vp, m->dtok, out, n_new, stepc, s));
+  if (m->smp_on)
+    CK(launch_sample(m->dlogits, B, m->V, m->Vp, m->smp_temp, m->smp_topk, m->smp_topp, m->smp_u, n_new, m->dtok, out,
+                     n_new, stepc, s));
+  else
+    CK(launch_argmax(m->dlogits, B, m->V, m->Vp, m->dtok, out, n_new, stepc, s));
   CK(launch_step_advance(stepc, s));
   return GPT_OK;
 }
@@ -661,15 +970,48 @@ static int decode_impl(gpt_model* m, const int32_t* prompt, int B, int Tp, int n
   const int C = m->C, H = m->H, d = m->d;
   CKI(forward_impl<T>(m, prompt, nullptr, nullptr, B, Tp, nullptr));
   m->logits_valid = false;
-  size_t kvl = (size_t)m->Bmax * H * m->Tmax * d;
+  size_t kvl = (size_t)m->Bmax * m->Hkv * m->Tmax * d;
+  const DecLayout DL = dec_layout(m);
   for (int l = 0; l < m->NL; ++l)
-    CK(launch_kv_fill<T>(A.qkv(l), (T*)m->kc + l * kvl, (T*)m->vc + l * kvl, B, Tp, H, d, m->Tmax, s));
+    CK(launch_kv_fill<T>(A.qkv(l), (T*)m->kc + l * kvl, (T*)m->vc + l * kvl, B, Tp, d, m->Tmax, DL, s));
   // first new token: from the prefill's last position
   CK(launch_gather_last<T>((const T*)m->xf, B, Tp, C, (T*)m->dxf, s));
   CK(dec_proj<T>(m, (const T*)m->dxf, B, C, A.W(m->o_head), m->Vp, nullptr, nullptr, 2, nullptr, nullptr,
                  m->dlogits, s));
-  CK(launch_argmax(m->dlogits, B, m->V, m->Vp, m->dtok, out, n_new, nullptr, s));
+  if (m->smp_on)
+    CK(launch_sample(m->dlogits, B, m->V, m->Vp, m->smp_temp, m->smp_topk, m->smp_topp, m->smp_u, n_new, m->dtok, out,
+                     n_new, nullptr, s));
+  else
+    CK(launch_argmax(m->dlogits, B, m->V, m->Vp, m->dtok, out, n_new, nullptr, s));
   if (n_new == 1) return GPT_OK;
+  if constexpr (sizeof(T) == 2) {
+    if (!m->smp_on && !m->fp16 && !m->llama && dec_fused_supported(B, C, H, m->F, m->Vp)) {
+      // every later token from one persistent kernel
+      const LayerOff& l0 = m->L[0];
+      DecFusedParams q;
+      memset(&q, 0, sizeof(q));
+      q.pw = (const bf16*)m->pw; q.p32 = m->p32;
+      q.o_wte = m->o_wte; q.o_wpe = m->o_wpe; q.o_lnf_g = m->o_lnf_g; q.o_lnf_b = m->o_lnf_b; q.o_head = m->o_head;
+      q.l_ln1_g = l0.ln1_g; q.l_ln1_b = l0.ln1_b; q.l_w_qkv = l0.w_qkv; q.l_b_qkv = l0.b_qkv; q.l_w_o = l0.w_o;
+      q.l_b_o = l0.b_o; q.l_ln2_g = l0.ln2_g; q.l_ln2_b = l0.ln2_b; q.l_w_fc = l0.w_fc; q.l_b_fc = l0.b_fc;
+      q.l_w_fc2 = l0.w_fc2; q.l_b_fc2 = l0.b_fc2;
+      q.l_stride = m->NL > 1 ? (long)(m->L[1].ln1_g - l0.ln1_g) : (long)(m->o_lnf_g - l0.ln1_g);
+      q.NL = m->NL; q.C = C; q.H = H; q.D = d; q.F = m->F; q.V = m->V; q.Vp = m->Vp; q.Tmax = m->Tmax;
+      q.eps = m->cfg.ln_eps;
+      q.kc = (bf16*)m->kc; q.vc = (bf16*)m->vc; q.kvl = (long)kvl;
+      q.B = B; q.pos_first = Tp; q.n_steps = n_new - 1;
+      q.tok = m->dtok; q.out = out; q.out_ld = n_new; q.out_col0 = 1;
+      q.qkv = (bf16*)m->dq; q.part = m->dpart; q.xmid = (bf16*)m->dh; q.abuf = (bf16*)m->da; q.xbuf = (bf16*)m->dx;
+      q.logits = m->dlogits; q.am_v = m->dam; q.am_i = (int*)(m->dam + (size_t)m->Bmax * DF_MAX_GRID);
+      q.cnt = (int*)(m->dam + (size_t)m->Bmax * DF_MAX_GRID * 2);
+      q.att = (bf16*)m->datt;
+      q.bar = &m->sc->dec_bar; q.abortf = &m->sc->dec_abort; q.err = &m->sc->err;
+      CK(cudaMemsetAsync(&m->sc->dec_bar, 0, 2 * sizeof(unsigned), s));
+      CK(cudaMemsetAsync(q.cnt, 0, (size_t)B * H * sizeof(int), s));
+      CK(launch_decode_fused(q, s));
+      return GPT_OK;
+    }
+  }
   const int one = 1;
   CK(cudaMemcpyAsync(&m->sc->dec_step, &one, sizeof(int), cudaMemcpyHostToDevice, s));
   // later tokens: one captured step (about 7 L + 5 kernels), replayed n_new - 1 times
@@ -678,7 +1020,9 @@ static int decode_impl(gpt_model* m, const int32_t* prompt, int B, int Tp, int n
     CK(cudaEventCreateWithFlags(&m->ev_a, cudaEventDisableTiming));
     CK(cudaEventCreateWithFlags(&m->ev_b, cudaEventDisableTiming));
   }
-  if (!m->dec_graph || m->dec_B != B || m->dec_Tp != Tp || m->dec_nnew != n_new || m->dec_out != out) {
+  const bool same_smp = m->dec_smp_on == m->smp_on && m->dec_smp_temp == m->smp_temp &&
+                        m->dec_smp_topk == m->smp_topk && m->dec_smp_topp == m->smp_topp && m->dec_smp_u == m->smp_u;
+  if (!m->dec_graph || m->dec_B != B || m->dec_Tp != Tp || m->dec_nnew != n_new || m->dec_out != out || !same_smp) {
     if (m->dec_graph) { cudaGraphExecDestroy(m->dec_graph); m->dec_graph = nullptr; }
     cudaGraph_t g = nullptr;
     unsigned long long n0 = g_kernel_launches;
@@ -695,6 +1039,8 @@ static int decode_impl(gpt_model* m, const int32_t* prompt, int B, int Tp, int n
     g_kernel_launches = n0;
     m->dec_kernels = 7 * m->NL + 5;
     m->dec_B = B; m->dec_Tp = Tp; m->dec_nnew = n_new; m->dec_out = out;
+    m->dec_smp_on = m->smp_on; m->dec_smp_temp = m->smp_temp; m->dec_smp_topk = m->smp_topk;
+    m->dec_smp_topp = m->smp_topp; m->dec_smp_u = m->smp_u;
   }
   CK(cudaEventRecord(m->ev_a, s));
   CK(cudaStreamWaitEvent(m->cap_stream, m->ev_a, 0));
@@ -716,9 +1062,21 @@ static int validate_cfg(const gpt_config* c, std::string& why) {
   if (d != 16 && d != 32 && d != 64 && d != 128) { why = "head size must be 16, 32, 64 or 128"; return 0; }
   if (c->d_mlp < 8 || c->d_mlp % 8) { why = "d_mlp must be a positive multiple of 8"; return 0; }
   if (c->n_layers < 1 || c->max_seq < 1 || c->max_batch < 1) { why = "n_layers, max_seq, max_batch >= 1"; return 0; }
-  if (c->precision != GPT_PRECISION_FP32 && c->precision != GPT_PRECISION_BF16) { why = "precision"; return 0; }
+  if (c->precision != GPT_PRECISION_FP32 && c->precision != GPT_PRECISION_BF16 && c->precision != GPT_PRECISION_FP16) {
+    why = "precision";
+    return 0;
+  }
   if (!(c->ln_eps > 0.f) || !(c->init_std >= 0.f)) { why = "ln_eps > 0, init_std >= 0"; return 0; }
   if (c->loss_scaling && !(c->init_loss_scale > 0.f)) { why = "init_loss_scale > 0"; return 0; }
+  if (c->arch != GPT_ARCH_GPT2 && c->arch != GPT_ARCH_LLAMA) { why = "arch"; return 0; }
+  if (c->arch == GPT_ARCH_LLAMA) {
+    if (c->precision == GPT_PRECISION_FP32) { why = "the Llama-style block needs 16-bit precision"; return 0; }
+    if (d != 64) { why = "the Llama-style block needs head size 64"; return 0; }
+    const int hkv = c->n_kv_heads ? c->n_kv_heads : c->n_heads;
+    if (hkv < 1 || c->n_heads % hkv) { why = "n_kv_heads must divide n_heads"; return 0; }
+    if (c->d_mlp % 16) { why = "d_mlp must be a multiple of 16 for the Llama-style block"; return 0; }
+    if (!(c->rope_base >= 0.f)) { why = "rope_base >= 0"; return 0; }
+  }
   return 1;
 }
 
@@ -740,26 +1098,45 @@ int gpt_create(const gpt_config* cfg, uint64_t seed, gpt_model** out) {
   int nsm = 0;
   if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, m->device) == cudaSuccess && nsm > 0)
     g_num_sms = nsm;
-  m->bf16 = cfg->precision == GPT_PRECISION_BF16;
+  m->lp = cfg->precision == GPT_PRECISION_BF16 || cfg->precision == GPT_PRECISION_FP16;
+  m->fp16 = cfg->precision == GPT_PRECISION_FP16;
   m->V = cfg->vocab; m->Vp = cfg->vocab_padded; m->C = cfg->d_model; m->H = cfg->n_heads;
   m->d = m->C / m->H; m->F = cfg->d_mlp; m->NL = cfg->n_layers; m->Tmax = cfg->max_seq;
   m->Bmax = cfg->max_batch; m->Mmax = (long)m->Bmax * m->Tmax;
   m->ldl = (m->Vp + 7) / 8 * 8;
+  m->llama = cfg->arch == GPT_ARCH_LLAMA;
+  m->Hkv = m->llama && cfg->n_kv_heads ? cfg->n_kv_heads : m->H;
+  m->QW = m->llama ? m->C + 2 * m->Hkv * m->d : 3 * m->C;
+  m->UW = m->llama ? 2 * m->F : m->F;
   layout_params(m);
   int r = build_arena(m);
   if (r != GPT_OK) { g_create_err = m->err; delete m; return r; }
   std::vector<float> h;
   init_host_params(m, seed, h);
   cudaError_t e = cudaMemcpy(m->p32, h.data(), m->N * 4, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && m->llama) {
+    // rotary table: (cos, sin) of p * base^(-2i/d), evaluated in double precision
+    const double base = cfg->rope_base > 0.f ? (double)cfg->rope_base : 10000.0;
+    const int hd = m->d / 2;
+    std::vector<float2> tab((size_t)m->Tmax * hd);
+    for (int p = 0; p < m->Tmax; ++p)
+      for (int i = 0; i < hd; ++i) {
+        const double a = (double)p * pow(base, -2.0 * i / m->d);
+        tab[(size_t)p * hd + i] = make_float2((float)cos(a), (float)sin(a));
+      }
+    e = cudaMemcpy(m->rope_tab, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice);
+  }
   if (e == cudaSuccess) e = cudaMemset(m->g32, 0, m->N * 4);
   if (e == cudaSuccess) e = cudaMemset(m->m32, 0, m->N * 4);
   if (e == cudaSuccess) e = cudaMemset(m->v32, 0, m->N * 4);
-  if (e == cudaSuccess && m->bf16) e = launch_cast<bf16>(m->p32, (bf16*)m->pw, m->N, 0);
+  if (e == cudaSuccess && m->fp16) e = launch_cast<f16>(m->p32, (f16*)m->pw, m->N, 0);
+  else if (e == cudaSuccess && m->lp) e = launch_cast<bf16>(m->p32, (bf16*)m->pw, m->N, 0);
   DevScalars sc;
   memset(&sc, 0, sizeof(sc));
   sc.loss_scale = cfg->loss_scaling ? cfg->init_loss_scale : 1.0f;
   sc.loss_scaling = cfg->loss_scaling ? 1 : 0;
   sc.coef = 1.f; sc.bc1 = 1.f; sc.bc2 = 1.f;
+  sc.loss_weight = 1.f;
   if (e == cudaSuccess) e = cudaMemcpy(m->sc, &sc, sizeof(sc), cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
@@ -797,7 +1174,8 @@ int gpt_forward_loss(gpt_model* m, const int32_t* tokens, const int32_t* targets
   if (!tokens) FAIL(GPT_ERR_ARG, "tokens is NULL");
   if (B < 1 || B > m->Bmax) FAIL(GPT_ERR_ARG, "B out of range [1, max_batch]");
   if (T < 1 || T > m->Tmax) FAIL(GPT_ERR_ARG, "T out of range [1, max_seq]");
-  if (m->bf16) return forward_impl<bf16>(m, tokens, targets, seg_ids, B, T, loss_dev);
+  if (m->fp16) return forward_impl<f16>(m, tokens, targets, seg_ids, B, T, loss_dev);
+  if (m->lp) return forward_impl<bf16>(m, tokens, targets, seg_ids, B, T, loss_dev);
   return forward_impl<float>(m, tokens, targets, seg_ids, B, T, loss_dev);
 }
 
@@ -805,8 +1183,29 @@ int gpt_backward(gpt_model* m) {
   if (!m) return GPT_ERR_ARG;
   m->err.clear();
   if (!m->have_targets) FAIL(GPT_ERR_STATE, "gpt_backward needs a preceding gpt_forward_loss with targets");
-  if (m->bf16) return backward_impl<bf16>(m);
+  m->accum_now = false;
+  if (m->fp16) return backward_impl<f16>(m);
+  if (m->lp) return backward_impl<bf16>(m);
   return backward_impl<float>(m);
+}
+
+int gpt_backward_accumulate(gpt_model* m) {
+  if (!m) return GPT_ERR_ARG;
+  m->err.clear();
+  if (!m->have_targets) FAIL(GPT_ERR_STATE, "gpt_backward_accumulate needs a preceding gpt_forward_loss with targets");
+  m->accum_now = true;
+  const int r = m->fp16 ? backward_impl<f16>(m) : m->lp ? backward_impl<bf16>(m) : backward_impl<float>(m);
+  m->accum_now = false;
+  return r;
+}
+
+int gpt_set_loss_weight(gpt_model* m, float w) {
+  if (!m) return GPT_ERR_ARG;
+  m->err.clear();
+  if (!(w > 0.f) || !(w < 1e30f)) FAIL(GPT_ERR_ARG, "loss weight must be positive and finite");
+  CK(cudaMemcpyAsync(&m->sc->loss_weight, &w, sizeof(float), cudaMemcpyHostToDevice, m->stream));
+  CK(cudaStreamSynchronize(m->stream));
+  return GPT_OK;
 }
 
 int gpt_clip_adamw_step(gpt_model* m, const gpt_adamw* hp, float* grad_norm_dev, int32_t* skipped_dev) {
@@ -814,16 +1213,78 @@ int gpt_clip_adamw_step(gpt_model* m, const gpt_adamw* hp, float* grad_norm_dev,
   m->err.clear();
   if (!(hp->clip_norm > 0.f)) FAIL(GPT_ERR_ARG, "clip_norm must be > 0");
   cudaStream_t s = m->stream;
-  ProfScope ps(m, PC_OPT, 0, (double)m->N * (m->bf16 ? 34.0 : 32.0));
+  ProfScope ps(m, PC_OPT, 0, (double)m->N * (m->lp ? 34.0 : 32.0));
+  {
+    // one cooperative launch; the three-launch form below if it cannot run
+    cudaError_t e;
+    if (m->fp16)
+      e = launch_clip_adamw_fused<f16>(m->p32, m->g32, m->m32, m->v32, (f16*)m->pw, m->N, m->normpart, m->normblk,
+                                       hp->clip_norm, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, hp->lr, m->sc,
+                                       grad_norm_dev, skipped_dev, s);
+    else if (m->lp)
+      e = launch_clip_adamw_fused<bf16>(m->p32, m->g32, m->m32, m->v32, (bf16*)m->pw, m->N, m->normpart, m->normblk,
+                                        hp->clip_norm, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, hp->lr, m->sc,
+                                        grad_norm_dev, skipped_dev, s);
+    else
+      e = launch_clip_adamw_fused<float>(m->p32, m->g32, m->m32, m->v32, nullptr, m->N, m->normpart, m->normblk,
+                                         hp->clip_norm, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, hp->lr,
+                                         m->sc, grad_norm_dev, skipped_dev, s);
+    if (e == cudaSuccess) return GPT_OK;
+    cudaGetLastError();
+  }
   CK(launch_sumsq(m->g32, m->N, m->normpart, m->normblk, s));
-  CK(launch_opt_finalize(m->normpart, m->normblk, hp->clip_norm, hp->beta1, hp->beta2, m->sc, grad_norm_dev,
-                         skipped_dev, s));
-  if (m->bf16)
-    CK(launch_adamw<bf16>(m->p32, m->g32, m->m32, m->v32, (bf16*)m->pw, m->N, hp->lr, hp->beta1, hp->beta2,
+  CK(launch_opt_finalize(m->normpart, m->normblk, hp->clip_norm, hp->beta1, hp->beta2, hp->lr, m->sc,
+                         grad_norm_dev, skipped_dev, s));
+  if (m->fp16)
+    CK(launch_adamw<f16>(m->p32, m->g32, m->m32, m->v32, (f16*)m->pw, m->N, hp->beta1, hp->beta2,
+                         hp->eps, hp->weight_decay, m->sc, s));
+  else if (m->lp)
+    CK(launch_adamw<bf16>(m->p32, m->g32, m->m32, m->v32, (bf16*)m->pw, m->N, hp->beta1, hp->beta2,
                           hp->eps, hp->weight_decay, m->sc, s));
   else
-    CK(launch_adamw<float>(m->p32, m->g32, m->m32, m->v32, nullptr, m->N, hp->lr, hp->beta1, hp->beta2,
+    CK(launch_adamw<float>(m->p32, m->g32, m->m32, m->v32, nullptr, m->N, hp->beta1, hp->beta2,
                            hp->eps, hp->weight_decay, m->sc, s));
+  return GPT_OK;
+}
+
+int gpt_set_lr_schedule(gpt_model* m, const gpt_lr_schedule* sched) {
+  if (!m) return GPT_ERR_ARG;
+  m->err.clear();
+  gpt_lr_schedule z;
+  memset(&z, 0, sizeof(z));
+  const gpt_lr_schedule& q = sched ? *sched : z;
+  if (q.kind != GPT_LR_CONSTANT && q.kind != GPT_LR_COSINE) FAIL(GPT_ERR_ARG, "unknown schedule kind");
+  if (q.kind == GPT_LR_COSINE) {
+    if (q.warmup_steps < 0 || q.total_steps <= q.warmup_steps) FAIL(GPT_ERR_ARG, "need 0 <= warmup_steps < total_steps");
+    if (!(q.min_lr >= 0.f) || !(q.max_lr >= q.min_lr)) FAIL(GPT_ERR_ARG, "need 0 <= min_lr <= max_lr");
+  }
+  DevScalars sc;
+  CK(cudaStreamSynchronize(m->stream));
+  CK(cudaMemcpy(&sc, m->sc, sizeof(sc), cudaMemcpyDeviceToHost));
+  sc.sched_kind = q.kind;
+  sc.sched_warmup = q.warmup_steps;
+  sc.sched_total = q.total_steps;
+  sc.sched_max_lr = q.max_lr;
+  sc.sched_min_lr = q.min_lr;
+  CK(cudaMemcpy(m->sc, &sc, sizeof(sc), cudaMemcpyHostToDevice));
+  return GPT_OK;
+}
+
+int gpt_train_steps(gpt_model* m, const int32_t* tokens, const int32_t* targets, const int32_t* seg_ids, int K,
+                    int B, int T, const gpt_adamw* hp, float* losses_dev, float* grad_norms_dev,
+                    int32_t* skipped_dev) {
+  if (!m) return GPT_ERR_ARG;
+  m->err.clear();
+  if (!tokens || !targets || !hp) FAIL(GPT_ERR_ARG, "tokens, targets and hp must be non-NULL");
+  if (K < 1) FAIL(GPT_ERR_ARG, "K must be >= 1");
+  const size_t bt = (size_t)B * T;
+  for (int k = 0; k < K; ++k) {
+    CKI(gpt_forward_loss(m, tokens + k * bt, targets + k * bt, seg_ids ? seg_ids + k * bt : nullptr, B, T,
+                         losses_dev ? losses_dev + k : nullptr));
+    CKI(gpt_backward(m));
+    CKI(gpt_clip_adamw_step(m, hp, grad_norms_dev ? grad_norms_dev + k : nullptr,
+                            skipped_dev ? skipped_dev + k : nullptr));
+  }
   return GPT_OK;
 }
 
@@ -835,8 +1296,32 @@ int gpt_greedy_decode(gpt_model* m, const int32_t* prompt, int B, int Tp, int n_
   if (Tp < 1 || n_new < 1) FAIL(GPT_ERR_ARG, "Tp and n_new must be >= 1");
   if ((long)Tp + n_new - 1 > m->Tmax) FAIL(GPT_ERR_STATE, "Tp + n_new - 1 exceeds max_seq");
   m->have_targets = false;
-  if (m->bf16) return decode_impl<bf16>(m, prompt, B, Tp, n_new, out);
+  if (m->fp16) return decode_impl<f16>(m, prompt, B, Tp, n_new, out);
+  if (m->lp) return decode_impl<bf16>(m, prompt, B, Tp, n_new, out);
   return decode_impl<float>(m, prompt, B, Tp, n_new, out);
+}
+
+int gpt_sample_decode(gpt_model* m, const int32_t* prompt, int B, int Tp, int n_new, const gpt_sampling* sp,
+                      const float* uniforms, int32_t* out) {
+  if (!m) return GPT_ERR_ARG;
+  m->err.clear();
+  if (!prompt || !out || !sp || !uniforms) FAIL(GPT_ERR_ARG, "prompt / out / sampling / uniforms is NULL");
+  if (!(sp->temperature >= 0.f) || sp->top_k < 0 || !(sp->top_p > 0.f && sp->top_p <= 1.f))
+    FAIL(GPT_ERR_ARG, "need temperature >= 0, top_k >= 0, 0 < top_p <= 1");
+  if (m->V > SMP_MAX_VOCAB) FAIL(GPT_ERR_ARG, "vocabulary too large for the sampling kernel");
+  if (B < 1 || B > m->Bmax || B > 32) FAIL(GPT_ERR_ARG, "B out of range [1, min(max_batch, 32)]");
+  if (Tp < 1 || n_new < 1) FAIL(GPT_ERR_ARG, "Tp and n_new must be >= 1");
+  if ((long)Tp + n_new - 1 > m->Tmax) FAIL(GPT_ERR_STATE, "Tp + n_new - 1 exceeds max_seq");
+  m->have_targets = false;
+  m->smp_on = true;
+  m->smp_temp = sp->temperature;
+  m->smp_topk = sp->top_k;
+  m->smp_topp = sp->top_p;
+  m->smp_u = uniforms;
+  const int r = m->fp16 ? decode_impl<f16>(m, prompt, B, Tp, n_new, out)
+                : m->lp ? decode_impl<bf16>(m, prompt, B, Tp, n_new, out) : decode_impl<float>(m, prompt, B, Tp, n_new, out);
+  m->smp_on = false;
+  return r;
 }
 
 int gpt_num_params(const gpt_model* m, size_t* n) {
@@ -864,7 +1349,10 @@ int gpt_set_adam_v(gpt_model* m, const float* src, size_t n) { return m ? copy_s
 int gpt_set_params(gpt_model* m, const float* src, size_t n) {
   if (!m) return GPT_ERR_ARG;
   CKI(copy_state(m, m->p32, src, n));
-  if (m->bf16) {
+  if (m->fp16) {
+    CK(launch_cast<f16>(m->p32, (f16*)m->pw, m->N, m->stream));
+    CK(cudaStreamSynchronize(m->stream));
+  } else if (m->lp) {
     CK(launch_cast<bf16>(m->p32, (bf16*)m->pw, m->N, m->stream));
     CK(cudaStreamSynchronize(m->stream));
   }
@@ -883,7 +1371,8 @@ int gpt_get_logits(gpt_model* m, float* dst, size_t n) {
   float* tmp = dst;
   if (!dev) CK(cudaMalloc((void**)&tmp, n * 4));
   cudaError_t e;
-  if (m->bf16) e = launch_to_f32<bf16>((const bf16*)m->logits, m->ldl, M, m->Vp, tmp, m->stream);
+  if (m->fp16) e = launch_to_f32<f16>((const f16*)m->logits, m->ldl, M, m->Vp, tmp, m->stream);
+  else if (m->lp) e = launch_to_f32<bf16>((const bf16*)m->logits, m->ldl, M, m->Vp, tmp, m->stream);
   else e = launch_to_f32<float>((const float*)m->logits, m->ldl, M, m->Vp, tmp, m->stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(m->stream);
   if (e == cudaSuccess && !dev) e = cudaMemcpy(dst, tmp, n * 4, cudaMemcpyDeviceToHost);
@@ -906,7 +1395,8 @@ int gpt_get_residual(gpt_model* m, int layer, float* dst, size_t n) {
   float* tmp = dst;
   if (!dev) CK(cudaMalloc((void**)&tmp, n * 4));
   cudaError_t e;
-  if (m->bf16) e = launch_to_f32<bf16>((const bf16*)m->xs + off, m->C, M, m->C, tmp, m->stream);
+  if (m->fp16) e = launch_to_f32<f16>((const f16*)m->xs + off, m->C, M, m->C, tmp, m->stream);
+  else if (m->lp) e = launch_to_f32<bf16>((const bf16*)m->xs + off, m->C, M, m->C, tmp, m->stream);
   else e = launch_to_f32<float>((const float*)m->xs + off, m->C, M, m->C, tmp, m->stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(m->stream);
   if (e == cudaSuccess && !dev) e = cudaMemcpy(dst, tmp, n * 4, cudaMemcpyDeviceToHost);
@@ -926,6 +1416,7 @@ int gpt_get_scalars(gpt_model* m, gpt_scalars* out) {
   out->last_loss = sc.loss;
   out->last_grad_norm = sc.grad_norm;
   out->last_skipped = sc.skipped;
+  out->last_lr = sc.lr;
   return GPT_OK;
 }
 
@@ -1002,13 +1493,15 @@ int gpt_profile_read(gpt_model* m, gpt_prof_entry* out, int max_entries, int* n_
   CK(cudaStreamSynchronize(m->stream));
   gpt_prof_entry acc[PC_COUNT];
   memset(acc, 0, sizeof(acc));
+  unsigned long long pairs = 0;
+  CK(cudaMemcpy(&pairs, &m->sc->attn_pairs, sizeof(pairs), cudaMemcpyDeviceToHost));
   for (auto& r : m->recs) {
     if (!r.b) continue;
     float ms = 0.f;
     CK(cudaEventElapsedTime(&ms, r.a, r.b));
     acc[r.cls].launches += 1;
     acc[r.cls].ms += ms;
-    acc[r.cls].flops += r.flops;
+    acc[r.cls].flops += r.flops + r.pair_mult * (double)pairs;
     acc[r.cls].bytes += r.bytes;
   }
   int n = 0;

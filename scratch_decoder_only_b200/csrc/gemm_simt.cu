@@ -82,3 +82,5 @@ template cudaError_t launch_gemm_simt<float>(int, int, int, const float*, long, 
                                              const EpiParams<float>&, int, cudaStream_t);
 template cudaError_t launch_gemm_simt<bf16>(int, int, int, const bf16*, long, bool, const bf16*, long, bool,
                                             const EpiParams<bf16>&, int, cudaStream_t);
+template cudaError_t launch_gemm_simt<f16>(int, int, int, const f16*, long, bool, const f16*, long, bool,
+                                           const EpiParams<f16>&, int, cudaStream_t);

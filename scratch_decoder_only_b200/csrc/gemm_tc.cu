@@ -51,13 +51,14 @@ __device__ __forceinline__ void stage_row128(uint32_t buf, int r, const uint4* w
                  : "memory");
   }
 }
-__device__ __forceinline__ void pack_bf16x64(const float* v, uint4* w) {
+template <bool F16>
+__device__ __forceinline__ void pack16x64(const float* v, uint4* w) {
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
-    w[q].x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
-    w[q].y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
-    w[q].z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
-    w[q].w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    w[q].x = pack16x2<F16>(v[8 * q + 0], v[8 * q + 1]);
+    w[q].y = pack16x2<F16>(v[8 * q + 2], v[8 * q + 3]);
+    w[q].z = pack16x2<F16>(v[8 * q + 4], v[8 * q + 5]);
+    w[q].w = pack16x2<F16>(v[8 * q + 6], v[8 * q + 7]);
   }
 }
 
@@ -88,15 +89,16 @@ __device__ __forceinline__ bool epi_sync(uint32_t bar, uint32_t& phase, volatile
   return ok;
 }
 
-// Row r of a 128-row, 128-byte-swizzled bf16 buffer (64 values) into fp32.
-__device__ __forceinline__ void load_row128_bf16(uint32_t buf, int r, float* x) {
+// Row r of a 128-row, 128-byte-swizzled 16-bit buffer (64 values) into fp32.
+template <bool F16>
+__device__ __forceinline__ void load_row128_16(uint32_t buf, int r, float* x) {
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
     uint4 w;
     const uint32_t a = buf + r * 128 + ((q ^ (r & 7)) << 4);
     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w) : "r"(a)
                  : "memory");
-    Vec<bf16>::load(reinterpret_cast<const bf16*>(&w), x + 8 * q);
+    unpack16x8<F16>(w, x + 8 * q);
   }
 }
 __device__ __forceinline__ float4 ld_shared_f4(uint32_t a) {
@@ -113,6 +115,9 @@ __device__ __forceinline__ float4 ld_shared_f4(uint32_t a) {
 // row and head, taken while the dO tile is in registers): its own
 // instantiation, the second operand of the dot read by TMA as a side input.
 #define EPI_STORE_DOT 8
+// Added to an epilogue kind in the kernel's template argument: the 16-bit
+// operands and outputs are fp16 instead of bf16.
+#define KIND_F16 16
 template <int KIND>
 struct EpiTraits {
   static constexpr bool SIDE = (KIND == EPI_STORE_RES || KIND == EPI_DGELU || KIND == EPI_STORE_DOT);   // reads a bf16 [M, N] input
@@ -142,11 +147,13 @@ struct TcCfg {
 // tcgen05.mma.cta_group::2 stream issued by the even CTA; each CTA loads its
 // 128 rows of A and half of the tile's B columns, and holds its 128 rows of
 // the accumulator in its own TMEM.
-template <int BN, bool A_MN, bool B_MN, int KIND, int CG>
+template <int BN, bool A_MN, bool B_MN, int KINDF, int CG>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2, int M, int N,
                int K, int splits, EpiParams<bf16> epi, unsigned* err) {
+  constexpr int KIND = KINDF & (KIND_F16 - 1);
+  constexpr bool F16 = (KINDF & KIND_F16) != 0;
   using Cfg = TcCfg<BN, KIND, CG>;
   constexpr int STAGES = Cfg::STAGES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -262,7 +269,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
   } else if (warp == 1 && lane == 0 && rank == 0) {
     // ---------------- MMA issuer (the even CTA of a pair issues for both)
-    constexpr uint32_t IDESC = instr_desc(BN, A_MN, B_MN, TM);
+    constexpr uint32_t IDESC = instr_desc_t(F16, BN, A_MN, B_MN, TM);
     // K-major: SBO = 8 rows x 128 B; k step (16 elements) = 32 B inside the swizzle row.
     // MN-major: LBO = one 64-element box (64 k-rows x 128 B), SBO = 8 k-rows x 128 B; k step = 16 rows.
     constexpr uint32_t A_LBO = A_MN ? 64 * TC_BK * 2 : 16, A_SBO = 1024, A_KSTEP = A_MN ? 16 * 128 : 32;
@@ -404,22 +411,22 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if constexpr (KIND == EPI_STORE || KIND == EPI_STORE_RES) {
           if constexpr (KIND == EPI_STORE_RES) {
             float rr[64];
-            load_row128_bf16(rbase + (sub & 1) * EPI_BUF_BYTES, rl, rr);
+            load_row128_16<F16>(rbase + (sub & 1) * EPI_BUF_BYTES, rl, rr);
 #pragma unroll
             for (int j = 0; j < 64; ++j) v[j] += rr[j];
           }
-          pack_bf16x64(v, w);
+          pack16x64<F16>(v, w);
           stage_row128(b0, rl, w);
         } else if constexpr (KIND == EPI_STORE_DOT) {
           float oo[64];
-          load_row128_bf16(rbase + (sub & 1) * EPI_BUF_BYTES, rl, oo);
+          load_row128_16<F16>(rbase + (sub & 1) * EPI_BUF_BYTES, rl, oo);
           float dot = 0.f;
 #pragma unroll
           for (int j = 0; j < 64; ++j) {
-            v[j] = __bfloat162float(__float2bfloat16_rn(v[j]));
+            v[j] = round16<F16>(v[j]);
             dot += v[j] * oo[j];
           }
-          pack_bf16x64(v, w);
+          pack16x64<F16>(v, w);
           stage_row128(b0, rl, w);
           const int row = m0 + rl;
           if (rows_in && row < M) {
@@ -430,20 +437,20 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           float a[64];
 #pragma unroll
           for (int j = 0; j < 64; ++j) {
-            const float uq = __bfloat162float(__float2bfloat16_rn(v[j]));
+            const float uq = round16<F16>(v[j]);
             v[j] = uq;
             a[j] = gelu_fast(uq);
           }
-          pack_bf16x64(v, w);
+          pack16x64<F16>(v, w);
           stage_row128(b0, rl, w);
-          pack_bf16x64(a, w);
+          pack16x64<F16>(a, w);
           stage_row128(b0 + 2 * EPI_BUF_BYTES, rl, w);
         } else if constexpr (KIND == EPI_DGELU) {
           float uu[64];
-          load_row128_bf16(rbase + (sub & 1) * EPI_BUF_BYTES, rl, uu);
+          load_row128_16<F16>(rbase + (sub & 1) * EPI_BUF_BYTES, rl, uu);
 #pragma unroll
           for (int j = 0; j < 64; ++j) v[j] *= gelu_grad_fast(uu[j]);
-          pack_bf16x64(v, w);
+          pack16x64<F16>(v, w);
           stage_row128(b0, rl, w);
           if (epi.colsum) {   // this warp's 32 rows, summed per column, to shared memory
             const float2 cs = warp_colsum64(v, lane);
@@ -519,12 +526,12 @@ bool gemm_tc_supported(int M, int N, int K, long lda, bool a_t, long ldb, bool b
 
 static int g_sms = 0;
 
-template <int BN, bool A_MN, bool B_MN, int KIND, int CG>
+template <int BN, bool A_MN, bool B_MN, int KINDF, int CG>
 static cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc,
                              const CUtensorMap& tc2, int M, int N, int K, int splits, const EpiParams<bf16>& epi,
                              unsigned* err, cudaStream_t s) {
-  using Cfg = TcCfg<BN, KIND, CG>;
-  auto kern = gemm_tc_kernel<BN, A_MN, B_MN, KIND, CG>;
+  using Cfg = TcCfg<BN, KINDF & (KIND_F16 - 1), CG>;
+  auto kern = gemm_tc_kernel<BN, A_MN, B_MN, KINDF, CG>;
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
@@ -557,33 +564,34 @@ static cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const
 
 // The (layout, epilogue) combinations the training step and the stand-alone
 // GEMM use; any other returns cudaErrorNotSupported.
-template <int BN, bool A_MN, bool B_MN, int CG>
+template <int BN, bool A_MN, bool B_MN, int CG, bool F16>
 static cudaError_t launch_kind(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc,
                                const CUtensorMap& tc2, int M, int N, int K, int splits, const EpiParams<bf16>& epi,
                                unsigned* err, cudaStream_t s) {
-  if (epi.kind == EPI_F32) return launch_tc<BN, A_MN, B_MN, EPI_F32, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+  constexpr int FK = F16 ? KIND_F16 : 0;
+  if (epi.kind == EPI_F32) return launch_tc<BN, A_MN, B_MN, EPI_F32 + FK, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
   if constexpr (!A_MN) {
     if (epi.kind == EPI_STORE && epi.resid)
-      return launch_tc<BN, A_MN, B_MN, EPI_STORE_RES, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+      return launch_tc<BN, A_MN, B_MN, EPI_STORE_RES + FK, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
     if constexpr (B_MN) {
       if (epi.kind == EPI_STORE && epi.rowdot)
-        return launch_tc<BN, A_MN, B_MN, EPI_STORE_DOT, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+        return launch_tc<BN, A_MN, B_MN, EPI_STORE_DOT + FK, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
     }
     if (epi.rowdot) return cudaErrorNotSupported;
     if (epi.kind == EPI_STORE)
-      return launch_tc<BN, A_MN, B_MN, EPI_STORE, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+      return launch_tc<BN, A_MN, B_MN, EPI_STORE + FK, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
     if constexpr (!B_MN) {
       if (epi.kind == EPI_GELU)
-        return launch_tc<BN, A_MN, B_MN, EPI_GELU, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+        return launch_tc<BN, A_MN, B_MN, EPI_GELU + FK, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
     } else {
       if (epi.kind == EPI_DGELU)
-        return launch_tc<BN, A_MN, B_MN, EPI_DGELU, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+        return launch_tc<BN, A_MN, B_MN, EPI_DGELU + FK, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
     }
   } else if constexpr (B_MN) {
     if (epi.kind == EPI_F32_SPLIT)
-      return launch_tc<BN, A_MN, B_MN, EPI_F32_SPLIT, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+      return launch_tc<BN, A_MN, B_MN, EPI_F32_SPLIT + FK, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
     if (epi.kind == EPI_F32_ADD)
-      return launch_tc<BN, A_MN, B_MN, EPI_F32_ADD, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+      return launch_tc<BN, A_MN, B_MN, EPI_F32_ADD + FK, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
   }
   return cudaErrorNotSupported;
 }
@@ -632,10 +640,16 @@ static cudaError_t launch_bn(int M, int N, int K, const bf16* A, long lda, bool 
       ok = false;
   }
   if (!ok) return cudaErrorInvalidValue;
-  if (!a_t && !b_t) return launch_kind<BN, false, false, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
-  if (!a_t && b_t) return launch_kind<BN, false, true, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
-  if (a_t && b_t) return launch_kind<BN, true, true, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
-  return launch_kind<BN, true, false, CG>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+  if (epi.f16) {
+    if (!a_t && !b_t) return launch_kind<BN, false, false, CG, true>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+    if (!a_t && b_t) return launch_kind<BN, false, true, CG, true>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+    if (a_t && b_t) return launch_kind<BN, true, true, CG, true>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+    return launch_kind<BN, true, false, CG, true>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+  }
+  if (!a_t && !b_t) return launch_kind<BN, false, false, CG, false>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+  if (!a_t && b_t) return launch_kind<BN, false, true, CG, false>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+  if (a_t && b_t) return launch_kind<BN, true, true, CG, false>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
+  return launch_kind<BN, true, false, CG, false>(ta, tb, tc, tc2, M, N, K, splits, epi, err, s);
 }
 
 cudaError_t launch_gemm_tc(int M, int N, int K, const bf16* A, long lda, bool a_t, const bf16* B, long ldb,

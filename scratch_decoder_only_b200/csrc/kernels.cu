@@ -31,6 +31,7 @@ __global__ void __launch_bounds__(1024) prep_kernel(const int32_t* __restrict__ 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   unsigned err = 0;
   int nv = 0;
+  unsigned long long pairs = 0;   // keys each query may attend to, summed (packed rows)
   int carry = 0;
   for (int t0 = 0; t0 < T; t0 += blockDim.x) {
     const int t = t0 + threadIdx.x;
@@ -81,6 +82,7 @@ __global__ void __launch_bounds__(1024) prep_kernel(const int32_t* __restrict__ 
       const int ds = seg ? v : 0;
       dstart_out[m] = ds;
       pos_out[m] = t - ds;
+      pairs += (unsigned long long)(t - ds + 1);
     }
     if (threadIdx.x == blockDim.x - 1) carry_s = v;
     __syncthreads();
@@ -96,6 +98,10 @@ __global__ void __launch_bounds__(1024) prep_kernel(const int32_t* __restrict__ 
     for (int w = 0; w < nw; ++w) tot += nv_s[w];
     atomicAdd(&sc->n_valid, tot);   // cleared before the launch
   }
+  if (seg) {
+    for (int o = 16; o > 0; o >>= 1) pairs += __shfl_xor_sync(0xffffffffu, pairs, o);
+    if (lane == 0) atomicAdd(&sc->attn_pairs, pairs);   // cleared before the launch
+  }
 }
 
 cudaError_t launch_prep(const int32_t* tokens, const int32_t* targets, const int32_t* seg, int B, int T,
@@ -103,6 +109,10 @@ cudaError_t launch_prep(const int32_t* tokens, const int32_t* targets, const int
                         DevScalars* sc, cudaStream_t s) {
   if (targets) {
     cudaError_t e = cudaMemsetAsync(&sc->n_valid, 0, sizeof(int), s);
+    if (e != cudaSuccess) return e;
+  }
+  if (seg) {
+    cudaError_t e = cudaMemsetAsync(&sc->attn_pairs, 0, sizeof(unsigned long long), s);
     if (e != cudaSuccess) return e;
   }
   int th = T >= 1024 ? 1024 : ((T + 31) / 32) * 32;
@@ -123,7 +133,7 @@ __global__ void embed_fwd_kernel(const int* __restrict__ tok, const int* __restr
   int lane = threadIdx.x & 31;
   if (row >= M) return;
   const float* a = wte + (long)tok[row] * C;
-  const float* b = wpe + (long)pos[row] * C;
+  const float* b = wpe ? wpe + (long)pos[row] * C : nullptr;
   T* o = x + (long)row * C;
   constexpr int NV = Vec<T>::N;
   for (int c = lane * NV; c < C; c += 32 * NV) {
@@ -131,10 +141,12 @@ __global__ void embed_fwd_kernel(const int* __restrict__ tok, const int* __restr
 #pragma unroll
     for (int i = 0; i < NV; i += 4) {
       Vec<float>::load(a + c + i, va + i);
-      Vec<float>::load(b + c + i, vb + i);
+      if (b) Vec<float>::load(b + c + i, vb + i);
     }
+    if (b) {
 #pragma unroll
-    for (int i = 0; i < NV; ++i) va[i] += vb[i];
+      for (int i = 0; i < NV; ++i) va[i] += vb[i];
+    }
     Vec<T>::store(o + c, va);
   }
 }
@@ -194,7 +206,8 @@ __global__ void __launch_bounds__(256, (NCH * Vec<T>::N <= 24 ? 4 : 2)) ln_fwd_k
     for (int i = 0; i < NCH; ++i)
 #pragma unroll
       for (int j = 0; j < NV; ++j) sum += v[i][j];
-    const float mu = warp_sum(sum) / C;
+    const bool rms = b == nullptr;   // RMSNorm: no mean, no shift
+    const float mu = rms ? 0.f : warp_sum(sum) / C;
     float sq = 0.f;
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
@@ -213,7 +226,7 @@ __global__ void __launch_bounds__(256, (NCH * Vec<T>::N <= 24 ? 4 : 2)) ln_fwd_k
 #pragma unroll
         for (int j = 0; j < NV; j += 4) {
           const float4 gv = __ldg(reinterpret_cast<const float4*>(g + ch * NV + j));
-          const float4 bv = __ldg(reinterpret_cast<const float4*>(b + ch * NV + j));
+          const float4 bv = rms ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldg(reinterpret_cast<const float4*>(b + ch * NV + j));
           o[j] = (v[i][j] - mu) * rs * gv.x + bv.x;
           o[j + 1] = (v[i][j + 1] - mu) * rs * gv.y + bv.y;
           o[j + 2] = (v[i][j + 2] - mu) * rs * gv.z + bv.z;
@@ -405,7 +418,7 @@ template <typename T>
 __global__ void __launch_bounds__(LNB2_THREADS, 2)
 ln_bwd2_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __restrict__ mean,
                const float* __restrict__ rstd, const float* __restrict__ g, const float* dres_in, float* dres_out,
-               T* __restrict__ dres_out_t, float* __restrict__ partials, int M, int C, int TPR, int G) {
+               T* __restrict__ dres_out_t, float* __restrict__ partials, int M, int C, int TPR, int G, int rms) {
   constexpr int NV = Vec<T>::N;
   __shared__ float2 slot[2][LNB2_THREADS / 32];
   const int grp = threadIdx.x / TPR, t = threadIdx.x % TPR;
@@ -473,7 +486,7 @@ ln_bwd2_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* _
       s1 += v.x;
       s2 += v.y;
     }
-    s1 /= C;
+    s1 = rms ? 0.f : s1 / C;   // RMSNorm: no mean term
     s2 /= C;
     if (live) {
       const long off = (long)row * C + col;
@@ -509,7 +522,7 @@ ln_bwd2_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* _
 template <typename T>
 cudaError_t launch_ln_bwd(const T* dy, const T* x, const float* mean, const float* rstd, const float* g,
                           const float* dres_in, float* dres_out, T* dres_out_t, float* partials,
-                          int M, int C, int* nblk_out, cudaStream_t s) {
+                          int M, int C, int* nblk_out, cudaStream_t s, bool rms) {
   constexpr int NV = Vec<T>::N;
   {
     // row-group kernel: C / NV threads per row (whole warps), several rows per block
@@ -528,10 +541,11 @@ cudaError_t launch_ln_bwd(const T* dy, const T* x, const float* mean, const floa
       }
       ++g_kernel_launches;
       ln_bwd2_kernel<T><<<nblk, G * tpr, smem, s>>>(dy, x, mean, rstd, g, dres_in, dres_out, dres_out_t, partials, M,
-                                                    C, tpr, G);
+                                                    C, tpr, G, rms ? 1 : 0);
       return cudaGetLastError();
     }
   }
+  if (rms) return cudaErrorNotSupported;   // the register-row form has no RMSNorm variant
   int nblk = (M + LNB_WARPS - 1) / LNB_WARPS;
   if (nblk > 148 * 3) nblk = 148 * 3;
   *nblk_out = nblk;
@@ -582,13 +596,14 @@ __global__ void __launch_bounds__(256) reduce_segs_kernel(RedSegList L) {
     float acc = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) acc += red[w][threadIdx.x];
-    if (n < sg.cols) sg.dst[n] = acc;
+    if (n < sg.cols) sg.dst[n] = L.add ? sg.dst[n] + acc : acc;
   }
 }
 
-cudaError_t launch_reduce_segs(const RedSeg* segs, int n, cudaStream_t s) {
+cudaError_t launch_reduce_segs(const RedSeg* segs, int n, bool add, cudaStream_t s) {
   for (int i0 = 0; i0 < n; i0 += RED_MAX_SEGS) {
     RedSegList L;
+    L.add = add ? 1 : 0;
     L.n = n - i0 < RED_MAX_SEGS ? n - i0 : RED_MAX_SEGS;
     int blk = 0;
     for (int i = 0; i < L.n; ++i) {
@@ -642,12 +657,13 @@ __global__ void __launch_bounds__(256) colsum_kernel(const Tin* __restrict__ x, 
   }
 }
 
-// bf16 column sums with 16-byte loads: a block covers 256 columns (32 lanes
+// 16-bit (bf16 or fp16) column sums with 16-byte loads: a block covers 256 columns (32 lanes
 // x 8 columns) and CS2_ROWS rows split over 8 warps, four rows in flight per
 // thread; one partial row per block row-chunk.
 #define CS2_ROWS 256
-__global__ void __launch_bounds__(256) colsum_bf16_kernel(const bf16* __restrict__ x, long ldx, int M, int N,
-                                                         float* __restrict__ partials) {
+template <typename T16>
+__global__ void __launch_bounds__(256) colsum16_kernel(const T16* __restrict__ x, long ldx, int M, int N,
+                                                       float* __restrict__ partials) {
   __shared__ float red[8][257];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c0 = blockIdx.x * 256 + lane * 8;
@@ -664,14 +680,14 @@ __global__ void __launch_bounds__(256) colsum_bf16_kernel(const bf16* __restrict
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         float v[8];
-        Vec<bf16>::load(reinterpret_cast<const bf16*>(&w[u]), v);
+        Vec<T16>::load(reinterpret_cast<const T16*>(&w[u]), v);
 #pragma unroll
         for (int j = 0; j < 8; ++j) a[j] += v[j];
       }
     }
     for (; r < re; r += 8) {
       float v[8];
-      Vec<bf16>::load(x + (long)r * ldx + c0, v);
+      Vec<T16>::load(x + (long)r * ldx + c0, v);
 #pragma unroll
       for (int j = 0; j < 8; ++j) a[j] += v[j];
     }
@@ -693,7 +709,7 @@ cudaError_t launch_colsum(const Tin* x, long ldx, int M, int N, float* partials,
       dim3 g2((N + 255) / 256, (M + CS2_ROWS - 1) / CS2_ROWS);
       *rows_out = (int)g2.y;
       ++g_kernel_launches;
-      colsum_bf16_kernel<<<g2, 256, 0, s>>>(reinterpret_cast<const bf16*>(x), ldx, M, N, partials);
+      colsum16_kernel<Tin><<<g2, 256, 0, s>>>(x, ldx, M, N, partials);
       return cudaGetLastError();
     }
   }
@@ -707,7 +723,7 @@ cudaError_t launch_colsum(const Tin* x, long ldx, int M, int N, float* partials,
 // ---------------------------------------------------------------------------
 // Fused softmax cross-entropy and its gradient, in place over the logits.
 // Per row: lse over the real vocabulary 0..V-1 (online max / sum), loss =
-// lse - z[target]; then dz = (softmax - onehot) * loss_scale / N_valid for
+// lse - z[target]; then dz = (softmax - onehot) * loss_scale * loss_weight / N_valid for
 // c < V, 0 for the padded columns and for ignored rows.  No fp32
 // probability tensor is written.  ("RustGPT", "Technical implementation":
 // cross-entropy loss.)
@@ -759,7 +775,7 @@ xent_kernel(T* __restrict__ logits, long ldl, const int* __restrict__ tgt, int V
   float lse = s_lse;
   if (threadIdx.x == 0) rowloss[row] = tg >= 0 ? lse - s_ztg : 0.f;
   int nv = sc->n_valid;
-  float scale = tg >= 0 ? sc->loss_scale / (float)(nv > 0 ? nv : 1) : 0.f;
+  float scale = tg >= 0 ? sc->loss_scale * sc->loss_weight / (float)(nv > 0 ? nv : 1) : 0.f;
   int nvp = Vp / NV;
   for (int i = threadIdx.x; i < nvp; i += XENT_THREADS) {
     float v[NV];
@@ -836,7 +852,7 @@ xent_smem_kernel(T* __restrict__ logits, long ldl, const int* __restrict__ tgt, 
   ssum = block_reduce(ssum, false, red);
   if (threadIdx.x == 0) rowloss[row] = tg >= 0 ? m + logf(ssum) - zt : 0.f;
   const int nv = sc->n_valid;
-  const float scale = tg >= 0 ? sc->loss_scale / (float)(nv > 0 ? nv : 1) : 0.f;
+  const float scale = tg >= 0 ? sc->loss_scale * sc->loss_weight / (float)(nv > 0 ? nv : 1) : 0.f;
   const float inv = scale / ssum;
   for (int i = threadIdx.x; i < nvec; i += XENT_THREADS) {
     float v[NV];
@@ -850,20 +866,21 @@ xent_smem_kernel(T* __restrict__ logits, long ldl, const int* __restrict__ tgt, 
   }
 }
 
-// bf16 logits: the row moves between HBM and shared memory as one bulk copy
+// 16-bit logits: the row moves between HBM and shared memory as one bulk copy
 // each way (the copy engine keeps the whole row in flight); the three passes
 // over it (max, exp and sum, scale) run on shared memory.  exp(z - max) is
-// kept in place as bf16 and summed in fp32.
+// kept in place as 16-bit values and summed in fp32.
 #define XB_THREADS 512
+template <typename T16>
 __global__ void __launch_bounds__(XB_THREADS, 2)
-xent_bulk_kernel(bf16* __restrict__ logits, long ldl, const int* __restrict__ tgt, int V, int Vp,
+xent_bulk_kernel(T16* __restrict__ logits, long ldl, const int* __restrict__ tgt, int V, int Vp,
                  float* __restrict__ rowloss, DevScalars* __restrict__ sc) {
   extern __shared__ __align__(128) uint8_t xb_raw[];
   __shared__ float red[33];
   __shared__ __align__(8) uint64_t bar;
-  bf16* zs = reinterpret_cast<bf16*>(xb_raw);
+  T16* zs = reinterpret_cast<T16*>(xb_raw);
   const int row = blockIdx.x;
-  bf16* z = logits + (long)row * ldl;
+  T16* z = logits + (long)row * ldl;
   const int tg = tgt[row];
   const int nvec = Vp / 8;
   const uint32_t bytes = (uint32_t)nvec * 16;
@@ -886,7 +903,7 @@ xent_bulk_kernel(bf16* __restrict__ logits, long ldl, const int* __restrict__ tg
   for (int i = threadIdx.x; i < nvec; i += XB_THREADS) {
     float v[8];
     const uint4 w = zv[i];
-    Vec<bf16>::load(reinterpret_cast<const bf16*>(&w), v);
+    Vec<T16>::load(reinterpret_cast<const T16*>(&w), v);
 #pragma unroll
     for (int j = 0; j < 8; ++j)
       if (i * 8 + j < V) m = fmaxf(m, v[j]);
@@ -899,7 +916,7 @@ xent_bulk_kernel(bf16* __restrict__ logits, long ldl, const int* __restrict__ tg
   for (int i = threadIdx.x; i < nvec; i += XB_THREADS) {
     float v[8];
     uint4 w = zv[i];
-    Vec<bf16>::load(reinterpret_cast<const bf16*>(&w), v);
+    Vec<T16>::load(reinterpret_cast<const T16*>(&w), v);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       float e;
@@ -907,21 +924,21 @@ xent_bulk_kernel(bf16* __restrict__ logits, long ldl, const int* __restrict__ tg
       v[j] = i * 8 + j < V ? e : 0.f;
       ssum += v[j];
     }
-    Vec<bf16>::store(reinterpret_cast<bf16*>(&w), v);
+    Vec<T16>::store(reinterpret_cast<T16*>(&w), v);
     reinterpret_cast<uint4*>(zs)[i] = w;
   }
   ssum = block_reduce(ssum, false, red);
   if (threadIdx.x == 0) rowloss[row] = tg >= 0 ? m + logf(ssum) - zt : 0.f;
   const int nv = sc->n_valid;
-  const float scale = tg >= 0 ? sc->loss_scale / (float)(nv > 0 ? nv : 1) : 0.f;
+  const float scale = tg >= 0 ? sc->loss_scale * sc->loss_weight / (float)(nv > 0 ? nv : 1) : 0.f;
   const float inv = scale / ssum;
   for (int i = threadIdx.x; i < nvec; i += XB_THREADS) {
     float v[8];
     uint4 w = zv[i];
-    Vec<bf16>::load(reinterpret_cast<const bf16*>(&w), v);
+    Vec<T16>::load(reinterpret_cast<const T16*>(&w), v);
 #pragma unroll
     for (int j = 0; j < 8; ++j) v[j] = v[j] * inv - (i * 8 + j == tg ? scale : 0.f);
-    Vec<bf16>::store(reinterpret_cast<bf16*>(&w), v);
+    Vec<T16>::store(reinterpret_cast<T16*>(&w), v);
     reinterpret_cast<uint4*>(zs)[i] = w;
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -945,12 +962,12 @@ cudaError_t launch_xent(T* logits, long ldl, const int* tgt, int M, int V, int V
     if (Vp % 8 == 0 && ldl % 8 == 0 && bytes <= 110 * 1024) {
       static size_t attr = 0;
       if (bytes > attr) {
-        cudaError_t e = cudaFuncSetAttribute(xent_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        cudaError_t e = cudaFuncSetAttribute(xent_bulk_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
         if (e != cudaSuccess) return e;
         attr = bytes;
       }
       ++g_kernel_launches;
-      xent_bulk_kernel<<<M, XB_THREADS, bytes, s>>>(logits, ldl, tgt, V, Vp, rowloss, sc);
+      xent_bulk_kernel<T><<<M, XB_THREADS, bytes, s>>>(logits, ldl, tgt, V, Vp, rowloss, sc);
       return cudaGetLastError();
     }
   }
@@ -1009,12 +1026,15 @@ __global__ void embed_bwd_kernel(const float* __restrict__ dres, const int* __re
   if (row >= M) return;
   const float* d = dres + (long)row * C;
   float* a = gwte + (long)tok[row] * C;
-  float* b = gwpe + (long)pos[row] * C;
+  float* b = gwpe ? gwpe + (long)pos[row] * C : nullptr;
   for (int c = lane * 4; c < C; c += 128) {
     float v[4];
     Vec<float>::load(d + c, v);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) { atomicAdd(a + c + j, v[j]); atomicAdd(b + c + j, v[j]); }
+    for (int j = 0; j < 4; ++j) {
+      atomicAdd(a + c + j, v[j]);
+      if (b) atomicAdd(b + c + j, v[j]);
+    }
   }
 }
 
@@ -1030,7 +1050,7 @@ cudaError_t launch_embed_bwd(const float* dres, const int* tok, const int* pos, 
 // Global L2 norm, clip, dynamic loss scale and AdamW over the flat fp32
 // parameter vector (one tensor: the canonical layout is contiguous).
 // ---------------------------------------------------------------------------
-__global__ void sumsq_kernel(const float* __restrict__ g, size_t n, double* __restrict__ partials) {
+__device__ __forceinline__ void sumsq_block(const float* __restrict__ g, size_t n, double* __restrict__ partials) {
   float acc = 0.f;
   size_t n4 = n / 4;
   const float4* g4 = reinterpret_cast<const float4*>(g);
@@ -1051,6 +1071,9 @@ __global__ void sumsq_kernel(const float* __restrict__ g, size_t n, double* __re
     partials[blockIdx.x] = t;
   }
 }
+__global__ void sumsq_kernel(const float* __restrict__ g, size_t n, double* __restrict__ partials) {
+  sumsq_block(g, n, partials);
+}
 
 cudaError_t launch_sumsq(const float* g, size_t n, double* partials, int nblk, cudaStream_t s) {
   ++g_kernel_launches;
@@ -1058,11 +1081,26 @@ cudaError_t launch_sumsq(const float* g, size_t n, double* partials, int nblk, c
   return cudaGetLastError();
 }
 
-__global__ void opt_finalize_kernel(const double* __restrict__ partials, int nblk, float clip, float beta1,
-                                    float beta2, DevScalars* sc, float* norm_out, int32_t* skipped_out) {
+// Learning rate of AdamW step s (0-based count of steps taken before it)
+// under the schedule in sc (cosine with linear warm-up and a floor).
+__device__ double sched_lr(const DevScalars* sc, int s, double lr_const) {
+  if (sc->sched_kind != 1) return lr_const;
+  const double mx = sc->sched_max_lr, mn = sc->sched_min_lr;
+  if (s < sc->sched_warmup) return mx * (double)(s + 1) / (double)sc->sched_warmup;
+  if (s >= sc->sched_total) return mn;
+  const double r = (double)(s - sc->sched_warmup) / (double)(sc->sched_total - sc->sched_warmup);
+  return mn + 0.5 * (mx - mn) * (1.0 + cos(3.14159265358979323846 * r));
+}
+
+// One block: the global norm from the per-block partials, the clip
+// coefficient, the skip decision, the loss-scale update and the bias
+// corrections, all into sc (thread 0 writes).
+__device__ __forceinline__ void opt_finalize_block(const double* partials, int nblk, float clip, float beta1,
+                                                   float beta2, float lr, DevScalars* sc, float* norm_out,
+                                                   int32_t* skipped_out) {
   __shared__ double red[32];
   double acc = 0.0;
-  for (int i = threadIdx.x; i < nblk; i += blockDim.x) acc += partials[i];
+  for (int i = threadIdx.x; i < nblk; i += blockDim.x) acc += __ldcg(partials + i);
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
   __syncthreads();
@@ -1082,6 +1120,7 @@ __global__ void opt_finalize_kernel(const double* __restrict__ partials, int nbl
     double coef = (double)clip / (norm + 1e-6);
     if (coef > 1.0) coef = 1.0;
     sc->coef = (float)(coef * inv);
+    sc->lr = (float)sched_lr(sc, sc->step, (double)lr);
     int t = sc->step + 1;
     sc->step = t;
     sc->bc1 = (float)(1.0 - pow((double)beta1, (double)t));
@@ -1094,24 +1133,31 @@ __global__ void opt_finalize_kernel(const double* __restrict__ partials, int nbl
   if (norm_out) *norm_out = (float)norm;
   if (skipped_out) *skipped_out = sc->skipped;
 }
+__global__ void opt_finalize_kernel(const double* __restrict__ partials, int nblk, float clip, float beta1,
+                                    float beta2, float lr, DevScalars* sc, float* norm_out, int32_t* skipped_out) {
+  opt_finalize_block(partials, nblk, clip, beta1, beta2, lr, sc, norm_out, skipped_out);
+}
 
-cudaError_t launch_opt_finalize(const double* partials, int nblk, float clip, float beta1, float beta2,
+cudaError_t launch_opt_finalize(const double* partials, int nblk, float clip, float beta1, float beta2, float lr,
                                 DevScalars* sc, float* norm_out, int32_t* skipped_out, cudaStream_t s) {
   ++g_kernel_launches;
-  opt_finalize_kernel<<<1, 1024, 0, s>>>(partials, nblk, clip, beta1, beta2, sc, norm_out, skipped_out);
+  opt_finalize_kernel<<<1, 1024, 0, s>>>(partials, nblk, clip, beta1, beta2, lr, sc, norm_out, skipped_out);
   return cudaGetLastError();
 }
 
 // AdamW ("Feste", "Manual Backpropagation from scratch": decoupled weight
-// decay) on the clipped, unscaled gradient g * coef:
+// decay) on the clipped, unscaled gradient g * coef, with lr = sc->lr:
 //   m = b1 m + (1-b1) g;  v = b2 v + (1-b2) g^2;
 //   p -= lr (m / bc1 / (sqrt(v / bc2) + eps) + wd p);  pw = T(p).
 template <typename T>
-__global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g, float* __restrict__ m,
-                             float* __restrict__ v, T* __restrict__ pw, size_t n, float lr, float beta1,
-                             float beta2, float eps, float wd, const DevScalars* __restrict__ sc) {
-  if (sc->skipped) return;
-  float coef = sc->coef, bc1 = sc->bc1, bc2 = sc->bc2;
+__device__ __forceinline__ void adamw_body(float* __restrict__ p, const float* __restrict__ g, float* __restrict__ m,
+                                           float* __restrict__ v, T* __restrict__ pw, size_t n, float beta1,
+                                           float beta2, float eps, float wd, const DevScalars* sc) {
+  // the scalars are read from L2: in the fused form another block wrote them
+  // in this kernel
+  if (__ldcg(&sc->skipped)) return;
+  const float lr = __ldcg(&sc->lr);
+  float coef = __ldcg(&sc->coef), bc1 = __ldcg(&sc->bc1), bc2 = __ldcg(&sc->bc2);
   float ib1 = 1.0f / bc1, ib2 = 1.0f / bc2;
   size_t n4 = n / 4;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
@@ -1149,11 +1195,92 @@ __global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g,
 }
 
 template <typename T>
-cudaError_t launch_adamw(float* p, const float* g, float* m, float* v, T* pw, size_t n, float lr,
+__global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g, float* __restrict__ m,
+                             float* __restrict__ v, T* __restrict__ pw, size_t n, float beta1,
+                             float beta2, float eps, float wd, const DevScalars* __restrict__ sc) {
+  adamw_body<T>(p, g, m, v, pw, n, beta1, beta2, eps, wd, sc);
+}
+
+// The whole optimiser step in one cooperative launch ("a single multi-tensor
+// kernel"): every block sums the squares of its share of the gradient (fp64
+// partials), a grid barrier, block 0 finalises the norm / clip / skip /
+// loss-scale / bias corrections, a second barrier, and every block updates
+// its share of p, m, v and the 16-bit copy.  The barriers count on
+// sc->opt_bar (zeroed before the launch) and give up after about a second,
+// setting GPT_DEVERR_TIMEOUT (no update then happens).
+__device__ __forceinline__ bool opt_grid_sync(DevScalars* sc, unsigned k) {
+  __shared__ int s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    __threadfence();
+    atomicAdd(&sc->opt_bar, 1u);
+    const unsigned target = k * gridDim.x;
+    const long long t0 = clock64();
+    while (true) {
+      unsigned v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(&sc->opt_bar) : "memory");
+      if (v >= target) break;
+      if (*(volatile unsigned*)&sc->opt_abort) { ok = 0; break; }
+      if (clock64() - t0 > (1ll << 31)) {
+        atomicOr(&sc->err, GPT_DEVERR_TIMEOUT);
+        atomicExch(&sc->opt_abort, 1u);
+        ok = 0;
+        break;
+      }
+    }
+    __threadfence();
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(512) clip_adamw_fused_kernel(float* __restrict__ p, const float* __restrict__ g,
+                                                              float* __restrict__ m, float* __restrict__ v,
+                                                              T* __restrict__ pw, size_t n, double* partials,
+                                                              float clip, float beta1, float beta2, float eps,
+                                                              float wd, float lr, DevScalars* sc, float* norm_out,
+                                                              int32_t* skipped_out) {
+  sumsq_block(g, n, partials);
+  if (!opt_grid_sync(sc, 1)) return;
+  if (blockIdx.x == 0) opt_finalize_block(partials, gridDim.x, clip, beta1, beta2, lr, sc, norm_out, skipped_out);
+  if (!opt_grid_sync(sc, 2)) return;
+  adamw_body<T>(p, g, m, v, pw, n, beta1, beta2, eps, wd, sc);
+}
+
+template <typename T>
+cudaError_t launch_clip_adamw_fused(float* p, const float* g, float* m, float* v, T* pw, size_t n, double* partials,
+                                    int max_blocks, float clip, float beta1, float beta2, float eps, float wd,
+                                    float lr, DevScalars* sc, float* norm_out, int32_t* skipped_out,
+                                    cudaStream_t s) {
+  static int grid = 0;
+  if (!grid) {
+    int dev = 0, sms = 0, per = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, clip_adamw_fused_kernel<T>, 512, 0);
+    if (e != cudaSuccess) return e;
+    if (per > 4) per = 4;
+    grid = sms * per;
+  }
+  const int G = grid < max_blocks ? grid : max_blocks;
+  if (G < 1) return cudaErrorNotSupported;
+  cudaError_t e = cudaMemsetAsync(&sc->opt_bar, 0, 2 * sizeof(unsigned), s);
+  if (e != cudaSuccess) return e;
+  void* args[] = {&p, (void*)&g, &m, &v, &pw, &n, &partials, &clip, &beta1, &beta2, &eps, &wd, &lr, &sc, &norm_out,
+                  &skipped_out};
+  ++g_kernel_launches;
+  return cudaLaunchCooperativeKernel((void*)clip_adamw_fused_kernel<T>, dim3(G), dim3(512), args, 0, s);
+}
+
+template <typename T>
+cudaError_t launch_adamw(float* p, const float* g, float* m, float* v, T* pw, size_t n,
                          float beta1, float beta2, float eps, float wd, const DevScalars* sc,
                          cudaStream_t s) {
   ++g_kernel_launches;
-  adamw_kernel<T><<<148 * 8, 256, 0, s>>>(p, g, m, v, pw, n, lr, beta1, beta2, eps, wd, sc);
+  adamw_kernel<T><<<148 * 8, 256, 0, s>>>(p, g, m, v, pw, n, beta1, beta2, eps, wd, sc);
   return cudaGetLastError();
 }
 
@@ -1216,14 +1343,19 @@ cudaError_t launch_wait_timeout_probe(unsigned* err, long long timeout_cycles, c
   template cudaError_t launch_ln_fwd<T>(const T*, const float*, const float*, T*, float*, float*, int, int, \
                                         float, cudaStream_t);                                            \
   template cudaError_t launch_ln_bwd<T>(const T*, const T*, const float*, const float*, const float*,      \
-                                        const float*, float*, T*, float*, int, int, int*, cudaStream_t);  \
+                                        const float*, float*, T*, float*, int, int, int*, cudaStream_t,   \
+                                        bool);                                                           \
   template cudaError_t launch_colsum<T>(const T*, long, int, int, float*, int*, cudaStream_t);            \
   template cudaError_t launch_xent<T>(T*, long, const int*, int, int, int, float*, DevScalars*, cudaStream_t); \
   template cudaError_t launch_embed_bwd<T>(const float*, const int*, const int*, float*, float*, int, int,  \
                                            cudaStream_t);                                                \
   template cudaError_t launch_adamw<T>(float*, const float*, float*, float*, T*, size_t, float, float,     \
-                                       float, float, float, const DevScalars*, cudaStream_t);            \
+                                       float, float, const DevScalars*, cudaStream_t);                   \
   template cudaError_t launch_cast<T>(const float*, T*, size_t, cudaStream_t);                            \
+  template cudaError_t launch_clip_adamw_fused<T>(float*, const float*, float*, float*, T*, size_t, double*, int, \
+                                                  float, float, float, float, float, float, DevScalars*, float*, \
+                                                  int32_t*, cudaStream_t);                               \
   template cudaError_t launch_to_f32<T>(const T*, long, int, int, float*, cudaStream_t);
 INST(float)
 INST(bf16)
+INST(f16)

@@ -25,24 +25,36 @@ struct DevScalars {
   int loss_scaling;   // 1: dynamic scale on
   unsigned err;       // sticky device error word
   int dec_step;       // decode step counter
+  unsigned dec_bar;   // grid-barrier counter of the fused decode kernel (zeroed per launch)
+  unsigned dec_abort; // its abort word (zeroed per launch)
+  unsigned long long attn_pairs;   // allowed (query, key) pairs of the latest packed forward
+  float lr;           // learning rate of the latest taken step (set by the finalize kernel)
+  float loss_weight;  // multiplies the loss gradient of later forwards (micro-batch weight)
+  int sched_kind;     // GPT_LR_CONSTANT / GPT_LR_COSINE
+  int sched_warmup, sched_total;
+  float sched_max_lr, sched_min_lr;
+  unsigned opt_bar, opt_abort;   // grid barrier of the fused optimiser step (zeroed per launch)
 };
 
 // ---- kernels.cu: embedding, LayerNorm, cross-entropy, reductions, optimiser
 cudaError_t launch_prep(const int32_t* tokens, const int32_t* targets, const int32_t* seg, int B, int T,
                         int V, int* tok_out, int* tgt_out, int* pos_out, int* dstart_out,
                         DevScalars* sc, cudaStream_t s);
+// wpe may be null (no position table)
 template <typename T>
 cudaError_t launch_embed_fwd(const int* tok, const int* pos, const float* wte, const float* wpe, T* x,
                              int M, int C, cudaStream_t s);
+// b == nullptr: RMSNorm (no mean subtracted, no shift; mean is written as 0)
 template <typename T>
 cudaError_t launch_ln_fwd(const T* x, const float* g, const float* b, T* y, float* mean, float* rstd,
                           int M, int C, float eps, cudaStream_t s);
 // partials: [nblk][3C] = dg | db | column sums of dres_out (the bias gradient of
 // the layer whose output gradient dres_out is)
+// rms: the RMSNorm backward (no mean term; the db partials are then unused)
 template <typename T>
 cudaError_t launch_ln_bwd(const T* dy, const T* x, const float* mean, const float* rstd, const float* g,
                           const float* dres_in, float* dres_out, T* dres_out_t, float* partials,
-                          int M, int C, int* nblk_out, cudaStream_t s);
+                          int M, int C, int* nblk_out, cudaStream_t s, bool rms = false);
 // Deferred column reductions: for each segment, dst[n] = sum_r src[r * ld + n]
 // (n < cols, r < rows, fixed summation order).  Segments are launched in
 // lists of RED_MAX_SEGS (the list travels as the kernel parameter).
@@ -54,9 +66,10 @@ struct RedSeg {
 #define RED_MAX_SEGS 96
 struct RedSegList {
   int n;
+  int add;   // 1: dst[n] += sum (gradient accumulation), 0: dst[n] = sum
   RedSeg seg[RED_MAX_SEGS];
 };
-cudaError_t launch_reduce_segs(const RedSeg* segs, int n, cudaStream_t s);
+cudaError_t launch_reduce_segs(const RedSeg* segs, int n, bool add, cudaStream_t s);
 // Column sums of x [M, N] as partial rows: partials[r][0..N), *rows_out rows
 // (at most (M + 127) / 128), to be summed by a reduction segment.
 template <typename Tin>
@@ -69,12 +82,19 @@ template <typename T>
 cudaError_t launch_embed_bwd(const float* dres, const int* tok, const int* pos, float* gwte, float* gwpe,
                              int M, int C, cudaStream_t s);
 cudaError_t launch_sumsq(const float* g, size_t n, double* partials, int nblk, cudaStream_t s);
-cudaError_t launch_opt_finalize(const double* partials, int nblk, float clip, float beta1, float beta2,
+// also sets sc->lr: the schedule's value at the step counter, or `lr`
+cudaError_t launch_opt_finalize(const double* partials, int nblk, float clip, float beta1, float beta2, float lr,
                                 DevScalars* sc, float* norm_out, int32_t* skipped_out, cudaStream_t s);
 template <typename T>
-cudaError_t launch_adamw(float* p, const float* g, float* m, float* v, T* pw, size_t n, float lr,
+cudaError_t launch_adamw(float* p, const float* g, float* m, float* v, T* pw, size_t n,
                          float beta1, float beta2, float eps, float wd, const DevScalars* sc,
                          cudaStream_t s);
+// norm, clip, skip / loss scale and AdamW in one cooperative launch (at most
+// max_blocks blocks: partials holds one double per block)
+template <typename T>
+cudaError_t launch_clip_adamw_fused(float* p, const float* g, float* m, float* v, T* pw, size_t n, double* partials,
+                                    int max_blocks, float clip, float beta1, float beta2, float eps, float wd,
+                                    float lr, DevScalars* sc, float* norm_out, int32_t* skipped_out, cudaStream_t s);
 template <typename T>
 cudaError_t launch_cast(const float* src, T* dst, size_t n, cudaStream_t s);
 template <typename T>
@@ -108,31 +128,119 @@ cudaError_t launch_attn_bwd_mma(const bf16* qkv, const bf16* out, const bf16* do
 
 // ---- attention_tc.cu: head size 64 on tcgen05 (dq_acc: fp32 [B*T, C] scratch)
 bool attn_tc_supported(int d);
+// Column layout of the fused q/k/v rows and of the key / value gradients.
+// One key / value head per query head: qkv rows [q | k | v] of C each.
+// Grouped heads (G query heads per key / value head): qkv rows of width qw
+// hold the H query heads at 0, the Hkv key heads at kcol and the Hkv value
+// heads at vcol; query head h reads key / value head h / G.  The backward
+// writes one key and one value gradient per query head: at dkv + row * ld_kv
+// + h d (keys) and + v_off + h d (values); grouped heads send them to a
+// scratch [rows, 2C] that a reduction sums into the shared heads.
+struct AttnLayout {
+  int qw, kcol, vcol, G;
+  bf16* dkv;
+  long ld_kv;
+  int v_off;
+};
+AttnLayout attn_layout_mha(bf16* dqkv, int C);
+// f16: the 16-bit tensors hold fp16 values (same layouts; bf16 otherwise);
+// lay: null for one key / value head per query head
 cudaError_t launch_attn_fwd_tc(const bf16* qkv, bf16* out, float* lse, const int* dstart, int B, int T, int H,
-                               unsigned* err, cudaStream_t s);
+                               unsigned* err, cudaStream_t s, bool f16 = false, const AttnLayout* lay = nullptr);
 // d_ready: Dbuf [B, H, T] already holds rowsum(dO o O) (written by the GEMM
 // epilogue that produced dO); otherwise a row-dot kernel computes it first
 cudaError_t launch_attn_bwd_tc(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* Dbuf,
                                bool d_ready, float* dq_acc, const int* dstart, bf16* dqkv, int B, int T, int H,
-                               unsigned* err, cudaStream_t s);
+                               unsigned* err, cudaStream_t s, bool f16 = false, const AttnLayout* lay = nullptr);
 
 // ---- decode.cu
 // decode kernels read the position as pos0 + *step (device counter)
+// wpe may be null (no position table)
 template <typename T>
 cudaError_t launch_dec_embed(const int* tok, const float* wte, const float* wpe, T* x, int B, int C, int pos0,
                              const int* step, int max_seq, unsigned* err, cudaStream_t s);
 template <typename T>
 cudaError_t launch_gemv(const T* X, int B, int K, const T* W, int N, const float* bias, const T* resid,
                         int mode, T* out, T* out2, float* outf, cudaStream_t s);
+// q|k|v row layout of a decode step: rows of width qw, query heads at 0, Hkv
+// key heads at kcol, Hkv value heads at vcol; the cache holds Hkv heads
+// ([B][Hkv][Tmax][d] per layer).  One key/value head per query head:
+// {3C, C, 2C, H}.
+struct DecLayout {
+  int qw, kcol, vcol, Hkv;
+};
 template <typename T>
-cudaError_t launch_kv_fill(const T* qkv, T* kc, T* vc, int B, int Tp, int H, int d, int Tmax, cudaStream_t s);
+cudaError_t launch_kv_fill(const T* qkv, T* kc, T* vc, int B, int Tp, int d, int Tmax, const DecLayout& L,
+                           cudaStream_t s);
 size_t dec_attn_part_floats(int B, int H, int d);
 template <typename T>
 cudaError_t launch_dec_attn(const T* qkv, T* kc, T* vc, T* out, float* part, int B, int H, int d, int Tmax, int pos0,
-                            const int* step, cudaStream_t s);
+                            const int* step, const DecLayout& L, cudaStream_t s);
 // out[b * out_ld + (*step or 0)] = argmax; tok[b] = argmax
 cudaError_t launch_argmax(const float* logits, int B, int V, int Vp, int* tok, int32_t* out, int out_ld,
                           const int* step, cudaStream_t s);
 cudaError_t launch_step_advance(int* step, cudaStream_t s);
+// sampled choice (temperature, top-k, top-p; temp <= 0: greedy) with the
+// uniform uni[b * u_ld + (*step or 0)]; writes tok[b] and out[b * out_ld + col].
+// Needs V * 4 bytes of shared memory (at most SMP_MAX_VOCAB tokens).
+#define SMP_MAX_VOCAB 55000
+cudaError_t launch_sample(const float* logits, int B, int V, int Vp, float temp, int top_k, float top_p,
+                          const float* uni, int u_ld, int* tok, int32_t* out, int out_ld, const int* step,
+                          cudaStream_t s);
 template <typename T>
 cudaError_t launch_gather_last(const T* x, int B, int Tp, int C, T* out, cudaStream_t s);
+
+// ---- llama.cu: the Llama-style block's elementwise kernels (16-bit T)
+// rotary positions in place on nq query heads at columns [0, nq d) and nk key
+// heads at [kcol, kcol + nk d) of rows of stride ld; position pos[r] (or
+// pos0 + *step when pos is null); tab: [max_seq][d/2] (cos, sin)
+template <typename T>
+cudaError_t launch_rope(T* x, long ld, int rows, int nq, int kcol, int nk, int d, const int* pos, int pos0,
+                        const int* step, const float2* tab, int max_seq, bool inverse, cudaStream_t s);
+// a [rows, F] = silu(gate) * up of gu [rows, 2F] = [gate | up]
+template <typename T>
+cudaError_t launch_swiglu(const T* gu, T* a, int rows, int F, cudaStream_t s);
+// dgu [rows, 2F] = [da * up * silu'(gate) | da * silu(gate)]
+template <typename T>
+cudaError_t launch_swiglu_bwd(const T* da, const T* gu, T* dgu, int rows, int F, cudaStream_t s);
+// per-query-head key / value gradients kvq [rows, 2 H d] summed into the
+// Hkv shared heads of dkv (row stride ld; keys at kcol, values at vcol)
+template <typename T>
+cudaError_t launch_gqa_reduce(const T* kvq, T* dkv, long ld, int kcol, int vcol, int rows, int Hkv, int G, int d,
+                              cudaStream_t s);
+
+// ---- decode_fused.cu: every remaining greedy step of a small batch in one
+// persistent kernel (bf16 weights; B <= 4)
+#define DF_MAX_GRID 256   // am_v / am_i hold [B][DF_MAX_GRID]
+struct DecFusedParams {
+  const bf16* pw;          // bf16 working copy of the parameters
+  const float* p32;        // fp32 master parameters (embeddings, LN, biases)
+  long o_wte, o_wpe, o_lnf_g, o_lnf_b, o_head;
+  // offsets of layer 0 and the stride between layers (canonical layout)
+  long l_ln1_g, l_ln1_b, l_w_qkv, l_b_qkv, l_w_o, l_b_o, l_ln2_g, l_ln2_b, l_w_fc, l_b_fc, l_w_fc2, l_b_fc2;
+  long l_stride;
+  int NL, C, H, D, F, V, Vp, Tmax;
+  float eps;
+  bf16* kc;                // [NL][Bmax][H][Tmax][D]
+  bf16* vc;
+  long kvl;                // elements per layer of the cache
+  int B, pos_first, n_steps, S;
+  int* tok;                // [B] current token (in: the prefill's choice)
+  int32_t* out;            // [B][out_ld], columns out_col0 .. out_col0 + n_steps - 1
+  int out_ld, out_col0;
+  bf16* qkv;               // [B][3C]
+  float* part;             // [B*H][S][D+2] attention partials
+  int* cnt;                // [B*H] splits finished per (row, head) (zero at launch)
+  bf16* att;               // [B][C] merged attention output
+  bf16* xmid;              // [B][C]
+  bf16* abuf;              // [B][F]
+  bf16* xbuf;              // [B][C]
+  float* logits;           // [B][Vp]
+  float* am_v;             // [B][grid] per-CTA maxima
+  int* am_i;
+  unsigned* bar;           // grid barrier counter (zero at launch)
+  unsigned* abortf;        // abort word (zero at launch)
+  unsigned* err;           // sticky device error word
+};
+bool dec_fused_supported(int B, int C, int H, int F, int Vp);
+cudaError_t launch_decode_fused(const DecFusedParams& prm, cudaStream_t s);

@@ -178,6 +178,31 @@ __host__ __device__ constexpr uint32_t instr_desc(int bn, bool a_mn, bool b_mn, 
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
          ((uint32_t)(bn >> 3) << 17) | ((uint32_t)(bm >> 4) << 24);
 }
+// The same with A and B in fp16 (their format fields 0): in one kind::f16
+// MMA both operands have the same type.
+__host__ __device__ constexpr uint32_t instr_desc_t(bool f16, int bn, bool a_mn, bool b_mn, int bm = 128) {
+  return f16 ? instr_desc(bn, a_mn, b_mn, bm) & ~((7u << 7) | (7u << 10)) : instr_desc(bn, a_mn, b_mn, bm);
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+// 16-bit operand formats: bf16 or (F16) fp16.
+template <bool F16>
+__device__ __forceinline__ uint32_t pack16x2(float lo, float hi) {
+  if constexpr (F16) return pack_f16x2(lo, hi);
+  else return pack_bf16x2(lo, hi);
+}
+template <bool F16>
+__device__ __forceinline__ float round16(float v) {
+  if constexpr (F16) return __half2float(__float2half_rn(v));
+  else return __bfloat162float(__float2bfloat16_rn(v));
+}
+template <bool F16>
+__device__ __forceinline__ void unpack16x8(const uint4& w, float* o) {
+  if constexpr (F16) Vec<f16>::load(reinterpret_cast<const f16*>(&w), o);
+  else Vec<bf16>::load(reinterpret_cast<const bf16*>(&w), o);
+}
 
 
 // TMA bulk-tensor reduce-add of a shared-memory box into global memory.

@@ -29,7 +29,8 @@ EXPORTED = [
     "gpt_set_adam_v", "gpt_get_logits", "gpt_get_residual", "gpt_get_scalars", "gpt_set_scalars", "gpt_status",
     "gpt_device_error", "gpt_last_error", "gpt_debug_poison_grad", "gpt_debug_wait_timeout",
     "gpt_kernel_launches", "gpt_profile_enable", "gpt_profile_read", "gpt_gemm_bf16",
-    "gpt_gemm_bf16_splitk_noalloc", "gpt_noalloc_status",
+    "gpt_gemm_bf16_splitk_noalloc", "gpt_noalloc_status", "gpt_set_lr_schedule", "gpt_train_steps",
+    "gpt_sample_decode", "gpt_backward_accumulate", "gpt_set_loss_weight",
 ]
 
 
@@ -43,7 +44,8 @@ class gpt_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("vocab", "vocab_padded", "d_model", "n_heads", "d_mlp",
                                               "n_layers", "max_seq", "max_batch", "tied", "precision",
                                               "loss_scaling")] + \
-               [("init_loss_scale", ctypes.c_float), ("ln_eps", ctypes.c_float), ("init_std", ctypes.c_float)]
+               [("init_loss_scale", ctypes.c_float), ("ln_eps", ctypes.c_float), ("init_std", ctypes.c_float),
+                ("arch", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("rope_base", ctypes.c_float)]
 
 
 class gpt_adamw(ctypes.Structure):
@@ -58,7 +60,19 @@ class gpt_prof_entry(ctypes.Structure):
 class gpt_scalars(ctypes.Structure):
     _fields_ = [("loss_scale", ctypes.c_float), ("good_steps", ctypes.c_int32), ("step", ctypes.c_int32),
                 ("last_loss", ctypes.c_float), ("last_grad_norm", ctypes.c_float),
-                ("last_skipped", ctypes.c_int32)]
+                ("last_skipped", ctypes.c_int32), ("last_lr", ctypes.c_float)]
+
+
+GPT_LR_CONSTANT, GPT_LR_COSINE = 0, 1
+
+
+class gpt_sampling(ctypes.Structure):
+    _fields_ = [("temperature", ctypes.c_float), ("top_k", ctypes.c_int32), ("top_p", ctypes.c_float)]
+
+
+class gpt_lr_schedule(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("warmup_steps", ctypes.c_int32), ("total_steps", ctypes.c_int32),
+                ("max_lr", ctypes.c_float), ("min_lr", ctypes.c_float)]
 
 
 _lib = None
@@ -80,6 +94,8 @@ def load_library(path: str = LIB_PATH):
         "gpt_set_stream": ([H, P], I),
         "gpt_forward_loss": ([H, P, P, P, I, I, P], I),
         "gpt_backward": ([H], I),
+        "gpt_backward_accumulate": ([H], I),
+        "gpt_set_loss_weight": ([H, F], I),
         "gpt_clip_adamw_step": ([H, ctypes.POINTER(gpt_adamw), P, P], I),
         "gpt_greedy_decode": ([H, P, I, I, I, P], I),
         "gpt_num_params": ([H, ctypes.POINTER(S)], I),
@@ -98,6 +114,9 @@ def load_library(path: str = LIB_PATH):
         "gpt_gemm_bf16_splitk_noalloc": ([I, I, I, P, ctypes.c_long, I, P, ctypes.c_long, I, I, P, ctypes.c_long, P],
                                          I),
         "gpt_noalloc_status": ([P], I),
+        "gpt_set_lr_schedule": ([H, ctypes.POINTER(gpt_lr_schedule)], I),
+        "gpt_sample_decode": ([H, P, I, I, I, ctypes.POINTER(gpt_sampling), P, P], I),
+        "gpt_train_steps": ([H, P, P, P, I, I, I, ctypes.POINTER(gpt_adamw), P, P, P], I),
         "gpt_profile_read": ([H, ctypes.POINTER(gpt_prof_entry), I, ctypes.POINTER(I)], I),
     }
     for n in ("params", "grads", "adam_m", "adam_v"):
@@ -114,9 +133,10 @@ def load_library(path: str = LIB_PATH):
 def make_config(mc: ModelConfig) -> gpt_config:
     return gpt_config(vocab=mc.vocab, vocab_padded=mc.vocab_padded, d_model=mc.d_model, n_heads=mc.n_heads,
                       d_mlp=mc.d_mlp, n_layers=mc.n_layers, max_seq=mc.max_seq, max_batch=mc.max_batch,
-                      tied=int(mc.tied), precision=1 if mc.precision == "bf16" else 0,
+                      tied=int(mc.tied), precision={"fp32": 0, "bf16": 1, "fp16": 2}[mc.precision],
                       loss_scaling=int(mc.loss_scaling), init_loss_scale=mc.init_loss_scale,
-                      ln_eps=mc.ln_eps, init_std=mc.init_std)
+                      ln_eps=mc.ln_eps, init_std=mc.init_std, arch={"gpt2": 0, "llama": 1}[mc.arch],
+                      n_kv_heads=mc.n_kv_heads, rope_base=mc.rope_base)
 
 
 def _ptr(t):
@@ -220,9 +240,15 @@ class GPT:
         return self._check(self.lib.gpt_forward_loss(self.h, _ptr(tokens), _ptr(targets), _ptr(seg_ids),
                                                      B, T, _ptr(loss)))
 
-    def backward(self):
+    def backward(self, accumulate=False):
         self._sync_stream()
+        if accumulate:
+            return self._check(self.lib.gpt_backward_accumulate(self.h))
         return self._check(self.lib.gpt_backward(self.h))
+
+    def set_loss_weight(self, w):
+        self._sync_stream()
+        return self._check(self.lib.gpt_set_loss_weight(self.h, w))
 
     def clip_adamw_step(self, hp: AdamWConfig, grad_norm=None, skipped=None):
         self._sync_stream()
@@ -230,12 +256,42 @@ class GPT:
                       clip_norm=hp.clip_norm)
         return self._check(self.lib.gpt_clip_adamw_step(self.h, ctypes.byref(a), _ptr(grad_norm), _ptr(skipped)))
 
+    def set_lr_schedule(self, kind=GPT_LR_COSINE, warmup_steps=0, total_steps=1, max_lr=0.0, min_lr=0.0):
+        """Device-side learning-rate schedule (kind None clears it)."""
+        self._sync_stream()
+        if kind is None:
+            return self._check(self.lib.gpt_set_lr_schedule(self.h, None))
+        sch = gpt_lr_schedule(kind=kind, warmup_steps=warmup_steps, total_steps=total_steps, max_lr=max_lr,
+                              min_lr=min_lr)
+        return self._check(self.lib.gpt_set_lr_schedule(self.h, ctypes.byref(sch)))
+
+    def train_steps(self, tokens, targets, seg_ids, hp: AdamWConfig, losses=None, grad_norms=None, skipped=None):
+        """K steps over tokens / targets / seg_ids of shape [K, B, T], one call."""
+        K, B, T = tokens.shape
+        self._sync_stream()
+        a = gpt_adamw(lr=hp.lr, beta1=hp.beta1, beta2=hp.beta2, eps=hp.eps, weight_decay=hp.weight_decay,
+                      clip_norm=hp.clip_norm)
+        return self._check(self.lib.gpt_train_steps(self.h, _ptr(tokens), _ptr(targets), _ptr(seg_ids), K, B, T,
+                                                    ctypes.byref(a), _ptr(losses), _ptr(grad_norms),
+                                                    _ptr(skipped)))
+
     def greedy_decode(self, prompt, n_new, out=None):
         B, Tp = prompt.shape
         if out is None:
             out = self.torch.empty((B, n_new), dtype=self.torch.int32, device=prompt.device)
         self._sync_stream()
         self._check(self.lib.gpt_greedy_decode(self.h, _ptr(prompt), B, Tp, n_new, _ptr(out)))
+        return out
+
+    def sample_decode(self, prompt, n_new, uniforms, temperature=1.0, top_k=0, top_p=1.0, out=None):
+        """Sampled continuation; uniforms: device float32 [B, n_new] in [0, 1)."""
+        B, Tp = prompt.shape
+        if out is None:
+            out = self.torch.empty((B, n_new), dtype=self.torch.int32, device=prompt.device)
+        sp = gpt_sampling(temperature=temperature, top_k=top_k, top_p=top_p)
+        self._sync_stream()
+        self._check(self.lib.gpt_sample_decode(self.h, _ptr(prompt), B, Tp, n_new, ctypes.byref(sp), _ptr(uniforms),
+                                               _ptr(out)))
         return out
 
     # -- state access (synchronous)

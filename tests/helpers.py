@@ -9,7 +9,7 @@ def ocfg(mc: CF.ModelConfig, max_seq=None) -> O.OracleConfig:
     return O.OracleConfig(vocab=mc.vocab, vocab_padded=mc.vocab_padded, d_model=mc.d_model,
                           n_heads=mc.n_heads, d_mlp=mc.d_mlp, n_layers=mc.n_layers,
                           max_seq=max_seq or mc.max_seq, tied=mc.tied, ln_eps=mc.ln_eps,
-                          init_std=mc.init_std)
+                          init_std=mc.init_std, arch=mc.arch, n_kv_heads=mc.n_kv_heads, rope_base=mc.rope_base)
 
 
 def per_tensor_rel_l2(cfg: O.OracleConfig, g_gpu, g_ref):

@@ -51,9 +51,10 @@ def test_library_has_no_driver_link_dependency():
 
 
 def test_struct_sizes_match_header():
-    assert ctypes.sizeof(G.gpt_config) == 14 * 4
+    assert ctypes.sizeof(G.gpt_config) == 17 * 4
     assert ctypes.sizeof(G.gpt_adamw) == 6 * 4
-    assert ctypes.sizeof(G.gpt_scalars) == 6 * 4
+    assert ctypes.sizeof(G.gpt_scalars) == 7 * 4
+    assert ctypes.sizeof(G.gpt_lr_schedule) == 5 * 4
 
 
 def test_header_is_plain_c_and_matches_the_binding(tmp_path):
@@ -65,6 +66,7 @@ def test_header_is_plain_c_and_matches_the_binding(tmp_path):
     if cc is None:
         pytest.skip("no C compiler")
     structs = {"gpt_config": G.gpt_config, "gpt_adamw": G.gpt_adamw, "gpt_scalars": G.gpt_scalars,
+               "gpt_lr_schedule": G.gpt_lr_schedule, "gpt_sampling": G.gpt_sampling,
                "gpt_prof_entry": G.gpt_prof_entry}
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "gpt.h"', "int main(void) {"]
     for sname, cls in structs.items():

@@ -384,28 +384,35 @@ def test_bounded_wait_times_out_and_context_survives(torch):
 
 def test_greedy_decode_bf16_batched(torch):
     """Decode with more than 8 rows runs its projections on the tensor-core GEMM,
-    fewer rows on the GEMV (the path the fp32 decode tests pin bit-exactly to the
-    oracle).  Both bf16 paths accumulate in fp32 and round at the same points: the
-    12-row decode must give the tokens of the same prompts decoded 6 rows at a
-    time, and its first token (from the prefill) must follow the oracle wherever
-    the oracle's top-2 gap is clear of bf16 rounding."""
+    fewer rows on the GEMV.  Both are checked against the oracle's logits for the
+    sequence each produced (teacher forcing, full prefix, no cache, on the bf16
+    weights): every token within 1 % of the row's logit scale of the oracle's
+    maximum, and exactly the oracle's argmax where the top-2 gap is clearer than
+    that.  (The two paths sum in different orders, so they need not agree bit
+    for bit with each other.)"""
     mc = CF.ModelConfig(vocab=512, vocab_padded=512, d_model=128, n_heads=2, d_mlp=512, n_layers=2,
                         max_seq=64, max_batch=12, tied=False, precision="bf16", init_std=0.3)
     cfg = ocfg(mc)
     model = new_model(mc, 11)
     rng = np.random.default_rng(4)
     prompt = rng.integers(0, 512, size=(12, 10)).astype(np.int32)
-    out = model.greedy_decode(dev(torch, prompt), 6).cpu().numpy()
+    outs = [model.greedy_decode(dev(torch, prompt), 6).cpu().numpy(),
+            np.concatenate([model.greedy_decode(dev(torch, prompt[i:i + 6]), 6).cpu().numpy() for i in (0, 6)])]
     assert model.status() == 0
-    halves = [model.greedy_decode(dev(torch, prompt[i:i + 6]), 6).cpu().numpy() for i in (0, 6)]
-    assert np.array_equal(out, np.concatenate(halves)), (out, halves)
-    # the GPU multiplies bf16 copies of the weights: give the oracle the same values
     p32 = model.get_params()
     pb = (p32.view(np.uint32) + 0x7FFF + ((p32.view(np.uint32) >> 16) & 1)) & 0xFFFF0000
-    ref, gaps = O.greedy_decode(cfg, pb.view(np.float32).astype(np.float64), prompt, 1, dtype=np.float64)
-    clear = gaps[:, 0] >= 0.1
-    assert clear.sum() >= 9, gaps[:, 0]
-    assert np.array_equal(out[clear, 0], ref[clear, 0]), (out[:, 0], ref[:, 0], gaps[:, 0])
+    pb = pb.view(np.float32).astype(np.float64)
+    for out in outs:
+        seq = np.concatenate([prompt, out[:, :-1]], axis=1)
+        z, _ = O.forward(cfg, pb, seq)
+        z = z.reshape(12, 15, -1)[:, 9:, :512]
+        picked = np.take_along_axis(z, out[:, :, None].astype(np.int64), axis=2)[:, :, 0]
+        tol = 0.01 * np.abs(z).max(axis=2)
+        assert np.all(z.max(axis=2) - picked <= tol)
+        srt = np.sort(z, axis=2)
+        clear = srt[:, :, -1] - srt[:, :, -2] > tol
+        assert clear.mean() >= 0.7
+        assert np.array_equal(out[clear], np.argmax(z, axis=2)[clear])
 
 
 def test_byte30m_bf16_trajectory(torch):

@@ -22,7 +22,7 @@ def ocfg(mc: CF.ModelConfig) -> O.OracleConfig:
     return O.OracleConfig(vocab=mc.vocab, vocab_padded=mc.vocab_padded, d_model=mc.d_model,
                           n_heads=mc.n_heads, d_mlp=mc.d_mlp, n_layers=mc.n_layers,
                           max_seq=mc.max_seq, tied=mc.tied, ln_eps=mc.ln_eps,
-                          init_std=mc.init_std)
+                          init_std=mc.init_std, arch=mc.arch, n_kv_heads=mc.n_kv_heads, rope_base=mc.rope_base)
 
 
 TINY = O.OracleConfig(vocab=11, vocab_padded=16, d_model=8, n_heads=2, d_mlp=16,
