@@ -33,7 +33,12 @@ What it computes, with the page each step follows:
 * dynamic loss scaling with skip-on-overflow -- LucilleAI, "Architecture"
   (GradScaler, AMP);
 * greedy decoding: take the argmax, append it, repeat -- RustGPT "Technical
-  implementation" (greedy decoding); Smallem "Ce qu'est un modele de langage".
+  implementation" (greedy decoding); Smallem "Ce qu'est un modele de langage";
+* sampled decoding (temperature, top-k, top-p) and beam search -- RustGPT,
+  roadmap "high-priority feature requests" (better sampling); the learning-rate
+  schedule -- LucilleAI, "Getting started" (cosine, warm-up, min-lr); the
+  Llama-style block (RMSNorm, rotary positions, grouped key/value heads,
+  SwiGLU) -- "NTransformer", key features.
 
 Where the pages leave a step open the plainest reading is taken (GPT-2's
 LayerNorm eps 1e-5 with biased variance, tanh-form GELU, biases on every
@@ -755,3 +760,56 @@ def sample_decode(cfg: OracleConfig, flat_params, prompt, n_new, temperature, to
             out[b, s] = sample_token(last[b], cfg.vocab, temperature, top_k, top_p, float(uniforms[b, s]))
         seq = np.concatenate([seq, out[:, s:s + 1]], axis=1)
     return out
+
+
+# ---------------------------------------------------------------------------
+# Beam search
+# ---------------------------------------------------------------------------
+
+def log_softmax_row(z, V):
+    """log p over the real vocabulary 0..V-1 of one row of logits."""
+    x = np.asarray(z[:V], dtype=np.float64)
+    m = np.max(x)
+    return x - (m + np.log(np.sum(np.exp(x - m))))
+
+
+def beam_decode(cfg: OracleConfig, flat_params, prompt, n_new, width, dtype=np.float64):
+    """Beam search by full-prefix recomputation (no cache).
+
+    "RustGPT" lists beam search beside top-k / top-p and temperature among
+    the sampling features its roadmap asks for (roadmap, "high-priority
+    feature requests"); the page gives no further rule, so the plainest
+    reading is taken: per prompt, keep the ``width`` continuations with the
+    largest sum of next-token log-probabilities (log-softmax over the real
+    vocabulary), extend every kept continuation by every token, keep the best
+    ``width`` again, for exactly ``n_new`` tokens (no end token, no length
+    normalisation).  Order: score descending, ties to the lower flat index
+    parent_rank * V + token, where parent_rank is the parent's place in the
+    previous step's order.  The first step extends the prompt alone.
+
+    Returns (tokens [B, width, n_new], scores [B, width], margins [B, n_new]):
+    beams best first; margins[b, s] is the gap between the last kept and the
+    first dropped candidate at step s (inf where nothing was dropped).
+    """
+    prompt = np.asarray(prompt, dtype=np.int64)
+    B, V = prompt.shape[0], cfg.vocab
+    toks = np.zeros((B, width, n_new), dtype=np.int64)
+    scores = np.zeros((B, width), dtype=np.float64)
+    margins = np.zeros((B, n_new), dtype=np.float64)
+    for b in range(B):
+        beams = [(0.0, [])]                      # (score, tokens so far), best first
+        for s in range(n_new):
+            seqs = np.array([np.concatenate([prompt[b], np.array(t, dtype=np.int64)]) for _, t in beams])
+            logits, _ = forward(cfg, flat_params, seqs, None, dtype)
+            last = logits.reshape(len(beams), seqs.shape[1], -1)[:, -1, :]
+            cand_score = np.concatenate([sc + log_softmax_row(last[r], V) for r, (sc, _) in enumerate(beams)])
+            flat = np.arange(cand_score.size)
+            order = np.lexsort((flat, -cand_score))   # score descending, then flat index ascending
+            keep = order[:width]
+            margins[b, s] = cand_score[keep[-1]] - cand_score[order[width]] if order.size > width else np.inf
+            beams = [(float(cand_score[i]), beams[i // V][1] + [int(i % V)]) for i in keep]
+        for w, (sc, t) in enumerate(beams):
+            toks[b, w] = t
+            scores[b, w] = sc
+    return toks, scores, margins
+

@@ -599,3 +599,74 @@ def test_llama_mask_and_packing_bit_identity():
     d0, _ = O.forward(cfg, flat, tok[:, :3])
     d1, _ = O.forward(cfg, flat, tok[:, 3:])
     assert np.array_equal(p[:3], d0) and np.array_equal(p[3:], d1)
+
+
+# ---------------------------------------------------------------------------
+# Beam search
+# ---------------------------------------------------------------------------
+
+def _seq_logprob_bruteforce(cfg, flat, prompt_row, cont):
+    """Total log-probability of a continuation from ONE forward pass over the
+    whole sequence (not step by step), log-softmax by scipy's logsumexp over
+    the real vocabulary."""
+    from scipy.special import logsumexp
+    seq = np.concatenate([prompt_row, cont])[None, :]
+    z, _ = O.forward(cfg, flat, seq, None, np.float64)
+    z = z.reshape(seq.shape[1], -1)[:, :cfg.vocab]
+    Tp = prompt_row.size
+    tot = 0.0
+    for i, t in enumerate(cont):
+        row = z[Tp - 1 + i]
+        tot += row[t] - logsumexp(row)
+    return tot
+
+
+def test_beam_exhaustive_when_width_covers_all_prefixes():
+    """With V = 3 and width 9 = V^2, the last step ranks every one of the 27
+    three-token continuations, so the beams are exactly the 9 best sequences
+    by total log-probability (each scored here by one full-sequence forward)."""
+    import itertools
+    cfg = O.OracleConfig(vocab=3, vocab_padded=8, d_model=8, n_heads=2, d_mlp=16, n_layers=2, max_seq=8)
+    flat = random_params(cfg, 61, scale=0.8)
+    prompt = np.array([[1, 0, 2], [2, 2, 1]])
+    toks, scores, _ = O.beam_decode(cfg, flat, prompt, 3, 9)
+    for b in range(2):
+        allseq = [np.array(c) for c in itertools.product(range(3), repeat=3)]
+        lp = np.array([_seq_logprob_bruteforce(cfg, flat, prompt[b], c) for c in allseq])
+        order = np.argsort(-lp, kind="stable")[:9]
+        assert np.allclose(scores[b], lp[order], rtol=0, atol=1e-12)
+        for w in range(9):
+            assert np.array_equal(toks[b, w], allseq[order[w]])
+
+
+def test_beam_width_one_is_greedy_and_scores_are_log_probs():
+    """Width 1 keeps the argmax every step (greedy decoding); every beam's
+    score is its continuation's total log-probability; scores descend; the
+    beams are distinct."""
+    cfg = O.OracleConfig(vocab=50, vocab_padded=64, d_model=16, n_heads=2, d_mlp=32, n_layers=2, max_seq=12)
+    flat = random_params(cfg, 62, scale=0.5)
+    prompt = np.array([[3, 7, 11, 2], [9, 9, 40, 1]])
+    g, _ = O.greedy_decode(cfg, flat, prompt, 5, dtype=np.float64)
+    t1, _, _ = O.beam_decode(cfg, flat, prompt, 5, 1)
+    assert np.array_equal(t1[:, 0], g)
+    toks, scores, margins = O.beam_decode(cfg, flat, prompt, 5, 4)
+    for b in range(2):
+        assert np.all(np.diff(scores[b]) <= 0)
+        assert len({tuple(t) for t in toks[b]}) == 4
+        for w in range(4):
+            assert abs(scores[b, w] - _seq_logprob_bruteforce(cfg, flat, prompt[b], toks[b, w])) < 1e-10
+    # a wider beam never ends below the narrower one's best
+    assert np.all(scores[:, 0] >= O.beam_decode(cfg, flat, prompt, 5, 2)[1][:, 0] - 1e-12)
+    assert np.all(margins >= 0)
+
+
+def test_beam_ties_go_to_lower_flat_index():
+    """A model whose logits ignore the input (zero weights, zero head): every
+    token has log-probability -log V, so the beams after two steps are the
+    lexicographically first continuations (0,0), (0,1), ..."""
+    cfg = O.OracleConfig(vocab=5, vocab_padded=8, d_model=8, n_heads=2, d_mlp=16, n_layers=1, max_seq=6)
+    flat = np.zeros(O.num_params(cfg))
+    toks, scores, margins = O.beam_decode(cfg, flat, np.array([[1, 2]]), 2, 3)
+    assert np.array_equal(toks[0], [[0, 0], [0, 1], [0, 2]])
+    assert np.allclose(scores, -2 * np.log(5))
+    assert np.all(margins == 0)
