@@ -254,6 +254,24 @@ typedef struct {
 int gpt_sample_decode(gpt_model* m, const int32_t* prompt, int B, int Tp, int n_new, const gpt_sampling* sp,
                       const float* uniforms, int32_t* out);
 
+/* Beam search ("RustGPT", roadmap "high-priority feature requests": beam
+ * search): per prompt, the `width` continuations of n_new tokens with the
+ * largest sum of next-token log-probabilities (fp32 log-softmax over the real
+ * vocabulary).  Each step extends every kept beam by every token and keeps
+ * the best `width` (score descending, ties to the lower parent * V + token,
+ * parents counted by their place in the previous order); the first step
+ * extends the prompt alone.  No end token, no length normalisation.
+ *  prompt  device int32 [B, Tp]
+ *  out     device int32 [B, width, n_new]: the beams' tokens, best first
+ *  scores  device float [B, width]: their summed log-probabilities
+ * The beams share the prompt's cache rows and never copy the key/value cache:
+ * each reads its earlier positions through a table of source rows.
+ * Requires 1 <= width <= 8, width <= vocab <= 55000, B * width <= max_batch
+ * and <= 32, Tp + n_new - 1 <= max_seq.
+ * Errors: GPT_ERR_ARG, GPT_ERR_STATE (sequence too long). */
+int gpt_beam_decode(gpt_model* m, const int32_t* prompt, int B, int Tp, int n_new, int width, int32_t* out,
+                    float* scores);
+
 /* Number of parameters N in the canonical layout:
  *  wte[Vp,C], wpe[max_seq,C]; per layer ln1_g[C], ln1_b[C], w_qkv[3C,C]
  *  (rows: q, then k, then v; head h = rows h*d..h*d+d-1 of each), b_qkv[3C],

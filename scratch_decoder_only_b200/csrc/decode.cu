@@ -270,8 +270,10 @@ dec_attn_split_kernel(const T* __restrict__ qkv, T* kc, T* vc, float* __restrict
   for (int j0 = (sp * NW + warp) * KPW; j0 <= pos; j0 += DA_SPLITS * NW * KPW) {
     const int j = j0 + grp;
     const bool live = j <= pos;
-    const T* kr = j == pos ? knew : kcb + (long)j * D;
-    const T* vr = j == pos ? vnew : vcb + (long)j * D;
+    long row = (long)j * D;
+    if (Ly.src && j < pos) row += ((long)Ly.src[(long)b * Tmax + j] - b) * Ly.Hkv * Tmax * D;
+    const T* kr = j == pos ? knew : kcb + row;
+    const T* vr = j == pos ? vnew : vcb + row;
     float kv[8], vv[8];
     if (live) {
       load8(kr + sub * 8, kv);

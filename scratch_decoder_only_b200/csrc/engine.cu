@@ -77,6 +77,15 @@ struct gpt_model {
   float smp_temp = 0.f, smp_topp = 1.f;
   int smp_topk = 0;
   const float* smp_u = nullptr;
+  // beam search (gpt_beam_decode); beam_w = 0: off.  dsrc [Bmax][Tmax]: the
+  // cache row of each (row, position); dbcs / dbct: per-row candidates
+  int beam_w = 0;
+  float* beam_scores = nullptr;
+  int* dsrc = nullptr;
+  float* dbcs = nullptr;
+  int* dbct = nullptr;
+  int dec_beam_w = 0;
+  float* dec_beam_scores = nullptr;
   bool dec_smp_on = false;   // the sampling state the captured graph was built with
   float dec_smp_temp = 0.f, dec_smp_topp = 1.f;
   int dec_smp_topk = 0;
@@ -360,6 +369,9 @@ static int build_arena(gpt_model* m) {
   cv.add((void**)&m->dtok, Bx * 4);
   cv.add((void**)&m->dpart, dec_attn_part_floats((int)Bx, m->H, m->d) * 4);
   cv.add((void**)&m->dam, Bx * DF_MAX_GRID * 8 + Bx * m->H * 4);   // argmax partials, then split counters
+  cv.add((void**)&m->dsrc, Bx * (size_t)m->Tmax * 4);
+  cv.add((void**)&m->dbcs, Bx * BEAM_MAX_WIDTH * 4);
+  cv.add((void**)&m->dbct, Bx * BEAM_MAX_WIDTH * 4);
   m->arena_bytes = cv.off + 256;
   cudaError_t e = cudaMalloc((void**)&m->arena, m->arena_bytes);
   if (e != cudaSuccess) {
@@ -915,6 +927,7 @@ static DecLayout dec_layout(const gpt_model* m) {
   L.kcol = m->C;
   L.vcol = m->C + m->Hkv * m->d;
   L.Hkv = m->Hkv;
+  L.src = m->beam_w ? m->dsrc : nullptr;
   return L;
 }
 
@@ -954,7 +967,12 @@ static int decode_step(gpt_model* m, int B, int Tp, int n_new, int32_t* out, cud
   }
   CK(launch_ln_fwd<T>(x, A.P(m->o_lnf_g), P0(m->o_lnf_b), xf, m->dmu, m->drs, B, C, eps, s));
   CK(dec_proj<T>(m, xf, B, C, A.W(m->o_head), m->Vp, nullptr, nullptr, 2, nullptr, nullptr, m->dlogits, s));
-  if (m->smp_on)
+  if (m->beam_w) {
+    const int W = m->beam_w;
+    CK(launch_beam_topk(m->dlogits, m->Vp, m->V, B / W, W, false, m->beam_scores, m->dbcs, m->dbct, s));
+    CK(launch_beam_merge(m->dbcs, m->dbct, B / W, W, m->V, Tp, m->dsrc, m->Tmax, m->beam_scores, m->dtok, out, n_new,
+                         stepc, s));
+  } else if (m->smp_on)
     CK(launch_sample(m->dlogits, B, m->V, m->Vp, m->smp_temp, m->smp_topk, m->smp_topp, m->smp_u, n_new, m->dtok, out,
                      n_new, stepc, s));
   else
@@ -978,14 +996,22 @@ static int decode_impl(gpt_model* m, const int32_t* prompt, int B, int Tp, int n
   CK(launch_gather_last<T>((const T*)m->xf, B, Tp, C, (T*)m->dxf, s));
   CK(dec_proj<T>(m, (const T*)m->dxf, B, C, A.W(m->o_head), m->Vp, nullptr, nullptr, 2, nullptr, nullptr,
                  m->dlogits, s));
-  if (m->smp_on)
+  if (m->beam_w) {
+    // every beam of a prompt starts from the prompt's prefill row
+    const int W = m->beam_w;
+    CK(launch_beam_init(m->dsrc, m->Tmax, m->beam_scores, B, W, Tp, s));
+    CK(launch_beam_topk(m->dlogits, m->Vp, m->V, B, W, true, m->beam_scores, m->dbcs, m->dbct, s));
+    CK(launch_beam_merge(m->dbcs, m->dbct, B, W, m->V, Tp, m->dsrc, m->Tmax, m->beam_scores, m->dtok, out, n_new,
+                         nullptr, s));
+  } else if (m->smp_on)
     CK(launch_sample(m->dlogits, B, m->V, m->Vp, m->smp_temp, m->smp_topk, m->smp_topp, m->smp_u, n_new, m->dtok, out,
                      n_new, nullptr, s));
   else
     CK(launch_argmax(m->dlogits, B, m->V, m->Vp, m->dtok, out, n_new, nullptr, s));
   if (n_new == 1) return GPT_OK;
+  const int Bd = m->beam_w ? B * m->beam_w : B;   // decode rows
   if constexpr (sizeof(T) == 2) {
-    if (!m->smp_on && !m->fp16 && !m->llama && dec_fused_supported(B, C, H, m->F, m->Vp)) {
+    if (!m->smp_on && !m->beam_w && !m->fp16 && !m->llama && dec_fused_supported(B, C, H, m->F, m->Vp)) {
       // every later token from one persistent kernel
       const LayerOff& l0 = m->L[0];
       DecFusedParams q;
@@ -1021,14 +1047,15 @@ static int decode_impl(gpt_model* m, const int32_t* prompt, int B, int Tp, int n
     CK(cudaEventCreateWithFlags(&m->ev_b, cudaEventDisableTiming));
   }
   const bool same_smp = m->dec_smp_on == m->smp_on && m->dec_smp_temp == m->smp_temp &&
-                        m->dec_smp_topk == m->smp_topk && m->dec_smp_topp == m->smp_topp && m->dec_smp_u == m->smp_u;
-  if (!m->dec_graph || m->dec_B != B || m->dec_Tp != Tp || m->dec_nnew != n_new || m->dec_out != out || !same_smp) {
+                        m->dec_smp_topk == m->smp_topk && m->dec_smp_topp == m->smp_topp && m->dec_smp_u == m->smp_u &&
+                        m->dec_beam_w == m->beam_w && m->dec_beam_scores == m->beam_scores;
+  if (!m->dec_graph || m->dec_B != Bd || m->dec_Tp != Tp || m->dec_nnew != n_new || m->dec_out != out || !same_smp) {
     if (m->dec_graph) { cudaGraphExecDestroy(m->dec_graph); m->dec_graph = nullptr; }
     cudaGraph_t g = nullptr;
     unsigned long long n0 = g_kernel_launches;
     CK(cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
     g_pdl = true;   // each captured kernel may start while its predecessor drains
-    int r = decode_step<T>(m, B, Tp, n_new, out, m->cap_stream);
+    int r = decode_step<T>(m, Bd, Tp, n_new, out, m->cap_stream);
     g_pdl = false;
     cudaError_t ec = cudaStreamEndCapture(m->cap_stream, &g);
     if (r != GPT_OK) { if (g) cudaGraphDestroy(g); return r; }
@@ -1036,11 +1063,12 @@ static int decode_impl(gpt_model* m, const int32_t* prompt, int B, int Tp, int n
     cudaError_t ei = cudaGraphInstantiate(&m->dec_graph, g, 0);
     cudaGraphDestroy(g);
     CK(ei);
+    m->dec_kernels = (int)(g_kernel_launches - n0);   // the kernels one replay launches
     g_kernel_launches = n0;
-    m->dec_kernels = 7 * m->NL + 5;
-    m->dec_B = B; m->dec_Tp = Tp; m->dec_nnew = n_new; m->dec_out = out;
+    m->dec_B = Bd; m->dec_Tp = Tp; m->dec_nnew = n_new; m->dec_out = out;
     m->dec_smp_on = m->smp_on; m->dec_smp_temp = m->smp_temp; m->dec_smp_topk = m->smp_topk;
     m->dec_smp_topp = m->smp_topp; m->dec_smp_u = m->smp_u;
+    m->dec_beam_w = m->beam_w; m->dec_beam_scores = m->beam_scores;
   }
   CK(cudaEventRecord(m->ev_a, s));
   CK(cudaStreamWaitEvent(m->cap_stream, m->ev_a, 0));
@@ -1321,6 +1349,29 @@ int gpt_sample_decode(gpt_model* m, const int32_t* prompt, int B, int Tp, int n_
   const int r = m->fp16 ? decode_impl<f16>(m, prompt, B, Tp, n_new, out)
                 : m->lp ? decode_impl<bf16>(m, prompt, B, Tp, n_new, out) : decode_impl<float>(m, prompt, B, Tp, n_new, out);
   m->smp_on = false;
+  return r;
+}
+
+int gpt_beam_decode(gpt_model* m, const int32_t* prompt, int B, int Tp, int n_new, int width, int32_t* out,
+                    float* scores) {
+  if (!m) return GPT_ERR_ARG;
+  m->err.clear();
+  if (!prompt || !out || !scores) FAIL(GPT_ERR_ARG, "prompt / out / scores is NULL");
+  if (width < 1 || width > BEAM_MAX_WIDTH) FAIL(GPT_ERR_ARG, "width out of range [1, 8]");
+  if (m->V < width) FAIL(GPT_ERR_ARG, "width exceeds the vocabulary");
+  if (m->V > SMP_MAX_VOCAB) FAIL(GPT_ERR_ARG, "vocabulary too large for the beam kernel");
+  if (B < 1 || (long)B * width > m->Bmax || (long)B * width > 32)
+    FAIL(GPT_ERR_ARG, "B * width out of range [1, min(max_batch, 32)]");
+  if (Tp < 1 || n_new < 1) FAIL(GPT_ERR_ARG, "Tp and n_new must be >= 1");
+  if ((long)Tp + n_new - 1 > m->Tmax) FAIL(GPT_ERR_STATE, "Tp + n_new - 1 exceeds max_seq");
+  if ((uintptr_t)scores & 3) FAIL(GPT_ERR_ARG, "scores must be 4-byte aligned");
+  m->have_targets = false;
+  m->beam_w = width;
+  m->beam_scores = scores;
+  const int r = m->fp16 ? decode_impl<f16>(m, prompt, B, Tp, n_new, out)
+                : m->lp ? decode_impl<bf16>(m, prompt, B, Tp, n_new, out) : decode_impl<float>(m, prompt, B, Tp, n_new, out);
+  m->beam_w = 0;
+  m->beam_scores = nullptr;
   return r;
 }
 

@@ -1021,19 +1021,26 @@ cudaError_t launch_loss_finalize(const float* rowloss, int M, DevScalars* sc, fl
 template <typename T>
 __global__ void embed_bwd_kernel(const float* __restrict__ dres, const int* __restrict__ tok,
                                  const int* __restrict__ pos, float* gwte, float* gwpe, int M, int C) {
+  // one warp per row; the row's fp32 gradient is loaded whole (up to 8
+  // 16-byte vectors per lane in flight), then added into the token's and the
+  // position's gradient rows with 16-byte vector atomics (a row's additions
+  // land in no fixed order among the rows that share a token or position)
   int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   int lane = threadIdx.x & 31;
   if (row >= M) return;
-  const float* d = dres + (long)row * C;
-  float* a = gwte + (long)tok[row] * C;
-  float* b = gwpe ? gwpe + (long)pos[row] * C : nullptr;
-  for (int c = lane * 4; c < C; c += 128) {
-    float v[4];
-    Vec<float>::load(d + c, v);
+  const float4* d = reinterpret_cast<const float4*>(dres + (long)row * C);
+  float4* a = reinterpret_cast<float4*>(gwte + (long)tok[row] * C);
+  float4* b = gwpe ? reinterpret_cast<float4*>(gwpe + (long)pos[row] * C) : nullptr;
+  const int n4 = C / 4;
+  float4 v[8];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      atomicAdd(a + c + j, v[j]);
-      if (b) atomicAdd(b + c + j, v[j]);
+  for (int k = 0; k < 8; ++k)
+    if (lane + 32 * k < n4) v[k] = __ldcs(d + lane + 32 * k);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    if (lane + 32 * k < n4) {
+      atomicAdd(a + lane + 32 * k, v[k]);
+      if (b) atomicAdd(b + lane + 32 * k, v[k]);
     }
   }
 }

@@ -168,6 +168,9 @@ cudaError_t launch_gemv(const T* X, int B, int K, const T* W, int N, const float
 // {3C, C, 2C, H}.
 struct DecLayout {
   int qw, kcol, vcol, Hkv;
+  // beam search: src[b * Tmax + t] = the cache row holding position t of
+  // row b's sequence (positions before the current one); null: row b itself
+  const int* src = nullptr;
 };
 template <typename T>
 cudaError_t launch_kv_fill(const T* qkv, T* kc, T* vc, int B, int Tp, int d, int Tmax, const DecLayout& L,
@@ -189,6 +192,25 @@ cudaError_t launch_sample(const float* logits, int B, int V, int Vp, float temp,
                           cudaStream_t s);
 template <typename T>
 cudaError_t launch_gather_last(const T* x, int B, int Tp, int C, T* out, cudaStream_t s);
+
+// ---- beam.cu: beam search over the decode rows (row r = b * W + w)
+#define BEAM_MAX_WIDTH 8
+// scores[b W + w] = 0 for w = 0, -inf otherwise; src rows of every beam of
+// prompt b point at prefill row b for the prompt's positions t < Tp.
+cudaError_t launch_beam_init(int* src, int Tmax, float* scores, int B, int W, int Tp, cudaStream_t s);
+// Per row: log-softmax over the real vocabulary (fp32) and the row's W best
+// candidates scores[r] + log p (ties to the lower token), into cand_s /
+// cand_t [B W][W].  first: the logits of beam (b, w) are row b and only w = 0
+// takes part (the others' candidates are -inf).  V * 4 bytes of shared memory.
+cudaError_t launch_beam_topk(const float* logits, int Vp, int V, int B, int W, bool first, const float* scores,
+                             float* cand_s, int* cand_t, cudaStream_t s);
+// Per prompt: the W best of the W x W candidates (score descending, ties to
+// the lower parent * V + token); reorders the token history out [B W][out_ld]
+// and the source-row table by parent, appends the chosen tokens at column
+// (*step or 0), sets scores and the next input tokens tok[B W].
+cudaError_t launch_beam_merge(const float* cand_s, const int* cand_t, int B, int W, int V, int Tp, int* src,
+                              int Tmax, float* scores, int* tok, int32_t* out, int out_ld, const int* step,
+                              cudaStream_t s);
 
 // ---- llama.cu: the Llama-style block's elementwise kernels (16-bit T)
 // rotary positions in place on nq query heads at columns [0, nq d) and nk key

@@ -30,7 +30,7 @@ EXPORTED = [
     "gpt_device_error", "gpt_last_error", "gpt_debug_poison_grad", "gpt_debug_wait_timeout",
     "gpt_kernel_launches", "gpt_profile_enable", "gpt_profile_read", "gpt_gemm_bf16",
     "gpt_gemm_bf16_splitk_noalloc", "gpt_noalloc_status", "gpt_set_lr_schedule", "gpt_train_steps",
-    "gpt_sample_decode", "gpt_backward_accumulate", "gpt_set_loss_weight",
+    "gpt_sample_decode", "gpt_backward_accumulate", "gpt_set_loss_weight", "gpt_beam_decode",
 ]
 
 
@@ -116,6 +116,7 @@ def load_library(path: str = LIB_PATH):
         "gpt_noalloc_status": ([P], I),
         "gpt_set_lr_schedule": ([H, ctypes.POINTER(gpt_lr_schedule)], I),
         "gpt_sample_decode": ([H, P, I, I, I, ctypes.POINTER(gpt_sampling), P, P], I),
+        "gpt_beam_decode": ([H, P, I, I, I, I, P, P], I),
         "gpt_train_steps": ([H, P, P, P, I, I, I, ctypes.POINTER(gpt_adamw), P, P, P], I),
         "gpt_profile_read": ([H, ctypes.POINTER(gpt_prof_entry), I, ctypes.POINTER(I)], I),
     }
@@ -293,6 +294,16 @@ class GPT:
         self._check(self.lib.gpt_sample_decode(self.h, _ptr(prompt), B, Tp, n_new, ctypes.byref(sp), _ptr(uniforms),
                                                _ptr(out)))
         return out
+
+    def beam_decode(self, prompt, n_new, width):
+        """Beam search: returns (tokens int32 [B, width, n_new], scores float32
+        [B, width]) on the prompt's device, beams best first."""
+        B, Tp = prompt.shape
+        out = self.torch.empty((B, width, n_new), dtype=self.torch.int32, device=prompt.device)
+        scores = self.torch.empty((B, width), dtype=self.torch.float32, device=prompt.device)
+        self._sync_stream()
+        self._check(self.lib.gpt_beam_decode(self.h, _ptr(prompt), B, Tp, n_new, width, _ptr(out), _ptr(scores)))
+        return out, scores
 
     # -- state access (synchronous)
     def _get(self, which, dst=None):
