@@ -152,7 +152,7 @@ __device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& y0, floa
 // Pairs k of a 32-score chunk (k = 0..15) with (k & 7) < FW_POLY_PAIRS take
 // the polynomial, the others the MUFU ex2: the two units run side by side.
 #ifndef FW_POLY_PAIRS
-#define FW_POLY_PAIRS 3
+#define FW_POLY_PAIRS 0
 #endif
 
 __device__ __forceinline__ float fmax3f(float a, float b, float c) {
@@ -764,43 +764,28 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
       // masking only where a key can be later than a query or before its document
       // (document starts never decrease, queries past T carry INT_MAX)
       const bool need_mask = q0 < k0 + AT_BLK || DSq[BW_QB - 1 - 64 * grp] > k0;
-      // four 16-column quarters of the group's 64 query columns, each
-      // quarter's S^T / dP^T loads issued before the previous quarter's
-      // arithmetic (a TMEM load wait covers every load in flight)
+      // two 32-column halves of the group's 64 query columns (a variant that
+      // pipelined 16-column quarters, each quarter's loads issued before the
+      // previous quarter's arithmetic, measured 4 % slower)
       uint32_t pw[32], dw[32];
-      uint32_t sa[16], da[16], sb[16], db[16];
-      const uint32_t tSg = tmem + lane_off + 64 * grp, tDg = tmem + lane_off + 128 + 64 * grp;
-      const int qf = q0 + 64 * grp;
-      tmem_ld16(tSg, sa);
-      tmem_ld16(tDg, da);
-      tmem_wait_ld();
 #pragma unroll
-      for (int qt = 0; qt < 4; qt += 2) {
-        tmem_ld16(tSg + 16 * (qt + 1), sb);
-        tmem_ld16(tDg + 16 * (qt + 1), db);
-        if (need_mask)
-          bwd_elementwise<true, F16, 16>(sa, da, L2 + 16 * qt, Dq + 16 * qt, DSq + 16 * qt, qf + 16 * qt, k, sl2,
-                                         pw + 8 * qt, dw + 8 * qt);
-        else
-          bwd_elementwise<false, F16, 16>(sa, da, L2 + 16 * qt, Dq + 16 * qt, DSq + 16 * qt, qf + 16 * qt, k, sl2,
-                                          pw + 8 * qt, dw + 8 * qt);
+      for (int half = 0; half < 2; ++half) {
+        uint32_t sr[32], dr[32];
+        tmem_ld32(tmem + lane_off + 64 * grp + 32 * half, sr);
+        tmem_ld32(tmem + lane_off + 128 + 64 * grp + 32 * half, dr);
         tmem_wait_ld();
-        if (qt + 2 < 4) {
-          tmem_ld16(tSg + 16 * (qt + 2), sa);
-          tmem_ld16(tDg + 16 * (qt + 2), da);
-        } else {
-          // every S^T / dP^T value of this block is in registers
+        if (half == 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(S_FREE));   // S^T / dP^T may be overwritten
         }
+        const int qf = q0 + 64 * grp + 32 * half;
         if (need_mask)
-          bwd_elementwise<true, F16, 16>(sb, db, L2 + 16 * (qt + 1), Dq + 16 * (qt + 1), DSq + 16 * (qt + 1),
-                                         qf + 16 * (qt + 1), k, sl2, pw + 8 * (qt + 1), dw + 8 * (qt + 1));
+          bwd_elementwise<true, F16, 32>(sr, dr, L2 + 32 * half, Dq + 32 * half, DSq + 32 * half, qf, k, sl2,
+                                         pw + 16 * half, dw + 16 * half);
         else
-          bwd_elementwise<false, F16, 16>(sb, db, L2 + 16 * (qt + 1), Dq + 16 * (qt + 1), DSq + 16 * (qt + 1),
-                                          qf + 16 * (qt + 1), k, sl2, pw + 8 * (qt + 1), dw + 8 * (qt + 1));
-        if (qt + 2 < 4) tmem_wait_ld();
+          bwd_elementwise<false, F16, 32>(sr, dr, L2 + 32 * half, Dq + 32 * half, DSq + 32 * half, qf, k, sl2,
+                                          pw + 16 * half, dw + 16 * half);
       }
       // the previous block's P^T / dS^T have been consumed and its dQ is complete
       if (i > 0 && !wait_w(bar(MMA_DONE), (i - 1) & 1)) { ok = false; break; }

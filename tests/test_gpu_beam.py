@@ -18,7 +18,7 @@ import pytest
 from oracle import gpt_oracle as O
 from scratch_decoder_only_b200 import configs as CF
 from scratch_decoder_only_b200 import synthetic as S
-from tests.helpers import ocfg
+from tests.helpers import ocfg, tame_attention
 
 pytestmark = pytest.mark.gpu
 
@@ -109,6 +109,7 @@ def test_beam_bf16_scores_are_log_probs(torch, B):
     from scratch_decoder_only_b200.gpt import GPT
     cfg = ocfg(DEC64)
     model = GPT(DEC64, 13)
+    tame_attention(model, cfg)
     rng = np.random.default_rng(70 + B)
     prompt = rng.integers(0, DEC64.vocab, size=(B, 16)).astype(np.int32)
     toks, scores = model.beam_decode(dev(torch, prompt), 20, 4)
@@ -123,6 +124,7 @@ def test_beam_llama_bf16(torch):
                         init_std=0.3)
     cfg = ocfg(mc)
     model = GPT(mc, 14)
+    tame_attention(model, cfg)
     rng = np.random.default_rng(77)
     prompt = rng.integers(0, 1000, size=(2, 16)).astype(np.int32)
     toks, scores = model.beam_decode(dev(torch, prompt), 16, 3)

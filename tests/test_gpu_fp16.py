@@ -19,7 +19,7 @@ import pytest
 from oracle import gpt_oracle as O
 from scratch_decoder_only_b200 import configs as CF
 from scratch_decoder_only_b200 import synthetic as S
-from tests.helpers import ocfg, per_tensor_rel_l2, rel
+from tests.helpers import ocfg, per_tensor_rel_l2, rel, tame_attention
 
 pytestmark = pytest.mark.gpu
 
@@ -123,6 +123,7 @@ def test_fp16_greedy_decode_against_oracle_logits(torch):
                         max_seq=64, max_batch=2, tied=False, precision="fp16", init_std=0.3)
     cfg = ocfg(mc)
     model = GPT(mc, 13)
+    tame_attention(model, cfg)
     rng = np.random.default_rng(42)
     Tp, n_new = 12, 16
     prompt = rng.integers(0, 1000, size=(2, Tp)).astype(np.int32)

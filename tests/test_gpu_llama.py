@@ -13,7 +13,7 @@ import pytest
 from oracle import gpt_oracle as O
 from scratch_decoder_only_b200 import configs as CF
 from scratch_decoder_only_b200 import synthetic as S
-from tests.helpers import ocfg, per_tensor_rel_l2, rel
+from tests.helpers import ocfg, tame_attention, per_tensor_rel_l2, rel
 
 pytestmark = pytest.mark.gpu
 
@@ -108,6 +108,7 @@ def test_llama_greedy_decode_against_oracle_logits(torch, B):
     mc = llama_cfg(max_seq=64, max_batch=12, init_std=0.3)
     cfg = ocfg(mc)
     model = GPT(mc, 14)
+    tame_attention(model, cfg)
     rng = np.random.default_rng(54 + B)
     Tp, n_new = 16, 20
     prompt = rng.integers(0, 1000, size=(B, Tp)).astype(np.int32)

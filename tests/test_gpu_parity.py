@@ -13,7 +13,7 @@ import pytest
 from oracle import gpt_oracle as O
 from scratch_decoder_only_b200 import configs as CF
 from scratch_decoder_only_b200 import synthetic as S
-from tests.helpers import ocfg, per_tensor_rel_l2, rel
+from tests.helpers import ocfg, per_tensor_rel_l2, rel, tame_attention
 
 pytestmark = pytest.mark.gpu
 
@@ -394,6 +394,7 @@ def test_greedy_decode_bf16_batched(torch):
                         max_seq=64, max_batch=12, tied=False, precision="bf16", init_std=0.3)
     cfg = ocfg(mc)
     model = new_model(mc, 11)
+    tame_attention(model, cfg)
     rng = np.random.default_rng(4)
     prompt = rng.integers(0, 512, size=(12, 10)).astype(np.int32)
     outs = [model.greedy_decode(dev(torch, prompt), 6).cpu().numpy(),

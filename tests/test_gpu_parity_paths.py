@@ -29,7 +29,7 @@ import pytest
 from oracle import gpt_oracle as O
 from scratch_decoder_only_b200 import configs as CF
 from scratch_decoder_only_b200 import synthetic as S
-from tests.helpers import ocfg, per_tensor_rel_l2, rel
+from tests.helpers import tame_attention, ocfg, per_tensor_rel_l2, rel
 
 pytestmark = pytest.mark.gpu
 
@@ -145,6 +145,7 @@ def test_greedy_decode_d64_bf16_against_oracle_logits(torch, B):
     attention over the cache at head size 64."""
     cfg = ocfg(DEC64)
     model = new_model(DEC64, 13)
+    tame_attention(model, cfg)
     rng = np.random.default_rng(30 + B)
     Tp, n_new = 16, 24
     prompt = rng.integers(0, DEC64.vocab, size=(B, Tp)).astype(np.int32)
