@@ -1,33 +1,32 @@
 // Flash attention on tcgen05 tensor cores (sm_100a), head size 64, causal
 // with the block-diagonal mask of packed documents (query i sees keys j with
 // dstart[i] <= j <= i).  Same layouts as the other attention kernels: qkv
-// [B*T, 3C], out / dout [B*T, C], lse / D [B, H, T].
+// [B*T, 3C] (or any column layout with the query, key and value heads at
+// given column offsets: grouped key/value heads), out / dout [B*T, C],
+// lse / D [B, H, T].
 //
-// Every kernel is a 192-thread CTA, warp-specialised like the GEMM:
+// Both kernels are warp-specialised, one CTA per SM (all 512 TMEM columns):
 //   warp 0     TMA producer (tiles of Q, K, V, dO with a 128-byte swizzle)
 //   warp 1     MMA issuer (one thread; tcgen05.mma kind::f16, M = 128)
-//   warps 2-5  elementwise warps: thread t owns accumulator row t (TMEM lane
-//              t); they read scores from TMEM, write P or dS to shared memory
-//              as the next MMA's operand, and run the epilogue.
-// A CTA works through its blocks one after another; latency is hidden by
-// running 2-3 CTAs per SM (each takes 128-256 TMEM columns, 64-96 KB smem).
+//   the rest   elementwise warps: thread t owns accumulator row t (TMEM lane
+//              t); they read scores from TMEM and write P (TMEM) or dS
+//              (shared memory) as the next MMA's operand.
 //
-//   forward  CTA = 128 queries, 64-key blocks: S = Q K^T (TMEM), P =
-//            exp2(S log2e / 8 - m) (smem), O_blk = P V (TMEM), accumulated in
-//            registers with the online-softmax correction; writes O, lse.
-//   dK / dV  CTA = 128 keys, 64-query blocks: S^T = K Q^T, dP^T = V dO^T
-//            (TMEM); P^T and dS^T = P^T (dP^T - D) (smem); dV += P^T dO and
-//            dK += dS^T Q accumulate in TMEM across query blocks.
-//   dQ       CTA = 128 queries, 64-key blocks: S, dP (TMEM); dS (smem);
-//            dQ += dS K in TMEM.
-// A 64-wide bf16 row is one 128-byte swizzle atom, so one shared-memory tile
-// serves as a K-major operand and as an MN-major one.  Blocks outside the
-// document ranges are skipped, not masked.
+//   forward   CTA = two 128-query tiles, 128-key blocks: S = Q K^T in one of
+//             three rotating TMEM buffers, P = exp2(S log2e / 8 - m) written
+//             back over S as 16-bit pairs, O += P V in TMEM (A from TMEM).
+//   backward  CTA = 128 keys, 128-query blocks: S^T = K Q^T, dP^T = V dO^T
+//             (TMEM); P^T (TMEM) and dS^T = P^T (dP^T - D) (smem); dV += P^T
+//             dO and dK += dS^T Q accumulate in TMEM across query blocks;
+//             dQ = dS K per block, added in fp32 to a global accumulator by
+//             TMA bulk reduce-add.
+// A 64-wide 16-bit row is one 128-byte swizzle atom, so one shared-memory
+// tile serves as a K-major operand and as an MN-major one.  Blocks outside
+// the document ranges are skipped, not masked.
 #include "tc_common.cuh"
 
 #define AT_D 64
 #define AT_BLK 128
-#define AT_THREADS 192
 #define AT_TILE_BYTES (AT_BLK * AT_D * 2)   // 16 KB: 128 rows x 128 B
 #define LOG2E_F 1.4426950408889634f
 #define LN2_F 0.6931471805599453f
@@ -162,16 +161,14 @@ __device__ __forceinline__ float fmax3f(float a, float b, float c) {
 }
 
 // One 32-score chunk of a row: fold the (masked) raw scores into mx
-// (three-input max), write P = exp2(s sl2 - mb) as 16 packed 16-bit pairs at
-// TMEM column tP and add their sum to sum.  Masked chunks keep key e (0..31)
-// when lo <= e <= hi (relative to the chunk), branch-free:
-// ((e - lo) | (hi - e)) >= 0.  The exponent arguments and the sums run as
-// packed fp32 pairs.
+// (three-input max), put P = exp2(s sl2 - mb) as 16 packed 16-bit pairs into
+// pw and add their sum to sum.  Masked chunks keep key e (0..31) when
+// lo <= e <= hi (relative to the chunk), branch-free: ((e - lo) | (hi - e))
+// >= 0.  The exponent arguments and the sums run as packed fp32 pairs.
 template <bool MASK, bool F16>
-__device__ __forceinline__ void fwd_chunk(const uint32_t* sr, int lo, int hi, float sl2, float mb, uint32_t tP,
+__device__ __forceinline__ void fwd_chunk(const uint32_t* sr, int lo, int hi, float sl2, float mb, uint32_t* pw,
                                           float& mx, float& sum) {
   float l0 = 0.f, l1 = 0.f;
-  uint32_t pw[16];
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
     float s0 = __uint_as_float(sr[e]), s1 = __uint_as_float(sr[e + 1]);
@@ -197,57 +194,143 @@ __device__ __forceinline__ void fwd_chunk(const uint32_t* sr, int lo, int hi, fl
     pw[e / 2] = pack16x2<F16>(p0, p1);
   }
   sum += l0 + l1;
-  tmem_st16(tP, pw);
 }
 
-// One pass over a row's 128 scores at tS (writing P at tP): four chunks of
-// 32, each chunk's TMEM load issued before the previous chunk's arithmetic
-// (tcgen05.wait::ld waits for every load in flight, so each wait covers a
-// load that had a chunk of arithmetic to land).  One code body per mask
-// variant keeps the score loop within the instruction cache.
+// One pass over a row's 128 scores at tS with the running max mb: four
+// chunks of 32, each chunk's TMEM load issued before the previous chunk's
+// arithmetic (tcgen05.wait::ld waits for every load in flight, so each wait
+// covers a load that had a chunk of arithmetic to land).  P of chunk c goes
+// over columns 16c..16c+15 of S, whose scores (chunk c/2) are already in
+// registers.  A chunk whose max exceeds thr (the running max + 2^8 in the
+// exp2 domain, voted warp-wide) stops the pass before its P is stored:
+// the return value is that chunk (4: none), and S of it and of every later
+// chunk is still intact.  sum collects the stored chunks' P.
 template <bool MASK, bool F16>
-__device__ __forceinline__ void fwd_pass(uint32_t tS, uint32_t tP, int lo, int hi, float sl2, float mb, float& mx,
-                                         float& sum) {
-  uint32_t ra[32], rb[32];
+__device__ __forceinline__ int fwd_pass(uint32_t tS, int lo, int hi, float sl2, float mb, float thr, float& mx,
+                                        float& sum) {
+  uint32_t ra[32], rb[32], pw[16];
   tmem_ld32(tS, ra);
   tmem_wait_ld();
-#pragma unroll 1
-  for (int c = 0; c < 4; c += 2) {
-    tmem_ld32(tS + 32 * (c + 1), rb);
-    fwd_chunk<MASK, F16>(ra, lo - 32 * c, hi - 32 * c, sl2, mb, tP + 16 * c, mx, sum);
-    tmem_wait_ld();
-    if (c + 2 < 4) tmem_ld32(tS + 32 * (c + 2), ra);
-    fwd_chunk<MASK, F16>(rb, lo - 32 * (c + 1), hi - 32 * (c + 1), sl2, mb, tP + 16 * (c + 1), mx, sum);
-    tmem_wait_ld();
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t* cur = (c & 1) ? rb : ra;
+    uint32_t* nxt = (c & 1) ? ra : rb;
+    if (c + 1 < 4) tmem_ld32(tS + 32 * (c + 1), nxt);
+    float csum = 0.f;
+    fwd_chunk<MASK, F16>(cur, lo - 32 * c, hi - 32 * c, sl2, mb, pw, mx, csum);
+    if (c + 1 < 4) tmem_wait_ld();
+    if (__any_sync(0xffffffffu, mx * sl2 > thr)) return c;
+    sum += csum;
+    tmem_st16(tS + 16 * c, pw);
   }
+  return 4;
+}
+
+// The rare continuation of a pass stopped at chunk ct (the block raised the
+// max past the threshold): the block max over the remaining chunks gives the
+// new running max m_new; the P already stored (chunks < ct, each <= 2^8) is
+// scaled by 2^(mb - m_new) in place (a power of two: exact unless it
+// underflows), and chunks ct..3 are exponentiated with m_new.  mb is the
+// max the stored P was computed with (0 where m_use is still -inf).
+template <bool MASK, bool F16>
+__device__ __noinline__ void fwd_raise(uint32_t tS, int lo, int hi, float sl2, float m_use, float mb, int ct,
+                                       float mx_before, float& m_new, float& sum) {
+  tmem_wait_st();   // the P of chunks < ct is read back below
+  float mx = mx_before;
+  for (int c = ct; c < 4; ++c) {
+    uint32_t ra[32];
+    tmem_ld32(tS + 32 * c, ra);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      float s0 = __uint_as_float(ra[e]);
+      if (MASK) s0 = ((e - (lo - 32 * c)) | ((hi - 32 * c) - e)) >= 0 ? s0 : -INFINITY;
+      mx = fmaxf(mx, s0);
+    }
+  }
+  m_new = fmaxf(m_use, mx * sl2);
+  // a row with no allowed key yet keeps m_new = -inf (all its P are 0)
+  const float mb_new = m_new == -INFINITY ? 0.f : m_new;
+  // no running max yet: the chunks already stored held no allowed key (any
+  // finite score stops the pass), so their P and sum are exactly 0
+  const float sc = m_use == -INFINITY ? 0.f : exp2f(mb - mb_new);
+  sum *= sc;
+  for (int c = 0; c < ct; ++c) {
+    uint32_t pw[16];
+    tmem_ld16(tS + 16 * c, pw);
+    tmem_wait_ld();
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float f[8];
+      unpack16x8<F16>(make_uint4(pw[4 * u], pw[4 * u + 1], pw[4 * u + 2], pw[4 * u + 3]), f);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) pw[4 * u + e] = pack16x2<F16>(f[2 * e] * sc, f[2 * e + 1] * sc);
+    }
+    tmem_st16(tS + 16 * c, pw);
+  }
+  for (int c = ct; c < 4; ++c) {
+    uint32_t ra[32], pw[16];
+    tmem_ld32(tS + 32 * c, ra);
+    tmem_wait_ld();
+    float dummy = -INFINITY;
+    fwd_chunk<MASK, F16>(ra, lo - 32 * c, hi - 32 * c, sl2, mb_new, pw, dummy, sum);
+    tmem_st16(tS + 16 * c, pw);
+  }
+}
+
+// The row's (masked) maximum score over a block, without exponentials: the
+// first block of a row sets the running max from it.
+template <bool MASK>
+__device__ __forceinline__ float fwd_max(uint32_t tS, int lo, int hi) {
+  uint32_t ra[32];
+  float mx = -INFINITY;
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {
+    tmem_ld32(tS + 32 * c, ra);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      float s0 = __uint_as_float(ra[e]), s1 = __uint_as_float(ra[e + 1]);
+      if (MASK) {
+        s0 = ((e - (lo - 32 * c)) | ((hi - 32 * c) - e)) >= 0 ? s0 : -INFINITY;
+        s1 = ((e + 1 - (lo - 32 * c)) | ((hi - 32 * c) - e - 1)) >= 0 ? s1 : -INFINITY;
+      }
+      mx = fmax3f(mx, s0, s1);
+    }
+  }
+  return mx;
 }
 
 // ============================================================== forward
 // CTA = two 128-query tiles (256 queries) sharing each 128-key block of K
 // and V.  Per tile g and key block j:
-//   S_g = Q_g K_j^T                (TMEM, 128 x 128 fp32)
-//   P_g = exp2(S_g log2e / 8 - m)  (bf16 pairs, TMEM columns beside O_g)
-//   O_g += P_g V_j                 (TMEM, 128 x 64 fp32, A operand from TMEM)
-// The MMA warp alternates between the tiles so that one tile's softmax runs
-// while the other tile's products are computed.  The running max m is only
-// raised (and O, l rescaled) when a row's block max exceeds it by more than
-// 2^8; otherwise the stale max is kept, which bounds every P by 256.  After a
-// row's first block, each half of the score row is read from TMEM once: the
-// exponentials use the running max while the block max is tracked, and only a
-// block whose max rose past the threshold is exponentiated again (S is still
-// intact, since P has its own columns).
+//   S = Q_g K_j^T                (TMEM, 128 x 128 fp32)
+//   P = exp2(S log2e / 8 - m)    (16-bit pairs, written over S's first 64 columns)
+//   O_g += P V_j                 (TMEM, 128 x 64 fp32, A operand from TMEM)
+// The (tile, key block) items run in the order (j, g); their score tiles
+// rotate through three TMEM buffers, so the MMA warp computes the next
+// items' S while the softmax warps work on the current ones and a tile's
+// softmax warps go from one block to the next without waiting for an MMA.
+// A buffer is reused three items later: its S MMA is issued after the P V
+// MMA that read its P (tcgen05.mma ops of one thread run in issue order).
+// The running max m is set by a row's first block (a max-only pass) and later
+// raised (O and l rescaled) only when a block's max exceeds it by more than
+// 2^8; otherwise the stale max is kept, which bounds every P by 256.  P is
+// held in registers until that check, so a block that does raise the max is
+// exponentiated again from S.
 // 320 threads: warp 0 loads, warp 1 issues MMAs, warps 2-5 (tile 0) and 6-9
 // (tile 1) run the softmax, thread t of a group owning query row t.
 #define FW_THREADS 320
 #define FW_QT 256                                    // queries per CTA
 #define FW_ST 3                                      // K / V stages
+#define FW_NB 3                                      // score buffers
 #define FW_RESCALE 8.0f                              // log2 of the largest tolerated P
 struct FwdSmem {
   static constexpr int Q = 0;                        // 2 tiles x 16 KB
   static constexpr int KV = Q + 2 * AT_TILE_BYTES;   // FW_ST stages x (K 16 KB, V 16 KB)
   static constexpr int BAR = KV + FW_ST * 2 * AT_TILE_BYTES;
   static constexpr int TOTAL = BAR + 256;
-  static constexpr int TMEM_COLS = 512;              // tile g: S at 256g, O at 256g + 128, P at 256g + 192
+  static constexpr int TMEM_COLS = 512;              // O_g at 64 g; score buffer k at 128 + 128 k
 };
 
 template <bool F16>
@@ -257,8 +340,10 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
   extern __shared__ __align__(1024) uint8_t at_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)at_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = (uint64_t*)(sm + FwdSmem::BAR);
-  enum { Q_FULL = 0, KV_FULL = 1, KV_EMPTY = 1 + FW_ST, S_FULL = 1 + 2 * FW_ST, P_FULL = S_FULL + 2,
-         O_DONE = P_FULL + 2, DRAIN = O_DONE + 2, NBARS = DRAIN + 1 };
+  // O_DONE + 2 g + (m & 1): P V of tile g's m-th block complete (two barriers
+  // per tile, alternating, so that a waiter is never two phases behind)
+  enum { Q_FULL = 0, KV_FULL = 1, KV_EMPTY = 1 + FW_ST, S_FULL = 1 + 2 * FW_ST, P_FULL = S_FULL + FW_NB,
+         O_DONE = P_FULL + FW_NB, DRAIN = O_DONE + 4, NBARS = DRAIN + 1 };
   uint32_t* tmem_slot = (uint32_t*)(bars + NBARS);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   int* s_info = (int*)(tmem_slot + 2);
@@ -274,6 +359,8 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
   const int q0 = qt * FW_QT;
   const long rowbase = (long)b * T;
   const int* dsr = dstart + rowbase;
+  griddep_wait();
+  griddep_release();
 
   if (threadIdx.x == 0) {
     mbar_init(bar(Q_FULL), 1);
@@ -281,11 +368,11 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
       mbar_init(bar(KV_FULL + i), 1);
       mbar_init(bar(KV_EMPTY + i), 1);
     }
-    for (int g = 0; g < 2; ++g) {
-      mbar_init(bar(S_FULL + g), 1);
-      mbar_init(bar(P_FULL + g), 4);
-      mbar_init(bar(O_DONE + g), 1);
+    for (int k = 0; k < FW_NB; ++k) {
+      mbar_init(bar(S_FULL + k), 1);
+      mbar_init(bar(P_FULL + k), 4);
     }
+    for (int k = 0; k < 4; ++k) mbar_init(bar(O_DONE + k), 1);
     mbar_init(bar(DRAIN), 1);
     *abort_flag = 0;
     // key blocks of each tile: from its first query's document start to its last query
@@ -304,8 +391,18 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
   const uint32_t tmem = *tmem_slot;
   const int lo0 = s_info[0], hi0 = s_info[1], lo1 = s_info[2], hi1 = s_info[3];
   const bool two = q0 + 128 < T;          // the second tile has queries
-  const int jlo = lo0, jhi = two ? hi1 : hi0;
+  const int jlo = lo0, jhi = two ? hi1 : hi0;   // document starts and last queries never decrease
   auto in_tile = [&](int g, int j) { return g == 0 ? (j >= lo0 && j <= hi0) : (two && j >= lo1 && j <= hi1); };
+  // items (tile g, block j) in (j, g) order: the index of (g, j) and the total
+  auto blocks_before = [&](int g, int j) {
+    if (g == 1 && !two) return 0;
+    const int lo_ = g ? lo1 : lo0, e = min(j, (g ? hi1 : hi0) + 1);
+    return e > lo_ ? e - lo_ : 0;
+  };
+  auto item_of = [&](int g, int j) {
+    return blocks_before(0, j) + blocks_before(1, j) + ((g == 1 && in_tile(0, j)) ? 1 : 0);
+  };
+  const int n_items = blocks_before(0, jhi + 1) + blocks_before(1, jhi + 1);
 
   if (warp == 0 && lane == 0) {
     // ---------------- producer
@@ -328,49 +425,58 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
     const int nj = jhi - jlo + 1;
     for (int n = max(0, nj - FW_ST); n < nj; ++n) mbar_wait(bar(KV_FULL + n % FW_ST), (n / FW_ST) & 1, &never, 1ll << 28);
   } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer: S_0(j+1) is issued right after P_0 V(j), then P_1 V(j), S_1(j+1)
+    // ---------------- MMA issuer: S of item i + FW_NB is issued right after P V of item i
     constexpr uint32_t ID_S = instr_desc_t(F16, 128, false, false);   // S = Q K^T: 128 x 128, K = 64
     constexpr uint32_t ID_O = instr_desc_t(F16, 64, false, true);     // O = P V: 128 x 64, K = 128 keys (V MN-major)
     bool ok = mbar_wait(bar(Q_FULL), 0, abort_flag);
-    int ns[2] = {0, 0}, np[2] = {0, 0};   // S and P V products issued per tile
-    auto kv_wait = [&](int j) {
-      const int n = j - jlo;
-      return mbar_wait(bar(KV_FULL + n % FW_ST), (n / FW_ST) & 1, abort_flag);
+    int np0 = 0, np1 = 0;   // P V products issued per tile
+    // item iterators: (g, j) of the next S and the next P V
+    auto advance = [&](int& g, int& j) {
+      do {
+        if (g == 0) g = 1;
+        else { g = 0; ++j; }
+      } while (j <= jhi && !in_tile(g, j));
     };
-    auto issue_s = [&](int g, int j) -> bool {
-      if (!in_tile(g, j)) return true;
-      // the softmax has turned the previous S into P (and P V was issued before this)
-      if (ns[g] > 0 && !mbar_wait(bar(P_FULL + g), (ns[g] - 1) & 1, abort_flag)) return false;
+    int sg = 0, sj = jlo, pg = 0, pj = jlo;
+    if (!in_tile(0, jlo)) { advance(sg, sj); advance(pg, pj); }
+    auto issue_s = [&](int i, int g, int j) -> bool {
+      const int n = j - jlo;
+      if (!mbar_wait(bar(KV_FULL + n % FW_ST), (n / FW_ST) & 1, abort_flag)) return false;
       tc_fence_after();
-      const uint32_t sK = sKV + ((j - jlo) % FW_ST) * 2 * AT_TILE_BYTES, q = sQ + g * AT_TILE_BYTES;
+      const uint32_t sK = sKV + (n % FW_ST) * 2 * AT_TILE_BYTES, q = sQ + g * AT_TILE_BYTES;
+      const uint32_t d = tmem + 128 + 128 * (i % FW_NB);
 #pragma unroll
-      for (int k = 0; k < AT_D / 16; ++k)
-        umma_bf16(tmem + 256 * g, kdesc(q + k * 32), kdesc(sK + k * 32), ID_S, k > 0);
-      umma_commit(bar(S_FULL + g));
-      ++ns[g];
+      for (int k = 0; k < AT_D / 16; ++k) umma_bf16(d, kdesc(q + k * 32), kdesc(sK + k * 32), ID_S, k > 0);
+      umma_commit(bar(S_FULL + i % FW_NB));
       return true;
     };
-    auto issue_pv = [&](int g, int j) -> bool {
-      if (!in_tile(g, j)) return true;
-      if (!mbar_wait(bar(P_FULL + g), np[g] & 1, abort_flag)) return false;
+    int is = 0;
+    for (; is < FW_NB && is < n_items && ok; ++is) {
+      ok = issue_s(is, sg, sj);
+      advance(sg, sj);
+    }
+    for (int i = 0; i < n_items && ok; ++i) {
+      // P V of item i, once its softmax has written P
+      if (!mbar_wait(bar(P_FULL + i % FW_NB), (i / FW_NB) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t sV = sKV + ((j - jlo) % FW_ST) * 2 * AT_TILE_BYTES + AT_TILE_BYTES;
+      const int n = pj - jlo;
+      const uint32_t sV = sKV + (n % FW_ST) * 2 * AT_TILE_BYTES + AT_TILE_BYTES;
+      const uint32_t pbuf = tmem + 128 + 128 * (i % FW_NB);
 #pragma unroll
       for (int kk = 0; kk < AT_BLK / 16; ++kk)
-        umma_bf16_ts(tmem + 256 * g + 128, tmem + 256 * g + 192 + 8 * kk, mndesc(sV + kk * 2048, 8192), ID_O,
-                     (np[g] > 0 || kk > 0));
-      umma_commit(bar(O_DONE + g));
-      ++np[g];
-      return true;
-    };
-    if (ok && jlo <= jhi) ok = kv_wait(jlo) && issue_s(0, jlo) && issue_s(1, jlo);
-    for (int j = jlo; j <= jhi && ok; ++j) {
-      const bool next = j + 1 <= jhi;
-      if (!issue_pv(0, j)) { ok = false; break; }
-      if (next && !(kv_wait(j + 1) && issue_s(0, j + 1))) { ok = false; break; }
-      if (!issue_pv(1, j)) { ok = false; break; }
-      umma_commit(bar(KV_EMPTY + (j - jlo) % FW_ST));   // K / V of block j no longer read
-      if (next && !issue_s(1, j + 1)) { ok = false; break; }
+        umma_bf16_ts(tmem + 64 * pg, pbuf + 8 * kk, mndesc(sV + kk * 2048, 8192), ID_O,
+                     ((pg ? np1 : np0) > 0 || kk > 0));
+      umma_commit(bar(O_DONE + 2 * pg + ((pg ? np1 : np0) & 1)));
+      if (pg) ++np1;
+      else ++np0;
+      const int pj_done = pj;
+      advance(pg, pj);
+      if (pj != pj_done) umma_commit(bar(KV_EMPTY + n % FW_ST));   // K / V of block pj_done no longer read
+      if (is < n_items) {
+        if (!issue_s(is, sg, sj)) { ok = false; break; }
+        advance(sg, sj);
+        ++is;
+      }
     }
     if (!ok) trap_timeout(abort_flag, err);
     umma_commit(bar(DRAIN));
@@ -389,67 +495,73 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
     const int lo = g == 0 ? lo0 : lo1, hi = g == 0 ? hi0 : hi1;
     const int qlast = min(q0 + 128 * g + 127, T - 1);
     const int ds_last = ld_once(dsr + qlast);
-    const uint32_t tS = tmem + 256 * g + ((uint32_t)(quarter * 32) << 16), tO = tS + 128, tP = tS + 192;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tO = tmem + lane_off + 64 * g;
     const float sl2 = 0.125f * LOG2E_F;   // 1/sqrt(64) in the exp2 domain
     auto wait_w = [&](uint32_t bb, uint32_t parity) { return __all_sync(0xffffffffu, mbar_wait(bb, parity, abort_flag)); };
+    // wait until P V of this tile's m-th block has completed.  Called for m
+    // in increasing order, each m at a point where P V of block m - 2 has been
+    // waited for and P V of block m + 2 cannot have been issued, so the
+    // barrier is within one phase of the one asked for.
+    auto wait_pv = [&](int m) { return wait_w(bar(O_DONE + 2 * g + (m & 1)), (m >> 1) & 1); };
     float m_use = -INFINITY, l = 0.f;
     bool ok = true;
     int n = 0;
     if (g == 0 || two) {
       for (int j = lo; j <= hi; ++j, ++n) {
-        if (!wait_w(bar(S_FULL + g), n & 1)) { ok = false; break; }
+        if (n >= 2 && !wait_pv(n - 2)) { ok = false; break; }
+        const int it = item_of(g, j);
+        const uint32_t tS = tmem + lane_off + 128 + 128 * (it % FW_NB);
+        if (!wait_w(bar(S_FULL + it % FW_NB), (it / FW_NB) & 1)) { ok = false; break; }
         tc_fence_after();
         const int kb0 = j * AT_BLK;
         // masked blocks: a key may be later than a query or before its document
         // (voted warp-wide so the warp runs one code path)
         const bool need_mask = __any_sync(0xffffffffu, kb0 + AT_BLK - 1 > q0 + 128 * g || ds_last > kb0 || !qv);
         const int lo_h = ds_q - kb0, hi_h = q - kb0;   // allowed keys relative to the block
-        // exponentiate with the running max while tracking the block max; a
-        // block whose max rose more than 2^FW_RESCALE above the running one
-        // (always the row's first block, whose running max is -inf) raises
-        // it, rescales O and l, and is exponentiated again (S is intact: P
-        // has its own columns)
-        float bsum, mx;
-        float mb = m_use == -INFINITY ? 0.f : m_use;
-        while (true) {
-          bsum = 0.f;
-          mx = -INFINITY;
-          if (need_mask) fwd_pass<true, F16>(tS, tP, lo_h, hi_h, sl2, mb, mx, bsum);
-          else fwd_pass<false, F16>(tS, tP, lo_h, hi_h, sl2, mb, mx, bsum);
-          mx *= sl2;
-          if (!__any_sync(0xffffffffu, mx > m_use + FW_RESCALE)) break;
-          const float m_new = fmaxf(m_use, mx);
-          if (n > 0) {
-            // O holds P V of every earlier block: wait for the last one, then scale it
-            const float sc = m_use == -INFINITY ? 0.f : exp2f(m_use - m_new);
-            if (!wait_w(bar(O_DONE + g), (n - 1) & 1)) { ok = false; break; }
-            tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < 2; ++c) {
-              uint32_t orr[32];
-              tmem_ld32(tO + 32 * c, orr);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * sc);
-              tmem_st32(tO + 32 * c, orr);
-            }
-            l *= sc;
-          }
-          m_use = m_new;
-          mb = m_use == -INFINITY ? 0.f : m_use;
-          tmem_wait_st();   // the first P of this block is replaced by the next pass
+        if (n == 0) {
+          // the row's first block sets the running max (no O or l to rescale yet)
+          const float m0 = (need_mask ? fwd_max<true>(tS, lo_h, hi_h) : fwd_max<false>(tS, lo_h, hi_h)) * sl2;
+          m_use = m0;
         }
-        if (!ok) break;
+        float bsum = 0.f, mx = -INFINITY;
+        const float mb = m_use == -INFINITY ? 0.f : m_use;
+        const float thr = m_use + FW_RESCALE;
+        const int ct = need_mask ? fwd_pass<true, F16>(tS, lo_h, hi_h, sl2, mb, thr, mx, bsum)
+                                 : fwd_pass<false, F16>(tS, lo_h, hi_h, sl2, mb, thr, mx, bsum);
+        if (ct < 4) {
+          // this block raised the max past the threshold (never the first
+          // block): finish it with the new max, then scale O (P V of the
+          // earlier blocks: wait for the last one) and l
+          float m_new;
+          if (need_mask) fwd_raise<true, F16>(tS, lo_h, hi_h, sl2, m_use, mb, ct, mx, m_new, bsum);
+          else fwd_raise<false, F16>(tS, lo_h, hi_h, sl2, m_use, mb, ct, mx, m_new, bsum);
+          const float sc = m_use == -INFINITY ? 0.f : exp2f(m_use - m_new);
+          if (!wait_pv(n - 1)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
+            uint32_t orr[32];
+            tmem_ld32(tO + 32 * c, orr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * sc);
+            tmem_st32(tO + 32 * c, orr);
+          }
+          l *= sc;
+          m_use = m_new;
+        }
         l += bsum;
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(P_FULL + g));
+        if (lane == 0) mbar_arrive(bar(P_FULL + it % FW_NB));
       }
     }
     if (!ok) trap_timeout(abort_flag, err);
-    // O / l for the row, after the last P V
-    if (ok && n > 0 && wait_w(bar(O_DONE + g), (n - 1) & 1)) {
+    // O / l for the row, after the last P V (and the one before it, in order)
+    if (ok && n >= 2) ok = wait_pv(n - 2);
+    if (ok && n > 0 && wait_pv(n - 1)) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       bf16* orow = out + (rowbase + q) * C + h * AT_D;
@@ -579,6 +691,8 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
   const int* dsr = dstart + rowbase;
   const int nqb = (T + BW_QB - 1) / BW_QB;
   const int qb_lo = k0 / BW_QB;
+  griddep_wait();
+  griddep_release();
 
   if (threadIdx.x == 0) {
     mbar_init(bar(KV_FULL), 1);
@@ -867,6 +981,8 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
 // dq[row, head h] = bf16 or fp16 (F16) of dQacc / 8; the accumulator is cleared for the next use.
 template <bool F16>
 __global__ void attn_dq_finish_kernel(float* __restrict__ dq_acc, bf16* __restrict__ dqkv, long rows, int C, long ld_q) {
+  griddep_wait();
+  griddep_release();
   const long n8 = rows * C / 8;
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n8; i += (long)gridDim.x * blockDim.x) {
     const long e = i * 8, row = e / C;
@@ -933,8 +1049,8 @@ static cudaError_t attn_fwd_tc_t(const bf16* qkv, bf16* out, float* lse, const i
   if (!attr) { cudaError_t e = tc_smem_attr(attn_fwd_tc<F16>, smem); if (e) return e; attr = true; }
   dim3 grid(B * H, (T + FW_QT - 1) / FW_QT);
   ++g_kernel_launches;
-  attn_fwd_tc<F16><<<grid, FW_THREADS, smem, s>>>(tqkv, out, lse, dstart, T, H, L.kcol, L.vcol, L.G, err);
-  return cudaGetLastError();
+  return launch_k(attn_fwd_tc<F16>, grid, dim3(FW_THREADS), smem, s, tqkv, out, lse, dstart, T, H, L.kcol, L.vcol, L.G,
+                  err);
 }
 
 static bool layout_ok(const AttnLayout& L, int H) {
@@ -978,12 +1094,11 @@ static cudaError_t attn_bwd_tc_t(const bf16* qkv, const bf16* out, const bf16* d
   }
   dim3 grid(B * H, (T + AT_BLK - 1) / AT_BLK);
   ++g_kernel_launches;
-  attn_bwd_tc<F16><<<grid, BW_THREADS, smem, s>>>(tqkv, tdo, tdq, lse, Dbuf, dstart, T, H, L.kcol, L.vcol, L.G,
-                                                  L.dkv, L.ld_kv, L.v_off, err);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  e = launch_k(attn_bwd_tc<F16>, grid, dim3(BW_THREADS), smem, s, tqkv, tdo, tdq, lse, Dbuf, dstart, T, H, L.kcol, L.vcol,
+               L.G, L.dkv, L.ld_kv, L.v_off, err);
+  if (e != cudaSuccess) return e;
   ++g_kernel_launches;
-  attn_dq_finish_kernel<F16><<<148 * 8, 256, 0, s>>>(dq_acc, dqkv, rows, C, (long)L.qw);
-  return cudaGetLastError();
+  return launch_k(attn_dq_finish_kernel<F16>, dim3(148 * 8), dim3(256), 0, s, dq_acc, dqkv, rows, C, (long)L.qw);
 }
 
 cudaError_t launch_attn_bwd_tc(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* Dbuf,

@@ -106,7 +106,13 @@ __device__ __forceinline__ float gelu_grad_f(float u) {
 // griddep_release() lets the successor start launching.
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-extern bool g_pdl;   // set while the decode step is captured: its launches overlap their predecessors
+// Every kernel launched through launch_k (and the tensor-core GEMM) calls
+// griddep_wait() before it touches global memory that another kernel writes,
+// so each may be launched with programmatic dependent launch: its blocks are
+// scheduled, and its set-up runs, while the previous kernel drains.  The
+// chain stays ordered because every kernel waits for its predecessor, which
+// waited for its own.  g_pdl (default on) turns the launch attribute on.
+extern bool g_pdl;
 template <typename... KArgs, typename... Args>
 static cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
   if (!g_pdl) {

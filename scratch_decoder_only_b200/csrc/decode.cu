@@ -217,13 +217,15 @@ cudaError_t launch_kv_fill(const T* qkv, T* kc, T* vc, int B, int Tp, int d, int
   return cudaGetLastError();
 }
 
-// Split decode attention: grid (B*H, DA_SPLITS); block (bh, sp) takes keys
-// sp, sp + DA_SPLITS, ... in chunks of DA_CHUNK and keeps an online softmax
-// (max, sum, output) per 8-lane group, each lane holding 8 of the head's
-// dimensions (one 16-byte load of a key or value row).  Its partial
-// (m, l, o[D]) goes to part[bh][sp]; dec_attn_combine merges the splits.
-// The new key / value of this step are read from qkv, and written to the
-// cache by split 0.
+// Split decode attention: grid (B*H, DA_SPLITS); the first `act` splits
+// of a (row, head) take the keys (act grows with the context, one split per
+// 64 keys, so that a short context is not spread over mostly idle blocks);
+// block (bh, sp < act) takes key groups sp, sp + act, ... and keeps an online
+// softmax (max, sum, output) per 8-lane group, each lane holding 8 of the
+// head's dimensions (one 16-byte load of a key or value row).  Its partial
+// (m, l, o[D]) goes to part[bh][sp]; splits past act write an empty partial.
+// dec_attn_combine merges the splits.  The new key / value of this step are
+// read from qkv, and written to the cache by split 0.
 #define DA_SPLITS 16
 #define DA_THREADS 128
 template <typename T>
@@ -247,6 +249,7 @@ dec_attn_split_kernel(const T* __restrict__ qkv, T* kc, T* vc, float* __restrict
   const int bh = blockIdx.x, sp = blockIdx.y;
   const int b = bh / H, h = bh % H;
   const int G = H / Ly.Hkv, hk = h / G;   // query head h reads key/value head hk
+  const int act = min(DA_SPLITS, pos / 64 + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = lane / LPK, sub = lane % LPK;
   const T* q = qkv + (long)b * Ly.qw + h * D;
@@ -266,8 +269,9 @@ dec_attn_split_kernel(const T* __restrict__ qkv, T* kc, T* vc, float* __restrict
   float m = -INFINITY, l = 0.f, o[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) o[i] = 0.f;
-  // key j belongs to this split when (j / KPW) % (DA_SPLITS * NW) == sp * NW + warp
-  for (int j0 = (sp * NW + warp) * KPW; j0 <= pos; j0 += DA_SPLITS * NW * KPW) {
+  // key j belongs to this split when (j / KPW) % (act * NW) == sp * NW + warp
+  // (no key at all for sp >= act: the partial stays empty)
+  for (int j0 = sp < act ? (sp * NW + warp) * KPW : pos + 1; j0 <= pos; j0 += act * NW * KPW) {
     const int j = j0 + grp;
     const bool live = j <= pos;
     long row = (long)j * D;

@@ -18,8 +18,9 @@
 //                 output projection (+ bias + residual)
 //              D  LN2 (every CTA), 16-row units of fc (+ bias, GELU)
 //              E  row units of fc2 (+ bias + residual)
-//   then       F  final LN (every CTA), 32-row chunks of the LM head (fp32
-//                 logits) with a per-CTA argmax; after the barrier every CTA
+//   then       F  final LN (every CTA), 16-row chunks of the LM head (fp32
+//                 logits, four chunks in flight) with a per-CTA argmax;
+//                 after the barrier every CTA
 //                 reduces the per-CTA maxima (lowest index on ties) into the
 //                 next token and embeds it for the next step.
 //
@@ -28,6 +29,10 @@
 // (cp.async.bulk, completion on an mbarrier) issued before it waits at the
 // barrier, so the weight stream overlaps the barrier, and it asks L2 to
 // prefetch its share of the next layer's weights at the start of a layer.
+// LayerNorm gamma / beta and the bias rows of the CTA's units travel the
+// same way into two small parameter areas, one phase ahead.  The key-range
+// partials of phase B are merged by the CTAs of phase C that need the
+// attention rows (no atomics, no fences).
 // Rounding points are those of the training forward: the residual stream,
 // LN outputs, q/k/v, the attention output, u and GELU(u) are bf16; all dot
 // products, LN statistics and the softmax are fp32; the logits are fp32.
@@ -42,6 +47,8 @@
 #define DF_WBUF (48 * 1024)             // bytes of each of the two weight buffers
 #define DF_MAX_SPLITS 16
 #define DF_BAR_LIMIT (1ll << 31)         // clock cycles (about a second)
+#define DF_PRM_BIAS 256                  // bias floats of one CTA's units in one phase (at most)
+#define DF_PRM(C) (2 * (C) + DF_PRM_BIAS)  // floats of one parameter area
 
 // DecFusedParams is declared in launch.h.
 
@@ -82,12 +89,29 @@ __device__ __forceinline__ bool df_grid_sync(const DecFusedParams& p, unsigned k
   return *s_flag == 0;
 }
 
+// Bounded wait for an mbarrier phase by one thread: the global abort word is
+// read only every 64 polls (every thread of every CTA reading it on each
+// poll made one L2 line a hot spot and delayed each wake-up by a round trip).
+__device__ __forceinline__ bool df_mbar_wait(uint32_t bar, uint32_t parity, const unsigned* abortf) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (unsigned it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63) == 0) {
+      if (*(volatile const unsigned*)abortf) return false;
+      if (clock64() - t0 > DF_BAR_LIMIT) return false;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ weight buffers
+// Two 48 KB buffers (slots 0 and 1); the LM-head phase splits them into four
+// 24 KB slots, slot s at buffer s & 1, half s >> 1.  Slot s completes on bar[s].
 struct WBufs {
   uint8_t* buf[2];
-  uint32_t bar[2];
-  uint32_t parity[2];
-  int inflight[2];   // a queued copy not yet waited for (same value in every thread)
+  uint32_t bar[4];
+  uint32_t parity[4];
+  int inflight[4];   // a queued copy not yet waited for (same value in every thread)
 };
 
 // Thread 0 queues `n` contiguous byte ranges into buffer `i` (total <= DF_WBUF);
@@ -101,9 +125,11 @@ __device__ __forceinline__ void wbuf_copy(uint32_t dst, const void* src, uint32_
                ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
                : "memory");
 }
-// Every thread of the CTA calls this; the outcome is the same in all of them.
+// Every thread of the CTA calls this; thread 0 waits and the block barrier
+// hands the data to the others; the outcome is the same in all of them.
 __device__ __forceinline__ bool wbuf_wait(WBufs& w, int i, const DecFusedParams& p) {
-  const bool ok = mbar_wait(w.bar[i], w.parity[i], (volatile int*)p.abortf, DF_BAR_LIMIT);
+  int ok = 1;
+  if (threadIdx.x == 0) ok = df_mbar_wait(w.bar[i], w.parity[i], p.abortf);
   if (!__syncthreads_or(!ok)) {
     w.parity[i] ^= 1u;
     w.inflight[i] = 0;
@@ -119,7 +145,7 @@ __device__ __forceinline__ bool wbuf_wait(WBufs& w, int i, const DecFusedParams&
 // copies still in flight into this CTA's shared memory.
 __device__ __forceinline__ void wbuf_drain(WBufs& w) {
   volatile int never = 0;
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < 4; ++i)
     if (w.inflight[i]) mbar_wait(w.bar[i], w.parity[i], &never, 1ll << 28);
 }
 
@@ -133,6 +159,7 @@ __device__ __forceinline__ float bfr(float v) { return __bfloat162float(__float2
 
 // LayerNorm of BB rows of C fp32 values in smem `x` into smem `y` (bf16-rounded
 // values kept as fp32), one warp per row; two-pass statistics as in training.
+// g and b are in shared memory (staged by a bulk copy one phase ahead).
 template <int BB>
 __device__ __forceinline__ void df_layernorm(const float* x, float* y, const float* g, const float* b, int B, int C,
                                              float eps) {
@@ -145,7 +172,7 @@ __device__ __forceinline__ void df_layernorm(const float* x, float* y, const flo
     float q = 0.f;
     for (int c = lane; c < C; c += 32) { const float d = xr[c] - mu; q += d * d; }
     const float rs = 1.0f / sqrtf(warp_sum(q) / C + eps);
-    for (int c = lane; c < C; c += 32) y[r * C + c] = bfr((xr[c] - mu) * rs * __ldg(g + c) + __ldg(b + c));
+    for (int c = lane; c < C; c += 32) y[r * C + c] = bfr((xr[c] - mu) * rs * g[c] + b[c]);
   }
 }
 
@@ -201,7 +228,8 @@ __device__ __forceinline__ void df_load_rows(const bf16* src, float* dst, int B,
 template <int BB>
 __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const DecFusedParams p) {
   extern __shared__ __align__(128) uint8_t df_smem[];
-  __shared__ __align__(8) uint64_t wbars[2];
+  __shared__ __align__(8) uint64_t wbars[4];
+  __shared__ __align__(8) uint64_t pbars[2];
   __shared__ int s_flag;
   __shared__ float s_rv[DF_WARPS][BB];
   __shared__ int s_ri[DF_WARPS][BB];
@@ -215,13 +243,23 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const DecFu
   float* xs = reinterpret_cast<float*>(df_smem + 2 * DF_WBUF);   // [BB][C] residual row (bf16 values)
   float* xm = xs + BB * C;                                        // [BB][C] x_mid
   float* xin = xm + BB * C;                                       // [BB][KX] projection input
-  wb.bar[0] = smem_u32(&wbars[0]);
-  wb.bar[1] = smem_u32(&wbars[1]);
-  wb.parity[0] = wb.parity[1] = 0;
-  wb.inflight[0] = wb.inflight[1] = 0;
+  // two parameter areas of DF_PRM(C) floats: LayerNorm gamma and beta (2C),
+  // then the bias slices of the CTA's units, staged one phase ahead
+  float* prm[2];
+  prm[0] = xin + BB * (C > F ? C : F);
+  prm[1] = prm[0] + DF_PRM(C);
+  uint32_t pbar[2] = {smem_u32(&pbars[0]), smem_u32(&pbars[1])};
+  uint32_t ppar[2] = {0u, 0u};
+  int pinf[2] = {0, 0};
+  for (int i = 0; i < 4; ++i) {
+    wb.bar[i] = smem_u32(&wbars[i]);
+    wb.parity[i] = 0;
+    wb.inflight[i] = 0;
+  }
   if (threadIdx.x == 0) {
-    mbar_init(wb.bar[0], 1);
-    mbar_init(wb.bar[1], 1);
+    for (int i = 0; i < 4; ++i) mbar_init(wb.bar[i], 1);
+    mbar_init(pbar[0], 1);
+    mbar_init(pbar[1], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (threadIdx.x < BB) s_tok[threadIdx.x] = threadIdx.x < B ? __ldcg(p.tok + threadIdx.x) : 0;
@@ -232,8 +270,11 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const DecFu
   const int nu_qkv = 3 * C / 16, nu_o = C / 16, nu_fc = F / 16;
   int rows_e = DF_WBUF / (F * 2);
   if (rows_e > 16) rows_e = 16;
+  rows_e &= ~3;   // bias slices of whole 16-byte groups
   const int nu_e = (C + rows_e - 1) / rows_e;
-  const int n_head = (p.Vp + 31) / 32;
+  int hr = (DF_WBUF / 2) / (2 * C);   // LM-head rows per 24 KB chunk
+  if (hr > 16) hr = 16;
+  const int n_head = (p.Vp + hr - 1) / hr;
   const int S = p.S, nu_att = B * H * S;
   const float* P32 = p.p32;
   const bf16* PW = p.pw;
@@ -265,9 +306,46 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const DecFu
     return cnt;
   };
   auto lw = [&](long off0, int l) -> long { return off0 + (long)l * p.l_stride; };
+  // queue parameter area k: gamma and beta (2C contiguous floats at ln, or
+  // none) and the bias rows of this CTA's units (rows_per_unit each)
+  auto issue_params = [&](int k, long ln, long bias, int nunits, int rows_per_unit, int nrows) {
+    pinf[k] = 1;
+    if (threadIdx.x == 0) {
+      uint32_t total = ln >= 0 ? (uint32_t)(2 * C * 4) : 0u;
+      for (int u = cta; u < nunits; u += G) total += (uint32_t)min(rows_per_unit, nrows - u * rows_per_unit) * 4;
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_expect_tx(pbar[k], total);
+      uint32_t off = 0;
+      if (ln >= 0) {
+        wbuf_copy(smem_u32(prm[k]), P32 + ln, (uint32_t)(2 * C * 4), pbar[k]);
+        off = (uint32_t)(2 * C * 4);
+      }
+      for (int u = cta; u < nunits; u += G) {
+        const int r0 = u * rows_per_unit;
+        const uint32_t bytes = (uint32_t)min(rows_per_unit, nrows - r0) * 4;
+        wbuf_copy(smem_u32(prm[k]) + off, P32 + bias + r0, bytes, pbar[k]);
+        off += bytes;
+      }
+    }
+  };
+  auto wait_params = [&](int k) -> bool {
+    int ok = 1;
+    if (threadIdx.x == 0) ok = df_mbar_wait(pbar[k], ppar[k], p.abortf);
+    if (__syncthreads_or(!ok)) {
+      if (threadIdx.x == 0) {
+        atomicOr(p.err, GPT_DEVERR_TIMEOUT);
+        atomicExch(p.abortf, 1u);
+      }
+      return false;
+    }
+    ppar[k] ^= 1u;
+    pinf[k] = 0;
+    return true;
+  };
 
-  // weights of layer 0's qkv units go first
+  // weights and parameters of layer 0's phase A go first
   int pend_a = issue_units(0, PW + lw(p.l_w_qkv, 0), nu_qkv, 16, 3 * C, C);
+  issue_params(0, lw(p.l_ln1_g, 0), lw(p.l_b_qkv, 0), nu_qkv, 16, 3 * C);
   int pend_c = 0, pend_d = 0, pend_e = 0;
 
   for (int st = 0; st < p.n_steps; ++st) {
@@ -297,23 +375,25 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const DecFu
         }
       }
       // ---- phase A: LN1, qkv units
-      df_layernorm<BB>(xs, xin, P32 + lw(p.l_ln1_g, l), P32 + lw(p.l_ln1_b, l), B, C, p.eps);
+      if (!wait_params(0)) goto abort;
+      df_layernorm<BB>(xs, xin, prm[0], prm[0] + C, B, C, p.eps);
       __syncthreads();
       if (pend_a) {
         if (!wbuf_wait(wb, 0, p)) goto abort;
-        const float* bq = P32 + lw(p.l_b_qkv, l);
+        const float* bq = prm[0] + 2 * C;
         int slot = 0;
         for (int u = cta; u < nu_qkv; u += G, ++slot) {
           const int r0 = u * 16;
           df_project<BB>(reinterpret_cast<const bf16*>(wb.buf[0]) + (long)slot * 16 * C, 16, C, xin, C, B,
                          [&](int r, int b, float y) {
-                           p.qkv[(long)b * 3 * C + r0 + r] = __float2bfloat16_rn(y + bq[r0 + r]);
+                           p.qkv[(long)b * 3 * C + r0 + r] = __float2bfloat16_rn(y + bq[slot * 16 + r]);
                          });
         }
       }
       __syncthreads();
-      // the out-projection's weights can move while the barrier and attention run
+      // the out-projection's weights and bias can move while the barrier and attention run
       pend_c = issue_units(1, PW + lw(p.l_w_o, l), nu_o, 16, C, C);
+      issue_params(1, -1, lw(p.l_b_o, l), nu_o, 16, C);
       if (!df_grid_sync(p, ++nbar, &s_flag)) goto abort;
 
       // ---- phase B: attention units (row b, head h, key range s)
@@ -404,40 +484,8 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const DecFu
               ll += sm[w2 * (D + 2) + 1] * f;
               oo += sm[w2 * (D + 2) + 2 + threadIdx.x] * f;
             }
-            if (S == 1) {
-              p.att[(long)b * C + h * D + threadIdx.x] = __float2bfloat16_rn(oo / ll);
-            } else {
-              dst[2 + threadIdx.x] = oo;
-              if (threadIdx.x == 0) { dst[0] = mm; dst[1] = ll; }
-            }
-          }
-          if (S > 1) {
-            // the last split of (b, h) to finish merges all S partials into att
-            __syncthreads();
-            if (threadIdx.x == 0) {
-              __threadfence();
-              s_flag = atomicAdd(p.cnt + bh, 1) == S - 1;
-            }
-            __syncthreads();
-            if (s_flag) {
-              __threadfence();
-              const float* pp = p.part + (long)bh * S * (D + 2);
-              for (int i = threadIdx.x; i < S * (D + 2); i += DF_THREADS) sm[i] = __ldcg(pp + i);
-              __syncthreads();
-              if (threadIdx.x < D) {
-                float mm = -INFINITY;
-                for (int s2 = 0; s2 < S; ++s2) mm = fmaxf(mm, sm[s2 * (D + 2)]);
-                float ll = 0.f, oo = 0.f;
-                for (int s2 = 0; s2 < S; ++s2) {
-                  const float ms = sm[s2 * (D + 2)];
-                  const float f = ms == -INFINITY ? 0.f : __expf(ms - mm);
-                  ll += sm[s2 * (D + 2) + 1] * f;
-                  oo += sm[s2 * (D + 2) + 2 + threadIdx.x] * f;
-                }
-                p.att[(long)b * C + h * D + threadIdx.x] = __float2bfloat16_rn(oo / ll);
-              }
-              if (threadIdx.x == 0) p.cnt[bh] = 0;   // ready for the next layer
-            }
+            dst[2 + threadIdx.x] = oo;
+            if (threadIdx.x == 0) { dst[0] = mm; dst[1] = ll; }
           }
           __syncthreads();
         }
@@ -445,54 +493,83 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const DecFu
       if (!df_grid_sync(p, ++nbar, &s_flag)) goto abort;
 
       // ---- phase C: out-projection units over the merged attention rows
+      if (!wait_params(1)) goto abort;
       if (pend_c) {
-        df_load_rows(p.att, xin, B, C);
+        // merge the key-range partials of every (row, head) into the
+        // attention rows: partials into shared memory (buffer 0 is free in
+        // this phase), then one output element per thread
+        {
+          float* ps = reinterpret_cast<float*>(wb.buf[0]);
+          const int npart = B * H * S * (D + 2), np4 = npart / 4;
+          for (int i = threadIdx.x; i < np4; i += DF_THREADS)
+            reinterpret_cast<float4*>(ps)[i] = __ldcg(reinterpret_cast<const float4*>(p.part) + i);
+          for (int i = np4 * 4 + threadIdx.x; i < npart; i += DF_THREADS) ps[i] = __ldcg(p.part + i);
+          __syncthreads();
+          for (int i = threadIdx.x; i < B * C; i += DF_THREADS) {
+            const int bh = i / D, d = i % D;
+            const float* pp = ps + (long)bh * S * (D + 2);
+            float mm = -INFINITY;
+            for (int s2 = 0; s2 < S; ++s2) mm = fmaxf(mm, pp[s2 * (D + 2)]);
+            float ll = 0.f, oo = 0.f;
+            for (int s2 = 0; s2 < S; ++s2) {
+              const float ms = pp[s2 * (D + 2)];
+              const float f = ms == -INFINITY ? 0.f : __expf(ms - mm);
+              ll += pp[s2 * (D + 2) + 1] * f;
+              oo += pp[s2 * (D + 2) + 2 + d] * f;
+            }
+            xin[i] = bfr(oo / ll);   // the attention output is rounded to bf16 as in training
+          }
+        }
         __syncthreads();
         if (!wbuf_wait(wb, 1, p)) goto abort;
-        const float* bo = P32 + lw(p.l_b_o, l);
+        const float* bo = prm[1];
         int slot = 0;
         for (int u = cta; u < nu_o; u += G, ++slot) {
           const int r0 = u * 16;
           df_project<BB>(reinterpret_cast<const bf16*>(wb.buf[1]) + (long)slot * 16 * C, 16, C, xin, C, B,
                          [&](int r, int b, float y) {
                            const int n = r0 + r;
-                           p.xmid[(long)b * C + n] = __float2bfloat16_rn(y + bo[n] + xs[b * C + n]);
+                           p.xmid[(long)b * C + n] = __float2bfloat16_rn(y + bo[slot * 16 + r] + xs[b * C + n]);
                          });
         }
       }
       __syncthreads();
       pend_d = issue_units(0, PW + lw(p.l_w_fc, l), nu_fc, 16, F, C);
+      issue_params(0, lw(p.l_ln2_g, l), lw(p.l_b_fc, l), nu_fc, 16, F);
       if (!df_grid_sync(p, ++nbar, &s_flag)) goto abort;
 
       // ---- phase D: LN2, fc units (u and GELU(u))
       df_load_rows(p.xmid, xm, B, C);
       __syncthreads();
-      df_layernorm<BB>(xm, xin, P32 + lw(p.l_ln2_g, l), P32 + lw(p.l_ln2_b, l), B, C, p.eps);
+      if (!wait_params(0)) goto abort;
+      df_layernorm<BB>(xm, xin, prm[0], prm[0] + C, B, C, p.eps);
       __syncthreads();
       if (pend_d) {
         if (!wbuf_wait(wb, 0, p)) goto abort;
-        const float* bf = P32 + lw(p.l_b_fc, l);
+        const float* bf = prm[0] + 2 * C;
         int slot = 0;
         for (int u = cta; u < nu_fc; u += G, ++slot) {
           const int r0 = u * 16;
           df_project<BB>(reinterpret_cast<const bf16*>(wb.buf[0]) + (long)slot * 16 * C, 16, C, xin, C, B,
                          [&](int r, int b, float y) {
                            const int n = r0 + r;
-                           const float uq = bfr(y + bf[n]);
+                           const float uq = bfr(y + bf[slot * 16 + r]);
                            p.abuf[(long)b * F + n] = __float2bfloat16_rn(gelu_f(uq));
                          });
         }
       }
       __syncthreads();
       pend_e = issue_units(1, PW + lw(p.l_w_fc2, l), nu_e, rows_e, C, F);
+      issue_params(1, -1, lw(p.l_b_fc2, l), nu_e, rows_e, C);
       if (!df_grid_sync(p, ++nbar, &s_flag)) goto abort;
 
       // ---- phase E: fc2 units (+ bias + residual)
+      if (!wait_params(1)) goto abort;
       if (pend_e) {
         df_load_rows(p.abuf, xin, B, F);
         __syncthreads();
         if (!wbuf_wait(wb, 1, p)) goto abort;
-        const float* b2 = P32 + lw(p.l_b_fc2, l);
+        const float* b2 = prm[1];
         int slot = 0;
         for (int u = cta; u < nu_e; u += G, ++slot) {
           const int r0 = u * rows_e;
@@ -500,12 +577,17 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const DecFu
           df_project<BB>(reinterpret_cast<const bf16*>(wb.buf[1]) + (long)slot * rows_e * F, rr, F, xin, F, B,
                          [&](int r, int b, float y) {
                            const int n = r0 + r;
-                           p.xbuf[(long)b * C + n] = __float2bfloat16_rn(y + b2[n] + xm[b * C + n]);
+                           p.xbuf[(long)b * C + n] = __float2bfloat16_rn(y + b2[slot * rows_e + r] + xm[b * C + n]);
                          });
         }
       }
       __syncthreads();
-      if (l + 1 < p.NL) pend_a = issue_units(0, PW + lw(p.l_w_qkv, l + 1), nu_qkv, 16, 3 * C, C);
+      if (l + 1 < p.NL) {
+        pend_a = issue_units(0, PW + lw(p.l_w_qkv, l + 1), nu_qkv, 16, 3 * C, C);
+        issue_params(0, lw(p.l_ln1_g, l + 1), lw(p.l_b_qkv, l + 1), nu_qkv, 16, 3 * C);
+      } else {
+        issue_params(0, p.o_lnf_g, 0, 0, 1, 1);   // the final LayerNorm's gamma and beta
+      }
       if (!df_grid_sync(p, ++nbar, &s_flag)) goto abort;
       df_load_rows(p.xbuf, xs, B, C);
       __syncthreads();
@@ -513,7 +595,8 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const DecFu
 
     // ---- phase F: final LN, LM head chunks with a per-CTA argmax
     {
-      df_layernorm<BB>(xs, xin, P32 + p.o_lnf_g, P32 + p.o_lnf_b, B, C, p.eps);
+      if (!wait_params(0)) goto abort;
+      df_layernorm<BB>(xs, xin, prm[0], prm[0] + C, B, C, p.eps);
       float bv[BB];
       int bi[BB];
 #pragma unroll
@@ -530,32 +613,33 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const DecFu
           if (len >= 8) l2_prefetch(PW + p.l_ln1_g + o, (uint32_t)(len & ~7L) * 2);
         }
       }
-      // chunk k of this CTA is head chunk cta + k * G, in buffer k & 1
+      // chunk k of this CTA is head chunk cta + k * G (hr rows), in slot k & 3:
+      // four 24 KB chunks in flight
       int nk = 0;
       for (int c2 = cta; c2 < n_head; c2 += G) ++nk;
+      auto slot_ptr = [&](int sl) { return wb.buf[sl & 1] + (sl >> 1) * (DF_WBUF / 2); };
       auto issue_chunk = [&](int k) {
-        const int ch = cta + k * G;
-        const int r0 = ch * 32, rr = min(32, p.Vp - r0);
-        wb.inflight[k & 1] = 1;
+        const int ch = cta + k * G, sl = k & 3;
+        const int r0 = ch * hr, rr = min(hr, p.Vp - r0);
+        wb.inflight[sl] = 1;
         if (threadIdx.x == 0) {
-          wbuf_issue_begin(wb, k & 1, (uint32_t)rr * C * 2);
-          wbuf_copy(smem_u32(wb.buf[k & 1]), Wh + (long)r0 * C, (uint32_t)rr * C * 2, wb.bar[k & 1]);
+          wbuf_issue_begin(wb, sl, (uint32_t)rr * C * 2);
+          wbuf_copy(smem_u32(slot_ptr(sl)), Wh + (long)r0 * C, (uint32_t)rr * C * 2, wb.bar[sl]);
         }
       };
       __syncthreads();
-      if (nk > 0) issue_chunk(0);
-      if (nk > 1) issue_chunk(1);
+      for (int k = 0; k < 4 && k < nk; ++k) issue_chunk(k);
       for (int k = 0; k < nk; ++k) {
         const int ch = cta + k * G;
-        const int r0 = ch * 32, rr = min(32, p.Vp - r0);
-        if (!wbuf_wait(wb, k & 1, p)) goto abort;
-        df_project<BB>(reinterpret_cast<const bf16*>(wb.buf[k & 1]), rr, C, xin, C, B, [&](int r, int b, float y) {
+        const int r0 = ch * hr, rr = min(hr, p.Vp - r0);
+        if (!wbuf_wait(wb, k & 3, p)) goto abort;
+        df_project<BB>(reinterpret_cast<const bf16*>(slot_ptr(k & 3)), rr, C, xin, C, B, [&](int r, int b, float y) {
           const int n = r0 + r;
           p.logits[(long)b * p.Vp + n] = y;
           if (n < p.V && (y > bv[b] || (y == bv[b] && n < bi[b]))) { bv[b] = y; bi[b] = n; }
         });
         __syncthreads();
-        if (k + 2 < nk) issue_chunk(k + 2);
+        if (k + 4 < nk) issue_chunk(k + 4);
       }
       // per-CTA maxima (lane 0 of every warp holds its own)
       if (lane == 0) {
@@ -577,8 +661,12 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const DecFu
       }
       __syncthreads();
       // the next step's (or the next layer 0's) qkv weights
-      if (st + 1 < p.n_steps) pend_a = issue_units(0, PW + lw(p.l_w_qkv, 0), nu_qkv, 16, 3 * C, C);
-      else pend_a = 0;
+      if (st + 1 < p.n_steps) {
+        pend_a = issue_units(0, PW + lw(p.l_w_qkv, 0), nu_qkv, 16, 3 * C, C);
+        issue_params(0, lw(p.l_ln1_g, 0), lw(p.l_b_qkv, 0), nu_qkv, 16, 3 * C);
+      } else {
+        pend_a = 0;
+      }
       if (!df_grid_sync(p, ++nbar, &s_flag)) goto abort;
       // every CTA reduces the maxima: warp b takes row b
       if (warp < B) {
@@ -612,6 +700,11 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const DecFu
 abort:
   // leave with no bulk copy in flight into this CTA's shared memory
   wbuf_drain(wb);
+  {
+    volatile int never = 0;
+    for (int k = 0; k < 2; ++k)
+      if (pinf[k]) mbar_wait(pbar[k], ppar[k], &never, 1ll << 28);
+  }
 }
 
 // ------------------------------------------------------------------ host side
@@ -646,22 +739,27 @@ bool dec_fused_supported(int B, int C, int H, int F, int Vp) {
   if (per_cta(3 * C / 16) * 16L * C * 2 > DF_WBUF) return false;   // qkv
   if (per_cta(C / 16) * 16L * C * 2 > DF_WBUF) return false;       // out-projection
   if (per_cta(F / 16) * 16L * C * 2 > DF_WBUF) return false;       // fc
-  if (32L * C * 2 > DF_WBUF) return false;                          // head chunks
+  if ((DF_WBUF / 2) / (2L * C) < 1) return false;                   // head chunks of at least a row
   long rows_e = DF_WBUF / (F * 2L);
-  if (rows_e < 1) return false;
   if (rows_e > 16) rows_e = 16;
+  rows_e &= ~3L;
+  if (rows_e < 4) return false;
   if (per_cta((C + rows_e - 1) / rows_e) * rows_e * F * 2 > DF_WBUF) return false;   // fc2
+  // bias slices of one CTA's units in one parameter area
+  if (per_cta(3 * C / 16) * 16 > DF_PRM_BIAS || per_cta(F / 16) * 16 > DF_PRM_BIAS ||
+      per_cta(C / 16) * 16 > DF_PRM_BIAS || per_cta((C + rows_e - 1) / rows_e) * rows_e > DF_PRM_BIAS)
+    return false;
   const int KX = C > F ? C : F;
   if (DF_WARPS * (D + 2) > KX) return false;                        // attention partials in xin
-  if (df_splits(B, H) * (D + 2) > KX) return false;                 // the merge of a head's splits in xin
-  const size_t smem = 2 * DF_WBUF + (size_t)4 * (2 * 4 * C + 4 * KX);
+  if ((long)B * H * df_splits(B, H) * (D + 2) * 4 > DF_WBUF) return false;   // the partials in buffer 0
+  const size_t smem = 2 * DF_WBUF + (size_t)4 * (2 * 4 * C + 4 * KX + 2 * DF_PRM(C));
   return smem <= 227 * 1024;
 }
 
 cudaError_t launch_decode_fused(const DecFusedParams& prm, cudaStream_t s) {
   const int BB = prm.B <= 1 ? 1 : prm.B <= 2 ? 2 : 4;
   const int KX = prm.C > prm.F ? prm.C : prm.F;
-  const size_t smem = 2 * DF_WBUF + (size_t)4 * (2 * BB * prm.C + BB * KX);
+  const size_t smem = 2 * DF_WBUF + (size_t)4 * (2 * BB * prm.C + BB * KX + 2 * DF_PRM(prm.C));
   void* fn = BB == 1 ? (void*)decode_fused_kernel<1> : BB == 2 ? (void*)decode_fused_kernel<2>
                                                                  : (void*)decode_fused_kernel<4>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -368,7 +368,7 @@ static int build_arena(gpt_model* m) {
   cv.add((void**)&m->drs, Bx * 4);
   cv.add((void**)&m->dtok, Bx * 4);
   cv.add((void**)&m->dpart, dec_attn_part_floats((int)Bx, m->H, m->d) * 4);
-  cv.add((void**)&m->dam, Bx * DF_MAX_GRID * 8 + Bx * m->H * 4);   // argmax partials, then split counters
+  cv.add((void**)&m->dam, Bx * DF_MAX_GRID * 8);   // fused decode: per-CTA argmax partials
   cv.add((void**)&m->dsrc, Bx * (size_t)m->Tmax * 4);
   cv.add((void**)&m->dbcs, Bx * BEAM_MAX_WIDTH * 4);
   cv.add((void**)&m->dbct, Bx * BEAM_MAX_WIDTH * 4);
@@ -891,18 +891,15 @@ static int backward_llama(gpt_model* m) {
 // Greedy decoding
 // ---------------------------------------------------------------------------
 // One projection of a decode step: y = x W^T with the gemv epilogue `mode`
-// (0: + bias + residual, 1: u = + bias and gelu(u), 2: fp32 logits).  A batch
-// of more than 8 rows runs on the tensor-core GEMM (rows past B are zero
-// tiles), fewer rows on the GEMV that streams each weight row once.
+// (0: + bias + residual, 1: u = + bias and gelu(u), 2: fp32 logits).  Up to 8
+// rows run on the GEMV that streams each weight row once; 9-32 rows (16-bit)
+// on the mma.sync kernel that spreads 16-row weight slices over every SM.
 template <typename T>
 static cudaError_t dec_proj(gpt_model* m, const T* X, int B, int K, const T* W, int N, const float* bias,
                             const T* resid, int mode, T* out, T* out2, float* outf, cudaStream_t s) {
   if constexpr (sizeof(T) == 2) {
-    if (B > 8 && gemm_tc_supported(B, N, K, K, false, K, false)) {
-      EpiParams<T> e = mode == 2 ? epi_f32<T>(outf, N)
-                                 : mode == 1 ? epi_gelu<T>(out, out2, N, bias) : epi_store<T>(out, N, bias, resid, N);
-      return tc_gemm<T>(B, N, K, X, K, false, W, K, false, e, 1, &m->sc->err, s);
-    }
+    if (B > 8 && dec_mma_supported(B, K, N))
+      return launch_dec_mma<T>(X, B, K, W, N, bias, resid, mode, out, out2, outf, &m->sc->err, s);
   }
   return launch_gemv<T>(X, B, K, W, N, bias, resid, mode, out, out2, outf, s);
 }
@@ -1029,11 +1026,8 @@ static int decode_impl(gpt_model* m, const int32_t* prompt, int B, int Tp, int n
       q.tok = m->dtok; q.out = out; q.out_ld = n_new; q.out_col0 = 1;
       q.qkv = (bf16*)m->dq; q.part = m->dpart; q.xmid = (bf16*)m->dh; q.abuf = (bf16*)m->da; q.xbuf = (bf16*)m->dx;
       q.logits = m->dlogits; q.am_v = m->dam; q.am_i = (int*)(m->dam + (size_t)m->Bmax * DF_MAX_GRID);
-      q.cnt = (int*)(m->dam + (size_t)m->Bmax * DF_MAX_GRID * 2);
-      q.att = (bf16*)m->datt;
       q.bar = &m->sc->dec_bar; q.abortf = &m->sc->dec_abort; q.err = &m->sc->err;
       CK(cudaMemsetAsync(&m->sc->dec_bar, 0, 2 * sizeof(unsigned), s));
-      CK(cudaMemsetAsync(q.cnt, 0, (size_t)B * H * sizeof(int), s));
       CK(launch_decode_fused(q, s));
       return GPT_OK;
     }
@@ -1054,9 +1048,7 @@ static int decode_impl(gpt_model* m, const int32_t* prompt, int B, int Tp, int n
     cudaGraph_t g = nullptr;
     unsigned long long n0 = g_kernel_launches;
     CK(cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
-    g_pdl = true;   // each captured kernel may start while its predecessor drains
     int r = decode_step<T>(m, Bd, Tp, n_new, out, m->cap_stream);
-    g_pdl = false;
     cudaError_t ec = cudaStreamEndCapture(m->cap_stream, &g);
     if (r != GPT_OK) { if (g) cudaGraphDestroy(g); return r; }
     CK(ec);

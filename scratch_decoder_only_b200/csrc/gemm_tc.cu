@@ -205,6 +205,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   if constexpr (CG == 2) cluster_sync_all();   // both CTAs' barriers exist before any remote arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the set-up above overlaps the previous kernel's tail; operands, side
+  // inputs and outputs are touched only after it has completed
+  griddep_wait();
+  griddep_release();
 
   constexpr int TM = TC_BM * CG;   // output rows per work unit
   const int tiles_m = (M + TM - 1) / TM, tiles_n = (N + BN - 1) / BN;
@@ -542,24 +546,28 @@ static cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const
   const int slots = g_sms / CG;
   const int grid = CG * (units < slots ? units : slots);
   ++g_kernel_launches;
-  if constexpr (CG == 1) {
-    kern<<<grid, TC_THREADS, Cfg::SMEM, s>>>(ta, tb, tc, tc2, M, N, K, splits, epi, err);
-    return cudaGetLastError();
-  } else {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid, 1, 1);
-    cfg.blockDim = dim3(TC_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = Cfg::SMEM;
-    cfg.stream = s;
-    cudaLaunchAttribute la[1];
-    la[0].id = cudaLaunchAttributeClusterDimension;
-    la[0].val.clusterDim.x = 2;
-    la[0].val.clusterDim.y = 1;
-    la[0].val.clusterDim.z = 1;
-    cfg.attrs = la;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, tc2, M, N, K, splits, epi, err);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(TC_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute la[2];
+  int na = 0;
+  if constexpr (CG == 2) {
+    la[na].id = cudaLaunchAttributeClusterDimension;
+    la[na].val.clusterDim.x = 2;
+    la[na].val.clusterDim.y = 1;
+    la[na].val.clusterDim.z = 1;
+    ++na;
   }
+  if (g_pdl) {   // the prologue may overlap the previous kernel's tail (the kernel waits before any access)
+    la[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    la[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = la;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, tc2, M, N, K, splits, epi, err);
 }
 
 // The (layout, epilogue) combinations the training step and the stand-alone

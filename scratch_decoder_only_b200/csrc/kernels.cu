@@ -7,7 +7,7 @@
 #include "tc_common.cuh"
 
 unsigned long long g_kernel_launches = 0;
-bool g_pdl = false;
+bool g_pdl = true;
 
 #define LN_MAXC 1024   // largest d_model the register-resident LayerNorm handles
 
@@ -21,6 +21,8 @@ __global__ void __launch_bounds__(1024) prep_kernel(const int32_t* __restrict__ 
                                                     const int32_t* __restrict__ seg, int B, int T, int V,
                                                     int* tok_out, int* tgt_out, int* pos_out, int* dstart_out,
                                                     DevScalars* sc) {
+  griddep_wait();
+  griddep_release();
   // one block per row; the document start of t is the largest run start <= t
   // (an inclusive max-scan of "t if a document starts at t"), carried across
   // chunks of blockDim.x positions
@@ -117,8 +119,8 @@ cudaError_t launch_prep(const int32_t* tokens, const int32_t* targets, const int
   }
   int th = T >= 1024 ? 1024 : ((T + 31) / 32) * 32;
   ++g_kernel_launches;
-  prep_kernel<<<B, th, 0, s>>>(tokens, targets, seg, B, T, V, tok_out, tgt_out, pos_out, dstart_out, sc);
-  return cudaGetLastError();
+  return launch_k(prep_kernel, dim3(B), dim3(th), 0, s,
+                  tokens, targets, seg, B, T, V, tok_out, tgt_out, pos_out, dstart_out, sc);
 }
 
 // ---------------------------------------------------------------------------
@@ -129,6 +131,8 @@ template <typename T>
 __global__ void embed_fwd_kernel(const int* __restrict__ tok, const int* __restrict__ pos,
                                  const float* __restrict__ wte, const float* __restrict__ wpe,
                                  T* __restrict__ x, int M, int C) {
+  griddep_wait();
+  griddep_release();
   int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   int lane = threadIdx.x & 31;
   if (row >= M) return;
@@ -155,8 +159,7 @@ template <typename T>
 cudaError_t launch_embed_fwd(const int* tok, const int* pos, const float* wte, const float* wpe, T* x,
                              int M, int C, cudaStream_t s) {
   ++g_kernel_launches;
-  embed_fwd_kernel<T><<<(M + 7) / 8, 256, 0, s>>>(tok, pos, wte, wpe, x, M, C);
-  return cudaGetLastError();
+  return launch_k(embed_fwd_kernel<T>, dim3((M + 7) / 8), dim3(256), 0, s, tok, pos, wte, wpe, x, M, C);
 }
 
 // ---------------------------------------------------------------------------
@@ -419,6 +422,8 @@ __global__ void __launch_bounds__(LNB2_THREADS, 2)
 ln_bwd2_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __restrict__ mean,
                const float* __restrict__ rstd, const float* __restrict__ g, const float* dres_in, float* dres_out,
                T* __restrict__ dres_out_t, float* __restrict__ partials, int M, int C, int TPR, int G, int rms) {
+  griddep_wait();
+  griddep_release();
   constexpr int NV = Vec<T>::N;
   __shared__ float2 slot[2][LNB2_THREADS / 32];
   const int grp = threadIdx.x / TPR, t = threadIdx.x % TPR;
@@ -540,9 +545,8 @@ cudaError_t launch_ln_bwd(const T* dy, const T* x, const float* mean, const floa
         attr = smem;
       }
       ++g_kernel_launches;
-      ln_bwd2_kernel<T><<<nblk, G * tpr, smem, s>>>(dy, x, mean, rstd, g, dres_in, dres_out, dres_out_t, partials, M,
-                                                    C, tpr, G, rms ? 1 : 0);
-      return cudaGetLastError();
+      return launch_k(ln_bwd2_kernel<T>, dim3(nblk), dim3(G * tpr), smem, s,
+                      dy, x, mean, rstd, g, dres_in, dres_out, dres_out_t, partials, M, C, tpr, G, rms ? 1 : 0);
     }
   }
   if (rms) return cudaErrorNotSupported;   // the register-row form has no RMSNorm variant
@@ -568,6 +572,8 @@ cudaError_t launch_ln_bwd(const T* dy, const T* x, const float* mean, const floa
 // A block takes 128 columns of one segment: 32 column quads x 8 row groups,
 // row group g summing rows g, g+8, ...; the groups are then added in order.
 __global__ void __launch_bounds__(256) reduce_segs_kernel(RedSegList L) {
+  griddep_wait();
+  griddep_release();
   __shared__ float red[8][129];
   int si = 0;
   while (si + 1 < L.n && (int)blockIdx.x >= L.seg[si + 1].blk0) ++si;
@@ -613,8 +619,7 @@ cudaError_t launch_reduce_segs(const RedSeg* segs, int n, bool add, cudaStream_t
     }
     if (blk == 0) continue;
     ++g_kernel_launches;
-    reduce_segs_kernel<<<blk, 256, 0, s>>>(L);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_k(reduce_segs_kernel, dim3(blk), dim3(256), 0, s, L);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -664,6 +669,8 @@ __global__ void __launch_bounds__(256) colsum_kernel(const Tin* __restrict__ x, 
 template <typename T16>
 __global__ void __launch_bounds__(256) colsum16_kernel(const T16* __restrict__ x, long ldx, int M, int N,
                                                        float* __restrict__ partials) {
+  griddep_wait();
+  griddep_release();
   __shared__ float red[8][257];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c0 = blockIdx.x * 256 + lane * 8;
@@ -709,8 +716,7 @@ cudaError_t launch_colsum(const Tin* x, long ldx, int M, int N, float* partials,
       dim3 g2((N + 255) / 256, (M + CS2_ROWS - 1) / CS2_ROWS);
       *rows_out = (int)g2.y;
       ++g_kernel_launches;
-      colsum16_kernel<Tin><<<g2, 256, 0, s>>>(x, ldx, M, N, partials);
-      return cudaGetLastError();
+      return launch_k(colsum16_kernel<Tin>, g2, dim3(256), 0, s, x, ldx, M, N, partials);
     }
   }
   dim3 grid((N + 127) / 128, (M + CS_ROWS - 1) / CS_ROWS);
@@ -875,6 +881,8 @@ template <typename T16>
 __global__ void __launch_bounds__(XB_THREADS, 2)
 xent_bulk_kernel(T16* __restrict__ logits, long ldl, const int* __restrict__ tgt, int V, int Vp,
                  float* __restrict__ rowloss, DevScalars* __restrict__ sc) {
+  griddep_wait();
+  griddep_release();
   extern __shared__ __align__(128) uint8_t xb_raw[];
   __shared__ float red[33];
   __shared__ __align__(8) uint64_t bar;
@@ -967,8 +975,7 @@ cudaError_t launch_xent(T* logits, long ldl, const int* tgt, int M, int V, int V
         attr = bytes;
       }
       ++g_kernel_launches;
-      xent_bulk_kernel<T><<<M, XB_THREADS, bytes, s>>>(logits, ldl, tgt, V, Vp, rowloss, sc);
-      return cudaGetLastError();
+      return launch_k(xent_bulk_kernel<T>, dim3(M), dim3(XB_THREADS), bytes, s, logits, ldl, tgt, V, Vp, rowloss, sc);
     }
   }
   size_t smem = (size_t)((Vp + NV - 1) / NV) * NV * sizeof(T);
@@ -990,6 +997,8 @@ cudaError_t launch_xent(T* logits, long ldl, const int* tgt, int M, int V, int V
 }
 
 __global__ void loss_finalize_kernel(const float* __restrict__ rowloss, int M, DevScalars* sc, float* loss_out) {
+  griddep_wait();
+  griddep_release();
   __shared__ float red[32];
   float acc = 0.f;
   for (int i = threadIdx.x; i < M; i += blockDim.x) acc += rowloss[i];
@@ -1010,8 +1019,7 @@ __global__ void loss_finalize_kernel(const float* __restrict__ rowloss, int M, D
 
 cudaError_t launch_loss_finalize(const float* rowloss, int M, DevScalars* sc, float* loss_out, cudaStream_t s) {
   ++g_kernel_launches;
-  loss_finalize_kernel<<<1, 1024, 0, s>>>(rowloss, M, sc, loss_out);
-  return cudaGetLastError();
+  return launch_k(loss_finalize_kernel, dim3(1), dim3(1024), 0, s, rowloss, M, sc, loss_out);
 }
 
 // ---------------------------------------------------------------------------
@@ -1021,6 +1029,8 @@ cudaError_t launch_loss_finalize(const float* rowloss, int M, DevScalars* sc, fl
 template <typename T>
 __global__ void embed_bwd_kernel(const float* __restrict__ dres, const int* __restrict__ tok,
                                  const int* __restrict__ pos, float* gwte, float* gwpe, int M, int C) {
+  griddep_wait();
+  griddep_release();
   // one warp per row; the row's fp32 gradient is loaded whole (up to 8
   // 16-byte vectors per lane in flight), then added into the token's and the
   // position's gradient rows with 16-byte vector atomics (a row's additions
@@ -1049,8 +1059,7 @@ template <typename T>
 cudaError_t launch_embed_bwd(const float* dres, const int* tok, const int* pos, float* gwte, float* gwpe,
                              int M, int C, cudaStream_t s) {
   ++g_kernel_launches;
-  embed_bwd_kernel<T><<<(M + 7) / 8, 256, 0, s>>>(dres, tok, pos, gwte, gwpe, M, C);
-  return cudaGetLastError();
+  return launch_k(embed_bwd_kernel<T>, dim3((M + 7) / 8), dim3(256), 0, s, dres, tok, pos, gwte, gwpe, M, C);
 }
 
 // ---------------------------------------------------------------------------

@@ -193,6 +193,14 @@ cudaError_t launch_sample(const float* logits, int B, int V, int Vp, float temp,
 template <typename T>
 cudaError_t launch_gather_last(const T* x, int B, int Tp, int C, T* out, cudaStream_t s);
 
+// ---- decode_mma.cu: decode projections of 9-32 rows on mma.sync (16-bit T),
+// same modes and outputs as the GEMV (0: + bias + residual, 1: + bias and
+// GELU into out / out2, 2: fp32 logits)
+bool dec_mma_supported(int B, int K, int N);
+template <typename T>
+cudaError_t launch_dec_mma(const T* X, int B, int K, const T* W, int N, const float* bias, const T* resid, int mode,
+                           T* out, T* out2, float* outf, unsigned* err, cudaStream_t s);
+
 // ---- beam.cu: beam search over the decode rows (row r = b * W + w)
 #define BEAM_MAX_WIDTH 8
 // scores[b W + w] = 0 for w = 0, -inf otherwise; src rows of every beam of
@@ -252,8 +260,6 @@ struct DecFusedParams {
   int out_ld, out_col0;
   bf16* qkv;               // [B][3C]
   float* part;             // [B*H][S][D+2] attention partials
-  int* cnt;                // [B*H] splits finished per (row, head) (zero at launch)
-  bf16* att;               // [B][C] merged attention output
   bf16* xmid;              // [B][C]
   bf16* abuf;              // [B][F]
   bf16* xbuf;              // [B][C]
