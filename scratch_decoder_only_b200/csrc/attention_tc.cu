@@ -154,6 +154,19 @@ __device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& y0, floa
 #define FW_POLY_PAIRS 0
 #endif
 
+// Optional: exponentials two at a time with ex2.approx.f16x2 on fp16 pairs of
+// arguments (at most 2^8 under the lazy running max; the row sums stay fp32).
+// Off by default: measured slower than two fp32 ex2 (the pair costs the MUFU
+// the same, and the conversions cost issue slots) and less accurate.
+#ifndef FW_EXP16
+#define FW_EXP16 0
+#endif
+__device__ __forceinline__ uint32_t ex2_f16x2(uint32_t a) {
+  uint32_t d;
+  asm("ex2.approx.f16x2 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+
 __device__ __forceinline__ float fmax3f(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -180,6 +193,15 @@ __device__ __forceinline__ void fwd_chunk(const uint32_t* sr, int lo, int hi, fl
     float x0, x1;
     fma_x2(x0, x1, s0, s1, sl2, -mb);
     float p0, p1;
+    if constexpr (FW_EXP16) {
+      const uint32_t e2 = ex2_f16x2(pack16x2<true>(x0, x1));
+      const float2 pf = __half22float2(*reinterpret_cast<const __half2*>(&e2));
+      p0 = pf.x;
+      p1 = pf.y;
+      add_x2(l0, l1, p0, p1);
+      pw[e / 2] = F16 ? e2 : pack16x2<false>(p0, p1);
+      continue;
+    }
     if (((e >> 1) & 7) < FW_POLY_PAIRS) {
       exp2_poly_x2(x0, x1, p0, p1);
       if (MASK) {   // the polynomial maps -inf to a tiny value, not 0
@@ -340,9 +362,13 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
   extern __shared__ __align__(1024) uint8_t at_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)at_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = (uint64_t*)(sm + FwdSmem::BAR);
+  // Parity waits need the waiter within one phase of the barrier, so
+  // S_FULL + 2 k + g: S of tile g's items in buffer k (a barrier per tile:
+  // a tile's first item can sit several items into the sequence, behind
+  // the other tile's uses of the same buffer);
   // O_DONE + 2 g + (m & 1): P V of tile g's m-th block complete (two barriers
   // per tile, alternating, so that a waiter is never two phases behind)
-  enum { Q_FULL = 0, KV_FULL = 1, KV_EMPTY = 1 + FW_ST, S_FULL = 1 + 2 * FW_ST, P_FULL = S_FULL + FW_NB,
+  enum { Q_FULL = 0, KV_FULL = 1, KV_EMPTY = 1 + FW_ST, S_FULL = 1 + 2 * FW_ST, P_FULL = S_FULL + 2 * FW_NB,
          O_DONE = P_FULL + FW_NB, DRAIN = O_DONE + 4, NBARS = DRAIN + 1 };
   uint32_t* tmem_slot = (uint32_t*)(bars + NBARS);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
@@ -369,7 +395,8 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
       mbar_init(bar(KV_EMPTY + i), 1);
     }
     for (int k = 0; k < FW_NB; ++k) {
-      mbar_init(bar(S_FULL + k), 1);
+      mbar_init(bar(S_FULL + 2 * k), 1);
+      mbar_init(bar(S_FULL + 2 * k + 1), 1);
       mbar_init(bar(P_FULL + k), 4);
     }
     for (int k = 0; k < 4; ++k) mbar_init(bar(O_DONE + k), 1);
@@ -447,7 +474,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
       const uint32_t d = tmem + 128 + 128 * (i % FW_NB);
 #pragma unroll
       for (int k = 0; k < AT_D / 16; ++k) umma_bf16(d, kdesc(q + k * 32), kdesc(sK + k * 32), ID_S, k > 0);
-      umma_commit(bar(S_FULL + i % FW_NB));
+      umma_commit(bar(S_FULL + 2 * (i % FW_NB) + g));
       return true;
     };
     int is = 0;
@@ -507,12 +534,14 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
     float m_use = -INFINITY, l = 0.f;
     bool ok = true;
     int n = 0;
+    uint32_t su = 0;   // bit k: parity of this tile's next use of score buffer k
     if (g == 0 || two) {
       for (int j = lo; j <= hi; ++j, ++n) {
         if (n >= 2 && !wait_pv(n - 2)) { ok = false; break; }
-        const int it = item_of(g, j);
-        const uint32_t tS = tmem + lane_off + 128 + 128 * (it % FW_NB);
-        if (!wait_w(bar(S_FULL + it % FW_NB), (it / FW_NB) & 1)) { ok = false; break; }
+        const int it = item_of(g, j), kb = it % FW_NB;
+        const uint32_t tS = tmem + lane_off + 128 + 128 * kb;
+        if (!wait_w(bar(S_FULL + 2 * kb + g), (su >> kb) & 1)) { ok = false; break; }
+        su ^= 1u << kb;
         tc_fence_after();
         const int kb0 = j * AT_BLK;
         // masked blocks: a key may be later than a query or before its document

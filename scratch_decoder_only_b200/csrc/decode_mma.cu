@@ -7,9 +7,8 @@
 // A decode step reads every weight once and multiplies it by a handful of
 // rows, so the work is a weight stream: the tensor-core GEMM's 128-row tiles
 // leave 3-12 CTAs busy on the 768-column projections at 32 rows.  Here the
-// weights are cut into 16-row slices spread over every SM; each slice moves
-// into shared memory by bulk copies (one per row, into rows padded by 16
-// bytes so that ldmatrix reads them without bank conflicts), several slices
+// weights are cut into 16-row slices spread over every SM; each slice (16
+// contiguous rows) moves into shared memory by one bulk copy, several slices
 // in flight per CTA, and the CTA's eight warps split the slice's k range,
 // each multiplying on the tensor cores with mma.sync m16n8k16 (A = 16 rows of
 // x, read from global memory and L1; B = the slice from shared memory).  The
@@ -47,8 +46,12 @@ __device__ __forceinline__ void dm_ldmatrix_x4(uint32_t* r, uint32_t addr) {
                : "r"(addr));
 }
 
-// MT = 16-row tiles of x (B <= 16 MT).  smem: nbuf slices of [16][K + 8]
-// 16-bit values, then the warps' partial tiles [DM_WARPS][16 MT][16] fp32.
+// MT = 16-row tiles of x (B <= 16 MT).  smem: nbuf slices of [16][K] 16-bit
+// values, then the warps' partial tiles [DM_WARPS][16 MT][16] fp32.  (The
+// ldmatrix reads of a slice meet bank conflicts, rows being K * 2 bytes
+// apart; they are a few hundred cycles per slice against microseconds of
+// copy, and one bulk copy per slice instead of one per padded row is what
+// keeps the weight stream at HBM speed.)
 template <typename T, int MT>
 __global__ void __launch_bounds__(DM_THREADS)
 dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, int N, const float* __restrict__ bias,
@@ -57,7 +60,7 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
   extern __shared__ __align__(128) uint8_t dm_smem[];
   __shared__ __align__(8) uint64_t bars[DM_MAXBUF];
   __shared__ int s_abort;
-  const int ldw = K + 8;
+  const int ldw = K;
   const uint32_t slice_bytes = (uint32_t)DM_ROWS * ldw * 2;
   float* red = reinterpret_cast<float*>(dm_smem + nbuf * slice_bytes);
   const int nslices = (N + DM_ROWS - 1) / DM_ROWS;
@@ -72,17 +75,16 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  // thread 0: slice i of this CTA into buffer i % nbuf (one bulk copy per row)
+  // thread 0: slice i of this CTA (rows r0 .. r0 + rr - 1, contiguous) into
+  // buffer i % nbuf with one bulk copy
   auto issue = [&](int i) {
     const int r0 = (blockIdx.x + i * gridDim.x) * DM_ROWS, rr = min(DM_ROWS, N - r0);
     const uint32_t dst = smem0 + (i % nbuf) * slice_bytes, bar = smem_u32(&bars[i % nbuf]);
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     mbar_expect_tx(bar, (uint32_t)rr * K * 2);
-    for (int r = 0; r < rr; ++r)
-      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                   ::"r"(dst + (uint32_t)r * ldw * 2), "l"(reinterpret_cast<uint64_t>(W + (long)(r0 + r) * K)),
-                   "r"((uint32_t)K * 2), "r"(bar)
-                   : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(reinterpret_cast<uint64_t>(W + (long)r0 * K)), "r"((uint32_t)rr * K * 2), "r"(bar)
+                 : "memory");
   };
   int issued = 0;
   if (threadIdx.x == 0)
@@ -171,7 +173,7 @@ static int g_dm_sms = 0;
 
 bool dec_mma_supported(int B, int K, int N) {
   if (B < 1 || B > 32 || K < 16 || K % 16 || N < 1) return false;
-  const size_t slice = (size_t)DM_ROWS * (K + 8) * 2, red = (size_t)DM_WARPS * 32 * 16 * 4;
+  const size_t slice = (size_t)DM_ROWS * K * 2, red = (size_t)DM_WARPS * 32 * 16 * 4;
   return 2 * slice + red <= 227 * 1024;
 }
 
@@ -187,7 +189,7 @@ cudaError_t launch_dec_mma(const T* X, int B, int K, const T* W, int N, const fl
     g_dm_sms = n > 0 ? n : 148;
   }
   const int MT = B <= 16 ? 1 : 2;
-  const size_t slice = (size_t)DM_ROWS * (K + 8) * 2, red = (size_t)DM_WARPS * 16 * MT * 16 * 4;
+  const size_t slice = (size_t)DM_ROWS * K * 2, red = (size_t)DM_WARPS * 16 * MT * 16 * 4;
   // buffers: up to four slices, two CTAs per SM where they fit in ~113 KB each
   int nbuf = (int)((113 * 1024 - red) / slice);
   if (nbuf > DM_MAXBUF) nbuf = DM_MAXBUF;
