@@ -621,8 +621,11 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
 }
 
 // ============================================================== backward
-// One CTA per 128-key block: it walks the 128-query blocks that can see its
-// keys and, per block,
+// Work items are (head, 128-key block) pairs; the grid is persistent (one CTA
+// per SM) and a CTA takes items blockIdx.x, blockIdx.x + gridDim.x, ... in
+// key-block-major order (the first key blocks see the most queries, so the
+// heaviest items go first).  For its item the CTA walks the 128-query blocks
+// that can see the keys and, per block,
 //   S^T = K Q^T, dP^T = V dO^T                  (TMEM, 128 x 128 each)
 //   P^T = exp2(S^T log2e / 8 - lse log2e)       (bf16, back into TMEM)
 //   dS^T = P^T (dP^T - D)                       (bf16, shared memory)
@@ -631,22 +634,32 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
 //                                                 global accumulator by a TMA
 //                                                 bulk reduce, scaled by 1/8
 //                                                 and rounded by a final pass)
+// K and V are double-buffered across items, so the next item's keys (and its
+// first query blocks) load while the current item finishes; the per-block
+// barriers run on a block counter that continues across items.
 // 352 threads: warp 0 loads, warp 1 issues MMAs, warps 2-9 are two groups of
 // four elementwise warps (group g handles query columns 64g..64g+63 of the
 // score tiles and d columns 32g..32g+31 of the dQ, dK, dV accumulators) and
 // warp 10 issues the dQ bulk reduces.
 #define BW_THREADS 352
 #define BW_QB 128                                    // queries per iterated block
-#define BW_ST 3                                      // Q / dO pipeline stages
+#ifndef BW_ST
+#define BW_ST 2                                      // Q / dO pipeline stages
+#endif
+#ifndef BW_KVB
+#define BW_KVB 2                                     // K / V buffers (items in flight)
+#endif
+#define BW_MAX_ITEMS 128                             // items per CTA (at most)
 struct BwdSmem {
-  static constexpr int K = 0;                        // 16 KB: 128 keys x 64
-  static constexpr int V = K + AT_TILE_BYTES;        // 16 KB
-  static constexpr int Q = V + AT_TILE_BYTES;        // BW_ST stages x 16 KB
+  static constexpr int K = 0;                        // BW_KVB buffers x 16 KB: 128 keys x 64
+  static constexpr int V = K + BW_KVB * AT_TILE_BYTES;
+  static constexpr int Q = V + BW_KVB * AT_TILE_BYTES;   // BW_ST stages x 16 KB
   static constexpr int DO = Q + BW_ST * AT_TILE_BYTES;
   static constexpr int DST = DO + BW_ST * AT_TILE_BYTES;   // 32 KB: [128 keys][128 queries] as two 64-query blocks
   static constexpr int DQS = DST + 2 * AT_TILE_BYTES;      // 2 groups x 16 KB: [128 queries][32 fp32]
   static constexpr int AUX = DQS + 2 * AT_TILE_BYTES;      // BW_ST stages x (lse2, D, dstart) x 128
-  static constexpr int BAR = AUX + BW_ST * 3 * BW_QB * 4;
+  static constexpr int NIT = AUX + BW_ST * 3 * BW_QB * 4;  // query blocks of each of the CTA's items
+  static constexpr int BAR = NIT + BW_MAX_ITEMS * 4;
   static constexpr int TOTAL = BAR + 256;
   // TMEM columns: S^T 0, dP^T 128, dV 256, dK 320, dQ 384, P^T (bf16 pairs) 448
   static constexpr int TMEM_COLS = 512;
@@ -686,45 +699,85 @@ __device__ __forceinline__ void bwd_elementwise(const uint32_t* sr, const uint32
   }
 }
 
+// Query blocks qb_lo .. nqb - 1 that can see a key block ending at last_key:
+// a prefix (document starts never decrease), counted from 8 loads at a time.
+__device__ __forceinline__ int bwd_niter(const int* dsr, int qb_lo, int nqb, int last_key) {
+  int n = 0;
+  for (int base = qb_lo; base < nqb; base += 8) {
+    int v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = base + u < nqb ? ld_once(dsr + (base + u) * BW_QB) : 0x7fffffff;
+    int c = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) c += v[u] <= last_key;
+    n += c;
+    if (c < 8) break;
+  }
+  return n;
+}
+
 template <bool F16>
 __global__ void __launch_bounds__(BW_THREADS, 1)
 attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
             const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ lse, const float* __restrict__ Dbuf,
-            const int* __restrict__ dstart, int T, int H, int kcol0, int vcol0, int G, bf16* __restrict__ dkv,
+            const int* __restrict__ dstart, int T, int H, int BH, int kcol0, int vcol0, int G, bf16* __restrict__ dkv,
             long ld_kv, int v_off, unsigned* err) {
   extern __shared__ __align__(1024) uint8_t at_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)at_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = (uint64_t*)(sm + BwdSmem::BAR);
-  // bars: 0 kv_full, 1-3 q_full (TMA tiles + per-query values), 4-6 q_empty, 7 s_full, 8 s_free,
-  //       9 p_full, 10 mma_done (P^T / dS^T read, dQ_blk complete), 11 dq_free, 12 drain,
-  //       13-14 staging written (per group, 128 arrivals), 15-16 staging free (per group)
-  uint32_t* tmem_slot = (uint32_t*)(bars + 17);
+  // bars: kv_full[2], kv_empty[2] (per item, by K/V buffer), q_full[BW_ST] (TMA tiles + per-query
+  //       values), q_empty[BW_ST], s_full, s_free, p_full, mma_done (P^T / dS^T read, dQ_blk
+  //       complete), dq_free, dkv_free (dK / dV read out), drain, staging written (per group,
+  //       128 arrivals), staging free (per group)
+  enum { KV_FULL = 0, KV_EMPTY = 2, Q_FULL = 4, Q_EMPTY = Q_FULL + BW_ST, S_FULL = Q_EMPTY + BW_ST,
+         S_FREE = S_FULL + 1, P_FULL = S_FREE + 1, MMA_DONE = P_FULL + 1, DQ_FREE = MMA_DONE + 1,
+         DKV_FREE = DQ_FREE + 1, DRAIN = DKV_FREE + 1, ST_FULL = DRAIN + 1, ST_FREE = ST_FULL + 2,
+         NBARS = ST_FREE + 2 };
+  uint32_t* tmem_slot = (uint32_t*)(bars + NBARS);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
-  int* s_info = (int*)(tmem_slot + 2);
   const uint32_t b0 = smem_u32(bars);
   auto bar = [&](int i) { return b0 + 8u * i; };
-  enum { KV_FULL = 0, Q_FULL = 1, Q_EMPTY = 4, S_FULL = 7, S_FREE = 8, P_FULL = 9, MMA_DONE = 10, DQ_FREE = 11,
-         DRAIN = 12, ST_FULL = 13, ST_FREE = 15 };
-  const uint32_t sK = smem_u32(sm + BwdSmem::K), sV = smem_u32(sm + BwdSmem::V);
+  const uint32_t sK0 = smem_u32(sm + BwdSmem::K), sV0 = smem_u32(sm + BwdSmem::V);
   const uint32_t sQ = smem_u32(sm + BwdSmem::Q), sDO = smem_u32(sm + BwdSmem::DO);
   const uint32_t sDST = smem_u32(sm + BwdSmem::DST);
   const uint32_t sDQ = smem_u32(sm + BwdSmem::DQS);
   float* aux = (float*)(sm + BwdSmem::AUX);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kb = blockIdx.y;   // earliest key blocks see the most queries: launched first
-  const int bh = blockIdx.x, b = bh / H, h = bh % H;
-  const int C = H * AT_D;
-  const int k0 = kb * AT_BLK;
-  const long rowbase = (long)b * T;
-  const int* dsr = dstart + rowbase;
-  const int nqb = (T + BW_QB - 1) / BW_QB;
-  const int qb_lo = k0 / BW_QB;
+  const int nqb = (T + BW_QB - 1) / BW_QB, nkb = (T + AT_BLK - 1) / AT_BLK;
+  const int n_items = nkb * BH;
+  int* s_nit = (int*)(sm + BwdSmem::NIT);
+  // item it (the ic-th of this CTA): key block it / BH, head-row bh = it % BH
+  struct Item { int bh, b, h, k0, qb_lo, niter; long rowbase; const int* dsr; };
+  auto item_at = [&](int it, int ic) {
+    Item I;
+    const int kb = it / BH;
+    I.bh = it % BH;
+    I.b = I.bh / H;
+    I.h = I.bh % H;
+    I.k0 = kb * AT_BLK;
+    I.rowbase = (long)I.b * T;
+    I.dsr = dstart + I.rowbase;
+    I.qb_lo = I.k0 / BW_QB;
+    I.niter = s_nit[ic];
+    return I;
+  };
   griddep_wait();
   griddep_release();
+  if (warp == 0) {
+    // the query-block count of every item of this CTA, one lane per item
+    for (int j = lane, it = blockIdx.x + lane * gridDim.x; it < n_items; j += 32, it += 32 * gridDim.x) {
+      const int k0 = (it / BH) * AT_BLK;
+      const int* dsr = dstart + (long)((it % BH) / H) * T;
+      s_nit[j] = bwd_niter(dsr, k0 / BW_QB, nqb, min(k0 + AT_BLK - 1, T - 1));
+    }
+  }
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(KV_FULL), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(KV_FULL + i), 1);
+      mbar_init(bar(KV_EMPTY + i), 1);
+    }
     for (int i = 0; i < BW_ST; ++i) {
       mbar_init(bar(Q_FULL + i), 1 + 32);   // TMA arrival + 32 lanes of per-query values
       mbar_init(bar(Q_EMPTY + i), 1);
@@ -734,6 +787,7 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
     mbar_init(bar(P_FULL), 8);
     mbar_init(bar(MMA_DONE), 1);
     mbar_init(bar(DQ_FREE), 8);
+    mbar_init(bar(DKV_FREE), 8);
     mbar_init(bar(DRAIN), 1);
     for (int g = 0; g < 2; ++g) {
       mbar_init(bar(ST_FULL + g), 128);
@@ -743,117 +797,140 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  if (warp == 0) {
-    // query blocks that can see these keys: a prefix (document starts never
-    // decrease), counted 32 blocks at a time with a ballot
-    const int last_key = min(k0 + AT_BLK - 1, T - 1);
-    int n = 0;
-    for (int base = qb_lo; base < nqb; base += 32) {
-      const int qb = base + lane;
-      const bool sees = qb < nqb && dsr[qb * BW_QB] <= last_key;
-      const unsigned m = __ballot_sync(0xffffffffu, sees);
-      n += __popc(m);
-      if (m != 0xffffffffu) break;
-    }
-    if (lane == 0) s_info[0] = n;
-  }
   if (warp == 0) tc_alloc(smem_u32(tmem_slot), BwdSmem::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int niter = s_info[0];
 
   if (warp == 0) {
     // ---------------- producer (lane 0: TMA; all lanes: per-query lse2, D, dstart)
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQKV)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmDO)) : "memory");
-      mbar_expect_tx(bar(KV_FULL), 2 * AT_TILE_BYTES);
-      tma_load_2d(sK, &tmQKV, bar(KV_FULL), kcol0 + (h / G) * AT_D, (int)(rowbase + k0));
-      tma_load_2d(sV, &tmQKV, bar(KV_FULL), vcol0 + (h / G) * AT_D, (int)(rowbase + k0));
     }
     bool ok = true;
-    for (int i = 0; i < niter; ++i) {
-      const int st = i % BW_ST;
-      const uint32_t ph = (i / BW_ST) & 1;
-      const int q0 = (qb_lo + i) * BW_QB;
-      // per-query values into registers before the stage is free
-      float l2v[4], dv[4];
-      int dsv[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int qq = q0 + lane + 32 * e;
-        const bool v = qq < T;
-        l2v[e] = v ? lse[(long)bh * T + qq] * LOG2E_F : 0.f;
-        dv[e] = v ? Dbuf[(long)bh * T + qq] : 0.f;
-        dsv[e] = v ? dsr[qq] : 0x7fffffff;
-      }
-      if (!mbar_wait(bar(Q_EMPTY + st), ph ^ 1, abort_flag)) { ok = false; break; }
+    int gb = 0, ic = 0, ic_loaded = 0;
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++ic) {
+      const Item I = item_at(it, ic);
+      const int kvb = ic % BW_KVB;
+      // the K / V buffer of item ic - BW_KVB has been read by its last MMA
+      if (!mbar_wait(bar(KV_EMPTY + kvb), ((ic / BW_KVB) & 1) ^ 1, abort_flag)) { ok = false; break; }
       if (lane == 0) {
-        mbar_expect_tx(bar(Q_FULL + st), 2 * AT_TILE_BYTES);
-        tma_load_2d(sQ + st * AT_TILE_BYTES, &tmQKV, bar(Q_FULL + st), h * AT_D, (int)(rowbase + q0));
-        tma_load_2d(sDO + st * AT_TILE_BYTES, &tmDO, bar(Q_FULL + st), h * AT_D, (int)(rowbase + q0));
+        mbar_expect_tx(bar(KV_FULL + kvb), 2 * AT_TILE_BYTES);
+        tma_load_2d(sK0 + kvb * AT_TILE_BYTES, &tmQKV, bar(KV_FULL + kvb), kcol0 + (I.h / G) * AT_D,
+                    (int)(I.rowbase + I.k0));
+        tma_load_2d(sV0 + kvb * AT_TILE_BYTES, &tmQKV, bar(KV_FULL + kvb), vcol0 + (I.h / G) * AT_D,
+                    (int)(I.rowbase + I.k0));
       }
-      float* L2 = aux + st * 3 * BW_QB;
-      float* Dq = L2 + BW_QB;
-      int* DSq = reinterpret_cast<int*>(Dq + BW_QB);
+      ic_loaded = ic + 1;
+      for (int i = 0; i < I.niter; ++i, ++gb) {
+        const int st = gb % BW_ST;
+        const uint32_t ph = (gb / BW_ST) & 1;
+        const int q0 = (I.qb_lo + i) * BW_QB;
+        // per-query values into registers before the stage is free
+        float l2v[4], dv[4];
+        int dsv[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        L2[lane + 32 * e] = l2v[e];
-        Dq[lane + 32 * e] = dv[e];
-        DSq[lane + 32 * e] = dsv[e];
+        for (int e = 0; e < 4; ++e) {
+          const int qq = q0 + lane + 32 * e;
+          const bool v = qq < T;
+          l2v[e] = v ? lse[(long)I.bh * T + qq] * LOG2E_F : 0.f;
+          dv[e] = v ? Dbuf[(long)I.bh * T + qq] : 0.f;
+          dsv[e] = v ? I.dsr[qq] : 0x7fffffff;
+        }
+        if (!mbar_wait(bar(Q_EMPTY + st), ph ^ 1, abort_flag)) { ok = false; break; }
+        if (lane == 0) {
+          mbar_expect_tx(bar(Q_FULL + st), 2 * AT_TILE_BYTES);
+          tma_load_2d(sQ + st * AT_TILE_BYTES, &tmQKV, bar(Q_FULL + st), I.h * AT_D, (int)(I.rowbase + q0));
+          tma_load_2d(sDO + st * AT_TILE_BYTES, &tmDO, bar(Q_FULL + st), I.h * AT_D, (int)(I.rowbase + q0));
+        }
+        float* L2 = aux + st * 3 * BW_QB;
+        float* Dq = L2 + BW_QB;
+        int* DSq = reinterpret_cast<int*>(Dq + BW_QB);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          L2[lane + 32 * e] = l2v[e];
+          Dq[lane + 32 * e] = dv[e];
+          DSq[lane + 32 * e] = dsv[e];
+        }
+        mbar_arrive(bar(Q_FULL + st));   // release: the values above are visible to whoever waits on q_full
       }
-      mbar_arrive(bar(Q_FULL + st));   // release: the values above are visible to whoever waits on q_full
     }
     if (!ok && lane == 0) trap_timeout(abort_flag, err);
     if (lane == 0) {
+      // every copy issued has landed before the CTA leaves
       volatile int never = 0;
-      mbar_wait(bar(KV_FULL), 0, &never, 1ll << 28);
-      for (int i = max(0, niter - BW_ST); i < niter; ++i)
+      for (int i = max(0, ic_loaded - BW_KVB); i < ic_loaded; ++i)
+        mbar_wait(bar(KV_FULL + i % BW_KVB), (i / BW_KVB) & 1, &never, 1ll << 28);
+      for (int i = max(0, gb - BW_ST); i < gb; ++i)
         mbar_wait(bar(Q_FULL + i % BW_ST), (i / BW_ST) & 1, &never, 1ll << 28);
     }
   } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
+    // ---------------- MMA issuer: the S^T / dP^T of the next block (next item
+    // included) go out before this block's dV, dK and dQ
     constexpr uint32_t ID_SS = instr_desc_t(F16, 128, false, false);   // S^T, dP^T: 128 keys x 128 queries, K = d
     constexpr uint32_t ID_KV = instr_desc_t(F16, 64, false, true);     // dV, dK: 128 keys x 64, K = 128 queries
     constexpr uint32_t ID_DQ = instr_desc_t(F16, 64, true, true);      // dQ: 128 queries x 64, K = 128 keys
-    bool ok = mbar_wait(bar(KV_FULL), 0, abort_flag);
-    auto issue_s = [&](int i) -> bool {   // S^T and dP^T of query block i
-      const int st = i % BW_ST;
-      if (!mbar_wait(bar(Q_FULL + st), (i / BW_ST) & 1, abort_flag)) return false;
-      if (!mbar_wait(bar(S_FREE), (i & 1) ^ 1, abort_flag)) return false;   // previous S^T / dP^T read
+    bool ok = true;
+    // S issue cursor: item it_s (ic_s-th of this CTA, niter_s blocks), block i_s, global block gs
+    int it_s = blockIdx.x, ic_s = 0, i_s = 0, gs = 0, niter_s = 0;
+    if (it_s < n_items) niter_s = s_nit[0];
+    auto issue_s = [&]() -> bool {   // S^T and dP^T of the block at the cursor, then advance it
+      const int st = gs % BW_ST, kvb = ic_s % BW_KVB;
+      if (i_s == 0 && !mbar_wait(bar(KV_FULL + kvb), (ic_s / BW_KVB) & 1, abort_flag)) return false;
+      if (!mbar_wait(bar(Q_FULL + st), (gs / BW_ST) & 1, abort_flag)) return false;
+      if (!mbar_wait(bar(S_FREE), (gs & 1) ^ 1, abort_flag)) return false;   // previous S^T / dP^T read
       tc_fence_after();
       const uint32_t q = sQ + st * AT_TILE_BYTES, o = sDO + st * AT_TILE_BYTES;
+      const uint32_t sK = sK0 + kvb * AT_TILE_BYTES, sV = sV0 + kvb * AT_TILE_BYTES;
 #pragma unroll
       for (int k = 0; k < AT_D / 16; ++k) {
         umma_bf16(tmem + 0, kdesc(sK + k * 32), kdesc(q + k * 32), ID_SS, k > 0);
         umma_bf16(tmem + 128, kdesc(sV + k * 32), kdesc(o + k * 32), ID_SS, k > 0);
       }
       umma_commit(bar(S_FULL));
+      ++gs;
+      if (++i_s == niter_s) {
+        i_s = 0;
+        ++ic_s;
+        it_s += gridDim.x;
+        niter_s = it_s < n_items ? s_nit[ic_s] : 0;
+      }
       return true;
     };
-    if (ok && niter > 0) ok = issue_s(0);
-    for (int i = 0; i < niter && ok; ++i) {
-      const int st = i % BW_ST;
-      if (i + 1 < niter && !issue_s(i + 1)) { ok = false; break; }
-      if (!mbar_wait(bar(P_FULL), i & 1, abort_flag)) { ok = false; break; }   // P^T, dS^T written
-      tc_fence_after();
-      const uint32_t q = sQ + st * AT_TILE_BYTES, o = sDO + st * AT_TILE_BYTES;
+    int g_total = 0;   // blocks of all of this CTA's items
+    for (int it = blockIdx.x, j = 0; it < n_items; it += gridDim.x, ++j) g_total += s_nit[j];
+    if (g_total > 0) ok = issue_s();
+    int gb = 0, ic = 0;
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++ic) {
+      const int niter = s_nit[ic], kvb = ic % BW_KVB;
+      const uint32_t sK = sK0 + kvb * AT_TILE_BYTES;
+      for (int i = 0; i < niter; ++i, ++gb) {
+        const int st = gb % BW_ST;
+        if (gb + 1 < g_total && !issue_s()) { ok = false; break; }
+        if (!mbar_wait(bar(P_FULL), gb & 1, abort_flag)) { ok = false; break; }   // P^T, dS^T written
+        // the previous item's dK / dV have been read out of TMEM before they are overwritten
+        if (i == 0 && ic > 0 && !mbar_wait(bar(DKV_FREE), (ic - 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t q = sQ + st * AT_TILE_BYTES, o = sDO + st * AT_TILE_BYTES;
 #pragma unroll
-      for (int kk = 0; kk < BW_QB / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * AT_TILE_BYTES + (kk & 3) * 32;
-        umma_bf16_ts(tmem + 256, tmem + 448 + 8 * kk, mndesc(o + kk * 2048, 8192), ID_KV, (i > 0 || kk > 0));
-        umma_bf16(tmem + 320, kdesc(sDST + off), mndesc(q + kk * 2048, 8192), ID_KV, (i > 0 || kk > 0));
+        for (int kk = 0; kk < BW_QB / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * AT_TILE_BYTES + (kk & 3) * 32;
+          umma_bf16_ts(tmem + 256, tmem + 448 + 8 * kk, mndesc(o + kk * 2048, 8192), ID_KV, (i > 0 || kk > 0));
+          umma_bf16(tmem + 320, kdesc(sDST + off), mndesc(q + kk * 2048, 8192), ID_KV, (i > 0 || kk > 0));
+        }
+        umma_commit(bar(Q_EMPTY + st));   // Q / dO stage free
+        // dQ_blk = dS K once the previous block's dQ has been read out
+        if (gb > 0 && !mbar_wait(bar(DQ_FREE), (gb - 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < AT_BLK / 16; ++kk)
+          umma_bf16(tmem + 384, mndesc(sDST + kk * 2048, AT_TILE_BYTES), mndesc(sK + kk * 2048, 8192), ID_DQ,
+                    kk > 0);
+        umma_commit(bar(MMA_DONE));
+        if (i + 1 == niter) umma_commit(bar(KV_EMPTY + kvb));   // this item's K / V no longer read
       }
-      umma_commit(bar(Q_EMPTY + st));   // Q / dO stage free
-      // dQ_blk = dS K once the previous block's dQ has been read out
-      if (i > 0 && !mbar_wait(bar(DQ_FREE), (i - 1) & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < AT_BLK / 16; ++kk)
-        umma_bf16(tmem + 384, mndesc(sDST + kk * 2048, AT_TILE_BYTES), mndesc(sK + kk * 2048, 8192), ID_DQ, kk > 0);
-      umma_commit(bar(MMA_DONE));
     }
     if (!ok) trap_timeout(abort_flag, err);
     umma_commit(bar(DRAIN));
@@ -864,7 +941,6 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
     const int quarter = warp & 3;
     const int grp = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
-    const int k = k0 + r;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = 0.125f * LOG2E_F;
     const uint32_t st_full = bar(ST_FULL + grp), st_free = bar(ST_FREE + grp);
@@ -873,8 +949,8 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
     // waits are voted warp-wide so that the .sync.aligned TMEM accesses after
     // them are never reached by part of a warp
     auto wait_w = [&](uint32_t bb, uint32_t parity) { return __all_sync(0xffffffffu, mbar_wait(bb, parity, abort_flag)); };
-    // dQ of block j: TMEM -> fp32 staging (128-byte swizzle); warp 10 issues
-    // the bulk reduce-add once all 128 rows of the group are written
+    // dQ of global block j: TMEM -> fp32 staging (128-byte swizzle); warp 10
+    // issues the bulk reduce-add once all 128 rows of the group are written
     auto flush_dq = [&](int j) -> bool {
       uint32_t rr[32];
       tmem_ld32(tmem + lane_off + 384 + 32 * grp, rr);
@@ -895,108 +971,119 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
       mbar_arrive(st_full);
       return true;
     };
-    for (int i = 0; i < niter; ++i) {
-      const int q0 = (qb_lo + i) * BW_QB;
-      const int st = i % BW_ST;
-      const float* L2 = aux + st * 3 * BW_QB + 64 * grp;
-      const float* Dq = L2 + BW_QB;
-      const int* DSq = reinterpret_cast<const int*>(L2 + 2 * BW_QB);
-      if (!wait_w(bar(Q_FULL + st), (i / BW_ST) & 1)) { ok = false; break; }   // per-query values
-      if (!wait_w(bar(S_FULL), i & 1)) { ok = false; break; }
-      tc_fence_after();
-      // masking only where a key can be later than a query or before its document
-      // (document starts never decrease, queries past T carry INT_MAX)
-      const bool need_mask = q0 < k0 + AT_BLK || DSq[BW_QB - 1 - 64 * grp] > k0;
-      // two 32-column halves of the group's 64 query columns (a variant that
-      // pipelined 16-column quarters, each quarter's loads issued before the
-      // previous quarter's arithmetic, measured 4 % slower)
-      uint32_t pw[32], dw[32];
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t sr[32], dr[32];
-        tmem_ld32(tmem + lane_off + 64 * grp + 32 * half, sr);
-        tmem_ld32(tmem + lane_off + 128 + 64 * grp + 32 * half, dr);
-        tmem_wait_ld();
-        if (half == 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(S_FREE));   // S^T / dP^T may be overwritten
-        }
-        const int qf = q0 + 64 * grp + 32 * half;
-        if (need_mask)
-          bwd_elementwise<true, F16, 32>(sr, dr, L2 + 32 * half, Dq + 32 * half, DSq + 32 * half, qf, k, sl2,
-                                         pw + 16 * half, dw + 16 * half);
-        else
-          bwd_elementwise<false, F16, 32>(sr, dr, L2 + 32 * half, Dq + 32 * half, DSq + 32 * half, qf, k, sl2,
-                                          pw + 16 * half, dw + 16 * half);
-      }
-      // the previous block's P^T / dS^T have been consumed and its dQ is complete
-      if (i > 0 && !wait_w(bar(MMA_DONE), (i - 1) & 1)) { ok = false; break; }
-      tc_fence_after();
-      tmem_st32(tmem + lane_off + 448 + 32 * grp, pw);
-      {
-        const uint32_t db = sDST + grp * AT_TILE_BYTES + r * 128;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint32_t sw = (u ^ (r & 7)) << 4;
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(db + sw), "r"(dw[4 * u]), "r"(dw[4 * u + 1]),
-                       "r"(dw[4 * u + 2]), "r"(dw[4 * u + 3])
-                       : "memory");
-        }
-      }
-      tmem_wait_st();
-      fence_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(P_FULL));
-      if (i > 0) {
+    int gb = 0, ic = 0;
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++ic) {
+      const Item I = item_at(it, ic);
+      const int k = I.k0 + r;
+      for (int i = 0; i < I.niter; ++i, ++gb) {
+        const int q0 = (I.qb_lo + i) * BW_QB;
+        const int st = gb % BW_ST;
+        const float* L2 = aux + st * 3 * BW_QB + 64 * grp;
+        const float* Dq = L2 + BW_QB;
+        const int* DSq = reinterpret_cast<const int*>(L2 + 2 * BW_QB);
+        if (!wait_w(bar(Q_FULL + st), (gb / BW_ST) & 1)) { ok = false; break; }   // per-query values
+        if (!wait_w(bar(S_FULL), gb & 1)) { ok = false; break; }
         tc_fence_after();
-        if (!flush_dq(i - 1)) { ok = false; break; }
-      }
-    }
-    // the last block's dQ, then dK and dV
-    if (ok && niter > 0 && wait_w(bar(MMA_DONE), (niter - 1) & 1)) {
-      tc_fence_after();
-      ok = flush_dq(niter - 1);
-      if (ok) {
-        bf16* row = dkv + (rowbase + k) * ld_kv;
+        // masking only where a key can be later than a query or before its document
+        // (document starts never decrease, queries past T carry INT_MAX)
+        const bool need_mask = q0 < I.k0 + AT_BLK || DSq[BW_QB - 1 - 64 * grp] > I.k0;
+        // two 32-column halves of the group's 64 query columns (a variant that
+        // pipelined 16-column quarters, each quarter's loads issued before the
+        // previous quarter's arithmetic, measured 4 % slower)
+        uint32_t pw[32], dw[32];
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          const float sc = part == 0 ? 0.125f : 1.f;
-          bf16* dst = row + (part == 0 ? 0 : v_off) + h * AT_D + 32 * grp;
-          uint32_t rr[32];
-          tmem_ld32(tmem + lane_off + (part == 0 ? 320 : 256) + 32 * grp, rr);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t sr[32], dr[32];
+          tmem_ld32(tmem + lane_off + 64 * grp + 32 * half, sr);
+          tmem_ld32(tmem + lane_off + 128 + 64 * grp + 32 * half, dr);
           tmem_wait_ld();
-          if (k >= T) continue;
+          if (half == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(S_FREE));   // S^T / dP^T may be overwritten
+          }
+          const int qf = q0 + 64 * grp + 32 * half;
+          if (need_mask)
+            bwd_elementwise<true, F16, 32>(sr, dr, L2 + 32 * half, Dq + 32 * half, DSq + 32 * half, qf, k, sl2,
+                                           pw + 16 * half, dw + 16 * half);
+          else
+            bwd_elementwise<false, F16, 32>(sr, dr, L2 + 32 * half, Dq + 32 * half, DSq + 32 * half, qf, k, sl2,
+                                            pw + 16 * half, dw + 16 * half);
+        }
+        // the previous block's P^T / dS^T have been consumed and its dQ is complete
+        if (gb > 0 && !wait_w(bar(MMA_DONE), (gb - 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        tmem_st32(tmem + lane_off + 448 + 32 * grp, pw);
+        {
+          const uint32_t db = sDST + grp * AT_TILE_BYTES + r * 128;
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            uint4 w;
-            w.x = pack16x2<F16>(__uint_as_float(rr[8 * u]) * sc, __uint_as_float(rr[8 * u + 1]) * sc);
-            w.y = pack16x2<F16>(__uint_as_float(rr[8 * u + 2]) * sc, __uint_as_float(rr[8 * u + 3]) * sc);
-            w.z = pack16x2<F16>(__uint_as_float(rr[8 * u + 4]) * sc, __uint_as_float(rr[8 * u + 5]) * sc);
-            w.w = pack16x2<F16>(__uint_as_float(rr[8 * u + 6]) * sc, __uint_as_float(rr[8 * u + 7]) * sc);
-            *reinterpret_cast<uint4*>(dst + 8 * u) = w;
+          for (int u = 0; u < 8; ++u) {
+            const uint32_t sw = (u ^ (r & 7)) << 4;
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(db + sw), "r"(dw[4 * u]),
+                         "r"(dw[4 * u + 1]), "r"(dw[4 * u + 2]), "r"(dw[4 * u + 3])
+                         : "memory");
           }
         }
+        tmem_wait_st();
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(P_FULL));
+        if (i > 0) {
+          tc_fence_after();
+          if (!flush_dq(gb - 1)) { ok = false; break; }
+        }
       }
-    } else if (niter > 0) {
-      ok = false;
+      if (!ok) break;
+      // the item's last dQ, then dK and dV
+      if (!wait_w(bar(MMA_DONE), (gb - 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      if (!flush_dq(gb - 1)) { ok = false; break; }
+      bf16* row = dkv + (I.rowbase + k) * ld_kv;
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        const float sc = part == 0 ? 0.125f : 1.f;
+        uint32_t rr[32];
+        tmem_ld32(tmem + lane_off + (part == 0 ? 320 : 256) + 32 * grp, rr);
+        tmem_wait_ld();
+        if (part == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(DKV_FREE));   // the next item's dV / dK may overwrite TMEM
+        }
+        if (k >= T) continue;
+        bf16* dst = row + (part == 0 ? 0 : v_off) + I.h * AT_D + 32 * grp;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          uint4 w;
+          w.x = pack16x2<F16>(__uint_as_float(rr[8 * u]) * sc, __uint_as_float(rr[8 * u + 1]) * sc);
+          w.y = pack16x2<F16>(__uint_as_float(rr[8 * u + 2]) * sc, __uint_as_float(rr[8 * u + 3]) * sc);
+          w.z = pack16x2<F16>(__uint_as_float(rr[8 * u + 4]) * sc, __uint_as_float(rr[8 * u + 5]) * sc);
+          w.w = pack16x2<F16>(__uint_as_float(rr[8 * u + 6]) * sc, __uint_as_float(rr[8 * u + 7]) * sc);
+          *reinterpret_cast<uint4*>(dst + 8 * u) = w;
+        }
+      }
     }
     if (!ok) trap_timeout(abort_flag, err);
   } else if (warp == 10 && lane == 0) {
     // ---------------- dQ reducer: per block, both groups' staging -> global fp32 accumulator
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmDQ)) : "memory");
     bool ok = true;
-    for (int j = 0; j < niter && ok; ++j) {
-      for (int gg = 0; gg < 2; ++gg) {
-        if (!mbar_wait(bar(ST_FULL + gg), j & 1, abort_flag)) { ok = false; break; }
-        tma_reduce_add_2d(&tmDQ, sDQ + gg * AT_TILE_BYTES, h * AT_D + 32 * gg, (int)(rowbase + (qb_lo + j) * BW_QB));
-        bulk_commit();
+    int gb = 0, ic = 0;
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++ic) {
+      const Item I = item_at(it, ic);
+      for (int j = 0; j < I.niter && ok; ++j, ++gb) {
+        for (int gg = 0; gg < 2; ++gg) {
+          if (!mbar_wait(bar(ST_FULL + gg), gb & 1, abort_flag)) { ok = false; break; }
+          tma_reduce_add_2d(&tmDQ, sDQ + gg * AT_TILE_BYTES, I.h * AT_D + 32 * gg,
+                            (int)(I.rowbase + (I.qb_lo + j) * BW_QB));
+          bulk_commit();
+        }
+        if (!ok) break;
+        bulk_wait_read<0>();   // both stagings read: the groups may overwrite them
+        mbar_arrive(bar(ST_FREE + 0));
+        mbar_arrive(bar(ST_FREE + 1));
       }
-      if (!ok) break;
-      bulk_wait_read<0>();   // both stagings read: the groups may overwrite them
-      mbar_arrive(bar(ST_FREE + 0));
-      mbar_arrive(bar(ST_FREE + 1));
     }
     if (!ok) trap_timeout(abort_flag, err);
     bulk_wait_all();
@@ -1121,10 +1208,19 @@ static cudaError_t attn_bwd_tc_t(const bf16* qkv, const bf16* out, const bf16* d
     attn_rowdot_kernel<F16><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(out, dout, Dbuf, B, T, H);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  dim3 grid(B * H, (T + AT_BLK - 1) / AT_BLK);
+  // persistent: one CTA per SM (or fewer, for fewer items)
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      sms = 148;
+  }
+  const int n_items = B * H * ((T + AT_BLK - 1) / AT_BLK);
+  const int grid = n_items < sms ? n_items : sms;
+  if (n_items > (long)grid * BW_MAX_ITEMS) return cudaErrorInvalidValue;
   ++g_kernel_launches;
-  e = launch_k(attn_bwd_tc<F16>, grid, dim3(BW_THREADS), smem, s, tqkv, tdo, tdq, lse, Dbuf, dstart, T, H, L.kcol, L.vcol,
-               L.G, L.dkv, L.ld_kv, L.v_off, err);
+  e = launch_k(attn_bwd_tc<F16>, dim3(grid), dim3(BW_THREADS), smem, s, tqkv, tdo, tdq, lse, Dbuf, dstart, T, H, B * H,
+               L.kcol, L.vcol, L.G, L.dkv, L.ld_kv, L.v_off, err);
   if (e != cudaSuccess) return e;
   ++g_kernel_launches;
   return launch_k(attn_dq_finish_kernel<F16>, dim3(148 * 8), dim3(256), 0, s, dq_acc, dqkv, rows, C, (long)L.qw);

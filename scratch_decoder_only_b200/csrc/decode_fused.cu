@@ -18,8 +18,9 @@
 //                 output projection (+ bias + residual)
 //              D  LN2 (every CTA), 16-row units of fc (+ bias, GELU)
 //              E  row units of fc2 (+ bias + residual)
-//   then       F  final LN (every CTA), 16-row chunks of the LM head (fp32
-//                 logits, four chunks in flight) with a per-CTA argmax;
+//   then       F  final LN (every CTA), the LM head (fp32 logits) in 4-row
+//                 chunks that every warp streams on its own (two in flight
+//                 per warp, no block barrier) with a per-CTA argmax;
 //                 after the barrier every CTA
 //                 reduces the per-CTA maxima (lowest index on ties) into the
 //                 next token and embeds it for the next step.
@@ -47,6 +48,7 @@
 #define DF_WBUF (48 * 1024)             // bytes of each of the two weight buffers
 #define DF_MAX_SPLITS 16
 #define DF_BAR_LIMIT (1ll << 31)         // clock cycles (about a second)
+#define DF_WSLOT (DF_WBUF / DF_WARPS)   // bytes of one LM-head slot (two per warp)
 #define DF_PRM_BIAS 256                  // bias floats of one CTA's units in one phase (at most)
 #define DF_PRM(C) (2 * (C) + DF_PRM_BIAS)  // floats of one parameter area
 
@@ -230,6 +232,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const DecFu
   extern __shared__ __align__(128) uint8_t df_smem[];
   __shared__ __align__(8) uint64_t wbars[4];
   __shared__ __align__(8) uint64_t pbars[2];
+  __shared__ __align__(8) uint64_t hbars[2 * DF_WARPS];   // LM head: two slots per warp
   __shared__ int s_flag;
   __shared__ float s_rv[DF_WARPS][BB];
   __shared__ int s_ri[DF_WARPS][BB];
@@ -258,6 +261,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const DecFu
   }
   if (threadIdx.x == 0) {
     for (int i = 0; i < 4; ++i) mbar_init(wb.bar[i], 1);
+    for (int i = 0; i < 2 * DF_WARPS; ++i) mbar_init(smem_u32(&hbars[i]), 1);
     mbar_init(pbar[0], 1);
     mbar_init(pbar[1], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -272,9 +276,13 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const DecFu
   if (rows_e > 16) rows_e = 16;
   rows_e &= ~3;   // bias slices of whole 16-byte groups
   const int nu_e = (C + rows_e - 1) / rows_e;
-  int hr = (DF_WBUF / 2) / (2 * C);   // LM-head rows per 24 KB chunk
-  if (hr > 16) hr = 16;
-  const int n_head = (p.Vp + hr - 1) / hr;
+  // LM head: warp-chunks of hw rows, each warp streaming its own through two
+  // DF_WSLOT-byte slots in the weight buffers (free during the head phase)
+  int hw = DF_WSLOT / (2 * C);
+  if (hw > 8) hw = 8;
+  const int n_wc = (p.Vp + hw - 1) / hw;
+  uint32_t hpar = 0;    // bit s: parity of this warp's next wait on slot s
+  int hpend = 0;        // this warp's slots with a copy in flight (bit s)
   const int S = p.S, nu_att = B * H * S;
   const float* P32 = p.p32;
   const bf16* PW = p.pw;
@@ -613,33 +621,90 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const DecFu
           if (len >= 8) l2_prefetch(PW + p.l_ln1_g + o, (uint32_t)(len & ~7L) * 2);
         }
       }
-      // chunk k of this CTA is head chunk cta + k * G (hr rows), in slot k & 3:
-      // four 24 KB chunks in flight
-      int nk = 0;
-      for (int c2 = cta; c2 < n_head; c2 += G) ++nk;
-      auto slot_ptr = [&](int sl) { return wb.buf[sl & 1] + (sl >> 1) * (DF_WBUF / 2); };
-      auto issue_chunk = [&](int k) {
-        const int ch = cta + k * G, sl = k & 3;
-        const int r0 = ch * hr, rr = min(hr, p.Vp - r0);
-        wb.inflight[sl] = 1;
-        if (threadIdx.x == 0) {
-          wbuf_issue_begin(wb, sl, (uint32_t)rr * C * 2);
-          wbuf_copy(smem_u32(slot_ptr(sl)), Wh + (long)r0 * C, (uint32_t)rr * C * 2, wb.bar[sl]);
+      // warp-chunk k of this warp is cta * DF_WARPS + warp + k * G * DF_WARPS
+      // (hw rows), in the warp's slot k & 1; each warp waits for its own copies
+      // and syncs only its own lanes, so warps stream independently
+      int nkw = 0;
+      for (int c2 = cta * DF_WARPS + warp; c2 < n_wc; c2 += G * DF_WARPS) ++nkw;
+      uint8_t* wsl = df_smem + warp * 2 * DF_WSLOT;
+      auto issue_w = [&](int k) {
+        const int sl = k & 1, wc = cta * DF_WARPS + warp + k * G * DF_WARPS;
+        const int r0 = wc * hw, rr = min(hw, p.Vp - r0);
+        hpend |= 1 << sl;
+        if (lane == 0) {
+          const uint32_t hb = smem_u32(&hbars[warp * 2 + sl]);
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          mbar_expect_tx(hb, (uint32_t)rr * C * 2);
+          wbuf_copy(smem_u32(wsl + sl * DF_WSLOT), Wh + (long)r0 * C, (uint32_t)rr * C * 2, hb);
         }
       };
-      __syncthreads();
-      for (int k = 0; k < 4 && k < nk; ++k) issue_chunk(k);
-      for (int k = 0; k < nk; ++k) {
-        const int ch = cta + k * G;
-        const int r0 = ch * hr, rr = min(hr, p.Vp - r0);
-        if (!wbuf_wait(wb, k & 3, p)) goto abort;
-        df_project<BB>(reinterpret_cast<const bf16*>(slot_ptr(k & 3)), rr, C, xin, C, B, [&](int r, int b, float y) {
-          const int n = r0 + r;
-          p.logits[(long)b * p.Vp + n] = y;
-          if (n < p.V && (y > bv[b] || (y == bv[b] && n < bi[b]))) { bv[b] = y; bi[b] = n; }
-        });
-        __syncthreads();
-        if (k + 4 < nk) issue_chunk(k + 4);
+      __syncthreads();   // the weight buffers are no longer read by the last layer
+      if (nkw > 0) issue_w(0);
+      if (nkw > 1) issue_w(1);
+      bool hok = true;
+      for (int k = 0; k < nkw; ++k) {
+        const int sl = k & 1, wc = cta * DF_WARPS + warp + k * G * DF_WARPS;
+        const int r0 = wc * hw, rr = min(hw, p.Vp - r0);
+        {
+          const uint32_t hb = smem_u32(&hbars[warp * 2 + sl]);
+          bool okw = true;
+          const long long t0 = clock64();
+          for (unsigned it = 1; !mbar_try_wait(hb, (hpar >> sl) & 1); ++it) {
+            if ((it & 63) == 0 && (*(volatile const unsigned*)p.abortf || clock64() - t0 > DF_BAR_LIMIT)) {
+              okw = false;
+              break;
+            }
+          }
+          if (!__all_sync(0xffffffffu, okw)) { hok = false; break; }
+          hpar ^= 1u << sl;
+          hpend &= ~(1 << sl);
+        }
+        const bf16* ws = reinterpret_cast<const bf16*>(wsl + sl * DF_WSLOT);
+        for (int r = 0; r < rr; ++r) {
+          float acc[BB];
+#pragma unroll
+          for (int b = 0; b < BB; ++b) acc[b] = 0.f;
+          for (int kk = lane * 8; kk < C; kk += 256) {
+            float w[8];
+            Vec<bf16>::load(ws + (long)r * C + kk, w);
+#pragma unroll
+            for (int b = 0; b < BB; ++b) {
+              if (b < B) {
+                const float4 x0 = *reinterpret_cast<const float4*>(xin + b * C + kk);
+                const float4 x1 = *reinterpret_cast<const float4*>(xin + b * C + kk + 4);
+                float a = acc[b];
+                a = fmaf(w[0], x0.x, a); a = fmaf(w[1], x0.y, a); a = fmaf(w[2], x0.z, a); a = fmaf(w[3], x0.w, a);
+                a = fmaf(w[4], x1.x, a); a = fmaf(w[5], x1.y, a); a = fmaf(w[6], x1.z, a); a = fmaf(w[7], x1.w, a);
+                acc[b] = a;
+              }
+            }
+          }
+#pragma unroll
+          for (int b = 0; b < BB; ++b) {
+            if (b < B) {
+              const float y = warp_sum(acc[b]);
+              const int n = r0 + r;
+              if (lane == 0) {
+                p.logits[(long)b * p.Vp + n] = y;
+                if (n < p.V && (y > bv[b] || (y == bv[b] && n < bi[b]))) { bv[b] = y; bi[b] = n; }
+              }
+            }
+          }
+        }
+        __syncwarp();   // every lane is done with the slot before it is refilled
+        if (k + 2 < nkw) issue_w(k + 2);
+      }
+      if (!hok && lane == 0) {
+        atomicOr(p.err, GPT_DEVERR_TIMEOUT);
+        atomicExch(p.abortf, 1u);
+      }
+      if (__syncthreads_or(!hok)) {
+        // leave with none of this warp's copies in flight
+        volatile int never = 0;
+        if (lane == 0)
+          for (int sl = 0; sl < 2; ++sl)
+            if (hpend & (1 << sl)) mbar_wait(smem_u32(&hbars[warp * 2 + sl]), (hpar >> sl) & 1, &never, 1ll << 28);
+        goto abort;
       }
       // per-CTA maxima (lane 0 of every warp holds its own)
       if (lane == 0) {
@@ -739,7 +804,7 @@ bool dec_fused_supported(int B, int C, int H, int F, int Vp) {
   if (per_cta(3 * C / 16) * 16L * C * 2 > DF_WBUF) return false;   // qkv
   if (per_cta(C / 16) * 16L * C * 2 > DF_WBUF) return false;       // out-projection
   if (per_cta(F / 16) * 16L * C * 2 > DF_WBUF) return false;       // fc
-  if ((DF_WBUF / 2) / (2L * C) < 1) return false;                   // head chunks of at least a row
+  if (DF_WSLOT / (2L * C) < 1) return false;                        // head warp-chunks of at least a row
   long rows_e = DF_WBUF / (F * 2L);
   if (rows_e > 16) rows_e = 16;
   rows_e &= ~3L;
