@@ -29,7 +29,6 @@
 #define AT_BLK 128
 #define AT_TILE_BYTES (AT_BLK * AT_D * 2)   // 16 KB: 128 rows x 128 B
 #define LOG2E_F 1.4426950408889634f
-#define LN2_F 0.6931471805599453f
 
 __device__ __forceinline__ uint64_t kdesc(uint32_t addr) { return smem_desc(addr, 16, 1024); }
 __device__ __forceinline__ uint64_t mndesc(uint32_t addr, uint32_t lbo) { return smem_desc(addr, lbo, 1024); }
@@ -611,7 +610,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
           }
         }
       }
-      if (qv) lse[(long)bh * T + q] = (m_use + log2f(l)) * LN2_F;
+      if (qv) lse[(long)bh * T + q] = m_use + log2f(l);   // base-2 log-sum-exp of the scaled scores
     }
   }
   tc_fence_before();
@@ -627,7 +626,8 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
 // heaviest items go first).  For its item the CTA walks the 128-query blocks
 // that can see the keys and, per block,
 //   S^T = K Q^T, dP^T = V dO^T                  (TMEM, 128 x 128 each)
-//   P^T = exp2(S^T log2e / 8 - lse log2e)       (bf16, back into TMEM)
+//   P^T = exp2(S^T log2e / 8 - lse2)            (bf16, back into TMEM; lse2 is
+//                                                 the forward's base-2 log-sum-exp)
 //   dS^T = P^T (dP^T - D)                       (bf16, shared memory)
 //   dV += P^T dO,  dK += dS^T Q                  (TMEM, across query blocks)
 //   dQ_blk = dS K                                (TMEM; added in fp32 to a
@@ -649,6 +649,10 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
 #ifndef BW_KVB
 #define BW_KVB 2                                     // K / V buffers (items in flight)
 #endif
+// The MMA warp issues the next item's first S^T before this item's last dV / dK
+// / dQ (whose completion frees this item's K / V buffer): one buffer would
+// deadlock that look-ahead.
+static_assert(BW_KVB >= 2, "the MMA look-ahead across items needs two K / V buffers");
 #define BW_MAX_ITEMS 128                             // items per CTA (at most)
 struct BwdSmem {
   static constexpr int K = 0;                        // BW_KVB buffers x 16 KB: 128 keys x 64
@@ -697,6 +701,14 @@ __device__ __forceinline__ void bwd_elementwise(const uint32_t* sr, const uint32
       dw[c8 / 2 + e] = pack16x2<F16>(gv[2 * e], gv[2 * e + 1]);
     }
   }
+}
+
+// Bulk copy of `bytes` (a multiple of 16, 16-byte aligned ends) from global to
+// shared memory, completing on mbarrier `bar`.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
 }
 
 // Query blocks qb_lo .. nqb - 1 that can see a key block ending at last_key:
@@ -779,7 +791,7 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
       mbar_init(bar(KV_EMPTY + i), 1);
     }
     for (int i = 0; i < BW_ST; ++i) {
-      mbar_init(bar(Q_FULL + i), 1 + 32);   // TMA arrival + 32 lanes of per-query values
+      mbar_init(bar(Q_FULL + i), 1);   // lane 0's arrival with the byte count
       mbar_init(bar(Q_EMPTY + i), 1);
     }
     mbar_init(bar(S_FULL), 1);
@@ -828,33 +840,47 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
         const int st = gb % BW_ST;
         const uint32_t ph = (gb / BW_ST) & 1;
         const int q0 = (I.qb_lo + i) * BW_QB;
-        // per-query values into registers before the stage is free
+        // per-query values (base-2 lse, D, document start): a full block with
+        // 16-byte aligned rows moves by bulk copy with the Q / dO tiles; a
+        // ragged one by lane loads (queries past T get INT_MAX starts)
+        const long lo_ = (long)I.bh * T + q0, ds_ = I.rowbase + q0;
+        const bool bulk = q0 + BW_QB <= T && ((lo_ | ds_) & 3) == 0;
         float l2v[4], dv[4];
         int dsv[4];
+        if (!bulk) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int qq = q0 + lane + 32 * e;
-          const bool v = qq < T;
-          l2v[e] = v ? lse[(long)I.bh * T + qq] * LOG2E_F : 0.f;
-          dv[e] = v ? Dbuf[(long)I.bh * T + qq] : 0.f;
-          dsv[e] = v ? I.dsr[qq] : 0x7fffffff;
+          for (int e = 0; e < 4; ++e) {
+            const int qq = q0 + lane + 32 * e;
+            const bool v = qq < T;
+            l2v[e] = v ? lse[(long)I.bh * T + qq] : 0.f;
+            dv[e] = v ? Dbuf[(long)I.bh * T + qq] : 0.f;
+            dsv[e] = v ? I.dsr[qq] : 0x7fffffff;
+          }
         }
         if (!mbar_wait(bar(Q_EMPTY + st), ph ^ 1, abort_flag)) { ok = false; break; }
-        if (lane == 0) {
-          mbar_expect_tx(bar(Q_FULL + st), 2 * AT_TILE_BYTES);
-          tma_load_2d(sQ + st * AT_TILE_BYTES, &tmQKV, bar(Q_FULL + st), I.h * AT_D, (int)(I.rowbase + q0));
-          tma_load_2d(sDO + st * AT_TILE_BYTES, &tmDO, bar(Q_FULL + st), I.h * AT_D, (int)(I.rowbase + q0));
-        }
         float* L2 = aux + st * 3 * BW_QB;
         float* Dq = L2 + BW_QB;
         int* DSq = reinterpret_cast<int*>(Dq + BW_QB);
+        if (!bulk) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          L2[lane + 32 * e] = l2v[e];
-          Dq[lane + 32 * e] = dv[e];
-          DSq[lane + 32 * e] = dsv[e];
+          for (int e = 0; e < 4; ++e) {
+            L2[lane + 32 * e] = l2v[e];
+            Dq[lane + 32 * e] = dv[e];
+            DSq[lane + 32 * e] = dsv[e];
+          }
+          __syncwarp();   // the lanes' values precede lane 0's arrival (release)
         }
-        mbar_arrive(bar(Q_FULL + st));   // release: the values above are visible to whoever waits on q_full
+        if (lane == 0) {
+          mbar_expect_tx(bar(Q_FULL + st), 2 * AT_TILE_BYTES + (bulk ? 3 * BW_QB * 4 : 0));
+          tma_load_2d(sQ + st * AT_TILE_BYTES, &tmQKV, bar(Q_FULL + st), I.h * AT_D, (int)(I.rowbase + q0));
+          tma_load_2d(sDO + st * AT_TILE_BYTES, &tmDO, bar(Q_FULL + st), I.h * AT_D, (int)(I.rowbase + q0));
+          if (bulk) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            bulk_g2s(smem_u32(L2), lse + lo_, BW_QB * 4, bar(Q_FULL + st));
+            bulk_g2s(smem_u32(Dq), Dbuf + lo_, BW_QB * 4, bar(Q_FULL + st));
+            bulk_g2s(smem_u32(DSq), dstart + ds_, BW_QB * 4, bar(Q_FULL + st));
+          }
+        }
       }
     }
     if (!ok && lane == 0) trap_timeout(abort_flag, err);

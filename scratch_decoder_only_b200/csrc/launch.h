@@ -145,6 +145,9 @@ struct AttnLayout {
 AttnLayout attn_layout_mha(bf16* dqkv, int C);
 // f16: the 16-bit tensors hold fp16 values (same layouts; bf16 otherwise);
 // lay: null for one key / value head per query head
+// lse of the tcgen05 pair is the base-2 log-sum-exp of the scaled scores
+// (log2e / sqrt(d) units), the form its backward consumes; the SIMT and
+// mma.sync pairs keep the natural log.
 cudaError_t launch_attn_fwd_tc(const bf16* qkv, bf16* out, float* lse, const int* dstart, int B, int T, int H,
                                unsigned* err, cudaStream_t s, bool f16 = false, const AttnLayout* lay = nullptr);
 // d_ready: Dbuf [B, H, T] already holds rowsum(dO o O) (written by the GEMM
