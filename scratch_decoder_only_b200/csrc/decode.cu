@@ -393,9 +393,30 @@ __global__ void argmax_kernel(const float* __restrict__ logits, int V, int Vp, i
   const float* z = logits + (long)b * Vp;
   float best = -INFINITY;
   int bi = 0x7fffffff;
-  for (int c = threadIdx.x; c < V; c += blockDim.x) {
-    float v = z[c];
-    if (v > best || (v == best && c < bi)) { best = v; bi = c; }
+  auto take = [&](float v, int c) {
+    if (c < V && (v > best || (v == best && c < bi))) { best = v; bi = c; }
+  };
+  // 16-byte aligned rows (Vp % 4 == 0, so 4 ceil(V / 4) <= Vp): four columns
+  // per load and four loads in flight per thread; columns from V on are padding
+  const bool vec = (Vp & 3) == 0 && (reinterpret_cast<uintptr_t>(logits) & 15) == 0;
+  const int nv = vec ? (V + 3) >> 2 : 0;
+  const float4* z4 = reinterpret_cast<const float4*>(z);
+  if (!vec)
+    for (int c = threadIdx.x; c < V; c += blockDim.x) take(z[c], c);
+  int q = threadIdx.x;
+  for (; q + 3 * (int)blockDim.x < nv; q += 4 * blockDim.x) {
+    float4 w[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) w[u] = z4[q + u * blockDim.x];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = 4 * (q + u * blockDim.x);
+      take(w[u].x, c); take(w[u].y, c + 1); take(w[u].z, c + 2); take(w[u].w, c + 3);
+    }
+  }
+  for (; q < nv; q += blockDim.x) {
+    const float4 w = z4[q];
+    take(w.x, 4 * q); take(w.y, 4 * q + 1); take(w.z, 4 * q + 2); take(w.w, 4 * q + 3);
   }
   __shared__ float sv[32];
   __shared__ int si[32];

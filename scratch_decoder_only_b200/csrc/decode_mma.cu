@@ -1,109 +1,159 @@
-// Decode projections for 9 to 32 rows ("RustGPT", "Technical implementation":
-// greedy decoding; "NTransformer" page, "No PyTorch, no cuBLAS": per-token
-// projections over a KV-cached step): y[b, n] = sum_k x[b, k] W[n, k] with
-// the epilogues of the decode GEMV (bias + residual, bias + GELU, fp32
-// logits).
+// Decode projections of 1 to 32 rows on the tensor cores ("RustGPT",
+// "Technical implementation": greedy decoding; "NTransformer" page, "No
+// PyTorch, no cuBLAS": per-token projections over a KV-cached step):
+// y[b, n] = sum_k x[b, k] W[n, k] with the epilogues of the decode GEMV
+// (bias + residual, bias + GELU, fp32 logits).
 //
 // A decode step reads every weight once and multiplies it by a handful of
-// rows, so the work is a weight stream: the tensor-core GEMM's 128-row tiles
-// leave 3-12 CTAs busy on the 768-column projections at 32 rows.  Here the
-// weights are cut into 16-row slices spread over every SM; each slice (16
-// contiguous rows) moves into shared memory by one bulk copy, several slices
-// in flight per CTA, and the CTA's eight warps split the slice's k range,
-// each multiplying on the tensor cores with mma.sync m16n8k16 (A = 16 rows of
-// x, read from global memory and L1; B = the slice from shared memory).  The
-// warps' partial tiles are summed in a fixed order in shared memory before
-// the epilogue, so results are deterministic.  Weight copies are issued
-// before the programmatic-dependent-launch wait: the stream starts while the
+// rows, so the work is a weight stream.  The weights are cut into 16-row
+// slices spread over every SM, two CTAs per SM.  A CTA owns one k range of
+// the input (all of K up to DM_KC columns, else a 1/nkc share) and a list of
+// slices:
+//   - each slice's k range moves into a ring of nbuf shared-memory slots by
+//     bulk copy (one copy for a whole-K slice, whose 16 rows are contiguous;
+//     one per row for a share of K), several slices in flight;
+//   - the eight warps split the k range in 32-column blocks and multiply
+//     with mma.sync m16n8k16, each warp keeping its blocks of x in registers
+//     as A fragments for the whole launch (loaded once from global memory);
+//   - the k order inside a 32-column block is permuted, the same way for x
+//     and W (a sum over k does not depend on its order): lane (g, t) takes
+//     columns 8t .. 8t + 7 of row g with one 16-byte load, columns 8t + 0..3
+//     serving the block's first MMA and 8t + 4..7 its second.  One 16-byte
+//     shared-memory load per lane and n tile then yields the B fragments of
+//     two MMAs, with at most two lanes of a quarter-warp on the same banks
+//     (ldmatrix of rows K * 2 bytes apart would put all eight on them);
+//   - the warps' partial tiles are summed in a fixed order in shared memory.
+// With a split k range each CTA writes its partial tile to a workspace and
+// the last of the slice's nkc CTAs (a per-slice arrival counter, reset by
+// that CTA) adds the nkc partials in k order and runs the epilogue: results
+// do not depend on which CTA finishes last.  Weight copies are issued before
+// the programmatic-dependent-launch wait: the stream starts while the
 // previous kernel drains.
 #include "launch.h"
 #include "tc_common.cuh"
 
 #define DM_THREADS 256
 #define DM_WARPS (DM_THREADS / 32)
-#define DM_ROWS 16        // weight rows per slice
-#define DM_MAXBUF 4       // slice buffers (at most)
+#define DM_ROWS 16                 // weight rows per slice
+#define DM_KC 768                  // k columns of one CTA's range (at most)
+#define DM_KB (DM_KC / 32 / DM_WARPS)   // 32-column blocks per warp (at most)
+#define DM_MAXBUF 6                // slice slots (at most)
+#define DM_SMEM_BUDGET (110 * 1024)     // two CTAs per SM
+#define DM_MAX_SPLIT 16
 
 template <bool F16>
-__device__ __forceinline__ void dm_mma(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+__device__ __forceinline__ void dm_mma(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                       uint32_t b1) {
   if constexpr (F16)
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
         "{%0, %1, %2, %3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
   else
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
         "{%0, %1, %2, %3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ void dm_ldmatrix_x4(uint32_t* r, uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
+__device__ __forceinline__ uint4 dm_lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
 }
 
-// MT = 16-row tiles of x (B <= 16 MT).  smem: nbuf slices of [16][K] 16-bit
-// values, then the warps' partial tiles [DM_WARPS][16 MT][16] fp32.  (The
-// ldmatrix reads of a slice meet bank conflicts, rows being K * 2 bytes
-// apart; they are a few hundred cycles per slice against microseconds of
-// copy, and one bulk copy per slice instead of one per padded row is what
-// keeps the weight stream at HBM speed.)
+template <typename T>
+__device__ __forceinline__ void dm_epilogue(float y, int bb, int n, int N, const float* bias, const T* resid, int mode,
+                                            T* out, T* out2, float* outf) {
+  const long oi = (long)bb * N + n;
+  if (mode == 2) {
+    outf[oi] = y;
+  } else if (mode == 1) {
+    const T uq = from_f<T>(y + bias[n]);
+    out[oi] = uq;
+    out2[oi] = from_f<T>(gelu_f(to_f(uq)));
+  } else {
+    out[oi] = from_f<T>(y + (bias ? bias[n] : 0.f) + (resid ? to_f(resid[oi]) : 0.f));
+  }
+}
+
+// MT = 16-row tiles of x (B <= 16 MT).  Grid = ngrp groups x nkc k ranges;
+// CTA (grp, kc) takes columns [kc kcl, min(K, (kc + 1) kcl)) of every slice
+// grp + j ngrp.  Shared memory: nbuf slots of [16 rows][kcl] 16-bit values,
+// then the warps' partial tiles [DM_WARPS][16 MT][16] fp32.
 template <typename T, int MT>
-__global__ void __launch_bounds__(DM_THREADS)
-dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, int N, const float* __restrict__ bias,
-               const T* resid, int mode, T* out, T* out2, float* outf, int nbuf, unsigned* err) {
+__global__ void __launch_bounds__(DM_THREADS, 2)
+dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, int N, int nkc, int kcl,
+               const float* __restrict__ bias, const T* resid, int mode, T* out, T* out2, float* outf, float* ws,
+               unsigned* cnt, int nbuf, unsigned* err) {
   constexpr bool F16 = std::is_same<T, f16>::value;
   extern __shared__ __align__(128) uint8_t dm_smem[];
   __shared__ __align__(8) uint64_t bars[DM_MAXBUF];
-  __shared__ int s_abort;
-  const int ldw = K;
-  const uint32_t slice_bytes = (uint32_t)DM_ROWS * ldw * 2;
-  float* red = reinterpret_cast<float*>(dm_smem + nbuf * slice_bytes);
+  __shared__ int s_abort, s_last;
+  const int kc = blockIdx.x % nkc, grp = blockIdx.x / nkc, ngrp = gridDim.x / nkc;
+  const int k0 = kc * kcl, kn = min(kcl, K - k0);   // this CTA's columns [k0, k0 + kn), kn % 32 == 0
   const int nslices = (N + DM_ROWS - 1) / DM_ROWS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tig = lane & 3;
   int nmine = 0;
-  for (int sl = blockIdx.x; sl < nslices; sl += gridDim.x) ++nmine;
-  const uint32_t smem0 = smem_u32(dm_smem);
+  for (int sl = grp; sl < nslices; sl += ngrp) ++nmine;
+  const uint32_t slot0 = smem_u32(dm_smem), slot_bytes = (uint32_t)DM_ROWS * kcl * 2;
+  float* red = reinterpret_cast<float*>(dm_smem + nbuf * slot_bytes);
   if (threadIdx.x == 0) {
     for (int i = 0; i < nbuf; ++i) mbar_init(smem_u32(&bars[i]), 1);
     s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  // thread 0: slice i of this CTA (rows r0 .. r0 + rr - 1, contiguous) into
-  // buffer i % nbuf with one bulk copy
-  auto issue = [&](int i) {
-    const int r0 = (blockIdx.x + i * gridDim.x) * DM_ROWS, rr = min(DM_ROWS, N - r0);
-    const uint32_t dst = smem0 + (i % nbuf) * slice_bytes, bar = smem_u32(&bars[i % nbuf]);
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    mbar_expect_tx(bar, (uint32_t)rr * K * 2);
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(dst), "l"(reinterpret_cast<uint64_t>(W + (long)r0 * K)), "r"((uint32_t)rr * K * 2), "r"(bar)
-                 : "memory");
+  // thread 0: this CTA's k range of slice j (rows past N are not copied)
+  // into slot j % nbuf, rows kcl values apart
+  auto issue = [&](int j) {
+    const int r0 = (grp + j * ngrp) * DM_ROWS, rr = min(DM_ROWS, N - r0);
+    const uint32_t dst = slot0 + (j % nbuf) * slot_bytes, bar = smem_u32(&bars[j % nbuf]);
+    mbar_expect_tx(bar, (uint32_t)rr * kn * 2);
+    if (nkc == 1) {
+      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                   ::"r"(dst), "l"(reinterpret_cast<uint64_t>(W + (long)r0 * K)), "r"((uint32_t)rr * K * 2),
+                   "r"(bar) : "memory");
+    } else {
+      for (int r = 0; r < rr; ++r)
+        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                     ::"r"(dst + (uint32_t)r * kcl * 2), "l"(reinterpret_cast<uint64_t>(W + (long)(r0 + r) * K + k0)),
+                     "r"((uint32_t)kn * 2), "r"(bar) : "memory");
+    }
   };
   int issued = 0;
   if (threadIdx.x == 0)
     for (; issued < nbuf && issued < nmine; ++issued) issue(issued);
-  // x, the residual and the outputs belong to the previous kernel until here
+  // x, the residual, the outputs and the workspace belong to the previous kernel until here
   griddep_wait();
   griddep_release();
-  // ldmatrix.x4 row addresses: matrices (rows 0-7, k0), (rows 0-7, k0 + 8),
-  // (rows 8-15, k0), (rows 8-15, k0 + 8) -> B fragments of two 8-row n tiles
-  const int lrow = (lane & 7) + ((lane >> 4) << 3), lcol = ((lane >> 3) & 1) * 8;
-  int i = 0;
-  for (; i < nmine; ++i) {
-    const int r0 = (blockIdx.x + i * gridDim.x) * DM_ROWS;
-    // a timed-out wait is voted block-wide so that every thread leaves together
-    const bool okw = mbar_wait(smem_u32(&bars[i % nbuf]), (i / nbuf) & 1, &s_abort);
-    if (__syncthreads_or(!okw)) {
-      if (threadIdx.x == 0) set_dev_err(err, GPT_DEVERR_TIMEOUT);
-      break;
-    }
+  // A fragments: this warp's 32-column blocks kb = warp + 8 j of the range;
+  // lane (g, t) holds columns 8t .. 8t + 7 of x rows g and g + 8 of each tile
+  uint4 xa[DM_KB][MT][2];
+#pragma unroll
+  for (int j = 0; j < DM_KB; ++j) {
+    const int col = 32 * (warp + DM_WARPS * j) + 8 * tig;
+#pragma unroll
+    for (int bt = 0; bt < MT; ++bt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int r = bt * 16 + h * 8 + g;
+        xa[j][bt][h] = (col < kn && r < B) ? *reinterpret_cast<const uint4*>(X + (long)r * K + k0 + col)
+                                           : make_uint4(0u, 0u, 0u, 0u);
+      }
+  }
+  // A timed-out wait is voted block-wide; the CTA then runs its remaining
+  // slices without data so that every slice counter still receives its nkc
+  // arrivals (and returns to zero), and drains its copies before leaving.
+  bool dead = false;
+  int landed = 0;   // slices whose copies completed
+  for (int j = 0; j < nmine; ++j) {
+    const int s = grp + j * ngrp, r0 = s * DM_ROWS;
+    if (!dead) dead = __syncthreads_or(!mbar_wait(smem_u32(&bars[j % nbuf]), (j / nbuf) & 1, &s_abort));
+    if (!dead) landed = j + 1;
     float acc[MT][2][4];
 #pragma unroll
     for (int bt = 0; bt < MT; ++bt)
@@ -111,22 +161,23 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[bt][nt][e] = 0.f;
-    const uint32_t ws = smem0 + (i % nbuf) * slice_bytes + (uint32_t)(lrow * ldw + lcol) * 2;
-#pragma unroll 2
-    for (int ks = warp; ks < K / 16; ks += DM_WARPS) {
-      const int k0 = ks * 16;
-      uint32_t b[4];
-      dm_ldmatrix_x4(b, ws + k0 * 2);
+    if (!dead) {
+      const uint32_t slot = slot0 + (j % nbuf) * slot_bytes;
 #pragma unroll
-      for (int bt = 0; bt < MT; ++bt) {
-        const int ra = bt * 16 + g, rb = ra + 8;
-        uint32_t a[4];
-        a[0] = ra < B ? *reinterpret_cast<const uint32_t*>(X + (long)ra * K + k0 + 2 * tig) : 0u;
-        a[1] = rb < B ? *reinterpret_cast<const uint32_t*>(X + (long)rb * K + k0 + 2 * tig) : 0u;
-        a[2] = ra < B ? *reinterpret_cast<const uint32_t*>(X + (long)ra * K + k0 + 2 * tig + 8) : 0u;
-        a[3] = rb < B ? *reinterpret_cast<const uint32_t*>(X + (long)rb * K + k0 + 2 * tig + 8) : 0u;
-        dm_mma<F16>(acc[bt][0], a, b[0], b[1]);
-        dm_mma<F16>(acc[bt][1], a, b[2], b[3]);
+      for (int jj = 0; jj < DM_KB; ++jj) {
+        const int col = 32 * (warp + DM_WARPS * jj) + 8 * tig;
+        if (32 * (warp + DM_WARPS * jj) < kn) {
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            const uint4 w = dm_lds128(slot + (uint32_t)((nt * 8 + g) * kcl + col) * 2);
+#pragma unroll
+            for (int bt = 0; bt < MT; ++bt) {
+              const uint4 p = xa[jj][bt][0], q = xa[jj][bt][1];
+              dm_mma<F16>(acc[bt][nt], p.x, q.x, p.y, q.y, w.x, w.y);
+              dm_mma<F16>(acc[bt][nt], p.z, q.z, p.w, q.w, w.z, w.w);
+            }
+          }
+        }
       }
     }
     // this warp's partial tile: rows b = x rows, columns n = slice rows
@@ -141,47 +192,59 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
         rw[8 * 16 + 1] = acc[bt][nt][3];
       }
     __syncthreads();
-    // every ldmatrix of this buffer is done: refill it
-    if (threadIdx.x == 0 && issued < nmine) issue(issued++);
+    // every read of this slot is done: refill it
+    if (threadIdx.x == 0 && !dead && issued < nmine) issue(issued++);
     for (int o = threadIdx.x; o < B * DM_ROWS; o += DM_THREADS) {
       const int bb = o / DM_ROWS, nn = o % DM_ROWS, n = r0 + nn;
       if (n >= N) continue;
       float y = 0.f;
 #pragma unroll
       for (int w = 0; w < DM_WARPS; ++w) y += red[((w * 16 * MT) + bb) * 16 + nn];
-      const long oi = (long)bb * N + n;
-      if (mode == 2) {
-        outf[oi] = y;
-      } else if (mode == 1) {
-        const T uq = from_f<T>(y + bias[n]);
-        out[oi] = uq;
-        out2[oi] = from_f<T>(gelu_f(to_f(uq)));
-      } else {
-        out[oi] = from_f<T>(y + (bias ? bias[n] : 0.f) + (resid ? to_f(resid[oi]) : 0.f));
+      if (nkc == 1) dm_epilogue<T>(y, bb, n, N, bias, resid, mode, out, out2, outf);
+      else ws[((long)kc * B + bb) * N + n] = y;
+    }
+    if (nkc > 1) {
+      __threadfence();
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        const unsigned prev = atomicAdd(&cnt[s], 1u);
+        s_last = prev == (unsigned)(nkc - 1);
+        if (s_last) atomicExch(&cnt[s], 0u);   // ready for the next launch
+      }
+      __syncthreads();
+      if (s_last) {
+        __threadfence();
+        for (int o = threadIdx.x; o < B * DM_ROWS; o += DM_THREADS) {
+          const int bb = o / DM_ROWS, n = r0 + o % DM_ROWS;
+          if (n >= N) continue;
+          float y = 0.f;
+          for (int q = 0; q < nkc; ++q) y += __ldcg(&ws[((long)q * B + bb) * N + n]);
+          dm_epilogue<T>(y, bb, n, N, bias, resid, mode, out, out2, outf);
+        }
       }
     }
     __syncthreads();   // the partial tiles are rewritten by the next slice
   }
-  // after a timeout: let the copies still in flight land before leaving
-  if (threadIdx.x == 0) {
+  if (dead && threadIdx.x == 0) {
+    set_dev_err(err, GPT_DEVERR_TIMEOUT);
+    // let the copies still in flight land before leaving
     volatile int never = 0;
-    for (int j = i; j < issued; ++j) mbar_wait(smem_u32(&bars[j % nbuf]), (j / nbuf) & 1, &never, 1ll << 28);
+    for (int q = landed; q < issued; ++q) mbar_wait(smem_u32(&bars[q % nbuf]), (q / nbuf) & 1, &never, 1ll << 28);
   }
 }
 
 static int g_dm_sms = 0;
 
 bool dec_mma_supported(int B, int K, int N) {
-  if (B < 1 || B > 32 || K < 16 || K % 16 || N < 1) return false;
-  const size_t slice = (size_t)DM_ROWS * K * 2, red = (size_t)DM_WARPS * 32 * 16 * 4;
-  return 2 * slice + red <= 227 * 1024;
+  return B >= 1 && B <= 32 && K >= 32 && K % 32 == 0 && N >= 1 && K <= DM_KC * DM_MAX_SPLIT;
 }
 
 template <typename T>
 cudaError_t launch_dec_mma(const T* X, int B, int K, const T* W, int N, const float* bias, const T* resid, int mode,
-                           T* out, T* out2, float* outf, unsigned* err, cudaStream_t s) {
+                           T* out, T* out2, float* outf, float* ws, size_t ws_floats, unsigned* cnt, int cnt_n,
+                           unsigned* err, cudaStream_t s) {
   if (!dec_mma_supported(B, K, N)) return cudaErrorInvalidValue;
-  if (((uintptr_t)X & 3) || ((uintptr_t)W & 15)) return cudaErrorInvalidValue;
+  if (((uintptr_t)X & 15) || ((uintptr_t)W & 15)) return cudaErrorInvalidValue;
   if (!g_dm_sms) {
     int dev = 0, n = 0;
     cudaGetDevice(&dev);
@@ -189,29 +252,33 @@ cudaError_t launch_dec_mma(const T* X, int B, int K, const T* W, int N, const fl
     g_dm_sms = n > 0 ? n : 148;
   }
   const int MT = B <= 16 ? 1 : 2;
-  const size_t slice = (size_t)DM_ROWS * K * 2, red = (size_t)DM_WARPS * 16 * MT * 16 * 4;
-  // buffers: up to four slices, two CTAs per SM where they fit in ~113 KB each
-  int nbuf = (int)((113 * 1024 - red) / slice);
+  const int nslices = (N + DM_ROWS - 1) / DM_ROWS;
+  // k ranges of at most DM_KC columns, multiples of 32
+  const int nkc = (K + DM_KC - 1) / DM_KC, kcl = ((K + nkc - 1) / nkc + 31) / 32 * 32;
+  if ((nkc - 1) * kcl >= K) return cudaErrorInvalidValue;   // no empty last range
+  if (nkc > 1 && (!ws || !cnt || (size_t)nkc * B * N > ws_floats || cnt_n < nslices)) return cudaErrorInvalidValue;
+  const size_t slot = (size_t)DM_ROWS * kcl * 2, red = (size_t)DM_WARPS * 16 * MT * 16 * 4;
+  int nbuf = (int)((DM_SMEM_BUDGET - (long)red) / (long)slot);
   if (nbuf > DM_MAXBUF) nbuf = DM_MAXBUF;
   if (nbuf < 2) nbuf = 2;
-  const size_t smem = nbuf * slice + red;
-  void (*kern)(const T*, int, int, const T*, int, const float*, const T*, int, T*, T*, float*, int, unsigned*) =
-      MT == 1 ? dec_mma_kernel<T, 1> : dec_mma_kernel<T, 2>;
+  const size_t smem = nbuf * slot + red;
+  void (*kern)(const T*, int, int, const T*, int, int, int, const float*, const T*, int, T*, T*, float*, float*,
+               unsigned*, int, unsigned*) = MT == 1 ? dec_mma_kernel<T, 1> : dec_mma_kernel<T, 2>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, DM_THREADS, smem);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) return cudaErrorInvalidValue;
-  const int nslices = (N + DM_ROWS - 1) / DM_ROWS;
-  int grid = g_dm_sms * per_sm;
-  if (grid > nslices) grid = nslices;
+  const int ngrp = std::min(g_dm_sms * per_sm / nkc, nslices);
+  if (ngrp < 1) return cudaErrorInvalidValue;
   ++g_kernel_launches;
-  return launch_k(kern, dim3(grid), dim3(DM_THREADS), smem, s, X, B, K, W, N, bias, resid, mode, out, out2, outf,
-                  nbuf, err);
+  return launch_k(kern, dim3(ngrp * nkc), dim3(DM_THREADS), smem, s, X, B, K, W, N, nkc, kcl, bias, resid, mode, out,
+                  out2, outf, ws, cnt, nbuf, err);
 }
 
 template cudaError_t launch_dec_mma<bf16>(const bf16*, int, int, const bf16*, int, const float*, const bf16*, int,
-                                          bf16*, bf16*, float*, unsigned*, cudaStream_t);
+                                          bf16*, bf16*, float*, float*, size_t, unsigned*, int, unsigned*,
+                                          cudaStream_t);
 template cudaError_t launch_dec_mma<f16>(const f16*, int, int, const f16*, int, const float*, const f16*, int, f16*,
-                                         f16*, float*, unsigned*, cudaStream_t);
+                                         f16*, float*, float*, size_t, unsigned*, int, unsigned*, cudaStream_t);

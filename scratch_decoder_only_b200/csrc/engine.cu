@@ -59,6 +59,10 @@ struct gpt_model {
   DevScalars* sc;
   void *kc, *vc, *dx, *dh, *dq, *datt, *du, *da, *dxf;
   float *dlogits, *dmu, *drs, *dpart;
+  float* dmws = nullptr;        // decode projections: partial tiles of a split k range
+  unsigned* dmcnt = nullptr;    // and their per-slice arrival counters (kept zero)
+  size_t dmws_n = 0;
+  int dmcnt_n = 0;
   float* dam;      // fused decode: per-CTA argmax partials [Bmax][DF_MAX_GRID] values, then indices
   int* dtok;
   int fwd_B = 0, fwd_T = 0;
@@ -368,6 +372,10 @@ static int build_arena(gpt_model* m) {
   cv.add((void**)&m->drs, Bx * 4);
   cv.add((void**)&m->dtok, Bx * 4);
   cv.add((void**)&m->dpart, dec_attn_part_floats((int)Bx, m->H, m->d) * 4);
+  m->dmws_n = 16 * Bx * (size_t)std::max<long>(std::max<long>(3 * C, m->UW), F);
+  m->dmcnt_n = (int)((std::max<long>(std::max<long>(3 * C, m->UW), std::max<long>(F, m->Vp)) + 15) / 16);
+  cv.add((void**)&m->dmws, m->dmws_n * 4);
+  cv.add((void**)&m->dmcnt, (size_t)m->dmcnt_n * 4);
   cv.add((void**)&m->dam, Bx * DF_MAX_GRID * 8);   // fused decode: per-CTA argmax partials
   cv.add((void**)&m->dsrc, Bx * (size_t)m->Tmax * 4);
   cv.add((void**)&m->dbcs, Bx * BEAM_MAX_WIDTH * 4);
@@ -382,6 +390,8 @@ static int build_arena(gpt_model* m) {
     return GPT_ERR_NOMEM;
   }
   for (auto& it : cv.items) *it.first = m->arena + it.second;
+  e = cudaMemset(m->dmcnt, 0, (size_t)m->dmcnt_n * 4);
+  if (e != cudaSuccess) { m->err = std::string("cudaMemset: ") + cudaGetErrorString(e); return GPT_ERR_CUDA; }
   if (!m->lp) m->pw = m->p32;
   return GPT_OK;
 }
@@ -899,7 +909,8 @@ static cudaError_t dec_proj(gpt_model* m, const T* X, int B, int K, const T* W, 
                             const T* resid, int mode, T* out, T* out2, float* outf, cudaStream_t s) {
   if constexpr (sizeof(T) == 2) {
     if (B > 8 && dec_mma_supported(B, K, N))
-      return launch_dec_mma<T>(X, B, K, W, N, bias, resid, mode, out, out2, outf, &m->sc->err, s);
+      return launch_dec_mma<T>(X, B, K, W, N, bias, resid, mode, out, out2, outf, m->dmws, m->dmws_n, m->dmcnt,
+                               m->dmcnt_n, &m->sc->err, s);
   }
   return launch_gemv<T>(X, B, K, W, N, bias, resid, mode, out, out2, outf, s);
 }

@@ -196,13 +196,18 @@ cudaError_t launch_sample(const float* logits, int B, int V, int Vp, float temp,
 template <typename T>
 cudaError_t launch_gather_last(const T* x, int B, int Tp, int C, T* out, cudaStream_t s);
 
-// ---- decode_mma.cu: decode projections of 9-32 rows on mma.sync (16-bit T),
+// ---- decode_mma.cu: decode projections of 1-32 rows on mma.sync (16-bit T),
 // same modes and outputs as the GEMV (0: + bias + residual, 1: + bias and
-// GELU into out / out2, 2: fp32 logits)
+// GELU into out / out2, 2: fp32 logits).  X and W 16-byte aligned.  ws
+// (ws_floats floats) holds the partial tiles of a split k range and cnt
+// (cnt_n counters, zero before the first launch; every launch leaves them
+// zero) the per-slice arrivals; with too small a workspace the k range is not
+// split.
 bool dec_mma_supported(int B, int K, int N);
 template <typename T>
 cudaError_t launch_dec_mma(const T* X, int B, int K, const T* W, int N, const float* bias, const T* resid, int mode,
-                           T* out, T* out2, float* outf, unsigned* err, cudaStream_t s);
+                           T* out, T* out2, float* outf, float* ws, size_t ws_floats, unsigned* cnt, int cnt_n,
+                           unsigned* err, cudaStream_t s);
 
 // ---- beam.cu: beam search over the decode rows (row r = b * W + w)
 #define BEAM_MAX_WIDTH 8
