@@ -217,15 +217,22 @@ cudaError_t launch_kv_fill(const T* qkv, T* kc, T* vc, int B, int Tp, int d, int
   return cudaGetLastError();
 }
 
-// Split decode attention: grid (B*H, DA_SPLITS); the first `act` splits
-// of a (row, head) take the keys (act grows with the context, one split per
-// 64 keys, so that a short context is not spread over mostly idle blocks);
-// block (bh, sp < act) takes key groups sp, sp + act, ... and keeps an online
-// softmax (max, sum, output) per 8-lane group, each lane holding 8 of the
-// head's dimensions (one 16-byte load of a key or value row).  Its partial
-// (m, l, o[D]) goes to part[bh][sp]; splits past act write an empty partial.
-// dec_attn_combine merges the splits.  The new key / value of this step are
-// read from qkv, and written to the cache by split 0.
+// Decode attention of the new query over the cache ("NTransformer" page,
+// KV cache; "Feste", scaled dot-product attention with the causal mask):
+// o = softmax(q K^T / sqrt(D)) V over keys 0 .. pos of the (row, head).
+// Grid (B*H, S): the key range of a (row, head) is cut into act <= S
+// contiguous pieces (act grows with the context, one per 64 keys), one CTA
+// each; S is chosen so that about two CTAs per SM have work.  A CTA's four
+// warps take 4 * (32 / (D / 8)) * U consecutive keys per pass (128 for D = 64
+// in 16 bits), a lane group of D / 8 lanes per key and U keys per lane group
+// in flight (each lane one load of 8 values of a key and of a value row,
+// kept packed until used), with an online softmax (max, sum, output) per lane
+// group updated once per U keys.  The lane groups and warps
+// merge in a fixed order; with act = 1 the CTA writes the output, otherwise
+// its partial (m, l, o[D]) goes to part and the last CTA of the (row, head)
+// (an arrival counter that it resets) merges the act partials in key order.
+// The new key / value of this step come from qkv and are written to the
+// cache by piece 0.
 #define DA_SPLITS 16
 #define DA_THREADS 128
 template <typename T>
@@ -233,23 +240,44 @@ __device__ __forceinline__ void load8(const T* p, float* v) {
 #pragma unroll
   for (int i = 0; i < 8; i += Vec<T>::N) Vec<T>::load(p + i, v + i);
 }
+__device__ __forceinline__ int dec_attn_act(int pos, int S) { return min(S, (pos + 64) / 64); }
+// 8 values of T kept packed in registers
+template <typename T>
+struct Pack8 {
+  uint4 w[sizeof(T) / 2];
+};
+template <typename T>
+__device__ __forceinline__ Pack8<T> ld_pack8(const T* p) {
+  Pack8<T> r;
+#pragma unroll
+  for (int i = 0; i < (int)(sizeof(T) / 2); ++i) r.w[i] = reinterpret_cast<const uint4*>(p)[i];
+  return r;
+}
+template <typename T>
+__device__ __forceinline__ void unpack8(const Pack8<T>& r, float* v) {
+  load8(reinterpret_cast<const T*>(r.w), v);
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(DA_THREADS)
-dec_attn_split_kernel(const T* __restrict__ qkv, T* kc, T* vc, float* __restrict__ part, int B, int H, int Tmax,
-                      int pos0, const int* __restrict__ step, DecLayout Ly) {
+dec_attn_kernel(const T* __restrict__ qkv, T* kc, T* vc, T* __restrict__ out, float* part, unsigned* cnt, int B,
+                int H, int Tmax, int pos0, const int* __restrict__ step, DecLayout Ly) {
   griddep_wait();
   griddep_release();
   static_assert(D % 8 == 0 && D <= 256, "head size");
   constexpr int LPK = D / 8;            // lanes per key row (16 bytes each)
-  constexpr int KPW = 32 / LPK;         // keys per warp pass
+  constexpr int KPW = 32 / LPK;         // lane groups (keys) per warp
   constexpr int NW = DA_THREADS / 32;
+  constexpr int U = sizeof(T) == 2 ? 8 : 4;   // keys per lane group in flight
+  constexpr int KPP = NW * KPW * U;           // keys per CTA pass
   int pos = pos0 + *step;
   if (pos < 0) pos = 0;
   if (pos >= Tmax) pos = Tmax - 1;
   const int bh = blockIdx.x, sp = blockIdx.y;
+  const int act = dec_attn_act(pos, gridDim.y);
+  if (sp >= act) return;
   const int b = bh / H, h = bh % H;
   const int G = H / Ly.Hkv, hk = h / G;   // query head h reads key/value head hk
-  const int act = min(DA_SPLITS, pos / 64 + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = lane / LPK, sub = lane % LPK;
   const T* q = qkv + (long)b * Ly.qw + h * D;
@@ -269,38 +297,58 @@ dec_attn_split_kernel(const T* __restrict__ qkv, T* kc, T* vc, float* __restrict
   float m = -INFINITY, l = 0.f, o[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) o[i] = 0.f;
-  // key j belongs to this split when (j / KPW) % (act * NW) == sp * NW + warp
-  // (no key at all for sp >= act: the partial stays empty)
-  for (int j0 = sp < act ? (sp * NW + warp) * KPW : pos + 1; j0 <= pos; j0 += act * NW * KPW) {
-    const int j = j0 + grp;
-    const bool live = j <= pos;
-    long row = (long)j * D;
-    if (Ly.src && j < pos) row += ((long)Ly.src[(long)b * Tmax + j] - b) * Ly.Hkv * Tmax * D;
-    const T* kr = j == pos ? knew : kcb + row;
-    const T* vr = j == pos ? vnew : vcb + row;
-    float kv[8], vv[8];
-    if (live) {
-      load8(kr + sub * 8, kv);
-      load8(vr + sub * 8, vv);
-    } else {
+  // this piece's keys [j_lo, j_hi)
+  const int per = (pos + act) / act;   // ceil((pos + 1) / act)
+  const int j_lo = sp * per, j_hi = min(pos + 1, j_lo + per);
+  for (int jb = j_lo + warp * KPW * U; jb < j_hi; jb += KPP) {
+    Pack8<T> kp[U], vp[U];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) { kv[i] = 0.f; vv[i] = 0.f; }
+    for (int u = 0; u < U; ++u) {
+      const int j = jb + u * KPW + grp;
+      if (j < j_hi) {
+        long row = (long)j * D;
+        if (Ly.src && j < pos) row += ((long)Ly.src[(long)b * Tmax + j] - b) * Ly.Hkv * Tmax * D;
+        const T* kr = j == pos ? knew : kcb + row;
+        const T* vr = j == pos ? vnew : vcb + row;
+        kp[u] = ld_pack8(kr + sub * 8);
+        vp[u] = ld_pack8(vr + sub * 8);
+      } else {
+#pragma unroll
+        for (int i = 0; i < (int)(sizeof(T) / 2); ++i) { kp[u].w[i] = make_uint4(0u, 0u, 0u, 0u); vp[u].w[i] = kp[u].w[i]; }
+      }
     }
-    float sc = 0.f;
+    float sc[U];
+    float mn = m;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) sc = fmaf(qv[i], kv[i], sc);
+    for (int u = 0; u < U; ++u) {
+      float kv[8];
+      unpack8(kp[u], kv);
+      float t = 0.f;
 #pragma unroll
-    for (int o2 = LPK / 2; o2 > 0; o2 >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o2);
-    if (live) {
-      const float mn = fmaxf(m, sc);
-      const float corr = expf(m - mn), p = expf(sc - mn);
-      l = l * corr + p;
+      for (int i = 0; i < 8; ++i) t = fmaf(qv[i], kv[i], t);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) o[i] = o[i] * corr + p * vv[i];
+      for (int o2 = LPK / 2; o2 > 0; o2 >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o2);
+      sc[u] = jb + u * KPW + grp < j_hi ? t : -INFINITY;
+      mn = fmaxf(mn, sc[u]);
+    }
+    if (mn != -INFINITY) {
+      const float corr = expf(m - mn);
+      l *= corr;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] *= corr;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const float p = expf(sc[u] - mn);
+        l += p;
+        float vv[8];
+        unpack8(vp[u], vv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) o[i] = fmaf(p, vv[i], o[i]);
+      }
       m = mn;
     }
   }
-  // merge the key groups of the warp (lanes with the same sub hold the same dimensions)
+  // merge the lane groups of the warp (lanes with the same sub hold the same dimensions)
 #pragma unroll
   for (int o2 = LPK; o2 < 32; o2 <<= 1) {
     const float m2 = __shfl_xor_sync(0xffffffffu, m, o2);
@@ -314,63 +362,84 @@ dec_attn_split_kernel(const T* __restrict__ qkv, T* kc, T* vc, float* __restrict
   }
   // merge the warps through shared memory
   __shared__ float sm_m[NW], sm_l[NW], sm_o[NW][D];
+  __shared__ int s_last;
   if (lane < LPK) {
     if (lane == 0) { sm_m[warp] = m; sm_l[warp] = l; }
 #pragma unroll
     for (int i = 0; i < 8; ++i) sm_o[warp][sub * 8 + i] = o[i];
   }
   __syncthreads();
-  float* dst = part + ((long)bh * DA_SPLITS + sp) * (D + 2);
+  float mm = -INFINITY, ll = 0.f, oo = 0.f;
   if (threadIdx.x < D) {
-    float mm = -INFINITY;
 #pragma unroll
     for (int w = 0; w < NW; ++w) mm = fmaxf(mm, sm_m[w]);
-    float ll = 0.f, oo = 0.f;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
       const float f = sm_m[w] == -INFINITY ? 0.f : expf(sm_m[w] - mm);
       ll += sm_l[w] * f;
       oo += sm_o[w][threadIdx.x] * f;
     }
-    dst[2 + threadIdx.x] = oo;
-    if (threadIdx.x == 0) { dst[0] = mm; dst[1] = ll; }
   }
-}
-
-// out[b, head h] = merge of the DA_SPLITS partials of (b, h).
-template <typename T, int D>
-__global__ void dec_attn_combine_kernel(const float* __restrict__ part, T* __restrict__ out, int H) {
-  griddep_wait();
-  griddep_release();
-  const int bh = blockIdx.x, b = bh / H, h = bh % H;
-  const float* p = part + (long)bh * DA_SPLITS * (D + 2);
-  float mm = -INFINITY;
-  for (int s2 = 0; s2 < DA_SPLITS; ++s2) mm = fmaxf(mm, p[s2 * (D + 2)]);
-  for (int i = threadIdx.x; i < D; i += blockDim.x) {
-    float ll = 0.f, oo = 0.f;
-    for (int s2 = 0; s2 < DA_SPLITS; ++s2) {
-      const float ms = p[s2 * (D + 2)];
-      const float f = ms == -INFINITY ? 0.f : expf(ms - mm);
-      ll += p[s2 * (D + 2) + 1] * f;
-      oo += p[s2 * (D + 2) + 2 + i] * f;
+  T* orow = out + (long)b * H * D + h * D;
+  if (act == 1) {
+    if (threadIdx.x < D) orow[threadIdx.x] = from_f<T>(oo / ll);
+    return;
+  }
+  float* pb = part + (long)bh * DA_SPLITS * (D + 2);
+  if (threadIdx.x < D) {
+    pb[sp * (D + 2) + 2 + threadIdx.x] = oo;
+    if (threadIdx.x == 0) { pb[sp * (D + 2)] = mm; pb[sp * (D + 2) + 1] = ll; }
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned prev = atomicAdd(&cnt[bh], 1u);
+    s_last = prev == (unsigned)(act - 1);
+    if (s_last) atomicExch(&cnt[bh], 0u);   // ready for the next launch
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  if (threadIdx.x < D) {
+    float gm = -INFINITY;
+    for (int s2 = 0; s2 < act; ++s2) gm = fmaxf(gm, __ldcg(pb + s2 * (D + 2)));
+    float gl = 0.f, go = 0.f;
+    for (int s2 = 0; s2 < act; ++s2) {
+      const float ms = __ldcg(pb + s2 * (D + 2));
+      const float f = ms == -INFINITY ? 0.f : expf(ms - gm);
+      gl += __ldcg(pb + s2 * (D + 2) + 1) * f;
+      go += __ldcg(pb + s2 * (D + 2) + 2 + threadIdx.x) * f;
     }
-    out[(long)b * H * D + h * D + i] = from_f<T>(oo / ll);
+    orow[threadIdx.x] = from_f<T>(go / gl);
   }
 }
 
 size_t dec_attn_part_floats(int B, int H, int d) { return (size_t)B * H * DA_SPLITS * (d + 2); }
 
+static int g_da_sms = 0;
+
 template <typename T>
-cudaError_t launch_dec_attn(const T* qkv, T* kc, T* vc, T* out, float* part, int B, int H, int d, int Tmax, int pos0,
-                            const int* step, const DecLayout& L, cudaStream_t s) {
-  dim3 g(B * H, DA_SPLITS);
+cudaError_t launch_dec_attn(const T* qkv, T* kc, T* vc, T* out, float* part, unsigned* cnt, int B, int H, int d,
+                            int Tmax, int pos0, const int* step, const DecLayout& L, cudaStream_t s) {
+  if (!g_da_sms) {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    g_da_sms = n > 0 ? n : 148;
+  }
+  // pieces per (row, head): about two working CTAs per SM (a split costs a
+  // fence, an arrival and a merge, more than one more pass over the keys)
+  int S = (2 * g_da_sms + B * H - 1) / (B * H);
+  if (S > DA_SPLITS) S = DA_SPLITS;
+  if (S < 1) S = 1;
+  dim3 g(B * H, S);
   cudaError_t e = cudaSuccess;
   switch (d) {
 #define DA_CASE(DD)                                                                                               \
   case DD:                                                                                                        \
-    g_kernel_launches += 2;                                                                                       \
-    e = launch_k(dec_attn_split_kernel<T, DD>, g, dim3(DA_THREADS), 0, s, qkv, kc, vc, part, B, H, Tmax, pos0, step, L); \
-    if (e == cudaSuccess) e = launch_k(dec_attn_combine_kernel<T, DD>, dim3(B * H), dim3(64), 0, s, (const float*)part, out, H); \
+    g_kernel_launches += 1;                                                                                       \
+    e = launch_k(dec_attn_kernel<T, DD>, g, dim3(DA_THREADS), 0, s, qkv, kc, vc, out, part, cnt, B, H, Tmax, pos0, \
+                 step, L);                                                                                        \
     break;
     DA_CASE(16)
     DA_CASE(32)
@@ -732,7 +801,7 @@ cudaError_t launch_gather_last(const T* x, int B, int Tp, int C, T* out, cudaStr
   template cudaError_t launch_gemv<T>(const T*, int, int, const T*, int, const float*, const T*, int, T*, T*, \
                                       float*, cudaStream_t);                                             \
   template cudaError_t launch_kv_fill<T>(const T*, T*, T*, int, int, int, int, const DecLayout&, cudaStream_t); \
-  template cudaError_t launch_dec_attn<T>(const T*, T*, T*, T*, float*, int, int, int, int, int, const int*,      \
+  template cudaError_t launch_dec_attn<T>(const T*, T*, T*, T*, float*, unsigned*, int, int, int, int, int, const int*,      \
                                           const DecLayout&, cudaStream_t);                               \
   template cudaError_t launch_gather_last<T>(const T*, int, int, int, T*, cudaStream_t);
 INSTD(float)

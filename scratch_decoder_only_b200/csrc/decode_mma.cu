@@ -23,6 +23,11 @@
 //     two MMAs, with at most two lanes of a quarter-warp on the same banks
 //     (ldmatrix of rows K * 2 bytes apart would put all eight on them);
 //   - the warps' partial tiles are summed in a fixed order in shared memory.
+// A LayerNorm (or RMSNorm) of x can run in the kernel (K <= DM_KC): the CTA
+// holds all of x's columns, so the row statistics come from the registers
+// (two passes, quad shuffles and a fixed-order sum over the warps) and the
+// normalised values, rounded to 16 bits as the LayerNorm kernel stores them,
+// replace the fragments.
 // With a split k range each CTA writes its partial tile to a workspace and
 // the last of the slice's nkc CTAs (a per-slice arrival counter, reset by
 // that CTA) adds the nkc partials in k order and runs the epilogue: results
@@ -40,6 +45,9 @@
 #define DM_MAXBUF 6                // slice slots (at most)
 #define DM_SMEM_BUDGET (110 * 1024)     // two CTAs per SM
 #define DM_MAX_SPLIT 16
+#ifndef DM_CTAS
+#define DM_CTAS 2                  // CTAs per SM in the grid
+#endif
 
 template <bool F16>
 __device__ __forceinline__ void dm_mma(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
@@ -64,30 +72,35 @@ __device__ __forceinline__ uint4 dm_lds128(uint32_t addr) {
   return v;
 }
 
+// Output (bb, n) from the dot product y, the bias value pb and the residual
+// value pr (both loaded ahead, zero where absent).
 template <typename T>
-__device__ __forceinline__ void dm_epilogue(float y, int bb, int n, int N, const float* bias, const T* resid, int mode,
-                                            T* out, T* out2, float* outf) {
+__device__ __forceinline__ void dm_epilogue(float y, float pb, float pr, int bb, int n, int N, int mode, T* out,
+                                            T* out2, float* outf) {
   const long oi = (long)bb * N + n;
   if (mode == 2) {
     outf[oi] = y;
   } else if (mode == 1) {
-    const T uq = from_f<T>(y + bias[n]);
+    const T uq = from_f<T>(y + pb);
     out[oi] = uq;
     out2[oi] = from_f<T>(gelu_f(to_f(uq)));
   } else {
-    out[oi] = from_f<T>(y + (bias ? bias[n] : 0.f) + (resid ? to_f(resid[oi]) : 0.f));
+    out[oi] = from_f<T>(y + pb + pr);
   }
 }
+#define DM_OPT (16 * 32 / DM_THREADS)   // outputs per thread and slice (at most)
 
 // MT = 16-row tiles of x (B <= 16 MT).  Grid = ngrp groups x nkc k ranges;
 // CTA (grp, kc) takes columns [kc kcl, min(K, (kc + 1) kcl)) of every slice
 // grp + j ngrp.  Shared memory: nbuf slots of [16 rows][kcl] 16-bit values,
-// then the warps' partial tiles [DM_WARPS][16 MT][16] fp32.
+// the warps' partial tiles [DM_WARPS][16 MT][16] fp32, then (LayerNorm) its
+// gains and shifts [2][K] fp32.
 template <typename T, int MT>
 __global__ void __launch_bounds__(DM_THREADS, 2)
 dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, int N, int nkc, int kcl,
                const float* __restrict__ bias, const T* resid, int mode, T* out, T* out2, float* outf, float* ws,
-               unsigned* cnt, int nbuf, unsigned* err) {
+               unsigned* cnt, int nbuf, unsigned* err, const float* __restrict__ lng, const float* __restrict__ lnb,
+               float eps) {
   constexpr bool F16 = std::is_same<T, f16>::value;
   extern __shared__ __align__(128) uint8_t dm_smem[];
   __shared__ __align__(8) uint64_t bars[DM_MAXBUF];
@@ -127,6 +140,13 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
   int issued = 0;
   if (threadIdx.x == 0)
     for (; issued < nbuf && issued < nmine; ++issued) issue(issued);
+  // the LayerNorm parameters (constant) can move before the wait
+  float* lns = red + DM_WARPS * 16 * MT * 16;
+  if (lng)
+    for (int i = threadIdx.x; i < K; i += DM_THREADS) {
+      lns[i] = lng[i];
+      lns[K + i] = lnb ? lnb[i] : 0.f;
+    }
   // x, the residual, the outputs and the workspace belong to the previous kernel until here
   griddep_wait();
   griddep_release();
@@ -145,6 +165,106 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
                                            : make_uint4(0u, 0u, 0u, 0u);
       }
   }
+  if (lng) {
+    // x <- LayerNorm(x) (RMSNorm without lnb), nkc == 1: columns [0, K).
+    // Statistics with one barrier: each lane takes the mean and the sum of
+    // squared deviations (M2) of its values of a row (registers only); the
+    // quad's four equal-count parts merge pairwise by shuffles (mean' = (ma +
+    // mb) / 2, M2' = M2a + M2b + d^2 n / 2 for n values each, d = mb - ma:
+    // the pairwise update of Chan, Golub and LeVeque); the warps' parts merge
+    // in warp order as mean = sum_w n_w mean_w / K and M2 = sum_w (M2_w +
+    // n_w (mean_w - mean)^2).  RMSNorm keeps every mean 0 and sums squares.
+    float2* sred = reinterpret_cast<float2*>(red);   // [DM_WARPS][16 MT] (mean, M2) of the warp's columns
+    float mu[MT][2], rs[MT][2];
+    const int nw = min(DM_KB, (kn / 32 - warp + DM_WARPS - 1) / DM_WARPS);   // this warp's blocks in range
+    const float nl = 8.f * nw;                                             // values per lane
+    const float inl = nw > 0 ? 1.f / nl : 0.f, inK = 1.f / K;
+#pragma unroll
+    for (int bt = 0; bt < MT; ++bt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float m = 0.f, q = 0.f;
+        if (nw > 0 && bt * 16 + h * 8 + g < B) {
+          float sum = 0.f;
+#pragma unroll
+          for (int j = 0; j < DM_KB; ++j)
+            if (j < nw) {
+              float v[8];
+              unpack16x8<F16>(xa[j][bt][h], v);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) sum += v[i];
+            }
+          m = lnb ? sum * inl : 0.f;
+#pragma unroll
+          for (int j = 0; j < DM_KB; ++j)
+            if (j < nw) {
+              float v[8];
+              unpack16x8<F16>(xa[j][bt][h], v);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) q = fmaf(v[i] - m, v[i] - m, q);
+            }
+        }
+        // quad merge: four lanes with equal counts
+        float n = nl;
+#pragma unroll
+        for (int o = 1; o <= 2; o <<= 1) {
+          const float m2 = __shfl_xor_sync(0xffffffffu, m, o), q2 = __shfl_xor_sync(0xffffffffu, q, o);
+          const float d = m2 - m;
+          q = q + q2 + d * d * (0.5f * n);   // na = nb = n: d^2 na nb / (2n) = d^2 n / 2
+          m = m + 0.5f * d;
+          n *= 2.f;
+        }
+        if (tig == 0) sred[warp * 16 * MT + bt * 16 + h * 8 + g] = make_float2(m, q);
+      }
+    __syncthreads();
+#pragma unroll
+    for (int bt = 0; bt < MT; ++bt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float sm = 0.f, q = 0.f;
+#pragma unroll
+        for (int w = 0; w < DM_WARPS; ++w) {
+          const float nb = 32.f * min(DM_KB, (kn / 32 - w + DM_WARPS - 1) / DM_WARPS);
+          sm = fmaf(nb, sred[w * 16 * MT + bt * 16 + h * 8 + g].x, sm);
+        }
+        const float m = lnb ? sm * inK : 0.f;
+#pragma unroll
+        for (int w = 0; w < DM_WARPS; ++w) {
+          const float nb = 32.f * min(DM_KB, (kn / 32 - w + DM_WARPS - 1) / DM_WARPS);
+          const float2 t = sred[w * 16 * MT + bt * 16 + h * 8 + g];
+          const float d = t.x - m;
+          q += t.y + nb * d * d;
+        }
+        mu[bt][h] = m;
+        // RMSNorm: q is the sum of squares (every mean stayed 0)
+        rs[bt][h] = 1.0f / sqrtf(q / K + eps);
+      }
+#pragma unroll
+    for (int j = 0; j < DM_KB; ++j) {
+      const int col = 32 * (warp + DM_WARPS * j) + 8 * tig;
+      if (col < kn) {
+        float gv[8], bv[8];
+        *reinterpret_cast<float4*>(gv) = *reinterpret_cast<const float4*>(lns + col);
+        *reinterpret_cast<float4*>(gv + 4) = *reinterpret_cast<const float4*>(lns + col + 4);
+        *reinterpret_cast<float4*>(bv) = *reinterpret_cast<const float4*>(lns + K + col);
+        *reinterpret_cast<float4*>(bv + 4) = *reinterpret_cast<const float4*>(lns + K + col + 4);
+#pragma unroll
+        for (int bt = 0; bt < MT; ++bt)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (bt * 16 + h * 8 + g >= B) continue;   // rows past B stay zero
+            float v[8];
+            unpack16x8<F16>(xa[j][bt][h], v);
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              w[i] = pack16x2<F16>((v[2 * i] - mu[bt][h]) * rs[bt][h] * gv[2 * i] + bv[2 * i],
+                                   (v[2 * i + 1] - mu[bt][h]) * rs[bt][h] * gv[2 * i + 1] + bv[2 * i + 1]);
+            xa[j][bt][h] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+      }
+    }
+  }
   // A timed-out wait is voted block-wide; the CTA then runs its remaining
   // slices without data so that every slice counter still receives its nkc
   // arrivals (and returns to zero), and drains its copies before leaving.
@@ -152,8 +272,20 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
   int landed = 0;   // slices whose copies completed
   for (int j = 0; j < nmine; ++j) {
     const int s = grp + j * ngrp, r0 = s * DM_ROWS;
+    // the vote is also the barrier after the previous slice's reads of red
     if (!dead) dead = __syncthreads_or(!mbar_wait(smem_u32(&bars[j % nbuf]), (j / nbuf) & 1, &s_abort));
+    else __syncthreads();
     if (!dead) landed = j + 1;
+    // this thread's outputs o = threadIdx.x + DM_THREADS t: bias and residual
+    // values load while the tensor cores run
+    float pb[DM_OPT], pr[DM_OPT];
+#pragma unroll
+    for (int t = 0; t < DM_OPT; ++t) {
+      const int o = threadIdx.x + DM_THREADS * t, bb = o / DM_ROWS, n = r0 + o % DM_ROWS;
+      const bool ok = o < B * DM_ROWS && n < N;
+      pb[t] = ok && bias && mode != 2 ? bias[n] : 0.f;
+      pr[t] = ok && resid && mode == 0 ? to_f(resid[(long)bb * N + n]) : 0.f;
+    }
     float acc[MT][2][4];
 #pragma unroll
     for (int bt = 0; bt < MT; ++bt)
@@ -194,13 +326,14 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
     __syncthreads();
     // every read of this slot is done: refill it
     if (threadIdx.x == 0 && !dead && issued < nmine) issue(issued++);
-    for (int o = threadIdx.x; o < B * DM_ROWS; o += DM_THREADS) {
-      const int bb = o / DM_ROWS, nn = o % DM_ROWS, n = r0 + nn;
-      if (n >= N) continue;
+#pragma unroll
+    for (int t = 0; t < DM_OPT; ++t) {
+      const int o = threadIdx.x + DM_THREADS * t, bb = o / DM_ROWS, nn = o % DM_ROWS, n = r0 + nn;
+      if (o >= B * DM_ROWS || n >= N) continue;
       float y = 0.f;
 #pragma unroll
       for (int w = 0; w < DM_WARPS; ++w) y += red[((w * 16 * MT) + bb) * 16 + nn];
-      if (nkc == 1) dm_epilogue<T>(y, bb, n, N, bias, resid, mode, out, out2, outf);
+      if (nkc == 1) dm_epilogue<T>(y, pb[t], pr[t], bb, n, N, mode, out, out2, outf);
       else ws[((long)kc * B + bb) * N + n] = y;
     }
     if (nkc > 1) {
@@ -214,16 +347,16 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
       __syncthreads();
       if (s_last) {
         __threadfence();
-        for (int o = threadIdx.x; o < B * DM_ROWS; o += DM_THREADS) {
-          const int bb = o / DM_ROWS, n = r0 + o % DM_ROWS;
-          if (n >= N) continue;
+#pragma unroll
+        for (int t = 0; t < DM_OPT; ++t) {
+          const int o = threadIdx.x + DM_THREADS * t, bb = o / DM_ROWS, n = r0 + o % DM_ROWS;
+          if (o >= B * DM_ROWS || n >= N) continue;
           float y = 0.f;
           for (int q = 0; q < nkc; ++q) y += __ldcg(&ws[((long)q * B + bb) * N + n]);
-          dm_epilogue<T>(y, bb, n, N, bias, resid, mode, out, out2, outf);
+          dm_epilogue<T>(y, pb[t], pr[t], bb, n, N, mode, out, out2, outf);
         }
       }
     }
-    __syncthreads();   // the partial tiles are rewritten by the next slice
   }
   if (dead && threadIdx.x == 0) {
     set_dev_err(err, GPT_DEVERR_TIMEOUT);
@@ -235,15 +368,15 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
 
 static int g_dm_sms = 0;
 
-bool dec_mma_supported(int B, int K, int N) {
-  return B >= 1 && B <= 32 && K >= 32 && K % 32 == 0 && N >= 1 && K <= DM_KC * DM_MAX_SPLIT;
+bool dec_mma_supported(int B, int K, int N, bool ln) {
+  return B >= 1 && B <= 32 && K >= 32 && K % 32 == 0 && N >= 1 && K <= (ln ? DM_KC : DM_KC * DM_MAX_SPLIT);
 }
 
 template <typename T>
 cudaError_t launch_dec_mma(const T* X, int B, int K, const T* W, int N, const float* bias, const T* resid, int mode,
                            T* out, T* out2, float* outf, float* ws, size_t ws_floats, unsigned* cnt, int cnt_n,
-                           unsigned* err, cudaStream_t s) {
-  if (!dec_mma_supported(B, K, N)) return cudaErrorInvalidValue;
+                           unsigned* err, cudaStream_t s, const float* lng, const float* lnb, float eps) {
+  if (!dec_mma_supported(B, K, N, lng != nullptr)) return cudaErrorInvalidValue;
   if (((uintptr_t)X & 15) || ((uintptr_t)W & 15)) return cudaErrorInvalidValue;
   if (!g_dm_sms) {
     int dev = 0, n = 0;
@@ -257,28 +390,31 @@ cudaError_t launch_dec_mma(const T* X, int B, int K, const T* W, int N, const fl
   const int nkc = (K + DM_KC - 1) / DM_KC, kcl = ((K + nkc - 1) / nkc + 31) / 32 * 32;
   if ((nkc - 1) * kcl >= K) return cudaErrorInvalidValue;   // no empty last range
   if (nkc > 1 && (!ws || !cnt || (size_t)nkc * B * N > ws_floats || cnt_n < nslices)) return cudaErrorInvalidValue;
-  const size_t slot = (size_t)DM_ROWS * kcl * 2, red = (size_t)DM_WARPS * 16 * MT * 16 * 4;
+  const size_t slot = (size_t)DM_ROWS * kcl * 2;
+  const size_t red = (size_t)DM_WARPS * 16 * MT * 16 * 4 + (lng ? (size_t)2 * K * 4 : 0);
   int nbuf = (int)((DM_SMEM_BUDGET - (long)red) / (long)slot);
   if (nbuf > DM_MAXBUF) nbuf = DM_MAXBUF;
   if (nbuf < 2) nbuf = 2;
   const size_t smem = nbuf * slot + red;
   void (*kern)(const T*, int, int, const T*, int, int, int, const float*, const T*, int, T*, T*, float*, float*,
-               unsigned*, int, unsigned*) = MT == 1 ? dec_mma_kernel<T, 1> : dec_mma_kernel<T, 2>;
+               unsigned*, int, unsigned*, const float*, const float*, float) =
+      MT == 1 ? dec_mma_kernel<T, 1> : dec_mma_kernel<T, 2>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, DM_THREADS, smem);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) return cudaErrorInvalidValue;
-  const int ngrp = std::min(g_dm_sms * per_sm / nkc, nslices);
+  const int ngrp = std::min(g_dm_sms * std::min(per_sm, DM_CTAS) / nkc, nslices);
   if (ngrp < 1) return cudaErrorInvalidValue;
   ++g_kernel_launches;
   return launch_k(kern, dim3(ngrp * nkc), dim3(DM_THREADS), smem, s, X, B, K, W, N, nkc, kcl, bias, resid, mode, out,
-                  out2, outf, ws, cnt, nbuf, err);
+                  out2, outf, ws, cnt, nbuf, err, lng, lnb, eps);
 }
 
 template cudaError_t launch_dec_mma<bf16>(const bf16*, int, int, const bf16*, int, const float*, const bf16*, int,
                                           bf16*, bf16*, float*, float*, size_t, unsigned*, int, unsigned*,
-                                          cudaStream_t);
+                                          cudaStream_t, const float*, const float*, float);
 template cudaError_t launch_dec_mma<f16>(const f16*, int, int, const f16*, int, const float*, const f16*, int, f16*,
-                                         f16*, float*, float*, size_t, unsigned*, int, unsigned*, cudaStream_t);
+                                         f16*, float*, float*, size_t, unsigned*, int, unsigned*, cudaStream_t,
+                                         const float*, const float*, float);

@@ -61,6 +61,7 @@ struct gpt_model {
   float *dlogits, *dmu, *drs, *dpart;
   float* dmws = nullptr;        // decode projections: partial tiles of a split k range
   unsigned* dmcnt = nullptr;    // and their per-slice arrival counters (kept zero)
+  unsigned* dacnt = nullptr;    // decode attention: per-(row, head) arrival counters (kept zero)
   size_t dmws_n = 0;
   int dmcnt_n = 0;
   float* dam;      // fused decode: per-CTA argmax partials [Bmax][DF_MAX_GRID] values, then indices
@@ -376,6 +377,7 @@ static int build_arena(gpt_model* m) {
   m->dmcnt_n = (int)((std::max<long>(std::max<long>(3 * C, m->UW), std::max<long>(F, m->Vp)) + 15) / 16);
   cv.add((void**)&m->dmws, m->dmws_n * 4);
   cv.add((void**)&m->dmcnt, (size_t)m->dmcnt_n * 4);
+  cv.add((void**)&m->dacnt, Bx * m->H * 4);
   cv.add((void**)&m->dam, Bx * DF_MAX_GRID * 8);   // fused decode: per-CTA argmax partials
   cv.add((void**)&m->dsrc, Bx * (size_t)m->Tmax * 4);
   cv.add((void**)&m->dbcs, Bx * BEAM_MAX_WIDTH * 4);
@@ -391,6 +393,7 @@ static int build_arena(gpt_model* m) {
   }
   for (auto& it : cv.items) *it.first = m->arena + it.second;
   e = cudaMemset(m->dmcnt, 0, (size_t)m->dmcnt_n * 4);
+  if (e == cudaSuccess) e = cudaMemset(m->dacnt, 0, Bx * m->H * 4);
   if (e != cudaSuccess) { m->err = std::string("cudaMemset: ") + cudaGetErrorString(e); return GPT_ERR_CUDA; }
   if (!m->lp) m->pw = m->p32;
   return GPT_OK;
@@ -901,18 +904,36 @@ static int backward_llama(gpt_model* m) {
 // Greedy decoding
 // ---------------------------------------------------------------------------
 // One projection of a decode step: y = x W^T with the gemv epilogue `mode`
-// (0: + bias + residual, 1: u = + bias and gelu(u), 2: fp32 logits).  Up to 8
-// rows run on the GEMV that streams each weight row once; 9-32 rows (16-bit)
-// on the mma.sync kernel that spreads 16-row weight slices over every SM.
+// (0: + bias + residual, 1: u = + bias and gelu(u), 2: fp32 logits).  Up to
+// 32 rows of a 16-bit model run on the mma.sync kernel that spreads 16-row
+// weight slices over every SM; fp32 models on the GEMV that streams each
+// weight row once.
 template <typename T>
 static cudaError_t dec_proj(gpt_model* m, const T* X, int B, int K, const T* W, int N, const float* bias,
                             const T* resid, int mode, T* out, T* out2, float* outf, cudaStream_t s) {
   if constexpr (sizeof(T) == 2) {
-    if (B > 8 && dec_mma_supported(B, K, N))
+    if (dec_mma_supported(B, K, N))
       return launch_dec_mma<T>(X, B, K, W, N, bias, resid, mode, out, out2, outf, m->dmws, m->dmws_n, m->dmcnt,
                                m->dmcnt_n, &m->sc->err, s);
   }
   return launch_gemv<T>(X, B, K, W, N, bias, resid, mode, out, out2, outf, s);
+}
+// LayerNorm of the residual rows x (gains g, shift b; Llama: RMSNorm, b
+// null) followed by a projection of the normalised rows: one kernel where the
+// mma.sync projection can normalise its own input, else the LayerNorm kernel
+// into h and the projection.
+template <typename T>
+static cudaError_t dec_ln_proj(gpt_model* m, const T* x, const float* g, const float* b, T* h, int B, int K,
+                               const T* W, int N, const float* bias, const T* resid, int mode, T* out, T* out2,
+                               float* outf, cudaStream_t s) {
+  if constexpr (sizeof(T) == 2) {
+    if (dec_mma_supported(B, K, N, true))
+      return launch_dec_mma<T>(x, B, K, W, N, bias, resid, mode, out, out2, outf, m->dmws, m->dmws_n, m->dmcnt,
+                               m->dmcnt_n, &m->sc->err, s, g, b, m->cfg.ln_eps);
+  }
+  cudaError_t e = launch_ln_fwd<T>(x, g, b, h, m->dmu, m->drs, B, K, m->cfg.ln_eps, s);
+  if (e != cudaSuccess) return e;
+  return dec_proj<T>(m, h, B, K, W, N, bias, resid, mode, out, out2, outf, s);
 }
 
 // The Llama-style kernels exist for the 16-bit types only (the block needs
@@ -943,7 +964,6 @@ template <typename T>
 static int decode_step(gpt_model* m, int B, int Tp, int n_new, int32_t* out, cudaStream_t s) {
   Acts<T> A(m);
   const int C = m->C, F = m->F, H = m->H, d = m->d, QW = m->QW;
-  const float eps = m->cfg.ln_eps;
   const bool ll = m->llama;
   const DecLayout DL = dec_layout(m);
   size_t kvl = (size_t)m->Bmax * m->Hkv * m->Tmax * d;
@@ -959,22 +979,24 @@ static int decode_step(gpt_model* m, int B, int Tp, int n_new, int32_t* out, cud
                          &m->sc->err, s));
   for (int l = 0; l < m->NL; ++l) {
     const LayerOff& lo = m->L[l];
-    CK(launch_ln_fwd<T>(x, A.P(lo.ln1_g), P0(lo.ln1_b), h, m->dmu, m->drs, B, C, eps, s));
-    CK(dec_proj<T>(m, h, B, C, A.W(lo.w_qkv), QW, P0(lo.b_qkv), nullptr, 0, q, nullptr, nullptr, s));
+    CK(dec_ln_proj<T>(m, x, A.P(lo.ln1_g), P0(lo.ln1_b), h, B, C, A.W(lo.w_qkv), QW, P0(lo.b_qkv), nullptr, 0, q,
+                      nullptr, nullptr, s));
     if (ll) CK(rope16<T>(q, QW, B, H, C, m->Hkv, d, nullptr, Tp - 1, stepc, m->rope_tab, m->Tmax, false, s));
-    CK(launch_dec_attn<T>(q, kc + l * kvl, vc + l * kvl, att, m->dpart, B, H, d, m->Tmax, Tp - 1, stepc, DL, s));
+    CK(launch_dec_attn<T>(q, kc + l * kvl, vc + l * kvl, att, m->dpart, m->dacnt, B, H, d, m->Tmax, Tp - 1, stepc, DL,
+                          s));
     CK(dec_proj<T>(m, att, B, C, A.W(lo.w_o), C, P0(lo.b_o), x, 0, x, nullptr, nullptr, s));
-    CK(launch_ln_fwd<T>(x, A.P(lo.ln2_g), P0(lo.ln2_b), h, m->dmu, m->drs, B, C, eps, s));
     if (ll) {
-      CK(dec_proj<T>(m, h, B, C, A.W(lo.w_fc), 2 * F, nullptr, nullptr, 0, u, nullptr, nullptr, s));
+      CK(dec_ln_proj<T>(m, x, A.P(lo.ln2_g), nullptr, h, B, C, A.W(lo.w_fc), 2 * F, nullptr, nullptr, 0, u, nullptr,
+                        nullptr, s));
       CK(swiglu16<T>(u, a, B, F, s));
     } else {
-      CK(dec_proj<T>(m, h, B, C, A.W(lo.w_fc), F, A.P(lo.b_fc), nullptr, 1, u, a, nullptr, s));
+      CK(dec_ln_proj<T>(m, x, A.P(lo.ln2_g), A.P(lo.ln2_b), h, B, C, A.W(lo.w_fc), F, A.P(lo.b_fc), nullptr, 1, u, a,
+                        nullptr, s));
     }
     CK(dec_proj<T>(m, a, B, F, A.W(lo.w_fc2), C, P0(lo.b_fc2), x, 0, x, nullptr, nullptr, s));
   }
-  CK(launch_ln_fwd<T>(x, A.P(m->o_lnf_g), P0(m->o_lnf_b), xf, m->dmu, m->drs, B, C, eps, s));
-  CK(dec_proj<T>(m, xf, B, C, A.W(m->o_head), m->Vp, nullptr, nullptr, 2, nullptr, nullptr, m->dlogits, s));
+  CK(dec_ln_proj<T>(m, x, A.P(m->o_lnf_g), P0(m->o_lnf_b), xf, B, C, A.W(m->o_head), m->Vp, nullptr, nullptr, 2,
+                    nullptr, nullptr, m->dlogits, s));
   if (m->beam_w) {
     const int W = m->beam_w;
     CK(launch_beam_topk(m->dlogits, m->Vp, m->V, B / W, W, false, m->beam_scores, m->dbcs, m->dbct, s));

@@ -180,8 +180,10 @@ cudaError_t launch_kv_fill(const T* qkv, T* kc, T* vc, int B, int Tp, int d, int
                            cudaStream_t s);
 size_t dec_attn_part_floats(int B, int H, int d);
 template <typename T>
-cudaError_t launch_dec_attn(const T* qkv, T* kc, T* vc, T* out, float* part, int B, int H, int d, int Tmax, int pos0,
-                            const int* step, const DecLayout& L, cudaStream_t s);
+// part: dec_attn_part_floats floats; cnt: B * H counters, zero before the
+// first launch (every launch leaves them zero)
+cudaError_t launch_dec_attn(const T* qkv, T* kc, T* vc, T* out, float* part, unsigned* cnt, int B, int H, int d,
+                            int Tmax, int pos0, const int* step, const DecLayout& L, cudaStream_t s);
 // out[b * out_ld + (*step or 0)] = argmax; tok[b] = argmax
 cudaError_t launch_argmax(const float* logits, int B, int V, int Vp, int* tok, int32_t* out, int out_ld,
                           const int* step, cudaStream_t s);
@@ -201,13 +203,15 @@ cudaError_t launch_gather_last(const T* x, int B, int Tp, int C, T* out, cudaStr
 // GELU into out / out2, 2: fp32 logits).  X and W 16-byte aligned.  ws
 // (ws_floats floats) holds the partial tiles of a split k range and cnt
 // (cnt_n counters, zero before the first launch; every launch leaves them
-// zero) the per-slice arrivals; with too small a workspace the k range is not
-// split.
-bool dec_mma_supported(int B, int K, int N);
+// zero) the per-slice arrivals, needed when K > 768.  With lng the kernel
+// first applies LayerNorm (lnb: shift; none: RMSNorm) with eps to the rows
+// of X, which then hold the raw residual (K <= 768).
+bool dec_mma_supported(int B, int K, int N, bool ln = false);
 template <typename T>
 cudaError_t launch_dec_mma(const T* X, int B, int K, const T* W, int N, const float* bias, const T* resid, int mode,
                            T* out, T* out2, float* outf, float* ws, size_t ws_floats, unsigned* cnt, int cnt_n,
-                           unsigned* err, cudaStream_t s);
+                           unsigned* err, cudaStream_t s, const float* lng = nullptr, const float* lnb = nullptr,
+                           float eps = 0.f);
 
 // ---- beam.cu: beam search over the decode rows (row r = b * W + w)
 #define BEAM_MAX_WIDTH 8
