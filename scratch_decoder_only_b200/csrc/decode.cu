@@ -221,7 +221,7 @@ cudaError_t launch_kv_fill(const T* qkv, T* kc, T* vc, int B, int Tp, int d, int
 // KV cache; "Feste", scaled dot-product attention with the causal mask):
 // o = softmax(q K^T / sqrt(D)) V over keys 0 .. pos of the (row, head).
 // Grid (B*H, S): the key range of a (row, head) is cut into act <= S
-// contiguous pieces (act grows with the context, one per 64 keys), one CTA
+// contiguous pieces (act grows with the context, one per 256 keys), one CTA
 // each; S is chosen so that about two CTAs per SM have work.  A CTA's four
 // warps take 4 * (32 / (D / 8)) * U consecutive keys per pass (128 for D = 64
 // in 16 bits), a lane group of D / 8 lanes per key and U keys per lane group
@@ -232,7 +232,8 @@ cudaError_t launch_kv_fill(const T* qkv, T* kc, T* vc, int B, int Tp, int d, int
 // its partial (m, l, o[D]) goes to part and the last CTA of the (row, head)
 // (an arrival counter that it resets) merges the act partials in key order.
 // The new key / value of this step come from qkv and are written to the
-// cache by piece 0.
+// cache by piece 0; the first pass's cached rows load before the
+// programmatic-dependent-launch wait, while the q / k / v projection runs.
 #define DA_SPLITS 16
 #define DA_THREADS 128
 template <typename T>
@@ -240,7 +241,7 @@ __device__ __forceinline__ void load8(const T* p, float* v) {
 #pragma unroll
   for (int i = 0; i < 8; i += Vec<T>::N) Vec<T>::load(p + i, v + i);
 }
-__device__ __forceinline__ int dec_attn_act(int pos, int S) { return min(S, (pos + 64) / 64); }
+__device__ __forceinline__ int dec_attn_act(int pos, int S) { return min(S, (pos + 256) / 256); }
 // 8 values of T kept packed in registers
 template <typename T>
 struct Pack8 {
@@ -262,8 +263,6 @@ template <typename T, int D>
 __global__ void __launch_bounds__(DA_THREADS)
 dec_attn_kernel(const T* __restrict__ qkv, T* kc, T* vc, T* __restrict__ out, float* part, unsigned* cnt, int B,
                 int H, int Tmax, int pos0, const int* __restrict__ step, DecLayout Ly) {
-  griddep_wait();
-  griddep_release();
   static_assert(D % 8 == 0 && D <= 256, "head size");
   constexpr int LPK = D / 8;            // lanes per key row (16 bytes each)
   constexpr int KPW = 32 / LPK;         // lane groups (keys) per warp
@@ -285,6 +284,34 @@ dec_attn_kernel(const T* __restrict__ qkv, T* kc, T* vc, T* __restrict__ out, fl
   const T* vnew = qkv + (long)b * Ly.qw + Ly.vcol + hk * D;
   T* kcb = kc + ((long)b * Ly.Hkv + hk) * Tmax * D;
   T* vcb = vc + ((long)b * Ly.Hkv + hk) * Tmax * D;
+  // this piece's keys [j_lo, j_hi); this warp's first pass starts at jb0
+  const int per = (pos + act) / act;   // ceil((pos + 1) / act)
+  const int j_lo = sp * per, j_hi = min(pos + 1, j_lo + per);
+  const int jb0 = j_lo + warp * KPW * U;
+  // The step counter, the beam source table and the cached keys before pos
+  // come from earlier steps: the first pass's cached rows load before the
+  // wait, while the q / k / v projection still runs.
+  auto load_kv = [&](int jb, Pack8<T>* kp, Pack8<T>* vp, bool cached, bool fresh) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = jb + u * KPW + grp;
+      const bool take = j < j_hi && ((j < pos && cached) || (j == pos && fresh));
+      if (take) {
+        long row = (long)j * D;
+        if (Ly.src && j < pos) row += ((long)Ly.src[(long)b * Tmax + j] - b) * Ly.Hkv * Tmax * D;
+        kp[u] = ld_pack8((j == pos ? knew : kcb + row) + sub * 8);
+        vp[u] = ld_pack8((j == pos ? vnew : vcb + row) + sub * 8);
+      } else if (cached) {
+#pragma unroll
+        for (int i = 0; i < (int)(sizeof(T) / 2); ++i) { kp[u].w[i] = make_uint4(0u, 0u, 0u, 0u); vp[u].w[i] = kp[u].w[i]; }
+      }
+    }
+  };
+  Pack8<T> kp[U], vp[U];
+  load_kv(jb0, kp, vp, true, false);
+  // q, k, v of this step belong to the previous kernel until here
+  griddep_wait();
+  griddep_release();
   if (sp == 0 && h % G == 0 && threadIdx.x < D) {
     kcb[(long)pos * D + threadIdx.x] = knew[threadIdx.x];
     vcb[(long)pos * D + threadIdx.x] = vnew[threadIdx.x];
@@ -297,26 +324,9 @@ dec_attn_kernel(const T* __restrict__ qkv, T* kc, T* vc, T* __restrict__ out, fl
   float m = -INFINITY, l = 0.f, o[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) o[i] = 0.f;
-  // this piece's keys [j_lo, j_hi)
-  const int per = (pos + act) / act;   // ceil((pos + 1) / act)
-  const int j_lo = sp * per, j_hi = min(pos + 1, j_lo + per);
-  for (int jb = j_lo + warp * KPW * U; jb < j_hi; jb += KPP) {
-    Pack8<T> kp[U], vp[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int j = jb + u * KPW + grp;
-      if (j < j_hi) {
-        long row = (long)j * D;
-        if (Ly.src && j < pos) row += ((long)Ly.src[(long)b * Tmax + j] - b) * Ly.Hkv * Tmax * D;
-        const T* kr = j == pos ? knew : kcb + row;
-        const T* vr = j == pos ? vnew : vcb + row;
-        kp[u] = ld_pack8(kr + sub * 8);
-        vp[u] = ld_pack8(vr + sub * 8);
-      } else {
-#pragma unroll
-        for (int i = 0; i < (int)(sizeof(T) / 2); ++i) { kp[u].w[i] = make_uint4(0u, 0u, 0u, 0u); vp[u].w[i] = kp[u].w[i]; }
-      }
-    }
+  for (int jb = jb0; jb < j_hi; jb += KPP) {
+    if (jb == jb0) load_kv(jb, kp, vp, false, true);   // the new key of this step
+    else load_kv(jb, kp, vp, true, true);
     float sc[U];
     float mn = m;
 #pragma unroll

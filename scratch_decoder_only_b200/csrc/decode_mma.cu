@@ -104,6 +104,7 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
   constexpr bool F16 = std::is_same<T, f16>::value;
   extern __shared__ __align__(128) uint8_t dm_smem[];
   __shared__ __align__(8) uint64_t bars[DM_MAXBUF];
+  __shared__ __align__(8) uint64_t lnbar;
   __shared__ int s_abort, s_last;
   const int kc = blockIdx.x % nkc, grp = blockIdx.x / nkc, ngrp = gridDim.x / nkc;
   const int k0 = kc * kcl, kn = min(kcl, K - k0);   // this CTA's columns [k0, k0 + kn), kn % 32 == 0
@@ -116,6 +117,7 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
   float* red = reinterpret_cast<float*>(dm_smem + nbuf * slot_bytes);
   if (threadIdx.x == 0) {
     for (int i = 0; i < nbuf; ++i) mbar_init(smem_u32(&bars[i]), 1);
+    mbar_init(smem_u32(&lnbar), 1);
     s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -140,13 +142,30 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
   int issued = 0;
   if (threadIdx.x == 0)
     for (; issued < nbuf && issued < nmine; ++issued) issue(issued);
-  // the LayerNorm parameters (constant) can move before the wait
+  // the LayerNorm parameters (constant) move before the wait: by bulk copy
+  // when 16-byte aligned (waited for after the statistics), else by loads
   float* lns = red + DM_WARPS * 16 * MT * 16;
-  if (lng)
+  const bool ln_bulk = lng && !((reinterpret_cast<uintptr_t>(lng) | reinterpret_cast<uintptr_t>(lnb)) & 15);
+  if (ln_bulk) {
+    if (threadIdx.x == 0) {
+      const uint32_t bar = smem_u32(&lnbar);
+      mbar_expect_tx(bar, (uint32_t)K * 4 * (lnb ? 2 : 1));
+      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                   ::"r"(smem_u32(lns)), "l"(reinterpret_cast<uint64_t>(lng)), "r"((uint32_t)K * 4), "r"(bar)
+                   : "memory");
+      if (lnb)
+        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                     ::"r"(smem_u32(lns + K)), "l"(reinterpret_cast<uint64_t>(lnb)), "r"((uint32_t)K * 4), "r"(bar)
+                     : "memory");
+    }
+    if (!lnb)
+      for (int i = threadIdx.x; i < K; i += DM_THREADS) lns[K + i] = 0.f;
+  } else if (lng) {
     for (int i = threadIdx.x; i < K; i += DM_THREADS) {
       lns[i] = lng[i];
       lns[K + i] = lnb ? lnb[i] : 0.f;
     }
+  }
   // x, the residual, the outputs and the workspace belong to the previous kernel until here
   griddep_wait();
   griddep_release();
@@ -165,6 +184,7 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
                                            : make_uint4(0u, 0u, 0u, 0u);
       }
   }
+  bool lnwait = false;   // a timed-out wait for the LayerNorm parameters
   if (lng) {
     // x <- LayerNorm(x) (RMSNorm without lnb), nkc == 1: columns [0, K).
     // Statistics with one barrier: each lane takes the mean and the sum of
@@ -237,8 +257,9 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
         }
         mu[bt][h] = m;
         // RMSNorm: q is the sum of squares (every mean stayed 0)
-        rs[bt][h] = 1.0f / sqrtf(q / K + eps);
+        rs[bt][h] = 1.0f / sqrtf(q * inK + eps);
       }
+    if (ln_bulk) lnwait = !mbar_wait(smem_u32(&lnbar), 0, &s_abort);
 #pragma unroll
     for (int j = 0; j < DM_KB; ++j) {
       const int col = 32 * (warp + DM_WARPS * j) + 8 * tig;
@@ -268,7 +289,7 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
   // A timed-out wait is voted block-wide; the CTA then runs its remaining
   // slices without data so that every slice counter still receives its nkc
   // arrivals (and returns to zero), and drains its copies before leaving.
-  bool dead = false;
+  bool dead = __syncthreads_or(lnwait);
   int landed = 0;   // slices whose copies completed
   for (int j = 0; j < nmine; ++j) {
     const int s = grp + j * ngrp, r0 = s * DM_ROWS;
@@ -362,6 +383,7 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
     set_dev_err(err, GPT_DEVERR_TIMEOUT);
     // let the copies still in flight land before leaving
     volatile int never = 0;
+    if (ln_bulk) mbar_wait(smem_u32(&lnbar), 0, &never, 1ll << 28);
     for (int q = landed; q < issued; ++q) mbar_wait(smem_u32(&bars[q % nbuf]), (q / nbuf) & 1, &never, 1ll << 28);
   }
 }

@@ -64,7 +64,6 @@ struct gpt_model {
   unsigned* dacnt = nullptr;    // decode attention: per-(row, head) arrival counters (kept zero)
   size_t dmws_n = 0;
   int dmcnt_n = 0;
-  float* dam;      // fused decode: per-CTA argmax partials [Bmax][DF_MAX_GRID] values, then indices
   int* dtok;
   int fwd_B = 0, fwd_T = 0;
   bool have_targets = false, logits_valid = false;
@@ -378,7 +377,6 @@ static int build_arena(gpt_model* m) {
   cv.add((void**)&m->dmws, m->dmws_n * 4);
   cv.add((void**)&m->dmcnt, (size_t)m->dmcnt_n * 4);
   cv.add((void**)&m->dacnt, Bx * m->H * 4);
-  cv.add((void**)&m->dam, Bx * DF_MAX_GRID * 8);   // fused decode: per-CTA argmax partials
   cv.add((void**)&m->dsrc, Bx * (size_t)m->Tmax * 4);
   cv.add((void**)&m->dbcs, Bx * BEAM_MAX_WIDTH * 4);
   cv.add((void**)&m->dbct, Bx * BEAM_MAX_WIDTH * 4);
@@ -1040,31 +1038,6 @@ static int decode_impl(gpt_model* m, const int32_t* prompt, int B, int Tp, int n
     CK(launch_argmax(m->dlogits, B, m->V, m->Vp, m->dtok, out, n_new, nullptr, s));
   if (n_new == 1) return GPT_OK;
   const int Bd = m->beam_w ? B * m->beam_w : B;   // decode rows
-  if constexpr (sizeof(T) == 2) {
-    if (!m->smp_on && !m->beam_w && !m->fp16 && !m->llama && dec_fused_supported(B, C, H, m->F, m->Vp)) {
-      // every later token from one persistent kernel
-      const LayerOff& l0 = m->L[0];
-      DecFusedParams q;
-      memset(&q, 0, sizeof(q));
-      q.pw = (const bf16*)m->pw; q.p32 = m->p32;
-      q.o_wte = m->o_wte; q.o_wpe = m->o_wpe; q.o_lnf_g = m->o_lnf_g; q.o_lnf_b = m->o_lnf_b; q.o_head = m->o_head;
-      q.l_ln1_g = l0.ln1_g; q.l_ln1_b = l0.ln1_b; q.l_w_qkv = l0.w_qkv; q.l_b_qkv = l0.b_qkv; q.l_w_o = l0.w_o;
-      q.l_b_o = l0.b_o; q.l_ln2_g = l0.ln2_g; q.l_ln2_b = l0.ln2_b; q.l_w_fc = l0.w_fc; q.l_b_fc = l0.b_fc;
-      q.l_w_fc2 = l0.w_fc2; q.l_b_fc2 = l0.b_fc2;
-      q.l_stride = m->NL > 1 ? (long)(m->L[1].ln1_g - l0.ln1_g) : (long)(m->o_lnf_g - l0.ln1_g);
-      q.NL = m->NL; q.C = C; q.H = H; q.D = d; q.F = m->F; q.V = m->V; q.Vp = m->Vp; q.Tmax = m->Tmax;
-      q.eps = m->cfg.ln_eps;
-      q.kc = (bf16*)m->kc; q.vc = (bf16*)m->vc; q.kvl = (long)kvl;
-      q.B = B; q.pos_first = Tp; q.n_steps = n_new - 1;
-      q.tok = m->dtok; q.out = out; q.out_ld = n_new; q.out_col0 = 1;
-      q.qkv = (bf16*)m->dq; q.part = m->dpart; q.xmid = (bf16*)m->dh; q.abuf = (bf16*)m->da; q.xbuf = (bf16*)m->dx;
-      q.logits = m->dlogits; q.am_v = m->dam; q.am_i = (int*)(m->dam + (size_t)m->Bmax * DF_MAX_GRID);
-      q.bar = &m->sc->dec_bar; q.abortf = &m->sc->dec_abort; q.err = &m->sc->err;
-      CK(cudaMemsetAsync(&m->sc->dec_bar, 0, 2 * sizeof(unsigned), s));
-      CK(launch_decode_fused(q, s));
-      return GPT_OK;
-    }
-  }
   const int one = 1;
   CK(cudaMemcpyAsync(&m->sc->dec_step, &one, sizeof(int), cudaMemcpyHostToDevice, s));
   // later tokens: one captured step (about 7 L + 5 kernels), replayed n_new - 1 times

@@ -25,8 +25,6 @@ struct DevScalars {
   int loss_scaling;   // 1: dynamic scale on
   unsigned err;       // sticky device error word
   int dec_step;       // decode step counter
-  unsigned dec_bar;   // grid-barrier counter of the fused decode kernel (zeroed per launch)
-  unsigned dec_abort; // its abort word (zeroed per launch)
   unsigned long long attn_pairs;   // allowed (query, key) pairs of the latest packed forward
   float lr;           // learning rate of the latest taken step (set by the finalize kernel)
   float loss_weight;  // multiplies the loss gradient of later forwards (micro-batch weight)
@@ -251,36 +249,3 @@ template <typename T>
 cudaError_t launch_gqa_reduce(const T* kvq, T* dkv, long ld, int kcol, int vcol, int rows, int Hkv, int G, int d,
                               cudaStream_t s);
 
-// ---- decode_fused.cu: every remaining greedy step of a small batch in one
-// persistent kernel (bf16 weights; B <= 4)
-#define DF_MAX_GRID 256   // am_v / am_i hold [B][DF_MAX_GRID]
-struct DecFusedParams {
-  const bf16* pw;          // bf16 working copy of the parameters
-  const float* p32;        // fp32 master parameters (embeddings, LN, biases)
-  long o_wte, o_wpe, o_lnf_g, o_lnf_b, o_head;
-  // offsets of layer 0 and the stride between layers (canonical layout)
-  long l_ln1_g, l_ln1_b, l_w_qkv, l_b_qkv, l_w_o, l_b_o, l_ln2_g, l_ln2_b, l_w_fc, l_b_fc, l_w_fc2, l_b_fc2;
-  long l_stride;
-  int NL, C, H, D, F, V, Vp, Tmax;
-  float eps;
-  bf16* kc;                // [NL][Bmax][H][Tmax][D]
-  bf16* vc;
-  long kvl;                // elements per layer of the cache
-  int B, pos_first, n_steps, S;
-  int* tok;                // [B] current token (in: the prefill's choice)
-  int32_t* out;            // [B][out_ld], columns out_col0 .. out_col0 + n_steps - 1
-  int out_ld, out_col0;
-  bf16* qkv;               // [B][3C]
-  float* part;             // [B*H][S][D+2] attention partials
-  bf16* xmid;              // [B][C]
-  bf16* abuf;              // [B][F]
-  bf16* xbuf;              // [B][C]
-  float* logits;           // [B][Vp]
-  float* am_v;             // [B][grid] per-CTA maxima
-  int* am_i;
-  unsigned* bar;           // grid barrier counter (zero at launch)
-  unsigned* abortf;        // abort word (zero at launch)
-  unsigned* err;           // sticky device error word
-};
-bool dec_fused_supported(int B, int C, int H, int F, int Vp);
-cudaError_t launch_decode_fused(const DecFusedParams& prm, cudaStream_t s);
