@@ -28,10 +28,11 @@
 // (two passes, quad shuffles and a fixed-order sum over the warps) and the
 // normalised values, rounded to 16 bits as the LayerNorm kernel stores them,
 // replace the fragments.
-// With a split k range each CTA writes its partial tile to a workspace and
-// the last of the slice's nkc CTAs (a per-slice arrival counter, reset by
-// that CTA) adds the nkc partials in k order and runs the epilogue: results
-// do not depend on which CTA finishes last.  Weight copies are issued before
+// With a split k range the nkc CTAs of a slice group form a thread-block
+// cluster: each stores its partial tile into the first CTA's shared memory
+// (distributed shared memory), one cluster barrier per slice, and the first
+// CTA adds the nkc partials in k order and runs the epilogue (two partial
+// areas alternate, so the next slice's stores never meet this one's reads).  Weight copies are issued before
 // the programmatic-dependent-launch wait: the stream starts while the
 // previous kernel drains.
 #include "launch.h"
@@ -44,7 +45,7 @@
 #define DM_KB (DM_KC / 32 / DM_WARPS)   // 32-column blocks per warp (at most)
 #define DM_MAXBUF 6                // slice slots (at most)
 #define DM_SMEM_BUDGET (110 * 1024)     // two CTAs per SM
-#define DM_MAX_SPLIT 16
+#define DM_MAX_SPLIT 8              // cluster size (portable limit)
 #ifndef DM_CTAS
 #define DM_CTAS 2                  // CTAs per SM in the grid
 #endif
@@ -90,22 +91,33 @@ __device__ __forceinline__ void dm_epilogue(float y, float pb, float pr, int bb,
 }
 #define DM_OPT (16 * 32 / DM_THREADS)   // outputs per thread and slice (at most)
 
+__device__ __forceinline__ void dm_cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Store v at this CTA's shared address addr mapped into cluster CTA rank.
+__device__ __forceinline__ void dm_st_cluster(uint32_t addr, uint32_t rank, float v) {
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(addr), "r"(rank));
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
+}
+
 // MT = 16-row tiles of x (B <= 16 MT).  Grid = ngrp groups x nkc k ranges;
 // CTA (grp, kc) takes columns [kc kcl, min(K, (kc + 1) kcl)) of every slice
-// grp + j ngrp.  Shared memory: nbuf slots of [16 rows][kcl] 16-bit values,
-// the warps' partial tiles [DM_WARPS][16 MT][16] fp32, then (LayerNorm) its
-// gains and shifts [2][K] fp32.
+// grp + j ngrp; with nkc > 1 the CTAs of a group form one cluster (rank kc).
+// Shared memory: nbuf slots of [16 rows][kcl] 16-bit values, the warps'
+// partial tiles [DM_WARPS][16 MT][16] fp32, then the LayerNorm's gains and
+// shifts [2][K] fp32 (nkc == 1) or the cluster's partial areas [2][nkc][B
+// 16] fp32 (nkc > 1).
 template <typename T, int MT>
 __global__ void __launch_bounds__(DM_THREADS, 2)
 dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, int N, int nkc, int kcl,
-               const float* __restrict__ bias, const T* resid, int mode, T* out, T* out2, float* outf, float* ws,
-               unsigned* cnt, int nbuf, unsigned* err, const float* __restrict__ lng, const float* __restrict__ lnb,
-               float eps) {
+               const float* __restrict__ bias, const T* resid, int mode, T* out, T* out2, float* outf, int nbuf,
+               unsigned* err, const float* __restrict__ lng, const float* __restrict__ lnb, float eps) {
   constexpr bool F16 = std::is_same<T, f16>::value;
   extern __shared__ __align__(128) uint8_t dm_smem[];
   __shared__ __align__(8) uint64_t bars[DM_MAXBUF];
   __shared__ __align__(8) uint64_t lnbar;
-  __shared__ int s_abort, s_last;
+  __shared__ int s_abort;
   const int kc = blockIdx.x % nkc, grp = blockIdx.x / nkc, ngrp = gridDim.x / nkc;
   const int k0 = kc * kcl, kn = min(kcl, K - k0);   // this CTA's columns [k0, k0 + kn), kn % 32 == 0
   const int nslices = (N + DM_ROWS - 1) / DM_ROWS;
@@ -145,6 +157,9 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
   // the LayerNorm parameters (constant) move before the wait: by bulk copy
   // when 16-byte aligned (waited for after the statistics), else by loads
   float* lns = red + DM_WARPS * 16 * MT * 16;
+  float* cred = lns;   // nkc > 1: [2][nkc][B 16] partial areas of the cluster's first CTA
+  // every CTA of the cluster has started before any partial crosses to rank 0
+  if (nkc > 1) dm_cluster_sync();
   const bool ln_bulk = lng && !((reinterpret_cast<uintptr_t>(lng) | reinterpret_cast<uintptr_t>(lnb)) & 15);
   if (ln_bulk) {
     if (threadIdx.x == 0) {
@@ -355,30 +370,25 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
 #pragma unroll
       for (int w = 0; w < DM_WARPS; ++w) y += red[((w * 16 * MT) + bb) * 16 + nn];
       if (nkc == 1) dm_epilogue<T>(y, pb[t], pr[t], bb, n, N, mode, out, out2, outf);
-      else ws[((long)kc * B + bb) * N + n] = y;
+      else dm_st_cluster(smem_u32(cred + ((j & 1) * nkc + kc) * (B * DM_ROWS) + o), 0u, y);
     }
     if (nkc > 1) {
-      __threadfence();
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        const unsigned prev = atomicAdd(&cnt[s], 1u);
-        s_last = prev == (unsigned)(nkc - 1);
-        if (s_last) atomicExch(&cnt[s], 0u);   // ready for the next launch
-      }
-      __syncthreads();
-      if (s_last) {
-        __threadfence();
+      // every CTA arrives here once per slice, a timed-out one included
+      dm_cluster_sync();
+      if (kc == 0) {
 #pragma unroll
         for (int t = 0; t < DM_OPT; ++t) {
           const int o = threadIdx.x + DM_THREADS * t, bb = o / DM_ROWS, n = r0 + o % DM_ROWS;
           if (o >= B * DM_ROWS || n >= N) continue;
           float y = 0.f;
-          for (int q = 0; q < nkc; ++q) y += __ldcg(&ws[((long)q * B + bb) * N + n]);
+          for (int q = 0; q < nkc; ++q) y += cred[((j & 1) * nkc + q) * (B * DM_ROWS) + o];
           dm_epilogue<T>(y, pb[t], pr[t], bb, n, N, mode, out, out2, outf);
         }
       }
     }
   }
+  // no CTA leaves while another may still store into its shared memory
+  if (nkc > 1) dm_cluster_sync();
   if (dead && threadIdx.x == 0) {
     set_dev_err(err, GPT_DEVERR_TIMEOUT);
     // let the copies still in flight land before leaving
@@ -396,8 +406,8 @@ bool dec_mma_supported(int B, int K, int N, bool ln) {
 
 template <typename T>
 cudaError_t launch_dec_mma(const T* X, int B, int K, const T* W, int N, const float* bias, const T* resid, int mode,
-                           T* out, T* out2, float* outf, float* ws, size_t ws_floats, unsigned* cnt, int cnt_n,
-                           unsigned* err, cudaStream_t s, const float* lng, const float* lnb, float eps) {
+                           T* out, T* out2, float* outf, unsigned* err, cudaStream_t s, const float* lng,
+                           const float* lnb, float eps) {
   if (!dec_mma_supported(B, K, N, lng != nullptr)) return cudaErrorInvalidValue;
   if (((uintptr_t)X & 15) || ((uintptr_t)W & 15)) return cudaErrorInvalidValue;
   if (!g_dm_sms) {
@@ -410,17 +420,16 @@ cudaError_t launch_dec_mma(const T* X, int B, int K, const T* W, int N, const fl
   const int nslices = (N + DM_ROWS - 1) / DM_ROWS;
   // k ranges of at most DM_KC columns, multiples of 32
   const int nkc = (K + DM_KC - 1) / DM_KC, kcl = ((K + nkc - 1) / nkc + 31) / 32 * 32;
-  if ((nkc - 1) * kcl >= K) return cudaErrorInvalidValue;   // no empty last range
-  if (nkc > 1 && (!ws || !cnt || (size_t)nkc * B * N > ws_floats || cnt_n < nslices)) return cudaErrorInvalidValue;
+  if ((nkc - 1) * kcl >= K || nkc > DM_MAX_SPLIT) return cudaErrorInvalidValue;   // no empty last range
   const size_t slot = (size_t)DM_ROWS * kcl * 2;
-  const size_t red = (size_t)DM_WARPS * 16 * MT * 16 * 4 + (lng ? (size_t)2 * K * 4 : 0);
+  const size_t red = (size_t)DM_WARPS * 16 * MT * 16 * 4 + (lng ? (size_t)2 * K * 4 : 0) +
+                     (nkc > 1 ? (size_t)2 * nkc * B * DM_ROWS * 4 : 0);
   int nbuf = (int)((DM_SMEM_BUDGET - (long)red) / (long)slot);
   if (nbuf > DM_MAXBUF) nbuf = DM_MAXBUF;
   if (nbuf < 2) nbuf = 2;
   const size_t smem = nbuf * slot + red;
-  void (*kern)(const T*, int, int, const T*, int, int, int, const float*, const T*, int, T*, T*, float*, float*,
-               unsigned*, int, unsigned*, const float*, const float*, float) =
-      MT == 1 ? dec_mma_kernel<T, 1> : dec_mma_kernel<T, 2>;
+  void (*kern)(const T*, int, int, const T*, int, int, int, const float*, const T*, int, T*, T*, float*, int,
+               unsigned*, const float*, const float*, float) = MT == 1 ? dec_mma_kernel<T, 1> : dec_mma_kernel<T, 2>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
@@ -430,13 +439,30 @@ cudaError_t launch_dec_mma(const T* X, int B, int K, const T* W, int N, const fl
   const int ngrp = std::min(g_dm_sms * std::min(per_sm, DM_CTAS) / nkc, nslices);
   if (ngrp < 1) return cudaErrorInvalidValue;
   ++g_kernel_launches;
-  return launch_k(kern, dim3(ngrp * nkc), dim3(DM_THREADS), smem, s, X, B, K, W, N, nkc, kcl, bias, resid, mode, out,
-                  out2, outf, ws, cnt, nbuf, err, lng, lnb, eps);
+  if (nkc == 1)
+    return launch_k(kern, dim3(ngrp), dim3(DM_THREADS), smem, s, X, B, K, W, N, nkc, kcl, bias, resid, mode, out, out2,
+                    outf, nbuf, err, lng, lnb, eps);
+  // clusters of nkc CTAs (and the programmatic dependent launch of launch_k)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ngrp * nkc);
+  cfg.blockDim = dim3(DM_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = nkc;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = g_pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kern, X, B, K, W, N, nkc, kcl, bias, resid, mode, out, out2, outf, nbuf, err, lng,
+                            lnb, eps);
 }
 
 template cudaError_t launch_dec_mma<bf16>(const bf16*, int, int, const bf16*, int, const float*, const bf16*, int,
-                                          bf16*, bf16*, float*, float*, size_t, unsigned*, int, unsigned*,
-                                          cudaStream_t, const float*, const float*, float);
+                                          bf16*, bf16*, float*, unsigned*, cudaStream_t, const float*, const float*,
+                                          float);
 template cudaError_t launch_dec_mma<f16>(const f16*, int, int, const f16*, int, const float*, const f16*, int, f16*,
-                                         f16*, float*, float*, size_t, unsigned*, int, unsigned*, cudaStream_t,
-                                         const float*, const float*, float);
+                                         f16*, float*, unsigned*, cudaStream_t, const float*, const float*, float);

@@ -59,11 +59,7 @@ struct gpt_model {
   DevScalars* sc;
   void *kc, *vc, *dx, *dh, *dq, *datt, *du, *da, *dxf;
   float *dlogits, *dmu, *drs, *dpart;
-  float* dmws = nullptr;        // decode projections: partial tiles of a split k range
-  unsigned* dmcnt = nullptr;    // and their per-slice arrival counters (kept zero)
   unsigned* dacnt = nullptr;    // decode attention: per-(row, head) arrival counters (kept zero)
-  size_t dmws_n = 0;
-  int dmcnt_n = 0;
   int* dtok;
   int fwd_B = 0, fwd_T = 0;
   bool have_targets = false, logits_valid = false;
@@ -372,10 +368,6 @@ static int build_arena(gpt_model* m) {
   cv.add((void**)&m->drs, Bx * 4);
   cv.add((void**)&m->dtok, Bx * 4);
   cv.add((void**)&m->dpart, dec_attn_part_floats((int)Bx, m->H, m->d) * 4);
-  m->dmws_n = 16 * Bx * (size_t)std::max<long>(std::max<long>(3 * C, m->UW), F);
-  m->dmcnt_n = (int)((std::max<long>(std::max<long>(3 * C, m->UW), std::max<long>(F, m->Vp)) + 15) / 16);
-  cv.add((void**)&m->dmws, m->dmws_n * 4);
-  cv.add((void**)&m->dmcnt, (size_t)m->dmcnt_n * 4);
   cv.add((void**)&m->dacnt, Bx * m->H * 4);
   cv.add((void**)&m->dsrc, Bx * (size_t)m->Tmax * 4);
   cv.add((void**)&m->dbcs, Bx * BEAM_MAX_WIDTH * 4);
@@ -390,8 +382,7 @@ static int build_arena(gpt_model* m) {
     return GPT_ERR_NOMEM;
   }
   for (auto& it : cv.items) *it.first = m->arena + it.second;
-  e = cudaMemset(m->dmcnt, 0, (size_t)m->dmcnt_n * 4);
-  if (e == cudaSuccess) e = cudaMemset(m->dacnt, 0, Bx * m->H * 4);
+  e = cudaMemset(m->dacnt, 0, Bx * m->H * 4);
   if (e != cudaSuccess) { m->err = std::string("cudaMemset: ") + cudaGetErrorString(e); return GPT_ERR_CUDA; }
   if (!m->lp) m->pw = m->p32;
   return GPT_OK;
@@ -911,8 +902,7 @@ static cudaError_t dec_proj(gpt_model* m, const T* X, int B, int K, const T* W, 
                             const T* resid, int mode, T* out, T* out2, float* outf, cudaStream_t s) {
   if constexpr (sizeof(T) == 2) {
     if (dec_mma_supported(B, K, N))
-      return launch_dec_mma<T>(X, B, K, W, N, bias, resid, mode, out, out2, outf, m->dmws, m->dmws_n, m->dmcnt,
-                               m->dmcnt_n, &m->sc->err, s);
+      return launch_dec_mma<T>(X, B, K, W, N, bias, resid, mode, out, out2, outf, &m->sc->err, s);
   }
   return launch_gemv<T>(X, B, K, W, N, bias, resid, mode, out, out2, outf, s);
 }
@@ -926,8 +916,8 @@ static cudaError_t dec_ln_proj(gpt_model* m, const T* x, const float* g, const f
                                float* outf, cudaStream_t s) {
   if constexpr (sizeof(T) == 2) {
     if (dec_mma_supported(B, K, N, true))
-      return launch_dec_mma<T>(x, B, K, W, N, bias, resid, mode, out, out2, outf, m->dmws, m->dmws_n, m->dmcnt,
-                               m->dmcnt_n, &m->sc->err, s, g, b, m->cfg.ln_eps);
+      return launch_dec_mma<T>(x, B, K, W, N, bias, resid, mode, out, out2, outf, &m->sc->err, s, g, b,
+                               m->cfg.ln_eps);
   }
   cudaError_t e = launch_ln_fwd<T>(x, g, b, h, m->dmu, m->drs, B, K, m->cfg.ln_eps, s);
   if (e != cudaSuccess) return e;

@@ -198,18 +198,15 @@ cudaError_t launch_gather_last(const T* x, int B, int Tp, int C, T* out, cudaStr
 
 // ---- decode_mma.cu: decode projections of 1-32 rows on mma.sync (16-bit T),
 // same modes and outputs as the GEMV (0: + bias + residual, 1: + bias and
-// GELU into out / out2, 2: fp32 logits).  X and W 16-byte aligned.  ws
-// (ws_floats floats) holds the partial tiles of a split k range and cnt
-// (cnt_n counters, zero before the first launch; every launch leaves them
-// zero) the per-slice arrivals, needed when K > 768.  With lng the kernel
+// GELU into out / out2, 2: fp32 logits).  X and W 16-byte aligned; K > 768
+// runs as clusters of CTAs that split the k range.  With lng the kernel
 // first applies LayerNorm (lnb: shift; none: RMSNorm) with eps to the rows
 // of X, which then hold the raw residual (K <= 768).
 bool dec_mma_supported(int B, int K, int N, bool ln = false);
 template <typename T>
 cudaError_t launch_dec_mma(const T* X, int B, int K, const T* W, int N, const float* bias, const T* resid, int mode,
-                           T* out, T* out2, float* outf, float* ws, size_t ws_floats, unsigned* cnt, int cnt_n,
-                           unsigned* err, cudaStream_t s, const float* lng = nullptr, const float* lnb = nullptr,
-                           float eps = 0.f);
+                           T* out, T* out2, float* outf, unsigned* err, cudaStream_t s, const float* lng = nullptr,
+                           const float* lnb = nullptr, float eps = 0.f);
 
 // ---- beam.cu: beam search over the decode rows (row r = b * W + w)
 #define BEAM_MAX_WIDTH 8
