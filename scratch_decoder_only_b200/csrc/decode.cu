@@ -7,11 +7,13 @@
 #include "launch.h"
 
 // pos = pos0 + *step (the step counter lives on the device so that one
-// captured decode step can be replayed).
+// captured decode step can be replayed).  st (C % 16 == 0, or null): per
+// 16-column group g of row b, st[g B + b] = (mean, sum of squared
+// deviations) of the stored values, for the LayerNorm of the next projection.
 template <typename T>
 __global__ void dec_embed_kernel(const int* __restrict__ tok, const float* __restrict__ wte,
                                  const float* __restrict__ wpe, T* __restrict__ x, int C, int pos0,
-                                 const int* __restrict__ step, int max_seq, unsigned* err) {
+                                 const int* __restrict__ step, int max_seq, unsigned* err, float2* st) {
   griddep_wait();
   griddep_release();
   int b = blockIdx.x;
@@ -22,14 +24,36 @@ __global__ void dec_embed_kernel(const int* __restrict__ tok, const float* __res
   }
   const float* a = wte + (long)tok[b] * C;
   const float* p = wpe ? wpe + (long)pos * C : nullptr;
-  for (int c = threadIdx.x; c < C; c += blockDim.x) x[(long)b * C + c] = from_f<T>(a[c] + (p ? p[c] : 0.f));
+  // blockDim.x is a multiple of 32: a group's 16 columns sit in 16 consecutive lanes
+  for (int c0 = 0; c0 < C; c0 += blockDim.x) {
+    const int c = c0 + threadIdx.x;
+    const bool ok = c < C;
+    float v = 0.f;
+    if (ok) {
+      const T t = from_f<T>(a[c] + (p ? p[c] : 0.f));
+      x[(long)b * C + c] = t;
+      v = to_f(t);
+    }
+    if (st) {
+      float sm = v;
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
+      const float mean = sm * (1.f / 16.f), d = ok ? v - mean : 0.f;
+      float q = d * d;
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+      if (ok && (threadIdx.x & 15) == 0) st[(long)(c / 16) * gridDim.x + b] = make_float2(mean, q);
+    }
+  }
 }
 
 template <typename T>
 cudaError_t launch_dec_embed(const int* tok, const float* wte, const float* wpe, T* x, int B, int C, int pos0,
-                             const int* step, int max_seq, unsigned* err, cudaStream_t s) {
+                             const int* step, int max_seq, unsigned* err, cudaStream_t s, float2* st) {
+  if (st && C % 16) return cudaErrorInvalidValue;
   ++g_kernel_launches;
-  cudaError_t e = launch_k(dec_embed_kernel<T>, dim3(B), dim3(256), 0, s, tok, wte, wpe, x, C, pos0, step, max_seq, err);
+  cudaError_t e = launch_k(dec_embed_kernel<T>, dim3(B), dim3(256), 0, s, tok, wte, wpe, x, C, pos0, step, max_seq, err,
+                           st);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -807,7 +831,7 @@ cudaError_t launch_gather_last(const T* x, int B, int Tp, int C, T* out, cudaStr
 
 #define INSTD(T)                                                                                         \
   template cudaError_t launch_dec_embed<T>(const int*, const float*, const float*, T*, int, int, int,      \
-                                           const int*, int, unsigned*, cudaStream_t);                    \
+                                           const int*, int, unsigned*, cudaStream_t, float2*);           \
   template cudaError_t launch_gemv<T>(const T*, int, int, const T*, int, const float*, const T*, int, T*, T*, \
                                       float*, cudaStream_t);                                             \
   template cudaError_t launch_kv_fill<T>(const T*, T*, T*, int, int, int, int, const DecLayout&, cudaStream_t); \

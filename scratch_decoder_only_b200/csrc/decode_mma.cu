@@ -76,18 +76,35 @@ __device__ __forceinline__ uint4 dm_lds128(uint32_t addr) {
 // Output (bb, n) from the dot product y, the bias value pb and the residual
 // value pr (both loaded ahead, zero where absent).
 template <typename T>
-__device__ __forceinline__ void dm_epilogue(float y, float pb, float pr, int bb, int n, int N, int mode, T* out,
-                                            T* out2, float* outf) {
+__device__ __forceinline__ float dm_epilogue(float y, float pb, float pr, int bb, int n, int N, int mode, T* out,
+                                             T* out2, float* outf) {
   const long oi = (long)bb * N + n;
   if (mode == 2) {
     outf[oi] = y;
+    return y;
   } else if (mode == 1) {
     const T uq = from_f<T>(y + pb);
     out[oi] = uq;
     out2[oi] = from_f<T>(gelu_f(to_f(uq)));
-  } else {
-    out[oi] = from_f<T>(y + pb + pr);
+    return to_f(uq);
   }
+  const T v = from_f<T>(y + pb + pr);
+  out[oi] = v;
+  return to_f(v);
+}
+// LayerNorm statistics of a row's 16-column group (the slice's outputs of
+// row bb, held by 16 consecutive lanes): mean and sum of squared deviations
+// into st[slice][bb] (an LN-fused projection merges the groups).  Every lane
+// of the warp calls it; ok: this lane holds a stored value v.
+__device__ __forceinline__ void dm_group_stats(float v, bool ok, float2* st, int slice, int B, int bb, int lane) {
+  float sm = ok ? v : 0.f;
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
+  const float mean = sm * (1.f / 16.f), d = ok ? v - mean : 0.f;
+  float q = d * d;
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+  if (ok && (lane & 15) == 0) st[(long)slice * B + bb] = make_float2(mean, q);
 }
 #define DM_OPT (16 * 32 / DM_THREADS)   // outputs per thread and slice (at most)
 
@@ -112,7 +129,8 @@ template <typename T, int MT>
 __global__ void __launch_bounds__(DM_THREADS, 2)
 dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, int N, int nkc, int kcl,
                const float* __restrict__ bias, const T* resid, int mode, T* out, T* out2, float* outf, int nbuf,
-               unsigned* err, const float* __restrict__ lng, const float* __restrict__ lnb, float eps) {
+               unsigned* err, const float* __restrict__ lng, const float* __restrict__ lnb, float eps,
+               float2* st_out, const float2* __restrict__ st_in) {
   constexpr bool F16 = std::is_same<T, f16>::value;
   extern __shared__ __align__(128) uint8_t dm_smem[];
   __shared__ __align__(8) uint64_t bars[DM_MAXBUF];
@@ -209,71 +227,108 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
     // the pairwise update of Chan, Golub and LeVeque); the warps' parts merge
     // in warp order as mean = sum_w n_w mean_w / K and M2 = sum_w (M2_w +
     // n_w (mean_w - mean)^2).  RMSNorm keeps every mean 0 and sums squares.
-    float2* sred = reinterpret_cast<float2*>(red);   // [DM_WARPS][16 MT] (mean, M2) of the warp's columns
     float mu[MT][2], rs[MT][2];
-    const int nw = min(DM_KB, (kn / 32 - warp + DM_WARPS - 1) / DM_WARPS);   // this warp's blocks in range
-    const float nl = 8.f * nw;                                             // values per lane
-    const float inl = nw > 0 ? 1.f / nl : 0.f, inK = 1.f / K;
+    const float inK = 1.f / K;
+    if (st_in) {
+      // statistics from the producer's 16-column groups: thread (r, p) takes
+      // groups p, p + TPR, ... of row r; the row's TPR lanes merge by shuffles
+      // as mean = 16 sum_g mean_g / K, M2 = sum_g (M2_g + 16 (mean_g - mean)^2)
+      constexpr int R = 16 * MT, TPR = DM_THREADS / R, GPL = (DM_KC / 16 + TPR - 1) / TPR;
+      float2* srow = reinterpret_cast<float2*>(red);   // [16 MT] (mean, rstd)
+      const int r = threadIdx.x / TPR, p = threadIdx.x % TPR, NG = K / 16;
+      float2 gv[GPL];
+      float sm = 0.f;
 #pragma unroll
-    for (int bt = 0; bt < MT; ++bt)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float m = 0.f, q = 0.f;
-        if (nw > 0 && bt * 16 + h * 8 + g < B) {
-          float sum = 0.f;
-#pragma unroll
-          for (int j = 0; j < DM_KB; ++j)
-            if (j < nw) {
-              float v[8];
-              unpack16x8<F16>(xa[j][bt][h], v);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) sum += v[i];
-            }
-          m = lnb ? sum * inl : 0.f;
-#pragma unroll
-          for (int j = 0; j < DM_KB; ++j)
-            if (j < nw) {
-              float v[8];
-              unpack16x8<F16>(xa[j][bt][h], v);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) q = fmaf(v[i] - m, v[i] - m, q);
-            }
-        }
-        // quad merge: four lanes with equal counts
-        float n = nl;
-#pragma unroll
-        for (int o = 1; o <= 2; o <<= 1) {
-          const float m2 = __shfl_xor_sync(0xffffffffu, m, o), q2 = __shfl_xor_sync(0xffffffffu, q, o);
-          const float d = m2 - m;
-          q = q + q2 + d * d * (0.5f * n);   // na = nb = n: d^2 na nb / (2n) = d^2 n / 2
-          m = m + 0.5f * d;
-          n *= 2.f;
-        }
-        if (tig == 0) sred[warp * 16 * MT + bt * 16 + h * 8 + g] = make_float2(m, q);
+      for (int i = 0; i < GPL; ++i) {
+        const int gi = p + TPR * i;
+        gv[i] = gi < NG && r < B ? st_in[(long)gi * B + r] : make_float2(0.f, 0.f);
+        sm += gv[i].x;
       }
-    __syncthreads();
 #pragma unroll
-    for (int bt = 0; bt < MT; ++bt)
+      for (int o = TPR / 2; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
+      const float m = lnb ? 16.f * sm * inK : 0.f;
+      float q = 0.f;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float sm = 0.f, q = 0.f;
+      for (int i = 0; i < GPL; ++i)
+        if (p + TPR * i < NG) q += gv[i].y + 16.f * (gv[i].x - m) * (gv[i].x - m);
 #pragma unroll
-        for (int w = 0; w < DM_WARPS; ++w) {
-          const float nb = 32.f * min(DM_KB, (kn / 32 - w + DM_WARPS - 1) / DM_WARPS);
-          sm = fmaf(nb, sred[w * 16 * MT + bt * 16 + h * 8 + g].x, sm);
+      for (int o = TPR / 2; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+      if (p == 0) srow[r] = make_float2(m, 1.0f / sqrtf(q * inK + eps));
+      __syncthreads();
+#pragma unroll
+      for (int bt = 0; bt < MT; ++bt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float2 t = srow[bt * 16 + h * 8 + g];
+          mu[bt][h] = t.x;
+          rs[bt][h] = t.y;
         }
-        const float m = lnb ? sm * inK : 0.f;
+    } else {
+      float2* sred = reinterpret_cast<float2*>(red);   // [DM_WARPS][16 MT] (mean, M2) of the warp's columns
+      const int nw = min(DM_KB, (kn / 32 - warp + DM_WARPS - 1) / DM_WARPS);   // this warp's blocks in range
+      const float nl = 8.f * nw;                                             // values per lane
+      const float inl = nw > 0 ? 1.f / nl : 0.f;
 #pragma unroll
-        for (int w = 0; w < DM_WARPS; ++w) {
-          const float nb = 32.f * min(DM_KB, (kn / 32 - w + DM_WARPS - 1) / DM_WARPS);
-          const float2 t = sred[w * 16 * MT + bt * 16 + h * 8 + g];
-          const float d = t.x - m;
-          q += t.y + nb * d * d;
+      for (int bt = 0; bt < MT; ++bt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float m = 0.f, q = 0.f;
+          if (nw > 0 && bt * 16 + h * 8 + g < B) {
+            float sum = 0.f;
+#pragma unroll
+            for (int j = 0; j < DM_KB; ++j)
+              if (j < nw) {
+                float v[8];
+                unpack16x8<F16>(xa[j][bt][h], v);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) sum += v[i];
+              }
+            m = lnb ? sum * inl : 0.f;
+#pragma unroll
+            for (int j = 0; j < DM_KB; ++j)
+              if (j < nw) {
+                float v[8];
+                unpack16x8<F16>(xa[j][bt][h], v);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) q = fmaf(v[i] - m, v[i] - m, q);
+              }
+          }
+          // quad merge: four lanes with equal counts
+          float n = nl;
+#pragma unroll
+          for (int o = 1; o <= 2; o <<= 1) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, m, o), q2 = __shfl_xor_sync(0xffffffffu, q, o);
+            const float d = m2 - m;
+            q = q + q2 + d * d * (0.5f * n);   // na = nb = n: d^2 na nb / (2n) = d^2 n / 2
+            m = m + 0.5f * d;
+            n *= 2.f;
+          }
+          if (tig == 0) sred[warp * 16 * MT + bt * 16 + h * 8 + g] = make_float2(m, q);
         }
-        mu[bt][h] = m;
-        // RMSNorm: q is the sum of squares (every mean stayed 0)
-        rs[bt][h] = 1.0f / sqrtf(q * inK + eps);
-      }
+      __syncthreads();
+#pragma unroll
+      for (int bt = 0; bt < MT; ++bt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float sm = 0.f, q = 0.f;
+#pragma unroll
+          for (int w = 0; w < DM_WARPS; ++w) {
+            const float nb = 32.f * min(DM_KB, (kn / 32 - w + DM_WARPS - 1) / DM_WARPS);
+            sm = fmaf(nb, sred[w * 16 * MT + bt * 16 + h * 8 + g].x, sm);
+          }
+          const float m = lnb ? sm * inK : 0.f;
+#pragma unroll
+          for (int w = 0; w < DM_WARPS; ++w) {
+            const float nb = 32.f * min(DM_KB, (kn / 32 - w + DM_WARPS - 1) / DM_WARPS);
+            const float2 t = sred[w * 16 * MT + bt * 16 + h * 8 + g];
+            const float d = t.x - m;
+            q += t.y + nb * d * d;
+          }
+          mu[bt][h] = m;
+          // RMSNorm: q is the sum of squares (every mean stayed 0)
+          rs[bt][h] = 1.0f / sqrtf(q * inK + eps);
+        }
+    }
     if (ln_bulk) lnwait = !mbar_wait(smem_u32(&lnbar), 0, &s_abort);
 #pragma unroll
     for (int j = 0; j < DM_KB; ++j) {
@@ -365,12 +420,15 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
 #pragma unroll
     for (int t = 0; t < DM_OPT; ++t) {
       const int o = threadIdx.x + DM_THREADS * t, bb = o / DM_ROWS, nn = o % DM_ROWS, n = r0 + nn;
-      if (o >= B * DM_ROWS || n >= N) continue;
-      float y = 0.f;
+      const bool ok = o < B * DM_ROWS && n < N;
+      float y = 0.f, v = 0.f;
+      if (ok) {
 #pragma unroll
-      for (int w = 0; w < DM_WARPS; ++w) y += red[((w * 16 * MT) + bb) * 16 + nn];
-      if (nkc == 1) dm_epilogue<T>(y, pb[t], pr[t], bb, n, N, mode, out, out2, outf);
-      else dm_st_cluster(smem_u32(cred + ((j & 1) * nkc + kc) * (B * DM_ROWS) + o), 0u, y);
+        for (int w = 0; w < DM_WARPS; ++w) y += red[((w * 16 * MT) + bb) * 16 + nn];
+        if (nkc == 1) v = dm_epilogue<T>(y, pb[t], pr[t], bb, n, N, mode, out, out2, outf);
+        else dm_st_cluster(smem_u32(cred + ((j & 1) * nkc + kc) * (B * DM_ROWS) + o), 0u, y);
+      }
+      if (nkc == 1 && st_out) dm_group_stats(v, ok, st_out, s, B, bb, lane);
     }
     if (nkc > 1) {
       // every CTA arrives here once per slice, a timed-out one included
@@ -379,10 +437,14 @@ dec_mma_kernel(const T* __restrict__ X, int B, int K, const T* __restrict__ W, i
 #pragma unroll
         for (int t = 0; t < DM_OPT; ++t) {
           const int o = threadIdx.x + DM_THREADS * t, bb = o / DM_ROWS, n = r0 + o % DM_ROWS;
-          if (o >= B * DM_ROWS || n >= N) continue;
-          float y = 0.f;
-          for (int q = 0; q < nkc; ++q) y += cred[((j & 1) * nkc + q) * (B * DM_ROWS) + o];
-          dm_epilogue<T>(y, pb[t], pr[t], bb, n, N, mode, out, out2, outf);
+          const bool ok = o < B * DM_ROWS && n < N;
+          float v = 0.f;
+          if (ok) {
+            float y = 0.f;
+            for (int q = 0; q < nkc; ++q) y += cred[((j & 1) * nkc + q) * (B * DM_ROWS) + o];
+            v = dm_epilogue<T>(y, pb[t], pr[t], bb, n, N, mode, out, out2, outf);
+          }
+          if (st_out) dm_group_stats(v, ok, st_out, s, B, bb, lane);
         }
       }
     }
@@ -407,8 +469,9 @@ bool dec_mma_supported(int B, int K, int N, bool ln) {
 template <typename T>
 cudaError_t launch_dec_mma(const T* X, int B, int K, const T* W, int N, const float* bias, const T* resid, int mode,
                            T* out, T* out2, float* outf, unsigned* err, cudaStream_t s, const float* lng,
-                           const float* lnb, float eps) {
+                           const float* lnb, float eps, float2* st_out, const float2* st_in) {
   if (!dec_mma_supported(B, K, N, lng != nullptr)) return cudaErrorInvalidValue;
+  if ((st_out && (mode != 0 || N % 16)) || (st_in && (!lng || K % 16))) return cudaErrorInvalidValue;
   if (((uintptr_t)X & 15) || ((uintptr_t)W & 15)) return cudaErrorInvalidValue;
   if (!g_dm_sms) {
     int dev = 0, n = 0;
@@ -429,7 +492,8 @@ cudaError_t launch_dec_mma(const T* X, int B, int K, const T* W, int N, const fl
   if (nbuf < 2) nbuf = 2;
   const size_t smem = nbuf * slot + red;
   void (*kern)(const T*, int, int, const T*, int, int, int, const float*, const T*, int, T*, T*, float*, int,
-               unsigned*, const float*, const float*, float) = MT == 1 ? dec_mma_kernel<T, 1> : dec_mma_kernel<T, 2>;
+               unsigned*, const float*, const float*, float, float2*, const float2*) =
+      MT == 1 ? dec_mma_kernel<T, 1> : dec_mma_kernel<T, 2>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
@@ -441,7 +505,7 @@ cudaError_t launch_dec_mma(const T* X, int B, int K, const T* W, int N, const fl
   ++g_kernel_launches;
   if (nkc == 1)
     return launch_k(kern, dim3(ngrp), dim3(DM_THREADS), smem, s, X, B, K, W, N, nkc, kcl, bias, resid, mode, out, out2,
-                    outf, nbuf, err, lng, lnb, eps);
+                    outf, nbuf, err, lng, lnb, eps, st_out, st_in);
   // clusters of nkc CTAs (and the programmatic dependent launch of launch_k)
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ngrp * nkc);
@@ -458,11 +522,12 @@ cudaError_t launch_dec_mma(const T* X, int B, int K, const T* W, int N, const fl
   cfg.attrs = at;
   cfg.numAttrs = g_pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, X, B, K, W, N, nkc, kcl, bias, resid, mode, out, out2, outf, nbuf, err, lng,
-                            lnb, eps);
+                            lnb, eps, st_out, st_in);
 }
 
 template cudaError_t launch_dec_mma<bf16>(const bf16*, int, int, const bf16*, int, const float*, const bf16*, int,
                                           bf16*, bf16*, float*, unsigned*, cudaStream_t, const float*, const float*,
-                                          float);
+                                          float, float2*, const float2*);
 template cudaError_t launch_dec_mma<f16>(const f16*, int, int, const f16*, int, const float*, const f16*, int, f16*,
-                                         f16*, float*, unsigned*, cudaStream_t, const float*, const float*, float);
+                                         f16*, float*, unsigned*, cudaStream_t, const float*, const float*, float,
+                                         float2*, const float2*);

@@ -60,6 +60,7 @@ struct gpt_model {
   void *kc, *vc, *dx, *dh, *dq, *datt, *du, *da, *dxf;
   float *dlogits, *dmu, *drs, *dpart;
   unsigned* dacnt = nullptr;    // decode attention: per-(row, head) arrival counters (kept zero)
+  float2* dxst = nullptr;       // decode: LayerNorm statistics of the residual rows per 16-column group
   int* dtok;
   int fwd_B = 0, fwd_T = 0;
   bool have_targets = false, logits_valid = false;
@@ -369,6 +370,7 @@ static int build_arena(gpt_model* m) {
   cv.add((void**)&m->dtok, Bx * 4);
   cv.add((void**)&m->dpart, dec_attn_part_floats((int)Bx, m->H, m->d) * 4);
   cv.add((void**)&m->dacnt, Bx * m->H * 4);
+  cv.add((void**)&m->dxst, (C / 16 + 1) * Bx * 8);
   cv.add((void**)&m->dsrc, Bx * (size_t)m->Tmax * 4);
   cv.add((void**)&m->dbcs, Bx * BEAM_MAX_WIDTH * 4);
   cv.add((void**)&m->dbct, Bx * BEAM_MAX_WIDTH * 4);
@@ -897,12 +899,17 @@ static int backward_llama(gpt_model* m) {
 // 32 rows of a 16-bit model run on the mma.sync kernel that spreads 16-row
 // weight slices over every SM; fp32 models on the GEMV that streams each
 // weight row once.
+// With st (the projections that write the residual rows) the kernel also
+// leaves their LayerNorm statistics there for the next dec_ln_proj; st is
+// dropped (and the next LayerNorm takes its own) where the kernel cannot.
 template <typename T>
 static cudaError_t dec_proj(gpt_model* m, const T* X, int B, int K, const T* W, int N, const float* bias,
-                            const T* resid, int mode, T* out, T* out2, float* outf, cudaStream_t s) {
+                            const T* resid, int mode, T* out, T* out2, float* outf, cudaStream_t s,
+                            float2* st = nullptr) {
   if constexpr (sizeof(T) == 2) {
     if (dec_mma_supported(B, K, N))
-      return launch_dec_mma<T>(X, B, K, W, N, bias, resid, mode, out, out2, outf, &m->sc->err, s);
+      return launch_dec_mma<T>(X, B, K, W, N, bias, resid, mode, out, out2, outf, &m->sc->err, s, nullptr, nullptr,
+                               0.f, mode == 0 && N % 16 == 0 ? st : nullptr);
   }
   return launch_gemv<T>(X, B, K, W, N, bias, resid, mode, out, out2, outf, s);
 }
@@ -913,11 +920,11 @@ static cudaError_t dec_proj(gpt_model* m, const T* X, int B, int K, const T* W, 
 template <typename T>
 static cudaError_t dec_ln_proj(gpt_model* m, const T* x, const float* g, const float* b, T* h, int B, int K,
                                const T* W, int N, const float* bias, const T* resid, int mode, T* out, T* out2,
-                               float* outf, cudaStream_t s) {
+                               float* outf, cudaStream_t s, const float2* st = nullptr) {
   if constexpr (sizeof(T) == 2) {
     if (dec_mma_supported(B, K, N, true))
       return launch_dec_mma<T>(x, B, K, W, N, bias, resid, mode, out, out2, outf, &m->sc->err, s, g, b,
-                               m->cfg.ln_eps);
+                               m->cfg.ln_eps, nullptr, K % 16 == 0 ? st : nullptr);
   }
   cudaError_t e = launch_ln_fwd<T>(x, g, b, h, m->dmu, m->drs, B, K, m->cfg.ln_eps, s);
   if (e != cudaSuccess) return e;
@@ -962,29 +969,36 @@ static int decode_step(gpt_model* m, int B, int Tp, int n_new, int32_t* out, cud
   int* stepc = &m->sc->dec_step;
   // LayerNorm parameters (Llama: RMSNorm, gains only) and biases (Llama: none)
   auto P0 = [&](size_t off) -> const float* { return ll ? nullptr : A.P(off); };
+  // LayerNorm statistics of the residual rows travel from the kernel that
+  // writes the rows (embedding, output projection, fc2) to the next
+  // LayerNorm-fused projection where both run the 16-bit decode kernels
+  float2* st = C % 16 == 0 ? m->dxst : nullptr;
+  const bool mma = sizeof(T) == 2;
+  const float2* st_o = mma && dec_mma_supported(B, C, C) ? st : nullptr;    // after the output projection
+  const float2* st_f2 = mma && dec_mma_supported(B, F, C) ? st : nullptr;   // after fc2
   // the token fed at step st sits at position Tp - 1 + st
   CK(launch_dec_embed<T>(m->dtok, A.P(m->o_wte), ll ? nullptr : A.P(m->o_wpe), x, B, C, Tp - 1, stepc, m->Tmax,
-                         &m->sc->err, s));
+                         &m->sc->err, s, st));
   for (int l = 0; l < m->NL; ++l) {
     const LayerOff& lo = m->L[l];
     CK(dec_ln_proj<T>(m, x, A.P(lo.ln1_g), P0(lo.ln1_b), h, B, C, A.W(lo.w_qkv), QW, P0(lo.b_qkv), nullptr, 0, q,
-                      nullptr, nullptr, s));
+                      nullptr, nullptr, s, l == 0 ? st : st_f2));
     if (ll) CK(rope16<T>(q, QW, B, H, C, m->Hkv, d, nullptr, Tp - 1, stepc, m->rope_tab, m->Tmax, false, s));
     CK(launch_dec_attn<T>(q, kc + l * kvl, vc + l * kvl, att, m->dpart, m->dacnt, B, H, d, m->Tmax, Tp - 1, stepc, DL,
                           s));
-    CK(dec_proj<T>(m, att, B, C, A.W(lo.w_o), C, P0(lo.b_o), x, 0, x, nullptr, nullptr, s));
+    CK(dec_proj<T>(m, att, B, C, A.W(lo.w_o), C, P0(lo.b_o), x, 0, x, nullptr, nullptr, s, st));
     if (ll) {
       CK(dec_ln_proj<T>(m, x, A.P(lo.ln2_g), nullptr, h, B, C, A.W(lo.w_fc), 2 * F, nullptr, nullptr, 0, u, nullptr,
-                        nullptr, s));
+                        nullptr, s, st_o));
       CK(swiglu16<T>(u, a, B, F, s));
     } else {
       CK(dec_ln_proj<T>(m, x, A.P(lo.ln2_g), A.P(lo.ln2_b), h, B, C, A.W(lo.w_fc), F, A.P(lo.b_fc), nullptr, 1, u, a,
-                        nullptr, s));
+                        nullptr, s, st_o));
     }
-    CK(dec_proj<T>(m, a, B, F, A.W(lo.w_fc2), C, P0(lo.b_fc2), x, 0, x, nullptr, nullptr, s));
+    CK(dec_proj<T>(m, a, B, F, A.W(lo.w_fc2), C, P0(lo.b_fc2), x, 0, x, nullptr, nullptr, s, st));
   }
   CK(dec_ln_proj<T>(m, x, A.P(m->o_lnf_g), P0(m->o_lnf_b), xf, B, C, A.W(m->o_head), m->Vp, nullptr, nullptr, 2,
-                    nullptr, nullptr, m->dlogits, s));
+                    nullptr, nullptr, m->dlogits, s, m->NL > 0 ? st_f2 : st));
   if (m->beam_w) {
     const int W = m->beam_w;
     CK(launch_beam_topk(m->dlogits, m->Vp, m->V, B / W, W, false, m->beam_scores, m->dbcs, m->dbct, s));

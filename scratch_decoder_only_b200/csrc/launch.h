@@ -156,10 +156,12 @@ cudaError_t launch_attn_bwd_tc(const bf16* qkv, const bf16* out, const bf16* dou
 
 // ---- decode.cu
 // decode kernels read the position as pos0 + *step (device counter)
-// wpe may be null (no position table)
+// wpe may be null (no position table); st (optional, C % 16 == 0): per
+// 16-column group g and row b, st[g B + b] = (mean, sum of squared
+// deviations) of the stored row
 template <typename T>
 cudaError_t launch_dec_embed(const int* tok, const float* wte, const float* wpe, T* x, int B, int C, int pos0,
-                             const int* step, int max_seq, unsigned* err, cudaStream_t s);
+                             const int* step, int max_seq, unsigned* err, cudaStream_t s, float2* st = nullptr);
 template <typename T>
 cudaError_t launch_gemv(const T* X, int B, int K, const T* W, int N, const float* bias, const T* resid,
                         int mode, T* out, T* out2, float* outf, cudaStream_t s);
@@ -201,12 +203,16 @@ cudaError_t launch_gather_last(const T* x, int B, int Tp, int C, T* out, cudaStr
 // GELU into out / out2, 2: fp32 logits).  X and W 16-byte aligned; K > 768
 // runs as clusters of CTAs that split the k range.  With lng the kernel
 // first applies LayerNorm (lnb: shift; none: RMSNorm) with eps to the rows
-// of X, which then hold the raw residual (K <= 768).
+// of X, which then hold the raw residual (K <= 768), from the statistics
+// st_in when given, else its own.  st_out (mode 0, N % 16 == 0): the kernel
+// also writes, per 16-column group g and row b, st_out[g B + b] = (mean,
+// sum of squared deviations) of the stored outputs.
 bool dec_mma_supported(int B, int K, int N, bool ln = false);
 template <typename T>
 cudaError_t launch_dec_mma(const T* X, int B, int K, const T* W, int N, const float* bias, const T* resid, int mode,
                            T* out, T* out2, float* outf, unsigned* err, cudaStream_t s, const float* lng = nullptr,
-                           const float* lnb = nullptr, float eps = 0.f);
+                           const float* lnb = nullptr, float eps = 0.f, float2* st_out = nullptr,
+                           const float2* st_in = nullptr);
 
 // ---- beam.cu: beam search over the decode rows (row r = b * W + w)
 #define BEAM_MAX_WIDTH 8
