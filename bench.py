@@ -483,6 +483,55 @@ def bench_decode(torch, dev, args):
     return res
 
 
+def decode_profile(torch, dev, batches=(1, 32), n_new=17):
+    """Per-kernel critical path of greedy decode (CUPTI kernel records through
+    torch.profiler): with programmatic dependent launch a kernel starts while
+    its predecessor drains, so each kernel is charged end_k - end_(k-1) in
+    stream order.  The projections are labelled by their place in the step
+    (q/k/v with LN1, output, fc with LN2, fc2; then the head with the final
+    LN).  Prints a table per batch; not a bench value."""
+    from torch.profiler import profile, ProfilerActivity
+    from scratch_decoder_only_b200.gpt import GPT
+    wl = CF.GPT2_DECODE
+    model = GPT(wl.model, wl.init_seed)
+    for B in batches:
+        prompt = torch.from_numpy(S.make_prompts(wl, B, 128)).to(dev)
+        model.greedy_decode(prompt, n_new)
+        torch.cuda.synchronize()
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            model.greedy_decode(prompt, n_new)
+            torch.cuda.synchronize()
+        evs = sorted([e for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA],
+                     key=lambda e: e.time_range.start)
+        adv = [i for i, e in enumerate(evs) if "step_advance" in e.name]
+        evs = evs[adv[0] + 1: adv[-1] + 1]   # the replayed steps after the first
+        nsteps = len(adv) - 1
+        agg, order = {}, []
+        prev_end, nmma = evs[0].time_range.start, 0
+        names = ["q/k/v + LN1", "out", "fc + LN2", "fc2"]
+        for e in evs:
+            d = max(0.0, e.time_range.end - prev_end)
+            prev_end = max(prev_end, e.time_range.end)
+            k = e.name.split("(")[0].replace("void ", "")
+            if "step_advance" in k:
+                nmma = 0
+            if "dec_mma" in k:
+                k = "dec_mma " + (names[nmma % 4] if nmma < 4 * wl.model.n_layers else "head + final LN")
+                nmma += 1
+            if k not in agg:
+                agg[k] = [0, 0.0]
+                order.append(k)
+            agg[k][0] += 1
+            agg[k][1] += d
+        tot = sum(v[1] for v in agg.values()) / nsteps
+        print(f"batch {B}: {nsteps} steps, critical path {tot:.1f} us per step ({B / tot * 1e6:.0f} tok/s)")
+        print(f"  {'kernel':48s} {'per step':>9s} {'us/step':>9s} {'us each':>8s} {'share':>6s}")
+        for k in sorted(order, key=lambda k: -agg[k][1]):
+            n, t = agg[k]
+            print(f"  {k[:48]:48s} {n // nsteps:9d} {t / nsteps:9.1f} {t / n:8.2f} {100 * t / nsteps / tot:5.1f}%")
+    model.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -494,7 +543,13 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None, help="override the batch (profiling of small cases)")
+    ap.add_argument("--decode-profile", action="store_true",
+                    help="print the per-kernel critical path of greedy decode and exit (no bench line)")
     args = ap.parse_args()
+    if args.decode_profile:
+        import torch
+        decode_profile(torch, torch.device("cuda", 0))
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

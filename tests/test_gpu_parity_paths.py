@@ -140,9 +140,10 @@ def test_greedy_decode_d64_bf16_against_oracle_logits(torch, B):
     sequence the GPU generated (teacher-forced: one full-prefix forward), up
     to a bf16 tolerance `tol` (1 % of the row's largest logit magnitude);
     where the oracle's top-2 gap exceeds tol the token must be exactly the
-    oracle's argmax.  Batches 1 and 4 run every step after the first in the
-    persistent decode kernel; batches 12 and 32 run the mma.sync slice kernel
-    for the projections and the split attention over the cache."""
+    oracle's argmax.  Every batch runs the mma.sync projection kernel (one
+    and two 16-row tiles of x: batches 1, 4, 12 and 32) with the LayerNorm
+    folded in, and the decode attention over the cache (one key piece at
+    batch 32, several at batch 1)."""
     cfg = ocfg(DEC64)
     model = new_model(DEC64, 13)
     tame_attention(model, cfg)
