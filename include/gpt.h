@@ -322,6 +322,20 @@ int gpt_set_scalars(gpt_model* m, const gpt_scalars* in);
  * warmup_steps, or not 0 <= min_lr <= max_lr). */
 int gpt_set_lr_schedule(gpt_model* m, const gpt_lr_schedule* sched);
 
+/* One training step, gpt_forward_loss + gpt_backward + gpt_clip_adamw_step
+ * with the same arguments and results, launched as one CUDA graph: the
+ * step's kernels are captured once and the graph is replayed while the
+ * pointers, B, T and the hyper-parameters match the captured call (any change
+ * captures anew).  Device buffers are read when the step runs, so new tokens
+ * written into the same buffers need no new capture.  Falls back to the three
+ * calls when profiling is on or the runtime refuses the capture.
+ *  tokens, targets  device int32 [B, T]; seg_ids device int32 [B, T] or NULL
+ *  loss_dev, grad_norm_dev (device float [1]) and skipped_dev (device int32
+ *  [1]) may be NULL.
+ * Errors: as the three calls (GPT_ERR_ARG for NULL targets). */
+int gpt_train_step(gpt_model* m, const int32_t* tokens, const int32_t* targets, const int32_t* seg_ids, int B, int T,
+                   const gpt_adamw* hp, float* loss_dev, float* grad_norm_dev, int32_t* skipped_dev);
+
 /* K training steps in one call, all enqueued without a host round trip:
  * for k = 0..K-1, gpt_forward_loss on tokens + k*B*T (targets, seg_ids
  * likewise; seg_ids may be NULL), gpt_backward and gpt_clip_adamw_step.

@@ -71,6 +71,16 @@ struct gpt_model {
   cudaStream_t cap_stream = nullptr;
   cudaEvent_t ev_a = nullptr, ev_b = nullptr;
   cudaGraphExec_t dec_graph = nullptr;
+  // gpt_train_step: one captured training step, replayed while its inputs match
+  cudaGraphExec_t train_graph = nullptr;
+  struct TrainKey {
+    const void *tok, *tgt, *seg, *loss, *gn, *skip;
+    int B, T;
+    float lr, beta1, beta2, eps, wd, clip;
+    bool operator==(const TrainKey& o) const { return memcmp(this, &o, sizeof(TrainKey)) == 0; }
+  } train_key;
+  int train_kernels = 0;
+  bool train_graph_ok = true;   // false once a capture failed: plain launches from then on
   int dec_B = 0, dec_Tp = 0, dec_nnew = 0, dec_kernels = 0;
   int32_t* dec_out = nullptr;
   // sampling decode (gpt_sample_decode); smp_on = false: greedy
@@ -484,7 +494,7 @@ static int gemm16(gpt_model* m, int M, int N, int K, const T16* A, long lda, boo
     // accumulating, onto the stored gradient instead
     EpiParams<T16> e2 = epi;
     e2.kind = EPI_F32_ADD;
-    if (!add_f32) CK(cudaMemsetAsync(epi.outf, 0, (size_t)M * N * 4, m->stream));
+    if (!add_f32) CK(launch_zero(epi.outf, (size_t)M * N * 4, m->stream));
     CK(tc_gemm<T16>(M, N, K, A, lda, a_t, B, ldb, b_t, e2, splits, &m->sc->err, m->stream));
   } else {
     CK(tc_gemm<T16>(M, N, K, A, lda, a_t, B, ldb, b_t, epi, 1, &m->sc->err, m->stream));
@@ -737,8 +747,8 @@ static int backward_impl(gpt_model* m) {
   // embeddings: scatter-add by token and by position
   ProfScope ps_emb(m, PC_EMBED, 0, (double)M * C * 12);
   if (!m->accum_now) {
-    if (!m->cfg.tied) CK(cudaMemsetAsync(A.G(m->o_wte), 0, (size_t)Vp * C * 4, s));
-    CK(cudaMemsetAsync(A.G(m->o_wpe), 0, (size_t)m->Tmax * C * 4, s));
+    if (!m->cfg.tied) CK(launch_zero(A.G(m->o_wte), (size_t)Vp * C * 4, s));
+    CK(launch_zero(A.G(m->o_wpe), (size_t)m->Tmax * C * 4, s));
   }
   CK(launch_embed_bwd<T>(m->dres32, m->tok, m->pos, A.G(m->o_wte), A.G(m->o_wpe), M, C, s));
   m->have_targets = false;
@@ -885,7 +895,7 @@ static int backward_llama(gpt_model* m) {
     CK(launch_reduce_segs(segs.data(), (int)segs.size(), m->accum_now, s));
   }
   ProfScope ps_emb(m, PC_EMBED, 0, (double)M * C * 8);
-  if (!m->cfg.tied && !m->accum_now) CK(cudaMemsetAsync(A.G(m->o_wte), 0, (size_t)Vp * C * 4, s));
+  if (!m->cfg.tied && !m->accum_now) CK(launch_zero(A.G(m->o_wte), (size_t)Vp * C * 4, s));
   CK(launch_embed_bwd<T>(m->dres32, m->tok, m->pos, A.G(m->o_wte), nullptr, M, C, s));
   m->have_targets = false;
   return GPT_OK;
@@ -1184,6 +1194,7 @@ void gpt_destroy(gpt_model* m) {
   cudaDeviceSynchronize();
   for (auto e : m->evpool) cudaEventDestroy(e);
   if (m->dec_graph) cudaGraphExecDestroy(m->dec_graph);
+  if (m->train_graph) cudaGraphExecDestroy(m->train_graph);
   if (m->ev_a) cudaEventDestroy(m->ev_a);
   if (m->ev_b) cudaEventDestroy(m->ev_b);
   if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
@@ -1297,6 +1308,75 @@ int gpt_set_lr_schedule(gpt_model* m, const gpt_lr_schedule* sched) {
   sc.sched_max_lr = q.max_lr;
   sc.sched_min_lr = q.min_lr;
   CK(cudaMemcpy(m->sc, &sc, sizeof(sc), cudaMemcpyHostToDevice));
+  return GPT_OK;
+}
+
+int gpt_train_step(gpt_model* m, const int32_t* tokens, const int32_t* targets, const int32_t* seg_ids, int B, int T,
+                   const gpt_adamw* hp, float* loss_dev, float* grad_norm_dev, int32_t* skipped_dev) {
+  if (!m) return GPT_ERR_ARG;
+  m->err.clear();
+  if (!tokens || !targets || !hp) FAIL(GPT_ERR_ARG, "tokens, targets and hp must be non-NULL");
+  if (B < 1 || B > m->Bmax) FAIL(GPT_ERR_ARG, "B out of range [1, max_batch]");
+  if (T < 1 || T > m->Tmax) FAIL(GPT_ERR_ARG, "T out of range [1, max_seq]");
+  if (!(hp->clip_norm > 0.f)) FAIL(GPT_ERR_ARG, "clip_norm must be > 0");
+  auto plain = [&]() -> int {
+    int r = gpt_forward_loss(m, tokens, targets, seg_ids, B, T, loss_dev);
+    if (r == GPT_OK) r = gpt_backward(m);
+    if (r == GPT_OK) r = gpt_clip_adamw_step(m, hp, grad_norm_dev, skipped_dev);
+    return r;
+  };
+  // profiling records host-side events per kernel class: no graph then
+  if (m->prof || !m->train_graph_ok) return plain();
+  gpt_model::TrainKey key;
+  memset(&key, 0, sizeof(key));
+  key.tok = tokens; key.tgt = targets; key.seg = seg_ids; key.loss = loss_dev; key.gn = grad_norm_dev;
+  key.skip = skipped_dev; key.B = B; key.T = T; key.lr = hp->lr; key.beta1 = hp->beta1; key.beta2 = hp->beta2;
+  key.eps = hp->eps; key.wd = hp->weight_decay; key.clip = hp->clip_norm;
+  if (!m->train_graph || !(key == m->train_key)) {
+    if (m->train_graph) { cudaGraphExecDestroy(m->train_graph); m->train_graph = nullptr; }
+    if (!m->cap_stream) CK(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking));
+    // capture on the library's own stream (the caller's may be the legacy
+    // default stream, which cannot be captured); nothing runs during capture
+    cudaStream_t s0 = m->stream;
+    m->stream = m->cap_stream;
+    const unsigned long long n0 = g_kernel_launches;
+    cudaGraph_t g = nullptr;
+    cudaError_t eb = cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal);
+    int r = GPT_ERR_CUDA;
+    unsigned long long n1 = n0;
+    if (eb == cudaSuccess) {
+      r = plain();
+      n1 = g_kernel_launches;
+      cudaError_t ec = cudaStreamEndCapture(m->cap_stream, &g);
+      if (r == GPT_OK && ec != cudaSuccess) r = GPT_ERR_CUDA;
+    }
+    m->stream = s0;
+    g_kernel_launches = n0;   // counted per replay below
+    cudaError_t ei = cudaErrorUnknown;
+    if (r == GPT_OK && g) ei = cudaGraphInstantiate(&m->train_graph, g, 0);
+    if (g) cudaGraphDestroy(g);
+    if (r != GPT_OK || ei != cudaSuccess) {
+      // an argument or state error is the caller's; a capture the runtime
+      // refused falls back to plain launches for good
+      cudaGetLastError();
+      m->train_graph = nullptr;
+      if (r == GPT_ERR_ARG || r == GPT_ERR_STATE) return r;
+      m->train_graph_ok = false;
+      m->err.clear();
+      return plain();
+    }
+    m->train_kernels = (int)(n1 - n0);
+    m->train_key = key;
+  }
+  CK(cudaGraphLaunch(m->train_graph, m->stream));
+  g_kernel_launches += (unsigned long long)m->train_kernels;
+  // the host-side state a plain step leaves
+  m->seg_used = seg_ids != nullptr;
+  m->fwd_B = B;
+  m->fwd_T = T;
+  m->have_targets = false;
+  m->logits_valid = false;
+  m->accum_now = false;
   return GPT_OK;
 }
 

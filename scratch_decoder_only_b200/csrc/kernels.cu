@@ -106,15 +106,52 @@ __global__ void __launch_bounds__(1024) prep_kernel(const int32_t* __restrict__ 
   }
 }
 
+// ---------------------------------------------------------------------------
+// Zero fill inside the dependent-launch chain (a memset node would end the
+// overlap of its neighbours).  The buffer belongs to no kernel still running
+// (the caller's contract), so the fill starts at once and overlaps the
+// previous kernel; the wait sits at the end, so this kernel completes only
+// after its predecessor and the chain's order holds for the next kernel.
+// ---------------------------------------------------------------------------
+__global__ void zero_fill_kernel(uint8_t* p, size_t bytes) {
+  griddep_release();
+  const size_t head = (16 - (reinterpret_cast<uintptr_t>(p) & 15)) & 15;
+  const size_t pre = head < bytes ? head : bytes;
+  const size_t n16 = (bytes - pre) / 16, tail0 = pre + n16 * 16;
+  const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x, nth = (size_t)gridDim.x * blockDim.x;
+  if (tid < pre) p[tid] = 0;
+  uint4* q = reinterpret_cast<uint4*>(p + pre);
+  for (size_t i = tid; i < n16; i += nth) q[i] = make_uint4(0u, 0u, 0u, 0u);
+  if (tid < bytes - tail0) p[tail0 + tid] = 0;
+  griddep_wait();
+}
+
+static int g_zero_sms = 0;
+
+cudaError_t launch_zero(void* p, size_t bytes, cudaStream_t s) {
+  if (!bytes) return cudaSuccess;
+  if (!g_zero_sms) {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    g_zero_sms = n > 0 ? n : 148;
+  }
+  size_t blocks = (bytes / 16 + 255) / 256;
+  if (blocks > (size_t)g_zero_sms * 4) blocks = (size_t)g_zero_sms * 4;
+  if (blocks < 1) blocks = 1;
+  ++g_kernel_launches;
+  return launch_k(zero_fill_kernel, dim3((unsigned)blocks), dim3(256), 0, s, (uint8_t*)p, bytes);
+}
+
 cudaError_t launch_prep(const int32_t* tokens, const int32_t* targets, const int32_t* seg, int B, int T,
                         int V, int* tok_out, int* tgt_out, int* pos_out, int* dstart_out,
                         DevScalars* sc, cudaStream_t s) {
   if (targets) {
-    cudaError_t e = cudaMemsetAsync(&sc->n_valid, 0, sizeof(int), s);
+    cudaError_t e = launch_zero(&sc->n_valid, sizeof(int), s);
     if (e != cudaSuccess) return e;
   }
   if (seg) {
-    cudaError_t e = cudaMemsetAsync(&sc->attn_pairs, 0, sizeof(unsigned long long), s);
+    cudaError_t e = launch_zero(&sc->attn_pairs, sizeof(unsigned long long), s);
     if (e != cudaSuccess) return e;
   }
   int th = T >= 1024 ? 1024 : ((T + 31) / 32) * 32;
@@ -1283,7 +1320,7 @@ cudaError_t launch_clip_adamw_fused(float* p, const float* g, float* m, float* v
   }
   const int G = grid < max_blocks ? grid : max_blocks;
   if (G < 1) return cudaErrorNotSupported;
-  cudaError_t e = cudaMemsetAsync(&sc->opt_bar, 0, 2 * sizeof(unsigned), s);
+  cudaError_t e = launch_zero(&sc->opt_bar, 2 * sizeof(unsigned), s);
   if (e != cudaSuccess) return e;
   void* args[] = {&p, (void*)&g, &m, &v, &pw, &n, &partials, &clip, &beta1, &beta2, &eps, &wd, &lr, &sc, &norm_out,
                   &skipped_out};

@@ -35,6 +35,9 @@ struct DevScalars {
 };
 
 // ---- kernels.cu: embedding, LayerNorm, cross-entropy, reductions, optimiser
+// zero `bytes` bytes at p as a kernel in the dependent-launch chain; p must
+// not be in use by a kernel that may still run (the fill starts at once)
+cudaError_t launch_zero(void* p, size_t bytes, cudaStream_t s);
 cudaError_t launch_prep(const int32_t* tokens, const int32_t* targets, const int32_t* seg, int B, int T,
                         int V, int* tok_out, int* tgt_out, int* pos_out, int* dstart_out,
                         DevScalars* sc, cudaStream_t s);

@@ -30,7 +30,7 @@ EXPORTED = [
     "gpt_device_error", "gpt_last_error", "gpt_debug_poison_grad", "gpt_debug_wait_timeout",
     "gpt_kernel_launches", "gpt_profile_enable", "gpt_profile_read", "gpt_gemm_bf16",
     "gpt_gemm_bf16_splitk_noalloc", "gpt_noalloc_status", "gpt_set_lr_schedule", "gpt_train_steps",
-    "gpt_sample_decode", "gpt_backward_accumulate", "gpt_set_loss_weight", "gpt_beam_decode",
+    "gpt_sample_decode", "gpt_backward_accumulate", "gpt_set_loss_weight", "gpt_beam_decode", "gpt_train_step",
 ]
 
 
@@ -118,6 +118,7 @@ def load_library(path: str = LIB_PATH):
         "gpt_sample_decode": ([H, P, I, I, I, ctypes.POINTER(gpt_sampling), P, P], I),
         "gpt_beam_decode": ([H, P, I, I, I, I, P, P], I),
         "gpt_train_steps": ([H, P, P, P, I, I, I, ctypes.POINTER(gpt_adamw), P, P, P], I),
+        "gpt_train_step": ([H, P, P, P, I, I, ctypes.POINTER(gpt_adamw), P, P, P], I),
         "gpt_profile_read": ([H, ctypes.POINTER(gpt_prof_entry), I, ctypes.POINTER(I)], I),
     }
     for n in ("params", "grads", "adam_m", "adam_v"):
@@ -388,7 +389,11 @@ class GPT:
         return self.lib.gpt_debug_wait_timeout(self.h, timeout_us)
 
     def train_step(self, tokens, targets, seg_ids, hp: AdamWConfig, loss=None, grad_norm=None, skipped=None):
-        """forward_loss + backward + clip_adamw_step, all enqueued on the current stream."""
-        self.forward_loss(tokens, targets, seg_ids, loss)
-        self.backward()
-        self.clip_adamw_step(hp, grad_norm, skipped)
+        """forward_loss + backward + clip_adamw_step on the current stream, as
+        one replayed CUDA graph (gpt_train_step)."""
+        B, T = tokens.shape
+        self._sync_stream()
+        a = gpt_adamw(lr=hp.lr, beta1=hp.beta1, beta2=hp.beta2, eps=hp.eps, weight_decay=hp.weight_decay,
+                      clip_norm=hp.clip_norm)
+        return self._check(self.lib.gpt_train_step(self.h, _ptr(tokens), _ptr(targets), _ptr(seg_ids), B, T,
+                                                   ctypes.byref(a), _ptr(loss), _ptr(grad_norm), _ptr(skipped)))

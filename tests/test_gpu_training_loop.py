@@ -12,6 +12,8 @@ learning-rate schedule, the multi-step call and the loss scaler's growth.
   taken with 1999 good steps behind it doubles the scale; a non-finite one
   halves it and resets the count.
 * Gradient accumulation over micro-batches with a loss weight.
+* gpt_train_step, the training step as one replayed CUDA graph, against the
+  three separate calls.
 """
 import numpy as np
 import pytest
@@ -177,3 +179,47 @@ def test_gradient_accumulation_equals_one_large_batch(torch, wl_name):
         assert errs[worst] <= bar, (worst, errs[worst])
     errs = per_tensor_rel_l2(cfg, g_acc, g_big.astype(np.float64))
     assert max(errs.values()) <= bar
+
+
+def test_graph_step_matches_three_calls(torch):
+    """gpt_train_step (one captured graph per call signature, replayed) leaves
+    what gpt_forward_loss + gpt_backward + gpt_clip_adamw_step leave, to the
+    rounding that the embedding gradients' atomic order allows: parameters,
+    Adam moments, losses and gradient norms after four steps, with
+    new tokens written into the captured buffers between replays, a second
+    buffer pair (a new capture) and a changed learning rate (another)."""
+    from scratch_decoder_only_b200.gpt import GPT
+    wl = CF.BYTE_30M
+    mc = CF.ModelConfig(**{**wl.model.as_dict(), "n_layers": 2, "max_batch": 2, "max_seq": 256})
+    hp = CF.AdamWConfig(lr=3e-4, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1, clip_norm=1.0)
+    hp2 = CF.AdamWConfig(lr=1e-4, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1, clip_norm=1.0)
+    a, b = GPT(mc, 11), GPT(mc, 11)
+    rng = np.random.default_rng(12)
+    batches = [rng.integers(0, mc.vocab, size=(2, 129)).astype(np.int32) for _ in range(4)]
+    tok_a, tgt_a = torch.zeros((2, 128), dtype=torch.int32, device="cuda"), torch.zeros((2, 128), dtype=torch.int32,
+                                                                                       device="cuda")
+    tok_c, tgt_c = tok_a.clone(), tgt_a.clone()
+    la, lb = torch.zeros(4, device="cuda"), torch.zeros(4, device="cuda")
+    ga, gb = torch.zeros(4, device="cuda"), torch.zeros(4, device="cuda")
+    for i, x in enumerate(batches):
+        ta, tg = (tok_a, tgt_a) if i != 2 else (tok_c, tgt_c)
+        ta.copy_(torch.from_numpy(x[:, :-1])); tg.copy_(torch.from_numpy(x[:, 1:]))
+        h = hp if i < 3 else hp2
+        a.train_step(ta, tg, None, h, la[i:i + 1], ga[i:i + 1])
+        b.forward_loss(ta, tg, None, lb[i:i + 1])
+        b.backward()
+        b.clip_adamw_step(h, gb[i:i + 1])
+    torch.cuda.synchronize()
+    assert a.status() == 0 and b.status() == 0
+    # losses and norms see the embedding rows, so they match to rounding
+    assert np.allclose(la.cpu().numpy(), lb.cpu().numpy(), rtol=1e-5, atol=0)
+    assert np.allclose(ga.cpu().numpy(), gb.cpu().numpy(), rtol=1e-5, atol=0)
+    # the embedding tables (token rows, then positions: the first
+    # (Vp + max_seq) C values) take their gradients by atomic scatter-add, whose
+    # order varies from run to run, and every later step sees them: the
+    # parameters and moments agree to rounding (their update is one fused pass
+    # over the same gradients, so a graph that dropped, repeated or reordered a
+    # kernel would differ by whole steps, not by rounding)
+    for ga_, gb_ in ((a.get_params(), b.get_params()), (a.get_adam_m(), b.get_adam_m()),
+                     (a.get_adam_v(), b.get_adam_v())):
+        assert np.allclose(ga_, gb_, rtol=1e-3, atol=1e-7), np.max(np.abs(ga_ - gb_))
