@@ -507,8 +507,10 @@ def decode_profile(torch, dev, batches=(1, 32), n_new=17):
             torch.cuda.synchronize()
         evs = sorted([e for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA],
                      key=lambda e: e.time_range.start)
-        adv = [i for i, e in enumerate(evs) if "step_advance" in e.name]
-        evs = evs[adv[0] + 1: adv[-1] + 1]   # the replayed steps after the first
+        # a greedy step ends with its argmax (which also embeds the next token
+        # and advances the step); the first one closes the prefill
+        adv = [i for i, e in enumerate(evs) if "argmax" in e.name]
+        evs = evs[adv[0] + 1: adv[-1] + 1]   # the replayed steps
         nsteps = len(adv) - 1
         agg, order = {}, []
         prev_end, nmma = evs[0].time_range.start, 0
@@ -517,11 +519,13 @@ def decode_profile(torch, dev, batches=(1, 32), n_new=17):
             d = max(0.0, e.time_range.end - prev_end)
             prev_end = max(prev_end, e.time_range.end)
             k = e.name.split("(")[0].replace("void ", "")
-            if "step_advance" in k:
+            if "argmax" in k:
                 nmma = 0
             if "dec_mma" in k:
                 k = "dec_mma " + (names[nmma % 4] if nmma < 4 * wl.model.n_layers else "head + final LN")
                 nmma += 1
+            elif "argmax" in k:
+                k = "argmax + next embedding + step advance"
             if k not in agg:
                 agg[k] = [0, 0.0]
                 order.append(k)

@@ -486,9 +486,14 @@ cudaError_t launch_dec_attn(const T* qkv, T* kc, T* vc, T* out, float* part, uns
 }
 
 // Greedy choice: argmax over the real vocabulary of fp32 logits, lowest
-// index on ties.  Writes tok[b] and out[b * out_ld + col].
+// index on ties.  Writes tok[b] and out[b * out_ld + col].  With nx.x (a
+// replayed greedy step) the CTA also embeds its row's chosen token at the
+// next position into x (with its LayerNorm group statistics), and the last
+// CTA to finish (an arrival counter it resets) advances the step counter: the
+// embedding and step-advance kernels of the step fold into this one.
+template <typename T>
 __global__ void argmax_kernel(const float* __restrict__ logits, int V, int Vp, int* tok, int32_t* out,
-                              int out_ld, const int* __restrict__ step) {
+                              int out_ld, const int* __restrict__ step, GreedyNext<T> nx) {
   griddep_wait();
   griddep_release();
   int b = blockIdx.x;
@@ -544,14 +549,59 @@ __global__ void argmax_kernel(const float* __restrict__ logits, int V, int Vp, i
       if (bi < 0 || bi >= V) bi = 0;   // all-NaN row: fall back to id 0
       tok[b] = bi;
       out[(long)b * out_ld + col] = bi;
+      si[0] = bi;
+    }
+  }
+  if (!nx.x) return;
+  __syncthreads();
+  const int t = si[0];
+  // the next step's input row: token t at position pos0 + col + 1 (the last
+  // replay embeds a position nobody reads; it is clamped, not flagged)
+  int pos = nx.pos0 + col + 1;
+  pos = pos < 0 ? 0 : pos >= nx.max_seq ? nx.max_seq - 1 : pos;
+  const float* a = nx.wte + (long)t * nx.C;
+  const float* p = nx.wpe ? nx.wpe + (long)pos * nx.C : nullptr;
+  for (int c0 = 0; c0 < nx.C; c0 += blockDim.x) {
+    const int c = c0 + threadIdx.x;
+    const bool ok = c < nx.C;
+    float v = 0.f;
+    if (ok) {
+      const T w = from_f<T>(a[c] + (p ? p[c] : 0.f));
+      nx.x[(long)b * nx.C + c] = w;
+      v = to_f(w);
+    }
+    if (nx.st) {
+      float sm = v;
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
+      const float mean = sm * (1.f / 16.f), d = ok ? v - mean : 0.f;
+      float q = d * d;
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+      if (ok && (threadIdx.x & 15) == 0) nx.st[(long)(c / 16) * gridDim.x + b] = make_float2(mean, q);
+    }
+  }
+  // every CTA read the step counter at its start: the last one advances it
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(nx.cnt, 1u) == gridDim.x - 1) {
+      *nx.step += 1;
+      *nx.cnt = 0;
     }
   }
 }
 
+template <typename T>
 cudaError_t launch_argmax(const float* logits, int B, int V, int Vp, int* tok, int32_t* out, int out_ld,
-                          const int* step, cudaStream_t s) {
+                          const int* step, cudaStream_t s, const GreedyNext<T>* nx) {
+  GreedyNext<T> n{};
+  if (nx) {
+    if (!nx->x || !nx->wte || !nx->cnt || !nx->step || nx->step != step || (nx->st && nx->C % 16))
+      return cudaErrorInvalidValue;
+    n = *nx;
+  }
   ++g_kernel_launches;
-  cudaError_t e = launch_k(argmax_kernel, dim3(B), dim3(1024), 0, s, logits, V, Vp, tok, out, out_ld, step);
+  cudaError_t e = launch_k(argmax_kernel<T>, dim3(B), dim3(1024), 0, s, logits, V, Vp, tok, out, out_ld, step, n);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -830,6 +880,8 @@ cudaError_t launch_gather_last(const T* x, int B, int Tp, int C, T* out, cudaStr
 }
 
 #define INSTD(T)                                                                                         \
+  template cudaError_t launch_argmax<T>(const float*, int, int, int, int*, int32_t*, int, const int*,     \
+                                        cudaStream_t, const GreedyNext<T>*);                             \
   template cudaError_t launch_dec_embed<T>(const int*, const float*, const float*, T*, int, int, int,      \
                                            const int*, int, unsigned*, cudaStream_t, float2*);           \
   template cudaError_t launch_gemv<T>(const T*, int, int, const T*, int, const float*, const T*, int, T*, T*, \

@@ -986,9 +986,13 @@ static int decode_step(gpt_model* m, int B, int Tp, int n_new, int32_t* out, cud
   const bool mma = sizeof(T) == 2;
   const float2* st_o = mma && dec_mma_supported(B, C, C) ? st : nullptr;    // after the output projection
   const float2* st_f2 = mma && dec_mma_supported(B, F, C) ? st : nullptr;   // after fc2
-  // the token fed at step st sits at position Tp - 1 + st
-  CK(launch_dec_embed<T>(m->dtok, A.P(m->o_wte), ll ? nullptr : A.P(m->o_wpe), x, B, C, Tp - 1, stepc, m->Tmax,
-                         &m->sc->err, s, st));
+  // the token fed at step st sits at position Tp - 1 + st; a greedy step's
+  // input row was embedded by the previous step's argmax (the first one by
+  // decode_impl)
+  const bool greedy = !m->beam_w && !m->smp_on;
+  if (!greedy)
+    CK(launch_dec_embed<T>(m->dtok, A.P(m->o_wte), ll ? nullptr : A.P(m->o_wpe), x, B, C, Tp - 1, stepc, m->Tmax,
+                           &m->sc->err, s, st));
   for (int l = 0; l < m->NL; ++l) {
     const LayerOff& lo = m->L[l];
     CK(dec_ln_proj<T>(m, x, A.P(lo.ln1_g), P0(lo.ln1_b), h, B, C, A.W(lo.w_qkv), QW, P0(lo.b_qkv), nullptr, 0, q,
@@ -1017,9 +1021,21 @@ static int decode_step(gpt_model* m, int B, int Tp, int n_new, int32_t* out, cud
   } else if (m->smp_on)
     CK(launch_sample(m->dlogits, B, m->V, m->Vp, m->smp_temp, m->smp_topk, m->smp_topp, m->smp_u, n_new, m->dtok, out,
                      n_new, stepc, s));
-  else
-    CK(launch_argmax(m->dlogits, B, m->V, m->Vp, m->dtok, out, n_new, stepc, s));
-  CK(launch_step_advance(stepc, s));
+  else {
+    // the choice, the next input row and the step advance in one kernel
+    GreedyNext<T> nx;
+    nx.wte = A.P(m->o_wte);
+    nx.wpe = ll ? nullptr : A.P(m->o_wpe);
+    nx.x = x;
+    nx.C = C;
+    nx.pos0 = Tp - 1;
+    nx.max_seq = m->Tmax;
+    nx.st = st;
+    nx.cnt = &m->sc->dec_cnt;
+    nx.step = stepc;
+    CK(launch_argmax<T>(m->dlogits, B, m->V, m->Vp, m->dtok, out, n_new, stepc, s, &nx));
+  }
+  if (!greedy) CK(launch_step_advance(stepc, s));
   return GPT_OK;
 }
 
@@ -1054,6 +1070,11 @@ static int decode_impl(gpt_model* m, const int32_t* prompt, int B, int Tp, int n
   const int Bd = m->beam_w ? B * m->beam_w : B;   // decode rows
   const int one = 1;
   CK(cudaMemcpyAsync(&m->sc->dec_step, &one, sizeof(int), cudaMemcpyHostToDevice, s));
+  if (!m->beam_w && !m->smp_on) {
+    // the first replayed step's input row (later ones come from the step's argmax)
+    CK(launch_dec_embed<T>(m->dtok, A.P(m->o_wte), m->llama ? nullptr : A.P(m->o_wpe), (T*)m->dx, B, C, Tp - 1,
+                           &m->sc->dec_step, m->Tmax, &m->sc->err, s, C % 16 == 0 ? m->dxst : nullptr));
+  }
   // later tokens: one captured step (about 7 L + 5 kernels), replayed n_new - 1 times
   if (!m->cap_stream) CK(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking));
   if (!m->ev_a) {

@@ -25,6 +25,7 @@ struct DevScalars {
   int loss_scaling;   // 1: dynamic scale on
   unsigned err;       // sticky device error word
   int dec_step;       // decode step counter
+  unsigned dec_cnt;   // arrival counter of the greedy step's argmax CTAs (kept zero)
   unsigned long long attn_pairs;   // allowed (query, key) pairs of the latest packed forward
   float lr;           // learning rate of the latest taken step (set by the finalize kernel)
   float loss_weight;  // multiplies the loss gradient of later forwards (micro-batch weight)
@@ -187,9 +188,24 @@ template <typename T>
 // first launch (every launch leaves them zero)
 cudaError_t launch_dec_attn(const T* qkv, T* kc, T* vc, T* out, float* part, unsigned* cnt, int B, int H, int d,
                             int Tmax, int pos0, const int* step, const DecLayout& L, cudaStream_t s);
+// The next step's input of a replayed greedy step, made by the argmax kernel:
+// x[b] = T(wte[token] + wpe[pos0 + *step + 1]) (wpe may be null), with the
+// LayerNorm group statistics in st (optional, C % 16 == 0); the last CTA
+// advances *step (== the argmax's step) and resets cnt (zero before use).
+template <typename T>
+struct GreedyNext {
+  const float* wte = nullptr;
+  const float* wpe = nullptr;
+  T* x = nullptr;
+  int C = 0, pos0 = 0, max_seq = 0;
+  float2* st = nullptr;
+  unsigned* cnt = nullptr;
+  int* step = nullptr;
+};
 // out[b * out_ld + (*step or 0)] = argmax; tok[b] = argmax
+template <typename T = float>
 cudaError_t launch_argmax(const float* logits, int B, int V, int Vp, int* tok, int32_t* out, int out_ld,
-                          const int* step, cudaStream_t s);
+                          const int* step, cudaStream_t s, const GreedyNext<T>* nx = nullptr);
 cudaError_t launch_step_advance(int* step, cudaStream_t s);
 // sampled choice (temperature, top-k, top-p; temp <= 0: greedy) with the
 // uniform uni[b * u_ld + (*step or 0)]; writes tok[b] and out[b * out_ld + col].
