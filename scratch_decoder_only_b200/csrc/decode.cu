@@ -246,9 +246,10 @@ cudaError_t launch_kv_fill(const T* qkv, T* kc, T* vc, int B, int Tp, int d, int
 // o = softmax(q K^T / sqrt(D)) V over keys 0 .. pos of the (row, head).
 // Grid (B*H, S): the key range of a (row, head) is cut into act <= S
 // contiguous pieces (act grows with the context, one per 256 keys), one CTA
-// each; S is chosen so that about two CTAs per SM have work.  A CTA's four
-// warps take 4 * (32 / (D / 8)) * U consecutive keys per pass (128 for D = 64
-// in 16 bits), a lane group of D / 8 lanes per key and U keys per lane group
+// each; S is chosen so that about two CTAs per SM have work.  A CTA's NW
+// warps (8 while the (row, head) pairs do not fill the SMs, else 4) take
+// NW * (32 / (D / 8)) * U consecutive keys per pass (256 or 128 for D = 64 in
+// 16 bits), a lane group of D / 8 lanes per key and U keys per lane group
 // in flight (each lane one load of 8 values of a key and of a value row,
 // kept packed until used), with an online softmax (max, sum, output) per lane
 // group updated once per U keys.  The lane groups and warps
@@ -259,7 +260,6 @@ cudaError_t launch_kv_fill(const T* qkv, T* kc, T* vc, int B, int Tp, int d, int
 // cache by piece 0; the first pass's cached rows load before the
 // programmatic-dependent-launch wait, while the q / k / v projection runs.
 #define DA_SPLITS 16
-#define DA_THREADS 128
 template <typename T>
 __device__ __forceinline__ void load8(const T* p, float* v) {
 #pragma unroll
@@ -283,14 +283,13 @@ __device__ __forceinline__ void unpack8(const Pack8<T>& r, float* v) {
   load8(reinterpret_cast<const T*>(r.w), v);
 }
 
-template <typename T, int D>
-__global__ void __launch_bounds__(DA_THREADS)
+template <typename T, int D, int NW>
+__global__ void __launch_bounds__(NW * 32)
 dec_attn_kernel(const T* __restrict__ qkv, T* kc, T* vc, T* __restrict__ out, float* part, unsigned* cnt, int B,
                 int H, int Tmax, int pos0, const int* __restrict__ step, DecLayout Ly) {
   static_assert(D % 8 == 0 && D <= 256, "head size");
   constexpr int LPK = D / 8;            // lanes per key row (16 bytes each)
   constexpr int KPW = 32 / LPK;         // lane groups (keys) per warp
-  constexpr int NW = DA_THREADS / 32;
   constexpr int U = sizeof(T) == 2 ? 8 : 4;   // keys per lane group in flight
   constexpr int KPP = NW * KPW * U;           // keys per CTA pass
   int pos = pos0 + *step;
@@ -467,13 +466,20 @@ cudaError_t launch_dec_attn(const T* qkv, T* kc, T* vc, T* out, float* part, uns
   if (S > DA_SPLITS) S = DA_SPLITS;
   if (S < 1) S = 1;
   dim3 g(B * H, S);
+  // eight warps (one pass per 256-key piece at d = 64) while the (row, head)
+  // pairs do not fill the SMs, else four (more CTAs resident per SM)
+  const bool wide = B * H <= g_da_sms;
   cudaError_t e = cudaSuccess;
   switch (d) {
 #define DA_CASE(DD)                                                                                               \
   case DD:                                                                                                        \
     g_kernel_launches += 1;                                                                                       \
-    e = launch_k(dec_attn_kernel<T, DD>, g, dim3(DA_THREADS), 0, s, qkv, kc, vc, out, part, cnt, B, H, Tmax, pos0, \
-                 step, L);                                                                                        \
+    if (wide)                                                                                                     \
+      e = launch_k(dec_attn_kernel<T, DD, 8>, g, dim3(256), 0, s, qkv, kc, vc, out, part, cnt, B, H, Tmax, pos0, \
+                   step, L);                                                                                      \
+    else                                                                                                          \
+      e = launch_k(dec_attn_kernel<T, DD, 4>, g, dim3(128), 0, s, qkv, kc, vc, out, part, cnt, B, H, Tmax, pos0, \
+                   step, L);                                                                                      \
     break;
     DA_CASE(16)
     DA_CASE(32)
