@@ -357,7 +357,9 @@ struct FwdSmem {
 template <bool F16>
 __global__ void __launch_bounds__(FW_THREADS, 1)
 attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, float* __restrict__ lse,
-            const int* __restrict__ dstart, int T, int H, int kcol0, int vcol0, int G, unsigned* err) {
+            const int* __restrict__ dstart, int T, int H, int kcol0, int vcol0, int G, unsigned* err, float sl2) {
+  // sl2 = log2(e) / sqrt(d): the score scale in the exp2 domain (d = 64, or
+  // the true head size of heads zero-padded to 64 columns)
   extern __shared__ __align__(1024) uint8_t at_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)at_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = (uint64_t*)(sm + FwdSmem::BAR);
@@ -523,7 +525,6 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tmQKV, bf16* __restrict__ out, f
     const int ds_last = ld_once(dsr + qlast);
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t tO = tmem + lane_off + 64 * g;
-    const float sl2 = 0.125f * LOG2E_F;   // 1/sqrt(64) in the exp2 domain
     auto wait_w = [&](uint32_t bb, uint32_t parity) { return __all_sync(0xffffffffu, mbar_wait(bb, parity, abort_flag)); };
     // wait until P V of this tile's m-th block has completed.  Called for m
     // in increasing order, each m at a point where P V of block m - 2 has been
@@ -733,7 +734,9 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
 attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
             const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ lse, const float* __restrict__ Dbuf,
             const int* __restrict__ dstart, int T, int H, int BH, int kcol0, int vcol0, int G, bf16* __restrict__ dkv,
-            long ld_kv, int v_off, unsigned* err) {
+            long ld_kv, int v_off, unsigned* err, float sl2) {
+  // sl2 = log2(e) / sqrt(d) as in the forward; dK carries the 1 / sqrt(d) factor
+  const float dk_scale = sl2 * (1.0f / LOG2E_F);
   extern __shared__ __align__(1024) uint8_t at_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)at_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = (uint64_t*)(sm + BwdSmem::BAR);
@@ -968,7 +971,6 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
     const int grp = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const float sl2 = 0.125f * LOG2E_F;
     const uint32_t st_full = bar(ST_FULL + grp), st_free = bar(ST_FREE + grp);
     const uint32_t sDQg = sDQ + grp * AT_TILE_BYTES;
     bool ok = true;
@@ -1068,7 +1070,7 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
       bf16* row = dkv + (I.rowbase + k) * ld_kv;
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
-        const float sc = part == 0 ? 0.125f : 1.f;
+        const float sc = part == 0 ? dk_scale : 1.f;
         uint32_t rr[32];
         tmem_ld32(tmem + lane_off + (part == 0 ? 320 : 256) + 32 * grp, rr);
         tmem_wait_ld();
@@ -1120,9 +1122,10 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
   if (warp == 0) tc_dealloc(tmem, BwdSmem::TMEM_COLS);
 }
 
-// dq[row, head h] = bf16 or fp16 (F16) of dQacc / 8; the accumulator is cleared for the next use.
+// dq[row, head h] = bf16 or fp16 (F16) of dQacc / sqrt(d); the accumulator is cleared for the next use.
 template <bool F16>
-__global__ void attn_dq_finish_kernel(float* __restrict__ dq_acc, bf16* __restrict__ dqkv, long rows, int C, long ld_q) {
+__global__ void attn_dq_finish_kernel(float* __restrict__ dq_acc, bf16* __restrict__ dqkv, long rows, int C, long ld_q,
+                                      float scale) {
   griddep_wait();
   griddep_release();
   const long n8 = rows * C / 8;
@@ -1132,10 +1135,10 @@ __global__ void attn_dq_finish_kernel(float* __restrict__ dq_acc, bf16* __restri
     float4* src = reinterpret_cast<float4*>(dq_acc + e);
     const float4 a = src[0], bq = src[1];
     uint4 w;
-    w.x = pack16x2<F16>(a.x * 0.125f, a.y * 0.125f);
-    w.y = pack16x2<F16>(a.z * 0.125f, a.w * 0.125f);
-    w.z = pack16x2<F16>(bq.x * 0.125f, bq.y * 0.125f);
-    w.w = pack16x2<F16>(bq.z * 0.125f, bq.w * 0.125f);
+    w.x = pack16x2<F16>(a.x * scale, a.y * scale);
+    w.y = pack16x2<F16>(a.z * scale, a.w * scale);
+    w.z = pack16x2<F16>(bq.x * scale, bq.y * scale);
+    w.w = pack16x2<F16>(bq.z * scale, bq.w * scale);
     *reinterpret_cast<uint4*>(dqkv + row * ld_q + c) = w;
     src[0] = make_float4(0.f, 0.f, 0.f, 0.f);
     src[1] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1145,16 +1148,17 @@ __global__ void attn_dq_finish_kernel(float* __restrict__ dq_acc, bf16* __restri
 // D[b, h, t] = dO[b*T+t, head h] . O[b*T+t, head h]   (one thread per (row, head))
 template <bool F16>
 __global__ void attn_rowdot_kernel(const bf16* __restrict__ out, const bf16* __restrict__ dout, float* __restrict__ Dbuf,
-                                   int B, int T, int H) {
+                                   int B, int T, int H, int d) {
+  griddep_wait();
+  griddep_release();
   long i = blockIdx.x * (long)blockDim.x + threadIdx.x;
   if (i >= (long)B * T * H) return;
   const int h = i % H;
   const long row = i / H;
   const int t = row % T, b = row / T;
-  const long off = row * H * AT_D + h * AT_D;
+  const long off = row * H * d + h * d;
   float acc = 0.f;
-#pragma unroll
-  for (int c = 0; c < AT_D; c += 8) {
+  for (int c = 0; c < d; c += 8) {
     float x[8], y[8];
     unpack16x8<F16>(*reinterpret_cast<const uint4*>(dout + off + c), x);
     unpack16x8<F16>(*reinterpret_cast<const uint4*>(out + off + c), y);
@@ -1181,7 +1185,7 @@ AttnLayout attn_layout_mha(bf16* dqkv, int C) {
 
 template <bool F16>
 static cudaError_t attn_fwd_tc_t(const bf16* qkv, bf16* out, float* lse, const int* dstart, int B, int T, int H,
-                                 unsigned* err, cudaStream_t s, const AttnLayout& L) {
+                                 unsigned* err, cudaStream_t s, const AttnLayout& L, int d_real) {
   const long rows = (long)B * T;
   CUtensorMap tqkv;
   if (!make_map_ex(&tqkv, MapKey{qkv, rows, (long)L.qw, (long)L.qw, 1, 0, AT_D, AT_BLK, 0, 128}))
@@ -1192,7 +1196,7 @@ static cudaError_t attn_fwd_tc_t(const bf16* qkv, bf16* out, float* lse, const i
   dim3 grid(B * H, (T + FW_QT - 1) / FW_QT);
   ++g_kernel_launches;
   return launch_k(attn_fwd_tc<F16>, grid, dim3(FW_THREADS), smem, s, tqkv, out, lse, dstart, T, H, L.kcol, L.vcol, L.G,
-                  err);
+                  err, LOG2E_F / sqrtf((float)d_real));
 }
 
 static bool layout_ok(const AttnLayout& L, int H) {
@@ -1202,18 +1206,19 @@ static bool layout_ok(const AttnLayout& L, int H) {
 }
 
 cudaError_t launch_attn_fwd_tc(const bf16* qkv, bf16* out, float* lse, const int* dstart, int B, int T, int H,
-                               unsigned* err, cudaStream_t s, bool f16, const AttnLayout* lay) {
+                               unsigned* err, cudaStream_t s, bool f16, const AttnLayout* lay, int d_real) {
   const AttnLayout L = lay ? *lay : attn_layout_mha(nullptr, H * AT_D);
-  if (!layout_ok(L, H)) return cudaErrorInvalidValue;
-  return f16 ? attn_fwd_tc_t<true>(qkv, out, lse, dstart, B, T, H, err, s, L)
-             : attn_fwd_tc_t<false>(qkv, out, lse, dstart, B, T, H, err, s, L);
+  if (!layout_ok(L, H) || d_real < 1 || d_real > AT_D) return cudaErrorInvalidValue;
+  return f16 ? attn_fwd_tc_t<true>(qkv, out, lse, dstart, B, T, H, err, s, L, d_real)
+             : attn_fwd_tc_t<false>(qkv, out, lse, dstart, B, T, H, err, s, L, d_real);
 }
 
 template <bool F16>
 static cudaError_t attn_bwd_tc_t(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* Dbuf,
                                  bool d_ready, float* dq_acc, const int* dstart, bf16* dqkv, int B, int T, int H,
-                                 unsigned* err, cudaStream_t s, const AttnLayout& L) {
+                                 unsigned* err, cudaStream_t s, const AttnLayout& L, int d_real) {
   const int C = H * AT_D;
+  const float scale = 1.0f / sqrtf((float)d_real);
   const long rows = (long)B * T;
   CUtensorMap tqkv, tdo, tdq;
   if (!make_map_ex(&tqkv, MapKey{qkv, rows, (long)L.qw, (long)L.qw, 1, 0, AT_D, AT_BLK, 0, 128}) ||
@@ -1231,7 +1236,7 @@ static cudaError_t attn_bwd_tc_t(const bf16* qkv, const bf16* out, const bf16* d
   if (!d_ready) {   // D = rowsum(dO o O), unless the producer of dO already wrote it
     long n = rows * H;
     ++g_kernel_launches;
-    attn_rowdot_kernel<F16><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(out, dout, Dbuf, B, T, H);
+    attn_rowdot_kernel<F16><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(out, dout, Dbuf, B, T, H, AT_D);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   // persistent: one CTA per SM (or fewer, for fewer items)
@@ -1246,17 +1251,65 @@ static cudaError_t attn_bwd_tc_t(const bf16* qkv, const bf16* out, const bf16* d
   if (n_items > (long)grid * BW_MAX_ITEMS) return cudaErrorInvalidValue;
   ++g_kernel_launches;
   e = launch_k(attn_bwd_tc<F16>, dim3(grid), dim3(BW_THREADS), smem, s, tqkv, tdo, tdq, lse, Dbuf, dstart, T, H, B * H,
-               L.kcol, L.vcol, L.G, L.dkv, L.ld_kv, L.v_off, err);
+               L.kcol, L.vcol, L.G, L.dkv, L.ld_kv, L.v_off, err, scale * LOG2E_F);
   if (e != cudaSuccess) return e;
   ++g_kernel_launches;
-  return launch_k(attn_dq_finish_kernel<F16>, dim3(148 * 8), dim3(256), 0, s, dq_acc, dqkv, rows, C, (long)L.qw);
+  return launch_k(attn_dq_finish_kernel<F16>, dim3(148 * 8), dim3(256), 0, s, dq_acc, dqkv, rows, C, (long)L.qw, scale);
 }
 
 cudaError_t launch_attn_bwd_tc(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* Dbuf,
                                bool d_ready, float* dq_acc, const int* dstart, bf16* dqkv, int B, int T, int H,
-                               unsigned* err, cudaStream_t s, bool f16, const AttnLayout* lay) {
+                               unsigned* err, cudaStream_t s, bool f16, const AttnLayout* lay, int d_real) {
   const AttnLayout L = lay ? *lay : attn_layout_mha(dqkv, H * AT_D);
-  if (!layout_ok(L, H) || !L.dkv) return cudaErrorInvalidValue;
-  return f16 ? attn_bwd_tc_t<true>(qkv, out, dout, lse, Dbuf, d_ready, dq_acc, dstart, dqkv, B, T, H, err, s, L)
-             : attn_bwd_tc_t<false>(qkv, out, dout, lse, Dbuf, d_ready, dq_acc, dstart, dqkv, B, T, H, err, s, L);
+  if (!layout_ok(L, H) || !L.dkv || d_real < 1 || d_real > AT_D) return cudaErrorInvalidValue;
+  return f16 ? attn_bwd_tc_t<true>(qkv, out, dout, lse, Dbuf, d_ready, dq_acc, dstart, dqkv, B, T, H, err, s, L, d_real)
+             : attn_bwd_tc_t<false>(qkv, out, dout, lse, Dbuf, d_ready, dq_acc, dstart, dqkv, B, T, H, err, s, L, d_real);
+}
+
+// ------------------------------------------------------------ zero-padded heads
+// Heads of d < 64 columns (64 % d == 0) run the d = 64 kernels on copies whose
+// heads are widened to 64 columns with zeros: a zero column adds nothing to a
+// score, a zero value column gives a zero output column, and the padded
+// gradient columns are dropped.  attn_pad: dst [rows][groups][64] <- src
+// [rows][groups][d] (zeros beyond d); attn_unpad: the reverse copy.
+template <bool PAD>
+__global__ void attn_pad_kernel(const bf16* __restrict__ src, bf16* __restrict__ dst, long rows, int groups, int d) {
+  griddep_wait();
+  griddep_release();
+  const int cpg = AT_D / 8;   // 16-byte chunks per padded group
+  const long n = rows * groups * cpg;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
+    const long rg = i / cpg;
+    const int c = (int)(i % cpg) * 8;
+    const long row = rg / groups;
+    const int g = (int)(rg % groups);
+    const long p = (row * groups + g) * AT_D + c, u = (row * groups + g) * d + c;
+    if (PAD) {
+      *reinterpret_cast<uint4*>(dst + p) = c < d ? *reinterpret_cast<const uint4*>(src + u) : make_uint4(0u, 0u, 0u, 0u);
+    } else if (c < d) {
+      *reinterpret_cast<uint4*>(dst + u) = *reinterpret_cast<const uint4*>(src + p);
+    }
+  }
+}
+
+cudaError_t launch_attn_rowdot(const bf16* out, const bf16* dout, float* Dbuf, int B, int T, int H, int d, bool f16,
+                               cudaStream_t s) {
+  if (d % 8) return cudaErrorInvalidValue;
+  const long n = (long)B * T * H;
+  ++g_kernel_launches;
+  return f16 ? launch_k(attn_rowdot_kernel<true>, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, out, dout, Dbuf, B,
+                        T, H, d)
+             : launch_k(attn_rowdot_kernel<false>, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, out, dout, Dbuf,
+                        B, T, H, d);
+}
+
+bool attn_tc_pad_supported(int d) { return d >= 8 && d < AT_D && AT_D % d == 0 && get_encode() != nullptr; }
+
+cudaError_t launch_attn_pad(const bf16* src, bf16* dst, long rows, int groups, int d, bool pad, cudaStream_t s) {
+  if (!attn_tc_pad_supported(d)) return cudaErrorInvalidValue;
+  const long n = rows * groups * (AT_D / 8);
+  const int blocks = (int)std::min<long>((n + 255) / 256, 148L * 8);
+  ++g_kernel_launches;
+  return pad ? launch_k(attn_pad_kernel<true>, dim3(blocks), dim3(256), 0, s, src, dst, rows, groups, d)
+             : launch_k(attn_pad_kernel<false>, dim3(blocks), dim3(256), 0, s, src, dst, rows, groups, d);
 }

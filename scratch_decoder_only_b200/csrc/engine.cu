@@ -53,6 +53,10 @@ struct gpt_model {
   float* dres32;
   void *dres_t, *dC, *dF, *dqkv;
   float *attD, *rowloss, *partials, *dq_acc;
+  // heads of d < 64 on the tensor-core attention: q|k|v, O / dO and the
+  // q|k|v gradient with every head zero-padded to 64 columns (16-bit)
+  void *apad = nullptr, *opad = nullptr, *dqkvpad = nullptr;
+  size_t dq_acc_n = 0;
   size_t partials_n;
   double* normpart;
   int normblk = 592;
@@ -351,7 +355,14 @@ static int build_arena(gpt_model* m) {
   }
   cv.add(&m->dqkv, Mx * 3 * C * es);
   cv.add((void**)&m->attD, Mx * m->H * 4);
-  cv.add((void**)&m->dq_acc, m->lp ? Mx * C * 4 : 4);
+  const bool pad_heads = m->lp && !m->llama && !attn_tc_supported(m->d) && attn_tc_pad_supported(m->d);
+  m->dq_acc_n = m->lp ? Mx * (size_t)(pad_heads ? m->H * 64 : C) : 1;
+  cv.add((void**)&m->dq_acc, m->dq_acc_n * 4);
+  if (pad_heads) {
+    cv.add(&m->apad, NL * Mx * 3 * m->H * 64 * es);   // per layer
+    cv.add(&m->opad, Mx * m->H * 64 * es);
+    cv.add(&m->dqkvpad, Mx * 3 * m->H * 64 * es);
+  }
   cv.add((void**)&m->rowloss, Mx * 4);
   {
     // partial rows of every deferred column reduction of one backward pass:
@@ -395,6 +406,8 @@ static int build_arena(gpt_model* m) {
   }
   for (auto& it : cv.items) *it.first = m->arena + it.second;
   e = cudaMemset(m->dacnt, 0, Bx * m->H * 4);
+  // the attention backward adds into dq_acc, and its finishing kernel clears it after each use
+  if (e == cudaSuccess) e = cudaMemset(m->dq_acc, 0, m->dq_acc_n * 4);
   if (e != cudaSuccess) { m->err = std::string("cudaMemset: ") + cudaGetErrorString(e); return GPT_ERR_CUDA; }
   if (!m->lp) m->pw = m->p32;
   return GPT_OK;
@@ -516,17 +529,27 @@ static int gemm(gpt_model* m, int M, int N, int K, const f16* A, long lda, bool 
 static double attn_pairs(int B, int T, int H, bool seg) { return seg ? 0.0 : (double)B * H * T * (T + 1) / 2.0; }
 static double attn_pair_mult(const gpt_model* m, double per_pair) { return m->seg_used ? per_pair * m->H : 0.0; }
 
-static int attn_fwd(gpt_model* m, const float* qkv, float* out, float* lse, int B, int T) {
+static int attn_fwd(gpt_model* m, const float* qkv, float* out, float* lse, int B, int T,
+                    const AttnLayout* = nullptr, int = 0) {
   ProfScope ps(m, PC_ATTN_FWD, 4.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0, attn_pair_mult(m, 4.0 * m->d));
   CK(launch_attn_fwd_simt<float>(qkv, out, lse, m->dstart, B, T, m->H, m->d, m->stream));
   return GPT_OK;
 }
 template <typename T16>
-static int attn_fwd(gpt_model* m, const T16* qkv, T16* out, float* lse, int B, int T, const AttnLayout* lay = nullptr) {
+static int attn_fwd(gpt_model* m, const T16* qkv, T16* out, float* lse, int B, int T, const AttnLayout* lay = nullptr,
+                    int layer = 0) {
   ProfScope ps(m, PC_ATTN_FWD, 4.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0, attn_pair_mult(m, 4.0 * m->d));
   constexpr bool F16 = std::is_same<T16, f16>::value;
   if (lay && !attn_tc_supported(m->d)) FAIL(GPT_ERR_ARG, "grouped key/value heads need the tensor-core attention");
-  if (attn_tc_supported(m->d))
+  if (!lay && m->apad) {
+    // heads of d < 64: the d = 64 tensor-core kernel on zero-padded copies
+    // (the layer's padded q|k|v stays for its backward)
+    const long rows = (long)B * T;
+    bf16 *qp = (bf16*)m->apad + (size_t)layer * m->Mmax * 3 * m->H * 64, *op = (bf16*)m->opad;
+    CK(launch_attn_pad(reinterpret_cast<const bf16*>(qkv), qp, rows, 3 * m->H, m->d, true, m->stream));
+    CK(launch_attn_fwd_tc(qp, op, lse, m->dstart, B, T, m->H, &m->sc->err, m->stream, F16, nullptr, m->d));
+    CK(launch_attn_pad(op, reinterpret_cast<bf16*>(out), rows, m->H, m->d, false, m->stream));
+  } else if (attn_tc_supported(m->d))
     CK(launch_attn_fwd_tc(reinterpret_cast<const bf16*>(qkv), reinterpret_cast<bf16*>(out), lse, m->dstart, B, T,
                           m->H, &m->sc->err, m->stream, F16, lay));
   else if (!F16 && attn_mma_supported(m->d))
@@ -536,7 +559,7 @@ static int attn_fwd(gpt_model* m, const T16* qkv, T16* out, float* lse, int B, i
   return GPT_OK;
 }
 static int attn_bwd(gpt_model* m, const float* qkv, const float* out, const float* dout, const float* lse,
-                    float* dqkv, int B, int T, bool) {
+                    float* dqkv, int B, int T, bool, const AttnLayout* = nullptr, int = 0) {
   ProfScope ps(m, PC_ATTN_BWD, 8.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0, attn_pair_mult(m, 8.0 * m->d));
   CK(launch_attn_bwd_simt<float>(qkv, out, dout, lse, m->attD, m->dstart, dqkv, B, T, m->H, m->d, m->stream));
   return GPT_OK;
@@ -544,12 +567,25 @@ static int attn_bwd(gpt_model* m, const float* qkv, const float* out, const floa
 // d_ready: m->attD already holds D = rowsum(dO o O) (tensor-core path only)
 template <typename T16>
 static int attn_bwd(gpt_model* m, const T16* qkv, const T16* out, const T16* dout, const float* lse,
-                    T16* dqkv, int B, int T, bool d_ready, const AttnLayout* lay = nullptr) {
+                    T16* dqkv, int B, int T, bool d_ready, const AttnLayout* lay = nullptr, int layer = 0) {
   ProfScope ps(m, PC_ATTN_BWD, 8.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0, attn_pair_mult(m, 8.0 * m->d));
   constexpr bool F16 = std::is_same<T16, f16>::value;
   auto cb = [](const T16* p) { return reinterpret_cast<const bf16*>(p); };
   if (lay && !attn_tc_supported(m->d)) FAIL(GPT_ERR_ARG, "grouped key/value heads need the tensor-core attention");
-  if (attn_tc_supported(m->d))
+  if (!lay && m->apad) {
+    // heads of d < 64 on the zero-padded copies (the forward took the same
+    // path: its base-2 logsumexp is in this scale); D = rowsum(dO o O) is the
+    // same over the padded columns, which add nothing
+    const long rows = (long)B * T;
+    // the layer's q|k|v as its forward padded them
+    const bf16* qp = (const bf16*)m->apad + (size_t)layer * m->Mmax * 3 * m->H * 64;
+    bf16 *dop = (bf16*)m->opad, *gp = (bf16*)m->dqkvpad;
+    if (!d_ready) CK(launch_attn_rowdot(cb(out), cb(dout), m->attD, B, T, m->H, m->d, F16, m->stream));
+    CK(launch_attn_pad(cb(dout), dop, rows, m->H, m->d, true, m->stream));
+    CK(launch_attn_bwd_tc(qp, nullptr, dop, lse, m->attD, true, m->dq_acc, m->dstart, gp, B, T, m->H, &m->sc->err,
+                          m->stream, F16, nullptr, m->d));
+    CK(launch_attn_pad(gp, reinterpret_cast<bf16*>(dqkv), rows, 3 * m->H, m->d, false, m->stream));
+  } else if (attn_tc_supported(m->d))
     CK(launch_attn_bwd_tc(cb(qkv), cb(out), cb(dout), lse, m->attD, d_ready, m->dq_acc, m->dstart,
                           reinterpret_cast<bf16*>(dqkv), B, T, m->H, &m->sc->err, m->stream, F16, lay));
   else if (!F16 && attn_mma_supported(m->d))
@@ -615,7 +651,7 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
       CK(launch_ln_fwd<T>(A.x(l), A.P(lo.ln1_g), A.P(lo.ln1_b), A.h1(l), A.mu1(l), A.rs1(l), M, C, eps, s)); }
     CKI(gemm(m, M, 3 * C, C, A.h1(l), C, false, A.W(lo.w_qkv), C, false,
              epi_store<T>(A.qkv(l), 3 * C, A.P(lo.b_qkv), nullptr, 0)));
-    CKI(attn_fwd(m, A.qkv(l), A.att(l), A.lse(l), B, T_));
+    CKI(attn_fwd(m, A.qkv(l), A.att(l), A.lse(l), B, T_, nullptr, l));
     CKI(gemm(m, M, C, C, A.att(l), C, false, A.W(lo.w_o), C, false,
              epi_store<T>(A.xmid(l), C, A.P(lo.b_o), A.x(l), C)));
     { ProfScope ps(m, PC_LN_FWD, 0, lnb);
@@ -717,13 +753,14 @@ static int backward_impl(gpt_model* m) {
     CKI(gemm(m, C, C, M, drt, C, true, A.att(l), C, true, epi_f32<T>(A.G(lo.w_o), C)));
     // dO = d(attention output); on the tensor-core path its GEMM epilogue also
     // takes D = rowsum(dO o O) per row and head for the attention backward
+    // (the row-dot epilogue sums 64-column heads: d = 64 only)
     const bool fuse_d = sizeof(T) == 2 && attn_tc_supported(m->d) && gemm_tc_supported(M, C, C, C, false, C, true);
     {
       EpiParams<T> e = epi_store<T>(dC, C, nullptr, nullptr, 0);
       if (fuse_d) { e.aux = A.att(l); e.ld_aux = C; e.rowdot = m->attD; e.rd_T = T_; }
       CKI(gemm(m, M, C, C, drt, C, false, A.W(lo.w_o), C, true, e));
     }
-    CKI(attn_bwd(m, A.qkv(l), A.att(l), dC, A.lse(l), dq, B, T_, fuse_d));
+    CKI(attn_bwd(m, A.qkv(l), A.att(l), dC, A.lse(l), dq, B, T_, fuse_d, nullptr, l));
     {
       float* qpart = take((size_t)((M + 127) / 128) * 3 * C);
       if (!qpart) FAIL(GPT_ERR_NOMEM, "partials arena too small");

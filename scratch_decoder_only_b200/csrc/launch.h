@@ -150,13 +150,24 @@ AttnLayout attn_layout_mha(bf16* dqkv, int C);
 // lse of the tcgen05 pair is the base-2 log-sum-exp of the scaled scores
 // (log2e / sqrt(d) units), the form its backward consumes; the SIMT and
 // mma.sync pairs keep the natural log.
+// d_real: the true head size of heads zero-padded to 64 columns (64: none)
 cudaError_t launch_attn_fwd_tc(const bf16* qkv, bf16* out, float* lse, const int* dstart, int B, int T, int H,
-                               unsigned* err, cudaStream_t s, bool f16 = false, const AttnLayout* lay = nullptr);
+                               unsigned* err, cudaStream_t s, bool f16 = false, const AttnLayout* lay = nullptr,
+                               int d_real = 64);
 // d_ready: Dbuf [B, H, T] already holds rowsum(dO o O) (written by the GEMM
 // epilogue that produced dO); otherwise a row-dot kernel computes it first
 cudaError_t launch_attn_bwd_tc(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* Dbuf,
                                bool d_ready, float* dq_acc, const int* dstart, bf16* dqkv, int B, int T, int H,
-                               unsigned* err, cudaStream_t s, bool f16 = false, const AttnLayout* lay = nullptr);
+                               unsigned* err, cudaStream_t s, bool f16 = false, const AttnLayout* lay = nullptr,
+                               int d_real = 64);
+// heads of d < 64 columns (64 % d == 0) on the d = 64 tensor-core kernels:
+// copies with every head widened to 64 columns by zeros (pad: src [rows]
+// [groups][d] -> dst [rows][groups][64]; !pad: back, the extra columns dropped)
+bool attn_tc_pad_supported(int d);
+// D[b, h, t] = dO . O over head h's d columns of row b T + t ([rows][H][d])
+cudaError_t launch_attn_rowdot(const bf16* out, const bf16* dout, float* Dbuf, int B, int T, int H, int d, bool f16,
+                               cudaStream_t s);
+cudaError_t launch_attn_pad(const bf16* src, bf16* dst, long rows, int groups, int d, bool pad, cudaStream_t s);
 
 // ---- decode.cu
 // decode kernels read the position as pos0 + *step (device counter)
