@@ -714,7 +714,7 @@ static int backward_impl(gpt_model* m) {
     float* part = take((size_t)444 * 3 * C);
     if (!part) FAIL(GPT_ERR_NOMEM, "partials arena too small");
     ProfScope ps(m, PC_LN_BWD, 0, lnbb);
-    CK(launch_ln_bwd<T>(dC, x, mu, rs, g, din, m->dres32, drt, part, M, C, &nblk, s));
+    CK(launch_ln_bwd<T>(dC, x, mu, rs, g, din, m->dres32, drt, part, M, C, &nblk, s, false, &m->sc->err));
     seg(part, gdst, nblk, 2 * C, 3 * C);
     if (bias_dst) seg(part + 2 * C, bias_dst, nblk, C, 3 * C);
     return GPT_OK;
@@ -894,7 +894,7 @@ static int backward_llama(gpt_model* m) {
     float* part = take((size_t)444 * 3 * C);
     if (!part) FAIL(GPT_ERR_NOMEM, "partials arena too small");
     ProfScope ps(m, PC_LN_BWD, 0, lnbb);
-    CK(launch_ln_bwd<T>(dC, x, mu, rs, g, din, m->dres32, drt, part, M, C, &nblk, s, true));
+    CK(launch_ln_bwd<T>(dC, x, mu, rs, g, din, m->dres32, drt, part, M, C, &nblk, s, true, &m->sc->err));
     segs.push_back({part, gdst, nblk, C, 3 * C, 0});
     return GPT_OK;
   };

@@ -3,6 +3,7 @@
 // cross-entropy with its logits gradient, deterministic row reductions,
 // global-norm clip and AdamW.  All are HBM-bound: 16-byte vector loads, one
 // warp per row where a row is reduced, no fp32 copies of bf16 tensors.
+#include <algorithm>
 #include "launch.h"
 #include "tc_common.cuh"
 
@@ -220,6 +221,7 @@ __global__ void __launch_bounds__(256, (NCH * Vec<T>::N <= 24 ? 4 : 2)) ln_fwd_k
   griddep_release();
   const int lane = threadIdx.x & 31;
   const int nch = C / NV;
+  const float inv_c = 1.0f / C;
   const int stride = gridDim.x * (blockDim.x >> 5);
   int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   uint4 nxt[NCH];
@@ -241,22 +243,25 @@ __global__ void __launch_bounds__(256, (NCH * Vec<T>::N <= 24 ? 4 : 2)) ln_fwd_k
         for (int j = 0; j < NV; ++j) v[i][j] = 0.f;
     }
     fetch(row + stride);
-    float sum = 0.f;
+    // two interleaved partial sums per lane halve the dependent-add chains;
+    // the row normalises as x * rs + (-mu * rs), then gamma and beta by one FMA
+    float sum2[2] = {0.f, 0.f};
 #pragma unroll
     for (int i = 0; i < NCH; ++i)
 #pragma unroll
-      for (int j = 0; j < NV; ++j) sum += v[i][j];
+      for (int j = 0; j < NV; ++j) sum2[j & 1] += v[i][j];
     const bool rms = b == nullptr;   // RMSNorm: no mean, no shift
-    const float mu = rms ? 0.f : warp_sum(sum) / C;
-    float sq = 0.f;
+    const float mu = rms ? 0.f : warp_sum(sum2[0] + sum2[1]) * inv_c;
+    float sq2[2] = {0.f, 0.f};
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
       if (lane + i * 32 < nch) {
 #pragma unroll
-        for (int j = 0; j < NV; ++j) { const float d = v[i][j] - mu; sq += d * d; }
+        for (int j = 0; j < NV; ++j) { const float d = v[i][j] - mu; sq2[j & 1] = fmaf(d, d, sq2[j & 1]); }
       }
     }
-    const float rs = 1.0f / sqrtf(warp_sum(sq) / C + eps);
+    const float rs = 1.0f / sqrtf(warp_sum(sq2[0] + sq2[1]) * inv_c + eps);
+    const float nb = -mu * rs;
     T* yr = y + (long)row * C;
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
@@ -267,10 +272,10 @@ __global__ void __launch_bounds__(256, (NCH * Vec<T>::N <= 24 ? 4 : 2)) ln_fwd_k
         for (int j = 0; j < NV; j += 4) {
           const float4 gv = __ldg(reinterpret_cast<const float4*>(g + ch * NV + j));
           const float4 bv = rms ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldg(reinterpret_cast<const float4*>(b + ch * NV + j));
-          o[j] = (v[i][j] - mu) * rs * gv.x + bv.x;
-          o[j + 1] = (v[i][j + 1] - mu) * rs * gv.y + bv.y;
-          o[j + 2] = (v[i][j + 2] - mu) * rs * gv.z + bv.z;
-          o[j + 3] = (v[i][j + 3] - mu) * rs * gv.w + bv.w;
+          o[j] = fmaf(fmaf(v[i][j], rs, nb), gv.x, bv.x);
+          o[j + 1] = fmaf(fmaf(v[i][j + 1], rs, nb), gv.y, bv.y);
+          o[j + 2] = fmaf(fmaf(v[i][j + 2], rs, nb), gv.z, bv.z);
+          o[j + 3] = fmaf(fmaf(v[i][j + 3], rs, nb), gv.w, bv.w);
         }
         Vec<T>::store(yr + ch * NV, o);
       }
@@ -561,10 +566,161 @@ ln_bwd2_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* _
   }
 }
 
+// The same row-group backward with the next LNB3_NS rows of every group (dy,
+// x and the incoming residual gradient) in a ring of shared-memory slots
+// filled by bulk copies: each group keeps LNB3_NS rows in flight without
+// holding them in registers, so a block moves three times the bytes of the
+// register-prefetch form per memory latency.  A slot is refilled by the
+// group's first thread once the group's named barrier shows that every thread
+// has read it; the arithmetic and its order are those of ln_bwd2_kernel, so the
+// results are the same bits.  Needs 16-byte aligned rows (C * sizeof(T) % 16
+// == 0 and aligned bases).
+#define LNB3_NS 2
+template <typename T>
+__global__ void __launch_bounds__(LNB2_THREADS, 2)
+ln_bwd3_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __restrict__ mean,
+               const float* __restrict__ rstd, const float* __restrict__ g, const float* dres_in, float* dres_out,
+               T* __restrict__ dres_out_t, float* __restrict__ partials, int M, int C, int TPR, int G, int rms,
+               unsigned* __restrict__ err) {
+  constexpr int NV = Vec<T>::N;
+  extern __shared__ __align__(16) uint8_t lb3_raw[];
+  __shared__ __align__(8) uint64_t full[LNB2_THREADS / 32][LNB3_NS];
+  __shared__ float2 slot[2][LNB2_THREADS / 32];
+  const int grp = threadIdx.x / TPR, t = threadIdx.x % TPR;
+  const int nch = C / NV;
+  const bool act = grp < G && t < nch;
+  const int wpg = TPR / 32, wig = t / 32, lane = threadIdx.x & 31;
+  const int col = t * NV;
+  // one slot: dy | x | incoming residual gradient (absent for the first backward)
+  const uint32_t tb = (uint32_t)C * sizeof(T), fb = dres_in ? (uint32_t)C * 4u : 0u;
+  const uint32_t sb = 2 * tb + fb;
+  const uint32_t ring = smem_u32(lb3_raw) + grp * LNB3_NS * sb;
+  const int stride = gridDim.x * G;
+  int row = blockIdx.x * G + grp;
+  auto fbar = [&](int s) { return smem_u32(&full[grp][s]); };
+  auto issue = [&](int r, int s) {
+    const uint32_t bar = fbar(s), dst = ring + s * sb;
+    mbar_expect_tx(bar, sb);
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(reinterpret_cast<uint64_t>(dy + (long)r * C)), "r"(tb), "r"(bar) : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst + tb), "l"(reinterpret_cast<uint64_t>(x + (long)r * C)), "r"(tb), "r"(bar) : "memory");
+    if (fb)
+      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                   ::"r"(dst + 2 * tb), "l"(reinterpret_cast<uint64_t>(dres_in + (long)r * C)), "r"(fb), "r"(bar)
+                   : "memory");
+  };
+  if (grp < G && t == 0) {
+    for (int s = 0; s < LNB3_NS; ++s) mbar_init(fbar(s), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  griddep_wait();
+  griddep_release();
+  if (grp < G && t == 0)
+    for (int s = 0; s < LNB3_NS; ++s)
+      if (row + s * stride < M) issue(row + s * stride, s);
+  float gg[NV], dg[NV], db[NV], dsm[NV];
+#pragma unroll
+  for (int j = 0; j < NV; ++j) { gg[j] = 0.f; dg[j] = 0.f; db[j] = 0.f; dsm[j] = 0.f; }
+  if (act) {
+#pragma unroll
+    for (int j = 0; j < NV; j += 4) Vec<float>::load(g + col + j, gg + j);
+  }
+  float mu = 0.f, rs = 0.f;
+  if (act && row < M) { mu = mean[row]; rs = rstd[row]; }
+  __syncthreads();   // the barriers are initialised before any thread waits on them
+  // every issued copy is waited for, each wait bounded (a wait that gives up
+  // flags the step and the kernel still ends)
+  volatile int never = 0;
+  const int iters = (M + stride - 1) / stride;
+  for (int it = 0; it < iters; ++it, row += stride) {
+    const int s = it % LNB3_NS;
+    const bool live = act && row < M;
+    float dv[NV], xh[NV], o[NV];
+    if (grp < G && row < M && !mbar_wait(fbar(s), (it / LNB3_NS) & 1, &never, 1ll << 28) && t == 0)
+      atomicOr(err, GPT_DEVERR_TIMEOUT);
+    if (live) {
+      const uint32_t src = ring + s * sb + col * (uint32_t)sizeof(T);
+      uint4 q;
+      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(q.x), "=r"(q.y), "=r"(q.z), "=r"(q.w) : "r"(src));
+      Vec<T>::load(reinterpret_cast<const T*>(&q), dv);
+      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(q.x), "=r"(q.y), "=r"(q.z), "=r"(q.w) : "r"(src + tb));
+      Vec<T>::load(reinterpret_cast<const T*>(&q), xh);
+      if (fb) {
+        const uint32_t fsrc = ring + s * sb + 2 * tb + col * 4u;
+#pragma unroll
+        for (int j = 0; j < NV; j += 4)
+          asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                       : "=f"(o[j]), "=f"(o[j + 1]), "=f"(o[j + 2]), "=f"(o[j + 3]) : "r"(fsrc + 4u * j));
+      } else {
+#pragma unroll
+        for (int j = 0; j < NV; ++j) o[j] = 0.f;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < NV; ++j) { dv[j] = 0.f; xh[j] = 0.f; o[j] = 0.f; }
+    }
+    const float mu_r = mu, rs_r = rs;
+    if (act && row + stride < M) { mu = mean[row + stride]; rs = rstd[row + stride]; }
+    float s1 = 0.f, s2 = 0.f, gh[NV];
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      xh[j] = (xh[j] - mu_r) * rs_r;
+      gh[j] = dv[j] * gg[j];
+      s1 += gh[j];
+      s2 += gh[j] * xh[j];
+      if (live) { dg[j] += dv[j] * xh[j]; db[j] += dv[j]; }
+    }
+    s1 = warp_sum(live ? s1 : 0.f);
+    s2 = warp_sum(live ? s2 : 0.f);
+    if (lane == 0 && grp < G) slot[it & 1][grp * wpg + wig] = make_float2(s1, s2);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // slot reads before the refill's writes
+    if (grp < G) asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(TPR) : "memory");
+    if (grp < G && t == 0 && row + LNB3_NS * stride < M) issue(row + LNB3_NS * stride, s);
+    s1 = 0.f; s2 = 0.f;
+    for (int w = 0; w < wpg; ++w) {
+      const float2 v = slot[it & 1][grp * wpg + w];
+      s1 += v.x;
+      s2 += v.y;
+    }
+    s1 = rms ? 0.f : s1 / C;   // RMSNorm: no mean term
+    s2 /= C;
+    if (live) {
+      const long off = (long)row * C + col;
+#pragma unroll
+      for (int j = 0; j < NV; ++j) {
+        o[j] += rs_r * (gh[j] - s1 - xh[j] * s2);
+        dsm[j] += o[j];
+      }
+#pragma unroll
+      for (int j = 0; j < NV; j += 4) Vec<float>::store(dres_out + off + j, o + j);
+      Vec<T>::store(dres_out_t + off, o);
+    }
+  }
+  // every issued copy has been waited for (each group consumes the rows it
+  // prefetched), so the ring is free for the group sums: [dg | db | dsm] per block
+  __syncthreads();
+  float* red2 = reinterpret_cast<float*>(lb3_raw);
+  if (act) {
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      red2[grp * 3 * C + col + j] = dg[j];
+      red2[grp * 3 * C + C + col + j] = db[j];
+      red2[grp * 3 * C + 2 * C + col + j] = dsm[j];
+    }
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < 3 * C; c += blockDim.x) {
+    float acc = 0.f;
+    for (int gi = 0; gi < G; ++gi) acc += red2[gi * 3 * C + c];
+    partials[(long)blockIdx.x * 3 * C + c] = acc;
+  }
+}
+
 template <typename T>
 cudaError_t launch_ln_bwd(const T* dy, const T* x, const float* mean, const float* rstd, const float* g,
                           const float* dres_in, float* dres_out, T* dres_out_t, float* partials,
-                          int M, int C, int* nblk_out, cudaStream_t s, bool rms) {
+                          int M, int C, int* nblk_out, cudaStream_t s, bool rms, unsigned* err) {
   constexpr int NV = Vec<T>::N;
   {
     // row-group kernel: C / NV threads per row (whole warps), several rows per block
@@ -574,6 +730,22 @@ cudaError_t launch_ln_bwd(const T* dy, const T* x, const float* mean, const floa
       int nblk = (M + G - 1) / G;
       if (nblk > 148 * 2) nblk = 148 * 2;
       *nblk_out = nblk;
+      // bulk-copied rows when every row starts on a 16-byte boundary
+      const bool bulk = err && (C * sizeof(T)) % 16 == 0 && ((uintptr_t)dy & 15) == 0 && ((uintptr_t)x & 15) == 0 &&
+                        ((uintptr_t)dres_in & 15) == 0;
+      if (bulk) {
+        const size_t sb = (size_t)C * (2 * sizeof(T) + (dres_in ? 4 : 0));
+        const size_t smem3 = std::max((size_t)G * LNB3_NS * sb, (size_t)G * 3 * C * sizeof(float));
+        static size_t attr3 = 0;
+        if (smem3 > 48 * 1024 && smem3 > attr3) {
+          cudaError_t e = cudaFuncSetAttribute(ln_bwd3_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3);
+          if (e != cudaSuccess) return e;
+          attr3 = smem3;
+        }
+        ++g_kernel_launches;
+        return launch_k(ln_bwd3_kernel<T>, dim3(nblk), dim3(G * tpr), smem3, s, dy, x, mean, rstd, g, dres_in,
+                        dres_out, dres_out_t, partials, M, C, tpr, G, rms ? 1 : 0, err);
+      }
       const size_t smem = (size_t)G * 3 * C * sizeof(float);
       static size_t attr = 0;
       if (smem > 48 * 1024 && smem > attr) {
@@ -1397,7 +1569,7 @@ cudaError_t launch_wait_timeout_probe(unsigned* err, long long timeout_cycles, c
                                         float, cudaStream_t);                                            \
   template cudaError_t launch_ln_bwd<T>(const T*, const T*, const float*, const float*, const float*,      \
                                         const float*, float*, T*, float*, int, int, int*, cudaStream_t,   \
-                                        bool);                                                           \
+                                        bool, unsigned*);                                                \
   template cudaError_t launch_colsum<T>(const T*, long, int, int, float*, int*, cudaStream_t);            \
   template cudaError_t launch_xent<T>(T*, long, const int*, int, int, int, float*, DevScalars*, cudaStream_t); \
   template cudaError_t launch_embed_bwd<T>(const float*, const int*, const int*, float*, float*, int, int,  \

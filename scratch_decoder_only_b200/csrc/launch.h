@@ -53,10 +53,11 @@ cudaError_t launch_ln_fwd(const T* x, const float* g, const float* b, T* y, floa
 // partials: [nblk][3C] = dg | db | column sums of dres_out (the bias gradient of
 // the layer whose output gradient dres_out is)
 // rms: the RMSNorm backward (no mean term; the db partials are then unused)
+// err: device error word for the bounded waits of the bulk-copy form (taken only when given)
 template <typename T>
 cudaError_t launch_ln_bwd(const T* dy, const T* x, const float* mean, const float* rstd, const float* g,
                           const float* dres_in, float* dres_out, T* dres_out_t, float* partials,
-                          int M, int C, int* nblk_out, cudaStream_t s, bool rms = false);
+                          int M, int C, int* nblk_out, cudaStream_t s, bool rms = false, unsigned* err = nullptr);
 // Deferred column reductions: for each segment, dst[n] = sum_r src[r * ld + n]
 // (n < cols, r < rows, fixed summation order).  Segments are launched in
 // lists of RED_MAX_SEGS (the list travels as the kernel parameter).
