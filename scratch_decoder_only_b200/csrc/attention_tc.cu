@@ -729,13 +729,32 @@ __device__ __forceinline__ int bwd_niter(const int* dsr, int qb_lo, int nqb, int
   return n;
 }
 
+// Column sums of a warp's 32 x 32 block (lane = row, a[j] = column j): five
+// exchange rounds, each keeping half of the columns, leave lane l with the sum
+// of column l over the 32 rows.
+__device__ __forceinline__ float warp_colsum32(float (&a)[32], int lane) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < o; ++j) {
+      const float send = up ? a[j] : a[j + o];
+      const float keep = up ? a[j + o] : a[j];
+      a[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  return a[0];
+}
+
 template <bool F16>
 __global__ void __launch_bounds__(BW_THREADS, 1)
 attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
             const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ lse, const float* __restrict__ Dbuf,
             const int* __restrict__ dstart, int T, int H, int BH, int kcol0, int vcol0, int G, bf16* __restrict__ dkv,
-            long ld_kv, int v_off, unsigned* err, float sl2) {
+            long ld_kv, int v_off, unsigned* err, float sl2, float* __restrict__ cpart, long cp_ld) {
   // sl2 = log2(e) / sqrt(d) as in the forward; dK carries the 1 / sqrt(d) factor
+  // cpart (optional): column sums of dK and dV per 32 keys, row ((b nkb + key
+  // block) 4 + quarter) at cpart + row cp_ld, dK columns from 0, dV from v_off
   const float dk_scale = sl2 * (1.0f / LOG2E_F);
   extern __shared__ __align__(1024) uint8_t at_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)at_raw + 1023) & ~(uintptr_t)1023);
@@ -1079,6 +1098,16 @@ attn_bwd_tc(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ C
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(DKV_FREE));   // the next item's dV / dK may overwrite TMEM
         }
+        if (cpart) {
+          // the warp's 32 keys summed per column (keys past T add nothing): lane l
+          // ends with column 32 grp + l of the head
+          float a[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) a[j] = k < T ? __uint_as_float(rr[j]) * sc : 0.f;
+          const float cs = warp_colsum32(a, lane);
+          const long crow = ((long)I.b * nkb + I.k0 / AT_BLK) * 4 + quarter;
+          cpart[crow * cp_ld + (part == 0 ? 0 : v_off) + I.h * AT_D + 32 * grp + lane] = cs;
+        }
         if (k >= T) continue;
         bf16* dst = row + (part == 0 ? 0 : v_off) + I.h * AT_D + 32 * grp;
 #pragma unroll
@@ -1142,6 +1171,59 @@ __global__ void attn_dq_finish_kernel(float* __restrict__ dq_acc, bf16* __restri
     *reinterpret_cast<uint4*>(dqkv + row * ld_q + c) = w;
     src[0] = make_float4(0.f, 0.f, 0.f, 0.f);
     src[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+// The same finish over one 32-row slab per block (rows b T + 128 kb + 32 q + [0, 32)
+// below T, slab (b nkb + kb) 4 + q), also writing the slab's column sums of dq to
+// cpart + slab cp_ld (the bias gradient's partial rows; zeros for an empty slab).
+// Thread (lane rl, chunk ch) takes 8 columns of rows rl, rl + RL, ...; the RL row
+// lanes' sums are added in a fixed order through shared memory.
+#define DQF_THREADS 384
+template <bool F16>
+__global__ void __launch_bounds__(DQF_THREADS) attn_dq_finish_cs_kernel(float* __restrict__ dq_acc,
+                                                                        bf16* __restrict__ dqkv, int T, int C,
+                                                                        long ld_q, float scale, int nkb,
+                                                                        float* __restrict__ cpart, long cp_ld) {
+  extern __shared__ float dqf_red[];   // [RL][C]
+  griddep_wait();
+  griddep_release();
+  const int slab = blockIdx.x, qq = slab & 3, bk = slab >> 2;
+  const int b = bk / nkb, t0 = (bk % nkb) * AT_BLK + 32 * qq;
+  const int nr = min(32, T - t0);
+  const long row0 = (long)b * T + t0;
+  const int nch = C / 8;
+  const int RL = nch >= DQF_THREADS ? 1 : DQF_THREADS / nch;
+  const int rl = threadIdx.x / nch;
+  for (int ch = threadIdx.x % nch; ch < nch && rl < RL; ch += DQF_THREADS) {
+    float cs[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) cs[j] = 0.f;
+#pragma unroll 4
+    for (int r = rl; r < nr; r += RL) {
+      float4* src = reinterpret_cast<float4*>(dq_acc + (row0 + r) * C + ch * 8);
+      const float4 a = src[0], bq = src[1];
+      const float v[8] = {a.x * scale, a.y * scale, a.z * scale, a.w * scale,
+                          bq.x * scale, bq.y * scale, bq.z * scale, bq.w * scale};
+      uint4 w;
+      w.x = pack16x2<F16>(v[0], v[1]);
+      w.y = pack16x2<F16>(v[2], v[3]);
+      w.z = pack16x2<F16>(v[4], v[5]);
+      w.w = pack16x2<F16>(v[6], v[7]);
+      *reinterpret_cast<uint4*>(dqkv + (row0 + r) * ld_q + ch * 8) = w;
+      src[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      src[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) cs[j] += v[j];
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) dqf_red[rl * C + ch * 8 + j] = cs[j];
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < C; c += DQF_THREADS) {
+    float acc = 0.f;
+    for (int i = 0; i < RL; ++i) acc += dqf_red[i * C + c];
+    cpart[(long)slab * cp_ld + c] = acc;
   }
 }
 
@@ -1216,7 +1298,7 @@ cudaError_t launch_attn_fwd_tc(const bf16* qkv, bf16* out, float* lse, const int
 template <bool F16>
 static cudaError_t attn_bwd_tc_t(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* Dbuf,
                                  bool d_ready, float* dq_acc, const int* dstart, bf16* dqkv, int B, int T, int H,
-                                 unsigned* err, cudaStream_t s, const AttnLayout& L, int d_real) {
+                                 unsigned* err, cudaStream_t s, const AttnLayout& L, int d_real, float* cpart) {
   const int C = H * AT_D;
   const float scale = 1.0f / sqrtf((float)d_real);
   const long rows = (long)B * T;
@@ -1250,20 +1332,34 @@ static cudaError_t attn_bwd_tc_t(const bf16* qkv, const bf16* out, const bf16* d
   const int grid = n_items < sms ? n_items : sms;
   if (n_items > (long)grid * BW_MAX_ITEMS) return cudaErrorInvalidValue;
   ++g_kernel_launches;
+  const long cp_ld = 3L * C;   // partial rows of the q|k|v bias gradient
   e = launch_k(attn_bwd_tc<F16>, dim3(grid), dim3(BW_THREADS), smem, s, tqkv, tdo, tdq, lse, Dbuf, dstart, T, H, B * H,
-               L.kcol, L.vcol, L.G, L.dkv, L.ld_kv, L.v_off, err, scale * LOG2E_F);
+               L.kcol, L.vcol, L.G, L.dkv, L.ld_kv, L.v_off, err, scale * LOG2E_F, cpart ? cpart + C : nullptr, cp_ld);
   if (e != cudaSuccess) return e;
   ++g_kernel_launches;
+  if (cpart) {
+    const int nkb = (T + AT_BLK - 1) / AT_BLK;
+    const int nch = C / 8, rl = nch >= DQF_THREADS ? 1 : DQF_THREADS / nch;
+    const size_t red = (size_t)rl * C * sizeof(float);
+    if (red > 48 * 1024) return cudaErrorInvalidValue;
+    return launch_k(attn_dq_finish_cs_kernel<F16>, dim3((unsigned)(B * nkb * 4)), dim3(DQF_THREADS), red, s, dq_acc,
+                    dqkv, T, C, (long)L.qw, scale, nkb, cpart, cp_ld);
+  }
   return launch_k(attn_dq_finish_kernel<F16>, dim3(148 * 8), dim3(256), 0, s, dq_acc, dqkv, rows, C, (long)L.qw, scale);
 }
 
 cudaError_t launch_attn_bwd_tc(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* Dbuf,
                                bool d_ready, float* dq_acc, const int* dstart, bf16* dqkv, int B, int T, int H,
-                               unsigned* err, cudaStream_t s, bool f16, const AttnLayout* lay, int d_real) {
+                               unsigned* err, cudaStream_t s, bool f16, const AttnLayout* lay, int d_real,
+                               float* bias_part) {
   const AttnLayout L = lay ? *lay : attn_layout_mha(dqkv, H * AT_D);
   if (!layout_ok(L, H) || !L.dkv || d_real < 1 || d_real > AT_D) return cudaErrorInvalidValue;
-  return f16 ? attn_bwd_tc_t<true>(qkv, out, dout, lse, Dbuf, d_ready, dq_acc, dstart, dqkv, B, T, H, err, s, L, d_real)
-             : attn_bwd_tc_t<false>(qkv, out, dout, lse, Dbuf, d_ready, dq_acc, dstart, dqkv, B, T, H, err, s, L, d_real);
+  // the bias column sums index q|k|v columns of one fused row: plain heads only
+  if (bias_part && (lay || d_real != AT_D)) return cudaErrorInvalidValue;
+  return f16 ? attn_bwd_tc_t<true>(qkv, out, dout, lse, Dbuf, d_ready, dq_acc, dstart, dqkv, B, T, H, err, s, L, d_real,
+                                   bias_part)
+             : attn_bwd_tc_t<false>(qkv, out, dout, lse, Dbuf, d_ready, dq_acc, dstart, dqkv, B, T, H, err, s, L, d_real,
+                                    bias_part);
 }
 
 // ------------------------------------------------------------ zero-padded heads

@@ -368,8 +368,10 @@ static int build_arena(gpt_model* m) {
     // partial rows of every deferred column reduction of one backward pass:
     // LayerNorm blocks (at most 444 rows of 3C) and bias column sums (at most
     // one row per 128 tokens), each region rounded to 16 bytes
-    const size_t ln = (size_t)444 * 3 * C + 4, cs = (size_t)(Mx + 127) / 128;
-    m->partials_n = ln + NL * (2 * ln + cs * F + 4 + cs * 3 * C + 4);
+    // (the q|k|v bias partials from the attention backward: one row per 32
+    // rows of each sequence's 128-row blocks, at most 4 (Mx / 128 + Bmax))
+    const size_t ln = (size_t)444 * 3 * C + 4, cs = (size_t)(Mx + 127) / 128, cq = 4 * (cs + m->Bmax);
+    m->partials_n = ln + NL * (2 * ln + cs * F + 4 + cq * 3 * C + 4);
   }
   cv.add((void**)&m->partials, m->partials_n * 4);
   cv.add((void**)&m->normpart, m->normblk * 8);
@@ -559,7 +561,7 @@ static int attn_fwd(gpt_model* m, const T16* qkv, T16* out, float* lse, int B, i
   return GPT_OK;
 }
 static int attn_bwd(gpt_model* m, const float* qkv, const float* out, const float* dout, const float* lse,
-                    float* dqkv, int B, int T, bool, const AttnLayout* = nullptr, int = 0) {
+                    float* dqkv, int B, int T, bool, const AttnLayout* = nullptr, int = 0, float* = nullptr) {
   ProfScope ps(m, PC_ATTN_BWD, 8.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0, attn_pair_mult(m, 8.0 * m->d));
   CK(launch_attn_bwd_simt<float>(qkv, out, dout, lse, m->attD, m->dstart, dqkv, B, T, m->H, m->d, m->stream));
   return GPT_OK;
@@ -567,7 +569,8 @@ static int attn_bwd(gpt_model* m, const float* qkv, const float* out, const floa
 // d_ready: m->attD already holds D = rowsum(dO o O) (tensor-core path only)
 template <typename T16>
 static int attn_bwd(gpt_model* m, const T16* qkv, const T16* out, const T16* dout, const float* lse,
-                    T16* dqkv, int B, int T, bool d_ready, const AttnLayout* lay = nullptr, int layer = 0) {
+                    T16* dqkv, int B, int T, bool d_ready, const AttnLayout* lay = nullptr, int layer = 0,
+                    float* bias_part = nullptr) {
   ProfScope ps(m, PC_ATTN_BWD, 8.0 * m->d * attn_pairs(B, T, m->H, m->seg_used), 0.0, attn_pair_mult(m, 8.0 * m->d));
   constexpr bool F16 = std::is_same<T16, f16>::value;
   auto cb = [](const T16* p) { return reinterpret_cast<const bf16*>(p); };
@@ -587,7 +590,7 @@ static int attn_bwd(gpt_model* m, const T16* qkv, const T16* out, const T16* dou
     CK(launch_attn_pad(gp, reinterpret_cast<bf16*>(dqkv), rows, 3 * m->H, m->d, false, m->stream));
   } else if (attn_tc_supported(m->d))
     CK(launch_attn_bwd_tc(cb(qkv), cb(out), cb(dout), lse, m->attD, d_ready, m->dq_acc, m->dstart,
-                          reinterpret_cast<bf16*>(dqkv), B, T, m->H, &m->sc->err, m->stream, F16, lay));
+                          reinterpret_cast<bf16*>(dqkv), B, T, m->H, &m->sc->err, m->stream, F16, lay, 64, bias_part));
   else if (!F16 && attn_mma_supported(m->d))
     CK(launch_attn_bwd_mma(cb(qkv), cb(out), cb(dout), lse, m->attD, m->dstart, reinterpret_cast<bf16*>(dqkv), B, T,
                            m->H, m->d, m->stream));
@@ -760,8 +763,18 @@ static int backward_impl(gpt_model* m) {
       if (fuse_d) { e.aux = A.att(l); e.ld_aux = C; e.rowdot = m->attD; e.rd_T = T_; }
       CKI(gemm(m, M, C, C, drt, C, false, A.W(lo.w_o), C, true, e));
     }
-    CKI(attn_bwd(m, A.qkv(l), A.att(l), dC, A.lse(l), dq, B, T_, fuse_d, nullptr, l));
-    {
+    // the q|k|v bias gradient: on the tensor-core attention of 64-column heads
+    // its column sums come out of the backward kernels (one partial row per 32
+    // rows), otherwise from a column-sum pass over dq
+    const bool fuse_bq = sizeof(T) == 2 && attn_tc_supported(m->d) && !m->apad;
+    if (fuse_bq) {
+      const int crows = B * ((T_ + 127) / 128) * 4;
+      float* qpart = take((size_t)crows * 3 * C);
+      if (!qpart) FAIL(GPT_ERR_NOMEM, "partials arena too small");
+      CKI(attn_bwd(m, A.qkv(l), A.att(l), dC, A.lse(l), dq, B, T_, fuse_d, nullptr, l, qpart));
+      seg(qpart, A.G(lo.b_qkv), crows, 3 * C, 3 * C);
+    } else {
+      CKI(attn_bwd(m, A.qkv(l), A.att(l), dC, A.lse(l), dq, B, T_, fuse_d, nullptr, l));
       float* qpart = take((size_t)((M + 127) / 128) * 3 * C);
       if (!qpart) FAIL(GPT_ERR_NOMEM, "partials arena too small");
       ProfScope ps(m, PC_BIAS, 0, (double)M * 3 * C * es);

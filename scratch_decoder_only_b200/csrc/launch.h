@@ -157,10 +157,13 @@ cudaError_t launch_attn_fwd_tc(const bf16* qkv, bf16* out, float* lse, const int
                                int d_real = 64);
 // d_ready: Dbuf [B, H, T] already holds rowsum(dO o O) (written by the GEMM
 // epilogue that produced dO); otherwise a row-dot kernel computes it first
+// bias_part (plain 64-column heads only): also write the column sums of the
+// q|k|v gradient as partial rows [B * ceil(T/128) * 4][3 H 64], one per 32 rows
+// (rows b T + 128 kb + 32 q + [0, 32) below T -> row (b ceil(T/128) + kb) 4 + q)
 cudaError_t launch_attn_bwd_tc(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* Dbuf,
                                bool d_ready, float* dq_acc, const int* dstart, bf16* dqkv, int B, int T, int H,
                                unsigned* err, cudaStream_t s, bool f16 = false, const AttnLayout* lay = nullptr,
-                               int d_real = 64);
+                               int d_real = 64, float* bias_part = nullptr);
 // heads of d < 64 columns (64 % d == 0) on the d = 64 tensor-core kernels:
 // copies with every head widened to 64 columns by zeros (pad: src [rows]
 // [groups][d] -> dst [rows][groups][64]; !pad: back, the extra columns dropped)
