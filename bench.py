@@ -540,6 +540,50 @@ def decode_profile(torch, dev, batches=(1, 32), n_new=17):
     model.close()
 
 
+def critical_path(evs):
+    """Charge each kernel record end_k - max(end_0..end_(k-1)) in start order:
+    with programmatic dependent launch a kernel starts while its predecessor
+    drains, so its own duration overstates what it adds to the chain.
+    Returns {name: [launches, total_us, summed_duration_us]} and the total."""
+    agg = {}
+    prev_end = evs[0][0] if evs else 0.0
+    for start, end, name in evs:
+        d = max(0.0, end - prev_end)
+        prev_end = max(prev_end, end)
+        a = agg.setdefault(name, [0, 0.0, 0.0])
+        a[0] += 1
+        a[1] += d
+        a[2] += end - start
+    return agg, sum(v[1] for v in agg.values())
+
+
+def train_profile(torch, dev, steps=3):
+    """Per-kernel critical path of the graph-replayed training step (CUPTI
+    kernel records through torch.profiler), headline workload.  Prints a
+    table; not a bench value."""
+    from torch.profiler import profile, ProfilerActivity
+    from scratch_decoder_only_b200.gpt import GPT
+    tok, tgt, _ = S.make_batch(WL)
+    d_tok, d_tgt = torch.from_numpy(tok).to(dev), torch.from_numpy(tgt).to(dev)
+    model = GPT(WL.model, WL.init_seed)
+    loss = torch.zeros(1, dtype=torch.float32, device=dev)
+    for _ in range(3):   # the first call captures the step's graph
+        model.train_step(d_tok, d_tgt, None, WL.adamw, loss)
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        for _ in range(steps):
+            model.train_step(d_tok, d_tgt, None, WL.adamw, loss)
+        torch.cuda.synchronize()
+    evs = sorted(((e.time_range.start, e.time_range.end, e.name.split("(")[0].replace("void ", ""))
+                  for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA), key=lambda r: r[0])
+    agg, tot = critical_path(evs)
+    print(f"{WL.name}: {steps} steps, critical path {tot / steps:.1f} us per step")
+    print(f"  {'kernel':60s} {'per step':>8s} {'us/step':>9s} {'us each':>8s} {'dur each':>9s}")
+    for k, (n, t, dur) in sorted(agg.items(), key=lambda kv: -kv[1][1]):
+        print(f"  {k[:60]:60s} {n // steps:8d} {t / steps:9.1f} {t / n:8.2f} {dur / n:9.2f}")
+    model.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -553,10 +597,17 @@ def main():
     ap.add_argument("--batch", type=int, default=None, help="override the batch (profiling of small cases)")
     ap.add_argument("--decode-profile", action="store_true",
                     help="print the per-kernel critical path of greedy decode and exit (no bench line)")
+    ap.add_argument("--train-profile", action="store_true",
+                    help="print the per-kernel critical path of the training step and exit (no bench line)")
     args = ap.parse_args()
     if args.decode_profile:
         import torch
         decode_profile(torch, torch.device("cuda", 0))
+        return
+    if args.train_profile:
+        import torch
+        torch.cuda.set_device(0)
+        train_profile(torch, torch.device("cuda", 0))
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

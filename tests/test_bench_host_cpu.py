@@ -1,5 +1,6 @@
 """Host-side pieces of bench.py that need no GPU: the clock/throttle summary
-taken from nvidia-smi's CSV lines, and the FLOP count behind MFU."""
+taken from nvidia-smi's CSV lines, the FLOP count behind MFU, and the
+critical-path charge of the profile modes."""
 import pytest
 
 
@@ -39,3 +40,18 @@ def test_flops_per_token_gpt2():
     # 6 N + 6 L C (T + 1) with N = 124,475,904 (tied, padded vocabulary)
     assert mc.num_params() == 124_475_904
     assert bench.flops_per_token(mc, 1024) == pytest.approx(6 * 124_475_904 + 6 * 12 * 768 * 1025)
+
+
+def test_critical_path_charges_only_what_extends_the_chain():
+    """Kernel records (start, end, name) in start order: a kernel is charged the
+    part of it that ends after everything before it, so the charges add up to
+    the span from the first start to the last end, a kernel hidden under its
+    predecessor costs nothing, and its own duration is kept beside."""
+    import bench
+    evs = [(0.0, 10.0, "a"), (5.0, 12.0, "b"), (6.0, 11.0, "c"), (13.0, 20.0, "a")]
+    agg, tot = bench.critical_path(evs)
+    assert tot == 20.0
+    assert agg["a"] == [2, 18.0, 17.0]
+    assert agg["b"] == [1, 2.0, 7.0]
+    assert agg["c"] == [1, 0.0, 5.0]
+    assert bench.critical_path([]) == ({}, 0.0)
