@@ -512,12 +512,9 @@ def decode_profile(torch, dev, batches=(1, 32), n_new=17):
         adv = [i for i, e in enumerate(evs) if "argmax" in e.name]
         evs = evs[adv[0] + 1: adv[-1] + 1]   # the replayed steps
         nsteps = len(adv) - 1
-        agg, order = {}, []
-        prev_end, nmma = evs[0].time_range.start, 0
+        labelled, nmma = [], 0
         names = ["q/k/v + LN1", "out", "fc + LN2", "fc2"]
         for e in evs:
-            d = max(0.0, e.time_range.end - prev_end)
-            prev_end = max(prev_end, e.time_range.end)
             k = e.name.split("(")[0].replace("void ", "")
             if "argmax" in k:
                 nmma = 0
@@ -526,16 +523,14 @@ def decode_profile(torch, dev, batches=(1, 32), n_new=17):
                 nmma += 1
             elif "argmax" in k:
                 k = "argmax + next embedding + step advance"
-            if k not in agg:
-                agg[k] = [0, 0.0]
-                order.append(k)
-            agg[k][0] += 1
-            agg[k][1] += d
-        tot = sum(v[1] for v in agg.values()) / nsteps
+            labelled.append((e.time_range.start, e.time_range.end, k))
+        agg, tot = critical_path(labelled)
+        order = list(agg)
+        tot /= nsteps
         print(f"batch {B}: {nsteps} steps, critical path {tot:.1f} us per step ({B / tot * 1e6:.0f} tok/s)")
         print(f"  {'kernel':48s} {'per step':>9s} {'us/step':>9s} {'us each':>8s} {'share':>6s}")
         for k in sorted(order, key=lambda k: -agg[k][1]):
-            n, t = agg[k]
+            n, t, _ = agg[k]
             print(f"  {k[:48]:48s} {n // nsteps:9d} {t / nsteps:9.1f} {t / n:8.2f} {100 * t / nsteps / tot:5.1f}%")
     model.close()
 
